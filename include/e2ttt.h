@@ -1,0 +1,162 @@
+/*
+ * e2ttt.h -- C ABI of the E2-TTT chunk-parallel closed-form fast-weight update
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Rethinking Expressivity and Efficiency in Test-Time Training"
+ * (E2-TTT, arXiv 2608.21308). Its abstract states that, with gradients taken
+ * at the chunk-start weights, a closed-form state transition reproduces
+ * exactly the chunk-end fast-weight and momentum states of the per-token
+ * recurrence; its "Approach" summary (atlas.scime.ai) says the transition is
+ * built from two scalar kernels (a momentum kernel and a weight kernel) made
+ * with log-space cumulative sums, and two weighted gradient aggregations; the
+ * "Limitations" summaries say the chunk output is taken at the chunk-start
+ * weights.
+ *
+ * Semantics implemented here, per batch row b and head h, for the chunk of
+ * tokens t = 1..C (chunk i holds tokens [iC, (i+1)C); the last may be short):
+ *   per-token recurrence (gates: eta = lr, mu = mom, lam = decay)
+ *       M_t = mu_t M_{t-1} - eta_t g_t ,   W_t = lam_t W_{t-1} + M_t
+ *   with g_t = grad_W l(W0; k_t, v_t) at the chunk-start weights W0, and
+ *       l = 1/2 |f_W(k) - v|^2   (E2TTT_LOSS_MSE)   or   -<f_W(k), v>   (E2TTT_LOSS_NEG_DOT)
+ *       f_W(x) = W x                          (E2TTT_LINEAR,  W  [d_v, d_k])
+ *       f_W(x) = W2 (silu(W1 x) * (W3 x))     (E2TTT_SWIGLU,  W1, W3 [d_h, d_k], W2 [d_v, d_h])
+ *   closed form (what the library computes):
+ *       a_t = eta_t U(t+1,C),  b_t = eta_t sum_{j=t..C} L(j+1,C) U(t+1,j)
+ *       M_end = U(1,C) M0 - sum_t a_t g_t
+ *       W_end = L(1,C) W0 + (sum_j L(j+1,C) U(1,j)) M0 - sum_t b_t g_t
+ *       out_t = f_{W0}(q_t)
+ *   where U(i,j) = prod_{s=i..j} mu_s and L(i,j) = prod_{s=i..j} lam_s.
+ *   W_end / M_end of a chunk are the W0 / M0 of the next one.
+ *
+ * Layouts (all row-major, contiguous, caller-owned DEVICE memory):
+ *   q, k        [B, H, T, d_k]   activation dtype (shape->act)
+ *   v, out      [B, H, T, d_v]   activation dtype
+ *   lr, mom, decay              [B, H, T] fp32 gate VALUES (not logits)
+ *   W0, M0, W_end, M_end        [B, H, S] fp32, S = e2ttt_state_elems(shape):
+ *        linear: W [d_v, d_k];  SwiGLU: [W1 | W3 | W2] concatenated
+ *   saved_states                [n_chunks, B, H, 2, S] fp32: (W, M) at the
+ *                               start of every chunk (written by the forward,
+ *                               read by the backward)
+ *
+ * Conventions:
+ *   - The library allocates no memory. Scratch comes from `workspace`
+ *     (device memory of at least e2ttt_workspace_bytes(shape, for_bwd) bytes,
+ *     256-byte aligned); its contents on entry do not matter.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream). Argument checks run on the host
+ *     before anything is launched and return E2TTT_ERR_INVALID_ARG or
+ *     E2TTT_ERR_UNSUPPORTED synchronously, with nothing written.
+ *     A failed launch returns E2TTT_ERR_CUDA. The library never exits, aborts
+ *     or traps; e2ttt_last_error() describes the last failure of the calling
+ *     thread.
+ *   - Outputs must not overlap inputs or each other (E2TTT_ERR_INVALID_ARG).
+ *   - Results are deterministic: no atomics in any reduction.
+ */
+#ifndef E2TTT_H
+#define E2TTT_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  E2TTT_OK = 0,
+  E2TTT_ERR_INVALID_ARG = 1,   /* null pointer, bad size, overlap, short workspace   */
+  E2TTT_ERR_UNSUPPORTED = 2,   /* valid but not implemented (see each entry point)    */
+  E2TTT_ERR_CUDA = 3,          /* a CUDA call or kernel launch failed                 */
+  E2TTT_ERR_TIMEOUT = 4        /* a device-side bounded wait gave up                  */
+} e2ttt_status;
+
+typedef enum { E2TTT_LINEAR = 0, E2TTT_SWIGLU = 1 } e2ttt_fast_kind;
+typedef enum { E2TTT_F32 = 0, E2TTT_BF16 = 1 } e2ttt_dtype;
+typedef enum { E2TTT_LOSS_MSE = 0, E2TTT_LOSS_NEG_DOT = 1 } e2ttt_loss;
+
+/* Problem description. kind/act/loss hold e2ttt_fast_kind / e2ttt_dtype /
+ * e2ttt_loss values. d_h is ignored (may be 0) for E2TTT_LINEAR.
+ * Limits: all sizes >= 1; B*H*T*max(d_k,d_v,d_h) < 2^31; 1 <= C <= 1024. */
+typedef struct {
+  int B, H, T, C;
+  int d_k, d_v, d_h;
+  int kind;
+  int act;
+  int loss;
+} e2ttt_shape;
+
+/* Fast-weight state size S per (b, h): d_v*d_k (linear) or 2*d_h*d_k + d_v*d_h
+ * (SwiGLU). Returns 0 for an invalid shape. */
+size_t e2ttt_state_elems(const e2ttt_shape* shape);
+
+/* Bytes of device scratch the forward (for_bwd = 0) or backward (for_bwd = 1)
+ * needs for `shape`. Returns 0 for an invalid shape. */
+size_t e2ttt_workspace_bytes(const e2ttt_shape* shape, int for_bwd);
+
+/* Number of chunks, ceil(T / C); 0 for an invalid shape. */
+int e2ttt_num_chunks(const e2ttt_shape* shape);
+
+/* The two scalar kernels of every chunk (atlas.scime.ai summary, "Approach":
+ * momentum kernel and weight kernel from unrolling the token-wise
+ * momentum-plus-decay recurrence, via log-space cumulative sums; arxivlens
+ * "Results": "log-space suffix, ratio sums").
+ *   a[b,h,t] = eta_t U(t+1,C)                       momentum kernel
+ *   b[b,h,t] = eta_t sum_{j=t..C} L(j+1,C) U(t+1,j) weight kernel
+ *   chunk_scalars [3, B, H, n_chunks]: U(1,C), L(1,C), sum_j L(j+1,C) U(1,j)
+ * t counts from the start of its chunk. Inputs lr/mom/decay [B,H,T] fp32;
+ * outputs a, b [B,H,T] fp32. Device pointers; asynchronous on `stream`. */
+e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* shape,
+                                const float* lr, const float* mom, const float* decay,
+                                float* a, float* b, float* chunk_scalars,
+                                void* stream);
+
+/* Forward over all T tokens (abstract: closed-form chunk state transition;
+ * "Limitations": output at the chunk-start weights).
+ *   Inputs:  q, k, v (act dtype), lr, mom, decay, W0 (fp32), M0 (fp32; may be
+ *            NULL, meaning a zero momentum state).
+ *   Outputs: out (act dtype), W_end, M_end (fp32, the states after the last
+ *            chunk), saved_states (may be NULL; needed by the backward).
+ *   Paths: bf16 activations with T % C == 0, C % 128 == 0, d_k % 64 == 0,
+ *   d_v % 64 == 0 (and d_h % 128 == 0 for SwiGLU) run on the tcgen05 tensor
+ *   cores (bf16 operands, fp32 accumulation and state); every other shape and
+ *   fp32 activations run on fp32 CUDA-core kernels. */
+e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* shape,
+                                  const void* q, const void* k, const void* v,
+                                  const float* lr, const float* mom, const float* decay,
+                                  const float* W0, const float* M0,
+                                  void* out, float* W_end, float* M_end,
+                                  float* saved_states,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Backward of e2ttt_chunk_scan_fwd for the scalar objective
+ *     L = sum_t <dout_t, out_t> + <dW_end, W_end> + <dM_end, M_end>
+ * (abstract: "fully parallelized chunk-level training"). Chunks run in reverse;
+ * the gradient of the chunk-end states flows into the previous chunk. Second
+ * order terms through g_t(W0, k_t, v_t) are included (no stop-gradient).
+ *   Inputs:  q, k, v, lr, mom, decay, saved_states (from the forward), dout
+ *            (act dtype), dW_end, dM_end (fp32 [B,H,S]; may be NULL = zero).
+ *   Outputs: dq, dk, dv (act dtype), dlr, dmom, ddecay (fp32 [B,H,T]),
+ *            dW0, dM0 (fp32 [B,H,S]). */
+e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
+                                  const void* q, const void* k, const void* v,
+                                  const float* lr, const float* mom, const float* decay,
+                                  const float* saved_states, const void* dout,
+                                  const float* dW_end, const float* dM_end,
+                                  void* dq, void* dk, void* dv,
+                                  float* dlr, float* dmom, float* ddecay,
+                                  float* dW0, float* dM0,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Static description of a status code. */
+const char* e2ttt_status_string(e2ttt_status status);
+
+/* Human-readable detail of the last failed call on the calling thread ("" if
+ * none). The pointer stays valid until the thread's next library call. */
+const char* e2ttt_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E2TTT_H */

@@ -313,19 +313,13 @@ def chunk_kernels(eta, mu, lam):
         a[t] = eta[t] * np.prod(mu[t + 1:])
         # R: sum over j >= t of L(j+1,C) * U(t+1, j)  (1-based), i.e. running
         # products of mu over tokens t+1..j (0-based)
-        run = 1.0
-        r = sufL[t + 1]                      # j = t: empty mu product
-        for j in range(t + 1, n):
-            run *= mu[j]
-            r += sufL[j + 1] * run
+        # running products mu_{t+1} ... mu_j for j = t+1 .. C-1 (0-based)
+        run = np.cumprod(mu[t + 1:])
+        r = sufL[t + 1] + np.sum(sufL[t + 2:] * run)   # first term: j = t, empty product
         b[t] = eta[t] * r
     P_U = float(np.prod(mu))
     P_L = float(np.prod(lam))
-    run = 1.0
-    c = 0.0
-    for j in range(n):
-        run *= mu[j]
-        c += sufL[j + 1] * run
+    c = float(np.sum(sufL[1:] * np.cumprod(mu)))
     return a, b, P_U, P_L, c
 
 

@@ -1,0 +1,41 @@
+// Shared device helpers of the E2-TTT chunk-scan library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace e2ttt {
+
+typedef __nv_bfloat16 bf16;
+
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<bf16>(bf16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+// silu(z) = z * sigmoid(z) and its first two derivatives (SwiGLU fast MLP).
+__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + expf(-z)); }
+__device__ __forceinline__ float silu_f(float z) { return z * sigmoid_f(z); }
+__device__ __forceinline__ float dsilu_f(float z) {
+  float s = sigmoid_f(z);
+  return s * (1.0f + z * (1.0f - s));
+}
+__device__ __forceinline__ float d2silu_f(float z) {
+  float s = sigmoid_f(z);
+  return s * (1.0f - s) * (2.0f + z * (1.0f - 2.0f * s));
+}
+
+// Sizes of one problem as the kernels see them.
+struct Dims {
+  int BH;      // batch rows x heads
+  int T, C, NC;
+  int d_k, d_v, d_h;
+  int kind, loss;
+  long long S; // state elements per head
+};
+
+}  // namespace e2ttt

@@ -1,0 +1,293 @@
+// K1: the two scalar kernels of E2-TTT and their adjoint.
+//
+// "Rethinking Expressivity and Efficiency in Test-Time Training", atlas.scime.ai
+// summary, "Approach": a momentum kernel and a weight kernel come from unrolling
+// the token-wise momentum-plus-decay recurrence and are computed with log-space
+// cumulative sums; arxivlens summary, "Results": the extra work is a log-space
+// suffix and ratio sums. Per chunk of n tokens (1-based t), with
+// U(i,j) = prod mu, L(i,j) = prod lam over tokens i..j:
+//   SU_t = sum_{s>t} log mu_s,  SL_t = sum_{s>t} log lam_s     (suffix log-sums)
+//   a_t  = eta_t exp(SU_t)                                     (momentum kernel)
+//   R_t  = exp(SL_t) + mu_{t+1} R_{t+1},  R_n = 1              (ratio sum; affine scan)
+//   b_t  = eta_t R_t                                           (weight kernel)
+//   U(1,n) = exp(SU_0), L(1,n) = exp(SL_0), c = mu_1 R_1        (chunk scalars)
+// No prefix sum is ever subtracted from another, so mu = 0 or lam = 0 (log = -inf)
+// gives exact zeros instead of NaN.
+//
+// Layout: one warp per (head, chunk); lane l owns a contiguous segment of
+// ceil(n/32) tokens; segment results are combined with warp shuffles.
+#include "common.cuh"
+
+namespace e2ttt {
+
+namespace {
+
+constexpr int kWarpsPerBlock = 4;
+
+__device__ __forceinline__ void seg_bounds(int n, int lane, int& s0, int& s1) {
+  int per = (n + 31) >> 5;
+  s0 = min(n, lane * per);
+  s1 = min(n, s0 + per);
+}
+
+// Inclusive suffix sum across lanes (lane l gets sum over lanes >= l).
+__device__ __forceinline__ float warp_suffix_sum(float x, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    float y = __shfl_down_sync(0xffffffffu, x, off);
+    if (lane + off < 32) x += y;
+  }
+  return x;
+}
+
+// Per chunk: exclusive suffix log-sums at the end of this lane's segment and
+// the chunk totals (lane-uniform).
+struct LogSums {
+  float su_excl, sl_excl;  // sum over tokens after this lane's segment
+  float su_all, sl_all;    // sum over the whole chunk
+};
+
+__device__ __forceinline__ LogSums chunk_log_sums(const float* mu, const float* lam, int s0, int s1,
+                                                  int lane) {
+  float su = 0.f, sl = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    su += logf(mu[t]);
+    sl += logf(lam[t]);
+  }
+  float su_inc = warp_suffix_sum(su, lane);
+  float sl_inc = warp_suffix_sum(sl, lane);
+  LogSums r;
+  r.su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
+  r.sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
+  if (lane == 31) { r.su_excl = 0.f; r.sl_excl = 0.f; }
+  r.su_all = __shfl_sync(0xffffffffu, su_inc, 0);
+  r.sl_all = __shfl_sync(0xffffffffu, sl_inc, 0);
+  return r;
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                    const float* __restrict__ decay, float* __restrict__ a_out,
+                    float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
+                    int NC) {
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (wid >= BH * NC) return;  // warp-uniform
+  const int bh = wid / NC, ci = wid % NC;
+  const int t0 = ci * C;
+  const int n = min(C, T - t0);
+  const size_t base = (size_t)bh * T + t0;
+  const float* eta = lr + base;
+  const float* mu = mom + base;
+  const float* lam = decay + base;
+  int s0, s1;
+  seg_bounds(n, lane, s0, s1);
+
+  LogSums ls = chunk_log_sums(mu, lam, s0, s1, lane);
+
+  // Reverse walk 1: momentum kernel a_t and the segment's ratio-sum map.
+  float su = ls.su_excl, sl = ls.sl_excl;
+  float Mseg = 1.f, Cseg = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    a_out[base + t] = eta[t] * expf(su);
+    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    Cseg = expf(sl) + m * Cseg;
+    Mseg = m * Mseg;
+    su += logf(mu[t]);
+    sl += logf(lam[t]);
+  }
+  float M = Mseg, Cc = Cseg;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    float Mr = __shfl_down_sync(0xffffffffu, M, off);
+    float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+    if (lane + off < 32) {
+      Cc = Cc + M * Cr;
+      M = M * Mr;
+    }
+  }
+  float r_next = __shfl_down_sync(0xffffffffu, Cc, 1);
+  if (lane == 31) r_next = 0.f;
+
+  // Reverse walk 2: R_t and the weight kernel b_t.
+  sl = ls.sl_excl;
+  float r1 = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float r = expf(sl) + m * r_next;
+    b_out[base + t] = eta[t] * r;
+    r_next = r;
+    if (t == 0) r1 = r;
+    sl += logf(lam[t]);
+  }
+  if (s0 == 0 && s1 > 0) {  // lane 0 holds token 1
+    const size_t plane = (size_t)BH * NC;
+    const size_t o = (size_t)bh * NC + ci;
+    scal[o] = expf(ls.su_all);
+    scal[plane + o] = expf(ls.sl_all);
+    scal[2 * plane + o] = mu[0] * r1;
+  }
+}
+
+// Adjoint of chunk_coeffs_kernel. Given abar, bbar (per token) and the chunk
+// scalar adjoints (PUbar, PLbar, cbar), with
+//   X_1 = PUbar, X_{s+1} = mu_s X_s + abar_s eta_s
+//   Y_1 = cbar,  Y_{s+1} = mu_s Y_s + bbar_s eta_s
+//   V_1 = PLbar, V_{s+1} = lam_s V_s + Y_{s+1}
+// the gate gradients are
+//   deta_t = abar_t U(t+1,n) + bbar_t R_t
+//   dmu_s  = U(s+1,n) X_s + R_s Y_s
+//   dlam_s = L(s+1,n) V_s
+// (derivatives of the product definitions with the factor s removed; no gate
+// is ever divided by). X and (Y, V) are forward affine scans.
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                        const float* __restrict__ decay, const float* __restrict__ abar,
+                        const float* __restrict__ bbar, const float* __restrict__ scal_bar,
+                        float* __restrict__ deta, float* __restrict__ dmu,
+                        float* __restrict__ dlam, int BH, int T, int C, int NC) {
+  extern __shared__ float sm[];
+  const int lane = threadIdx.x & 31;
+  const int wl = threadIdx.x >> 5;
+  const int wid = blockIdx.x * kWarpsPerBlock + wl;
+  if (wid >= BH * NC) return;
+  float* sR = sm + (size_t)wl * 3 * C;
+  float* sU = sR + C;
+  float* sL = sU + C;
+  const int bh = wid / NC, ci = wid % NC;
+  const int t0 = ci * C;
+  const int n = min(C, T - t0);
+  const size_t base = (size_t)bh * T + t0;
+  const float* eta = lr + base;
+  const float* mu = mom + base;
+  const float* lam = decay + base;
+  const float* ab = abar + base;
+  const float* bb = bbar + base;
+  int s0, s1;
+  seg_bounds(n, lane, s0, s1);
+  LogSums ls = chunk_log_sums(mu, lam, s0, s1, lane);
+
+  // Reverse walks: U(t+1,n), L(t+1,n), R_t into shared memory; deta.
+  float su = ls.su_excl, sl = ls.sl_excl;
+  float Mseg = 1.f, Cseg = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float cl = expf(sl);
+    sU[t] = expf(su);
+    sL[t] = cl;
+    Cseg = cl + m * Cseg;
+    Mseg = m * Mseg;
+    su += logf(mu[t]);
+    sl += logf(lam[t]);
+  }
+  float M = Mseg, Cc = Cseg;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    float Mr = __shfl_down_sync(0xffffffffu, M, off);
+    float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+    if (lane + off < 32) {
+      Cc = Cc + M * Cr;
+      M = M * Mr;
+    }
+  }
+  float r_next = __shfl_down_sync(0xffffffffu, Cc, 1);
+  if (lane == 31) r_next = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float r = sL[t] + m * r_next;
+    sR[t] = r;
+    deta[base + t] = ab[t] * sU[t] + bb[t] * r;
+    r_next = r;
+  }
+
+  // Forward scans. Segment maps: X -> pX X + uX ;  (Y, V) -> [[p,0],[q,r]] (Y,V) + (u,w).
+  float pX = 1.f, uX = 0.f;
+  float p = 1.f, q = 0.f, r = 1.f, u = 0.f, w = 0.f;
+  for (int s = s0; s < s1; ++s) {
+    float m_ = mu[s], l_ = lam[s];
+    float al = ab[s] * eta[s], be = bb[s] * eta[s];
+    uX = m_ * uX + al;
+    pX = m_ * pX;
+    float q2 = m_ * p + l_ * q;
+    float w2 = m_ * u + l_ * w + be;
+    p = m_ * p;
+    r = l_ * r;
+    u = m_ * u + be;
+    q = q2;
+    w = w2;
+  }
+  // inclusive prefix composition (later o earlier) across lanes
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    float pXe = __shfl_up_sync(0xffffffffu, pX, off);
+    float uXe = __shfl_up_sync(0xffffffffu, uX, off);
+    float pe = __shfl_up_sync(0xffffffffu, p, off);
+    float qe = __shfl_up_sync(0xffffffffu, q, off);
+    float re = __shfl_up_sync(0xffffffffu, r, off);
+    float ue = __shfl_up_sync(0xffffffffu, u, off);
+    float we = __shfl_up_sync(0xffffffffu, w, off);
+    if (lane >= off) {
+      // self o earlier
+      uX = pX * uXe + uX;
+      pX = pX * pXe;
+      float np = p * pe;
+      float nq = q * pe + r * qe;
+      float nr = r * re;
+      float nu = p * ue + u;
+      float nw = q * ue + r * we + w;
+      p = np; q = nq; r = nr; u = nu; w = nw;
+    }
+  }
+  // exclusive: the composition of all earlier lanes, applied to the initial values
+  float epX = __shfl_up_sync(0xffffffffu, pX, 1), euX = __shfl_up_sync(0xffffffffu, uX, 1);
+  float ep = __shfl_up_sync(0xffffffffu, p, 1), eq = __shfl_up_sync(0xffffffffu, q, 1);
+  float er = __shfl_up_sync(0xffffffffu, r, 1), eu = __shfl_up_sync(0xffffffffu, u, 1);
+  float ew = __shfl_up_sync(0xffffffffu, w, 1);
+  if (lane == 0) { epX = 1.f; euX = 0.f; ep = 1.f; eq = 0.f; er = 1.f; eu = 0.f; ew = 0.f; }
+  const size_t plane = (size_t)BH * NC;
+  const size_t o = (size_t)bh * NC + ci;
+  const float PUb = scal_bar[o], PLb = scal_bar[plane + o], cb = scal_bar[2 * plane + o];
+  float X = epX * PUb + euX;
+  float Y = ep * cb + eu;
+  float V = eq * cb + er * PLb + ew;
+  for (int s = s0; s < s1; ++s) {
+    dmu[base + s] = sU[s] * X + sR[s] * Y;
+    dlam[base + s] = sL[s] * V;
+    float m_ = mu[s], l_ = lam[s];
+    X = m_ * X + ab[s] * eta[s];
+    float Yn = m_ * Y + bb[s] * eta[s];
+    V = l_ * V + Yn;
+    Y = Yn;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
+                                float* b, float* scal, int BH, int T, int C, int NC,
+                                cudaStream_t st) {
+  int warps = BH * NC;
+  int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  chunk_coeffs_kernel<<<blocks, kWarpsPerBlock * 32, 0, st>>>(lr, mom, decay, a, b, scal, BH, T,
+                                                               C, NC);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const float* decay,
+                                    const float* abar, const float* bbar, const float* scal_bar,
+                                    float* deta, float* dmu, float* dlam, int BH, int T, int C,
+                                    int NC, cudaStream_t st) {
+  int warps = BH * NC;
+  int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  size_t smem = (size_t)kWarpsPerBlock * 3 * C * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(chunk_coeffs_bwd_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  chunk_coeffs_bwd_kernel<<<blocks, kWarpsPerBlock * 32, smem, st>>>(
+      lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC);
+  return cudaGetLastError();
+}
+
+}  // namespace e2ttt

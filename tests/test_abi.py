@@ -1,0 +1,96 @@
+"""The C ABI without a GPU: the library loads, exports every function the header
+declares, and rejects bad arguments on the host (no launch, nothing written)."""
+import ctypes
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "test_weight_layers_chunk_b200", "libe2ttt.so")
+
+
+@pytest.fixture(scope="module")
+def E():
+    if not os.path.exists(LIB):
+        from test_weight_layers_chunk_b200 import build as b
+        b.build()
+    import test_weight_layers_chunk_b200 as E
+    return E
+
+
+def test_exports_every_declared_symbol(E):
+    names = E.header_functions()
+    assert set(names) >= {"e2ttt_chunk_scan_fwd", "e2ttt_chunk_scan_bwd", "e2ttt_chunk_coeffs",
+                          "e2ttt_workspace_bytes", "e2ttt_state_elems", "e2ttt_status_string",
+                          "e2ttt_last_error", "e2ttt_num_chunks"}
+    lib = ctypes.CDLL(LIB)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_sizes(E):
+    s = E.make_shape(4, 8, 2048, 512, 256, 256, 512, E.SWIGLU, E.BF16)
+    assert E.e2ttt_state_elems(s) == 2 * 512 * 256 + 256 * 512
+    assert E.e2ttt_num_chunks(s) == 4
+    assert E.e2ttt_workspace_bytes(s, 0) > 0
+    lin = E.make_shape(1, 1, 256, 64, 32, 32, 0, E.LINEAR, E.F32)
+    assert E.e2ttt_state_elems(lin) == 32 * 32
+    assert E.e2ttt_num_chunks(E.make_shape(1, 1, 257, 64, 32, 32, 0, E.LINEAR, E.F32)) == 5
+    for bad in (E.make_shape(0, 1, 8, 4, 4, 4, 4), E.make_shape(1, 1, 8, 2048, 4, 4, 4),
+                E.make_shape(1, 1, 8, 4, 4, 4, 0, E.SWIGLU), E.make_shape(1, 1, 8, 4, 4, 4, 4, 7)):
+        assert E.e2ttt_state_elems(bad) == 0 and E.e2ttt_workspace_bytes(bad, 0) == 0
+
+
+def test_status_strings(E):
+    for s in range(5):
+        assert E.e2ttt_status_string(s).startswith("E2TTT_")
+
+
+FAKE = 1 << 40  # never dereferenced: every call below fails its host-side checks
+
+
+def _fwd(E, shape, **over):
+    S = max(E.e2ttt_state_elems(shape), 1)
+    n = 1 << 30
+    args = dict(q=FAKE, k=FAKE + n, v=FAKE + 2 * n, lr=FAKE + 3 * n, mom=FAKE + 4 * n,
+                decay=FAKE + 5 * n, W0=FAKE + 6 * n, M0=FAKE + 7 * n, out=FAKE + 8 * n,
+                W_end=FAKE + 9 * n, M_end=FAKE + 10 * n, saved_states=None, workspace=FAKE + 12 * n,
+                workspace_bytes=E.e2ttt_workspace_bytes(shape, 0))
+    args.update(over)
+    return E.e2ttt_chunk_scan_fwd(shape, raw=True, stream=None, **args)
+
+
+def test_fwd_rejects_bad_arguments(E):
+    s = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32)
+    for over in (dict(q=None), dict(W0=None), dict(out=None), dict(workspace=None),
+                 dict(workspace_bytes=16), dict(workspace=FAKE + 12 * (1 << 30) + 8),
+                 dict(out=FAKE + 7),                       # out overlaps q
+                 dict(W_end=FAKE + 6 * (1 << 30)),         # W_end aliases W0
+                 dict(M_end=FAKE + 9 * (1 << 30) + 4)):    # M_end overlaps W_end
+        assert _fwd(E, s, **over) == E.ERR_INVALID_ARG, over
+        assert E.e2ttt_last_error() != ""
+    bad = E.make_shape(1, 2, 64, 0, 8, 8, 16, E.SWIGLU, E.F32)
+    assert _fwd(E, bad) == E.ERR_INVALID_ARG
+    assert "sizes" in E.e2ttt_last_error()
+
+
+def test_bwd_rejects_bad_arguments(E):
+    s = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32)
+    n = 1 << 30
+    args = dict(q=FAKE, k=FAKE + n, v=FAKE + 2 * n, lr=FAKE + 3 * n, mom=FAKE + 4 * n,
+                decay=FAKE + 5 * n, saved_states=FAKE + 6 * n, dout=FAKE + 7 * n, dW_end=None,
+                dM_end=None, dq=FAKE + 8 * n, dk=FAKE + 9 * n, dv=FAKE + 10 * n, dlr=FAKE + 11 * n,
+                dmom=FAKE + 12 * n, ddecay=FAKE + 13 * n, dW0=FAKE + 14 * n, dM0=FAKE + 15 * n,
+                workspace=FAKE + 16 * n, workspace_bytes=E.e2ttt_workspace_bytes(s, 1))
+    for over in (dict(saved_states=None), dict(dq=None), dict(workspace_bytes=0),
+                 dict(dk=FAKE + 8 * n + 2)):
+        a = dict(args)
+        a.update(over)
+        assert E.e2ttt_chunk_scan_bwd(s, raw=True, stream=None, **a) == E.ERR_INVALID_ARG, over
+
+
+def test_coeffs_rejects_bad_arguments(E):
+    s = E.make_shape(1, 1, 64, 16, 8, 8, 0, E.LINEAR, E.F32)
+    assert E.e2ttt_chunk_coeffs(s, None, FAKE, FAKE, FAKE, FAKE, FAKE, raw=True) == E.ERR_INVALID_ARG
+    assert E.e2ttt_chunk_coeffs(s, FAKE, FAKE + 4096, FAKE + 8192, FAKE, FAKE + (1 << 20),
+                                FAKE + (1 << 21), raw=True) == E.ERR_INVALID_ARG  # a aliases lr
