@@ -86,6 +86,18 @@ WORKLOADS = [
 BY_NAME = {w.name: w for w in WORKLOADS}
 
 
+def state_preserving(w: Workload) -> Workload:
+    """The same shapes with gates that keep the fast-weight state O(1) over many
+    chunks: lr ~ U(0.002, 0.02), decay ~ U(0.999, 1) (momentum unchanged).
+
+    With the stated distributions (decay ~ U(0.95, 1) over 256-512 token chunks)
+    the per-chunk decay product is about e^-13, so the SwiGLU state collapses to
+    the W = 0 fixed point within two or three chunks and later chunks carry
+    little signal. Parity tests run both variants."""
+    return w.replace(name=w.name + "_preserving", lr_dist="uniform", lr_lo=0.002, lr_hi=0.02,
+                     decay_lo=max(w.decay_lo, 0.999))
+
+
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding bf16 values."""
     x = np.ascontiguousarray(x, dtype=np.float32)

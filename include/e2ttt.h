@@ -95,6 +95,11 @@ size_t e2ttt_workspace_bytes(const e2ttt_shape* shape, int for_bwd);
 /* Number of chunks, ceil(T / C); 0 for an invalid shape. */
 int e2ttt_num_chunks(const e2ttt_shape* shape);
 
+/* 1 if e2ttt_chunk_scan_fwd runs `shape` on the tcgen05 tensor cores (given
+ * 16-byte aligned pointers), 0 if on the fp32 CUDA-core kernels, -1 if the
+ * shape is invalid. */
+int e2ttt_fwd_uses_tensor_cores(const e2ttt_shape* shape);
+
 /* The two scalar kernels of every chunk (atlas.scime.ai summary, "Approach":
  * momentum kernel and weight kernel from unrolling the token-wise
  * momentum-plus-decay recurrence, via log-space cumulative sums; arxivlens
@@ -147,6 +152,13 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
                                   float* dW0, float* dM0,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream);
+
+/* Status of the device-side bounded waits of the last compute call that used
+ * `workspace`: synchronizes `stream`, then returns E2TTT_ERR_TIMEOUT if a
+ * tensor-core kernel gave up waiting (its outputs are then invalid; the CUDA
+ * context stays usable), else E2TTT_OK. The status word is the first 4 bytes
+ * of the workspace and is reset by every compute call. */
+e2ttt_status e2ttt_workspace_status(const void* workspace, void* stream);
 
 /* Static description of a status code. */
 const char* e2ttt_status_string(e2ttt_status status);

@@ -11,7 +11,7 @@ The functions named e2ttt_* mirror the C entry points of include/e2ttt.h one to
 one: they only marshal arguments (torch tensors or raw device pointers) and
 raise E2TTTError on a non-zero status. All computation happens in the CUDA
 library; there is no Python or CPU fallback, and importing this package fails
-if the library has not been built (python -m test_weight_layers_chunk_b200.build).
+if the library has not been built (python test_weight_layers_chunk_b200/build.py).
 chunk_scan_fwd / chunk_scan_bwd are conveniences that allocate the outputs and
 the workspace with torch and call the same entry points.
 """
@@ -44,7 +44,7 @@ class E2TTTError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      f"`python -m test_weight_layers_chunk_b200.build` (needs nvcc)")
+                      f"`python test_weight_layers_chunk_b200/build.py` (needs nvcc)")
 _lib = ctypes.CDLL(LIB_PATH)
 
 _P = ctypes.c_void_p
@@ -53,9 +53,11 @@ _SIGS = {
     "e2ttt_state_elems": (ctypes.c_size_t, [_S]),
     "e2ttt_workspace_bytes": (ctypes.c_size_t, [_S, ctypes.c_int]),
     "e2ttt_num_chunks": (ctypes.c_int, [_S]),
+    "e2ttt_fwd_uses_tensor_cores": (ctypes.c_int, [_S]),
     "e2ttt_chunk_coeffs": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "e2ttt_chunk_scan_fwd": (ctypes.c_int, [_S] + [_P] * 13 + [ctypes.c_size_t, _P]),
     "e2ttt_chunk_scan_bwd": (ctypes.c_int, [_S] + [_P] * 19 + [ctypes.c_size_t, _P]),
+    "e2ttt_workspace_status": (ctypes.c_int, [_P, _P]),
     "e2ttt_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "e2ttt_last_error": (ctypes.c_char_p, []),
 }
@@ -106,6 +108,13 @@ def e2ttt_last_error() -> str:
     return _lib.e2ttt_last_error().decode()
 
 
+def e2ttt_workspace_status(workspace, stream=None, raw=False):
+    st = _lib.e2ttt_workspace_status(_ptr(workspace), _stream(stream) if not raw else stream)
+    if raw:
+        return st
+    _check(st)
+
+
 def e2ttt_state_elems(shape: e2ttt_shape) -> int:
     return _lib.e2ttt_state_elems(ctypes.byref(shape))
 
@@ -116,6 +125,10 @@ def e2ttt_workspace_bytes(shape: e2ttt_shape, for_bwd: int = 0) -> int:
 
 def e2ttt_num_chunks(shape: e2ttt_shape) -> int:
     return _lib.e2ttt_num_chunks(ctypes.byref(shape))
+
+
+def e2ttt_fwd_uses_tensor_cores(shape: e2ttt_shape) -> int:
+    return _lib.e2ttt_fwd_uses_tensor_cores(ctypes.byref(shape))
 
 
 def e2ttt_chunk_coeffs(shape, lr, mom, decay, a, b, chunk_scalars, stream=None, raw=False):

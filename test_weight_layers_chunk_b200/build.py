@@ -1,6 +1,8 @@
 """Build the E2-TTT chunk-scan library (libe2ttt.so) for sm_100a with nvcc.
 
-    python -m test_weight_layers_chunk_b200.build [--debug] [-v]
+    python test_weight_layers_chunk_b200/build.py [--debug] [-v]
+
+(run by path: importing the package itself needs the built library)
 
 Each csrc/*.cu compiles to an object under _build/ (in parallel), then links
 into test_weight_layers_chunk_b200/libe2ttt.so with the CUDA runtime linked
@@ -37,6 +39,15 @@ def flags(debug: bool) -> list[str]:
     if debug:
         f += ["-DE2TTT_DEBUG=1"]
     return f
+
+
+def load_builder():
+    """This module, loaded by file path without importing the package."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_e2ttt_build", os.path.abspath(__file__))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
 
 
 def build(debug: bool = False, verbose: bool = False) -> str:

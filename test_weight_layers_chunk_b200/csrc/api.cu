@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <cstdio>
+#include <initializer_list>
 #include <string>
 
 #include "../../include/e2ttt.h"
@@ -83,28 +84,43 @@ struct Bump {
 };
 
 struct FwdWs {
+  size_t status;                    // device status word (bounded waits)
   size_t a, b, scal, st, H, E, dH;  // fp32 CUDA-core path
   size_t tc;                        // tensor-core path scratch
   size_t total;
 };
 
-FwdWs fwd_layout(const Dims& d, bool tc) {
+// Coefficients and one spare state pair, then one region shared by the
+// tensor-core scratch and the CUDA-core scratch (only one path runs per call).
+FwdWs fwd_layout(const Dims& d, bool tc_shape) {
   Bump w;
   FwdWs L{};
   const size_t f = sizeof(float);
+  L.status = w.take(256);
   L.a = w.take((size_t)d.BH * d.T * f);
   L.b = w.take((size_t)d.BH * d.T * f);
   L.scal = w.take((size_t)3 * d.BH * d.NC * f);
   L.st = w.take((size_t)2 * d.BH * d.S * f);
-  if (tc) {
-    L.tc = w.take(tc_fwd_scratch_bytes(d));
-  } else {
-    if (d.kind == 1) L.H = w.take((size_t)d.BH * 2 * d.C * 2 * d.d_h * f);
-    L.E = w.take((size_t)d.BH * d.C * d.d_v * f);
-    if (d.kind == 1) L.dH = w.take((size_t)d.BH * d.C * 2 * d.d_h * f);
+  const size_t region = w.off;
+  Bump s;
+  s.off = region;
+  if (d.kind == 1) L.H = s.take((size_t)d.BH * 2 * d.C * 2 * d.d_h * f);
+  L.E = s.take((size_t)d.BH * d.C * d.d_v * f);
+  if (d.kind == 1) L.dH = s.take((size_t)d.BH * d.C * 2 * d.d_h * f);
+  size_t end = s.off;
+  L.tc = region;
+  if (tc_shape) {
+    size_t tend = align_up(region + tc_fwd_scratch_bytes(d));
+    if (tend > end) end = tend;
   }
-  L.total = w.off;
+  L.total = end;
   return L;
+}
+
+bool aligned16(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (((uintptr_t)p) & 15) return false;
+  return true;
 }
 
 struct Range {
@@ -149,6 +165,12 @@ int e2ttt_num_chunks(const e2ttt_shape* s) {
   return make_dims(s).NC;
 }
 
+int e2ttt_fwd_uses_tensor_cores(const e2ttt_shape* s) {
+  std::string why;
+  if (!shape_ok(s, &why)) return -1;
+  return tc_fwd_supported(make_dims(s), s->act == E2TTT_BF16) ? 1 : 0;
+}
+
 size_t e2ttt_workspace_bytes(const e2ttt_shape* s, int for_bwd) {
   std::string why;
   if (!shape_ok(s, &why)) return 0;
@@ -169,6 +191,18 @@ const char* e2ttt_status_string(e2ttt_status st) {
 }
 
 const char* e2ttt_last_error(void) { return g_last_error.c_str(); }
+
+e2ttt_status e2ttt_workspace_status(const void* ws, void* stream) {
+  g_last_error.clear();
+  if (!ws) return fail(E2TTT_ERR_INVALID_ARG, "workspace is NULL");
+  int word = 0;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status word");
+  if (word != 0)
+    return fail(E2TTT_ERR_TIMEOUT, "a device-side wait gave up (code %d: 1 = TMA producer, 2 = MMA issuer, 3 = epilogue)", word);
+  return E2TTT_OK;
+}
 
 e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* s, const float* lr, const float* mom,
                                 const float* decay, float* a, float* b, float* scal,
@@ -201,8 +235,9 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
     return fail(E2TTT_ERR_INVALID_ARG, "e2ttt_chunk_scan_fwd: NULL pointer argument (only M0 and saved_states may be NULL)");
   Dims d = make_dims(s);
   const bool bf = s->act == E2TTT_BF16;
-  const bool tc = tc_fwd_supported(d, bf);
-  FwdWs L = fwd_layout(d, tc);
+  const bool tc_shape = tc_fwd_supported(d, bf);
+  FwdWs L = fwd_layout(d, tc_shape);
+  const bool tc = tc_shape && aligned16({q, k, v, out, W0, M0, W_end, M_end, saved});
   if (!ws) return fail(E2TTT_ERR_INVALID_ARG, "workspace is NULL (needs %zu bytes)", L.total);
   if (ws_bytes < L.total)
     return fail(E2TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.total);
@@ -222,11 +257,14 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   float* cb = (float*)(w + L.b);
   float* scal = (float*)(w + L.scal);
   float* stbuf = (float*)(w + L.st);
-  cudaError_t e = launch_chunk_coeffs(lr, mom, decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, st);
+  int* status = (int*)(w + L.status);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "status word reset");
+  e = launch_chunk_coeffs(lr, mom, decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, st);
   if (e != cudaSuccess) return cuda_fail(e, "chunk coefficient kernel");
   if (tc) {
     e = tc_fwd(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal, W0, M0,
-               W_end, M_end, saved, stbuf, w + L.tc, st);
+               W_end, M_end, saved, stbuf, w + L.tc, status, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward");
     return E2TTT_OK;
   }

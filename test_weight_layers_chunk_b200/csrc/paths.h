@@ -29,7 +29,7 @@ size_t tc_fwd_scratch_bytes(const Dims& d);
 cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, bf16* out,
                    const float* ca, const float* cb, const float* scal, const float* W0,
                    const float* M0, float* W_end, float* M_end, float* saved, float* stbuf,
-                   void* scratch, cudaStream_t st);
+                   void* scratch, int* status, cudaStream_t st);
 
 // Backward (bwd.cu).
 struct BwdArgs {

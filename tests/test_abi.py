@@ -12,8 +12,12 @@ LIB = os.path.join(ROOT, "test_weight_layers_chunk_b200", "libe2ttt.so")
 @pytest.fixture(scope="module")
 def E():
     if not os.path.exists(LIB):
-        from test_weight_layers_chunk_b200 import build as b
-        b.build()
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(
+            "_e2ttt_build", os.path.join(ROOT, "test_weight_layers_chunk_b200", "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
     import test_weight_layers_chunk_b200 as E
     return E
 

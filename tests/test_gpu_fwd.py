@@ -98,9 +98,10 @@ F32_CASES = {
     "linear_ragged": gen.Workload("lr", gen.LINEAR, gen.F32, 2, 3, 40, 24, 0, 203, 48, "uniform",
                                   0.99, seed=11),
     "swiglu_f32": gen.Workload("sf", gen.SWIGLU, gen.F32, 2, 2, 24, 20, 40, 100, 32, "uniform",
-                               0.995, seed=12),
+                               0.99, seed=12, lr_lo=0.002, lr_hi=0.02),
     "swiglu_f32_dot": gen.Workload("sd", gen.SWIGLU, gen.F32, 1, 2, 16, 16, 32, 96, 32, "uniform",
-                                   0.995, seed=13, loss=gen.LOSS_NEG_DOT),
+                                   0.99, seed=13, loss=gen.LOSS_NEG_DOT, lr_lo=0.0005, lr_hi=0.005,
+                                   mom_lo=0.5, mom_hi=0.9),
 }
 
 
@@ -122,7 +123,8 @@ def test_fwd_f32_matches_oracle(E, name):
 
 def test_fwd_bf16_untiled_shape_matches_oracle(E):
     """bf16 activations on a shape the tensor-core path does not tile."""
-    w = gen.Workload("bu", gen.SWIGLU, gen.BF16, 1, 3, 48, 40, 72, 150, 64, "uniform", 0.995, seed=14)
+    w = gen.Workload("bu", gen.SWIGLU, gen.BF16, 1, 3, 48, 40, 72, 150, 64, "uniform", 0.99, seed=14,
+                     lr_lo=0.002, lr_hi=0.02)
     x = gen.generate(w, m0_scale=0.5)
     out, W_end, M_end, _ = run_fwd(E, w, device_inputs(w, x))
     ro, rW, rM, _ = oracle_fwd(w, x)
@@ -135,7 +137,7 @@ def test_fwd_bf16_untiled_shape_matches_oracle(E):
 STRUCT_CASES = {
     "f32": F32_CASES["swiglu_f32"],
     "bf16_tc": gen.Workload("bt", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform",
-                            0.999, seed=15),
+                            0.999, seed=15, lr_lo=0.002, lr_hi=0.02),
 }
 
 
