@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Throughput of the E2-TTT chunk-parallel closed-form fast-weight update on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload layer_1p3b_2k] [--mode fwd|train]
+
+One step = one e2ttt_chunk_scan_fwd call (mode train: forward then
+e2ttt_chunk_scan_bwd) over the whole workload, inputs resident in HBM. The
+default workload is the 1.3B-shaped layer (B=4, H=8 heads of 256, SwiGLU fast
+hidden 512, T=2048, C=512) with seeded synthetic inputs. The working set
+(inputs, fp32 state, workspace) is larger than the 126 MB L2, so no flush is
+needed between steps. Time is taken with CUDA events on the launch stream,
+max over ranks. Prints one JSON line (rank 0).
+
+N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
+workload (independent batch rows, no collective on the data path; weak
+scaling); the only collectives are the timing barrier and the max over ranks.
+
+--impl reference: the fp64 CPU oracle (closed form) on a bounded sample of the
+same workload, timed on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import e2ttt_inputs as gen  # noqa: E402
+
+METRIC = "E2-TTT layer tokens/sec (fwd, fwd+bwd) at T=2K/16K; % of bf16 TC roofline"
+UNIT = "tokens/s"
+KERNEL_SOURCES = ["test_weight_layers_chunk_b200/csrc/tc_gemm.cuh",
+                  "test_weight_layers_chunk_b200/csrc/tc_fwd.cu"]
+
+
+# ----------------------------------------------------------------- algorithmic work
+def phase_flops_per_token_head(w) -> dict:
+    """Algorithmic FLOPs per token and head of each forward GEMM phase."""
+    dk, dv, dh = w.d_k, w.d_v, w.d_h
+    if w.kind == gen.LINEAR:
+        return {"tc_g1_linear_out_e": 4 * dk * dv, "tc_g4_aggregate_state": 4 * dv * dk}
+    return {"tc_g1_h_act": 8 * dk * dh,            # [q; k] x [W1; W3]^T
+            "tc_g2_y_out_e": 4 * dh * dv,          # [A_q; A_k] x W2^T
+            "tc_g3_da_dh": 2 * dv * dh,            # E x W2
+            "tc_g4_aggregate_state": 8 * dh * dk + 4 * dv * dh}  # two aggregations x 3 matrices
+
+
+def fwd_flops(w) -> float:
+    return float(sum(phase_flops_per_token_head(w).values())) * w.B * w.H * w.T
+
+
+def algorithmic_bytes(w) -> float:
+    """q, k, v, out once (act dtype), gates, W0/M0 in and W_end/M_end out (fp32)."""
+    es = 2 if w.act == gen.BF16 else 4
+    toks = w.B * w.H * w.T
+    return toks * (2 * w.d_k + 2 * w.d_v) * es + toks * 12 + 4 * w.B * w.H * w.state_elems * 4
+
+
+# ----------------------------------------------------------------- environment
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel, if it
+    was taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    tb = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not sha or not tb or sha.group(1) != kernel_source_sha():
+        return None
+    return float(tb.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+def oracle_sample(w, x, budget_s: float, max_heads=None):
+    """Run the fp64 closed-form oracle head by head until `budget_s` is spent.
+    Returns (layer tokens processed, seconds, heads, threads)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if max_heads:
+        heads = heads[:max_heads]
+    done = 0
+    t0 = time.perf_counter()
+    for hh in heads:
+        O.closed_fwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"],
+                     x["M0"], w.C, d_h=w.d_h, loss=w.loss, heads=[hh])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done * w.T / w.H, dt, done, threads
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    x = gen.generate(w)
+    for _ in range(args.warmup):
+        oracle_sample(w, x, 0.0, max_heads=1)
+    tok = 0.0
+    t0 = time.perf_counter()
+    threads = 1
+    for _ in range(args.steps):
+        t, _, _, threads = oracle_sample(w, x, 0.0, max_heads=1)
+        tok += t
+    dt = time.perf_counter() - t0
+    v = tok / dt
+    sample = f"closed-form fp64 oracle, 1 of {w.B * w.H} heads x {w.T} tokens per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, args),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+
+
+def config_dict(w, args):
+    return {"workload": w.name, "kind": "swiglu" if w.kind == gen.SWIGLU else "linear",
+            "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "d_h": w.d_h, "T": w.T, "C": w.C,
+            "global_batch": w.B * args.gpus, "seq_len": w.T, "mode": args.mode,
+            "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
+            "l2": "working set larger than L2 (no flush)"}
+
+
+# ----------------------------------------------------------------- our path
+def run_ours(args, w):
+    import torch
+    import test_weight_layers_chunk_b200 as E
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xs = gen.generate(w)
+        tok, dt, nh, threads = oracle_sample(w, xs, args.cpu_budget)
+        cpu_baseline = {"value": tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+                        "sample": f"closed-form fp64 oracle on {nh} of {w.B * w.H} heads "
+                                  f"x {w.T} tokens ({dt:.1f} s)"}
+        del xs
+
+    x = gen.generate(w, seed=w.seed + 1000 * rank)
+    ad = torch.bfloat16 if w.act == gen.BF16 else torch.float32
+    f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
+    q, k, v = f(x["q"], ad), f(x["k"], ad), f(x["v"], ad)
+    lr, mom, decay, W0 = f(x["lr"]), f(x["mom"]), f(x["decay"]), f(x["W0"])
+    M0 = None if not np.any(x["M0"]) else f(x["M0"])   # the workload's M0 is zero
+    shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss)
+    assert E.e2ttt_fwd_uses_tensor_cores(shape) == 1
+    nc = E.e2ttt_num_chunks(shape)
+    out = torch.empty_like(v)
+    W_end = torch.empty_like(W0)
+    M_end = torch.empty_like(W0)
+    train = args.mode == "train"
+    saved = torch.empty((nc, w.B, w.H, 2, w.state_elems), device=dev) if train else None
+    ws = E.workspace(shape, False, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, M0, out, W_end, M_end, saved, ws,
+                               stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    E.e2ttt_workspace_status(ws, stream=stream)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    E.e2ttt_trace_enable(True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    trace = E.e2ttt_trace_summary()
+    E.e2ttt_trace_enable(False)
+    if world > 1:
+        torch.distributed.barrier()
+    E.e2ttt_workspace_status(ws, stream=stream)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world, dev)
+    tokens = w.B * w.T * args.steps * world
+    value = tokens / (ms_max / 1e3)
+
+    # roofline of the dominant kernel
+    peaks = measured_peaks()
+    ph = phase_flops_per_token_head(w)
+    kern = trace["kernels"]
+    dom = max((n for n in kern if n in ph), key=lambda n: kern[n]["total_ms"])
+    avg_ms = kern[dom]["total_ms"] / kern[dom]["launches"]
+    flops_launch = ph[dom] * w.B * w.H * w.C   # one launch = one chunk of every head
+    achieved = flops_launch / (avg_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": peaks["source"] + " (burst bf16 GEMM)",
+                "traffic": recorded_traffic(dom, w.name),
+                "share_of_step": kern[dom]["total_ms"] / ms}
+    step_flops = fwd_flops(w)
+    whole = {"achieved_tflops": step_flops / (ms / args.steps / 1e3) / 1e12}
+    whole["frac"] = whole["achieved_tflops"] / peaks["bf16_tflops"]
+    kernels = {n: {"launches": kv["launches"], "avg_us": 1e3 * kv["total_ms"] / kv["launches"],
+                   "share": kv["total_ms"] / ms} for n, kv in kern.items()}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hlr, hmom, hdec, hW0 = (t.cpu().pin_memory() for t in (lr, mom, decay, W0))
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hWe = torch.empty(W_end.shape, dtype=torch.float32, pin_memory=True)
+        hMe = torch.empty(M_end.shape, dtype=torch.float32, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hlr, hmom, hdec, hW0))
+        d2h = sum(t.numel() * t.element_size() for t in (hout, hWe, hMe))
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (lr, hlr), (mom, hmom), (decay, hdec),
+                             (W0, hW0)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+            hWe.copy_(W_end, non_blocking=True)
+            hMe.copy_(M_end, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+        e2e = {"value": w.B * w.T * args.e2e_steps * world / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if w.act == gen.BF16 else "f32",
+                "data": "synthetic (seeded numpy; shapes and distributions of the workload)",
+                "config": config_dict(w, argparse.Namespace(gpus=world, mode=args.mode)),
+                "roofline": roofline, "step_roofline": whole, "kernels": kernels,
+                "gpu_launches": trace["launches"], "clocks": clk.summary(),
+                "cpu_baseline": cpu_baseline, "e2e": e2e}
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="layer_1p3b_2k", choices=[w.name for w in gen.WORKLOADS])
+    ap.add_argument("--mode", choices=["fwd", "train"], default="fwd")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = gen.BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -160,6 +160,16 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
  * of the workspace and is reset by every compute call. */
 e2ttt_status e2ttt_workspace_status(const void* workspace, void* stream);
 
+/* Launch tracing. While enabled, every kernel the library launches is
+ * bracketed by a pair of CUDA events recorded on its launch stream (events are
+ * created by the library and reused; no device memory is allocated).
+ * e2ttt_trace_enable(1) starts a fresh record, (0) stops and discards it.
+ * e2ttt_trace_summary() waits for the recorded events, returns a JSON object
+ * {"launches": N, "kernels": {name: {"launches": n, "total_ms": t}}} and
+ * starts a fresh record; the string stays valid until the next call. */
+void e2ttt_trace_enable(int on);
+const char* e2ttt_trace_summary(void);
+
 /* Static description of a status code. */
 const char* e2ttt_status_string(e2ttt_status status);
 

@@ -60,6 +60,8 @@ _SIGS = {
     "e2ttt_workspace_status": (ctypes.c_int, [_P, _P]),
     "e2ttt_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "e2ttt_last_error": (ctypes.c_char_p, []),
+    "e2ttt_trace_enable": (None, [ctypes.c_int]),
+    "e2ttt_trace_summary": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -113,6 +115,15 @@ def e2ttt_workspace_status(workspace, stream=None, raw=False):
     if raw:
         return st
     _check(st)
+
+
+def e2ttt_trace_enable(on: bool = True) -> None:
+    _lib.e2ttt_trace_enable(int(bool(on)))
+
+
+def e2ttt_trace_summary() -> dict:
+    import json
+    return json.loads(_lib.e2ttt_trace_summary().decode())
 
 
 def e2ttt_state_elems(shape: e2ttt_shape) -> int:

@@ -17,6 +17,7 @@
 // Layout: one warp per (head, chunk); lane l owns a contiguous segment of
 // ceil(n/32) tokens; segment results are combined with warp shuffles.
 #include "common.cuh"
+#include "trace.h"
 
 namespace e2ttt {
 
@@ -268,6 +269,7 @@ cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* 
                                 cudaStream_t st) {
   int warps = BH * NC;
   int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  E2TTT_TRACE("k1_chunk_coeffs", st);
   chunk_coeffs_kernel<<<blocks, kWarpsPerBlock * 32, 0, st>>>(lr, mom, decay, a, b, scal, BH, T,
                                                                C, NC);
   return cudaGetLastError();
@@ -285,6 +287,7 @@ cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const flo
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
+  E2TTT_TRACE("k1_chunk_coeffs_bwd", st);
   chunk_coeffs_bwd_kernel<<<blocks, kWarpsPerBlock * 32, smem, st>>>(
       lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC);
   return cudaGetLastError();

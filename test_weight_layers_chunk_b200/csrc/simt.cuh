@@ -9,6 +9,7 @@
 // tensor-core path does not tile.
 #pragma once
 #include "common.cuh"
+#include "trace.h"
 
 namespace e2ttt {
 
@@ -84,8 +85,10 @@ simt_gemm_kernel(int M, int N, int K, LA la, LB lb, SC sc, EPI epi) {
 }
 
 template <int NACC, class LA, class LB, class SC, class EPI>
-cudaError_t simt_gemm(int Z, int M, int N, int K, LA la, LB lb, SC sc, EPI epi, cudaStream_t st) {
+cudaError_t simt_gemm(int Z, int M, int N, int K, LA la, LB lb, SC sc, EPI epi, cudaStream_t st,
+                      const char* name = "simt_gemm") {
   if (M <= 0 || N <= 0 || Z <= 0) return cudaSuccess;
+  E2TTT_TRACE(name, st);
   dim3 grid((N + kSimtBN - 1) / kSimtBN, (M + kSimtBM - 1) / kSimtBM, Z);
   simt_gemm_kernel<NACC><<<grid, 256, 0, st>>>(M, N, K, la, lb, sc, epi);
   return cudaGetLastError();

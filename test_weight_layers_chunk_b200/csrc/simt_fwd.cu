@@ -66,7 +66,15 @@ template <typename TA> struct LoadAct {
     return silu_f(h[j]) * h[c.d.d_h + j];
   }
 };
-// For the aggregations, A(i, t) = L[t, i] with L [n, ld] per head in workspace
+// A(t, kk) = L[t, kk] with L [C, ld] per head in workspace
+template <typename TA> struct LoadRow {
+  const float* base;
+  int C, ld;
+  __device__ __forceinline__ float operator()(int z, int t, int kk) const {
+    return base[((size_t)z * C + t) * ld + kk];
+  }
+};
+// For the aggregations, A(i, t) = L[t, i] with L [C, ld] per head in workspace
 template <typename TA> struct LoadTok {
   const float* base;
   int C, ld;
@@ -145,26 +153,26 @@ cudaError_t fwd_chunk(const Fwd<TA>& c, cudaStream_t st) {
   cudaError_t e;
   if (d.kind == 0) {
     e = simt_gemm<1>(d.BH, 2 * n, d.d_v, d.d_k, LoadX<TA>{c}, LoadWT<TA>{c, 0, d.d_k}, UnitScale{},
-                     EpiOutE<TA>{c}, st);
+                     EpiOutE<TA>{c}, st, "simt_linear_out_e");
     if (e != cudaSuccess) return e;
     return simt_gemm<2>(d.BH, d.d_v, d.d_k, n, LoadTok<TA>{c.E, d.C, d.d_v}, LoadK<TA>{c},
-                        ScaleAB<TA>{c}, EpiState<TA>{c, 0, d.d_k}, st);
+                        ScaleAB<TA>{c}, EpiState<TA>{c, 0, d.d_k}, st, "simt_aggregate_state");
   }
   const long long o2 = 2LL * d.d_h * d.d_k;
   e = simt_gemm<1>(d.BH, 2 * n, 2 * d.d_h, d.d_k, LoadX<TA>{c}, LoadWT<TA>{c, 0, d.d_k},
-                   UnitScale{}, EpiStoreH<TA>{c}, st);
+                   UnitScale{}, EpiStoreH<TA>{c}, st, "simt_g1_h");
   if (e != cudaSuccess) return e;
   e = simt_gemm<1>(d.BH, 2 * n, d.d_v, d.d_h, LoadAct<TA>{c, 0}, LoadWT<TA>{c, o2, d.d_h},
-                   UnitScale{}, EpiOutE<TA>{c}, st);
+                   UnitScale{}, EpiOutE<TA>{c}, st, "simt_g2_y_out_e");
   if (e != cudaSuccess) return e;
-  e = simt_gemm<1>(d.BH, n, d.d_h, d.d_v, LoadTok<TA>{c.E, d.C, d.d_v}, LoadW<TA>{c, o2, d.d_h},
-                   UnitScale{}, EpiDH<TA>{c}, st);
+  e = simt_gemm<1>(d.BH, n, d.d_h, d.d_v, LoadRow<TA>{c.E, d.C, d.d_v}, LoadW<TA>{c, o2, d.d_h},
+                   UnitScale{}, EpiDH<TA>{c}, st, "simt_g3_da_dh");
   if (e != cudaSuccess) return e;
   e = simt_gemm<2>(d.BH, 2 * d.d_h, d.d_k, n, LoadTok<TA>{c.dH, d.C, 2 * d.d_h}, LoadK<TA>{c},
-                   ScaleAB<TA>{c}, EpiState<TA>{c, 0, d.d_k}, st);
+                   ScaleAB<TA>{c}, EpiState<TA>{c, 0, d.d_k}, st, "simt_g4_aggregate_w13");
   if (e != cudaSuccess) return e;
   return simt_gemm<2>(d.BH, d.d_v, d.d_h, n, LoadTok<TA>{c.E, d.C, d.d_v}, LoadActK<TA>{c},
-                      ScaleAB<TA>{c}, EpiState<TA>{c, o2, d.d_h}, st);
+                      ScaleAB<TA>{c}, EpiState<TA>{c, o2, d.d_h}, st, "simt_g4_aggregate_w2");
 }
 
 }  // namespace

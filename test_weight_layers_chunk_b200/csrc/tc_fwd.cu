@@ -22,6 +22,7 @@
 #include "paths.h"
 #include "state.cuh"
 #include "tc_gemm.cuh"
+#include "trace.h"
 
 namespace e2ttt {
 namespace {
@@ -348,6 +349,13 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <class Epi> struct EpiName;
+template <> struct EpiName<struct EpiG1> { static constexpr const char* v = "tc_g1_h_act"; };
+template <> struct EpiName<struct EpiG2> { static constexpr const char* v = "tc_g2_y_out_e"; };
+template <> struct EpiName<struct EpiG3> { static constexpr const char* v = "tc_g3_da_dh"; };
+template <> struct EpiName<struct EpiG4> { static constexpr const char* v = "tc_g4_aggregate_state"; };
+template <> struct EpiName<struct EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
+
 template <int BN, int NUM_A, int STAGES, class Epi>
 cudaError_t launch(const tc::Job& job, const FwdP& p, cudaStream_t st) {
   constexpr size_t smem = tc::smem_bytes<BN, NUM_A, STAGES>();
@@ -357,6 +365,7 @@ cudaError_t launch(const tc::Job& job, const FwdP& p, cudaStream_t st) {
   if (attr != cudaSuccess) return attr;
   int tiles = 0;
   for (int c = 0; c < job.n_cls; ++c) tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
+  E2TTT_TRACE(EpiName<Epi>::v, st);
   kern<<<tiles, kThreads, smem, st>>>(job, p);
   return cudaGetLastError();
 }
@@ -431,8 +440,14 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
 
   cudaError_t e = save_initial_state(d, W0, M0, saved, st);
   if (e != cudaSuccess) return e;
-  transpose_keys_kernel<<<dim3(T / 32, dk / 32, BH), dim3(32, 8), 0, st>>>(k, s.KT, T, C, NC, dk);
-  shadow_init_kernel<<<1184, 256, 0, st>>>(p, W0);
+  {
+    E2TTT_TRACE("tc_transpose_keys", st);
+    transpose_keys_kernel<<<dim3(T / 32, dk / 32, BH), dim3(32, 8), 0, st>>>(k, s.KT, T, C, NC, dk);
+  }
+  {
+    E2TTT_TRACE("tc_shadow_init", st);
+    shadow_init_kernel<<<1184, 256, 0, st>>>(p, W0);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
