@@ -133,6 +133,31 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* shape,
                                   void* workspace, size_t workspace_bytes,
                                   void* stream);
 
+/* e2ttt_chunk_scan_fwd for callers that cannot allocate device memory: the
+ * same forward, same arguments minus the workspace, with the scratch taken from
+ * a 32 MiB array owned by the library (no counterpart in the paper; this is a
+ * deployment convenience). Callers such as applications whose device memory is
+ * already claimed by their own pool allocator, C hosts without a device
+ * allocator, or loops that cannot afford cudaMalloc's implicit synchronisation
+ * use it instead of providing a workspace.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The array lives in device memory of every GPU on which the library's
+ *     kernels are loaded, for the life of the process.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Shapes whose workspace (e2ttt_workspace_bytes(shape, 0)) exceeds 32 MiB
+ *     return E2TTT_ERR_INVALID_ARG with the sizes in e2ttt_last_error(); the
+ *     tiny linear and the d=128 SwiGLU workloads fit, the 1.3B layer does not.
+ *   - All calls share the array and it keeps the last call's contents; calls
+ *     that overlap on the GPU (several streams or host threads) race on it and
+ *     must be serialised by the caller. */
+e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
+                                          const void* q, const void* k, const void* v,
+                                          const float* lr, const float* mom, const float* decay,
+                                          const float* W0, const float* M0,
+                                          void* out, float* W_end, float* M_end,
+                                          float* saved_states, void* stream);
+
 /* Backward of e2ttt_chunk_scan_fwd for the scalar objective
  *     L = sum_t <dout_t, out_t> + <dW_end, W_end> + <dM_end, M_end>
  * (abstract: "fully parallelized chunk-level training"). Chunks run in reverse;

@@ -56,6 +56,7 @@ _SIGS = {
     "e2ttt_fwd_uses_tensor_cores": (ctypes.c_int, [_S]),
     "e2ttt_chunk_coeffs": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "e2ttt_chunk_scan_fwd": (ctypes.c_int, [_S] + [_P] * 13 + [ctypes.c_size_t, _P]),
+    "e2ttt_chunk_scan_fwd_noalloc": (ctypes.c_int, [_S] + [_P] * 13),
     "e2ttt_chunk_scan_bwd": (ctypes.c_int, [_S] + [_P] * 19 + [ctypes.c_size_t, _P]),
     "e2ttt_workspace_status": (ctypes.c_int, [_P, _P]),
     "e2ttt_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -158,6 +159,19 @@ def e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, M0, out, W_end, M_e
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(mom), _ptr(decay), _ptr(W0),
         _ptr(M0), _ptr(out), _ptr(W_end), _ptr(M_end), _ptr(saved_states), _ptr(workspace),
         workspace_bytes, _stream(stream) if not raw else stream)
+    if raw:
+        return st
+    _check(st)
+
+
+def e2ttt_chunk_scan_fwd_noalloc(shape, q, k, v, lr, mom, decay, W0, M0, out, W_end, M_end,
+                                 saved_states, stream=None, raw=False):
+    """The forward without a workspace (library-owned static scratch, at most
+    32 MiB of it): for callers that cannot allocate device memory."""
+    st = _lib.e2ttt_chunk_scan_fwd_noalloc(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(mom), _ptr(decay), _ptr(W0),
+        _ptr(M0), _ptr(out), _ptr(W_end), _ptr(M_end), _ptr(saved_states),
+        _stream(stream) if not raw else stream)
     if raw:
         return st
     _check(st)

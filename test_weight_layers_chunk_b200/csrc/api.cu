@@ -147,6 +147,11 @@ bool check_overlaps(const Range* in, int nin, const Range* out, int nout, std::s
 }
 
 }  // namespace
+
+// Lets other translation units of the library report a failure through
+// e2ttt_last_error().
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 }  // namespace e2ttt
 
 using namespace e2ttt;
