@@ -85,13 +85,13 @@ struct Bump {
 
 struct FwdWs {
   size_t status;                    // device status word (bounded waits)
-  size_t a, b, scal, st, H, E, dH;  // fp32 CUDA-core path
+  size_t a, b, scal, H, E, dH;      // fp32 CUDA-core path
   size_t tc;                        // tensor-core path scratch
   size_t total;
 };
 
-// Coefficients and one spare state pair, then one region shared by the
-// tensor-core scratch and the CUDA-core scratch (only one path runs per call).
+// Status word and coefficients, then one region shared by the tensor-core
+// scratch and the CUDA-core scratch (only one path runs per call).
 FwdWs fwd_layout(const Dims& d, bool tc_shape) {
   Bump w;
   FwdWs L{};
@@ -100,7 +100,6 @@ FwdWs fwd_layout(const Dims& d, bool tc_shape) {
   L.a = w.take((size_t)d.BH * d.T * f);
   L.b = w.take((size_t)d.BH * d.T * f);
   L.scal = w.take((size_t)3 * d.BH * d.NC * f);
-  L.st = w.take((size_t)2 * d.BH * d.S * f);
   const size_t region = w.off;
   Bump s;
   s.off = region;
@@ -261,7 +260,6 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   float* ca = (float*)(w + L.a);
   float* cb = (float*)(w + L.b);
   float* scal = (float*)(w + L.scal);
-  float* stbuf = (float*)(w + L.st);
   int* status = (int*)(w + L.status);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "status word reset");
@@ -269,7 +267,7 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   if (e != cudaSuccess) return cuda_fail(e, "chunk coefficient kernel");
   if (tc) {
     e = tc_fwd(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal, W0, M0,
-               W_end, M_end, saved, stbuf, w + L.tc, status, st);
+               W_end, M_end, saved, w + L.tc, status, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward");
     return E2TTT_OK;
   }
@@ -278,10 +276,10 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   float* dH = (float*)(w + L.dH);
   if (bf)
     e = simt_fwd<bf16>(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal,
-                       W0, M0, W_end, M_end, saved, stbuf, H, E, dH, st);
+                       W0, M0, W_end, M_end, saved, H, E, dH, st);
   else
     e = simt_fwd<float>(d, (const float*)q, (const float*)k, (const float*)v, (float*)out, ca, cb,
-                        scal, W0, M0, W_end, M_end, saved, stbuf, H, E, dH, st);
+                        scal, W0, M0, W_end, M_end, saved, H, E, dH, st);
   if (e != cudaSuccess) return cuda_fail(e, "CUDA-core forward");
   return E2TTT_OK;
 }

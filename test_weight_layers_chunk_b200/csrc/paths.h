@@ -20,16 +20,16 @@ cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const flo
 template <typename TA>
 cudaError_t simt_fwd(const Dims& d, const TA* q, const TA* k, const TA* v, TA* out,
                      const float* ca, const float* cb, const float* scal, const float* W0,
-                     const float* M0, float* W_end, float* M_end, float* saved, float* stbuf,
-                     float* H, float* E, float* dH, cudaStream_t st);
+                     const float* M0, float* W_end, float* M_end, float* saved, float* H,
+                     float* E, float* dH, cudaStream_t st);
 
 // tcgen05 tensor-core forward for bf16 activations (tc_fwd.cu).
 bool tc_fwd_supported(const Dims& d, bool bf16_act);
 size_t tc_fwd_scratch_bytes(const Dims& d);
 cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, bf16* out,
                    const float* ca, const float* cb, const float* scal, const float* W0,
-                   const float* M0, float* W_end, float* M_end, float* saved, float* stbuf,
-                   void* scratch, int* status, cudaStream_t st);
+                   const float* M0, float* W_end, float* M_end, float* saved, void* scratch,
+                   int* status, cudaStream_t st);
 
 // Backward (bwd.cu).
 struct BwdArgs {

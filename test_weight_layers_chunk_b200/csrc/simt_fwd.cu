@@ -180,8 +180,8 @@ cudaError_t fwd_chunk(const Fwd<TA>& c, cudaStream_t st) {
 template <typename TA>
 cudaError_t simt_fwd(const Dims& d, const TA* q, const TA* k, const TA* v, TA* out,
                      const float* ca, const float* cb, const float* scal, const float* W0,
-                     const float* M0, float* W_end, float* M_end, float* saved, float* stbuf,
-                     float* H, float* E, float* dH, cudaStream_t st) {
+                     const float* M0, float* W_end, float* M_end, float* saved, float* H,
+                     float* E, float* dH, cudaStream_t st) {
   Fwd<TA> c;
   c.d = d;
   c.q = q; c.k = k; c.v = v; c.out = out;
@@ -193,7 +193,7 @@ cudaError_t simt_fwd(const Dims& d, const TA* q, const TA* k, const TA* v, TA* o
     c.ci = ci;
     c.t0 = ci * d.C;
     c.n = d.T - c.t0 < d.C ? d.T - c.t0 : d.C;
-    chunk_states(d, ci, W0, M0, W_end, M_end, saved, stbuf, &c.src, &c.dst);
+    chunk_states(d, ci, W0, M0, W_end, M_end, saved, &c.src, &c.dst);
     e = fwd_chunk(c, st);
     if (e != cudaSuccess) return e;
   }
@@ -203,10 +203,10 @@ cudaError_t simt_fwd(const Dims& d, const TA* q, const TA* k, const TA* v, TA* o
 template cudaError_t simt_fwd<float>(const Dims&, const float*, const float*, const float*, float*,
                                      const float*, const float*, const float*, const float*,
                                      const float*, float*, float*, float*, float*, float*, float*,
-                                     float*, cudaStream_t);
+                                     cudaStream_t);
 template cudaError_t simt_fwd<bf16>(const Dims&, const bf16*, const bf16*, const bf16*, bf16*,
                                     const float*, const float*, const float*, const float*,
                                     const float*, float*, float*, float*, float*, float*, float*,
-                                    float*, cudaStream_t);
+                                    cudaStream_t);
 
 }  // namespace e2ttt

@@ -7,8 +7,8 @@
 //   with saved_states [NC, BH, 2, S]: chunk 0 reads the caller's W0/M0 (a copy
 //     goes to saved[0]); chunk i writes saved[i+1]; the last chunk writes
 //     W_end/M_end;
-//   without: chunk i writes X_i, alternating between the caller's W_end/M_end
-//     and one workspace pair so that the last chunk lands in W_end/M_end.
+//   without: chunk 0 reads W0/M0 and writes W_end/M_end; later chunks update
+//     W_end/M_end in place.
 #pragma once
 #include "common.cuh"
 
@@ -40,7 +40,7 @@ __device__ __forceinline__ void state_update(const StateIn& src, const StateOut&
 }
 
 inline void chunk_states(const Dims& d, int ci, const float* W0, const float* M0, float* W_end,
-                         float* M_end, float* saved, float* stbuf, StateIn* src, StateOut* dst) {
+                         float* M_end, float* saved, StateIn* src, StateOut* dst) {
   const long long S = d.S;
   const size_t per_chunk = (size_t)d.BH * 2 * S;
   if (saved) {
@@ -50,16 +50,12 @@ inline void chunk_states(const Dims& d, int ci, const float* W0, const float* M0
     else *dst = StateOut{W_end, M_end, S};
     return;
   }
-  auto X = [&](int i) {
-    if (((d.NC - 1 - i) & 1) == 0) return StateOut{W_end, M_end, S};
-    return StateOut{stbuf, stbuf + (size_t)d.BH * S, S};
-  };
+  // In place after the first chunk: every state element is read and then
+  // written by the same thread, and no other kernel of the chunk reads the
+  // fp32 state while the aggregation kernel updates it.
   if (ci == 0) *src = StateIn{W0, M0, S};
-  else {
-    StateOut p = X(ci - 1);
-    *src = StateIn{p.W, p.M, p.stride};
-  }
-  *dst = X(ci);
+  else *src = StateIn{W_end, M_end, S};
+  *dst = StateOut{W_end, M_end, S};
 }
 
 inline cudaError_t save_initial_state(const Dims& d, const float* W0, const float* M0, float* saved,

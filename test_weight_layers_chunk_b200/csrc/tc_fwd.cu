@@ -4,30 +4,32 @@
 // Test-Time Training" (abstract: closed-form chunk transition with chunk-start
 // gradients; atlas "Approach": two weighted gradient aggregations; arxivlens
 // "Limitations": output at the chunk-start weights), SwiGLU fast weight:
-//   G1  H = [Q; K] [W1; W3]^T     epilogue: A = silu(H1) * H3 (bf16, both row
-//                                 sets), A_k^T, and silu(H1_k), H3_k silu'(H1_k)
-//   G2  Y = A W2^T                epilogue: out = Y_q; E = Y_k - V, and the
-//                                 transposed, a- and b-scaled copies of E
-//   G3  dA = E W2                 epilogue: dH1 = dA H3 silu'(H1), dH3 = dA
-//                                 silu(H1), transposed and a-/b-scaled
-//   G4  [dM | dW] = [Da | Db]^T K  and  [Ea | Eb]^T A_k   (two accumulators)
+//   G1  H = [Q; K] [W1; W3]^T     epilogue: A = silu(H1) * H3 for both row sets,
+//                                 silu(H1_k) and H3_k silu'(H1_k)
+//   G2  Y = A W2^T                epilogue: out = Y_q; E = Y_k - V and its a-/b-
+//                                 scaled copies
+//   G3  dA = E W2                 epilogue: dH1 = dA H3 silu'(H1), dH3 = dA silu(H1)
+//   G4  [dM | dW] of [W1; W3] = dH^T [diag(a) K | diag(b) K]  (one A, two B)
+//       [dM | dW] of W2       = [diag(a) E | diag(b) E]^T A_k  (two A, one B)
 //                                 epilogue: M_end = U M0 - dM, W_end = L W0 + c M0 - dW
 //                                 in fp32, plus the bf16 operand copies of W_end
-//                                 that the next chunk's GEMMs read.
-// Linear fast weight: G1 gives out and the scaled E^T; G4 aggregates E^T K.
-// Every GEMM operand is K-major in global memory: the epilogues write the
-// transposed operands directly, and the keys are transposed once per call.
+// Linear fast weight: G1 gives out and the scaled E; G4 aggregates them with K.
+// All intermediates are stored token-major (natural rows); the aggregations read
+// them as MN-major operands, so nothing is ever transposed.
 #include <cuda.h>
 
 #include "paths.h"
 #include "state.cuh"
-#include "tc_gemm.cuh"
+#include "tc_gemm2.cuh"
 #include "trace.h"
 
 namespace e2ttt {
 namespace {
 
-using tc::EpiCtx;
+using tc2::EpiCtx;
+using tc2::tmem_ld32_nowait;
+using tc2::tmem_wait_ld;
+using tc2::tmem_wait_ld2;
 
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
@@ -41,8 +43,8 @@ struct FwdP {
   const float *ca, *cb, *scal;
   StateIn src;
   StateOut dst;
-  bf16 *Wsh13, *W2sh, *W2Tsh;  // bf16 copies of the chunk-start weights (Wsh13 = W for linear)
-  bf16 *KT, *A, *AkT, *Sk, *E, *EaT, *EbT, *DaT, *DbT;
+  bf16 *Wsh13, *W2sh;  // bf16 copies of the chunk-start weights (Wsh13 = W for linear)
+  bf16 *A, *Sk, *E, *Ea, *Eb, *dH, *Ka, *Kb;
 };
 
 // ---------------------------------------------------------------- small helpers
@@ -65,8 +67,7 @@ __device__ __forceinline__ void ld_row32(const bf16* src, float (&v)[32]) {
     uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
-      float2 f = __bfloat1622float2(h);
+      float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[j]));
       v[8 * i + 2 * j] = f.x;
       v[8 * i + 2 * j + 1] = f.y;
     }
@@ -85,9 +86,31 @@ __device__ __forceinline__ void st_row32_f(float* dst, const float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
+__device__ __forceinline__ float fast_sigmoid(float z) { return __frcp_rn(1.0f + __expf(-z)); }
 // Row of the interleaved [W1; W3] operand copy that holds row r of W1 (which=0) or W3 (which=1).
 __device__ __forceinline__ int w13_row(int r, int which) {
   return (r / HB) * (2 * HB) + which * HB + (r % HB);
+}
+template <int BN>
+__device__ __forceinline__ void ld2(const EpiCtx<BN>& c, int acc0, int col0, int acc1, int col1,
+                                    float (&x)[32], float (&y)[32]) {
+  uint32_t r[32], s[32];
+  tmem_ld32_nowait(c.taddr + (uint32_t)(acc0 * BN + col0), r);
+  tmem_ld32_nowait(c.taddr + (uint32_t)(acc1 * BN + col1), s);
+  tmem_wait_ld2(r, s);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    x[i] = __uint_as_float(r[i]);
+    y[i] = __uint_as_float(s[i]);
+  }
+}
+template <int BN>
+__device__ __forceinline__ void ld1(const EpiCtx<BN>& c, int acc, int col, float (&x)[32]) {
+  uint32_t r[32];
+  tmem_ld32_nowait(c.taddr + (uint32_t)(acc * BN + col), r);
+  tmem_wait_ld(r);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
 }
 
 // ---------------------------------------------------------------- epilogues
@@ -99,55 +122,52 @@ struct EpiG1 {
     const int t = c.m0 + c.row;
     const int j0 = (c.n0 / (2 * HB)) * HB;
     const int per = HB / c.nparts;
-    const size_t arow = ((size_t)c.z * 2 * d.C + (size_t)c.cls * d.C + t) * d.d_h;
+    bf16* arow = p.A + ((size_t)c.z * 2 * d.C + (size_t)c.cls * d.C + t) * d.d_h + j0;
+    bf16* srow = p.Sk + ((size_t)c.z * d.C + t) * 2 * d.d_h + j0;
     for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
-      float h1[32], h3[32], u[32];
-      c.ld(0, g, h1);
-      c.ld(0, HB + g, h3);
+      float h1[32], h3[32];
+      ld2(c, 0, g, 0, HB + g, h1, h3);
       if (c.cls == 0) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = silu_f(h1[i]) * h3[i];
-        st_row32(p.A + arow + j0 + g, u);
+        for (int i = 0; i < 32; ++i) h1[i] = h1[i] * fast_sigmoid(h1[i]) * h3[i];
+        st_row32(arow + g, h1);
       } else {
-        float s1[32], s2[32];
+        float s2[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float sg = sigmoid_f(h1[i]);
-          s1[i] = h1[i] * sg;
+          const float sg = fast_sigmoid(h1[i]);
+          const float s1 = h1[i] * sg;
           s2[i] = h3[i] * sg * (1.0f + h1[i] * (1.0f - sg));
-          u[i] = s1[i] * h3[i];
+          h3[i] = s1 * h3[i];  // u
+          h1[i] = s1;
         }
-        st_row32(p.A + arow + j0 + g, u);
-        const size_t srow = ((size_t)c.z * d.C + t) * 2 * d.d_h;
-        st_row32(p.Sk + srow + j0 + g, s1);
-        st_row32(p.Sk + srow + d.d_h + j0 + g, s2);
-        bf16* akt = p.AkT + ((size_t)c.z * d.d_h + j0 + g) * d.C + t;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) akt[(size_t)i * d.C] = __float2bfloat16_rn(u[i]);
+        st_row32(arow + g, h3);
+        st_row32(srow + g, h1);
+        st_row32(srow + d.d_h + g, s2);
       }
     }
   }
 };
 
-// Key-row epilogue shared by G2 (SwiGLU) and G1 (linear): e = y - v (or -v);
-// writes E (if requested) and the a-/b-scaled transposes.
+// Key rows: e = y - v (or -v); E (if requested) and its a-/b-scaled copies.
 template <int BN>
 __device__ __forceinline__ void key_rows_epilogue(const FwdP& p, const EpiCtx<BN>& c, int t, int col0,
-                                                  const float (&y)[32], bool write_e) {
+                                                  float (&y)[32], bool write_e) {
   const Dims& d = p.d;
   const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-  float vv[32], e[32];
+  float vv[32];
   ld_row32(p.v + tok * d.d_v + col0, vv);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) e[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
-  if (write_e) st_row32(p.E + ((size_t)c.z * d.C + t) * d.d_v + col0, e);
+  for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
+  const size_t o = ((size_t)c.z * d.C + t) * d.d_v + col0;
+  if (write_e) st_row32(p.E + o, y);
   const float at = p.ca[tok], bt = p.cb[tok];
-  const size_t o = ((size_t)c.z * d.d_v + col0) * d.C + t;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    p.EaT[o + (size_t)i * d.C] = __float2bfloat16_rn(at * e[i]);
-    p.EbT[o + (size_t)i * d.C] = __float2bfloat16_rn(bt * e[i]);
-  }
+  for (int i = 0; i < 32; ++i) vv[i] = at * y[i];
+  st_row32(p.Ea + o, vv);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) vv[i] = bt * y[i];
+  st_row32(p.Eb + o, vv);
 }
 
 // G2, SwiGLU: rows [0, C) are queries (-> out), [C, 2C) keys (-> E).
@@ -159,18 +179,15 @@ struct EpiG2 {
     const int per = BN / c.nparts;
     for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
       float y[32];
-      c.ld(0, g, y);
+      ld1(c, 0, g, y);
       const int col = c.n0 + g;
-      if (m < d.C) {
-        st_row32(p.out + ((size_t)c.z * d.T + p.t0 + m) * d.d_v + col, y);
-      } else {
-        key_rows_epilogue(p, c, m - d.C, col, y, true);
-      }
+      if (m < d.C) st_row32(p.out + ((size_t)c.z * d.T + p.t0 + m) * d.d_v + col, y);
+      else key_rows_epilogue(p, c, m - d.C, col, y, true);
     }
   }
 };
 
-// G1, linear: class 0 = queries (-> out), class 1 = keys (-> scaled E^T).
+// G1, linear: class 0 = queries (-> out), class 1 = keys (-> scaled E).
 struct EpiG1Lin {
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
@@ -179,7 +196,7 @@ struct EpiG1Lin {
     const int per = BN / c.nparts;
     for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
       float y[32];
-      c.ld(0, g, y);
+      ld1(c, 0, g, y);
       const int col = c.n0 + g;
       if (c.cls == 0) st_row32(p.out + ((size_t)c.z * d.T + p.t0 + t) * d.d_v + col, y);
       else key_rows_epilogue(p, c, t, col, y, false);
@@ -187,32 +204,27 @@ struct EpiG1Lin {
   }
 };
 
-// G3, SwiGLU: dA -> dH1, dH3, transposed and scaled by a_t and b_t.
+// G3, SwiGLU: dA -> dH1 = dA H3 silu'(H1), dH3 = dA silu(H1) (rows: tokens).
 struct EpiG3 {
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
     const int t = c.m0 + c.row;
-    const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-    const float at = p.ca[tok], bt = p.cb[tok];
     const int per = BN / c.nparts;
-    const size_t srow = ((size_t)c.z * d.C + t) * 2 * d.d_h;
+    const size_t row = ((size_t)c.z * d.C + t) * 2 * d.d_h;
     for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
       float da[32], s1[32], s2[32];
-      c.ld(0, g, da);
       const int j = c.n0 + g;
-      ld_row32(p.Sk + srow + j, s1);
-      ld_row32(p.Sk + srow + d.d_h + j, s2);
-      const size_t o1 = ((size_t)c.z * 2 * d.d_h + j) * d.C + t;
-      const size_t o3 = o1 + (size_t)d.d_h * d.C;
+      ld_row32(p.Sk + row + j, s1);
+      ld_row32(p.Sk + row + d.d_h + j, s2);
+      ld1(c, 0, g, da);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float dh1 = da[i] * s2[i], dh3 = da[i] * s1[i];
-        p.DaT[o1 + (size_t)i * d.C] = __float2bfloat16_rn(at * dh1);
-        p.DbT[o1 + (size_t)i * d.C] = __float2bfloat16_rn(bt * dh1);
-        p.DaT[o3 + (size_t)i * d.C] = __float2bfloat16_rn(at * dh3);
-        p.DbT[o3 + (size_t)i * d.C] = __float2bfloat16_rn(bt * dh3);
+        s2[i] *= da[i];  // dH1
+        s1[i] *= da[i];  // dH3
       }
+      st_row32(p.dH + row + j, s2);
+      st_row32(p.dH + row + d.d_h + j, s1);
     }
   }
 };
@@ -231,18 +243,20 @@ struct EpiG4 {
     const int ld = c.cls == 0 ? d.d_k : d.d_h;
     const long long base = c.cls == 0 ? 0 : 2LL * d.d_h * d.d_k;
     const int per = BN / c.nparts;
+    const float* srcW = p.src.W + c.z * p.src.stride + base + (long long)i * ld;
+    const float* srcM = p.src.M ? p.src.M + c.z * p.src.stride + base + (long long)i * ld : nullptr;
+    float* dstW = p.dst.W + c.z * p.dst.stride + base + (long long)i * ld;
+    float* dstM = p.dst.M + c.z * p.dst.stride + base + (long long)i * ld;
     for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
-      float dM[32], dW[32], w0[32], m0[32];
-      c.ld(0, g, dM);
-      c.ld(1, g, dW);
       const int j = c.n0 + g;
-      const long long idx = base + (long long)i * ld + j;
-      ld_row32_f(p.src.W + c.z * p.src.stride + idx, w0);
-      if (p.src.M) ld_row32_f(p.src.M + c.z * p.src.stride + idx, m0);
+      float w0[32], m0[32], dM[32], dW[32];
+      ld_row32_f(srcW + j, w0);
+      if (srcM) ld_row32_f(srcM + j, m0);
       else {
 #pragma unroll
         for (int q = 0; q < 32; ++q) m0[q] = 0.f;
       }
+      ld2(c, 0, g, 1, g, dM, dW);
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
         const float mn = PU * m0[q] - dM[q];
@@ -250,8 +264,8 @@ struct EpiG4 {
         dM[q] = mn;
         dW[q] = wn;
       }
-      st_row32_f(p.dst.M + c.z * p.dst.stride + idx, dM);
-      st_row32_f(p.dst.W + c.z * p.dst.stride + idx, dW);
+      st_row32_f(dstM + j, dM);
+      st_row32_f(dstW + j, dW);
       if (!p.write_shadow) continue;
       if (c.cls == 0) {
         const int row = swiglu ? w13_row(i % d.d_h, i / d.d_h) : i;
@@ -259,61 +273,64 @@ struct EpiG4 {
         st_row32(p.Wsh13 + ((size_t)c.z * rows + row) * d.d_k + j, dW);
       } else {
         st_row32(p.W2sh + ((size_t)c.z * d.d_v + i) * d.d_h + j, dW);
-        bf16* wt = p.W2Tsh + ((size_t)c.z * d.d_h + j) * d.d_v + i;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) wt[(size_t)q * d.d_v] = __float2bfloat16_rn(dW[q]);
       }
     }
   }
 };
 
-template <class Epi>
-struct EpiAdapter {
-  template <int BN>
-  static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
-    Epi::template run<BN>(p, c);
-  }
-};
+template <class Epi> struct EpiName;
+template <> struct EpiName<EpiG1> { static constexpr const char* v = "tc_g1_h_act"; };
+template <> struct EpiName<EpiG2> { static constexpr const char* v = "tc_g2_y_out_e"; };
+template <> struct EpiName<EpiG3> { static constexpr const char* v = "tc_g3_da_dh"; };
+template <> struct EpiName<EpiG4> { static constexpr const char* v = "tc_g4_aggregate_state"; };
+template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 
-// ---------------------------------------------------------------- prep kernels
-// K [BH, T, d_k] -> per-chunk transposes KT [BH, NC, d_k, C] (32x32 tiles).
-__global__ void transpose_keys_kernel(const bf16* __restrict__ k, bf16* __restrict__ KT, int T, int C,
-                                      int NC, int d_k) {
-  __shared__ bf16 tile[32][33];
-  const int z = blockIdx.z;
-  const int t0 = blockIdx.x * 32, j0 = blockIdx.y * 32;
-  for (int r = threadIdx.y; r < 32; r += 8)
-    tile[r][threadIdx.x] = k[((size_t)z * T + t0 + r) * d_k + j0 + threadIdx.x];
-  __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += 8) {
-    const int j = j0 + r, t = t0 + threadIdx.x;
-    KT[(((size_t)z * NC + t / C) * d_k + j) * C + (t % C)] = tile[threadIdx.x][r];
+// ---------------------------------------------------------------- prep kernel
+// bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
+__global__ void shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
+  const Dims& d = p.d;
+  const long long total4 = (long long)d.BH * d.S / 4;
+  const long long n13 = d.kind == 1 ? 2LL * d.d_h * d.d_k : 0;
+  for (long long e4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e4 < total4;
+       e4 += (long long)gridDim.x * blockDim.x) {
+    const long long e = e4 * 4;
+    const int z = (int)(e / d.S);
+    const long long idx = e - (long long)z * d.S;
+    const float4 f = reinterpret_cast<const float4*>(W0)[e4];
+    const uint2 packed = make_uint2(pack2(f.x, f.y), pack2(f.z, f.w));
+    bf16* dst;
+    if (d.kind == 0) {
+      dst = p.Wsh13 + e;
+    } else if (idx < n13) {
+      const int i = (int)(idx / d.d_k), j = (int)(idx % d.d_k);
+      dst = p.Wsh13 + ((size_t)z * 2 * d.d_h + w13_row(i % d.d_h, i / d.d_h)) * d.d_k + j;
+    } else {
+      dst = p.W2sh + (size_t)z * d.d_v * d.d_h + (idx - n13);
+    }
+    *reinterpret_cast<uint2*>(dst) = packed;
   }
 }
 
-// bf16 operand copies of the caller's W0.
-__global__ void shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
-  const Dims& d = p.d;
-  const long long total = (long long)d.BH * d.S;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int z = (int)(e / d.S);
-    const long long idx = e - (long long)z * d.S;
-    const bf16 w = __float2bfloat16_rn(W0[e]);
-    if (d.kind == 0) {
-      p.Wsh13[e] = w;
-      continue;
+// diag(a) K and diag(b) K for every token (B operands of the W1/W3 aggregation).
+__global__ void scale_keys_kernel(const bf16* __restrict__ k, const float* __restrict__ ca,
+                                  const float* __restrict__ cb, bf16* __restrict__ Ka,
+                                  bf16* __restrict__ Kb, long long tokens, int d_k) {
+  const long long n8 = tokens * d_k / 8;
+  for (long long e8 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e8 < n8;
+       e8 += (long long)gridDim.x * blockDim.x) {
+    const long long tok = e8 * 8 / d_k;
+    const float a = ca[tok], b = cb[tok];
+    const uint4 u = reinterpret_cast<const uint4*>(k)[e8];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t oa[4], ob[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      oa[i] = pack2(a * f.x, a * f.y);
+      ob[i] = pack2(b * f.x, b * f.y);
     }
-    const long long n13 = 2LL * d.d_h * d.d_k;
-    if (idx < n13) {
-      const int i = (int)(idx / d.d_k), j = (int)(idx % d.d_k);
-      p.Wsh13[((size_t)z * 2 * d.d_h + w13_row(i % d.d_h, i / d.d_h)) * d.d_k + j] = w;
-    } else {
-      const long long r2 = idx - n13;
-      const int i = (int)(r2 / d.d_h), j = (int)(r2 % d.d_h);
-      p.W2sh[((size_t)z * d.d_v + i) * d.d_h + j] = w;
-      p.W2Tsh[((size_t)z * d.d_h + j) * d.d_v + i] = w;
-    }
+    reinterpret_cast<uint4*>(Ka)[e8] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+    reinterpret_cast<uint4*>(Kb)[e8] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
   }
 }
 
@@ -336,7 +353,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a row-major [rows, cols] matrix; box = 64 columns x box_rows rows, 128B swizzle.
+// 2-D bf16 map over a row-major [rows, cols] matrix; box = 64 columns x box_rows
+// rows, 128B swizzle (K-major operand: box_rows = tile rows; MN-major: 64).
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -349,36 +367,28 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <class Epi> struct EpiName;
-template <> struct EpiName<struct EpiG1> { static constexpr const char* v = "tc_g1_h_act"; };
-template <> struct EpiName<struct EpiG2> { static constexpr const char* v = "tc_g2_y_out_e"; };
-template <> struct EpiName<struct EpiG3> { static constexpr const char* v = "tc_g3_da_dh"; };
-template <> struct EpiName<struct EpiG4> { static constexpr const char* v = "tc_g4_aggregate_state"; };
-template <> struct EpiName<struct EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
 
-template <int BN, int NUM_A, int STAGES, class Epi>
-cudaError_t launch(const tc::Job& job, const FwdP& p, cudaStream_t st) {
-  constexpr size_t smem = tc::smem_bytes<BN, NUM_A, STAGES>();
-  auto kern = tc::gemm_kernel<BN, NUM_A, STAGES, kEpiWarps, EpiAdapter<Epi>, FwdP>;
-  cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)smem);
-  if (attr != cudaSuccess) return attr;
-  int tiles = 0;
-  for (int c = 0; c < job.n_cls; ++c) tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
+template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, class Epi>
+cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
+  constexpr size_t smem = tc2::smem_bytes<BN, NUM_ACC, A_MN, B_MN, STAGES>();
+  auto kern = tc2::gemm_persistent<BN, NUM_ACC, A_MN, B_MN, STAGES, kEpiWarps, Epi, FwdP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  job.total_tiles = 0;
+  for (int c = 0; c < job.n_cls; ++c) job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
+  const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
   E2TTT_TRACE(EpiName<Epi>::v, st);
-  kern<<<tiles, kThreads, smem, st>>>(job, p);
+  kern<<<grid, kThreads, smem, st>>>(job, p);
   return cudaGetLastError();
 }
 
-// BN = 256 when N allows, else 128 (N is always a multiple of 128 here).
-template <int NUM_A, int STAGES256, int STAGES128, class Epi>
-cudaError_t launch_bn(bool bn256, const tc::Job& job, const FwdP& p, cudaStream_t st) {
-  if (bn256) return launch<256, NUM_A, STAGES256, Epi>(job, p, st);
-  return launch<128, NUM_A, STAGES128, Epi>(job, p, st);
-}
-
 struct Scratch {
-  bf16 *Wsh13, *W2sh, *W2Tsh, *KT, *A, *AkT, *Sk, *E, *EaT, *EbT, *DaT, *DbT;
+  bf16 *Wsh13, *W2sh, *A, *Sk, *E, *Ea, *Eb, *dH, *Ka, *Kb;
 };
 
 size_t carve(const Dims& d, char* base, Scratch* s) {
@@ -386,27 +396,24 @@ size_t carve(const Dims& d, char* base, Scratch* s) {
   auto take = [&](size_t bytes) {
     char* p = base ? base + off : nullptr;
     off = (off + bytes + 255) & ~size_t(255);
-    return p;
+    return (bf16*)p;
   };
   const size_t e = sizeof(bf16), BH = d.BH;
-  Scratch t;
+  Scratch t{};
   if (d.kind == 0) {
-    t.Wsh13 = (bf16*)take(BH * d.d_v * d.d_k * e);
-    t.W2sh = t.W2Tsh = t.A = t.AkT = t.Sk = t.E = t.DaT = t.DbT = nullptr;
+    t.Wsh13 = take(BH * d.d_v * d.d_k * e);
   } else {
-    t.Wsh13 = (bf16*)take(BH * 2 * d.d_h * d.d_k * e);
-    t.W2sh = (bf16*)take(BH * d.d_v * d.d_h * e);
-    t.W2Tsh = (bf16*)take(BH * d.d_h * d.d_v * e);
-    t.A = (bf16*)take(BH * 2 * d.C * d.d_h * e);
-    t.AkT = (bf16*)take(BH * d.d_h * d.C * e);
-    t.Sk = (bf16*)take(BH * d.C * 2 * d.d_h * e);
-    t.E = (bf16*)take(BH * d.C * d.d_v * e);
-    t.DaT = (bf16*)take(BH * 2 * d.d_h * d.C * e);
-    t.DbT = (bf16*)take(BH * 2 * d.d_h * d.C * e);
+    t.Wsh13 = take(BH * 2 * d.d_h * d.d_k * e);
+    t.W2sh = take(BH * d.d_v * d.d_h * e);
+    t.A = take(BH * 2 * d.C * d.d_h * e);
+    t.Sk = take(BH * d.C * 2 * d.d_h * e);
+    t.E = take(BH * d.C * d.d_v * e);
+    t.dH = take(BH * d.C * 2 * d.d_h * e);
+    t.Ka = take(BH * d.T * d.d_k * e);
+    t.Kb = take(BH * d.T * d.d_k * e);
   }
-  t.KT = (bf16*)take(BH * d.T * d.d_k * e);
-  t.EaT = (bf16*)take(BH * d.d_v * d.C * e);
-  t.EbT = (bf16*)take(BH * d.d_v * d.C * e);
+  t.Ea = take(BH * d.C * d.d_v * e);
+  t.Eb = take(BH * d.C * d.d_v * e);
   if (s) *s = t;
   return off;
 }
@@ -425,82 +432,88 @@ size_t tc_fwd_scratch_bytes(const Dims& d) { return carve(d, nullptr, nullptr); 
 
 cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, bf16* out,
                    const float* ca, const float* cb, const float* scal, const float* W0,
-                   const float* M0, float* W_end, float* M_end, float* saved, float* stbuf,
-                   void* scratch, int* status, cudaStream_t st) {
+                   const float* M0, float* W_end, float* M_end, float* saved, void* scratch,
+                   int* status, cudaStream_t st) {
   Scratch s;
   carve(d, (char*)scratch, &s);
   FwdP p;
   p.d = d;
   p.q = q; p.k = k; p.v = v; p.out = out;
   p.ca = ca; p.cb = cb; p.scal = scal;
-  p.Wsh13 = s.Wsh13; p.W2sh = s.W2sh; p.W2Tsh = s.W2Tsh;
-  p.KT = s.KT; p.A = s.A; p.AkT = s.AkT; p.Sk = s.Sk; p.E = s.E;
-  p.EaT = s.EaT; p.EbT = s.EbT; p.DaT = s.DaT; p.DbT = s.DbT;
+  p.Wsh13 = s.Wsh13; p.W2sh = s.W2sh;
+  p.A = s.A; p.Sk = s.Sk; p.E = s.E; p.Ea = s.Ea; p.Eb = s.Eb; p.dH = s.dH; p.Ka = s.Ka;
+  p.Kb = s.Kb;
   const int BH = d.BH, T = d.T, C = d.C, NC = d.NC, dk = d.d_k, dv = d.d_v, dh = d.d_h;
 
   cudaError_t e = save_initial_state(d, W0, M0, saved, st);
   if (e != cudaSuccess) return e;
   {
-    E2TTT_TRACE("tc_transpose_keys", st);
-    transpose_keys_kernel<<<dim3(T / 32, dk / 32, BH), dim3(32, 8), 0, st>>>(k, s.KT, T, C, NC, dk);
-  }
-  {
     E2TTT_TRACE("tc_shadow_init", st);
-    shadow_init_kernel<<<1184, 256, 0, st>>>(p, W0);
+    shadow_init_kernel<<<4 * num_sms(), 256, 0, st>>>(p, W0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (d.kind == 1) {
+    E2TTT_TRACE("tc_scale_keys", st);
+    scale_keys_kernel<<<4 * num_sms(), 256, 0, st>>>(k, ca, cb, s.Ka, s.Kb, (long long)BH * T, dk);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
 
-  // Operand maps (chunk-independent: coordinates carry the chunk offset).
-  tc::Job g1{}, g2{}, g3{}, g4{};
+  // Operand maps (chunk-independent; the chunk offset goes into the coordinates).
+  tc2::Job g1{}, g2{}, g3{}, g4{};
   bool ok = true;
-  const bool bn_v = dv % 256 == 0, bn_k = dk % 256 == 0, bn_h = dh % 256 == 0;
-  for (tc::Job* j : {&g1, &g2, &g3, &g4}) {
+  const bool bn_v = dv % 256 == 0;
+  for (tc2::Job* j : {&g1, &g2, &g3, &g4}) {
     j->heads = BH;
     j->status = status;
   }
+  using tc2::kModeA1B2;
+  using tc2::kModeA2B1;
   if (d.kind == 1) {
     // G1: classes = query rows, key rows; B = interleaved [W1; W3]
-    ok &= make_map(&g1.maps[0].a0, q, (uint64_t)BH * T, dk, 128);
-    ok &= make_map(&g1.maps[1].a0, k, (uint64_t)BH * T, dk, 128);
-    ok &= make_map(&g1.maps[0].b, s.Wsh13, (uint64_t)BH * 2 * dh, dk, 256);
-    g1.maps[1].b = g1.maps[0].b;
+    ok &= make_map(&g1.maps[0].op0, q, (uint64_t)BH * T, dk, 128);
+    ok &= make_map(&g1.maps[1].op0, k, (uint64_t)BH * T, dk, 128);
+    ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * 2 * dh, dk, 256);
+    g1.maps[1].op2 = g1.maps[0].op2;
     g1.n_cls = 2;
-    for (int c = 0; c < 2; ++c) g1.cls[c] = tc::Class{C / 128, 2 * dh / 256, dk / 64, T, 0, 2 * dh, 0};
-    // G2: A = [A_q; A_k] (2C rows per head), B = W2 (N = d_v)
-    ok &= make_map(&g2.maps[0].a0, s.A, (uint64_t)BH * 2 * C, dh, 128);
-    ok &= make_map(&g2.maps[0].b, s.W2sh, (uint64_t)BH * dv, dh, bn_v ? 256 : 128);
+    for (int c = 0; c < 2; ++c)
+      g1.cls[c] = tc2::Class{C / 128, 2 * dh / 256, dk / 64, {T, 0, 0}, {2 * dh, 0, 0}, 0};
+    // G2: A = [A_q; A_k], B = W2 (N = d_v)
+    ok &= make_map(&g2.maps[0].op0, s.A, (uint64_t)BH * 2 * C, dh, 128);
+    ok &= make_map(&g2.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 128);
     g2.n_cls = 1;
-    g2.cls[0] = tc::Class{2 * C / 128, dv / (bn_v ? 256 : 128), dh / 64, 2 * C, 0, dv, 0};
-    // G3: A = E, B = W2^T (N = d_h)
-    ok &= make_map(&g3.maps[0].a0, s.E, (uint64_t)BH * C, dv, 128);
-    ok &= make_map(&g3.maps[0].b, s.W2Tsh, (uint64_t)BH * dh, dv, bn_h ? 256 : 128);
+    g2.cls[0] = tc2::Class{2 * C / 128, dv / 128, dh / 64, {2 * C, 0, 0}, {dv, 0, 0}, 0};
+    // G3: A = E, B = W2 read MN-major (N = d_h, K = d_v)
+    ok &= make_map(&g3.maps[0].op0, s.E, (uint64_t)BH * C, dv, 128);
+    ok &= make_map(&g3.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 64);
     g3.n_cls = 1;
-    g3.cls[0] = tc::Class{C / 128, dh / (bn_h ? 256 : 128), dv / 64, C, 0, dh, 0};
-    // G4: class 0 = [W1; W3] rows (A = Da/Db, B = K^T), class 1 = W2 rows (A = Ea/Eb, B = A_k^T)
-    const bool bn4 = bn_k && bn_h;
-    const uint32_t b4 = bn4 ? 256 : 128;
-    ok &= make_map(&g4.maps[0].a0, s.DaT, (uint64_t)BH * 2 * dh, C, 128);
-    ok &= make_map(&g4.maps[0].a1, s.DbT, (uint64_t)BH * 2 * dh, C, 128);
-    ok &= make_map(&g4.maps[0].b, s.KT, (uint64_t)BH * NC * dk, C, b4);
-    ok &= make_map(&g4.maps[1].a0, s.EaT, (uint64_t)BH * dv, C, 128);
-    ok &= make_map(&g4.maps[1].a1, s.EbT, (uint64_t)BH * dv, C, 128);
-    ok &= make_map(&g4.maps[1].b, s.AkT, (uint64_t)BH * dh, C, b4);
+    g3.cls[0] = tc2::Class{C / 128, dh / 128, dv / 64, {C, 0, 0}, {dv, 0, 0}, 0};
+    // G4 class 0: A = dH (M = [W1; W3] rows, K = tokens), B0 = diag(a) K, B1 = diag(b) K
+    ok &= make_map(&g4.maps[0].op0, s.dH, (uint64_t)BH * C, 2 * dh, 64);
+    ok &= make_map(&g4.maps[0].op1, s.Ka, (uint64_t)BH * T, dk, 64);
+    ok &= make_map(&g4.maps[0].op2, s.Kb, (uint64_t)BH * T, dk, 64);
+    // G4 class 1: A0 = diag(a) E, A1 = diag(b) E (M = W2 rows), B = A_k (rows [C, 2C) of A)
+    ok &= make_map(&g4.maps[1].op0, s.Ea, (uint64_t)BH * C, dv, 64);
+    ok &= make_map(&g4.maps[1].op1, s.Eb, (uint64_t)BH * C, dv, 64);
+    ok &= make_map(&g4.maps[1].op2, s.A, (uint64_t)BH * 2 * C, dh, 64);
     g4.n_cls = 2;
-    g4.cls[0] = tc::Class{2 * dh / 128, dk / (int)b4, C / 64, 2 * dh, 0, NC * dk, 0};
-    g4.cls[1] = tc::Class{dv / 128, dh / (int)b4, C / 64, dv, 0, dh, 0};
+    g4.cls[0] = tc2::Class{2 * dh / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, kModeA1B2};
+    g4.cls[1] = tc2::Class{dv / 128, dh / 128, C / 64, {C, 0, 0}, {2 * C, C, 0}, kModeA2B1};
   } else {
-    ok &= make_map(&g1.maps[0].a0, q, (uint64_t)BH * T, dk, 128);
-    ok &= make_map(&g1.maps[1].a0, k, (uint64_t)BH * T, dk, 128);
-    ok &= make_map(&g1.maps[0].b, s.Wsh13, (uint64_t)BH * dv, dk, bn_v ? 256 : 128);
-    g1.maps[1].b = g1.maps[0].b;
+    ok &= make_map(&g1.maps[0].op0, q, (uint64_t)BH * T, dk, 128);
+    ok &= make_map(&g1.maps[1].op0, k, (uint64_t)BH * T, dk, 128);
+    ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * dv, dk, bn_v ? 256 : 128);
+    g1.maps[1].op2 = g1.maps[0].op2;
     g1.n_cls = 2;
-    for (int c = 0; c < 2; ++c) g1.cls[c] = tc::Class{C / 128, dv / (bn_v ? 256 : 128), dk / 64, T, 0, dv, 0};
-    ok &= make_map(&g4.maps[0].a0, s.EaT, (uint64_t)BH * dv, C, 128);
-    ok &= make_map(&g4.maps[0].a1, s.EbT, (uint64_t)BH * dv, C, 128);
-    ok &= make_map(&g4.maps[0].b, s.KT, (uint64_t)BH * NC * dk, C, bn_k ? 256 : 128);
+    for (int c = 0; c < 2; ++c)
+      g1.cls[c] = tc2::Class{C / 128, dv / (bn_v ? 256 : 128), dk / 64, {T, 0, 0}, {dv, 0, 0}, 0};
+    // G4: A0 = diag(a) E, A1 = diag(b) E (M = rows of W), B = K (N = d_k, K = tokens)
+    ok &= make_map(&g4.maps[0].op0, s.Ea, (uint64_t)BH * C, dv, 64);
+    ok &= make_map(&g4.maps[0].op1, s.Eb, (uint64_t)BH * C, dv, 64);
+    ok &= make_map(&g4.maps[0].op2, k, (uint64_t)BH * T, dk, 64);
     g4.n_cls = 1;
-    g4.cls[0] = tc::Class{dv / 128, dk / (bn_k ? 256 : 128), C / 64, dv, 0, NC * dk, 0};
+    g4.cls[0] = tc2::Class{dv / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, kModeA2B1};
   }
   if (!ok) return cudaErrorInvalidValue;
 
@@ -508,18 +521,18 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     p.ci = ci;
     p.t0 = ci * C;
     p.write_shadow = ci + 1 < NC;
-    chunk_states(d, ci, W0, M0, W_end, M_end, saved, stbuf, &p.src, &p.dst);
-    for (int c = 0; c < g1.n_cls; ++c) g1.cls[c].a_row_base = ci * C;
-    for (int c = 0; c < g4.n_cls; ++c)
-      if (c == 0) g4.cls[c].b_row_base = ci * dk;
+    chunk_states(d, ci, W0, M0, W_end, M_end, saved, &p.src, &p.dst);
+    g1.cls[0].a.y_base = g1.cls[1].a.y_base = ci * C;  // query / key rows of this chunk
+    g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
     if (d.kind == 1) {
-      e = launch<256, 1, 2, EpiG1>(g1, p, st);
-      if (e == cudaSuccess) e = launch_bn<1, 2, 3, EpiG2>(bn_v, g2, p, st);
-      if (e == cudaSuccess) e = launch_bn<1, 2, 3, EpiG3>(bn_h, g3, p, st);
-      if (e == cudaSuccess) e = launch_bn<2, 3, 2, EpiG4>(bn_k && bn_h, g4, p, st);
+      e = launch<256, 1, false, false, 4, EpiG1>(g1, p, st);
+      if (e == cudaSuccess) e = launch<128, 1, false, false, 6, EpiG2>(g2, p, st);
+      if (e == cudaSuccess) e = launch<128, 1, false, true, 6, EpiG3>(g3, p, st);
+      if (e == cudaSuccess) e = launch<128, 2, true, true, 4, EpiG4>(g4, p, st);
     } else {
-      e = launch_bn<1, 2, 3, EpiG1Lin>(bn_v, g1, p, st);
-      if (e == cudaSuccess) e = launch_bn<2, 3, 2, EpiG4>(bn_k, g4, p, st);
+      e = bn_v ? launch<256, 1, false, false, 4, EpiG1Lin>(g1, p, st)
+               : launch<128, 1, false, false, 6, EpiG1Lin>(g1, p, st);
+      if (e == cudaSuccess) e = launch<128, 2, true, true, 4, EpiG4>(g4, p, st);
     }
     if (e != cudaSuccess) return e;
   }

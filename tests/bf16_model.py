@@ -3,7 +3,8 @@
 Not the oracle: this restates the closed-form chunk transition with every GEMM
 operand rounded to bf16 at the points where the tcgen05 path rounds it (bf16
 copies of the chunk-start weights, the activations A = silu(H1) H3, the
-residual E, the a-/b-scaled gradient factors, silu(H1_k) and H3_k silu'(H1_k)),
+residual E and its a-/b-scaled copies, dH1 and dH3, the a-/b-scaled keys,
+silu(H1_k) and H3_k silu'(H1_k)),
 everything else in fp64, the fast-weight state rounded to fp32 once per chunk.
 Comparing the GPU with this model separates kernel mistakes (GPU far from the
 model) from the precision bf16 operands allow (model far from the oracle).
@@ -58,13 +59,12 @@ def model_fwd(w, x, heads):
                 out[b, h, t0:t1] = bf(Aq @ W2s.T)
                 e = f32(Ak @ W2s.T) - V if w.loss == gen.LOSS_MSE else -V
                 dA = f32(bf(e) @ W2s)
-                dH1, dH3 = dA * s2, dA * s1
-                Da1, Db1 = bf(a[:, None] * dH1), bf(bb[:, None] * dH1)
-                Da3, Db3 = bf(a[:, None] * dH3), bf(bb[:, None] * dH3)
+                dH1, dH3 = bf(dA * s2), bf(dA * s1)
+                Ka, Kb = bf(a[:, None] * K), bf(bb[:, None] * K)
                 Ea, Eb = bf(a[:, None] * e), bf(bb[:, None] * e)
-                dM = np.concatenate([(Da1.T @ K).reshape(-1), (Da3.T @ K).reshape(-1),
+                dM = np.concatenate([(dH1.T @ Ka).reshape(-1), (dH3.T @ Ka).reshape(-1),
                                      (Ea.T @ Ak).reshape(-1)])
-                dW = np.concatenate([(Db1.T @ K).reshape(-1), (Db3.T @ K).reshape(-1),
+                dW = np.concatenate([(dH1.T @ Kb).reshape(-1), (dH3.T @ Kb).reshape(-1),
                                      (Eb.T @ Ak).reshape(-1)])
             M_new = f32(PU * M - dM)
             W = f32(PL * W + c * M - dW)
