@@ -32,12 +32,16 @@ using tc2::tmem_wait_ld;
 using tc2::tmem_wait_ld2;
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr int HB = 128;  // hidden units per G1 tile (its 256 columns hold h1 then h3)
 
 struct FwdP {
+  // fp32 state tiles of the aggregation epilogue (3-D maps: columns, rows, heads)
+  // and the bf16 operand copies it writes; index = tile class (0: [W1; W3] or W,
+  // 1: W2). Rebuilt for every chunk.
+  CUtensorMap srcW[2], srcM[2], dstW[2], dstM[2], shadow[2];
   Dims d;
   int ci, t0, write_shadow;
+  int* status;
   const bf16 *q, *k, *v;
   bf16* out;
   const float *ca, *cb, *scal;
@@ -72,19 +76,6 @@ __device__ __forceinline__ void ld_row32(const bf16* src, float (&v)[32]) {
       v[8 * i + 2 * j + 1] = f.y;
     }
   }
-}
-__device__ __forceinline__ void ld_row32_f(const float* src, float (&v)[32]) {
-  const float4* p = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4 f = p[i];
-    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
-  }
-}
-__device__ __forceinline__ void st_row32_f(float* dst, const float (&v)[32]) {
-  float4* p = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 __device__ __forceinline__ float fast_sigmoid(float z) { return __frcp_rn(1.0f + __expf(-z)); }
 // Row of the interleaved [W1; W3] operand copy that holds row r of W1 (which=0) or W3 (which=1).
@@ -231,49 +222,91 @@ struct EpiG3 {
 
 // G4: accumulator 0 = dM = sum_t a_t g_t, accumulator 1 = dW = sum_t b_t g_t.
 // Class 0 covers rows of [W1; W3] (or W for linear), class 1 the rows of W2.
+// Each of the four epilogue warps owns 32 rows x 128 columns of the tile and
+// moves the fp32 state with TMA through two 10 KB slots of its shared memory:
+// the W0/M0 tiles of column group g+2 load while group g is computed; results
+// are written back into the slot (W, M fp32 and the bf16 copy of W) and stored
+// with TMA, so the state never passes through the load/store units.
 struct EpiG4 {
+  static constexpr int kSlot = 10240;  // W 4 KB | M 4 KB | bf16 copy 2 KB
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int i = c.m0 + c.row;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;  // first state row of this warp
+    constexpr int kGroups = BN / 32;
+    const bool hasM = p.src.M != nullptr;
+    const uint32_t tx = hasM ? 8192u : 4096u;
     const size_t plane = (size_t)d.BH * d.NC;
     const size_t so = (size_t)c.z * d.NC + p.ci;
     const float PU = p.scal[so], PL = p.scal[plane + so], cc = p.scal[2 * plane + so];
-    const bool swiglu = d.kind == 1;
-    const int ld = c.cls == 0 ? d.d_k : d.d_h;
-    const long long base = c.cls == 0 ? 0 : 2LL * d.d_h * d.d_k;
-    const int per = BN / c.nparts;
-    const float* srcW = p.src.W + c.z * p.src.stride + base + (long long)i * ld;
-    const float* srcM = p.src.M ? p.src.M + c.z * p.src.stride + base + (long long)i * ld : nullptr;
-    float* dstW = p.dst.W + c.z * p.dst.stride + base + (long long)i * ld;
-    float* dstM = p.dst.M + c.z * p.dst.stride + base + (long long)i * ld;
-    for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
-      const int j = c.n0 + g;
-      float w0[32], m0[32], dM[32], dW[32];
-      ld_row32_f(srcW + j, w0);
-      if (srcM) ld_row32_f(srcM + j, m0);
-      else {
+    int sh_row;
+    if (c.cls == 0 && d.kind == 1) {
+      const int which = r0 / d.d_h, rr = r0 % d.d_h;
+      sh_row = c.z * 2 * d.d_h + w13_row(rr, which);
+    } else {
+      sh_row = c.z * d.d_v + r0;
+    }
+    auto issue = [&](int g) {  // lane 0: TMA loads of column group g into slot g & 1
+      const int sidx = g & 1;
+      uint8_t* slot = c.wsmem + sidx * kSlot;
+      tc::mbar_expect_tx(&c.wbar[sidx], tx);
+      tc::tma_load_3d(slot, &p.srcW[c.cls], &c.wbar[sidx], c.n0 + g * 32, r0, c.z);
+      if (hasM) tc::tma_load_3d(slot + 4096, &p.srcM[c.cls], &c.wbar[sidx], c.n0 + g * 32, r0, c.z);
+    };
+    if (lane == 0) {
+      tc::bulk_wait_read<0>();  // the previous tile's stores no longer read our slots
+      issue(0);
+      if (kGroups > 1) issue(1);
+    }
+    __syncwarp();
+    for (int g = 0; g < kGroups; ++g) {
+      const int sidx = g & 1;
+      uint8_t* slot = c.wsmem + sidx * kSlot;
+      float dM[32], dW[32];
+      ld2(c, 0, g * 32, 1, g * 32, dM, dW);
+      const bool ok = tc::mbar_wait(&c.wbar[sidx], c.uses[sidx] & 1u);
+      c.uses[sidx] += 1;
+      if (!ok) {
+        if (lane == 0) atomicExch(p.status, tc2::kErrEpilogue);
+        return;
+      }
+      // row `lane` of the 128B-swizzled fp32 tiles; 64B-swizzled bf16 row
+      uint8_t* wrow = slot + lane * 128;
+      uint8_t* mrow = slot + 4096 + lane * 128;
+      uint8_t* srow = slot + 8192 + lane * 64;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) m0[q] = 0.f;
+      for (int q = 0; q < 8; ++q) {
+        const int off = (q ^ (lane & 7)) << 4;
+        const float4 w = *reinterpret_cast<const float4*>(wrow + off);
+        const float4 m = hasM ? *reinterpret_cast<const float4*>(mrow + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 wn, mn;
+        mn.x = PU * m.x - dM[4 * q + 0];
+        mn.y = PU * m.y - dM[4 * q + 1];
+        mn.z = PU * m.z - dM[4 * q + 2];
+        mn.w = PU * m.w - dM[4 * q + 3];
+        wn.x = PL * w.x + cc * m.x - dW[4 * q + 0];
+        wn.y = PL * w.y + cc * m.y - dW[4 * q + 1];
+        wn.z = PL * w.z + cc * m.z - dW[4 * q + 2];
+        wn.w = PL * w.w + cc * m.w - dW[4 * q + 3];
+        *reinterpret_cast<float4*>(wrow + off) = wn;
+        *reinterpret_cast<float4*>(mrow + off) = mn;
+        *reinterpret_cast<uint2*>(srow + ((((q >> 1) ^ ((lane >> 1) & 3)) << 4) | ((q & 1) << 3))) =
+            make_uint2(pack2(wn.x, wn.y), pack2(wn.z, wn.w));
       }
-      ld2(c, 0, g, 1, g, dM, dW);
-#pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const float mn = PU * m0[q] - dM[q];
-        const float wn = PL * w0[q] + cc * m0[q] - dW[q];
-        dM[q] = mn;
-        dW[q] = wn;
+      tc::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tc::tma_store_3d(&p.dstW[c.cls], slot, c.n0 + g * 32, r0, c.z);
+        tc::tma_store_3d(&p.dstM[c.cls], slot + 4096, c.n0 + g * 32, r0, c.z);
+        if (p.write_shadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 8192, c.n0 + g * 32, sh_row);
+        tc::bulk_commit();
+        if (g + 2 < kGroups) {
+          tc::bulk_wait_read<0>();  // slot reused for group g + 2
+          issue(g + 2);
+        }
       }
-      st_row32_f(dstM + j, dM);
-      st_row32_f(dstW + j, dW);
-      if (!p.write_shadow) continue;
-      if (c.cls == 0) {
-        const int row = swiglu ? w13_row(i % d.d_h, i / d.d_h) : i;
-        const int rows = swiglu ? 2 * d.d_h : d.d_v;
-        st_row32(p.Wsh13 + ((size_t)c.z * rows + row) * d.d_k + j, dW);
-      } else {
-        st_row32(p.W2sh + ((size_t)c.z * d.d_v + i) * d.d_h + j, dW);
-      }
+      __syncwarp();
     }
   }
 };
@@ -367,23 +400,53 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 map over the state rows [rows, cols] of every head (head stride in
+// elements), box 32 x 32 x 1, 128B swizzle.
+bool make_state_map(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint64_t heads,
+                    uint64_t head_stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, heads};
+  cuuint64_t strides[2] = {cols * 4, head_stride * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 map, box 32 columns x 32 rows, 64B swizzle (epilogue stores).
+bool make_map_box32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n;
 }
 
-template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, class Epi>
+template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, class Epi, int EW = kEpiWarps,
+          int ESM = 0>
 cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
-  constexpr size_t smem = tc2::smem_bytes<BN, NUM_ACC, A_MN, B_MN, STAGES>();
-  auto kern = tc2::gemm_persistent<BN, NUM_ACC, A_MN, B_MN, STAGES, kEpiWarps, Epi, FwdP>;
+  constexpr size_t smem = tc2::smem_bytes<BN, NUM_ACC, A_MN, B_MN, STAGES, EW, ESM>();
+  static_assert(smem <= 232448, "shared memory per CTA");
+  auto kern = tc2::gemm_persistent<BN, NUM_ACC, A_MN, B_MN, STAGES, EW, Epi, FwdP, ESM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   job.total_tiles = 0;
   for (int c = 0; c < job.n_cls; ++c) job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
   const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
   E2TTT_TRACE(EpiName<Epi>::v, st);
-  kern<<<grid, kThreads, smem, st>>>(job, p);
+  kern<<<grid, (2 + EW) * 32, smem, st>>>(job, p);
   return cudaGetLastError();
 }
 
@@ -440,6 +503,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   p.d = d;
   p.q = q; p.k = k; p.v = v; p.out = out;
   p.ca = ca; p.cb = cb; p.scal = scal;
+  p.status = status;
   p.Wsh13 = s.Wsh13; p.W2sh = s.W2sh;
   p.A = s.A; p.Sk = s.Sk; p.E = s.E; p.Ea = s.Ea; p.Eb = s.Eb; p.dH = s.dH; p.Ka = s.Ka;
   p.Kb = s.Kb;
@@ -522,17 +586,34 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     p.t0 = ci * C;
     p.write_shadow = ci + 1 < NC;
     chunk_states(d, ci, W0, M0, W_end, M_end, saved, &p.src, &p.dst);
+    {
+      const int ncls = d.kind == 1 ? 2 : 1;
+      for (int c = 0; c < ncls; ++c) {
+        const long long off = c == 0 ? 0 : 2LL * dh * dk;
+        const uint64_t rows = c == 0 ? (d.kind == 1 ? 2 * dh : dv) : dv;
+        const uint64_t cols = c == 0 ? dk : dh;
+        ok &= make_state_map(&p.srcW[c], p.src.W + off, rows, cols, BH, p.src.stride);
+        if (p.src.M) ok &= make_state_map(&p.srcM[c], p.src.M + off, rows, cols, BH, p.src.stride);
+        ok &= make_state_map(&p.dstW[c], p.dst.W + off, rows, cols, BH, p.dst.stride);
+        ok &= make_state_map(&p.dstM[c], p.dst.M + off, rows, cols, BH, p.dst.stride);
+      }
+      if (ci == 0) {
+        ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * (d.kind == 1 ? 2 * dh : dv), dk);
+        if (d.kind == 1) ok &= make_map_box32(&p.shadow[1], s.W2sh, (uint64_t)BH * dv, dh);
+      }
+      if (!ok) return cudaErrorInvalidValue;
+    }
     g1.cls[0].a.y_base = g1.cls[1].a.y_base = ci * C;  // query / key rows of this chunk
     g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
     if (d.kind == 1) {
       e = launch<256, 1, false, false, 4, EpiG1>(g1, p, st);
       if (e == cudaSuccess) e = launch<128, 1, false, false, 6, EpiG2>(g2, p, st);
       if (e == cudaSuccess) e = launch<128, 1, false, true, 6, EpiG3>(g3, p, st);
-      if (e == cudaSuccess) e = launch<128, 2, true, true, 4, EpiG4>(g4, p, st);
+      if (e == cudaSuccess) e = launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
     } else {
       e = bn_v ? launch<256, 1, false, false, 4, EpiG1Lin>(g1, p, st)
                : launch<128, 1, false, false, 6, EpiG1Lin>(g1, p, st);
-      if (e == cudaSuccess) e = launch<128, 2, true, true, 4, EpiG4>(g4, p, st);
+      if (e == cudaSuccess) e = launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
     }
     if (e != cudaSuccess) return e;
   }

@@ -100,9 +100,13 @@ struct Job {
 template <int BN>
 struct EpiCtx {
   int cls, z, m0, n0;
-  int row;
-  int part, nparts;
-  uint32_t taddr;  // TMEM address of (this warp's lane quadrant, this tile's accumulator set)
+  int row;            // this thread's row inside the tile (its TMEM lane)
+  int quad;           // this warp's lane quadrant (rows [32 quad, 32 quad + 32))
+  int part, nparts;   // this warp's column share
+  uint32_t taddr;     // TMEM address of (this warp's lane quadrant, this tile's accumulator set)
+  uint8_t* wsmem;     // this warp's epilogue shared memory (EPI_SMEM bytes, 1024-aligned)
+  uint64_t* wbar;     // two mbarriers owned by this warp (epilogue TMA loads)
+  uint32_t* uses;     // completed-phase counters of wbar[0..1], kept across tiles
   __device__ __forceinline__ void ld(int acc, int col, float (&v)[32]) const {
     tmem_ld32(taddr + (uint32_t)(acc * BN + col), v);
   }
@@ -120,10 +124,12 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 2 * kAccCols <= 128 ? 128 : 2 * kAccCols <= 256 ? 256 : 512;
 };
 
-template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES>
+template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, int EPI_WARPS = 8, int EPI_SMEM = 0>
 constexpr size_t smem_bytes() {
-  // ring + barriers; at least 116 KB so that one CTA is resident per SM
-  size_t s = 1024 + (size_t)STAGES * Cfg<BN, NUM_ACC, A_MN, B_MN>::kStage + 256;
+  // ring + per-warp epilogue buffers + barriers; at least 116 KB so that one
+  // CTA is resident per SM
+  size_t s = 1024 + (size_t)STAGES * Cfg<BN, NUM_ACC, A_MN, B_MN>::kStage +
+             (size_t)EPI_WARPS * EPI_SMEM + 256 + 16 * EPI_WARPS;
   return s < 118784 ? 118784 : s;
 }
 
@@ -156,19 +162,23 @@ __device__ __forceinline__ void load_opnd(uint8_t* dst, const CUtensorMap* map, 
   }
 }
 
-template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, int EPI_WARPS, class Epi, class P>
+template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, int EPI_WARPS, class Epi, class P,
+          int EPI_SMEM = 0>
 __global__ void __launch_bounds__((2 + EPI_WARPS) * 32, 1)
 gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) {
   using C_ = Cfg<BN, NUM_ACC, A_MN, B_MN>;
+  static_assert(EPI_SMEM % 1024 == 0, "epilogue buffers stay 1024-byte aligned");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * C_::kStage);
+  uint8_t* epi_smem = smem + (size_t)STAGES * C_::kStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + (size_t)EPI_WARPS * EPI_SMEM);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* epi_bar = acc_empty + 2;     // [2 per epilogue warp]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + 2 * EPI_WARPS);
   __shared__ int s_err;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -182,6 +192,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS);
     }
+    for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&epi_bar[w], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -291,6 +302,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
     // ---------------- epilogue
     const int ew = warp - 2;
     const int quad = warp & 3;
+    uint32_t uses[2] = {0u, 0u};
     int i = 0;
     for (int t = blockIdx.x; t < job.total_tiles; t += gridDim.x, ++i) {
       int c, z, mt, nt;
@@ -308,14 +320,20 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       ctx.m0 = mt * BM;
       ctx.n0 = nt * BN;
       ctx.row = quad * 32 + lane;
+      ctx.quad = quad;
       ctx.nparts = EPI_WARPS / 4;
       ctx.part = ew >> 2;
       ctx.taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * C_::kAccCols);
+      ctx.wsmem = epi_smem + (size_t)ew * EPI_SMEM;
+      ctx.wbar = epi_bar + 2 * ew;
+      ctx.uses = uses;
       if (!s_err) Epi::run(prm, ctx);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
+    if (EPI_SMEM > 0 && lane == 0) tc::bulk_wait_all();  // our TMA stores have completed
+    __syncwarp();
   }
   __syncthreads();
   if (warp == 1) {
