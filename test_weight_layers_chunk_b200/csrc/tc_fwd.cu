@@ -39,6 +39,8 @@ struct FwdP {
   // and the bf16 operand copies it writes; index = tile class (0: [W1; W3] or W,
   // 1: W2). Rebuilt for every chunk.
   CUtensorMap srcW[2], srcM[2], dstW[2], dstM[2], shadow[2];
+  // 32 x 32 bf16 tiles (64B swizzle) moved by the other epilogues
+  CUtensorMap mA, mSk, mOut, mV, mE, mEa, mEb, mdH;
   Dims d;
   int ci, t0, write_shadow;
   int* status;
@@ -56,32 +58,45 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ void st_row32(bf16* dst, const float (&v)[32]) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    p[i] = make_uint4(pack2(v[8 * i], v[8 * i + 1]), pack2(v[8 * i + 2], v[8 * i + 3]),
-                      pack2(v[8 * i + 4], v[8 * i + 5]), pack2(v[8 * i + 6], v[8 * i + 7]));
-}
-__device__ __forceinline__ void ld_row32(const bf16* src, float (&v)[32]) {
-  const uint4* p = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 u = p[i];
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[j]));
-      v[8 * i + 2 * j] = f.x;
-      v[8 * i + 2 * j + 1] = f.y;
-    }
-  }
-}
-__device__ __forceinline__ float fast_sigmoid(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 // Row of the interleaved [W1; W3] operand copy that holds row r of W1 (which=0) or W3 (which=1).
 __device__ __forceinline__ int w13_row(int r, int which) {
   return (r / HB) * (2 * HB) + which * HB + (r % HB);
 }
+// Staging tile = one TMA box of make_map_box32: 32 rows x 32 bf16, row r at
+// r * 64 bytes with its 16-byte chunks permuted by the 64B swizzle.
+__device__ __forceinline__ int sw64(int r, int q) { return r * 64 + ((q ^ ((r >> 1) & 3)) << 4); }
+__device__ __forceinline__ void stage32(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(buf + sw64(r, q)) =
+        make_uint4(pack2(v[8 * q], v[8 * q + 1]), pack2(v[8 * q + 2], v[8 * q + 3]),
+                   pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
+}
+__device__ __forceinline__ void unstage32(const uint8_t* buf, int r, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = *reinterpret_cast<const uint4*>(buf + sw64(r, q));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      v[8 * q + 2 * j] = f.x;
+      v[8 * q + 2 * j + 1] = f.y;
+    }
+  }
+}
+// Before refilling staging tiles: this warp's earlier TMA stores must have read them.
+__device__ __forceinline__ void staging_free(int lane) {
+  if (lane == 0) tc::bulk_wait_read<0>();
+  __syncwarp();
+}
+// After filling staging tiles: make them visible to the TMA (async) proxy.
+__device__ __forceinline__ void staging_ready() {
+  tc::fence_async_smem();
+  __syncwarp();
+}
+
 template <int BN>
 __device__ __forceinline__ void ld2(const EpiCtx<BN>& c, int acc0, int col0, int acc1, int col1,
                                     float (&x)[32], float (&y)[32]) {
@@ -105,23 +120,31 @@ __device__ __forceinline__ void ld1(const EpiCtx<BN>& c, int acc, int col, float
 }
 
 // ---------------------------------------------------------------- epilogues
+// Epilogues of G1-G3: each warp owns 32 rows (its TMEM lane quadrant) and a
+// share of the tile's columns; results are staged in shared memory and written
+// with TMA stores, inputs they need (V, silu factors) are prefetched with TMA.
+
 // G1, SwiGLU. Class 0 = query rows, class 1 = key rows of the chunk.
 struct EpiG1 {
+  static constexpr int kSmem = 6144;  // A | silu(H1) | H3 silu'(H1) staging
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;  // first token row of this warp
     const int j0 = (c.n0 / (2 * HB)) * HB;
     const int per = HB / c.nparts;
-    bf16* arow = p.A + ((size_t)c.z * 2 * d.C + (size_t)c.cls * d.C + t) * d.d_h + j0;
-    bf16* srow = p.Sk + ((size_t)c.z * d.C + t) * 2 * d.d_h + j0;
+    const int yA = c.z * 2 * d.C + c.cls * d.C + r0;
+    const int ySk = c.z * d.C + r0;
+    uint8_t* S = c.wsmem;
     for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
       float h1[32], h3[32];
       ld2(c, 0, g, 0, HB + g, h1, h3);
       if (c.cls == 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) h1[i] = h1[i] * fast_sigmoid(h1[i]) * h3[i];
-        st_row32(arow + g, h1);
+        staging_free(lane);
+        stage32(S, lane, h1);
       } else {
         float s2[32];
 #pragma unroll
@@ -132,90 +155,171 @@ struct EpiG1 {
           h3[i] = s1 * h3[i];  // u
           h1[i] = s1;
         }
-        st_row32(arow + g, h3);
-        st_row32(srow + g, h1);
-        st_row32(srow + d.d_h + g, s2);
+        staging_free(lane);
+        stage32(S, lane, h3);
+        stage32(S + 2048, lane, h1);
+        stage32(S + 4096, lane, s2);
       }
+      staging_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mA, S, j0 + g, yA);
+        if (c.cls == 1) {
+          tc::tma_store_2d(&p.mSk, S + 2048, j0 + g, ySk);
+          tc::tma_store_2d(&p.mSk, S + 4096, d.d_h + j0 + g, ySk);
+        }
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
 
-// Key rows: e = y - v (or -v); E (if requested) and its a-/b-scaled copies.
+// Query rows -> out, key rows -> E (optional) and its a-/b-scaled copies, for a
+// warp's 32 rows and its column groups; V of the key rows is prefetched.
 template <int BN>
-__device__ __forceinline__ void key_rows_epilogue(const FwdP& p, const EpiCtx<BN>& c, int t, int col0,
-                                                  float (&y)[32], bool write_e) {
+__device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>& c, bool key_rows,
+                                                int r0, bool write_e) {
   const Dims& d = p.d;
-  const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-  float vv[32];
-  ld_row32(p.v + tok * d.d_v + col0, vv);
+  const int lane = c.row & 31;
+  const int per = BN / c.nparts;
+  const int col0 = c.n0 + c.part * per;
+  static_assert(BN <= 128, "two V buffers: at most two 32-column groups per warp");
+  const int ngroups = per / 32;
+  uint8_t* V = c.wsmem;            // [2][2 KB]
+  uint8_t* S = c.wsmem + 4096;     // E | Ea | Eb staging
+  const int ytok = c.z * d.T + p.t0 + r0;
+  const int yrow = c.z * d.C + r0;
+  if (key_rows) {
+    if (lane == 0) {
+      tc::mbar_expect_tx(&c.wbar[0], 2048u * ngroups);
+      for (int gi = 0; gi < ngroups; ++gi)
+        tc::tma_load_2d(V + gi * 2048, &p.mV, &c.wbar[0], col0 + gi * 32, ytok);
+    }
+    __syncwarp();
+  }
+  float at = 0.f, bt = 0.f;
+  if (key_rows) {
+    const size_t tok = (size_t)ytok + lane;
+    at = p.ca[tok];
+    bt = p.cb[tok];
+  }
+  for (int gi = 0; gi < ngroups; ++gi) {
+    const int col = col0 + gi * 32;
+    float y[32];
+    ld1(c, 0, c.part * per + gi * 32, y);
+    if (!key_rows) {
+      staging_free(lane);
+      stage32(S, lane, y);
+      staging_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mOut, S, col, ytok);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+      continue;
+    }
+    if (gi == 0) {
+      const bool ok = tc::mbar_wait(&c.wbar[0], c.uses[0] & 1u);
+      c.uses[0] += 1;
+      if (!ok) {
+        if (lane == 0) atomicExch(p.status, tc2::kErrEpilogue);
+        return;
+      }
+    }
+    float vv[32];
+    unstage32(V + gi * 2048, lane, vv);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
-  const size_t o = ((size_t)c.z * d.C + t) * d.d_v + col0;
-  if (write_e) st_row32(p.E + o, y);
-  const float at = p.ca[tok], bt = p.cb[tok];
+    for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
+    staging_free(lane);
+    if (write_e) stage32(S, lane, y);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) vv[i] = at * y[i];
-  st_row32(p.Ea + o, vv);
+    for (int i = 0; i < 32; ++i) vv[i] = at * y[i];
+    stage32(S + 2048, lane, vv);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) vv[i] = bt * y[i];
-  st_row32(p.Eb + o, vv);
+    for (int i = 0; i < 32; ++i) vv[i] = bt * y[i];
+    stage32(S + 4096, lane, vv);
+    staging_ready();
+    if (lane == 0) {
+      if (write_e) tc::tma_store_2d(&p.mE, S, col, yrow);
+      tc::tma_store_2d(&p.mEa, S + 2048, col, yrow);
+      tc::tma_store_2d(&p.mEb, S + 4096, col, yrow);
+      tc::bulk_commit();
+    }
+    __syncwarp();
+  }
 }
 
 // G2, SwiGLU: rows [0, C) are queries (-> out), [C, 2C) keys (-> E).
 struct EpiG2 {
+  static constexpr int kSmem = 10240;  // V[2] | E | Ea | Eb
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
-    const Dims& d = p.d;
-    const int m = c.m0 + c.row;
-    const int per = BN / c.nparts;
-    for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
-      float y[32];
-      ld1(c, 0, g, y);
-      const int col = c.n0 + g;
-      if (m < d.C) st_row32(p.out + ((size_t)c.z * d.T + p.t0 + m) * d.d_v + col, y);
-      else key_rows_epilogue(p, c, m - d.C, col, y, true);
-    }
+    const int r0 = c.m0 + c.quad * 32;
+    const bool key_rows = c.m0 >= p.d.C;
+    out_or_residual(p, c, key_rows, key_rows ? r0 - p.d.C : r0, true);
   }
 };
 
 // G1, linear: class 0 = queries (-> out), class 1 = keys (-> scaled E).
 struct EpiG1Lin {
+  static constexpr int kSmem = 10240;
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
-    const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    const int per = BN / c.nparts;
-    for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
-      float y[32];
-      ld1(c, 0, g, y);
-      const int col = c.n0 + g;
-      if (c.cls == 0) st_row32(p.out + ((size_t)c.z * d.T + p.t0 + t) * d.d_v + col, y);
-      else key_rows_epilogue(p, c, t, col, y, false);
-    }
+    out_or_residual(p, c, c.cls == 1, c.m0 + c.quad * 32, false);
   }
 };
 
 // G3, SwiGLU: dA -> dH1 = dA H3 silu'(H1), dH3 = dA silu(H1) (rows: tokens).
 struct EpiG3 {
+  static constexpr int kSmem = 12288;  // silu factors [2 groups][2] | dH1 | dH3
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;
     const int per = BN / c.nparts;
-    const size_t row = ((size_t)c.z * d.C + t) * 2 * d.d_h;
-    for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
+    const int col0 = c.n0 + c.part * per;
+    static_assert(BN <= 128, "silu-factor buffers for at most two column groups per warp");
+    const int ngroups = per / 32;
+    const int y = c.z * d.C + r0;
+    uint8_t* F = c.wsmem;          // [group][s1 | s2] 2 KB each
+    uint8_t* S = c.wsmem + 8192;   // dH1 | dH3 staging
+    if (lane == 0) {
+      tc::mbar_expect_tx(&c.wbar[0], 4096u * ngroups);
+      for (int gi = 0; gi < ngroups; ++gi) {
+        tc::tma_load_2d(F + gi * 4096, &p.mSk, &c.wbar[0], col0 + gi * 32, y);
+        tc::tma_load_2d(F + gi * 4096 + 2048, &p.mSk, &c.wbar[0], d.d_h + col0 + gi * 32, y);
+      }
+    }
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
       float da[32], s1[32], s2[32];
-      const int j = c.n0 + g;
-      ld_row32(p.Sk + row + j, s1);
-      ld_row32(p.Sk + row + d.d_h + j, s2);
-      ld1(c, 0, g, da);
+      ld1(c, 0, c.part * per + gi * 32, da);
+      if (gi == 0) {
+        const bool ok = tc::mbar_wait(&c.wbar[0], c.uses[0] & 1u);
+        c.uses[0] += 1;
+        if (!ok) {
+          if (lane == 0) atomicExch(p.status, tc2::kErrEpilogue);
+          return;
+        }
+      }
+      unstage32(F + gi * 4096, lane, s1);
+      unstage32(F + gi * 4096 + 2048, lane, s2);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         s2[i] *= da[i];  // dH1
         s1[i] *= da[i];  // dH3
       }
-      st_row32(p.dH + row + j, s2);
-      st_row32(p.dH + row + d.d_h + j, s1);
+      staging_free(lane);
+      stage32(S, lane, s2);
+      stage32(S + 2048, lane, s1);
+      staging_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mdH, S, col0 + gi * 32, y);
+        tc::tma_store_2d(&p.mdH, S + 2048, d.d_h + col0 + gi * 32, y);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -527,7 +631,6 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   // Operand maps (chunk-independent; the chunk offset goes into the coordinates).
   tc2::Job g1{}, g2{}, g3{}, g4{};
   bool ok = true;
-  const bool bn_v = dv % 256 == 0;
   for (tc2::Job* j : {&g1, &g2, &g3, &g4}) {
     j->heads = BH;
     j->status = status;
@@ -567,17 +670,28 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   } else {
     ok &= make_map(&g1.maps[0].op0, q, (uint64_t)BH * T, dk, 128);
     ok &= make_map(&g1.maps[1].op0, k, (uint64_t)BH * T, dk, 128);
-    ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * dv, dk, bn_v ? 256 : 128);
+    ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * dv, dk, 128);
     g1.maps[1].op2 = g1.maps[0].op2;
     g1.n_cls = 2;
     for (int c = 0; c < 2; ++c)
-      g1.cls[c] = tc2::Class{C / 128, dv / (bn_v ? 256 : 128), dk / 64, {T, 0, 0}, {dv, 0, 0}, 0};
+      g1.cls[c] = tc2::Class{C / 128, dv / 128, dk / 64, {T, 0, 0}, {dv, 0, 0}, 0};
     // G4: A0 = diag(a) E, A1 = diag(b) E (M = rows of W), B = K (N = d_k, K = tokens)
     ok &= make_map(&g4.maps[0].op0, s.Ea, (uint64_t)BH * C, dv, 64);
     ok &= make_map(&g4.maps[0].op1, s.Eb, (uint64_t)BH * C, dv, 64);
     ok &= make_map(&g4.maps[0].op2, k, (uint64_t)BH * T, dk, 64);
     g4.n_cls = 1;
     g4.cls[0] = tc2::Class{dv / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, kModeA2B1};
+  }
+  // 32 x 32 tiles of the epilogues (bf16, 64B swizzle)
+  ok &= make_map_box32(&p.mOut, out, (uint64_t)BH * T, dv);
+  ok &= make_map_box32(&p.mV, v, (uint64_t)BH * T, dv);
+  ok &= make_map_box32(&p.mEa, s.Ea, (uint64_t)BH * C, dv);
+  ok &= make_map_box32(&p.mEb, s.Eb, (uint64_t)BH * C, dv);
+  if (d.kind == 1) {
+    ok &= make_map_box32(&p.mA, s.A, (uint64_t)BH * 2 * C, dh);
+    ok &= make_map_box32(&p.mSk, s.Sk, (uint64_t)BH * C, 2 * dh);
+    ok &= make_map_box32(&p.mE, s.E, (uint64_t)BH * C, dv);
+    ok &= make_map_box32(&p.mdH, s.dH, (uint64_t)BH * C, 2 * dh);
   }
   if (!ok) return cudaErrorInvalidValue;
 
@@ -606,13 +720,12 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     g1.cls[0].a.y_base = g1.cls[1].a.y_base = ci * C;  // query / key rows of this chunk
     g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
     if (d.kind == 1) {
-      e = launch<256, 1, false, false, 4, EpiG1>(g1, p, st);
-      if (e == cudaSuccess) e = launch<128, 1, false, false, 6, EpiG2>(g2, p, st);
-      if (e == cudaSuccess) e = launch<128, 1, false, true, 6, EpiG3>(g3, p, st);
+      e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
+      if (e == cudaSuccess) e = launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
+      if (e == cudaSuccess) e = launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st);
       if (e == cudaSuccess) e = launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
     } else {
-      e = bn_v ? launch<256, 1, false, false, 4, EpiG1Lin>(g1, p, st)
-               : launch<128, 1, false, false, 6, EpiG1Lin>(g1, p, st);
+      e = launch<128, 1, false, false, 4, EpiG1Lin, kEpiWarps, EpiG1Lin::kSmem>(g1, p, st);
       if (e == cudaSuccess) e = launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
     }
     if (e != cudaSuccess) return e;
