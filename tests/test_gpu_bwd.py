@@ -1,0 +1,111 @@
+"""GPU parity of e2ttt_chunk_scan_bwd against the fp64 oracle's adjoint.
+
+The oracle's closed-form adjoint is pinned on the CPU to the per-token reverse
+loop and to finite differences (tests/test_oracle.py). Here the GPU forward
+saves the chunk-start states, the GPU backward consumes them, and every
+gradient (dq, dk, dv, dlr, dmom, ddecay, dW0, dM0) is compared with the oracle
+at tensor level: 1e-4 relative Frobenius error for fp32 activations, 2e-2 for
+bf16 activations (bf16 inputs and forward operands).
+"""
+import numpy as np
+import pytest
+
+import e2ttt_inputs as gen
+import oracle as O
+from gpu_util import dev, device_inputs, host, run_fwd
+
+pytestmark = pytest.mark.gpu
+NAMES = ("dq", "dk", "dv", "dlr", "dmom", "ddecay", "dW0", "dM0")
+
+
+@pytest.fixture(scope="module")
+def E():
+    import torch
+    assert torch.cuda.is_available()
+    import test_weight_layers_chunk_b200 as E
+    return E
+
+
+def err(x, ref):
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-30 * np.sqrt(ref.size)))
+
+
+def run_bwd(E, w, x, dW, dM, heads=None):
+    import torch
+    d = device_inputs(w, x)
+    _, _, _, saved = run_fwd(E, w, d, save=True)
+    g = E.chunk_scan_bwd(d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], saved, d["dout"],
+                         None if dW is None else dev(dW), None if dM is None else dev(dM),
+                         C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss)
+    torch.cuda.synchronize()
+    gpu = {n: host(t) for n, t in g.items()}
+    ref = O.closed_bwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"],
+                       x["M0"], w.C, x["dout"], dW, dM, d_h=w.d_h, loss=w.loss, heads=heads)
+    return gpu, ref
+
+
+def check(gpu, ref, tol, heads=None, label=""):
+    if heads is None:
+        errs = {n: err(gpu[n], ref[n]) for n in NAMES}
+    else:
+        bi = tuple(np.array(heads).T)
+        errs = {n: err(gpu[n][bi], ref[n][bi]) for n in NAMES}
+    print(f"\n{label}: " + " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
+    bad = {n: e for n, e in errs.items() if not e < tol}
+    assert not bad, (label, bad)
+
+
+F32 = {
+    "linear_mse": gen.Workload("bl", gen.LINEAR, gen.F32, 1, 2, 24, 16, 0, 70, 32, "uniform", 0.99,
+                               seed=41),
+    "linear_dot": gen.Workload("bld", gen.LINEAR, gen.F32, 2, 1, 16, 24, 0, 64, 16, "uniform", 0.99,
+                               seed=42, loss=gen.LOSS_NEG_DOT),
+    "swiglu_mse": gen.Workload("bs", gen.SWIGLU, gen.F32, 1, 2, 16, 12, 24, 50, 16, "uniform", 0.99,
+                               seed=43, lr_lo=0.002, lr_hi=0.02, mom_lo=0.7, mom_hi=0.95),
+    "swiglu_dot": gen.Workload("bsd", gen.SWIGLU, gen.F32, 2, 1, 12, 16, 20, 48, 16, "uniform", 0.99,
+                               seed=44, loss=gen.LOSS_NEG_DOT, lr_lo=0.001, lr_hi=0.005,
+                               mom_lo=0.5, mom_hi=0.9),
+}
+
+
+@pytest.mark.parametrize("name", list(F32))
+@pytest.mark.parametrize("upstream", [True, False])
+def test_bwd_f32_matches_oracle(E, name, upstream):
+    w = F32[name]
+    x = gen.generate(w, m0_scale=0.5)
+    dW, dM = gen.upstream_state_grads(w, seed=7, scale=0.3) if upstream else (None, None)
+    gpu, ref = run_bwd(E, w, x, dW, dM)
+    check(gpu, ref, 1e-4, label=f"{name} upstream={upstream}")
+
+
+def test_bwd_tiny_linear_workload(E):
+    """The tiny linear fp32 workload at its full size (256 tokens, 4 chunks)."""
+    w = gen.BY_NAME["tiny_linear"]
+    x = gen.generate(w)
+    dW, dM = gen.upstream_state_grads(w, seed=0)
+    gpu, ref = run_bwd(E, w, x, dW, dM)
+    check(gpu, ref, 1e-4, label="tiny_linear")
+
+
+def test_bwd_bf16_small(E):
+    w = gen.Workload("bb", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform", 0.999,
+                     seed=45, lr_lo=0.002, lr_hi=0.02)
+    x = gen.generate(w, m0_scale=0.5)
+    dW, dM = gen.upstream_state_grads(w, seed=8, scale=0.1)
+    gpu, ref = run_bwd(E, w, x, dW, dM)
+    check(gpu, ref, 2e-2, label="swiglu_bf16_small")
+
+
+@pytest.mark.parametrize("variant", ["stated", "preserving"])
+def test_bwd_training_workload(E, variant):
+    """fwd then bwd at the 1.3B layer's shapes (B=4, H=8, d=256, d_h=512, T=2048,
+    C=512), upstream dOut ~ N(0,1); the oracle recomputes two heads."""
+    w = gen.BY_NAME["train_1p3b_2k"]
+    if variant == "preserving":
+        w = gen.state_preserving(w)
+    x = gen.generate(w, m0_scale=0.0 if variant == "stated" else 0.5)
+    heads = [(0, 0), (3, 7)]
+    gpu, ref = run_bwd(E, w, x, None, None, heads=heads)
+    check(gpu, ref, 2e-2, heads=heads, label=f"train_1p3b_2k {variant}")
