@@ -57,8 +57,28 @@ def phase_flops_per_token_head(w) -> dict:
             "tc_g4_aggregate_state": 8 * dh * dk + 4 * dv * dh}  # two aggregations x 3 matrices
 
 
+# Backward kernels of the CUDA-core path (fp32 FMA), algorithmic FLOPs per token
+# and head (SwiGLU, d_k = d_v); bwd_h / bwd_residual / bwd_da recompute the
+# forward internals at the chunk-start weights.
+BWD_SIMT_FLOPS = {"bwd_dk": 12, "bwd_dw2": 6, "bwd_dir_w13": 8, "bwd_h": 8, "bwd_dw13": 8,
+                  "bwd_dir_w2": 4, "bwd_residual": 2, "bwd_ub_dir": 4, "bwd_dq": 4, "bwd_eb": 2,
+                  "bwd_q_rows": 2, "bwd_da": 2, "bwd_ub_eb": 2}
+
+
 def fwd_flops(w) -> float:
     return float(sum(phase_flops_per_token_head(w).values())) * w.B * w.H * w.T
+
+
+def train_flops(w) -> float:
+    """Forward 26 d d_h plus backward 52 d d_h per token and head (SwiGLU,
+    d_k = d_v = d; the backward's recomputation of the forward is not counted)."""
+    return 78.0 * w.d_k * w.d_h * w.B * w.H * w.T
+
+
+def fp32_fma_peak_tflops(sm_mhz: float) -> float:
+    """CUDA-core fp32 peak from unit counts: 148 SMs x 128 FP32 lanes x 2 FLOP
+    per FMA x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 def algorithmic_bytes(w) -> float:
@@ -231,6 +251,59 @@ def config_dict(w, args):
             "l2": "working set larger than L2 (no flush)"}
 
 
+# ----------------------------------------------------------------- extra lines
+def _timed(torch, stream, fn, steps):
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        fn()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1) / steps
+
+
+def measure_extras(E, torch, dev, stream, args):
+    """The metric's other operating points, device-timed like the main line:
+    forward at T = 16K (the 8x length-extrapolation layer) and forward+backward at
+    T = 2K (the training workload), each with its own warm-up."""
+    out = {}
+    f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
+    for name, train, steps in (("layer_1p3b_16k", False, args.extra_steps),
+                               ("train_1p3b_2k", True, max(2, args.extra_steps // 8))):
+        w = gen.BY_NAME[name]
+        x = gen.generate(w)
+        q, k, v = f(x["q"], torch.bfloat16), f(x["k"], torch.bfloat16), f(x["v"], torch.bfloat16)
+        lr, mom, decay, W0 = f(x["lr"]), f(x["mom"]), f(x["decay"]), f(x["W0"])
+        shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss)
+        nc = E.e2ttt_num_chunks(shape)
+        outb, We, Me = torch.empty_like(v), torch.empty_like(W0), torch.empty_like(W0)
+        saved = torch.empty((nc, w.B, w.H, 2, w.state_elems), device=dev) if train else None
+        ws = E.workspace(shape, False, dev)
+        if train:
+            dout = f(x["dout"], torch.bfloat16)
+            g = [torch.empty_like(t) for t in (q, k, v, lr, mom, decay, W0, W0)]
+            wsb = E.workspace(shape, True, dev)
+
+        def step():
+            E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, None, outb, We, Me, saved, ws,
+                                   stream=stream)
+            if train:
+                E.e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved, dout, None, None, *g,
+                                       wsb, stream=stream)
+
+        for _ in range(3):
+            step()
+        ms = _timed(torch, stream, step, steps)
+        flops = train_flops(w) if train else fwd_flops(w)
+        out[("fwd_bwd_" if train else "fwd_") + name] = {
+            "value": w.B * w.T / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "tflops": flops / (ms / 1e3) / 1e12, "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / measured_peaks()["bf16_tflops"]}
+        del q, k, v, outb, We, Me, saved, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------- our path
 def run_ours(args, w):
     import torch
@@ -270,9 +343,21 @@ def run_ours(args, w):
     ws = E.workspace(shape, False, dev)
     stream = torch.cuda.current_stream(dev)
 
+    if train:
+        dout = f(x["dout"], ad)
+        grads = {n: torch.empty_like(t) for n, t in (("dq", q), ("dk", k), ("dv", v), ("dlr", lr),
+                                                       ("dmom", mom), ("ddecay", decay))}
+        dW0g = torch.empty_like(W0)
+        dM0g = torch.empty_like(W0)
+        wsb = E.workspace(shape, True, dev)
+
     def step():
         E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, M0, out, W_end, M_end, saved, ws,
                                stream=stream)
+        if train:
+            E.e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved, dout, None, None,
+                                   grads["dq"], grads["dk"], grads["dv"], grads["dlr"],
+                                   grads["dmom"], grads["ddecay"], dW0g, dM0g, wsb, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -302,23 +387,36 @@ def run_ours(args, w):
 
     # roofline of the dominant kernel
     peaks = measured_peaks()
+    clocks = clk.summary()
     ph = phase_flops_per_token_head(w)
     kern = trace["kernels"]
-    dom = max((n for n in kern if n in ph), key=lambda n: kern[n]["total_ms"])
+    known = {n: ("tensor", f) for n, f in ph.items()}
+    if w.kind == gen.SWIGLU and w.d_k == w.d_v:
+        known.update({n: ("alu", f) for n, f in BWD_SIMT_FLOPS.items()})
+    dom = max((n for n in kern if n in known), key=lambda n: kern[n]["total_ms"])
+    bound, per_th = known[dom]
     avg_ms = kern[dom]["total_ms"] / kern[dom]["launches"]
-    flops_launch = ph[dom] * w.B * w.H * w.C   # one launch = one chunk of every head
+    flops_launch = per_th * w.d_k * w.d_h * w.B * w.H * w.C if bound == "alu" else \
+        ph[dom] * w.B * w.H * w.C  # one launch = one chunk of every head
     achieved = flops_launch / (avg_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"],
-                "peak_source": peaks["source"] + " (burst bf16 GEMM)",
+    if bound == "tensor":
+        peak, psrc = peaks["bf16_tflops"], peaks["source"] + " (burst bf16 GEMM)"
+    else:
+        peak = fp32_fma_peak_tflops(clocks.get("sm_max_mhz") or 1965.0)
+        psrc = "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"
+    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": psrc,
                 "traffic": recorded_traffic(dom, w.name),
                 "share_of_step": kern[dom]["total_ms"] / ms}
-    step_flops = fwd_flops(w)
+    step_flops = train_flops(w) if train else fwd_flops(w)
     whole = {"achieved_tflops": step_flops / (ms / args.steps / 1e3) / 1e12}
     whole["frac"] = whole["achieved_tflops"] / peaks["bf16_tflops"]
     kernels = {n: {"launches": kv["launches"], "avg_us": 1e3 * kv["total_ms"] / kv["launches"],
                    "share": kv["total_ms"] / ms} for n, kv in kern.items()}
+
+    extras = {}
+    if args.extras and rank == 0 and world == 1 and not train:
+        extras = measure_extras(E, torch, dev, stream, args)
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -363,8 +461,8 @@ def run_ours(args, w):
                 "data": "synthetic (seeded numpy; shapes and distributions of the workload)",
                 "config": config_dict(w, argparse.Namespace(gpus=world, mode=args.mode)),
                 "roofline": roofline, "step_roofline": whole, "kernels": kernels,
-                "gpu_launches": trace["launches"], "clocks": clk.summary(),
-                "cpu_baseline": cpu_baseline, "e2e": e2e}
+                "gpu_launches": trace["launches"], "clocks": clocks,
+                "cpu_baseline": cpu_baseline, "e2e": e2e, "extra": extras}
         print(json.dumps(line))
     if world > 1:
         torch.distributed.barrier()
@@ -377,14 +475,19 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="layer_1p3b_2k", choices=[w.name for w in gen.WORKLOADS])
+    ap.add_argument("--workload", default=None, choices=[w.name for w in gen.WORKLOADS],
+                    help="default: layer_1p3b_2k (fwd) or train_1p3b_2k (train)")
     ap.add_argument("--mode", choices=["fwd", "train"], default="fwd")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extras", type=int, default=1, help="also time T=16K fwd and T=2K fwd+bwd")
+    ap.add_argument("--extra-steps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload is None:
+        args.workload = "train_1p3b_2k" if args.mode == "train" else "layer_1p3b_2k"
     w = gen.BY_NAME[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
