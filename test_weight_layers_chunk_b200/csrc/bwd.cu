@@ -20,6 +20,10 @@
 //   h1b = dh1b du h3 s'' + sb s',  dv = -eb,
 //   dk = -(G1^T dh1 + G3^T dh3) + W1^T h1b + W3^T h3b,
 //   dW2 += e dub^T + eb u^T (MSE),  dW1 += h1b k^T,  dW3 += h3b k^T.
+#include <stdint.h>
+
+#include <initializer_list>
+
 #include "paths.h"
 #include "simt.cuh"
 #include "state.cuh"
@@ -29,7 +33,7 @@ namespace {
 
 // Scratch of the backward (fp32), per head, C rows per chunk.
 struct BwdWs {
-  size_t a, b, scal, abar, bbar, sbar, part;
+  size_t status, a, b, scal, abar, bbar, sbar, part;
   size_t H, E, dA, P, P2, UB, DUB, EB, UB5, HB, GK;
   size_t total;
 };
@@ -43,6 +47,7 @@ BwdWs bwd_layout(const Dims& d) {
   };
   const size_t BH = d.BH, C = d.C, dh = d.d_h, dv = d.d_v;
   BwdWs L{};
+  L.status = take(64);  // status word (read by e2ttt_workspace_status; always 0 here)
   L.a = take(BH * d.T);
   L.b = take(BH * d.T);
   L.scal = take(3 * BH * d.NC);
@@ -559,11 +564,27 @@ cudaError_t chunk_bwd(const Bwd<TA>& c, cudaStream_t st) {
 
 }  // namespace
 
-size_t bwd_workspace_bytes(const Dims& d, bool) { return bwd_layout(d).total; }
+size_t bwd_workspace_bytes(const Dims& d, bool bf16_act) {
+  size_t n = bwd_layout(d).total;
+  if (tc_bwd_supported(d, bf16_act)) {
+    const size_t t = tc_bwd_workspace_bytes(d);
+    if (t > n) n = t;
+  }
+  return n;
+}
+
+static bool aligned16(std::initializer_list<const void*> ps) {
+  for (const void* q : ps)
+    if (((uintptr_t)q) & 15) return false;
+  return true;
+}
 
 template <typename TA>
 cudaError_t bwd_run(const BwdArgs& A) {
   const Dims& d = A.d;
+  if (sizeof(TA) == 2 && tc_bwd_supported(d, true) &&
+      aligned16({A.q, A.k, A.v, A.dout, A.dq, A.dk, A.dv, A.saved, A.dW0, A.dM0}))
+    return tc_bwd(A);
   BwdWs L = bwd_layout(d);
   char* w = (char*)A.ws;
   Bwd<TA> c;
@@ -583,7 +604,9 @@ cudaError_t bwd_run(const BwdArgs& A) {
   c.DM = A.dM0;
   cudaStream_t st = A.st;
   const size_t sbytes = (size_t)d.BH * d.S * sizeof(float);
-  cudaError_t e = launch_chunk_coeffs(A.lr, A.mom, A.decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, st);
+  cudaError_t e = cudaMemsetAsync(w + L.status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  e = launch_chunk_coeffs(A.lr, A.mom, A.decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, st);
   if (e != cudaSuccess) return e;
   e = A.dW_end ? cudaMemcpyAsync(A.dW0, A.dW_end, sbytes, cudaMemcpyDeviceToDevice, st)
                : cudaMemsetAsync(A.dW0, 0, sbytes, st);

@@ -47,4 +47,9 @@ size_t bwd_workspace_bytes(const Dims& d, bool bf16_act);
 template <typename TA>
 cudaError_t bwd_run(const BwdArgs& a);
 
+// tcgen05 tensor-core backward (tc_bwd.cu): SwiGLU, bf16, tile-aligned shapes.
+bool tc_bwd_supported(const Dims& d, bool bf16_act);
+size_t tc_bwd_workspace_bytes(const Dims& d);
+cudaError_t tc_bwd(const BwdArgs& a);
+
 }  // namespace e2ttt

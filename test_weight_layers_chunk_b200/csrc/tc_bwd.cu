@@ -1,0 +1,830 @@
+// tcgen05 tensor-core backward of the chunk scan (SwiGLU, bf16 activations).
+//
+// Same mathematics as the CUDA-core backward (bwd.cu): the adjoint of the
+// closed-form chunk transition ("Rethinking Expressivity and Efficiency in
+// Test-Time Training": abstract, fully parallelized chunk-level training),
+// chunks in reverse, second-order terms through the loss gradient included.
+// Per chunk, all heads at once (token-major bf16 operands, fp32 epilogue data):
+//   R1  [K; Q] -> H1 = X W1^T, H3 = X W3^T (two accumulators) ; u = silu(H1) H3
+//   R2  E = U_k W2^T - V            R3  du = E W2 -> dH1 = du H3 silu'(H1), dH3 = du silu(H1)
+//   D1  K [D_M13 | D_W13]^T -> dh1b/dh3b = -(a P_M + b P_W) and the abar/bbar dot products
+//   D2  U_k [D_M2 | D_W2]^T -> G2u = -(a P_M + b P_W) and the abar/bbar dot products
+//   E3  E [D_M2 | D_W2] -> -(a . + b .) ; dub = dh1b H3 silu'(H1) + dh3b silu(H1)
+//   E4  eb = dub W2^T + G2u (dv = -eb)    E5  ub = E3 term + eb W2 -> h1b, h3b
+//   Q1  dout W2 -> query-row h1b, h3b
+//   dk = -(a dH D_M13 + b dH D_W13) + [h1b | h3b] [W1; W3] ;  dq = query-row [h1b | h3b] [W1; W3]
+//   dW13 += [h1b | h3b]^T [K; Q] ,  dW2 += [E; EB; dout]^T [dub; U_k; U_q]  (into D_W in place)
+//   dM0 = U(1,n) D_M + c D_W ; abar, bbar and the chunk-scalar adjoints for the gate gradients.
+#include <cuda.h>
+
+#include "paths.h"
+#include "state.cuh"
+#include "tc_gemm2.cuh"
+#include "trace.h"
+
+namespace e2ttt {
+namespace {
+
+using tc2::EpiCtx;
+
+constexpr int kEW = 8;  // epilogue warps
+
+struct BwdP {
+  Dims d;
+  int ci, t0;
+  const bf16 *v;
+  bf16 *dq, *dk, *dv;
+  const float *ca, *cb, *scal;
+  float *DW, *DM;  // fp32 state adjoints (head stride S), in place
+  // bf16 token-major operands (per head)
+  bf16 *X;    // [2C, d_k]   rows: keys, then queries
+  bf16 *Y3;   // [3C, d_h]   rows: dub | u_k | u_q
+  bf16 *Z3;   // [3C, d_v]   rows: E | EB | dout
+  bf16 *Hc;   // [2C, 2 d_h] h1 | h3 (keys, then queries)
+  bf16 *DH;   // [C, 2 d_h]  dH1 | dH3
+  bf16 *HB;   // [2C, 2 d_h] h1b | h3b (keys, then queries)
+  // fp32 epilogue data (per head)
+  float *du;     // [C, d_h]
+  float *DB;     // [C, 2 d_h]  dh1b | dh3b
+  float *G2U;    // [C, d_v]
+  float *UBd;    // [C, d_h]
+  float *dkp;    // [C, d_k]
+  float *part;   // [C, NG]   partial dot products for abar (and bbar at + BH*C*NG)
+  int NG;
+  int* status;
+};
+
+// ---------------------------------------------------------------- row helpers
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ void st32(bf16* dst, const float (&v)[32]) {
+  uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    p[i] = make_uint4(pack2(v[8 * i], v[8 * i + 1]), pack2(v[8 * i + 2], v[8 * i + 3]),
+                      pack2(v[8 * i + 4], v[8 * i + 5]), pack2(v[8 * i + 6], v[8 * i + 7]));
+}
+__device__ __forceinline__ void ld32(const bf16* src, float (&v)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = p[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      v[8 * i + 2 * j] = f.x;
+      v[8 * i + 2 * j + 1] = f.y;
+    }
+  }
+}
+__device__ __forceinline__ void ld32f(const float* src, float (&v)[32]) {
+  const float4* p = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 f = p[i];
+    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+  }
+}
+__device__ __forceinline__ void st32f(float* dst, const float (&v)[32]) {
+  float4* p = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <int BN>
+__device__ __forceinline__ void acc1(const EpiCtx<BN>& c, int col, float (&x)[32]) {
+  uint32_t r[32];
+  tc2::tmem_ld32_nowait(c.taddr + (uint32_t)col, r);
+  tc2::tmem_wait_ld(r);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+}
+template <int BN>
+__device__ __forceinline__ void acc2(const EpiCtx<BN>& c, int col, float (&x)[32], float (&y)[32]) {
+  uint32_t r[32], s[32];
+  tc2::tmem_ld32_nowait(c.taddr + (uint32_t)col, r);
+  tc2::tmem_ld32_nowait(c.taddr + (uint32_t)(BN + col), s);
+  tc2::tmem_wait_ld2(r, s);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    x[i] = __uint_as_float(r[i]);
+    y[i] = __uint_as_float(s[i]);
+  }
+}
+// sigmoid with the fast exponential and reciprocal; silu, silu', silu'' from it.
+struct Act {
+  float s, d1, d2;  // silu(z), silu'(z), silu''(z)
+  __device__ __forceinline__ explicit Act(float z) {
+    const float sg = __fdividef(1.0f, 1.0f + __expf(-z));
+    s = z * sg;
+    d1 = sg * (1.0f + z * (1.0f - sg));
+    d2 = sg * (1.0f - sg) * (2.0f + z * (1.0f - 2.0f * sg));
+  }
+};
+__device__ __forceinline__ float fsilu(float z) { return z * __fdividef(1.0f, 1.0f + __expf(-z)); }
+// 8 consecutive bf16 / fp32 values
+__device__ __forceinline__ void ld8(const bf16* src, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(src);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void ld8f(const float* src, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void st8(bf16* dst, const float (&v)[8]) {
+  *reinterpret_cast<uint4*>(dst) =
+      make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
+}
+// Column groups of 32 owned by this thread inside the tile.
+#define FOR_GROUPS(c, BN, g) \
+  for (int g = (c).part * ((BN) / (c).nparts); g < ((c).part + 1) * ((BN) / (c).nparts); g += 32)
+
+// ---------------------------------------------------------------- epilogues
+// R1: rows of X (keys then queries); h1 = acc0, h3 = acc1.
+struct EpiR1 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int r = c.m0 + c.row;
+    bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + r) * 2 * d.d_h;
+    bf16* urow = p.Y3 + ((size_t)c.z * 3 * d.C + d.C + r) * d.d_h;
+    FOR_GROUPS(c, BN, g) {
+      const int j = c.n0 + g;
+      float h1[32], h3[32];
+      acc2(c, g, h1, h3);
+      st32(hrow + j, h1);
+      st32(hrow + d.d_h + j, h3);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h1[i] = fsilu(h1[i]) * h3[i];
+      st32(urow + j, h1);
+    }
+  }
+};
+// R2: E = y - v (or -v) of the key rows.
+struct EpiR2 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const bf16* vrow = p.v + ((size_t)c.z * d.T + p.t0 + t) * d.d_v;
+    bf16* erow = p.Z3 + ((size_t)c.z * 3 * d.C + t) * d.d_v;
+    FOR_GROUPS(c, BN, g) {
+      const int col = c.n0 + g;
+      float y[32], vv[32];
+      acc1(c, g, y);
+      ld32(vrow + col, vv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
+      st32(erow + col, y);
+    }
+  }
+};
+// R3: du, dH1 = du H3 silu'(H1), dH3 = du silu(H1).
+struct EpiR3 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
+    float* durow = p.du + ((size_t)c.z * d.C + t) * d.d_h;
+    bf16* dhrow = p.DH + ((size_t)c.z * d.C + t) * 2 * d.d_h;
+    FOR_GROUPS(c, BN, g) {
+      const int j = c.n0 + g;
+      float du[32], h1[32], h3[32];
+      acc1(c, g, du);
+      st32f(durow + j, du);
+      ld32(hrow + j, h1);
+      ld32(hrow + d.d_h + j, h3);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const Act f(h1[i]);
+        const float dh1 = du[i] * h3[i] * f.d1;
+        h3[i] = du[i] * f.s;  // dH3
+        h1[i] = dh1;
+      }
+      st32(dhrow + j, h1);
+      st32(dhrow + d.d_h + j, h3);
+    }
+  }
+};
+// D1: acc0 = K D_M13^T, acc1 = K D_W13^T over columns [0, 2 d_h).
+struct EpiD1 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const size_t tok = (size_t)c.z * d.T + p.t0 + t;
+    const float a = p.ca[tok], b = p.cb[tok];
+    const bf16* dhrow = p.DH + ((size_t)c.z * d.C + t) * 2 * d.d_h;
+    float* dbrow = p.DB + ((size_t)c.z * d.C + t) * 2 * d.d_h;
+    float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG;
+    float* pb = pa + (size_t)d.BH * d.C * p.NG;
+    FOR_GROUPS(c, BN, g) {
+      const int jj = c.n0 + g;
+      float pm[32], pw[32], dh[32];
+      acc2(c, g, pm, pw);
+      ld32(dhrow + jj, dh);
+      float sa = 0.f, sb = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        sa += dh[i] * pm[i];
+        sb += dh[i] * pw[i];
+        pm[i] = -(a * pm[i] + b * pw[i]);
+      }
+      st32f(dbrow + jj, pm);
+      pa[jj / 32] = sa;
+      pb[jj / 32] = sb;
+    }
+  }
+};
+// D2: acc0 = U_k D_M2^T, acc1 = U_k D_W2^T over columns [0, d_v).
+struct EpiD2 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const size_t tok = (size_t)c.z * d.T + p.t0 + t;
+    const float a = p.ca[tok], b = p.cb[tok];
+    const bf16* erow = p.Z3 + ((size_t)c.z * 3 * d.C + t) * d.d_v;
+    float* grow = p.G2U + ((size_t)c.z * d.C + t) * d.d_v;
+    float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG + 2 * d.d_h / 32;
+    float* pb = pa + (size_t)d.BH * d.C * p.NG;
+    FOR_GROUPS(c, BN, g) {
+      const int col = c.n0 + g;
+      float pm[32], pw[32], e[32];
+      acc2(c, g, pm, pw);
+      ld32(erow + col, e);
+      float sa = 0.f, sb = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        sa += e[i] * pm[i];
+        sb += e[i] * pw[i];
+        pm[i] = -(a * pm[i] + b * pw[i]);
+      }
+      st32f(grow + col, pm);
+      pa[col / 32] = sa;
+      pb[col / 32] = sb;
+    }
+  }
+};
+// E3: acc0 = E D_M2, acc1 = E D_W2 (columns = hidden units); dub.
+struct EpiE3 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const size_t tok = (size_t)c.z * d.T + p.t0 + t;
+    const float a = p.ca[tok], b = p.cb[tok];
+    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
+    const float* dbrow = p.DB + ((size_t)c.z * d.C + t) * 2 * d.d_h;
+    float* ubrow = p.UBd + ((size_t)c.z * d.C + t) * d.d_h;
+    bf16* dubrow = p.Y3 + ((size_t)c.z * 3 * d.C + t) * d.d_h;
+    FOR_GROUPS(c, BN, g) {
+      const int j = c.n0 + g;
+      float m[32], w[32], h1[32], h3[32];
+      acc2(c, g, m, w);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
+      st32f(ubrow + j, m);
+      ld32(hrow + j, h1);
+      ld32(hrow + d.d_h + j, h3);
+      ld32f(dbrow + j, m);           // dh1b
+      ld32f(dbrow + d.d_h + j, w);   // dh3b
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const Act f(h1[i]);
+        m[i] = m[i] * h3[i] * f.d1 + w[i] * f.s;
+      }
+      st32(dubrow + j, m);
+    }
+  }
+};
+// E4: eb = dub W2^T + G2u; EB row (zero for the dot loss), dv = -eb.
+struct EpiE4 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const float* grow = p.G2U + ((size_t)c.z * d.C + t) * d.d_v;
+    bf16* ebrow = p.Z3 + ((size_t)c.z * 3 * d.C + d.C + t) * d.d_v;
+    bf16* dvrow = p.dv + ((size_t)c.z * d.T + p.t0 + t) * d.d_v;
+    FOR_GROUPS(c, BN, g) {
+      const int col = c.n0 + g;
+      float eb[32], gu[32];
+      acc1(c, g, eb);
+      ld32f(grow + col, gu);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        eb[i] += gu[i];
+        gu[i] = -eb[i];
+      }
+      st32(dvrow + col, gu);
+      if (d.loss != 0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) eb[i] = 0.f;
+      }
+      st32(ebrow + col, eb);
+    }
+  }
+};
+// E5: ub = E3 term + eb W2 (MSE); the key rows' h1b, h3b (8 columns at a time).
+struct EpiE5 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const size_t row = (size_t)c.z * d.C + t;
+    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
+    bf16* hbrow = p.HB + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
+    FOR_GROUPS(c, BN, g) {
+      float acc[32];
+      acc1(c, g, acc);
+#pragma unroll
+      for (int s8 = 0; s8 < 4; ++s8) {
+        const int j = c.n0 + g + 8 * s8;
+        float ubd[8], h1[8], h3[8], du[8], b1[8], b3[8];
+        ld8f(p.UBd + row * d.d_h + j, ubd);
+        ld8(hrow + j, h1);
+        ld8(hrow + d.d_h + j, h3);
+        ld8f(p.du + row * d.d_h + j, du);
+        ld8f(p.DB + row * 2 * d.d_h + j, b1);           // dh1b
+        ld8f(p.DB + row * 2 * d.d_h + d.d_h + j, b3);   // dh3b
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float ub = ubd[i] + (d.loss == 0 ? acc[8 * s8 + i] : 0.f);
+          const Act f(h1[i]);
+          const float sb = b3[i] * du[i] + ub * h3[i];
+          const float h3b = b1[i] * du[i] * f.d1 + ub * f.s;
+          const float h1b = b1[i] * du[i] * h3[i] * f.d2 + sb * f.d1;
+          h1[i] = h1b;
+          h3[i] = h3b;
+        }
+        st8(hbrow + j, h1);
+        st8(hbrow + d.d_h + j, h3);
+      }
+    }
+  }
+};
+// Q1: ub_q = dout W2 -> query-row h1b = ub H3 silu'(H1), h3b = ub silu(H1).
+struct EpiQ1 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + d.C + t) * 2 * d.d_h;
+    bf16* hbrow = p.HB + ((size_t)c.z * 2 * d.C + d.C + t) * 2 * d.d_h;
+    FOR_GROUPS(c, BN, g) {
+      const int j = c.n0 + g;
+      float ub[32], h1[32], h3[32];
+      acc1(c, g, ub);
+      ld32(hrow + j, h1);
+      ld32(hrow + d.d_h + j, h3);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const Act f(h1[i]);
+        const float a1 = ub[i] * h3[i] * f.d1;
+        h3[i] = ub[i] * f.s;
+        h1[i] = a1;
+      }
+      st32(hbrow + j, h1);
+      st32(hbrow + d.d_h + j, h3);
+    }
+  }
+};
+// dk part 1: -(a dH D_M13 + b dH D_W13) (fp32).
+struct EpiDk1 {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    const size_t tok = (size_t)c.z * d.T + p.t0 + t;
+    const float a = p.ca[tok], b = p.cb[tok];
+    float* o = p.dkp + ((size_t)c.z * d.C + t) * d.d_k;
+    FOR_GROUPS(c, BN, g) {
+      float m[32], w[32];
+      acc2(c, g, m, w);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
+      st32f(o + c.n0 + g, m);
+    }
+  }
+};
+// dk part 2 (adds part 1) and dq: [h1b | h3b] [W1; W3] -> act output.
+template <bool KEYS>
+struct EpiDkq {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int t = c.m0 + c.row;
+    bf16* o = (KEYS ? p.dk : p.dq) + ((size_t)c.z * d.T + p.t0 + t) * d.d_k;
+    FOR_GROUPS(c, BN, g) {
+      const int col = c.n0 + g;
+      float x[32];
+      acc1(c, g, x);
+      if (KEYS) {
+        float y[32];
+        ld32f(p.dkp + ((size_t)c.z * d.C + t) * d.d_k + col, y);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] += y[i];
+      }
+      st32(o + col, x);
+    }
+  }
+};
+// dW: D_W <- L(1,n) D_W + acc, class 0 = rows of [W1; W3], class 1 = rows of W2.
+struct EpiDW {
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int i = c.m0 + c.row;
+    const size_t plane = (size_t)d.BH * d.NC;
+    const float PL = p.scal[plane + (size_t)c.z * d.NC + p.ci];
+    const int ld = c.cls == 0 ? d.d_k : d.d_h;
+    const long long base = c.cls == 0 ? 0 : 2LL * d.d_h * d.d_k;
+    float* row = p.DW + (size_t)c.z * d.S + base + (long long)i * ld;
+    FOR_GROUPS(c, BN, g) {
+      float x[32], y[32];
+      acc1(c, g, x);
+      ld32f(row + c.n0 + g, y);
+#pragma unroll
+      for (int q = 0; q < 32; ++q) y[q] = PL * y[q] + x[q];
+      st32f(row + c.n0 + g, y);
+    }
+  }
+};
+
+template <class Epi> struct Name { static constexpr const char* v = "tc_bwd"; };
+template <> struct Name<EpiR1> { static constexpr const char* v = "tcb_r1_h"; };
+template <> struct Name<EpiR2> { static constexpr const char* v = "tcb_r2_e"; };
+template <> struct Name<EpiR3> { static constexpr const char* v = "tcb_r3_du"; };
+template <> struct Name<EpiD1> { static constexpr const char* v = "tcb_d1_dir13"; };
+template <> struct Name<EpiD2> { static constexpr const char* v = "tcb_d2_dir2"; };
+template <> struct Name<EpiE3> { static constexpr const char* v = "tcb_e3_ub_dub"; };
+template <> struct Name<EpiE4> { static constexpr const char* v = "tcb_e4_eb"; };
+template <> struct Name<EpiE5> { static constexpr const char* v = "tcb_e5_hb"; };
+template <> struct Name<EpiQ1> { static constexpr const char* v = "tcb_q1_hbq"; };
+template <> struct Name<EpiDk1> { static constexpr const char* v = "tcb_dk1"; };
+template <> struct Name<EpiDkq<true>> { static constexpr const char* v = "tcb_dk2"; };
+template <> struct Name<EpiDkq<false>> { static constexpr const char* v = "tcb_dq"; };
+template <> struct Name<EpiDW> { static constexpr const char* v = "tcb_dw"; };
+
+// ---------------------------------------------------------------- elementwise kernels
+// bf16 copies of the chunk-start weights and of the state adjoints, each split
+// into a [W1; W3] block [BH, 2 d_h, d_k] and a W2 block [BH, d_v, d_h]; plus the
+// partial sums of <D_M, M0>, <D_W, W0>, <D_W, M0> (64 blocks per head).
+__global__ void bwd_shadow_kernel(const float* __restrict__ W0, const float* __restrict__ M0,
+                                  long long sst, const float* __restrict__ DW,
+                                  const float* __restrict__ DM, bf16* W13, bf16* W2, bf16* DW13,
+                                  bf16* DW2, bf16* DM13, bf16* DM2, float* part, Dims d) {
+  const int z = blockIdx.y, blk = blockIdx.x;
+  const long long S = d.S, n13 = 2LL * d.d_h * d.d_k;
+  const float* w0 = W0 + z * sst;
+  const float* m0 = M0 + z * sst;
+  const float* dw = DW + z * S;
+  const float* dm = DM + z * S;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f;
+  for (long long i4 = (long long)blk * blockDim.x + threadIdx.x; i4 < S / 4;
+       i4 += (long long)gridDim.x * blockDim.x) {
+    const long long i = i4 * 4;
+    const float4 w = *reinterpret_cast<const float4*>(w0 + i);
+    const float4 m = *reinterpret_cast<const float4*>(m0 + i);
+    const float4 a = *reinterpret_cast<const float4*>(dw + i);
+    const float4 b = *reinterpret_cast<const float4*>(dm + i);
+    s0 += b.x * m.x + b.y * m.y + b.z * m.z + b.w * m.w;
+    s1 += a.x * w.x + a.y * w.y + a.z * w.z + a.w * w.w;
+    s2 += a.x * m.x + a.y * m.y + a.z * m.z + a.w * m.w;
+    size_t o13, o2;
+    bf16 *pw, *pa, *pb;
+    if (i < n13) {
+      o13 = (size_t)z * n13 + i;
+      pw = W13 + o13; pa = DW13 + o13; pb = DM13 + o13;
+    } else {
+      o2 = (size_t)z * (S - n13) + (i - n13);
+      pw = W2 + o2; pa = DW2 + o2; pb = DM2 + o2;
+    }
+    *reinterpret_cast<uint2*>(pw) = make_uint2(pack2(w.x, w.y), pack2(w.z, w.w));
+    *reinterpret_cast<uint2*>(pa) = make_uint2(pack2(a.x, a.y), pack2(a.z, a.w));
+    *reinterpret_cast<uint2*>(pb) = make_uint2(pack2(b.x, b.y), pack2(b.z, b.w));
+  }
+  __shared__ float red[3][256];
+  red[0][threadIdx.x] = s0;
+  red[1][threadIdx.x] = s1;
+  red[2][threadIdx.x] = s2;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o)
+      for (int q = 0; q < 3; ++q) red[q][threadIdx.x] += red[q][threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0)
+    for (int q = 0; q < 3; ++q) part[((size_t)q * d.BH + z) * 64 + blk] = red[q][0];
+}
+// chunk-scalar adjoints from the partials; dM0 = U D_M + c D_W in place.
+__global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci) {
+  const int z = blockIdx.x * blockDim.x + threadIdx.x;
+  if (z >= d.BH) return;
+  const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
+  for (int q = 0; q < 3; ++q) {
+    float s = 0.f;
+    for (int b = 0; b < 64; ++b) s += part[((size_t)q * d.BH + z) * 64 + b];
+    sbar[q * plane + o] = s;
+  }
+}
+__global__ void bwd_dm_kernel(float* DM, const float* DW, const float* scal, Dims d, int ci) {
+  const long long total4 = (long long)d.BH * d.S / 4;
+  const size_t plane = (size_t)d.BH * d.NC;
+  for (long long e4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e4 < total4;
+       e4 += (long long)gridDim.x * blockDim.x) {
+    const int z = (int)(e4 * 4 / d.S);
+    const size_t o = (size_t)z * d.NC + ci;
+    const float U = scal[o], c = scal[2 * plane + o];
+    float4 m = reinterpret_cast<float4*>(DM)[e4];
+    const float4 w = reinterpret_cast<const float4*>(DW)[e4];
+    m.x = U * m.x + c * w.x; m.y = U * m.y + c * w.y; m.z = U * m.z + c * w.z; m.w = U * m.w + c * w.w;
+    reinterpret_cast<float4*>(DM)[e4] = m;
+  }
+}
+// abar_t, bbar_t = -(sum of the partial dot products), fixed order.
+__global__ void bwd_rows_kernel(const float* part, float* abar, float* bbar, Dims d, int t0, int NG) {
+  const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= (long long)d.BH * d.C) return;
+  const int z = (int)(r / d.C), t = (int)(r % d.C);
+  const float* pa = part + (size_t)r * NG;
+  const float* pb = pa + (size_t)d.BH * d.C * NG;
+  float sa = 0.f, sb = 0.f;
+  for (int g = 0; g < NG; ++g) {
+    sa += pa[g];
+    sb += pb[g];
+  }
+  abar[(size_t)z * d.T + t0 + t] = -sa;
+  bbar[(size_t)z * d.T + t0 + t] = -sb;
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+// 2-D bf16 map over [rows, cols]; box 64 columns x box_rows, 128B swizzle.
+bool mk(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+template <int NUM_ACC, bool A_MN, bool B_MN, class Epi>
+cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
+  constexpr int STAGES = NUM_ACC == 1 ? 6 : 4;
+  constexpr size_t smem = tc2::smem_bytes<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, 0>();
+  auto kern = tc2::gemm_persistent<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, Epi, BwdP, 0>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  job.total_tiles = 0;
+  for (int c = 0; c < job.n_cls; ++c) job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
+  const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
+  E2TTT_TRACE(Name<Epi>::v, st);
+  kern<<<grid, (2 + kEW) * 32, smem, st>>>(job, p);
+  return cudaGetLastError();
+}
+
+struct Buf {
+  int* status;
+  bf16 *X, *Y3, *Z3, *Hc, *DH, *HB, *W13, *W2, *DW13, *DW2, *DM13, *DM2;
+  float *a, *b, *scal, *abar, *bbar, *sbar, *spart, *du, *DB, *G2U, *UBd, *dkp, *part;
+  size_t total;
+};
+Buf carve(const Dims& d, char* base) {
+  Buf B{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = (off + bytes + 255) & ~size_t(255);
+    return p;
+  };
+  const size_t BH = d.BH, C = d.C, dk = d.d_k, dv = d.d_v, dh = d.d_h, h = 2, f = 4;
+  const int NG = (int)(2 * dh / 32 + dv / 32);
+  B.status = (int*)take(256);  // first bytes of the workspace (read by e2ttt_workspace_status)
+  B.a = (float*)take(BH * d.T * f);
+  B.b = (float*)take(BH * d.T * f);
+  B.scal = (float*)take(3 * BH * d.NC * f);
+  B.abar = (float*)take(BH * d.T * f);
+  B.bbar = (float*)take(BH * d.T * f);
+  B.sbar = (float*)take(3 * BH * d.NC * f);
+  B.spart = (float*)take(3 * BH * 64 * f);
+  B.X = (bf16*)take(BH * 2 * C * dk * h);
+  B.Y3 = (bf16*)take(BH * 3 * C * dh * h);
+  B.Z3 = (bf16*)take(BH * 3 * C * dv * h);
+  B.Hc = (bf16*)take(BH * 2 * C * 2 * dh * h);
+  B.DH = (bf16*)take(BH * C * 2 * dh * h);
+  B.HB = (bf16*)take(BH * 2 * C * 2 * dh * h);
+  B.W13 = (bf16*)take(BH * 2 * dh * dk * h);
+  B.W2 = (bf16*)take(BH * dv * dh * h);
+  B.DW13 = (bf16*)take(BH * 2 * dh * dk * h);
+  B.DW2 = (bf16*)take(BH * dv * dh * h);
+  B.DM13 = (bf16*)take(BH * 2 * dh * dk * h);
+  B.DM2 = (bf16*)take(BH * dv * dh * h);
+  B.du = (float*)take(BH * C * dh * f);
+  B.DB = (float*)take(BH * C * 2 * dh * f);
+  B.G2U = (float*)take(BH * C * dv * f);
+  B.UBd = (float*)take(BH * C * dh * f);
+  B.dkp = (float*)take(BH * C * dk * f);
+  B.part = (float*)take(2 * BH * C * NG * f);
+  B.total = off;
+  return B;
+}
+
+tc2::Class cls(int tm, int tn, int kb, tc2::Opnd a, tc2::Opnd b, int mode = 0) {
+  return tc2::Class{tm, tn, kb, a, b, mode};
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const Dims& d, bool bf16_act) {
+  return d.kind == 1 && tc_fwd_supported(d, bf16_act);
+}
+size_t tc_bwd_workspace_bytes(const Dims& d) { return carve(d, nullptr).total; }
+
+cudaError_t tc_bwd(const BwdArgs& A) {
+  const Dims& d = A.d;
+  const int BH = d.BH, T = d.T, C = d.C, NC = d.NC, dk = d.d_k, dv = d.d_v, dh = d.d_h;
+  Buf B = carve(d, (char*)A.ws);
+  cudaStream_t st = A.st;
+  const size_t sbytes = (size_t)BH * d.S * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(B.status, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  e = launch_chunk_coeffs(A.lr, A.mom, A.decay, B.a, B.b, B.scal, BH, T, C, NC, st);
+  if (e != cudaSuccess) return e;
+  e = A.dW_end ? cudaMemcpyAsync(A.dW0, A.dW_end, sbytes, cudaMemcpyDeviceToDevice, st)
+               : cudaMemsetAsync(A.dW0, 0, sbytes, st);
+  if (e == cudaSuccess)
+    e = A.dM_end ? cudaMemcpyAsync(A.dM0, A.dM_end, sbytes, cudaMemcpyDeviceToDevice, st)
+                 : cudaMemsetAsync(A.dM0, 0, sbytes, st);
+  if (e != cudaSuccess) return e;
+
+  BwdP p{};
+  p.d = d;
+  p.v = (const bf16*)A.v;
+  p.dq = (bf16*)A.dq; p.dk = (bf16*)A.dk; p.dv = (bf16*)A.dv;
+  p.ca = B.a; p.cb = B.b; p.scal = B.scal;
+  p.DW = A.dW0; p.DM = A.dM0;
+  p.X = B.X; p.Y3 = B.Y3; p.Z3 = B.Z3; p.Hc = B.Hc; p.DH = B.DH; p.HB = B.HB;
+  p.du = B.du; p.DB = B.DB; p.G2U = B.G2U; p.UBd = B.UBd; p.dkp = B.dkp; p.part = B.part;
+  p.NG = (int)(2 * dh / 32 + dv / 32);
+  p.status = B.status;
+
+  // operand maps (per call; the chunk only changes the copies and the epilogue data)
+  tc2::Job r1{}, r2{}, r3{}, d1{}, d2{}, e3{}, e4{}, e5{}, q1{}, k1{}, k2{}, dq{}, dw{};
+  bool ok = true;
+  const uint64_t rX = (uint64_t)BH * 2 * C, rY = (uint64_t)BH * 3 * C, rZ = rY;
+  const uint64_t rH = (uint64_t)BH * 2 * C, rD = (uint64_t)BH * C;
+  const uint64_t r13 = (uint64_t)BH * 2 * dh, r2w = (uint64_t)BH * dv;
+  for (tc2::Job* j : {&r1, &r2, &r3, &d1, &d2, &e3, &e4, &e5, &q1, &k1, &k2, &dq, &dw}) {
+    j->heads = BH;
+    j->n_cls = 1;
+    j->status = B.status;
+  }
+  // R1: X [2C x dk] x {W1, W3}^T (two B operands)
+  ok &= mk(&r1.maps[0].op0, B.X, rX, dk, 128);
+  ok &= mk(&r1.maps[0].op1, B.W13, r13, dk, 128);
+  ok &= mk(&r1.maps[0].op2, B.W13 + (size_t)dh * dk, r13 - dh, dk, 128);
+  r1.cls[0] = cls(2 * C / 128, dh / 128, dk / 64, {2 * C, 0, 0}, {2 * dh, 0, 0}, tc2::kModeA1B2);
+  // R2: U_k (rows [C, 2C) of Y3) x W2^T
+  ok &= mk(&r2.maps[0].op0, B.Y3, rY, dh, 128);
+  ok &= mk(&r2.maps[0].op2, B.W2, r2w, dh, 128);
+  r2.cls[0] = cls(C / 128, dv / 128, dh / 64, {3 * C, C, 0}, {dv, 0, 0});
+  // R3: E (rows [0, C) of Z3) x W2 (MN-major)
+  ok &= mk(&r3.maps[0].op0, B.Z3, rZ, dv, 128);
+  ok &= mk(&r3.maps[0].op2, B.W2, r2w, dh, 64);
+  r3.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, 0, 0}, {dv, 0, 0});
+  // D1: keys (rows [0, C) of X) x {D_M13, D_W13}^T
+  ok &= mk(&d1.maps[0].op0, B.X, rX, dk, 128);
+  ok &= mk(&d1.maps[0].op1, B.DM13, r13, dk, 128);
+  ok &= mk(&d1.maps[0].op2, B.DW13, r13, dk, 128);
+  d1.cls[0] = cls(C / 128, 2 * dh / 128, dk / 64, {2 * C, 0, 0}, {2 * dh, 0, 0}, tc2::kModeA1B2);
+  // D2: U_k x {D_M2, D_W2}^T
+  ok &= mk(&d2.maps[0].op0, B.Y3, rY, dh, 128);
+  ok &= mk(&d2.maps[0].op1, B.DM2, r2w, dh, 128);
+  ok &= mk(&d2.maps[0].op2, B.DW2, r2w, dh, 128);
+  d2.cls[0] = cls(C / 128, dv / 128, dh / 64, {3 * C, C, 0}, {dv, 0, 0}, tc2::kModeA1B2);
+  // E3: E x {D_M2, D_W2} (MN-major)
+  ok &= mk(&e3.maps[0].op0, B.Z3, rZ, dv, 128);
+  ok &= mk(&e3.maps[0].op1, B.DM2, r2w, dh, 64);
+  ok &= mk(&e3.maps[0].op2, B.DW2, r2w, dh, 64);
+  e3.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, 0, 0}, {dv, 0, 0}, tc2::kModeA1B2);
+  // E4: dub (rows [0, C) of Y3) x W2^T
+  ok &= mk(&e4.maps[0].op0, B.Y3, rY, dh, 128);
+  ok &= mk(&e4.maps[0].op2, B.W2, r2w, dh, 128);
+  e4.cls[0] = cls(C / 128, dv / 128, dh / 64, {3 * C, 0, 0}, {dv, 0, 0});
+  // E5: EB (rows [C, 2C) of Z3) x W2 (MN-major);  Q1: dout (rows [2C, 3C)) x W2
+  ok &= mk(&e5.maps[0].op0, B.Z3, rZ, dv, 128);
+  ok &= mk(&e5.maps[0].op2, B.W2, r2w, dh, 64);
+  e5.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, C, 0}, {dv, 0, 0});
+  q1.maps[0] = e5.maps[0];
+  q1.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, 2 * C, 0}, {dv, 0, 0});
+  // dk1: dH x {D_M13, D_W13} (MN-major: N = d_k, K = 2 d_h)
+  ok &= mk(&k1.maps[0].op0, B.DH, rD, 2 * dh, 128);
+  ok &= mk(&k1.maps[0].op1, B.DM13, r13, dk, 64);
+  ok &= mk(&k1.maps[0].op2, B.DW13, r13, dk, 64);
+  k1.cls[0] = cls(C / 128, dk / 128, 2 * dh / 64, {C, 0, 0}, {2 * dh, 0, 0}, tc2::kModeA1B2);
+  // dk2 / dq: [h1b | h3b] (rows [0, C) / [C, 2C) of HB) x [W1; W3] (MN-major)
+  ok &= mk(&k2.maps[0].op0, B.HB, rH, 2 * dh, 128);
+  ok &= mk(&k2.maps[0].op2, B.W13, r13, dk, 64);
+  k2.cls[0] = cls(C / 128, dk / 128, 2 * dh / 64, {2 * C, 0, 0}, {2 * dh, 0, 0});
+  dq.maps[0] = k2.maps[0];
+  dq.cls[0] = cls(C / 128, dk / 128, 2 * dh / 64, {2 * C, C, 0}, {2 * dh, 0, 0});
+  // dW: class 0 = [h1b | h3b]^T [K; Q] (2C tokens), class 1 = [E; EB; dout]^T [dub; u_k; u_q]
+  ok &= mk(&dw.maps[0].op0, B.HB, rH, 2 * dh, 64);
+  ok &= mk(&dw.maps[0].op2, B.X, rX, dk, 64);
+  ok &= mk(&dw.maps[1].op0, B.Z3, rZ, dv, 64);
+  ok &= mk(&dw.maps[1].op2, B.Y3, rY, dh, 64);
+  dw.n_cls = 2;
+  dw.cls[0] = cls(2 * dh / 128, dk / 128, 2 * C / 64, {2 * C, 0, 0}, {2 * C, 0, 0});
+  dw.cls[1] = cls(dv / 128, dh / 128, 3 * C / 64, {3 * C, 0, 0}, {3 * C, 0, 0});
+  if (!ok) return cudaErrorInvalidValue;
+
+  const size_t per_chunk = (size_t)BH * 2 * d.S;
+  const Dims dd = d;
+  for (int ci = NC - 1; ci >= 0; --ci) {
+    const int t0 = ci * C;
+    p.ci = ci;
+    p.t0 = t0;
+    const float* W0 = A.saved + ci * per_chunk;
+    const float* M0 = W0 + d.S;
+    // chunk rows of keys, queries, dout into the stacked operands
+    e = cudaMemcpy2DAsync(B.X, (size_t)2 * C * dk * 2, (const bf16*)A.k + (size_t)t0 * dk,
+                          (size_t)T * dk * 2, (size_t)C * dk * 2, BH, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(B.X + (size_t)C * dk, (size_t)2 * C * dk * 2,
+                            (const bf16*)A.q + (size_t)t0 * dk, (size_t)T * dk * 2, (size_t)C * dk * 2,
+                            BH, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(B.Z3 + (size_t)2 * C * dv, (size_t)3 * C * dv * 2,
+                            (const bf16*)A.dout + (size_t)t0 * dv, (size_t)T * dv * 2,
+                            (size_t)C * dv * 2, BH, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return e;
+    {
+      E2TTT_TRACE("tcb_shadow", st);
+      bwd_shadow_kernel<<<dim3(64, BH), 256, 0, st>>>(W0, M0, 2 * d.S, A.dW0, A.dM0, B.W13, B.W2,
+                                                       B.DW13, B.DW2, B.DM13, B.DM2, B.spart, dd);
+      bwd_scalars_kernel<<<(BH + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci);
+      bwd_dm_kernel<<<4 * num_sms(), 256, 0, st>>>(A.dM0, A.dW0, B.scal, dd, ci);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    using tc2::kModeA1B2;
+    if ((e = run_gemm<2, false, false, EpiR1>(r1, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, false, EpiR2>(r2, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, true, EpiR3>(r3, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<2, false, false, EpiD1>(d1, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<2, false, false, EpiD2>(d2, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<2, false, true, EpiE3>(e3, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, false, EpiE4>(e4, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, true, EpiE5>(e5, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, true, EpiQ1>(q1, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<2, false, true, EpiDk1>(k1, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, true, EpiDkq<true>>(k2, p, st)) != cudaSuccess) return e;
+    if ((e = run_gemm<1, false, true, EpiDkq<false>>(dq, p, st)) != cudaSuccess) return e;
+    {
+      E2TTT_TRACE("tcb_rows", st);
+      const long long rows = (long long)BH * C;
+      bwd_rows_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(B.part, B.abar, B.bbar, dd, t0, p.NG);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    if ((e = run_gemm<1, true, true, EpiDW>(dw, p, st)) != cudaSuccess) return e;
+  }
+  return launch_chunk_coeffs_bwd(A.lr, A.mom, A.decay, B.abar, B.bbar, B.sbar, A.dlr, A.dmom,
+                                 A.ddecay, BH, T, C, NC, st);
+}
+
+}  // namespace e2ttt

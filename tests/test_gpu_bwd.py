@@ -109,3 +109,27 @@ def test_bwd_training_workload(E, variant):
     heads = [(0, 0), (3, 7)]
     gpu, ref = run_bwd(E, w, x, None, None, heads=heads)
     check(gpu, ref, 2e-2, heads=heads, label=f"train_1p3b_2k {variant}")
+
+
+def test_bwd_tensor_core_and_cuda_core_agree(E):
+    """One bf16 problem through both backward paths: a 2-byte offset view of dout
+    makes the pointers unaligned for TMA, which routes the call to the CUDA-core
+    backward."""
+    import torch
+    w = gen.Workload("agreeb", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform", 0.999,
+                     seed=46, lr_lo=0.002, lr_hi=0.02)
+    x = gen.generate(w, m0_scale=0.5)
+    d = device_inputs(w, x)
+    _, _, _, saved = run_fwd(E, w, d, save=True)
+    dW, dM = (dev(a) for a in gen.upstream_state_grads(w, seed=9, scale=0.1))
+    args = (d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], saved)
+    kw = dict(C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss)
+    g_tc = E.chunk_scan_bwd(*args, d["dout"], dW, dM, **kw)
+    buf = torch.empty(d["dout"].numel() + 1, dtype=torch.bfloat16, device="cuda")
+    dout_u = buf[1:].view_as(d["dout"])
+    dout_u.copy_(d["dout"])
+    g_cc = E.chunk_scan_bwd(*args, dout_u, dW, dM, **kw)
+    torch.cuda.synchronize()
+    errs = {n: err(host(g_tc[n]), host(g_cc[n])) for n in NAMES}
+    print("\ntensor-core vs CUDA-core backward:", " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
+    assert all(e < 2e-2 for e in errs.values()), errs
