@@ -41,8 +41,11 @@ import e2ttt_inputs as gen  # noqa: E402
 
 METRIC = "E2-TTT layer tokens/sec (fwd, fwd+bwd) at T=2K/16K; % of bf16 TC roofline"
 UNIT = "tokens/s"
-KERNEL_SOURCES = ["test_weight_layers_chunk_b200/csrc/tc_gemm.cuh",
-                  "test_weight_layers_chunk_b200/csrc/tc_fwd.cu"]
+_CSRC = "test_weight_layers_chunk_b200/csrc/"
+# the sources a kernel's recorded ncu traffic depends on, by kernel-name prefix
+KERNEL_SOURCES = {"tcb_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_bwd.cu"],
+                  "tc_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_fwd.cu"],
+                  "": [_CSRC + "scan.cu", _CSRC + "simt.cuh", _CSRC + "simt_fwd.cu", _CSRC + "bwd.cu"]}
 
 
 # ----------------------------------------------------------------- algorithmic work
@@ -63,6 +66,56 @@ def phase_flops_per_token_head(w) -> dict:
 BWD_SIMT_FLOPS = {"bwd_dk": 12, "bwd_dw2": 6, "bwd_dir_w13": 8, "bwd_h": 8, "bwd_dw13": 8,
                   "bwd_dir_w2": 4, "bwd_residual": 2, "bwd_ub_dir": 4, "bwd_dq": 4, "bwd_eb": 2,
                   "bwd_q_rows": 2, "bwd_da": 2, "bwd_ub_eb": 2}
+
+
+# Backward GEMM phases of the tensor-core path, FLOPs per token and head in units
+# of d d_h (SwiGLU, d_k = d_v = d): 52 for the adjoint plus 12 for recomputing
+# H, E and du at the chunk-start weights (r1, r2, r3).
+TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_du": 2, "tcb_d1_dir13": 8,
+                "tcb_d2_dir2": 4, "tcb_e3_ub_dub": 4, "tcb_e4_eb": 2, "tcb_e5_hb": 2,
+                "tcb_q1_hbq": 2, "tcb_dk1": 8, "tcb_dk2": 4, "tcb_dq": 4, "tcb_dw": 14}
+
+
+def kernel_work(w, has_m0: bool) -> dict:
+    """Algorithmic work of one launch of each kernel: (FLOPs, bytes). One launch
+    covers one chunk of every head (the prep kernels: the whole step). Bytes count
+    every operand read once from HBM and every result written once; the fp32
+    state traffic of the aggregation is averaged over the chunks of a step (the
+    first chunk reads M0 only if one is given, the last writes no bf16 copy)."""
+    BH, C, T, NC = w.B * w.H, w.C, w.T, w.T // w.C
+    dk, dv, dh = w.d_k, w.d_v, w.d_h
+    out = {"k1_chunk_coeffs": (0.0, 20.0 * BH * T), "k1_chunk_coeffs_bwd": (0.0, 32.0 * BH * T)}
+    if w.kind != gen.SWIGLU:
+        return out
+    S13, S2 = 2 * dh * dk, dv * dh
+    S = S13 + S2
+    N, Mk, Mv = C * dh, C * dk, C * dv
+    st_read = (4 + 4 * has_m0) + 8 * (NC - 1)       # per state element, summed over chunks
+    st_write = 8 * NC + 2 * (NC - 1)
+    fl = phase_flops_per_token_head(w)
+    per_head = {
+        "tc_g1_h_act": (fl["tc_g1_h_act"] * C, 2 * (2 * Mk + S13 + 2 * N + 2 * N)),
+        "tc_g2_y_out_e": (fl["tc_g2_y_out_e"] * 2 * C, 2 * (2 * N + S2 + Mv + 4 * Mv)),
+        "tc_g3_da_dh": (fl["tc_g3_da_dh"] * C, 2 * (Mv + S2 + 2 * N + 2 * N)),
+        "tc_g4_aggregate_state": (fl["tc_g4_aggregate_state"] * C,
+                                  2 * (2 * N + 2 * Mk + 2 * Mv + N) + S * (st_read + st_write) / NC),
+    }
+    if dk == dv:
+        dd = dk * dh
+        b = {"tcb_r1_h": 4 * Mk + 2 * S13 + 12 * N, "tcb_r2_e": 2 * N + 2 * S2 + 4 * Mv,
+             "tcb_r3_du": 2 * Mv + 2 * S2 + 12 * N, "tcb_d1_dir13": 2 * Mk + 4 * S13 + 12 * N,
+             "tcb_d2_dir2": 2 * N + 4 * S2 + 6 * Mv, "tcb_e3_ub_dub": 2 * Mv + 4 * S2 + 18 * N,
+             "tcb_e4_eb": 2 * N + 2 * S2 + 8 * Mv, "tcb_e5_hb": 2 * Mv + 2 * S2 + 24 * N,
+             "tcb_q1_hbq": 2 * Mv + 2 * S2 + 8 * N, "tcb_dk1": 4 * N + 4 * S13 + 4 * Mk,
+             "tcb_dk2": 4 * N + 2 * S13 + 6 * Mk, "tcb_dq": 4 * N + 2 * S13 + 2 * Mk,
+             "tcb_dw": 14 * N + 4 * Mk + 6 * Mv + 8 * S}
+        for n, by in b.items():
+            per_head[n] = (TC_BWD_FLOPS[n] * dd * C, by)
+        per_head["tcb_shadow"] = (0.0, 26 * S)
+    out.update({n: (f * BH, by * BH) for n, (f, by) in per_head.items()})
+    out["tc_shadow_init"] = (0.0, 6.0 * S * BH)
+    out["tc_scale_keys"] = (0.0, 6.0 * T * dk * BH)
+    return out
 
 
 def fwd_flops(w) -> float:
@@ -117,9 +170,10 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(kernel: str) -> str:
+    prefix = next(p for p in KERNEL_SOURCES if kernel.startswith(p))
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[prefix]:
         h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()[:16]
 
@@ -133,7 +187,7 @@ def recorded_traffic(kernel: str, workload: str):
     txt = open(p).read()
     sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
     tb = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    if not sha or not tb or sha.group(1) != kernel_source_sha():
+    if not sha or not tb or sha.group(1) != kernel_source_sha(kernel):
         return None
     return float(tb.group(1))
 
@@ -368,51 +422,79 @@ def run_ours(args, w):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    E.e2ttt_trace_enable(True)
     with ClockSampler(local) as clk:
         ev0.record(stream)
         for _ in range(args.steps):
             step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
-    trace = E.e2ttt_trace_summary()
-    E.e2ttt_trace_enable(False)
     if world > 1:
         torch.distributed.barrier()
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    # Per-kernel durations: a second timed pass of the same step with a CUDA event
+    # pair around every launch on the launching stream (kept out of the first pass,
+    # whose step time the events would inflate).
+    tsteps = max(1, min(args.steps, 50))
+    E.e2ttt_trace_enable(True)
+    ev0.record(stream)
+    for _ in range(tsteps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    trace = E.e2ttt_trace_summary()
+    E.e2ttt_trace_enable(False)
+    ms = ev0.elapsed_time(ev1)   # the traced pass: denominators of the kernel shares
     E.e2ttt_workspace_status(ws, stream=stream)
-    ms = ev0.elapsed_time(ev1)
-    ms_max = max_over_ranks(ms, world, dev)
     tokens = w.B * w.T * args.steps * world
     value = tokens / (ms_max / 1e3)
 
     # roofline of the dominant kernel
     peaks = measured_peaks()
     clocks = clk.summary()
-    ph = phase_flops_per_token_head(w)
     kern = trace["kernels"]
-    known = {n: ("tensor", f) for n, f in ph.items()}
+    work = kernel_work(w, M0 is not None)
     if w.kind == gen.SWIGLU and w.d_k == w.d_v:
-        known.update({n: ("alu", f) for n, f in BWD_SIMT_FLOPS.items()})
-    dom = max((n for n in kern if n in known), key=lambda n: kern[n]["total_ms"])
-    bound, per_th = known[dom]
+        dd = w.d_k * w.d_h * w.B * w.H * w.C
+        for n, f in BWD_SIMT_FLOPS.items():
+            work[n] = ("alu", f * dd)
+    dom = max((n for n in kern if n in work), key=lambda n: kern[n]["total_ms"])
     avg_ms = kern[dom]["total_ms"] / kern[dom]["launches"]
-    flops_launch = per_th * w.d_k * w.d_h * w.B * w.H * w.C if bound == "alu" else \
-        ph[dom] * w.B * w.H * w.C  # one launch = one chunk of every head
-    achieved = flops_launch / (avg_ms / 1e3) / 1e12
-    if bound == "tensor":
-        peak, psrc = peaks["bf16_tflops"], peaks["source"] + " (burst bf16 GEMM)"
-    else:
+    if isinstance(work[dom][0], str):      # CUDA-core backward kernel: fp32 FMA bound
+        bound, flops_launch = work[dom]
+        achieved = flops_launch / (avg_ms / 1e3) / 1e12
         peak = fp32_fma_peak_tflops(clocks.get("sm_max_mhz") or 1965.0)
-        psrc = "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"
+        psrc, unit, alg = "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock", "TFLOP/s", flops_launch
+    else:
+        flops_launch, bytes_launch = work[dom]
+        t_tensor = flops_launch / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = bytes_launch / (peaks["hbm_gbs"] * 1e9)
+        if t_tensor >= t_hbm:
+            bound, alg, unit = "tensor", flops_launch, "TFLOP/s"
+            achieved = flops_launch / (avg_ms / 1e3) / 1e12
+            peak, psrc = peaks["bf16_tflops"], peaks["source"] + " (burst bf16 GEMM)"
+        else:
+            bound, alg, unit = "hbm", bytes_launch, "GB/s"
+            achieved = bytes_launch / (avg_ms / 1e3) / 1e9
+            peak, psrc = peaks["hbm_gbs"], peaks["source"] + " (copy bandwidth)"
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": psrc,
+                "unit": unit, "frac": achieved / peak, "peak_source": psrc,
+                "algorithmic_per_launch": alg, "avg_launch_us": avg_ms * 1e3,
                 "traffic": recorded_traffic(dom, w.name),
                 "share_of_step": kern[dom]["total_ms"] / ms}
     step_flops = train_flops(w) if train else fwd_flops(w)
-    whole = {"achieved_tflops": step_flops / (ms / args.steps / 1e3) / 1e12}
+    whole = {"achieved_tflops": step_flops / (ms_max / args.steps / 1e3) / 1e12,
+             "traced_ms_per_step": ms / tsteps, "traced_steps": tsteps}
     whole["frac"] = whole["achieved_tflops"] / peaks["bf16_tflops"]
-    kernels = {n: {"launches": kv["launches"], "avg_us": 1e3 * kv["total_ms"] / kv["launches"],
-                   "share": kv["total_ms"] / ms} for n, kv in kern.items()}
+    kernels = {}
+    for n, kv in kern.items():
+        avg_s = kv["total_ms"] / kv["launches"] / 1e3
+        kernels[n] = {"launches": kv["launches"], "avg_us": avg_s * 1e6, "share": kv["total_ms"] / ms}
+        if n in work and not isinstance(work[n][0], str):
+            f, by = work[n]
+            kernels[n]["tflops"] = f / avg_s / 1e12
+            kernels[n]["gbs"] = by / avg_s / 1e9
+            kernels[n]["frac"] = max(f / avg_s / 1e12 / peaks["bf16_tflops"],
+                                     by / avg_s / 1e9 / peaks["hbm_gbs"])
 
     extras = {}
     if args.extras and rank == 0 and world == 1 and not train:
@@ -461,7 +543,7 @@ def run_ours(args, w):
                 "data": "synthetic (seeded numpy; shapes and distributions of the workload)",
                 "config": config_dict(w, argparse.Namespace(gpus=world, mode=args.mode)),
                 "roofline": roofline, "step_roofline": whole, "kernels": kernels,
-                "gpu_launches": trace["launches"], "clocks": clocks,
+                "gpu_launches": trace["launches"] // tsteps * args.steps, "clocks": clocks,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "extra": extras}
         print(json.dumps(line))
     if world > 1:

@@ -478,41 +478,60 @@ template <> struct Name<EpiDW> { static constexpr const char* v = "tcb_dw"; };
 
 // ---------------------------------------------------------------- elementwise kernels
 // bf16 copies of the chunk-start weights and of the state adjoints, each split
-// into a [W1; W3] block [BH, 2 d_h, d_k] and a W2 block [BH, d_v, d_h]; plus the
-// partial sums of <D_M, M0>, <D_W, W0>, <D_W, M0> (64 blocks per head).
-__global__ void bwd_shadow_kernel(const float* __restrict__ W0, const float* __restrict__ M0,
-                                  long long sst, const float* __restrict__ DW,
-                                  const float* __restrict__ DM, bf16* W13, bf16* W2, bf16* DW13,
-                                  bf16* DW2, bf16* DM13, bf16* DM2, float* part, Dims d) {
+// into a [W1; W3] block [BH, 2 d_h, d_k] and a W2 block [BH, d_v, d_h]; the
+// partial sums of <D_M, M0>, <D_W, W0>, <D_W, M0> (64 blocks per head); and,
+// once the old D_M is read, D_M <- U(1,n) D_M + c D_W in place (the chunk-start
+// adjoint of M; the GEMM phases read only the bf16 copies).
+__device__ __forceinline__ void shadow4(const float4 w, const float4 m, const float4 a, const float4 b,
+                                        long long i, long long n13, long long S, int z, bf16* W13,
+                                        bf16* W2, bf16* DW13, bf16* DW2, bf16* DM13, bf16* DM2,
+                                        float& s0, float& s1, float& s2) {
+  s0 += b.x * m.x + b.y * m.y + b.z * m.z + b.w * m.w;
+  s1 += a.x * w.x + a.y * w.y + a.z * w.z + a.w * w.w;
+  s2 += a.x * m.x + a.y * m.y + a.z * m.z + a.w * m.w;
+  size_t o;
+  bf16 *pw, *pa, *pb;
+  if (i < n13) {
+    o = (size_t)z * n13 + i;
+    pw = W13 + o; pa = DW13 + o; pb = DM13 + o;
+  } else {
+    o = (size_t)z * (S - n13) + (i - n13);
+    pw = W2 + o; pa = DW2 + o; pb = DM2 + o;
+  }
+  *reinterpret_cast<uint2*>(pw) = make_uint2(pack2(w.x, w.y), pack2(w.z, w.w));
+  *reinterpret_cast<uint2*>(pa) = make_uint2(pack2(a.x, a.y), pack2(a.z, a.w));
+  *reinterpret_cast<uint2*>(pb) = make_uint2(pack2(b.x, b.y), pack2(b.z, b.w));
+}
+__global__ void __launch_bounds__(256) bwd_shadow_kernel(
+    const float* __restrict__ W0, const float* __restrict__ M0, long long sst,
+    const float* __restrict__ DW, float* __restrict__ DM, bf16* W13, bf16* W2, bf16* DW13,
+    bf16* DW2, bf16* DM13, bf16* DM2, float* part, const float* __restrict__ scal, Dims d, int ci) {
   const int z = blockIdx.y, blk = blockIdx.x;
   const long long S = d.S, n13 = 2LL * d.d_h * d.d_k;
-  const float* w0 = W0 + z * sst;
-  const float* m0 = M0 + z * sst;
-  const float* dw = DW + z * S;
-  const float* dm = DM + z * S;
+  const size_t plane = (size_t)d.BH * d.NC, so = (size_t)z * d.NC + ci;
+  const float U = scal[so], cc = scal[2 * plane + so];
+  const float4* w0 = reinterpret_cast<const float4*>(W0 + z * sst);
+  const float4* m0 = reinterpret_cast<const float4*>(M0 + z * sst);
+  const float4* dw = reinterpret_cast<const float4*>(DW + z * S);
+  float4* dm = reinterpret_cast<float4*>(DM + z * S);
   float s0 = 0.f, s1 = 0.f, s2 = 0.f;
-  for (long long i4 = (long long)blk * blockDim.x + threadIdx.x; i4 < S / 4;
-       i4 += (long long)gridDim.x * blockDim.x) {
-    const long long i = i4 * 4;
-    const float4 w = *reinterpret_cast<const float4*>(w0 + i);
-    const float4 m = *reinterpret_cast<const float4*>(m0 + i);
-    const float4 a = *reinterpret_cast<const float4*>(dw + i);
-    const float4 b = *reinterpret_cast<const float4*>(dm + i);
-    s0 += b.x * m.x + b.y * m.y + b.z * m.z + b.w * m.w;
-    s1 += a.x * w.x + a.y * w.y + a.z * w.z + a.w * w.w;
-    s2 += a.x * m.x + a.y * m.y + a.z * m.z + a.w * m.w;
-    size_t o13, o2;
-    bf16 *pw, *pa, *pb;
-    if (i < n13) {
-      o13 = (size_t)z * n13 + i;
-      pw = W13 + o13; pa = DW13 + o13; pb = DM13 + o13;
-    } else {
-      o2 = (size_t)z * (S - n13) + (i - n13);
-      pw = W2 + o2; pa = DW2 + o2; pb = DM2 + o2;
-    }
-    *reinterpret_cast<uint2*>(pw) = make_uint2(pack2(w.x, w.y), pack2(w.z, w.w));
-    *reinterpret_cast<uint2*>(pa) = make_uint2(pack2(a.x, a.y), pack2(a.z, a.w));
-    *reinterpret_cast<uint2*>(pb) = make_uint2(pack2(b.x, b.y), pack2(b.z, b.w));
+  const long long n4 = S / 4, step = (long long)gridDim.x * blockDim.x;
+  long long i4 = (long long)blk * blockDim.x + threadIdx.x;
+  // two float4 groups per thread and iteration: eight 16-byte loads in flight
+  for (; i4 + step < n4; i4 += 2 * step) {
+    const long long j4 = i4 + step;
+    const float4 w = w0[i4], m = m0[i4], a = dw[i4], b = dm[i4];
+    const float4 w2 = w0[j4], m2 = m0[j4], a2 = dw[j4], b2 = dm[j4];
+    dm[i4] = make_float4(U * b.x + cc * a.x, U * b.y + cc * a.y, U * b.z + cc * a.z, U * b.w + cc * a.w);
+    dm[j4] = make_float4(U * b2.x + cc * a2.x, U * b2.y + cc * a2.y, U * b2.z + cc * a2.z,
+                         U * b2.w + cc * a2.w);
+    shadow4(w, m, a, b, i4 * 4, n13, S, z, W13, W2, DW13, DW2, DM13, DM2, s0, s1, s2);
+    shadow4(w2, m2, a2, b2, j4 * 4, n13, S, z, W13, W2, DW13, DW2, DM13, DM2, s0, s1, s2);
+  }
+  if (i4 < n4) {
+    const float4 w = w0[i4], m = m0[i4], a = dw[i4], b = dm[i4];
+    dm[i4] = make_float4(U * b.x + cc * a.x, U * b.y + cc * a.y, U * b.z + cc * a.z, U * b.w + cc * a.w);
+    shadow4(w, m, a, b, i4 * 4, n13, S, z, W13, W2, DW13, DW2, DM13, DM2, s0, s1, s2);
   }
   __shared__ float red[3][256];
   red[0][threadIdx.x] = s0;
@@ -527,7 +546,7 @@ __global__ void bwd_shadow_kernel(const float* __restrict__ W0, const float* __r
   if (threadIdx.x == 0)
     for (int q = 0; q < 3; ++q) part[((size_t)q * d.BH + z) * 64 + blk] = red[q][0];
 }
-// chunk-scalar adjoints from the partials; dM0 = U D_M + c D_W in place.
+// chunk-scalar adjoints from the partials.
 __global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci) {
   const int z = blockIdx.x * blockDim.x + threadIdx.x;
   if (z >= d.BH) return;
@@ -536,20 +555,6 @@ __global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* 
     float s = 0.f;
     for (int b = 0; b < 64; ++b) s += part[((size_t)q * d.BH + z) * 64 + b];
     sbar[q * plane + o] = s;
-  }
-}
-__global__ void bwd_dm_kernel(float* DM, const float* DW, const float* scal, Dims d, int ci) {
-  const long long total4 = (long long)d.BH * d.S / 4;
-  const size_t plane = (size_t)d.BH * d.NC;
-  for (long long e4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e4 < total4;
-       e4 += (long long)gridDim.x * blockDim.x) {
-    const int z = (int)(e4 * 4 / d.S);
-    const size_t o = (size_t)z * d.NC + ci;
-    const float U = scal[o], c = scal[2 * plane + o];
-    float4 m = reinterpret_cast<float4*>(DM)[e4];
-    const float4 w = reinterpret_cast<const float4*>(DW)[e4];
-    m.x = U * m.x + c * w.x; m.y = U * m.y + c * w.y; m.z = U * m.z + c * w.z; m.w = U * m.w + c * w.w;
-    reinterpret_cast<float4*>(DM)[e4] = m;
   }
 }
 // abar_t, bbar_t = -(sum of the partial dot products), fixed order.
@@ -795,9 +800,9 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     {
       E2TTT_TRACE("tcb_shadow", st);
       bwd_shadow_kernel<<<dim3(64, BH), 256, 0, st>>>(W0, M0, 2 * d.S, A.dW0, A.dM0, B.W13, B.W2,
-                                                       B.DW13, B.DW2, B.DM13, B.DM2, B.spart, dd);
+                                                       B.DW13, B.DW2, B.DM13, B.DM2, B.spart,
+                                                       B.scal, dd, ci);
       bwd_scalars_kernel<<<(BH + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci);
-      bwd_dm_kernel<<<4 * num_sms(), 256, 0, st>>>(A.dM0, A.dW0, B.scal, dd, ci);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }

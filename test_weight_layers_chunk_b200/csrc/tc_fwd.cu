@@ -424,27 +424,38 @@ template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_l
 
 // ---------------------------------------------------------------- prep kernel
 // bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
-__global__ void shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
+__global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
+  // One warp per state row: rows [0, 2 d_h) of a head are W1 then W3 (d_k wide),
+  // rows [2 d_h, 2 d_h + d_v) are W2 (d_h wide); the linear state is d_v rows of d_k.
   const Dims& d = p.d;
-  const long long total4 = (long long)d.BH * d.S / 4;
-  const long long n13 = d.kind == 1 ? 2LL * d.d_h * d.d_k : 0;
-  for (long long e4 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e4 < total4;
-       e4 += (long long)gridDim.x * blockDim.x) {
-    const long long e = e4 * 4;
-    const int z = (int)(e / d.S);
-    const long long idx = e - (long long)z * d.S;
-    const float4 f = reinterpret_cast<const float4*>(W0)[e4];
-    const uint2 packed = make_uint2(pack2(f.x, f.y), pack2(f.z, f.w));
+  const int lane = threadIdx.x & 31;
+  const int r13 = d.kind == 1 ? 2 * d.d_h : d.d_v;
+  const int rows = d.kind == 1 ? r13 + d.d_v : r13;
+  const long long total = (long long)d.BH * rows;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
+  for (long long gr = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); gr < total;
+       gr += nwarps) {
+    const int z = (int)(gr / rows), r = (int)(gr - (long long)z * rows);
+    const float* src;
     bf16* dst;
-    if (d.kind == 0) {
-      dst = p.Wsh13 + e;
-    } else if (idx < n13) {
-      const int i = (int)(idx / d.d_k), j = (int)(idx % d.d_k);
-      dst = p.Wsh13 + ((size_t)z * 2 * d.d_h + w13_row(i % d.d_h, i / d.d_h)) * d.d_k + j;
+    int len;
+    if (r < r13) {
+      src = W0 + (size_t)z * d.S + (size_t)r * d.d_k;
+      const int sr = d.kind == 1 ? w13_row(r % d.d_h, r / d.d_h) : r;
+      dst = p.Wsh13 + ((size_t)z * r13 + sr) * d.d_k;
+      len = d.d_k;
     } else {
-      dst = p.W2sh + (size_t)z * d.d_v * d.d_h + (idx - n13);
+      src = W0 + (size_t)z * d.S + (size_t)r13 * d.d_k + (size_t)(r - r13) * d.d_h;
+      dst = p.W2sh + ((size_t)z * d.d_v + (r - r13)) * d.d_h;
+      len = d.d_h;
     }
-    *reinterpret_cast<uint2*>(dst) = packed;
+    // len is a multiple of 128: every lane moves whole 8-float groups
+    for (int c = lane * 8; c < len; c += 256) {
+      const float4 f0 = *reinterpret_cast<const float4*>(src + c);
+      const float4 f1 = *reinterpret_cast<const float4*>(src + c + 4);
+      *reinterpret_cast<uint4*>(dst + c) =
+          make_uint4(pack2(f0.x, f0.y), pack2(f0.z, f0.w), pack2(f1.x, f1.y), pack2(f1.z, f1.w));
+    }
   }
 }
 
@@ -617,7 +628,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   if (e != cudaSuccess) return e;
   {
     E2TTT_TRACE("tc_shadow_init", st);
-    shadow_init_kernel<<<4 * num_sms(), 256, 0, st>>>(p, W0);
+    shadow_init_kernel<<<8 * num_sms(), 256, 0, st>>>(p, W0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
