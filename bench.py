@@ -305,6 +305,21 @@ def config_dict(w, args):
             "l2": "working set larger than L2 (no flush)"}
 
 
+def capture_graph(torch, dev, stream, fn):
+    """One step (every launch of the C-ABI calls) captured as a CUDA graph, for
+    replay without the host-side launch cost. fn(st) must launch on st."""
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        fn(cap)
+    cap.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        fn(cap)
+    torch.cuda.synchronize(dev)
+    return g
+
+
 # ----------------------------------------------------------------- extra lines
 def _timed(torch, stream, fn, steps):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -339,16 +354,21 @@ def measure_extras(E, torch, dev, stream, args):
             g = [torch.empty_like(t) for t in (q, k, v, lr, mom, decay, W0, W0)]
             wsb = E.workspace(shape, True, dev)
 
-        def step():
+        def step(st=stream):
             E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, None, outb, We, Me, saved, ws,
-                                   stream=stream)
+                                   stream=st)
             if train:
                 E.e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved, dout, None, None, *g,
-                                       wsb, stream=stream)
+                                       wsb, stream=st)
 
         for _ in range(3):
             step()
-        ms = _timed(torch, stream, step, steps)
+        graph = capture_graph(torch, dev, stream, step) if args.graph else None
+        run = graph.replay if graph is not None else step
+        for _ in range(3):
+            run()
+        ms = _timed(torch, stream, run, steps)
+        del graph
         flops = train_flops(w) if train else fwd_flops(w)
         out[("fwd_bwd_" if train else "fwd_") + name] = {
             "value": w.B * w.T / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
@@ -405,18 +425,25 @@ def run_ours(args, w):
         dM0g = torch.empty_like(W0)
         wsb = E.workspace(shape, True, dev)
 
-    def step():
+    def step(st=stream):
         E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, M0, out, W_end, M_end, saved, ws,
-                               stream=stream)
+                               stream=st)
         if train:
             E.e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved, dout, None, None,
                                    grads["dq"], grads["dk"], grads["dv"], grads["dlr"],
-                                   grads["dmom"], grads["ddecay"], dW0g, dM0g, wsb, stream=stream)
+                                   grads["dmom"], grads["ddecay"], dW0g, dM0g, wsb, stream=st)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     E.e2ttt_workspace_status(ws, stream=stream)
+    # The timed step replays a CUDA graph of the same C-ABI calls (all kernels,
+    # copies and memsets of one step); --graph 0 times plain stream launches.
+    graph = capture_graph(torch, dev, stream, step) if args.graph else None
+    run_step = graph.replay if graph is not None else step
+    for _ in range(3):
+        run_step()
+    torch.cuda.synchronize(dev)
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -425,12 +452,14 @@ def run_ours(args, w):
     with ClockSampler(local) as clk:
         ev0.record(stream)
         for _ in range(args.steps):
-            step()
+            run_step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     ms_max = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    # the same step with plain stream launches, for reference
+    stream_ms = _timed(torch, stream, step, max(1, min(args.steps, 50))) if graph is not None else None
     # Per-kernel durations: a second timed pass of the same step with a CUDA event
     # pair around every launch on the launching stream (kept out of the first pass,
     # whose step time the events would inflate).
@@ -483,7 +512,9 @@ def run_ours(args, w):
                 "share_of_step": kern[dom]["total_ms"] / ms}
     step_flops = train_flops(w) if train else fwd_flops(w)
     whole = {"achieved_tflops": step_flops / (ms_max / args.steps / 1e3) / 1e12,
-             "traced_ms_per_step": ms / tsteps, "traced_steps": tsteps}
+             "traced_ms_per_step": ms / tsteps, "traced_steps": tsteps,
+             "timed_as": "cuda_graph_replay" if graph is not None else "stream_launches",
+             "stream_launch_ms_per_step": stream_ms}
     whole["frac"] = whole["achieved_tflops"] / peaks["bf16_tflops"]
     kernels = {}
     for n, kv in kern.items():
@@ -546,6 +577,7 @@ def run_ours(args, w):
                 "gpu_launches": trace["launches"] // tsteps * args.steps, "clocks": clocks,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "extra": extras}
         print(json.dumps(line))
+    del graph, run_step  # release the captured graph before the process group
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -565,6 +597,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extras", type=int, default=1, help="also time T=16K fwd and T=2K fwd+bwd")
     ap.add_argument("--extra-steps", type=int, default=20)
+    ap.add_argument("--graph", type=int, default=1,
+                    help="time replays of a CUDA graph of the step (0: plain stream launches)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -14,8 +14,10 @@
 // No prefix sum is ever subtracted from another, so mu = 0 or lam = 0 (log = -inf)
 // gives exact zeros instead of NaN.
 //
-// Layout: one warp per (head, chunk); lane l owns a contiguous segment of
-// ceil(n/32) tokens; segment results are combined with warp shuffles.
+// Layout: one 128-thread block per (head, chunk) for chunks up to 8192 tokens
+// (thread i owns a contiguous segment of ceil(n/128) tokens; segment results are
+// combined with warp shuffles, then across warps), else one warp per (head,
+// chunk) with segments of ceil(n/32) tokens.
 #include "common.cuh"
 #include "trace.h"
 
@@ -127,6 +129,128 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
     scal[o] = expf(ls.su_all);
     scal[plane + o] = expf(ls.sl_all);
     scal[2 * plane + o] = mu[0] * r1;
+  }
+}
+
+// Block version of chunk_coeffs_kernel: one 128-thread block per (head, chunk),
+// thread i owning a contiguous segment of ceil(n/128) tokens. The gates and their
+// logs are staged in shared memory (each log computed once); the segment
+// log-sums and the segment maps of the ratio-sum recurrence are combined with
+// warp shuffles and then across the four warps, suffix-wise and by additions and
+// products only (never by subtracting a prefix), as in the warp version.
+constexpr int kK1Threads = 128;
+constexpr int kK1Warps = kK1Threads / 32;
+constexpr int kK1MaxC = 8192;  // 4 C floats of shared memory
+
+__global__ void __launch_bounds__(kK1Threads)
+chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                          const float* __restrict__ decay, float* __restrict__ a_out,
+                          float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
+                          int NC) {
+  extern __shared__ float k1s[];
+  float* s_eta = k1s;
+  float* s_mu = k1s + C;
+  float* s_lmu = k1s + 2 * C;
+  float* s_llam = k1s + 3 * C;
+  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
+  const int t0 = ci * C;
+  const int n = min(C, T - t0);
+  const size_t base = (size_t)bh * T + t0;
+  for (int t = tid; t < n; t += kK1Threads) {
+    const float mu = mom[base + t];
+    s_eta[t] = lr[base + t];
+    s_mu[t] = mu;
+    s_lmu[t] = logf(mu);
+    s_llam[t] = logf(decay[base + t]);
+  }
+  __syncthreads();
+  const int per = (n + kK1Threads - 1) / kK1Threads;
+  const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
+
+  // suffix log-sums: exclusive (tokens after this segment) and chunk totals
+  float su = 0.f, sl = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    su += s_lmu[t];
+    sl += s_llam[t];
+  }
+  const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
+  if (lane == 0) {
+    w_su[warp] = su_inc;
+    w_sl[warp] = sl_inc;
+  }
+  __syncthreads();
+  float su_later = 0.f, sl_later = 0.f;  // warps after this one
+  for (int w = kK1Warps - 1; w > warp; --w) {
+    su_later += w_su[w];
+    sl_later += w_sl[w];
+  }
+  float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
+  float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
+  if (lane == 31) {
+    su_excl = 0.f;
+    sl_excl = 0.f;
+  }
+  su_excl += su_later;
+  sl_excl += sl_later;
+  float su_all = 0.f, sl_all = 0.f;
+  for (int w = kK1Warps - 1; w >= 0; --w) {
+    su_all += w_su[w];
+    sl_all += w_sl[w];
+  }
+
+  // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map
+  su = su_excl;
+  sl = sl_excl;
+  float Mseg = 1.f, Cseg = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    a_out[base + t] = s_eta[t] * expf(su);
+    const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
+    Cseg = expf(sl) + m * Cseg;
+    Mseg = m * Mseg;
+    su += s_lmu[t];
+    sl += s_llam[t];
+  }
+  // inclusive suffix composition of the maps within the warp, then across warps
+  float M = Mseg, Cc = Cseg;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float Mr = __shfl_down_sync(0xffffffffu, M, off);
+    const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+    if (lane + off < 32) {
+      Cc = Cc + M * Cr;
+      M = M * Mr;
+    }
+  }
+  if (lane == 0) {
+    w_M[warp] = M;
+    w_C[warp] = Cc;
+  }
+  __syncthreads();
+  float r_end = 0.f;  // R at the first token after this warp's segments
+  for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
+  const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
+  const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
+  float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
+
+  // reverse walk 2: R_t and the weight kernel b_t
+  sl = sl_excl;
+  float r1 = 0.f;
+  for (int t = s1 - 1; t >= s0; --t) {
+    const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
+    const float r = expf(sl) + m * r_next;
+    b_out[base + t] = s_eta[t] * r;
+    r_next = r;
+    if (t == 0) r1 = r;
+    sl += s_llam[t];
+  }
+  if (s0 == 0 && s1 > 0) {  // the thread holding token 1
+    const size_t plane = (size_t)BH * NC;
+    const size_t o = (size_t)bh * NC + ci;
+    scal[o] = expf(su_all);
+    scal[plane + o] = expf(sl_all);
+    scal[2 * plane + o] = s_mu[0] * r1;
   }
 }
 
@@ -267,9 +391,20 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
 cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
                                 float* b, float* scal, int BH, int T, int C, int NC,
                                 cudaStream_t st) {
+  E2TTT_TRACE("k1_chunk_coeffs", st);
+  if (C <= kK1MaxC) {
+    const size_t smem = (size_t)4 * C * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(chunk_coeffs_block_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    chunk_coeffs_block_kernel<<<BH * NC, kK1Threads, smem, st>>>(lr, mom, decay, a, b, scal, BH, T,
+                                                                 C, NC);
+    return cudaGetLastError();
+  }
   int warps = BH * NC;
   int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  E2TTT_TRACE("k1_chunk_coeffs", st);
   chunk_coeffs_kernel<<<blocks, kWarpsPerBlock * 32, 0, st>>>(lr, mom, decay, a, b, scal, BH, T,
                                                                C, NC);
   return cudaGetLastError();

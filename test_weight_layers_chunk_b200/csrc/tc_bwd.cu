@@ -609,13 +609,19 @@ int num_sms() {
 }
 template <int NUM_ACC, bool A_MN, bool B_MN, class Epi>
 cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
-  constexpr int STAGES = NUM_ACC == 1 ? 6 : 4;
-  constexpr size_t smem = tc2::smem_bytes<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, 0>();
-  auto kern = tc2::gemm_persistent<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, Epi, BwdP, 0>;
+  // two 64-wide k-blocks per ring slot (one producer/MMA handshake per 128 of K)
+  constexpr int KG = 2;
+  constexpr int STAGES = NUM_ACC == 1 ? 3 : 2;
+  constexpr size_t smem = tc2::smem_bytes<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, 0, KG>();
+  static_assert(smem <= 232448, "shared memory per CTA");
+  auto kern = tc2::gemm_persistent<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, Epi, BwdP, 0, KG>;
+  job.total_tiles = 0;
+  for (int c = 0; c < job.n_cls; ++c) {
+    if (job.cls[c].kblocks % KG != 0) return cudaErrorInvalidValue;
+    job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  job.total_tiles = 0;
-  for (int c = 0; c < job.n_cls; ++c) job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
   const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
   E2TTT_TRACE(Name<Epi>::v, st);
   kern<<<grid, (2 + kEW) * 32, smem, st>>>(job, p);

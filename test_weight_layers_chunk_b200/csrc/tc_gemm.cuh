@@ -68,6 +68,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if ((i & 63) == 0 && globaltimer() - t0 > kWaitNs) return false;
   }
 }
+// Bounded wait for the hot producer / MMA loops: try_wait with a short
+// suspend-time hint (20 ns), so a thread whose phase completes while it is
+// suspended resumes promptly instead of after the default suspend interval.
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20u)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255) == 255 && globaltimer() - t0 > kWaitNs) return false;
+  }
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }

@@ -20,6 +20,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "tc_gemm.cuh"
 
@@ -31,6 +33,7 @@ using tc::BK;
 using tc::smem_u32;
 using tc::mbar_init;
 using tc::mbar_wait;
+using tc::mbar_wait_hint;
 using tc::mbar_try_wait;
 using tc::mbar_expect_tx;
 using tc::fence_mbar_init;
@@ -46,6 +49,7 @@ using tc::mma_commit;
 using tc::tmem_ld32;
 
 enum : int { kErrProducer = 1, kErrMma = 2, kErrEpilogue = 3 };
+constexpr int kEpiBars = 4;  // epilogue-load mbarriers per epilogue warp
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -105,12 +109,27 @@ struct EpiCtx {
   int part, nparts;   // this warp's column share
   uint32_t taddr;     // TMEM address of (this warp's lane quadrant, this tile's accumulator set)
   uint8_t* wsmem;     // this warp's epilogue shared memory (EPI_SMEM bytes, 1024-aligned)
-  uint64_t* wbar;     // two mbarriers owned by this warp (epilogue TMA loads)
-  uint32_t* uses;     // completed-phase counters of wbar[0..1], kept across tiles
+  uint64_t* wbar;     // kEpiBars mbarriers owned by this warp (epilogue TMA loads)
+  uint32_t* uses;     // completed-phase counters of wbar[], kept across tiles
+  int slot;           // this tile's epilogue input buffer / wbar index (tile ordinal & 1)
+  int iter;           // ordinal of this tile among the CTA's tiles
+  // the CTA's next tile (nxt_valid = 0 if this is its last), for epilogues that
+  // start loading the next tile's inputs while finishing this one
+  int nxt_valid, nxt_cls, nxt_z, nxt_m0, nxt_n0;
   __device__ __forceinline__ void ld(int acc, int col, float (&v)[32]) const {
     tmem_ld32(taddr + (uint32_t)(acc * BN + col), v);
   }
 };
+
+// Epilogues that define kPrefetch = true also provide bool prefetch(prm, ctx):
+// TMA loads of the tile's epilogue inputs into input buffer ctx.slot, signalled
+// on ctx.wbar[ctx.slot]; it returns (warp-uniformly) whether it issued any. The
+// core issues them one tile ahead, before it waits for the previous tile's
+// accumulator, so the loads overlap that tile's epilogue.
+template <class E, class = void>
+struct EpiPrefetch : std::false_type {};
+template <class E>
+struct EpiPrefetch<E, std::void_t<decltype(E::kPrefetch)>> : std::bool_constant<E::kPrefetch> {};
 
 template <int BN, int NUM_ACC, bool A_MN, bool B_MN>
 struct Cfg {
@@ -124,12 +143,13 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = 2 * kAccCols <= 128 ? 128 : 2 * kAccCols <= 256 ? 256 : 512;
 };
 
-template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, int EPI_WARPS = 8, int EPI_SMEM = 0>
+template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, int EPI_WARPS = 8, int EPI_SMEM = 0,
+          int KG = 1>
 constexpr size_t smem_bytes() {
   // ring + per-warp epilogue buffers + barriers; at least 116 KB so that one
   // CTA is resident per SM
-  size_t s = 1024 + (size_t)STAGES * Cfg<BN, NUM_ACC, A_MN, B_MN>::kStage +
-             (size_t)EPI_WARPS * EPI_SMEM + 256 + 16 * EPI_WARPS;
+  size_t s = 1024 + (size_t)STAGES * KG * Cfg<BN, NUM_ACC, A_MN, B_MN>::kStage +
+             (size_t)EPI_WARPS * EPI_SMEM + 256 + 8 * kEpiBars * EPI_WARPS;
   return s < 118784 ? 118784 : s;
 }
 
@@ -163,22 +183,25 @@ __device__ __forceinline__ void load_opnd(uint8_t* dst, const CUtensorMap* map, 
 }
 
 template <int BN, int NUM_ACC, bool A_MN, bool B_MN, int STAGES, int EPI_WARPS, class Epi, class P,
-          int EPI_SMEM = 0>
+          int EPI_SMEM = 0, int KG = 1>
 __global__ void __launch_bounds__((2 + EPI_WARPS) * 32, 1)
 gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) {
   using C_ = Cfg<BN, NUM_ACC, A_MN, B_MN>;
   static_assert(EPI_SMEM % 1024 == 0, "epilogue buffers stay 1024-byte aligned");
+  // One ring slot holds KG consecutive 64-wide k-blocks (one full/empty handshake
+  // per KG k-blocks); every class's k-block count is a multiple of KG.
+  constexpr uint32_t kSlot = KG * C_::kStage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint8_t* epi_smem = smem + (size_t)STAGES * C_::kStage;
+  uint8_t* epi_smem = smem + (size_t)STAGES * kSlot;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + (size_t)EPI_WARPS * EPI_SMEM);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
-  uint64_t* epi_bar = acc_empty + 2;     // [2 per epilogue warp]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + 2 * EPI_WARPS);
+  uint64_t* epi_bar = acc_empty + 2;     // [kEpiBars per epilogue warp]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + kEpiBars * EPI_WARPS);
   __shared__ int s_err;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -192,7 +215,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS);
     }
-    for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&epi_bar[w], 1);
+    for (int w = 0; w < kEpiBars * EPI_WARPS; ++w) mbar_init(&epi_bar[w], 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -221,26 +244,29 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       decode_tile(job, t, c, z, mt, nt);
       const Class& K = job.cls[c];
       const Maps& M = job.maps[c];
-      for (int kb = 0; kb < K.kblocks; ++kb, ++it) {
+      for (int kb = 0; kb < K.kblocks; kb += KG, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (it >= STAGES && !mbar_wait(&empty[s], ph ^ 1u)) {
+        if (it >= STAGES && !mbar_wait_hint(&empty[s], ph ^ 1u)) {
           atomicExch(job.status, kErrProducer);
           s_err = 1;
           ok = false;
           break;
         }
-        uint8_t* st = ring + (size_t)s * C_::kStage;
-        mbar_expect_tx(&full[s], C_::kStage);
-        load_opnd<A_MN, BM>(st, &M.op0, &full[s], K.a, z, mt * BM, kb);
-        if (NUM_ACC == 1) {
-          load_opnd<B_MN, BN>(st + C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb);
-        } else if (K.mode == kModeA2B1) {
-          load_opnd<A_MN, BM>(st + C_::kTileA, &M.op1, &full[s], K.a, z, mt * BM, kb);
-          load_opnd<B_MN, BN>(st + 2 * C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb);
-        } else {
-          load_opnd<B_MN, BN>(st + C_::kTileA, &M.op1, &full[s], K.b, z, nt * BN, kb);
-          load_opnd<B_MN, BN>(st + 2 * C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb);
+        mbar_expect_tx(&full[s], kSlot);
+#pragma unroll
+        for (int g = 0; g < KG; ++g) {
+          uint8_t* st = ring + (size_t)s * kSlot + g * C_::kStage;
+          load_opnd<A_MN, BM>(st, &M.op0, &full[s], K.a, z, mt * BM, kb + g);
+          if (NUM_ACC == 1) {
+            load_opnd<B_MN, BN>(st + C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
+          } else if (K.mode == kModeA2B1) {
+            load_opnd<A_MN, BM>(st + C_::kTileA, &M.op1, &full[s], K.a, z, mt * BM, kb + g);
+            load_opnd<B_MN, BN>(st + 2 * C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
+          } else {
+            load_opnd<B_MN, BN>(st + C_::kTileA, &M.op1, &full[s], K.b, z, nt * BN, kb + g);
+            load_opnd<B_MN, BN>(st + 2 * C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
+          }
         }
       }
     }
@@ -250,8 +276,12 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     constexpr uint32_t id = idesc(BM, BN, A_MN, B_MN);
-    constexpr uint32_t kStepA = A_MN ? 2048 : 32;
-    constexpr uint32_t kStepB = B_MN ? 2048 : 32;
+    // descriptors = ring-base descriptor + (byte offset >> 4): the start-address
+    // field is the low 14 bits and every operand lies below 256 KB of smem
+    constexpr uint32_t kStepA = (A_MN ? 2048 : 32) >> 4;
+    constexpr uint32_t kStepB = (B_MN ? 2048 : 32) >> 4;
+    const uint64_t dA0 = sdesc(smem_u32(ring), A_MN);
+    const uint64_t dB0 = sdesc(smem_u32(ring), B_MN);
     int it = 0, i = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < job.total_tiles && ok; t += gridDim.x, ++i) {
@@ -267,30 +297,33 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       }
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t)(b * C_::kAccCols);
-      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+      for (int kb = 0; kb < kblocks; kb += KG, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (!mbar_wait(&full[s], ph)) {
+        if (!mbar_wait_hint(&full[s], ph)) {
           atomicExch(job.status, kErrMma);
           s_err = 1;
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t st = smem_u32(ring + (size_t)s * C_::kStage);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k) {
-          const uint32_t accum = (kb | k) != 0;
-          const uint64_t ad = sdesc(st + k * kStepA, A_MN);
-          if (NUM_ACC == 1) {
-            mma_bf16(acc, ad, sdesc(st + C_::kTileA + k * kStepB, B_MN), id, accum);
-          } else if (!a1b2) {
-            const uint64_t bd = sdesc(st + 2 * C_::kTileA + k * kStepB, B_MN);
-            mma_bf16(acc, ad, bd, id, accum);
-            mma_bf16(acc + BN, sdesc(st + C_::kTileA + k * kStepA, A_MN), bd, id, accum);
-          } else {
-            mma_bf16(acc, ad, sdesc(st + C_::kTileA + k * kStepB, B_MN), id, accum);
-            mma_bf16(acc + BN, ad, sdesc(st + 2 * C_::kTileA + k * kStepB, B_MN), id, accum);
+        for (int g = 0; g < KG; ++g) {
+          const uint32_t so = ((uint32_t)s * kSlot + (uint32_t)g * C_::kStage) >> 4;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t accum = ((kb + g) | k) != 0;
+            const uint64_t ad = dA0 + (so + k * kStepA);
+            if (NUM_ACC == 1) {
+              mma_bf16(acc, ad, dB0 + (so + (C_::kTileA >> 4) + k * kStepB), id, accum);
+            } else if (!a1b2) {
+              const uint64_t bd = dB0 + (so + ((2 * C_::kTileA) >> 4) + k * kStepB);
+              mma_bf16(acc, ad, bd, id, accum);
+              mma_bf16(acc + BN, dA0 + (so + (C_::kTileA >> 4) + k * kStepA), bd, id, accum);
+            } else {
+              mma_bf16(acc, ad, dB0 + (so + (C_::kTileA >> 4) + k * kStepB), id, accum);
+              mma_bf16(acc + BN, ad, dB0 + (so + ((2 * C_::kTileA) >> 4) + k * kStepB), id, accum);
+            }
           }
         }
         mma_commit(&empty[s]);
@@ -302,18 +335,11 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
     // ---------------- epilogue
     const int ew = warp - 2;
     const int quad = warp & 3;
-    uint32_t uses[2] = {0u, 0u};
-    int i = 0;
-    for (int t = blockIdx.x; t < job.total_tiles; t += gridDim.x, ++i) {
+    uint32_t uses[kEpiBars] = {0u, 0u, 0u, 0u};
+    bool pend[2] = {false, false};  // prefetched input buffers not yet consumed
+    auto make_ctx = [&](int t, int i) {
       int c, z, mt, nt;
       decode_tile(job, t, c, z, mt, nt);
-      const int b = i & 1;
-      if (!mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u)) {
-        atomicExch(job.status, kErrEpilogue);
-        s_err = 1;
-        break;
-      }
-      tc_fence_after();
       EpiCtx<BN> ctx;
       ctx.cls = c;
       ctx.z = z;
@@ -323,15 +349,53 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       ctx.quad = quad;
       ctx.nparts = EPI_WARPS / 4;
       ctx.part = ew >> 2;
-      ctx.taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * C_::kAccCols);
+      ctx.taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)((i & 1) * C_::kAccCols);
       ctx.wsmem = epi_smem + (size_t)ew * EPI_SMEM;
-      ctx.wbar = epi_bar + 2 * ew;
+      ctx.wbar = epi_bar + kEpiBars * ew;
       ctx.uses = uses;
-      if (!s_err) Epi::run(prm, ctx);
+      ctx.slot = i & 1;
+      ctx.iter = i;
+      ctx.nxt_valid = t + (int)gridDim.x < job.total_tiles;
+      ctx.nxt_cls = ctx.nxt_z = ctx.nxt_m0 = ctx.nxt_n0 = 0;
+      if (ctx.nxt_valid) {
+        int c2, z2, mt2, nt2;
+        decode_tile(job, t + gridDim.x, c2, z2, mt2, nt2);
+        ctx.nxt_cls = c2;
+        ctx.nxt_z = z2;
+        ctx.nxt_m0 = mt2 * BM;
+        ctx.nxt_n0 = nt2 * BN;
+      }
+      return ctx;
+    };
+    constexpr bool kPre = EpiPrefetch<Epi>::value;
+    if constexpr (kPre) {
+      if ((int)blockIdx.x < job.total_tiles) pend[0] = Epi::prefetch(prm, make_ctx(blockIdx.x, 0));
+    }
+    int i = 0;
+    for (int t = blockIdx.x; t < job.total_tiles; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      const EpiCtx<BN> ctx = make_ctx(t, i);
+      if constexpr (kPre) {
+        if (t + (int)gridDim.x < job.total_tiles && !s_err)
+          pend[(i + 1) & 1] = Epi::prefetch(prm, make_ctx(t + gridDim.x, i + 1));
+      }
+      if (!mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u)) {
+        atomicExch(job.status, kErrEpilogue);
+        s_err = 1;
+        break;
+      }
+      tc_fence_after();
+      if (!s_err) {
+        Epi::run(prm, ctx);
+        pend[b] = false;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
+    // no prefetch of ours may still be in flight when the CTA exits
+    for (int k = 0; k < 2; ++k)
+      if (kPre && pend[k]) (void)mbar_wait(&epi_bar[kEpiBars * ew + k], uses[k] & 1u);
     if (EPI_SMEM > 0 && lane == 0) tc::bulk_wait_all();  // our TMA stores have completed
     __syncwarp();
   }
