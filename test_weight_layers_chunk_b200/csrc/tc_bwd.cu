@@ -17,6 +17,8 @@
 //   dM0 = U(1,n) D_M + c D_W ; abar, bbar and the chunk-scalar adjoints for the gate gradients.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "paths.h"
 #include "state.cuh"
 #include "tc_gemm2.cuh"
@@ -30,6 +32,8 @@ using tc2::EpiCtx;
 constexpr int kEW = 8;  // epilogue warps
 
 struct BwdP {
+  // 32 x 32 boxes for the epilogues' TMA-staged I/O (bf16: 64B swizzle, fp32: 128B)
+  CUtensorMap mHc, mY3, mDH, mHB, fdu, fDB, fUBd;
   Dims d;
   int ci, t0;
   const bf16 *v;
@@ -143,28 +147,108 @@ __device__ __forceinline__ void st8(bf16* dst, const float (&v)[8]) {
   *reinterpret_cast<uint4*>(dst) =
       make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
 }
+// ---------------------------------------------------------------- staged tile I/O
+// A warp's 32 rows x 32 columns move between global memory and shared memory as
+// one TMA box: bf16 boxes (2 KB) use the 64B swizzle, fp32 boxes (4 KB) the 128B
+// swizzle; lane r reads or writes row r. Buffers are 1024-byte aligned.
+__device__ __forceinline__ int swz64(int r, int q) { return r * 64 + ((q ^ ((r >> 1) & 3)) << 4); }
+__device__ __forceinline__ int swz128(int r, int q) { return r * 128 + ((q ^ (r & 7)) << 4); }
+__device__ __forceinline__ void stage_h(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(buf + swz64(r, q)) =
+        make_uint4(pack2(v[8 * q], v[8 * q + 1]), pack2(v[8 * q + 2], v[8 * q + 3]),
+                   pack2(v[8 * q + 4], v[8 * q + 5]), pack2(v[8 * q + 6], v[8 * q + 7]));
+}
+__device__ __forceinline__ void unstage_h(const uint8_t* buf, int r, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = *reinterpret_cast<const uint4*>(buf + swz64(r, q));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      v[8 * q + 2 * j] = f.x;
+      v[8 * q + 2 * j + 1] = f.y;
+    }
+  }
+}
+__device__ __forceinline__ void stage_f(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4*>(buf + swz128(r, q)) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+__device__ __forceinline__ void unstage_f(const uint8_t* buf, int r, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 f = *reinterpret_cast<const float4*>(buf + swz128(r, q));
+    v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+  }
+}
+// Before refilling the output staging: this warp's earlier TMA stores have read it.
+__device__ __forceinline__ void out_free(int lane) {
+  if (lane == 0) tc::bulk_wait_read<0>();
+  __syncwarp();
+}
+// After filling the output staging: visible to the TMA (async) proxy.
+__device__ __forceinline__ void out_ready() {
+  tc::fence_async_smem();
+  __syncwarp();
+}
+// Input loads are single-buffered and chained: group g + 1's boxes (or the next
+// tile's first group) are requested as soon as group g's are in registers, on the
+// warp's barrier 0. in_wait() consumes one completed load set.
+template <int BN>
+__device__ __forceinline__ bool in_wait(const BwdP& p, const EpiCtx<BN>& c) {
+  const bool ok = tc::mbar_wait(&c.wbar[0], c.uses[0] & 1u);
+  c.uses[0] += 1;
+  if (!ok && (c.row & 31) == 0) atomicExch(p.status, tc2::kErrEpilogue);
+  return ok;
+}
+// Where a warp's group gi (of ngroups) lies: this tile, or the next tile's first group.
+struct GroupAt {
+  int valid, z, m0, col;
+};
+template <int BN>
+__device__ __forceinline__ GroupAt group_at(const EpiCtx<BN>& c, int gi) {
+  const int per = BN / c.nparts;
+  if (gi < per / 32) return GroupAt{1, c.z, c.m0, c.n0 + c.part * per + gi * 32};
+  return GroupAt{c.nxt_valid, c.nxt_z, c.nxt_m0, c.nxt_n0 + c.part * per};
+}
+
 // Column groups of 32 owned by this thread inside the tile.
 #define FOR_GROUPS(c, BN, g) \
   for (int g = (c).part * ((BN) / (c).nparts); g < ((c).part + 1) * ((BN) / (c).nparts); g += 32)
 
 // ---------------------------------------------------------------- epilogues
-// R1: rows of X (keys then queries); h1 = acc0, h3 = acc1.
+// R1: rows of X (keys then queries); h1 = acc0, h3 = acc1 -> Hc, u = silu(h1) h3 -> Y3.
 struct EpiR1 {
+  static constexpr int kSmem = 6144;  // h1 | h3 | u staging (bf16)
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int r = c.m0 + c.row;
-    bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + r) * 2 * d.d_h;
-    bf16* urow = p.Y3 + ((size_t)c.z * 3 * d.C + d.C + r) * d.d_h;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;
+    const int yH = c.z * 2 * d.C + r0, yU = c.z * 3 * d.C + d.C + r0;
+    uint8_t* S = c.wsmem;
     FOR_GROUPS(c, BN, g) {
       const int j = c.n0 + g;
       float h1[32], h3[32];
       acc2(c, g, h1, h3);
-      st32(hrow + j, h1);
-      st32(hrow + d.d_h + j, h3);
+      out_free(lane);
+      stage_h(S, lane, h1);
+      stage_h(S + 2048, lane, h3);
 #pragma unroll
       for (int i = 0; i < 32; ++i) h1[i] = fsilu(h1[i]) * h3[i];
-      st32(urow + j, h1);
+      stage_h(S + 4096, lane, h1);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mHc, S, j, yH);
+        tc::tma_store_2d(&p.mHc, S + 2048, d.d_h + j, yH);
+        tc::tma_store_2d(&p.mY3, S + 4096, j, yU);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -187,22 +271,42 @@ struct EpiR2 {
     }
   }
 };
-// R3: du, dH1 = du H3 silu'(H1), dH3 = du silu(H1).
+// R3: du = E W2 -> du (fp32), dH1 = du H3 silu'(H1), dH3 = du silu(H1) (key rows).
 struct EpiR3 {
+  static constexpr int kIn = 4096;            // h1 | h3 (bf16)
+  static constexpr int kSmem = kIn + 8192;    // | du (fp32) | dH1 | dH3 (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    const int y = ga.z * 2 * p.d.C + ga.m0 + c.quad * 32;
+    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::tma_load_2d(c.wsmem, &p.mHc, &c.wbar[0], ga.col, y);
+    tc::tma_load_2d(c.wsmem + 2048, &p.mHc, &c.wbar[0], p.d.d_h + ga.col, y);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
-    float* durow = p.du + ((size_t)c.z * d.C + t) * d.d_h;
-    bf16* dhrow = p.DH + ((size_t)c.z * d.C + t) * 2 * d.d_h;
-    FOR_GROUPS(c, BN, g) {
-      const int j = c.n0 + g;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int yD = c.z * d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* F = c.wsmem + kIn;
+    uint8_t* Hs = c.wsmem + kIn + 4096;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
       float du[32], h1[32], h3[32];
       acc1(c, g, du);
-      st32f(durow + j, du);
-      ld32(hrow + j, h1);
-      ld32(hrow + d.d_h + j, h3);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, h1);
+      unstage_h(IN + 2048, lane, h3);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const Act f(h1[i]);
@@ -210,28 +314,59 @@ struct EpiR3 {
         h3[i] = du[i] * f.s;  // dH3
         h1[i] = dh1;
       }
-      st32(dhrow + j, h1);
-      st32(dhrow + d.d_h + j, h3);
+      out_free(lane);
+      stage_f(F, lane, du);
+      stage_h(Hs, lane, h1);
+      stage_h(Hs + 2048, lane, h3);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fdu, F, j, yD);
+        tc::tma_store_2d(&p.mDH, Hs, j, yD);
+        tc::tma_store_2d(&p.mDH, Hs + 2048, d.d_h + j, yD);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
-// D1: acc0 = K D_M13^T, acc1 = K D_W13^T over columns [0, 2 d_h).
+// D1: acc0 = K D_M13^T, acc1 = K D_W13^T over columns [0, 2 d_h) -> DB = -(a P_M + b P_W)
+// (fp32) and the abar / bbar partial dot products with dH.
 struct EpiD1 {
+  static constexpr int kIn = 2048;           // dH (bf16)
+  static constexpr int kSmem = kIn + 4096;   // | DB (fp32)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
+    tc::tma_load_2d(c.wsmem, &p.mDH, &c.wbar[0], ga.col, ga.z * p.d.C + ga.m0 + c.quad * 32);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
     const float a = p.ca[tok], b = p.cb[tok];
-    const bf16* dhrow = p.DH + ((size_t)c.z * d.C + t) * 2 * d.d_h;
-    float* dbrow = p.DB + ((size_t)c.z * d.C + t) * 2 * d.d_h;
+    const int yD = c.z * d.C + c.m0 + c.quad * 32;
     float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG;
     float* pb = pa + (size_t)d.BH * d.C * p.NG;
-    FOR_GROUPS(c, BN, g) {
-      const int jj = c.n0 + g;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* F = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, jj = c.n0 + g;
       float pm[32], pw[32], dh[32];
       acc2(c, g, pm, pw);
-      ld32(dhrow + jj, dh);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, dh);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
       float sa = 0.f, sb = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -239,7 +374,14 @@ struct EpiD1 {
         sb += dh[i] * pw[i];
         pm[i] = -(a * pm[i] + b * pw[i]);
       }
-      st32f(dbrow + jj, pm);
+      out_free(lane);
+      stage_f(F, lane, pm);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fDB, F, jj, yD);
+        tc::bulk_commit();
+      }
+      __syncwarp();
       pa[jj / 32] = sa;
       pb[jj / 32] = sb;
     }
@@ -275,35 +417,71 @@ struct EpiD2 {
     }
   }
 };
-// E3: acc0 = E D_M2, acc1 = E D_W2 (columns = hidden units); dub.
+// E3: acc0 = E D_M2, acc1 = E D_W2 (columns = hidden units) -> UBd = -(a . + b .)
+// (fp32) and dub = dh1b H3 silu'(H1) + dh3b silu(H1) (bf16, rows [0, C) of Y3).
 struct EpiE3 {
+  static constexpr int kWarps = 4;
+  static constexpr int kIn = 12288;          // dh1b | dh3b (fp32) | h1 | h3 (bf16)
+  static constexpr int kSmem = kIn + 6144;   // | UBd (fp32) | dub (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    const Dims& d = p.d;
+    const int r = ga.m0 + c.quad * 32;
+    uint64_t* bar = &c.wbar[0];
+    tc::mbar_expect_tx(bar, 12288u);
+    tc::tma_load_2d(c.wsmem, &p.fDB, bar, ga.col, ga.z * d.C + r);
+    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, d.d_h + ga.col, ga.z * d.C + r);
+    tc::tma_load_2d(c.wsmem + 8192, &p.mHc, bar, ga.col, ga.z * 2 * d.C + r);
+    tc::tma_load_2d(c.wsmem + 10240, &p.mHc, bar, d.d_h + ga.col, ga.z * 2 * d.C + r);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
     const float a = p.ca[tok], b = p.cb[tok];
-    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
-    const float* dbrow = p.DB + ((size_t)c.z * d.C + t) * 2 * d.d_h;
-    float* ubrow = p.UBd + ((size_t)c.z * d.C + t) * d.d_h;
-    bf16* dubrow = p.Y3 + ((size_t)c.z * 3 * d.C + t) * d.d_h;
-    FOR_GROUPS(c, BN, g) {
-      const int j = c.n0 + g;
-      float m[32], w[32], h1[32], h3[32];
+    const int r0 = c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* F = c.wsmem + kIn;
+    uint8_t* Hs = c.wsmem + kIn + 4096;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
+      float m[32], w[32];
       acc2(c, g, m, w);
 #pragma unroll
       for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
-      st32f(ubrow + j, m);
-      ld32(hrow + j, h1);
-      ld32(hrow + d.d_h + j, h3);
-      ld32f(dbrow + j, m);           // dh1b
-      ld32f(dbrow + d.d_h + j, w);   // dh3b
+      out_free(lane);
+      stage_f(F, lane, m);
+      if (!in_wait(p, c)) return;
+      float b1[32], b3[32];
+      unstage_f(IN, lane, b1);
+      unstage_f(IN + 4096, lane, b3);
+      unstage_h(IN + 8192, lane, m);       // h1
+      unstage_h(IN + 10240, lane, w);      // h3
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const Act f(h1[i]);
-        m[i] = m[i] * h3[i] * f.d1 + w[i] * f.s;
+        const Act f(m[i]);
+        b1[i] = b1[i] * w[i] * f.d1 + b3[i] * f.s;
       }
-      st32(dubrow + j, m);
+      stage_h(Hs, lane, b1);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fUBd, F, j, c.z * d.C + r0);
+        tc::tma_store_2d(&p.mY3, Hs, j, c.z * 3 * d.C + r0);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -335,28 +513,69 @@ struct EpiE4 {
     }
   }
 };
-// E5: ub = E3 term + eb W2 (MSE); the key rows' h1b, h3b (8 columns at a time).
+// E5: ub = UBd + eb W2 (MSE); the key rows' h1b, h3b (8 columns at a time).
 struct EpiE5 {
+  static constexpr int kWarps = 4;
+  static constexpr int kIn = 20480;          // UBd | du | dh1b | dh3b (fp32) | h1 | h3 (bf16)
+  static constexpr int kSmem = kIn + 4096;   // | h1b | h3b (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    const Dims& d = p.d;
+    const int r = ga.m0 + c.quad * 32;
+    const int yC = ga.z * d.C + r, yH = ga.z * 2 * d.C + r;
+    uint64_t* bar = &c.wbar[0];
+    tc::mbar_expect_tx(bar, 20480u);
+    tc::tma_load_2d(c.wsmem, &p.fUBd, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 4096, &p.fdu, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 8192, &p.fDB, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 12288, &p.fDB, bar, d.d_h + ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 16384, &p.mHc, bar, ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 18432, &p.mHc, bar, d.d_h + ga.col, yH);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    const size_t row = (size_t)c.z * d.C + t;
-    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
-    bf16* hbrow = p.HB + ((size_t)c.z * 2 * d.C + t) * 2 * d.d_h;
-    FOR_GROUPS(c, BN, g) {
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int yH = c.z * 2 * d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
       float acc[32];
       acc1(c, g, acc);
+      if (!in_wait(p, c)) return;
+      out_free(lane);
 #pragma unroll
       for (int s8 = 0; s8 < 4; ++s8) {
-        const int j = c.n0 + g + 8 * s8;
-        float ubd[8], h1[8], h3[8], du[8], b1[8], b3[8];
-        ld8f(p.UBd + row * d.d_h + j, ubd);
-        ld8(hrow + j, h1);
-        ld8(hrow + d.d_h + j, h3);
-        ld8f(p.du + row * d.d_h + j, du);
-        ld8f(p.DB + row * 2 * d.d_h + j, b1);           // dh1b
-        ld8f(p.DB + row * 2 * d.d_h + d.d_h + j, b3);   // dh3b
+        // 8 consecutive columns: one 16-byte chunk of a bf16 row, two of an fp32 row
+        const float4 u0 = *reinterpret_cast<const float4*>(IN + swz128(lane, 2 * s8));
+        const float4 u1 = *reinterpret_cast<const float4*>(IN + swz128(lane, 2 * s8 + 1));
+        const float4 d0 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8));
+        const float4 d1 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8 + 1));
+        const float4 p0 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8));
+        const float4 p1 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8 + 1));
+        const float4 q0 = *reinterpret_cast<const float4*>(IN + 12288 + swz128(lane, 2 * s8));
+        const float4 q1 = *reinterpret_cast<const float4*>(IN + 12288 + swz128(lane, 2 * s8 + 1));
+        const float ubd[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        const float du[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        const float b1[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        const float b3[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        float h1[8], h3[8];
+        const uint4 x1 = *reinterpret_cast<const uint4*>(IN + 16384 + swz64(lane, s8));
+        const uint4 x3 = *reinterpret_cast<const uint4*>(IN + 18432 + swz64(lane, s8));
+        const uint32_t w1[4] = {x1.x, x1.y, x1.z, x1.w}, w3[4] = {x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w1[k]));
+          const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w3[k]));
+          h1[2 * k] = f1.x; h1[2 * k + 1] = f1.y;
+          h3[2 * k] = f3.x; h3[2 * k + 1] = f3.y;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float ub = ubd[i] + (d.loss == 0 ? acc[8 * s8 + i] : 0.f);
@@ -367,26 +586,61 @@ struct EpiE5 {
           h1[i] = h1b;
           h3[i] = h3b;
         }
-        st8(hbrow + j, h1);
-        st8(hbrow + d.d_h + j, h3);
+        *reinterpret_cast<uint4*>(OUT + swz64(lane, s8)) =
+            make_uint4(pack2(h1[0], h1[1]), pack2(h1[2], h1[3]), pack2(h1[4], h1[5]), pack2(h1[6], h1[7]));
+        *reinterpret_cast<uint4*>(OUT + 2048 + swz64(lane, s8)) =
+            make_uint4(pack2(h3[0], h3[1]), pack2(h3[2], h3[3]), pack2(h3[4], h3[5]), pack2(h3[6], h3[7]));
       }
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mHB, OUT, j, yH);
+        tc::tma_store_2d(&p.mHB, OUT + 2048, d.d_h + j, yH);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
 // Q1: ub_q = dout W2 -> query-row h1b = ub H3 silu'(H1), h3b = ub silu(H1).
 struct EpiQ1 {
+  static constexpr int kIn = 4096;           // query h1 | h3 (bf16)
+  static constexpr int kSmem = kIn + 4096;   // | h1b | h3b (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    const int y = ga.z * 2 * p.d.C + p.d.C + ga.m0 + c.quad * 32;
+    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::tma_load_2d(c.wsmem, &p.mHc, &c.wbar[0], ga.col, y);
+    tc::tma_load_2d(c.wsmem + 2048, &p.mHc, &c.wbar[0], p.d.d_h + ga.col, y);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    const bf16* hrow = p.Hc + ((size_t)c.z * 2 * d.C + d.C + t) * 2 * d.d_h;
-    bf16* hbrow = p.HB + ((size_t)c.z * 2 * d.C + d.C + t) * 2 * d.d_h;
-    FOR_GROUPS(c, BN, g) {
-      const int j = c.n0 + g;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int y = c.z * 2 * d.C + d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
       float ub[32], h1[32], h3[32];
       acc1(c, g, ub);
-      ld32(hrow + j, h1);
-      ld32(hrow + d.d_h + j, h3);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, h1);
+      unstage_h(IN + 2048, lane, h3);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const Act f(h1[i]);
@@ -394,8 +648,16 @@ struct EpiQ1 {
         h3[i] = ub[i] * f.s;
         h1[i] = a1;
       }
-      st32(hbrow + j, h1);
-      st32(hbrow + d.d_h + j, h3);
+      out_free(lane);
+      stage_h(OUT, lane, h1);
+      stage_h(OUT + 2048, lane, h3);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mHB, OUT, j, y);
+        tc::tma_store_2d(&p.mHB, OUT + 2048, d.d_h + j, y);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -602,19 +864,53 @@ bool mk(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// 2-D map, box 32 columns x 32 rows: bf16 with 64B swizzle, fp32 with 128B swizzle
+// (the epilogues' staged I/O).
+bool box32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, bool f32) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * es};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t el[2] = {1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n;
 }
+// Per-epilogue launch shape: shared memory per epilogue warp (kSmem, default 0)
+// and epilogue warps (kWarps, default 8).
+template <class E, class = void>
+struct EpiSmemOf { static constexpr int v = 0; };
+template <class E>
+struct EpiSmemOf<E, std::void_t<decltype(E::kSmem)>> { static constexpr int v = E::kSmem; };
+template <class E, class = void>
+struct EpiWarpsOf { static constexpr int v = kEW; };
+template <class E>
+struct EpiWarpsOf<E, std::void_t<decltype(E::kWarps)>> { static constexpr int v = E::kWarps; };
+
 template <int NUM_ACC, bool A_MN, bool B_MN, class Epi>
 cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
-  // two 64-wide k-blocks per ring slot (one producer/MMA handshake per 128 of K)
-  constexpr int KG = 2;
-  constexpr int STAGES = NUM_ACC == 1 ? 3 : 2;
-  constexpr size_t smem = tc2::smem_bytes<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, 0, KG>();
+  constexpr int EW = EpiWarpsOf<Epi>::v;
+  constexpr int ESM = EpiSmemOf<Epi>::v;
+  constexpr uint32_t kStage = tc2::Cfg<128, NUM_ACC, A_MN, B_MN>::kStage;
+  // Epilogues without staging buffers: two 64-wide k-blocks per ring slot (one
+  // producer/MMA handshake per 128 of K). With staging: single k-block slots, as
+  // many (up to 4) as the shared memory left over holds.
+  constexpr int KG = ESM == 0 ? 2 : 1;
+  constexpr long long kFree = 232448LL - 1024 - 256 - 8LL * tc2::kEpiBars * EW - (long long)EW * ESM;
+  constexpr int kFit = (int)(kFree / ((long long)KG * kStage));
+  constexpr int STAGES = ESM == 0 ? (NUM_ACC == 1 ? 3 : 2) : (kFit > 4 ? 4 : kFit);
+  static_assert(STAGES >= 2, "at least two ring slots");
+  constexpr size_t smem = tc2::smem_bytes<128, NUM_ACC, A_MN, B_MN, STAGES, EW, ESM, KG>();
   static_assert(smem <= 232448, "shared memory per CTA");
-  auto kern = tc2::gemm_persistent<128, NUM_ACC, A_MN, B_MN, STAGES, kEW, Epi, BwdP, 0, KG>;
+  auto kern = tc2::gemm_persistent<128, NUM_ACC, A_MN, B_MN, STAGES, EW, Epi, BwdP, ESM, KG>;
   job.total_tiles = 0;
   for (int c = 0; c < job.n_cls; ++c) {
     if (job.cls[c].kblocks % KG != 0) return cudaErrorInvalidValue;
@@ -624,7 +920,7 @@ cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
   E2TTT_TRACE(Name<Epi>::v, st);
-  kern<<<grid, (2 + kEW) * 32, smem, st>>>(job, p);
+  kern<<<grid, (2 + EW) * 32, smem, st>>>(job, p);
   return cudaGetLastError();
 }
 
@@ -712,6 +1008,17 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   p.du = B.du; p.DB = B.DB; p.G2U = B.G2U; p.UBd = B.UBd; p.dkp = B.dkp; p.part = B.part;
   p.NG = (int)(2 * dh / 32 + dv / 32);
   p.status = B.status;
+  {
+    const uint64_t rC = (uint64_t)BH * C;
+    bool mok = box32(&p.mHc, B.Hc, 2 * rC, 2 * dh, false);
+    mok &= box32(&p.mY3, B.Y3, 3 * rC, dh, false);
+    mok &= box32(&p.mDH, B.DH, rC, 2 * dh, false);
+    mok &= box32(&p.mHB, B.HB, 2 * rC, 2 * dh, false);
+    mok &= box32(&p.fdu, B.du, rC, dh, true);
+    mok &= box32(&p.fDB, B.DB, rC, 2 * dh, true);
+    mok &= box32(&p.fUBd, B.UBd, rC, dh, true);
+    if (!mok) return cudaErrorInvalidValue;
+  }
 
   // operand maps (per call; the chunk only changes the copies and the epilogue data)
   tc2::Job r1{}, r2{}, r3{}, d1{}, d2{}, e3{}, e4{}, e5{}, q1{}, k1{}, k2{}, dq{}, dw{};
