@@ -34,6 +34,7 @@ constexpr int kEW = 8;  // epilogue warps
 struct BwdP {
   // 32 x 32 boxes for the epilogues' TMA-staged I/O (bf16: 64B swizzle, fp32: 128B)
   CUtensorMap mHc, mY3, mDH, mHB, fdu, fDB, fUBd;
+  CUtensorMap mZ3, mv, mdv, mdk, mdq, fG2U, fdkp, fDW[2];
   Dims d;
   int ci, t0;
   const bf16 *v;
@@ -62,40 +63,6 @@ struct BwdP {
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ void st32(bf16* dst, const float (&v)[32]) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    p[i] = make_uint4(pack2(v[8 * i], v[8 * i + 1]), pack2(v[8 * i + 2], v[8 * i + 3]),
-                      pack2(v[8 * i + 4], v[8 * i + 5]), pack2(v[8 * i + 6], v[8 * i + 7]));
-}
-__device__ __forceinline__ void ld32(const bf16* src, float (&v)[32]) {
-  const uint4* p = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 u = p[i];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-      v[8 * i + 2 * j] = f.x;
-      v[8 * i + 2 * j + 1] = f.y;
-    }
-  }
-}
-__device__ __forceinline__ void ld32f(const float* src, float (&v)[32]) {
-  const float4* p = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 f = p[i];
-    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
-  }
-}
-__device__ __forceinline__ void st32f(float* dst, const float (&v)[32]) {
-  float4* p = reinterpret_cast<float4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) p[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 template <int BN>
 __device__ __forceinline__ void acc1(const EpiCtx<BN>& c, int col, float (&x)[32]) {
@@ -128,25 +95,6 @@ struct Act {
   }
 };
 __device__ __forceinline__ float fsilu(float z) { return z * __fdividef(1.0f, 1.0f + __expf(-z)); }
-// 8 consecutive bf16 / fp32 values
-__device__ __forceinline__ void ld8(const bf16* src, float (&v)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4*>(src);
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-    v[2 * j] = f.x;
-    v[2 * j + 1] = f.y;
-  }
-}
-__device__ __forceinline__ void ld8f(const float* src, float (&v)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void st8(bf16* dst, const float (&v)[8]) {
-  *reinterpret_cast<uint4*>(dst) =
-      make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
-}
 // ---------------------------------------------------------------- staged tile I/O
 // A warp's 32 rows x 32 columns move between global memory and shared memory as
 // one TMA box: bf16 boxes (2 KB) use the 64B swizzle, fp32 boxes (4 KB) the 128B
@@ -207,13 +155,13 @@ __device__ __forceinline__ bool in_wait(const BwdP& p, const EpiCtx<BN>& c) {
 }
 // Where a warp's group gi (of ngroups) lies: this tile, or the next tile's first group.
 struct GroupAt {
-  int valid, z, m0, col;
+  int valid, cls, z, m0, col;
 };
 template <int BN>
 __device__ __forceinline__ GroupAt group_at(const EpiCtx<BN>& c, int gi) {
   const int per = BN / c.nparts;
-  if (gi < per / 32) return GroupAt{1, c.z, c.m0, c.n0 + c.part * per + gi * 32};
-  return GroupAt{c.nxt_valid, c.nxt_z, c.nxt_m0, c.nxt_n0 + c.part * per};
+  if (gi < per / 32) return GroupAt{1, c.cls, c.z, c.m0, c.n0 + c.part * per + gi * 32};
+  return GroupAt{c.nxt_valid, c.nxt_cls, c.nxt_z, c.nxt_m0, c.nxt_n0 + c.part * per};
 }
 
 // Column groups of 32 owned by this thread inside the tile.
@@ -252,22 +200,48 @@ struct EpiR1 {
     }
   }
 };
-// R2: E = y - v (or -v) of the key rows.
+// R2: E = y - v (or -v) of the key rows -> rows [0, C) of Z3.
 struct EpiR2 {
+  static constexpr int kIn = 2048;           // v (bf16)
+  static constexpr int kSmem = kIn + 2048;   // | E (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
+    tc::tma_load_2d(c.wsmem, &p.mv, &c.wbar[0], ga.col, ga.z * p.d.T + p.t0 + ga.m0 + c.quad * 32);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    const bf16* vrow = p.v + ((size_t)c.z * d.T + p.t0 + t) * d.d_v;
-    bf16* erow = p.Z3 + ((size_t)c.z * 3 * d.C + t) * d.d_v;
-    FOR_GROUPS(c, BN, g) {
-      const int col = c.n0 + g;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int yE = c.z * 3 * d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, col = c.n0 + g;
       float y[32], vv[32];
       acc1(c, g, y);
-      ld32(vrow + col, vv);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, vv);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
-      st32(erow + col, y);
+      out_free(lane);
+      stage_h(OUT, lane, y);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mZ3, OUT, col, yE);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -387,23 +361,44 @@ struct EpiD1 {
     }
   }
 };
-// D2: acc0 = U_k D_M2^T, acc1 = U_k D_W2^T over columns [0, d_v).
+// D2: acc0 = U_k D_M2^T, acc1 = U_k D_W2^T over columns [0, d_v) -> G2u = -(a P_M + b P_W)
+// (fp32) and the abar / bbar partial dot products with E.
 struct EpiD2 {
+  static constexpr int kIn = 2048;           // E (bf16)
+  static constexpr int kSmem = kIn + 4096;   // | G2u (fp32)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
+    tc::tma_load_2d(c.wsmem, &p.mZ3, &c.wbar[0], ga.col, ga.z * 3 * p.d.C + ga.m0 + c.quad * 32);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
     const float a = p.ca[tok], b = p.cb[tok];
-    const bf16* erow = p.Z3 + ((size_t)c.z * 3 * d.C + t) * d.d_v;
-    float* grow = p.G2U + ((size_t)c.z * d.C + t) * d.d_v;
+    const int yG = c.z * d.C + c.m0 + c.quad * 32;
     float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG + 2 * d.d_h / 32;
     float* pb = pa + (size_t)d.BH * d.C * p.NG;
-    FOR_GROUPS(c, BN, g) {
-      const int col = c.n0 + g;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* F = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, col = c.n0 + g;
       float pm[32], pw[32], e[32];
       acc2(c, g, pm, pw);
-      ld32(erow + col, e);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, e);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
       float sa = 0.f, sb = 0.f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -411,7 +406,14 @@ struct EpiD2 {
         sb += e[i] * pw[i];
         pm[i] = -(a * pm[i] + b * pw[i]);
       }
-      st32f(grow + col, pm);
+      out_free(lane);
+      stage_f(F, lane, pm);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fG2U, F, col, yG);
+        tc::bulk_commit();
+      }
+      __syncwarp();
       pa[col / 32] = sa;
       pb[col / 32] = sb;
     }
@@ -485,31 +487,58 @@ struct EpiE3 {
     }
   }
 };
-// E4: eb = dub W2^T + G2u; EB row (zero for the dot loss), dv = -eb.
+// E4: eb = dub W2^T + G2u; EB row (zero for the dot loss) -> rows [C, 2C) of Z3, dv = -eb.
 struct EpiE4 {
+  static constexpr int kIn = 4096;           // G2u (fp32)
+  static constexpr int kSmem = kIn + 4096;   // | dv | EB (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::tma_load_2d(c.wsmem, &p.fG2U, &c.wbar[0], ga.col, ga.z * p.d.C + ga.m0 + c.quad * 32);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    const float* grow = p.G2U + ((size_t)c.z * d.C + t) * d.d_v;
-    bf16* ebrow = p.Z3 + ((size_t)c.z * 3 * d.C + d.C + t) * d.d_v;
-    bf16* dvrow = p.dv + ((size_t)c.z * d.T + p.t0 + t) * d.d_v;
-    FOR_GROUPS(c, BN, g) {
-      const int col = c.n0 + g;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int r0 = c.m0 + c.quad * 32;
+    const int yV = c.z * d.T + p.t0 + r0, yB = c.z * 3 * d.C + d.C + r0;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, col = c.n0 + g;
       float eb[32], gu[32];
       acc1(c, g, eb);
-      ld32f(grow + col, gu);
+      if (!in_wait(p, c)) return;
+      unstage_f(IN, lane, gu);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         eb[i] += gu[i];
         gu[i] = -eb[i];
       }
-      st32(dvrow + col, gu);
       if (d.loss != 0) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) eb[i] = 0.f;
       }
-      st32(ebrow + col, eb);
+      out_free(lane);
+      stage_h(OUT, lane, gu);
+      stage_h(OUT + 2048, lane, eb);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mdv, OUT, col, yV);
+        tc::tma_store_2d(&p.mZ3, OUT + 2048, col, yB);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -661,64 +690,128 @@ struct EpiQ1 {
     }
   }
 };
-// dk part 1: -(a dH D_M13 + b dH D_W13) (fp32).
+// dk part 1: -(a dH D_M13 + b dH D_W13) (fp32) -> dkp.
 struct EpiDk1 {
+  static constexpr int kSmem = 4096;  // dkp staging (fp32)
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
+    const int lane = c.row & 31;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
     const float a = p.ca[tok], b = p.cb[tok];
-    float* o = p.dkp + ((size_t)c.z * d.C + t) * d.d_k;
+    const int y = c.z * d.C + c.m0 + c.quad * 32;
+    uint8_t* F = c.wsmem;
     FOR_GROUPS(c, BN, g) {
       float m[32], w[32];
       acc2(c, g, m, w);
 #pragma unroll
       for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
-      st32f(o + c.n0 + g, m);
+      out_free(lane);
+      stage_f(F, lane, m);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fdkp, F, c.n0 + g, y);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
-// dk part 2 (adds part 1) and dq: [h1b | h3b] [W1; W3] -> act output.
+// dk part 2 (adds part 1) and dq: [h1b | h3b] [W1; W3] -> the activation-dtype output.
 template <bool KEYS>
 struct EpiDkq {
+  static constexpr int kIn = KEYS ? 4096 : 0;  // dkp (fp32)
+  static constexpr int kSmem = kIn + 2048;     // | dk or dq (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::tma_load_2d(c.wsmem, &p.fdkp, &c.wbar[0], ga.col, ga.z * p.d.C + ga.m0 + c.quad * 32);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int t = c.m0 + c.row;
-    bf16* o = (KEYS ? p.dk : p.dq) + ((size_t)c.z * d.T + p.t0 + t) * d.d_k;
-    FOR_GROUPS(c, BN, g) {
-      const int col = c.n0 + g;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int yO = c.z * d.T + p.t0 + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (KEYS && c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, col = c.n0 + g;
       float x[32];
       acc1(c, g, x);
       if (KEYS) {
         float y[32];
-        ld32f(p.dkp + ((size_t)c.z * d.C + t) * d.d_k + col, y);
+        if (!in_wait(p, c)) return;
+        unstage_f(IN, lane, y);
+        __syncwarp();
+        if (lane == 0) {
+          tc::fence_async_smem();
+          issue(p, c, gi + 1);
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] += y[i];
       }
-      st32(o + col, x);
+      out_free(lane);
+      stage_h(OUT, lane, x);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(KEYS ? &p.mdk : &p.mdq, OUT, col, yO);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
-// dW: D_W <- L(1,n) D_W + acc, class 0 = rows of [W1; W3], class 1 = rows of W2.
+// dW: D_W <- L(1,n) D_W + acc in place, class 0 = rows of [W1; W3], class 1 = rows
+// of W2; the fp32 rows of D_W move through shared memory with TMA.
 struct EpiDW {
+  static constexpr int kIn = 4096;           // D_W block (fp32)
+  static constexpr int kSmem = kIn + 4096;   // | updated block (fp32)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::tma_load_3d(c.wsmem, &p.fDW[ga.cls], &c.wbar[0], ga.col, ga.m0 + c.quad * 32, ga.z);
+  }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
-    const int i = c.m0 + c.row;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
     const size_t plane = (size_t)d.BH * d.NC;
     const float PL = p.scal[plane + (size_t)c.z * d.NC + p.ci];
-    const int ld = c.cls == 0 ? d.d_k : d.d_h;
-    const long long base = c.cls == 0 ? 0 : 2LL * d.d_h * d.d_k;
-    float* row = p.DW + (size_t)c.z * d.S + base + (long long)i * ld;
-    FOR_GROUPS(c, BN, g) {
+    const int r0 = c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32;
       float x[32], y[32];
       acc1(c, g, x);
-      ld32f(row + c.n0 + g, y);
+      if (!in_wait(p, c)) return;
+      unstage_f(IN, lane, y);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
 #pragma unroll
       for (int q = 0; q < 32; ++q) y[q] = PL * y[q] + x[q];
-      st32f(row + c.n0 + g, y);
+      out_free(lane);
+      stage_f(OUT, lane, y);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_3d(&p.fDW[c.cls], OUT, c.n0 + g, r0, c.z);
+        tc::bulk_commit();
+      }
+      __syncwarp();
     }
   }
 };
@@ -879,6 +972,20 @@ bool box32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, bool 
             f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// 3-D fp32 map over [heads, rows, cols] of one block of every head's state
+// (head stride S), box 32 x 32 x 1, 128B swizzle.
+bool state_box32(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols, uint64_t heads,
+                 uint64_t head_stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, heads};
+  cuuint64_t strides[2] = {cols * 4, head_stride * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t el[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, el,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -1017,6 +1124,16 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     mok &= box32(&p.fdu, B.du, rC, dh, true);
     mok &= box32(&p.fDB, B.DB, rC, 2 * dh, true);
     mok &= box32(&p.fUBd, B.UBd, rC, dh, true);
+    const uint64_t rT = (uint64_t)BH * T;
+    mok &= box32(&p.mZ3, B.Z3, 3 * rC, dv, false);
+    mok &= box32(&p.mv, A.v, rT, dv, false);
+    mok &= box32(&p.mdv, A.dv, rT, dv, false);
+    mok &= box32(&p.mdk, A.dk, rT, dk, false);
+    mok &= box32(&p.mdq, A.dq, rT, dk, false);
+    mok &= box32(&p.fG2U, B.G2U, rC, dv, true);
+    mok &= box32(&p.fdkp, B.dkp, rC, dk, true);
+    mok &= state_box32(&p.fDW[0], A.dW0, 2 * dh, dk, BH, d.S);
+    mok &= state_box32(&p.fDW[1], A.dW0 + 2 * (size_t)dh * dk, dv, dh, BH, d.S);
     if (!mok) return cudaErrorInvalidValue;
   }
 
