@@ -34,7 +34,11 @@ Functions, and what each follows:
                  aggregations (abstract; atlas "Approach");
   seq_bwd        the reverse of seq_fwd's loop, token by token, with the second
                  order terms through g_t(W_chunk_start, k_t, v_t);
-  closed_bwd     the adjoint of closed_fwd (a second route; pinned to seq_bwd).
+  closed_bwd     the adjoint of closed_fwd (a second route; pinned to seq_bwd);
+  chunk_mean_kernels  the chunk-averaged variant (atlas "Surprising findings":
+                 per-token factors collapsed to chunk scalars), read as the
+                 chunk means of a_t and b_t; closed_fwd / closed_bwd take it
+                 with coef=COEF_CHUNK_MEAN.
 State layout per (b, h): linear W [d_v, d_k]; SwiGLU [W1 (d_h x d_k) | W3
 (d_h x d_k) | W2 (d_v x d_h)], each row-major, concatenated.
 """
@@ -47,6 +51,8 @@ LINEAR = 0
 SWIGLU = 1
 LOSS_MSE = 0
 LOSS_NEG_DOT = 1
+COEF_PER_TOKEN = 0     # per-token momentum / weight kernels (the method)
+COEF_CHUNK_MEAN = 1    # the chunk-averaged variant
 
 
 # --------------------------------------------------------------------------- layout
@@ -323,8 +329,24 @@ def chunk_kernels(eta, mu, lam):
     return a, b, P_U, P_L, c
 
 
-def all_chunk_kernels(lr, mom, decay, C):
-    """chunk_kernels over [B,H,T] gates: a, b [B,H,T]; P_U, P_L, c [B,H,n_chunks]."""
+def chunk_mean_kernels(eta, mu, lam):
+    """The chunk-averaged variant (atlas.scime.ai summary, "Surprising findings":
+    the per-token factors collapsed to chunk scalars): chunk_kernels' momentum
+    and weight kernels replaced by their means over the chunk's tokens, so every
+    token of the chunk carries a_bar = mean_t a_t and b_bar = mean_t b_t; the
+    chunk scalars P_U, P_L, c are those of the recurrence. Reading: "collapsed to
+    chunk scalars" = the arithmetic mean."""
+    a, b, P_U, P_L, c = chunk_kernels(eta, mu, lam)
+    return np.full_like(a, a.mean()), np.full_like(b, b.mean()), P_U, P_L, c
+
+
+def _kernels(coef):
+    return chunk_mean_kernels if coef == COEF_CHUNK_MEAN else chunk_kernels
+
+
+def all_chunk_kernels(lr, mom, decay, C, coef=COEF_PER_TOKEN):
+    """chunk_kernels (or chunk_mean_kernels) over [B,H,T] gates: a, b [B,H,T];
+    P_U, P_L, c [B,H,n_chunks]."""
     lr, mom, decay = _f64(lr), _f64(mom), _f64(decay)
     B, H, T = lr.shape
     chunks = _chunks(T, C)
@@ -334,8 +356,8 @@ def all_chunk_kernels(lr, mom, decay, C):
     for bb in range(B):
         for hh in range(H):
             for ci, (t0, t1) in enumerate(chunks):
-                aa, bbv, pu, pl, cc = chunk_kernels(lr[bb, hh, t0:t1], mom[bb, hh, t0:t1],
-                                                    decay[bb, hh, t0:t1])
+                aa, bbv, pu, pl, cc = _kernels(coef)(lr[bb, hh, t0:t1], mom[bb, hh, t0:t1],
+                                                     decay[bb, hh, t0:t1])
                 a[bb, hh, t0:t1] = aa
                 b[bb, hh, t0:t1] = bbv
                 sc[:, bb, hh, ci] = (pu, pl, cc)
@@ -369,13 +391,14 @@ def weighted_sum(factors, w):
 
 
 def closed_fwd(kind, q, k, v, lr, mom, decay, W0, M0, C, d_h=0, loss=LOSS_MSE,
-               return_starts=False, heads=None):
+               return_starts=False, heads=None, coef=COEF_PER_TOKEN):
     """Closed-form chunk transition: per chunk
         out_t = f_{W0}(q_t),
         M_end = P_U M0 - sum_t a_t g_t,
         W_end = P_L W0 + c M0 - sum_t b_t g_t,
-    with g_t at the chunk-start weights W0. ``heads`` optionally restricts the
-    computation to a list of (b, h) pairs (the others are left zero)."""
+    with g_t at the chunk-start weights W0 (a_t, b_t the chunk means for
+    coef=COEF_CHUNK_MEAN). ``heads`` optionally restricts the computation to a
+    list of (b, h) pairs (the others are left zero)."""
     q, k, v, lr, mom, decay, W0, M0 = map(_f64, (q, k, v, lr, mom, decay, W0, M0))
     B, H, T = lr.shape
     d_k, d_v, S = _dims(kind, q, v, W0, d_h)
@@ -395,7 +418,8 @@ def closed_fwd(kind, q, k, v, lr, mom, decay, W0, M0, C, d_h=0, loss=LOSS_MSE,
             P = unpack(kind, W, d_k, d_v, d_h)
             Q = q[b, h, t0:t1]
             out[b, h, t0:t1] = _fast_apply_rows(kind, P, Q)
-            a, bb, P_U, P_L, c = chunk_kernels(lr[b, h, t0:t1], mom[b, h, t0:t1], decay[b, h, t0:t1])
+            a, bb, P_U, P_L, c = _kernels(coef)(lr[b, h, t0:t1], mom[b, h, t0:t1],
+                                                decay[b, h, t0:t1])
             fac = chunk_grads(kind, loss, P, k[b, h, t0:t1], v[b, h, t0:t1])
             dM = pack(kind, weighted_sum(fac, a))
             dW = pack(kind, weighted_sum(fac, bb))
@@ -545,14 +569,16 @@ def chunk_kernels_vjp(eta, mu, lam, abar, bbar, PUbar, PLbar, cbar):
 
 
 def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_end=None,
-               d_h=0, loss=LOSS_MSE, heads=None):
+               d_h=0, loss=LOSS_MSE, heads=None, coef=COEF_PER_TOKEN):
     """Adjoint of closed_fwd, chunk by chunk in reverse. With D_W, D_M the
     adjoints of the chunk-end states and G_t = a_t D_M + b_t D_W:
         dM0 = P_U D_M + c D_W
         dW0 = P_L D_W + grad_W0 sum_t <dout_t, f_W0(q_t)> - sum_t VJP_g(G_t)
         abar_t = -<D_M, g_t>,  bbar_t = -<D_W, g_t>
         PUbar = <D_M, M0>,  PLbar = <D_W, W0>,  cbar = <D_W, M0>
-    then chunk_kernels_vjp gives the gate gradients."""
+    then chunk_kernels_vjp gives the gate gradients. For the chunk-averaged
+    variant every token's a_t is the mean of the per-token kernels, so each
+    per-token kernel receives the mean of abar (and of bbar) before the VJP."""
     q, k, v, lr, mom, decay, W0, M0, dout = map(_f64, (q, k, v, lr, mom, decay, W0, M0, dout))
     B, H, T = lr.shape
     d_k, d_v, S = _dims(kind, q, v, W0, d_h)
@@ -563,7 +589,7 @@ def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_e
            (("dq", q), ("dk", k), ("dv", v), ("dlr", lr), ("dmom", mom), ("ddecay", decay),
             ("dW0", W0), ("dM0", M0))}
     _, _, _, starts = closed_fwd(kind, q, k, v, lr, mom, decay, W0, M0, C, d_h, loss,
-                                 return_starts=True, heads=heads)
+                                 return_starts=True, heads=heads, coef=coef)
     hl = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     for (b, h) in hl:
         DW = dW_end[b, h].copy()
@@ -573,7 +599,7 @@ def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_e
             Ws, Ms = starts[ci, b, h, 0], starts[ci, b, h, 1]
             P = unpack(kind, Ws, d_k, d_v, d_h)
             eta, mu, lam = lr[b, h, t0:t1], mom[b, h, t0:t1], decay[b, h, t0:t1]
-            a, bb, P_U, P_L, c = chunk_kernels(eta, mu, lam)
+            a, bb, P_U, P_L, c = _kernels(coef)(eta, mu, lam)
             abar = np.zeros(t1 - t0)
             bbar = np.zeros(t1 - t0)
             Pbar = P_L * DW
@@ -589,6 +615,9 @@ def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_e
                 Pb, qb = fast_apply_vjp(kind, P, q[b, h, t], dout[b, h, t])
                 Pbar += pack(kind, Pb)
                 res["dq"][b, h, t] = qb
+            if coef == COEF_CHUNK_MEAN:
+                abar = np.full_like(abar, abar.mean())
+                bbar = np.full_like(bbar, bbar.mean())
             PUbar = np.dot(DM, Ms)
             PLbar = np.dot(DW, Ws)
             cbar = np.dot(DW, Ms)

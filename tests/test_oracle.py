@@ -408,3 +408,91 @@ def test_bf16_rounding_ties_to_even():
     x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5], np.float32)
     r = gen.round_to_bf16(x)
     np.testing.assert_array_equal(r, np.array([1.0, 1.0, 1.0 + 2 ** -6, 1.0, -2.5], np.float32))
+
+
+# ------------------------------------------------------------------ chunk-averaged variant
+# atlas.scime.ai summary, "Surprising findings": the per-token factors collapsed to
+# chunk scalars (read as the chunk means of a_t and b_t; P_U, P_L, c unchanged).
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+def test_chunk_mean_chunk_size_one_is_tokenwise(kind):
+    """With one token per chunk the mean is the token's own factor: the variant is
+    token-wise TTT (the independent third loop)."""
+    w, x = small_case(kind, T=9, C=1, seed=21)
+    o1, W1, M1 = O.closed_fwd(*fwd_args(w, x), d_h=w.d_h, coef=O.COEF_CHUNK_MEAN)
+    o2, W2, M2 = O.tokenwise_fwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"],
+                                 x["W0"], x["M0"], d_h=w.d_h)
+    assert O.rel_fro(o1, o2) < 1e-13 and O.rel_fro(W1, W2) < 1e-13 and O.rel_fro(M1, M2) < 1e-13
+
+
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+def test_chunk_mean_no_momentum_unit_decay(kind):
+    """mu = 0, lam = 1: a_t = eta_t [t = C] and b_t = eta_t, so the variant is the
+    plain chunk update with the chunk's mean learning rate,
+        W <- W - mean(eta) sum_t g_t(W),   M <- -(eta_C / C) sum_t g_t(W),
+    written here as its own loop over chunks."""
+    w, x = small_case(kind, T=12, C=4, H=1, seed=23)
+    x["mom"][:] = 0.0
+    x["decay"][:] = 1.0
+    _, W_end, M_end = O.closed_fwd(*fwd_args(w, x), d_h=w.d_h, coef=O.COEF_CHUNK_MEAN)
+    W = x["W0"][0, 0].astype(np.float64)
+    M = x["M0"][0, 0].astype(np.float64)
+    for t0 in range(0, 12, 4):
+        P = O.unpack(kind, W, w.d_k, w.d_v, w.d_h)
+        gsum = sum(O.pack(kind, O.loss_grad(kind, O.LOSS_MSE, P, x["k"][0, 0, t].astype(np.float64),
+                                            x["v"][0, 0, t].astype(np.float64)))
+                   for t in range(t0, t0 + 4))
+        eta = x["lr"][0, 0, t0:t0 + 4].astype(np.float64)
+        W = W - eta.mean() * gsum
+        M = -(eta[-1] / 4) * gsum
+    np.testing.assert_allclose(W_end[0, 0], W, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(M_end[0, 0], M, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("mu,lam", [(0.9, 0.97), (0.5, 0.8), (0.95, 0.95), (0.0, 0.9)])
+def test_chunk_mean_constant_gates_geometric(mu, lam):
+    """Constant gates: mean_t eta mu^(C-t) = eta (1 - mu^C) / (C (1 - mu)) and
+    mean_t eta R_t = eta / C * sum_{j=1..C} (lam^j - mu^j) / (lam - mu) (or
+    eta / C * sum_j j lam^(j-1) when mu = lam)."""
+    C, eta = 9, 0.3
+    a, b, PU, PL, c = O.chunk_mean_kernels(np.full(C, eta), np.full(C, mu), np.full(C, lam))
+    abar = eta * (1 - mu ** C) / (C * (1 - mu))
+    j = np.arange(1, C + 1)
+    if mu != lam:
+        bbar = eta / C * np.sum((lam ** j - mu ** j) / (lam - mu))
+    else:
+        bbar = eta / C * np.sum(j * lam ** (j - 1))
+    np.testing.assert_allclose(a, abar, rtol=1e-13)
+    np.testing.assert_allclose(b, bbar, rtol=1e-13)
+    assert abs(PU - mu ** C) <= 1e-15 and abs(PL - lam ** C) <= 1e-15
+
+
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+def test_chunk_mean_bwd_matches_fd(kind):
+    """closed_bwd of the variant against central finite differences of closed_fwd
+    of the variant, every input group, ragged last chunk."""
+    w, x = small_case(kind, B=1, H=1, T=7, C=3, d_k=4, d_v=4, d_h=6, seed=27)
+    x = {n: np.asarray(a, np.float64) for n, a in x.items()}
+    rng = np.random.default_rng(4)
+    S = w.state_elems
+    dW = rng.standard_normal((1, 1, S))
+    dM = rng.standard_normal((1, 1, S))
+    args = lambda y: (w.kind, y["q"], y["k"], y["v"], y["lr"], y["mom"], y["decay"], y["W0"],
+                      y["M0"], w.C)
+    g = O.closed_bwd(*args(x), x["dout"], dW, dM, d_h=w.d_h, coef=O.COEF_CHUNK_MEAN)
+
+    def L(y):
+        out, W_end, M_end = O.closed_fwd(*args(y), d_h=w.d_h, coef=O.COEF_CHUNK_MEAN)
+        return float(np.sum(out * x["dout"]) + np.sum(W_end * dW) + np.sum(M_end * dM))
+
+    for name, gname in NAMES:
+        d = rng.standard_normal(x[name].shape)
+        eps = 1e-6
+        yp, ym = dict(x), dict(x)
+        yp[name] = x[name] + eps * d
+        ym[name] = x[name] - eps * d
+        fd = (L(yp) - L(ym)) / (2 * eps)
+        an = float(np.sum(g[gname] * d))
+        assert abs(fd - an) <= 2e-7 * max(1.0, abs(fd)), (name, fd, an)
+    # and the variant really differs from the per-token kernels
+    g0 = O.closed_bwd(*args(x), x["dout"], dW, dM, d_h=w.d_h)
+    assert O.rel_fro(g["dlr"], g0["dlr"]) > 1e-3
