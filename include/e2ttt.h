@@ -72,9 +72,16 @@ typedef enum {
 typedef enum { E2TTT_LINEAR = 0, E2TTT_SWIGLU = 1 } e2ttt_fast_kind;
 typedef enum { E2TTT_F32 = 0, E2TTT_BF16 = 1 } e2ttt_dtype;
 typedef enum { E2TTT_LOSS_MSE = 0, E2TTT_LOSS_NEG_DOT = 1 } e2ttt_loss;
+/* Momentum / weight kernels. PER_TOKEN: a_t, b_t of every token (the method).
+ * CHUNK_MEAN: the chunk-averaged variant ("Rethinking Expressivity and
+ * Efficiency in Test-Time Training", atlas.scime.ai summary, "Surprising
+ * findings": per-token factors collapsed to chunk scalars), every token of a
+ * chunk carrying the chunk means of a_t and b_t; the chunk scalars U(1,n),
+ * L(1,n), c are unchanged. Forward and backward honour it. */
+typedef enum { E2TTT_COEF_PER_TOKEN = 0, E2TTT_COEF_CHUNK_MEAN = 1 } e2ttt_coef;
 
-/* Problem description. kind/act/loss hold e2ttt_fast_kind / e2ttt_dtype /
- * e2ttt_loss values. d_h is ignored (may be 0) for E2TTT_LINEAR.
+/* Problem description. kind/act/loss/coef hold e2ttt_fast_kind / e2ttt_dtype /
+ * e2ttt_loss / e2ttt_coef values. d_h is ignored (may be 0) for E2TTT_LINEAR.
  * Limits: all sizes >= 1; B*H*T*max(d_k,d_v,d_h) < 2^31; 1 <= C <= 1024. */
 typedef struct {
   int B, H, T, C;
@@ -82,6 +89,7 @@ typedef struct {
   int kind;
   int act;
   int loss;
+  int coef;
 } e2ttt_shape;
 
 /* Fast-weight state size S per (b, h): d_v*d_k (linear) or 2*d_h*d_k + d_v*d_h

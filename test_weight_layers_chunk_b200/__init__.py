@@ -28,12 +28,13 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "e2ttt.h")
 LINEAR, SWIGLU = 0, 1
 F32, BF16 = 0, 1
 LOSS_MSE, LOSS_NEG_DOT = 0, 1
+COEF_PER_TOKEN, COEF_CHUNK_MEAN = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 
 
 class e2ttt_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss")]
+                ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss", "coef")]
 
 
 class E2TTTError(RuntimeError):
@@ -77,8 +78,9 @@ def header_functions() -> list[str]:
     return sorted(set(re.findall(r"\b(e2ttt_[a-z_]+)\s*\(", src)))
 
 
-def make_shape(B, H, T, C, d_k, d_v, d_h=0, kind=SWIGLU, act=BF16, loss=LOSS_MSE) -> e2ttt_shape:
-    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss)
+def make_shape(B, H, T, C, d_k, d_v, d_h=0, kind=SWIGLU, act=BF16, loss=LOSS_MSE,
+               coef=COEF_PER_TOKEN) -> e2ttt_shape:
+    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef)
 
 
 def _ptr(x):
@@ -193,11 +195,11 @@ def e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved_states, dout, dW_
 
 
 # ---------------------------------------------------------------- conveniences
-def _shape_of(q, v, lr, C, d_h, kind, loss):
+def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN):
     import torch
     B, H, T, d_k = q.shape
     act = BF16 if q.dtype == torch.bfloat16 else F32
-    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss)
+    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef)
 
 
 def workspace(shape, for_bwd=False, device="cuda"):
@@ -209,11 +211,11 @@ def workspace(shape, for_bwd=False, device="cuda"):
 
 
 def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGLU,
-                   loss=LOSS_MSE, save_states=False, ws=None, stream=None):
+                   loss=LOSS_MSE, coef=COEF_PER_TOKEN, save_states=False, ws=None, stream=None):
     """Allocate out / W_end / M_end (and saved_states) and run the forward.
     Returns (out, W_end, M_end, saved_states or None)."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef)
     nc = e2ttt_num_chunks(shape)
     out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     W_end = torch.empty_like(W0)
@@ -228,10 +230,10 @@ def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGL
 
 
 def chunk_scan_bwd(q, k, v, lr, mom, decay, saved_states, dout, dW_end=None, dM_end=None, *, C,
-                   d_h=0, kind=SWIGLU, loss=LOSS_MSE, ws=None, stream=None):
+                   d_h=0, kind=SWIGLU, loss=LOSS_MSE, coef=COEF_PER_TOKEN, ws=None, stream=None):
     """Allocate the gradients and run the backward. Returns a dict."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef)
     g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
              dlr=torch.empty_like(lr), dmom=torch.empty_like(mom), ddecay=torch.empty_like(decay),
              dW0=torch.empty(saved_states.shape[1:3] + saved_states.shape[-1:], dtype=torch.float32,

@@ -46,6 +46,7 @@ bool shape_ok(const e2ttt_shape* s, std::string* why) {
   if (s->kind != E2TTT_LINEAR && s->kind != E2TTT_SWIGLU) { *why = "unknown fast-weight kind"; return false; }
   if (s->act != E2TTT_F32 && s->act != E2TTT_BF16) { *why = "unknown activation dtype"; return false; }
   if (s->loss != E2TTT_LOSS_MSE && s->loss != E2TTT_LOSS_NEG_DOT) { *why = "unknown loss"; return false; }
+  if (s->coef != E2TTT_COEF_PER_TOKEN && s->coef != E2TTT_COEF_CHUNK_MEAN) { *why = "unknown coef"; return false; }
   if (s->kind == E2TTT_SWIGLU && s->d_h < 1) { *why = "SwiGLU needs d_h >= 1"; return false; }
   if (s->C > 1024) { *why = "chunk size C must be <= 1024"; return false; }
   long long BH = (long long)s->B * s->H;
@@ -68,6 +69,7 @@ Dims make_dims(const e2ttt_shape* s) {
   d.d_h = s->kind == E2TTT_SWIGLU ? s->d_h : 0;
   d.kind = s->kind;
   d.loss = s->loss;
+  d.coef = s->coef;
   d.S = s->kind == E2TTT_LINEAR ? (long long)s->d_v * s->d_k
                                 : 2LL * s->d_h * s->d_k + (long long)s->d_v * s->d_h;
   return d;
@@ -221,7 +223,7 @@ e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* s, const float* lr, const flo
   Range in[] = {{lr, g, "lr"}, {mom, g, "mom"}, {decay, g, "decay"}};
   Range out[] = {{a, g, "a"}, {b, g, "b"}, {scal, (size_t)3 * d.BH * d.NC * sizeof(float), "chunk_scalars"}};
   if (!check_overlaps(in, 3, out, 3, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
-  cudaError_t e = launch_chunk_coeffs(lr, mom, decay, a, b, scal, d.BH, d.T, d.C, d.NC,
+  cudaError_t e = launch_chunk_coeffs(lr, mom, decay, a, b, scal, d.BH, d.T, d.C, d.NC, d.coef,
                                       (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "chunk coefficient kernel");
   return E2TTT_OK;
@@ -263,7 +265,7 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   int* status = (int*)(w + L.status);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
   if (e != cudaSuccess) return cuda_fail(e, "status word reset");
-  e = launch_chunk_coeffs(lr, mom, decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, st);
+  e = launch_chunk_coeffs(lr, mom, decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, d.coef, st);
   if (e != cudaSuccess) return cuda_fail(e, "chunk coefficient kernel");
   if (tc) {
     e = tc_fwd(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal, W0, M0,

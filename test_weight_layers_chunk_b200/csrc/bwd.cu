@@ -606,7 +606,7 @@ cudaError_t bwd_run(const BwdArgs& A) {
   const size_t sbytes = (size_t)d.BH * d.S * sizeof(float);
   cudaError_t e = cudaMemsetAsync(w + L.status, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
-  e = launch_chunk_coeffs(A.lr, A.mom, A.decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, st);
+  e = launch_chunk_coeffs(A.lr, A.mom, A.decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, d.coef, st);
   if (e != cudaSuccess) return e;
   e = A.dW_end ? cudaMemcpyAsync(A.dW0, A.dW_end, sbytes, cudaMemcpyDeviceToDevice, st)
                : cudaMemsetAsync(A.dW0, 0, sbytes, st);
@@ -626,7 +626,7 @@ cudaError_t bwd_run(const BwdArgs& A) {
     if (e != cudaSuccess) return e;
   }
   return launch_chunk_coeffs_bwd(A.lr, A.mom, A.decay, c.abar, c.bbar, c.sbar, A.dlr, A.dmom,
-                                 A.ddecay, d.BH, d.T, d.C, d.NC, st);
+                                 A.ddecay, d.BH, d.T, d.C, d.NC, d.coef, st);
 }
 
 template cudaError_t bwd_run<float>(const BwdArgs&);

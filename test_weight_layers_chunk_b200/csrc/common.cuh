@@ -35,6 +35,7 @@ struct Dims {
   int T, C, NC;
   int d_k, d_v, d_h;
   int kind, loss;
+  int coef;    // 0: per-token kernels, 1: chunk means (the chunk-averaged variant)
   long long S; // state elements per head
 };
 

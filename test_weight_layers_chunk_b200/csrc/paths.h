@@ -7,14 +7,16 @@
 
 namespace e2ttt {
 
-// K1 (scan.cu): scalar kernels of every chunk, and their adjoint.
+// K1 (scan.cu): scalar kernels of every chunk, and their adjoint. coef = 1 gives
+// every token of a chunk the chunk means of a_t, b_t (and, in the adjoint, the
+// chunk means of abar, bbar).
 cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
-                                float* b, float* scal, int BH, int T, int C, int NC,
+                                float* b, float* scal, int BH, int T, int C, int NC, int coef,
                                 cudaStream_t st);
 cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const float* decay,
                                     const float* abar, const float* bbar, const float* scal_bar,
                                     float* deta, float* dmu, float* dlam, int BH, int T, int C,
-                                    int NC, cudaStream_t st);
+                                    int NC, int coef, cudaStream_t st);
 
 // fp32 CUDA-core forward (simt_fwd.cu).
 template <typename TA>

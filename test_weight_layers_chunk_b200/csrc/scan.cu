@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
                     const float* __restrict__ decay, float* __restrict__ a_out,
                     float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
-                    int NC) {
+                    int NC, int coef) {
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   if (wid >= BH * NC) return;  // warp-uniform
@@ -91,8 +91,11 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   // Reverse walk 1: momentum kernel a_t and the segment's ratio-sum map.
   float su = ls.su_excl, sl = ls.sl_excl;
   float Mseg = 1.f, Cseg = 0.f;
+  float asum = 0.f, bsum = 0.f;  // segment sums (chunk means for coef = 1)
   for (int t = s1 - 1; t >= s0; --t) {
-    a_out[base + t] = eta[t] * expf(su);
+    const float at = eta[t] * expf(su);
+    a_out[base + t] = at;
+    asum += at;
     float m = (t + 1 < n) ? mu[t + 1] : 0.f;
     Cseg = expf(sl) + m * Cseg;
     Mseg = m * Mseg;
@@ -118,10 +121,20 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   for (int t = s1 - 1; t >= s0; --t) {
     float m = (t + 1 < n) ? mu[t + 1] : 0.f;
     float r = expf(sl) + m * r_next;
-    b_out[base + t] = eta[t] * r;
+    const float bt = eta[t] * r;
+    b_out[base + t] = bt;
+    bsum += bt;
     r_next = r;
     if (t == 0) r1 = r;
     sl += logf(lam[t]);
+  }
+  if (coef) {  // the chunk-averaged variant: every token carries the chunk means
+    const float am = __shfl_sync(0xffffffffu, warp_suffix_sum(asum, lane), 0) / (float)n;
+    const float bm = __shfl_sync(0xffffffffu, warp_suffix_sum(bsum, lane), 0) / (float)n;
+    for (int t = s0; t < s1; ++t) {
+      a_out[base + t] = am;
+      b_out[base + t] = bm;
+    }
   }
   if (s0 == 0 && s1 > 0) {  // lane 0 holds token 1
     const size_t plane = (size_t)BH * NC;
@@ -146,7 +159,7 @@ __global__ void __launch_bounds__(kK1Threads)
 chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
                           const float* __restrict__ decay, float* __restrict__ a_out,
                           float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
-                          int NC) {
+                          int NC, int coef) {
   extern __shared__ float k1s[];
   float* s_eta = k1s;
   float* s_mu = k1s + C;
@@ -204,8 +217,11 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   su = su_excl;
   sl = sl_excl;
   float Mseg = 1.f, Cseg = 0.f;
+  float asum = 0.f, bsum = 0.f;  // segment sums (chunk means for coef = 1)
   for (int t = s1 - 1; t >= s0; --t) {
-    a_out[base + t] = s_eta[t] * expf(su);
+    const float at = s_eta[t] * expf(su);
+    a_out[base + t] = at;
+    asum += at;
     const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
     Cseg = expf(sl) + m * Cseg;
     Mseg = m * Mseg;
@@ -240,10 +256,31 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   for (int t = s1 - 1; t >= s0; --t) {
     const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
     const float r = expf(sl) + m * r_next;
-    b_out[base + t] = s_eta[t] * r;
+    const float bt = s_eta[t] * r;
+    b_out[base + t] = bt;
+    bsum += bt;
     r_next = r;
     if (t == 0) r1 = r;
     sl += s_llam[t];
+  }
+  if (coef) {  // the chunk-averaged variant: every token carries the chunk means
+    const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
+    __syncthreads();  // w_su / w_sl are free again
+    if (lane == 0) {
+      w_su[warp] = ai;
+      w_sl[warp] = bi;
+    }
+    __syncthreads();
+    float at = 0.f, bt = 0.f;
+    for (int w = kK1Warps - 1; w >= 0; --w) {
+      at += w_su[w];
+      bt += w_sl[w];
+    }
+    const float am = at / (float)n, bm = bt / (float)n;
+    for (int t = s0; t < s1; ++t) {
+      a_out[base + t] = am;
+      b_out[base + t] = bm;
+    }
   }
   if (s0 == 0 && s1 > 0) {  // the thread holding token 1
     const size_t plane = (size_t)BH * NC;
@@ -270,7 +307,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
                         const float* __restrict__ decay, const float* __restrict__ abar,
                         const float* __restrict__ bbar, const float* __restrict__ scal_bar,
                         float* __restrict__ deta, float* __restrict__ dmu,
-                        float* __restrict__ dlam, int BH, int T, int C, int NC) {
+                        float* __restrict__ dlam, int BH, int T, int C, int NC, int coef) {
   extern __shared__ float sm[];
   const int lane = threadIdx.x & 31;
   const int wl = threadIdx.x >> 5;
@@ -291,6 +328,20 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   int s0, s1;
   seg_bounds(n, lane, s0, s1);
   LogSums ls = chunk_log_sums(mu, lam, s0, s1, lane);
+  // The chunk-averaged variant: each token's per-token kernel receives the
+  // chunk mean of the adjoints of the (averaged) factors.
+  float abm = 0.f, bbm = 0.f;
+  if (coef) {
+    float sa = 0.f, sb = 0.f;
+    for (int t = s0; t < s1; ++t) {
+      sa += ab[t];
+      sb += bb[t];
+    }
+    abm = __shfl_sync(0xffffffffu, warp_suffix_sum(sa, lane), 0) / (float)n;
+    bbm = __shfl_sync(0xffffffffu, warp_suffix_sum(sb, lane), 0) / (float)n;
+  }
+  auto AB = [&](int t) { return coef ? abm : ab[t]; };
+  auto BB = [&](int t) { return coef ? bbm : bb[t]; };
 
   // Reverse walks: U(t+1,n), L(t+1,n), R_t into shared memory; deta.
   float su = ls.su_excl, sl = ls.sl_excl;
@@ -321,7 +372,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
     float m = (t + 1 < n) ? mu[t + 1] : 0.f;
     float r = sL[t] + m * r_next;
     sR[t] = r;
-    deta[base + t] = ab[t] * sU[t] + bb[t] * r;
+    deta[base + t] = AB(t) * sU[t] + BB(t) * r;
     r_next = r;
   }
 
@@ -330,7 +381,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float p = 1.f, q = 0.f, r = 1.f, u = 0.f, w = 0.f;
   for (int s = s0; s < s1; ++s) {
     float m_ = mu[s], l_ = lam[s];
-    float al = ab[s] * eta[s], be = bb[s] * eta[s];
+    float al = AB(s) * eta[s], be = BB(s) * eta[s];
     uX = m_ * uX + al;
     pX = m_ * pX;
     float q2 = m_ * p + l_ * q;
@@ -379,8 +430,8 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
     dmu[base + s] = sU[s] * X + sR[s] * Y;
     dlam[base + s] = sL[s] * V;
     float m_ = mu[s], l_ = lam[s];
-    X = m_ * X + ab[s] * eta[s];
-    float Yn = m_ * Y + bb[s] * eta[s];
+    X = m_ * X + AB(s) * eta[s];
+    float Yn = m_ * Y + BB(s) * eta[s];
     V = l_ * V + Yn;
     Y = Yn;
   }
@@ -389,7 +440,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
 }  // namespace
 
 cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
-                                float* b, float* scal, int BH, int T, int C, int NC,
+                                float* b, float* scal, int BH, int T, int C, int NC, int coef,
                                 cudaStream_t st) {
   E2TTT_TRACE("k1_chunk_coeffs", st);
   if (C <= kK1MaxC) {
@@ -400,20 +451,20 @@ cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* 
       if (e != cudaSuccess) return e;
     }
     chunk_coeffs_block_kernel<<<BH * NC, kK1Threads, smem, st>>>(lr, mom, decay, a, b, scal, BH, T,
-                                                                 C, NC);
+                                                                 C, NC, coef);
     return cudaGetLastError();
   }
   int warps = BH * NC;
   int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
   chunk_coeffs_kernel<<<blocks, kWarpsPerBlock * 32, 0, st>>>(lr, mom, decay, a, b, scal, BH, T,
-                                                               C, NC);
+                                                               C, NC, coef);
   return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const float* decay,
                                     const float* abar, const float* bbar, const float* scal_bar,
                                     float* deta, float* dmu, float* dlam, int BH, int T, int C,
-                                    int NC, cudaStream_t st) {
+                                    int NC, int coef, cudaStream_t st) {
   int warps = BH * NC;
   int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
   size_t smem = (size_t)kWarpsPerBlock * 3 * C * sizeof(float);
@@ -424,7 +475,7 @@ cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const flo
   }
   E2TTT_TRACE("k1_chunk_coeffs_bwd", st);
   chunk_coeffs_bwd_kernel<<<blocks, kWarpsPerBlock * 32, smem, st>>>(
-      lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC);
+      lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC, coef);
   return cudaGetLastError();
 }
 

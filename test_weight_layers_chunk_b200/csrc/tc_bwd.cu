@@ -1096,7 +1096,7 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   const size_t sbytes = (size_t)BH * d.S * sizeof(float);
   cudaError_t e = cudaMemsetAsync(B.status, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
-  e = launch_chunk_coeffs(A.lr, A.mom, A.decay, B.a, B.b, B.scal, BH, T, C, NC, st);
+  e = launch_chunk_coeffs(A.lr, A.mom, A.decay, B.a, B.b, B.scal, BH, T, C, NC, d.coef, st);
   if (e != cudaSuccess) return e;
   e = A.dW_end ? cudaMemcpyAsync(A.dW0, A.dW_end, sbytes, cudaMemcpyDeviceToDevice, st)
                : cudaMemsetAsync(A.dW0, 0, sbytes, st);
@@ -1259,7 +1259,7 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     if ((e = run_gemm<1, true, true, EpiDW>(dw, p, st)) != cudaSuccess) return e;
   }
   return launch_chunk_coeffs_bwd(A.lr, A.mom, A.decay, B.abar, B.bbar, B.sbar, A.dlr, A.dmom,
-                                 A.ddecay, BH, T, C, NC, st);
+                                 A.ddecay, BH, T, C, NC, d.coef, st);
 }
 
 }  // namespace e2ttt

@@ -41,7 +41,8 @@ def test_sizes(E):
     assert E.e2ttt_state_elems(lin) == 32 * 32
     assert E.e2ttt_num_chunks(E.make_shape(1, 1, 257, 64, 32, 32, 0, E.LINEAR, E.F32)) == 5
     for bad in (E.make_shape(0, 1, 8, 4, 4, 4, 4), E.make_shape(1, 1, 8, 2048, 4, 4, 4),
-                E.make_shape(1, 1, 8, 4, 4, 4, 0, E.SWIGLU), E.make_shape(1, 1, 8, 4, 4, 4, 4, 7)):
+                E.make_shape(1, 1, 8, 4, 4, 4, 0, E.SWIGLU), E.make_shape(1, 1, 8, 4, 4, 4, 4, 7),
+                E.make_shape(1, 1, 8, 4, 4, 4, 4, E.SWIGLU, coef=2)):
         assert E.e2ttt_state_elems(bad) == 0 and E.e2ttt_workspace_bytes(bad, 0) == 0
 
 
