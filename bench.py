@@ -335,19 +335,21 @@ def _timed(torch, stream, fn, steps):
 def measure_extras(E, torch, dev, stream, args):
     """The metric's other operating points, device-timed like the main line:
     forward at T = 16K (the 8x length-extrapolation layer), forward+backward at
-    T = 2K (the training workload), and the chunk-averaged variant's forward at
-    T = 2K, each with its own warm-up."""
+    T = 2K (the training workload), and the forward at T = 2K of the
+    chunk-averaged variant and of the no-momentum mode, each with its own
+    warm-up."""
     out = {}
     f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
-    for name, train, steps, coef in (("layer_1p3b_16k", False, args.extra_steps, 0),
-                                     ("train_1p3b_2k", True, max(2, args.extra_steps // 8), 0),
-                                     ("layer_1p3b_2k", False, args.extra_steps, 1)):
+    for name, train, steps, coef, nomom in (("layer_1p3b_16k", False, args.extra_steps, 0, 0),
+                                            ("train_1p3b_2k", True, max(2, args.extra_steps // 8), 0, 0),
+                                            ("layer_1p3b_2k", False, args.extra_steps, 1, 0),
+                                            ("layer_1p3b_2k", False, args.extra_steps, 0, 1)):
         w = gen.BY_NAME[name]
         x = gen.generate(w)
         q, k, v = f(x["q"], torch.bfloat16), f(x["k"], torch.bfloat16), f(x["v"], torch.bfloat16)
         lr, mom, decay, W0 = f(x["lr"]), f(x["mom"]), f(x["decay"]), f(x["W0"])
         shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss,
-                             coef=coef)
+                             coef=coef, momentum=nomom)
         nc = E.e2ttt_num_chunks(shape)
         outb, We, Me = torch.empty_like(v), torch.empty_like(W0), torch.empty_like(W0)
         saved = torch.empty((nc, w.B, w.H, 2, w.state_elems), device=dev) if train else None
@@ -357,8 +359,10 @@ def measure_extras(E, torch, dev, stream, args):
             g = [torch.empty_like(t) for t in (q, k, v, lr, mom, decay, W0, W0)]
             wsb = E.workspace(shape, True, dev)
 
+        mm, Mo = (None, None) if nomom else (mom, Me)
+
         def step(st=stream):
-            E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, None, outb, We, Me, saved, ws,
+            E.e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mm, decay, W0, None, outb, We, Mo, saved, ws,
                                    stream=st)
             if train:
                 E.e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved, dout, None, None, *g,
@@ -373,7 +377,8 @@ def measure_extras(E, torch, dev, stream, args):
         ms = _timed(torch, stream, run, steps)
         del graph
         flops = train_flops(w) if train else fwd_flops(w)
-        out[("fwd_bwd_" if train else "fwd_") + name + ("_chunk_mean" if coef else "")] = {
+        out[("fwd_bwd_" if train else "fwd_") + name + ("_chunk_mean" if coef else "") +
+            ("_no_momentum" if nomom else "")] = {
             "value": w.B * w.T / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
             "tflops": flops / (ms / 1e3) / 1e12, "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / measured_peaks()["bf16_tflops"]}
         del q, k, v, outb, We, Me, saved, ws

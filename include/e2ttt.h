@@ -79,9 +79,17 @@ typedef enum { E2TTT_LOSS_MSE = 0, E2TTT_LOSS_NEG_DOT = 1 } e2ttt_loss;
  * chunk carrying the chunk means of a_t and b_t; the chunk scalars U(1,n),
  * L(1,n), c are unchanged. Forward and backward honour it. */
 typedef enum { E2TTT_COEF_PER_TOKEN = 0, E2TTT_COEF_CHUNK_MEAN = 1 } e2ttt_coef;
+/* Momentum. E2TTT_NO_MOMENTUM runs the recurrence without momentum,
+ * W_t = lam_t W_{t-1} - eta_t g_t (mu = 0; the pages' repository names a
+ * no-momentum kernel builder): no momentum state exists, so mom, M0 and M_end
+ * must be NULL in the forward (saved states then hold zero M), and mom, dM_end,
+ * dmom and dM0 must be NULL in the backward. The forward moves only W through
+ * HBM (about half the state traffic). */
+typedef enum { E2TTT_MOMENTUM = 0, E2TTT_NO_MOMENTUM = 1 } e2ttt_momentum;
 
-/* Problem description. kind/act/loss/coef hold e2ttt_fast_kind / e2ttt_dtype /
- * e2ttt_loss / e2ttt_coef values. d_h is ignored (may be 0) for E2TTT_LINEAR.
+/* Problem description. kind/act/loss/coef/momentum hold e2ttt_fast_kind /
+ * e2ttt_dtype / e2ttt_loss / e2ttt_coef / e2ttt_momentum values. d_h is ignored
+ * (may be 0) for E2TTT_LINEAR.
  * Limits: all sizes >= 1; B*H*T*max(d_k,d_v,d_h) < 2^31; 1 <= C <= 1024. */
 typedef struct {
   int B, H, T, C;
@@ -90,6 +98,7 @@ typedef struct {
   int act;
   int loss;
   int coef;
+  int momentum;
 } e2ttt_shape;
 
 /* Fast-weight state size S per (b, h): d_v*d_k (linear) or 2*d_h*d_k + d_v*d_h
@@ -115,8 +124,9 @@ int e2ttt_fwd_uses_tensor_cores(const e2ttt_shape* shape);
  *   a[b,h,t] = eta_t U(t+1,C)                       momentum kernel
  *   b[b,h,t] = eta_t sum_{j=t..C} L(j+1,C) U(t+1,j) weight kernel
  *   chunk_scalars [3, B, H, n_chunks]: U(1,C), L(1,C), sum_j L(j+1,C) U(1,j)
- * t counts from the start of its chunk. Inputs lr/mom/decay [B,H,T] fp32;
- * outputs a, b [B,H,T] fp32. Device pointers; asynchronous on `stream`. */
+ * t counts from the start of its chunk. Inputs lr/mom/decay [B,H,T] fp32
+ * (mom NULL, i.e. mu = 0, in no-momentum mode); outputs a, b [B,H,T] fp32.
+ * Device pointers; asynchronous on `stream`. */
 e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* shape,
                                 const float* lr, const float* mom, const float* decay,
                                 float* a, float* b, float* chunk_scalars,
@@ -128,6 +138,8 @@ e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* shape,
  *            NULL, meaning a zero momentum state).
  *   Outputs: out (act dtype), W_end, M_end (fp32, the states after the last
  *            chunk), saved_states (may be NULL; needed by the backward).
+ *   No-momentum mode (shape->momentum = E2TTT_NO_MOMENTUM): mom, M0 and M_end
+ *   must be NULL; saved_states then hold W and a zero M for every chunk.
  *   Paths: bf16 activations with T % C == 0, C % 128 == 0, d_k % 64 == 0,
  *   d_v % 64 == 0 (and d_h % 128 == 0 for SwiGLU) run on the tcgen05 tensor
  *   cores (bf16 operands, fp32 accumulation and state); every other shape and
@@ -174,7 +186,8 @@ e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
  *   Inputs:  q, k, v, lr, mom, decay, saved_states (from the forward), dout
  *            (act dtype), dW_end, dM_end (fp32 [B,H,S]; may be NULL = zero).
  *   Outputs: dq, dk, dv (act dtype), dlr, dmom, ddecay (fp32 [B,H,T]),
- *            dW0, dM0 (fp32 [B,H,S]). */
+ *            dW0, dM0 (fp32 [B,H,S]).
+ *   No-momentum mode: mom, dM_end, dmom and dM0 must be NULL. */
 e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
                                   const void* q, const void* k, const void* v,
                                   const float* lr, const float* mom, const float* decay,

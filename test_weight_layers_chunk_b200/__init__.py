@@ -29,12 +29,13 @@ LINEAR, SWIGLU = 0, 1
 F32, BF16 = 0, 1
 LOSS_MSE, LOSS_NEG_DOT = 0, 1
 COEF_PER_TOKEN, COEF_CHUNK_MEAN = 0, 1
+MOMENTUM, NO_MOMENTUM = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 
 
 class e2ttt_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss", "coef")]
+                ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss", "coef", "momentum")]
 
 
 class E2TTTError(RuntimeError):
@@ -79,8 +80,8 @@ def header_functions() -> list[str]:
 
 
 def make_shape(B, H, T, C, d_k, d_v, d_h=0, kind=SWIGLU, act=BF16, loss=LOSS_MSE,
-               coef=COEF_PER_TOKEN) -> e2ttt_shape:
-    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef)
+               coef=COEF_PER_TOKEN, momentum=MOMENTUM) -> e2ttt_shape:
+    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef, momentum)
 
 
 def _ptr(x):
@@ -195,11 +196,11 @@ def e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved_states, dout, dW_
 
 
 # ---------------------------------------------------------------- conveniences
-def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN):
+def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN, momentum=MOMENTUM):
     import torch
     B, H, T, d_k = q.shape
     act = BF16 if q.dtype == torch.bfloat16 else F32
-    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef)
+    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef, momentum)
 
 
 def workspace(shape, for_bwd=False, device="cuda"):
@@ -211,15 +212,17 @@ def workspace(shape, for_bwd=False, device="cuda"):
 
 
 def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGLU,
-                   loss=LOSS_MSE, coef=COEF_PER_TOKEN, save_states=False, ws=None, stream=None):
+                   loss=LOSS_MSE, coef=COEF_PER_TOKEN, momentum=MOMENTUM, save_states=False,
+                   ws=None, stream=None):
     """Allocate out / W_end / M_end (and saved_states) and run the forward.
-    Returns (out, W_end, M_end, saved_states or None)."""
+    Returns (out, W_end, M_end, saved_states or None); M_end is None without
+    momentum (momentum=NO_MOMENTUM: pass mom=None, M0=None)."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum)
     nc = e2ttt_num_chunks(shape)
     out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     W_end = torch.empty_like(W0)
-    M_end = torch.empty_like(W0)
+    M_end = None if momentum == NO_MOMENTUM else torch.empty_like(W0)
     saved = (torch.empty((nc,) + tuple(W0.shape[:2]) + (2, W0.shape[-1]), dtype=torch.float32,
                          device=q.device) if save_states else None)
     if ws is None:
@@ -230,15 +233,19 @@ def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGL
 
 
 def chunk_scan_bwd(q, k, v, lr, mom, decay, saved_states, dout, dW_end=None, dM_end=None, *, C,
-                   d_h=0, kind=SWIGLU, loss=LOSS_MSE, coef=COEF_PER_TOKEN, ws=None, stream=None):
-    """Allocate the gradients and run the backward. Returns a dict."""
+                   d_h=0, kind=SWIGLU, loss=LOSS_MSE, coef=COEF_PER_TOKEN, momentum=MOMENTUM,
+                   ws=None, stream=None):
+    """Allocate the gradients and run the backward. Returns a dict (dmom and dM0
+    are None without momentum)."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum)
+    nomom = momentum == NO_MOMENTUM
     g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
-             dlr=torch.empty_like(lr), dmom=torch.empty_like(mom), ddecay=torch.empty_like(decay),
+             dlr=torch.empty_like(lr), dmom=None if nomom else torch.empty_like(mom),
+             ddecay=torch.empty_like(decay),
              dW0=torch.empty(saved_states.shape[1:3] + saved_states.shape[-1:], dtype=torch.float32,
                              device=q.device))
-    g["dM0"] = torch.empty_like(g["dW0"])
+    g["dM0"] = None if nomom else torch.empty_like(g["dW0"])
     if ws is None:
         ws = workspace(shape, True, q.device)
     e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved_states, dout, dW_end, dM_end,

@@ -47,6 +47,7 @@ bool shape_ok(const e2ttt_shape* s, std::string* why) {
   if (s->act != E2TTT_F32 && s->act != E2TTT_BF16) { *why = "unknown activation dtype"; return false; }
   if (s->loss != E2TTT_LOSS_MSE && s->loss != E2TTT_LOSS_NEG_DOT) { *why = "unknown loss"; return false; }
   if (s->coef != E2TTT_COEF_PER_TOKEN && s->coef != E2TTT_COEF_CHUNK_MEAN) { *why = "unknown coef"; return false; }
+  if (s->momentum != E2TTT_MOMENTUM && s->momentum != E2TTT_NO_MOMENTUM) { *why = "unknown momentum mode"; return false; }
   if (s->kind == E2TTT_SWIGLU && s->d_h < 1) { *why = "SwiGLU needs d_h >= 1"; return false; }
   if (s->C > 1024) { *why = "chunk size C must be <= 1024"; return false; }
   long long BH = (long long)s->B * s->H;
@@ -70,6 +71,7 @@ Dims make_dims(const e2ttt_shape* s) {
   d.kind = s->kind;
   d.loss = s->loss;
   d.coef = s->coef;
+  d.nomom = s->momentum == E2TTT_NO_MOMENTUM;
   d.S = s->kind == E2TTT_LINEAR ? (long long)s->d_v * s->d_k
                                 : 2LL * s->d_h * s->d_k + (long long)s->d_v * s->d_h;
   return d;
@@ -88,6 +90,7 @@ struct Bump {
 struct FwdWs {
   size_t status;                    // device status word (bounded waits)
   size_t a, b, scal, H, E, dH;      // fp32 CUDA-core path
+  size_t mscr;                      // no-momentum mode: the CUDA-core path's M_end scratch
   size_t tc;                        // tensor-core path scratch
   size_t total;
 };
@@ -114,8 +117,24 @@ FwdWs fwd_layout(const Dims& d, bool tc_shape) {
     size_t tend = align_up(region + tc_fwd_scratch_bytes(d));
     if (tend > end) end = tend;
   }
+  L.mscr = 0;
+  if (d.nomom) {
+    L.mscr = align_up(end);
+    end = L.mscr + (size_t)d.BH * d.S * sizeof(float);
+  }
   L.total = end;
   return L;
+}
+// The backward's workspace; in no-momentum mode followed by the scratch that
+// stands in for dM0 (the momentum adjoint, identically zero there).
+size_t bwd_total_bytes(const Dims& d, bool bf, size_t* dm_off) {
+  size_t n = bwd_workspace_bytes(d, bf);
+  *dm_off = 0;
+  if (d.nomom) {
+    *dm_off = align_up(n);
+    n = *dm_off + (size_t)d.BH * d.S * sizeof(float);
+  }
+  return n;
 }
 
 bool aligned16(std::initializer_list<const void*> ps) {
@@ -181,7 +200,8 @@ size_t e2ttt_workspace_bytes(const e2ttt_shape* s, int for_bwd) {
   std::string why;
   if (!shape_ok(s, &why)) return 0;
   Dims d = make_dims(s);
-  if (for_bwd) return bwd_workspace_bytes(d, s->act == E2TTT_BF16);
+  size_t dm_off;
+  if (for_bwd) return bwd_total_bytes(d, s->act == E2TTT_BF16, &dm_off);
   return fwd_layout(d, tc_fwd_supported(d, s->act == E2TTT_BF16)).total;
 }
 
@@ -216,9 +236,12 @@ e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* s, const float* lr, const flo
   g_last_error.clear();
   std::string why;
   if (!shape_ok(s, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
-  if (!lr || !mom || !decay || !a || !b || !scal)
+  if (!lr || !decay || !a || !b || !scal)
     return fail(E2TTT_ERR_INVALID_ARG, "e2ttt_chunk_coeffs: NULL pointer argument");
   Dims d = make_dims(s);
+  if (d.nomom != (mom == nullptr))
+    return fail(E2TTT_ERR_INVALID_ARG, d.nomom ? "no-momentum mode: mom must be NULL"
+                                               : "e2ttt_chunk_coeffs: mom is NULL");
   size_t g = (size_t)d.BH * d.T * sizeof(float);
   Range in[] = {{lr, g, "lr"}, {mom, g, "mom"}, {decay, g, "decay"}};
   Range out[] = {{a, g, "a"}, {b, g, "b"}, {scal, (size_t)3 * d.BH * d.NC * sizeof(float), "chunk_scalars"}};
@@ -237,9 +260,13 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   g_last_error.clear();
   std::string why;
   if (!shape_ok(s, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
-  if (!q || !k || !v || !lr || !mom || !decay || !W0 || !out || !W_end || !M_end)
+  if (!q || !k || !v || !lr || !decay || !W0 || !out || !W_end)
     return fail(E2TTT_ERR_INVALID_ARG, "e2ttt_chunk_scan_fwd: NULL pointer argument (only M0 and saved_states may be NULL)");
   Dims d = make_dims(s);
+  if (d.nomom && (mom || M0 || M_end))
+    return fail(E2TTT_ERR_INVALID_ARG, "no-momentum mode: mom, M0 and M_end must be NULL");
+  if (!d.nomom && (!mom || !M_end))
+    return fail(E2TTT_ERR_INVALID_ARG, "e2ttt_chunk_scan_fwd: mom and M_end are required");
   const bool bf = s->act == E2TTT_BF16;
   const bool tc_shape = tc_fwd_supported(d, bf);
   FwdWs L = fwd_layout(d, tc_shape);
@@ -267,6 +294,12 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   if (e != cudaSuccess) return cuda_fail(e, "status word reset");
   e = launch_chunk_coeffs(lr, mom, decay, ca, cb, scal, d.BH, d.T, d.C, d.NC, d.coef, st);
   if (e != cudaSuccess) return cuda_fail(e, "chunk coefficient kernel");
+  if (d.nomom && saved) {
+    // no momentum state: the saved M parts hold zeros (the backward reads them)
+    const size_t row = (size_t)d.S * sizeof(float);
+    e = cudaMemset2DAsync(saved + d.S, 2 * row, 0, row, (size_t)d.NC * d.BH, st);
+    if (e != cudaSuccess) return cuda_fail(e, "saved-state reset");
+  }
   if (tc) {
     e = tc_fwd(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal, W0, M0,
                W_end, M_end, saved, w + L.tc, status, st);
@@ -276,6 +309,7 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   float* H = (float*)(w + L.H);
   float* E = (float*)(w + L.E);
   float* dH = (float*)(w + L.dH);
+  if (d.nomom) M_end = (float*)(w + L.mscr);  // the CUDA-core path's momentum scratch
   if (bf)
     e = simt_fwd<bf16>(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal,
                        W0, M0, W_end, M_end, saved, H, E, dH, st);
@@ -295,12 +329,17 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* s, const void* q, const voi
   g_last_error.clear();
   std::string why;
   if (!shape_ok(s, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
-  if (!q || !k || !v || !lr || !mom || !decay || !saved || !dout || !dq || !dk || !dv || !dlr ||
-      !dmom || !ddecay || !dW0 || !dM0)
+  if (!q || !k || !v || !lr || !decay || !saved || !dout || !dq || !dk || !dv || !dlr ||
+      !ddecay || !dW0)
     return fail(E2TTT_ERR_INVALID_ARG, "e2ttt_chunk_scan_bwd: NULL pointer argument (only dW_end and dM_end may be NULL)");
   Dims d = make_dims(s);
+  if (d.nomom && (mom || dM_end || dmom || dM0))
+    return fail(E2TTT_ERR_INVALID_ARG, "no-momentum mode: mom, dM_end, dmom and dM0 must be NULL");
+  if (!d.nomom && (!mom || !dmom || !dM0))
+    return fail(E2TTT_ERR_INVALID_ARG, "e2ttt_chunk_scan_bwd: mom, dmom and dM0 are required");
   const bool bf = s->act == E2TTT_BF16;
-  size_t need = bwd_workspace_bytes(d, bf);
+  size_t dm_off = 0;
+  size_t need = bwd_total_bytes(d, bf, &dm_off);
   if (!ws) return fail(E2TTT_ERR_INVALID_ARG, "workspace is NULL (needs %zu bytes)", need);
   if (ws_bytes < need) return fail(E2TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   if (((uintptr_t)ws) & 255) return fail(E2TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
@@ -314,6 +353,7 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* s, const void* q, const voi
                   {dmom, ng, "dmom"}, {ddecay, ng, "ddecay"}, {dW0, ns, "dW0"}, {dM0, ns, "dM0"},
                   {ws, need, "workspace"}};
   if (!check_overlaps(in, 10, outr, 9, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
+  if (d.nomom) dM0 = (float*)((char*)ws + dm_off);  // zero momentum adjoint, kept internal
   BwdArgs A{d, q, k, v, lr, mom, decay, saved, dout, dW_end, dM_end, dq, dk, dv,
             dlr, dmom, ddecay, dW0, dM0, ws, (cudaStream_t)stream};
   cudaError_t e = bf ? bwd_run<bf16>(A) : bwd_run<float>(A);

@@ -36,6 +36,7 @@ struct Dims {
   int d_k, d_v, d_h;
   int kind, loss;
   int coef;    // 0: per-token kernels, 1: chunk means (the chunk-averaged variant)
+  int nomom;   // 1: no momentum (mu = 0, no M state)
   long long S; // state elements per head
 };
 

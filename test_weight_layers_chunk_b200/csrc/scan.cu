@@ -43,6 +43,9 @@ __device__ __forceinline__ float warp_suffix_sum(float x, int lane) {
   return x;
 }
 
+// Momentum gate of token t (mu == nullptr: no-momentum mode, mu = 0).
+__device__ __forceinline__ float mu_at(const float* mu, int t) { return mu ? mu[t] : 0.f; }
+
 // Per chunk: exclusive suffix log-sums at the end of this lane's segment and
 // the chunk totals (lane-uniform).
 struct LogSums {
@@ -54,7 +57,7 @@ __device__ __forceinline__ LogSums chunk_log_sums(const float* mu, const float* 
                                                   int lane) {
   float su = 0.f, sl = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
-    su += logf(mu[t]);
+    su += logf(mu_at(mu, t));
     sl += logf(lam[t]);
   }
   float su_inc = warp_suffix_sum(su, lane);
@@ -81,7 +84,7 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   const int n = min(C, T - t0);
   const size_t base = (size_t)bh * T + t0;
   const float* eta = lr + base;
-  const float* mu = mom + base;
+  const float* mu = mom ? mom + base : nullptr;
   const float* lam = decay + base;
   int s0, s1;
   seg_bounds(n, lane, s0, s1);
@@ -96,10 +99,10 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
     const float at = eta[t] * expf(su);
     a_out[base + t] = at;
     asum += at;
-    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
     Cseg = expf(sl) + m * Cseg;
     Mseg = m * Mseg;
-    su += logf(mu[t]);
+    su += logf(mu_at(mu, t));
     sl += logf(lam[t]);
   }
   float M = Mseg, Cc = Cseg;
@@ -119,7 +122,7 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   sl = ls.sl_excl;
   float r1 = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
-    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
     float r = expf(sl) + m * r_next;
     const float bt = eta[t] * r;
     b_out[base + t] = bt;
@@ -141,7 +144,7 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
     const size_t o = (size_t)bh * NC + ci;
     scal[o] = expf(ls.su_all);
     scal[plane + o] = expf(ls.sl_all);
-    scal[2 * plane + o] = mu[0] * r1;
+    scal[2 * plane + o] = mu_at(mu, 0) * r1;
   }
 }
 
@@ -172,7 +175,7 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   const int n = min(C, T - t0);
   const size_t base = (size_t)bh * T + t0;
   for (int t = tid; t < n; t += kK1Threads) {
-    const float mu = mom[base + t];
+    const float mu = mom ? mom[base + t] : 0.f;  // NULL: no-momentum mode
     s_eta[t] = lr[base + t];
     s_mu[t] = mu;
     s_lmu[t] = logf(mu);
@@ -321,7 +324,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   const int n = min(C, T - t0);
   const size_t base = (size_t)bh * T + t0;
   const float* eta = lr + base;
-  const float* mu = mom + base;
+  const float* mu = mom ? mom + base : nullptr;
   const float* lam = decay + base;
   const float* ab = abar + base;
   const float* bb = bbar + base;
@@ -347,13 +350,13 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float su = ls.su_excl, sl = ls.sl_excl;
   float Mseg = 1.f, Cseg = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
-    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
     float cl = expf(sl);
     sU[t] = expf(su);
     sL[t] = cl;
     Cseg = cl + m * Cseg;
     Mseg = m * Mseg;
-    su += logf(mu[t]);
+    su += logf(mu_at(mu, t));
     sl += logf(lam[t]);
   }
   float M = Mseg, Cc = Cseg;
@@ -369,7 +372,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float r_next = __shfl_down_sync(0xffffffffu, Cc, 1);
   if (lane == 31) r_next = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
-    float m = (t + 1 < n) ? mu[t + 1] : 0.f;
+    float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
     float r = sL[t] + m * r_next;
     sR[t] = r;
     deta[base + t] = AB(t) * sU[t] + BB(t) * r;
@@ -380,7 +383,7 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float pX = 1.f, uX = 0.f;
   float p = 1.f, q = 0.f, r = 1.f, u = 0.f, w = 0.f;
   for (int s = s0; s < s1; ++s) {
-    float m_ = mu[s], l_ = lam[s];
+    float m_ = mu_at(mu, s), l_ = lam[s];
     float al = AB(s) * eta[s], be = BB(s) * eta[s];
     uX = m_ * uX + al;
     pX = m_ * pX;
@@ -427,9 +430,9 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float Y = ep * cb + eu;
   float V = eq * cb + er * PLb + ew;
   for (int s = s0; s < s1; ++s) {
-    dmu[base + s] = sU[s] * X + sR[s] * Y;
+    if (dmu) dmu[base + s] = sU[s] * X + sR[s] * Y;  // NULL in no-momentum mode
     dlam[base + s] = sL[s] * V;
-    float m_ = mu[s], l_ = lam[s];
+    float m_ = mu_at(mu, s), l_ = lam[s];
     X = m_ * X + AB(s) * eta[s];
     float Yn = m_ * Y + BB(s) * eta[s];
     V = l_ * V + Yn;

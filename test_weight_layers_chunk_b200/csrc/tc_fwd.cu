@@ -43,6 +43,7 @@ struct FwdP {
   CUtensorMap mA, mSk, mOut, mV, mE, mEa, mEb, mdH;
   Dims d;
   int ci, t0, write_shadow;
+  int nomom;  // no momentum: no a-scaled operands, W-only aggregation epilogue
   int* status;
   const bf16 *q, *k, *v;
   bf16* out;
@@ -232,16 +233,18 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
     for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
     staging_free(lane);
     if (write_e) stage32(S, lane, y);
+    if (!p.nomom) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) vv[i] = at * y[i];
-    stage32(S + 2048, lane, vv);
+      for (int i = 0; i < 32; ++i) vv[i] = at * y[i];
+      stage32(S + 2048, lane, vv);
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) vv[i] = bt * y[i];
     stage32(S + 4096, lane, vv);
     staging_ready();
     if (lane == 0) {
       if (write_e) tc::tma_store_2d(&p.mE, S, col, yrow);
-      tc::tma_store_2d(&p.mEa, S + 2048, col, yrow);
+      if (!p.nomom) tc::tma_store_2d(&p.mEa, S + 2048, col, yrow);
       tc::tma_store_2d(&p.mEb, S + 4096, col, yrow);
       tc::bulk_commit();
     }
@@ -415,11 +418,94 @@ struct EpiG4 {
   }
 };
 
+// G4 without momentum: one accumulator dW = sum_t b_t g_t and the update
+// W_end = L(1,n) W0 - dW; the fp32 W (no M) moves through three 6 KB slots per
+// warp in one sequence of 32-column groups across the CTA's tiles, as in EpiG4.
+struct EpiG4W {
+  static constexpr int kSlot = 6144;  // W 4 KB | bf16 copy 2 KB
+  static constexpr int kSlots = 3;
+  static constexpr int kSmem = kSlots * kSlot;
+  static __device__ __forceinline__ void issue(const FwdP& p, const uint8_t* wsmem, uint64_t* wbar,
+                                               int q, int g, int cls, int z, int r0, int n0) {
+    const int sidx = q % kSlots;
+    uint8_t* slot = const_cast<uint8_t*>(wsmem) + sidx * kSlot;
+    tc::mbar_expect_tx(&wbar[sidx], 4096u);
+    tc::tma_load_3d(slot, &p.srcW[cls], &wbar[sidx], n0 + g * 32, r0, z);
+  }
+  template <int BN>
+  static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;
+    constexpr int kGroups = BN / 32;
+    static_assert(kGroups >= 2, "two groups ahead");
+    const size_t plane = (size_t)d.BH * d.NC;
+    const float PL = p.scal[plane + (size_t)c.z * d.NC + p.ci];
+    int sh_row;
+    if (c.cls == 0 && d.kind == 1) {
+      const int which = r0 / d.d_h, rr = r0 % d.d_h;
+      sh_row = c.z * 2 * d.d_h + w13_row(rr, which);
+    } else {
+      sh_row = c.z * d.d_v + r0;
+    }
+    const int q0 = c.iter * kGroups;
+    if (c.iter == 0 && lane == 0) {
+      issue(p, c.wsmem, c.wbar, q0, 0, c.cls, c.z, r0, c.n0);
+      issue(p, c.wsmem, c.wbar, q0 + 1, 1, c.cls, c.z, r0, c.n0);
+    }
+    __syncwarp();
+    for (int g = 0; g < kGroups; ++g) {
+      const int q = q0 + g, sidx = q % kSlots;
+      uint8_t* slot = c.wsmem + sidx * kSlot;
+      float dW[32];
+      ld1(c, 0, g * 32, dW);
+      const bool ok = tc::mbar_wait(&c.wbar[sidx], c.uses[sidx] & 1u);
+      c.uses[sidx] += 1;
+      if (!ok) {
+        if (lane == 0) atomicExch(p.status, tc2::kErrEpilogue);
+        return;
+      }
+      uint8_t* wrow = slot + lane * 128;
+      uint8_t* srow = slot + 4096 + lane * 64;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int off = (k ^ (lane & 7)) << 4;
+        const float4 w = *reinterpret_cast<const float4*>(wrow + off);
+        float4 wn;
+        wn.x = PL * w.x - dW[4 * k + 0];
+        wn.y = PL * w.y - dW[4 * k + 1];
+        wn.z = PL * w.z - dW[4 * k + 2];
+        wn.w = PL * w.w - dW[4 * k + 3];
+        *reinterpret_cast<float4*>(wrow + off) = wn;
+        *reinterpret_cast<uint2*>(srow + ((((k >> 1) ^ ((lane >> 1) & 3)) << 4) | ((k & 1) << 3))) =
+            make_uint2(pack2(wn.x, wn.y), pack2(wn.z, wn.w));
+      }
+      tc::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tc::tma_store_3d(&p.dstW[c.cls], slot, c.n0 + g * 32, r0, c.z);
+        if (p.write_shadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 4096, c.n0 + g * 32, sh_row);
+        tc::bulk_commit();
+        tc::bulk_wait_read<1>();  // the slot of group q - 1 is free for group q + 2
+        const int gn = g + 2;
+        if (gn < kGroups) {
+          issue(p, c.wsmem, c.wbar, q + 2, gn, c.cls, c.z, r0, c.n0);
+        } else if (c.nxt_valid) {
+          issue(p, c.wsmem, c.wbar, q + 2, gn - kGroups, c.nxt_cls, c.nxt_z,
+                c.nxt_m0 + c.quad * 32, c.nxt_n0);
+        }
+      }
+      __syncwarp();
+    }
+  }
+};
+
 template <class Epi> struct EpiName;
 template <> struct EpiName<EpiG1> { static constexpr const char* v = "tc_g1_h_act"; };
 template <> struct EpiName<EpiG2> { static constexpr const char* v = "tc_g2_y_out_e"; };
 template <> struct EpiName<EpiG3> { static constexpr const char* v = "tc_g3_da_dh"; };
 template <> struct EpiName<EpiG4> { static constexpr const char* v = "tc_g4_aggregate_state"; };
+template <> struct EpiName<EpiG4W> { static constexpr const char* v = "tc_g4_aggregate_w"; };
 template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 
 // ---------------------------------------------------------------- prep kernel
@@ -477,7 +563,7 @@ __global__ void scale_keys_kernel(const bf16* __restrict__ k, const float* __res
       oa[i] = pack2(a * f.x, a * f.y);
       ob[i] = pack2(b * f.x, b * f.y);
     }
-    reinterpret_cast<uint4*>(Ka)[e8] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+    if (Ka) reinterpret_cast<uint4*>(Ka)[e8] = make_uint4(oa[0], oa[1], oa[2], oa[3]);  // NULL: no momentum
     reinterpret_cast<uint4*>(Kb)[e8] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
   }
 }
@@ -619,6 +705,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   p.q = q; p.k = k; p.v = v; p.out = out;
   p.ca = ca; p.cb = cb; p.scal = scal;
   p.status = status;
+  p.nomom = d.nomom;
   p.Wsh13 = s.Wsh13; p.W2sh = s.W2sh;
   p.A = s.A; p.Sk = s.Sk; p.E = s.E; p.Ea = s.Ea; p.Eb = s.Eb; p.dH = s.dH; p.Ka = s.Ka;
   p.Kb = s.Kb;
@@ -634,7 +721,8 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   }
   if (d.kind == 1) {
     E2TTT_TRACE("tc_scale_keys", st);
-    scale_keys_kernel<<<4 * num_sms(), 256, 0, st>>>(k, ca, cb, s.Ka, s.Kb, (long long)BH * T, dk);
+    scale_keys_kernel<<<4 * num_sms(), 256, 0, st>>>(k, ca, cb, d.nomom ? nullptr : s.Ka, s.Kb,
+                                                     (long long)BH * T, dk);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -693,6 +781,26 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     g4.n_cls = 1;
     g4.cls[0] = tc2::Class{dv / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, kModeA2B1};
   }
+  // Without momentum: one accumulator (the b-weighted aggregation), W only.
+  tc2::Job g4w{};
+  g4w.heads = BH;
+  g4w.status = status;
+  if (d.nomom) {
+    if (d.kind == 1) {
+      ok &= make_map(&g4w.maps[0].op0, s.dH, (uint64_t)BH * C, 2 * dh, 64);
+      ok &= make_map(&g4w.maps[0].op2, s.Kb, (uint64_t)BH * T, dk, 64);
+      ok &= make_map(&g4w.maps[1].op0, s.Eb, (uint64_t)BH * C, dv, 64);
+      ok &= make_map(&g4w.maps[1].op2, s.A, (uint64_t)BH * 2 * C, dh, 64);
+      g4w.n_cls = 2;
+      g4w.cls[0] = tc2::Class{2 * dh / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, 0};
+      g4w.cls[1] = tc2::Class{dv / 128, dh / 128, C / 64, {C, 0, 0}, {2 * C, C, 0}, 0};
+    } else {
+      ok &= make_map(&g4w.maps[0].op0, s.Eb, (uint64_t)BH * C, dv, 64);
+      ok &= make_map(&g4w.maps[0].op2, k, (uint64_t)BH * T, dk, 64);
+      g4w.n_cls = 1;
+      g4w.cls[0] = tc2::Class{dv / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, 0};
+    }
+  }
   // 32 x 32 tiles of the epilogues (bf16, 64B swizzle)
   ok &= make_map_box32(&p.mOut, out, (uint64_t)BH * T, dv);
   ok &= make_map_box32(&p.mV, v, (uint64_t)BH * T, dv);
@@ -720,7 +828,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
         ok &= make_state_map(&p.srcW[c], p.src.W + off, rows, cols, BH, p.src.stride);
         if (p.src.M) ok &= make_state_map(&p.srcM[c], p.src.M + off, rows, cols, BH, p.src.stride);
         ok &= make_state_map(&p.dstW[c], p.dst.W + off, rows, cols, BH, p.dst.stride);
-        ok &= make_state_map(&p.dstM[c], p.dst.M + off, rows, cols, BH, p.dst.stride);
+        if (p.dst.M) ok &= make_state_map(&p.dstM[c], p.dst.M + off, rows, cols, BH, p.dst.stride);
       }
       if (ci == 0) {
         ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * (d.kind == 1 ? 2 * dh : dv), dk);
@@ -730,14 +838,21 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     }
     g1.cls[0].a.y_base = g1.cls[1].a.y_base = ci * C;  // query / key rows of this chunk
     g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
+    g4w.cls[0].b.y_base = ci * C;
     if (d.kind == 1) {
       e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
       if (e == cudaSuccess) e = launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
       if (e == cudaSuccess) e = launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st);
-      if (e == cudaSuccess) e = launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
+      if (e == cudaSuccess) {
+        e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)
+                    : launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
+      }
     } else {
       e = launch<128, 1, false, false, 4, EpiG1Lin, kEpiWarps, EpiG1Lin::kSmem>(g1, p, st);
-      if (e == cudaSuccess) e = launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
+      if (e == cudaSuccess) {
+        e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)
+                    : launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
+      }
     }
     if (e != cudaSuccess) return e;
   }

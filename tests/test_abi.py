@@ -99,3 +99,33 @@ def test_coeffs_rejects_bad_arguments(E):
     assert E.e2ttt_chunk_coeffs(s, None, FAKE, FAKE, FAKE, FAKE, FAKE, raw=True) == E.ERR_INVALID_ARG
     assert E.e2ttt_chunk_coeffs(s, FAKE, FAKE + 4096, FAKE + 8192, FAKE, FAKE + (1 << 20),
                                 FAKE + (1 << 21), raw=True) == E.ERR_INVALID_ARG  # a aliases lr
+
+
+def test_no_momentum_pointer_rules(E):
+    """No-momentum mode (E2TTT_NO_MOMENTUM): mom, M0, M_end (forward) and mom, dM_end,
+    dmom, dM0 (backward) must be NULL; with momentum, mom and M_end are required.
+    All checks run on the host before any CUDA call."""
+    nm = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32, momentum=E.NO_MOMENTUM)
+    ws = E.e2ttt_workspace_bytes(nm, 0)
+    assert ws > E.e2ttt_workspace_bytes(E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32), 0)
+    for over in (dict(), dict(M0=None), dict(M0=None, M_end=None)):     # mom given
+        assert _fwd(E, nm, workspace_bytes=ws, **over) == E.ERR_INVALID_ARG, over
+        assert "no-momentum" in E.e2ttt_last_error()
+    s = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32)
+    assert _fwd(E, s, mom=None) == E.ERR_INVALID_ARG
+    assert _fwd(E, s, M_end=None) == E.ERR_INVALID_ARG
+    n = 1 << 30
+    args = dict(q=FAKE, k=FAKE + n, v=FAKE + 2 * n, lr=FAKE + 3 * n, mom=None,
+                decay=FAKE + 5 * n, saved_states=FAKE + 6 * n, dout=FAKE + 7 * n, dW_end=None,
+                dM_end=None, dq=FAKE + 8 * n, dk=FAKE + 9 * n, dv=FAKE + 10 * n, dlr=FAKE + 11 * n,
+                dmom=None, ddecay=FAKE + 13 * n, dW0=FAKE + 14 * n, dM0=None,
+                workspace=FAKE + 16 * n, workspace_bytes=E.e2ttt_workspace_bytes(nm, 1))
+    for over in (dict(mom=FAKE + 4 * n), dict(dmom=FAKE + 12 * n), dict(dM0=FAKE + 15 * n),
+                 dict(dM_end=FAKE + 15 * n)):
+        a = dict(args)
+        a.update(over)
+        assert E.e2ttt_chunk_scan_bwd(nm, raw=True, stream=None, **a) == E.ERR_INVALID_ARG, over
+    assert E.e2ttt_chunk_coeffs(nm, FAKE, FAKE + n, FAKE + 2 * n, FAKE + 3 * n, FAKE + 4 * n,
+                                FAKE + 5 * n, raw=True) == E.ERR_INVALID_ARG   # mom given
+    bad = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32, momentum=3)
+    assert E.e2ttt_state_elems(bad) == 0
