@@ -18,7 +18,8 @@ Efficiency in Test-Time Training", abstract and "Key results"):
     train_1p3b_2k    = layer_1p3b_2k, plus an upstream gradient dOut ~ N(0,1)
 
 Draw order (one numpy PCG64 generator seeded with the workload index):
-q, k, v, lr, mom, decay, W0 (W1, W3, W2 for SwiGLU; W for linear), M0, dout.
+q, k, v, lr, mom, decay, W0 (W1, W3, W2 for SwiGLU; W1, W2 for the GELU MLP; W
+for linear), M0, dout.
 q and k are N(0,1) then scaled to unit L2 norm per token and head; v ~ N(0,1).
 Fast-weight matrices are N(0, 1/fan_in). M0 is zero unless ``m0_scale`` > 0, in
 which case it is N(0, m0_scale^2 / fan_in) (tests use this to exercise the M0
@@ -32,6 +33,7 @@ import numpy as np
 
 LINEAR = 0
 SWIGLU = 1
+GELU = 2      # two-matrix GELU MLP fast weight W2 gelu(W1 x)
 F32 = 0
 BF16 = 1
 LOSS_MSE = 0
@@ -69,6 +71,8 @@ class Workload:
     def state_elems(self) -> int:
         if self.kind == LINEAR:
             return self.d_v * self.d_k
+        if self.kind == GELU:
+            return self.d_h * self.d_k + self.d_v * self.d_h
         return 2 * self.d_h * self.d_k + self.d_v * self.d_h
 
     def replace(self, **kw) -> "Workload":
@@ -151,6 +155,12 @@ def generate(w: Workload, m0_scale: float = 0.0, seed: int | None = None,
         W = rng.standard_normal((B, H, w.d_v, w.d_k)) / np.sqrt(w.d_k)
         W0 = W.reshape(B, H, -1)
         fan = np.full(W0.shape[-1], float(w.d_k))
+    elif w.kind == GELU:
+        W1 = rng.standard_normal((B, H, w.d_h, w.d_k)) / np.sqrt(w.d_k)
+        W2 = rng.standard_normal((B, H, w.d_v, w.d_h)) / np.sqrt(w.d_h)
+        W0 = np.concatenate([W1.reshape(B, H, -1), W2.reshape(B, H, -1)], axis=-1)
+        fan = np.concatenate([np.full(w.d_h * w.d_k, float(w.d_k)),
+                              np.full(w.d_v * w.d_h, float(w.d_h))])
     else:
         W1 = rng.standard_normal((B, H, w.d_h, w.d_k)) / np.sqrt(w.d_k)
         W3 = rng.standard_normal((B, H, w.d_h, w.d_k)) / np.sqrt(w.d_k)

@@ -19,7 +19,10 @@ equations. What they fix:
 Readings the pages leave open (all written out here):
   * recurrence  M_t = mu_t M_{t-1} - eta_t g_t ,  W_t = lam_t W_{t-1} + M_t ;
   * loss  l(W; k, v) = 1/2 |f_W(k) - v|^2  (or -<f_W(k), v> for the dot loss);
-  * fast weight  f(x) = W x  (linear)  or  W2 (silu(W1 x) * (W3 x))  (SwiGLU);
+  * fast weight  f(x) = W x  (linear),  W2 (silu(W1 x) * (W3 x))  (SwiGLU), or
+    W2 gelu(W1 x)  (the MLP variant: atlas "Key results" names E2-TTT_MLP and
+    the codewithpapers JSON a gelu_derivative function; read as the exact GELU
+    z Phi(z) of the standard normal CDF, no biases);
   * out_t = f_{W_chunk_start}(q_t); gates are values (not logits); chunk i holds
     tokens [iC, (i+1)C), the last chunk may be short.
 
@@ -40,15 +43,18 @@ Functions, and what each follows:
                  chunk means of a_t and b_t; closed_fwd / closed_bwd take it
                  with coef=COEF_CHUNK_MEAN.
 State layout per (b, h): linear W [d_v, d_k]; SwiGLU [W1 (d_h x d_k) | W3
-(d_h x d_k) | W2 (d_v x d_h)], each row-major, concatenated.
+(d_h x d_k) | W2 (d_v x d_h)]; GELU MLP [W1 (d_h x d_k) | W2 (d_v x d_h)]; each
+row-major, concatenated.
 """
 from __future__ import annotations
 
 import math
 import numpy as np
+from scipy.special import erf
 
 LINEAR = 0
 SWIGLU = 1
+GELU = 2               # the two-matrix GELU MLP fast weight (E2-TTT_MLP)
 LOSS_MSE = 0
 LOSS_NEG_DOT = 1
 COEF_PER_TOKEN = 0     # per-token momentum / weight kernels (the method)
@@ -59,6 +65,8 @@ COEF_CHUNK_MEAN = 1    # the chunk-averaged variant
 def state_elems(kind, d_k, d_v, d_h):
     if kind == LINEAR:
         return d_v * d_k
+    if kind == GELU:
+        return d_h * d_k + d_v * d_h
     return 2 * d_h * d_k + d_v * d_h
 
 
@@ -67,6 +75,8 @@ def unpack(kind, s, d_k, d_v, d_h):
     if kind == LINEAR:
         return {"W": s.reshape(d_v, d_k)}
     n1 = d_h * d_k
+    if kind == GELU:
+        return {"W1": s[:n1].reshape(d_h, d_k), "W2": s[n1:].reshape(d_v, d_h)}
     return {"W1": s[:n1].reshape(d_h, d_k),
             "W3": s[n1:2 * n1].reshape(d_h, d_k),
             "W2": s[2 * n1:].reshape(d_v, d_h)}
@@ -75,6 +85,8 @@ def unpack(kind, s, d_k, d_v, d_h):
 def pack(kind, P):
     if kind == LINEAR:
         return P["W"].reshape(-1).copy()
+    if kind == GELU:
+        return np.concatenate([P["W1"].reshape(-1), P["W2"].reshape(-1)])
     return np.concatenate([P["W1"].reshape(-1), P["W3"].reshape(-1), P["W2"].reshape(-1)])
 
 
@@ -99,11 +111,37 @@ def d2silu(z):
     return s * (1.0 - s) * (2.0 + z * (1.0 - 2.0 * s))
 
 
+def Phi(z):
+    """Standard normal CDF."""
+    return 0.5 * (1.0 + erf(z / math.sqrt(2.0)))
+
+
+def phi(z):
+    """Standard normal density."""
+    return np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+
+
+def gelu(z):
+    return z * Phi(z)
+
+
+def dgelu(z):
+    """d/dz [z Phi(z)] = Phi(z) + z phi(z)."""
+    return Phi(z) + z * phi(z)
+
+
+def d2gelu(z):
+    """d^2/dz^2 [z Phi(z)] = 2 phi(z) + z phi'(z) = phi(z) (2 - z^2)."""
+    return phi(z) * (2.0 - z * z)
+
+
 # --------------------------------------------------------------------------- fast weight
 def fast_apply(kind, P, x):
     """f_W(x) for one token x [d_k] -> [d_v]."""
     if kind == LINEAR:
         return P["W"] @ x
+    if kind == GELU:
+        return P["W2"] @ gelu(P["W1"] @ x)
     h1 = P["W1"] @ x
     h3 = P["W3"] @ x
     return P["W2"] @ (silu(h1) * h3)
@@ -122,6 +160,13 @@ def loss_grad(kind, loss, P, k, v):
         y = P["W"] @ k
         e = (y - v) if loss == LOSS_MSE else -v
         return {"W": np.outer(e, k)}
+    if kind == GELU:
+        h = P["W1"] @ k
+        u = gelu(h)
+        y = P["W2"] @ u
+        e = (y - v) if loss == LOSS_MSE else -v
+        dh = (P["W2"].T @ e) * dgelu(h)
+        return {"W1": np.outer(dh, k), "W2": np.outer(e, u)}
     h1 = P["W1"] @ k
     h3 = P["W3"] @ k
     s = silu(h1)
@@ -150,6 +195,38 @@ def loss_grad_vjp(kind, loss, P, k, v, gbar):
             Wbar += np.outer(ebar, k)  # y = W k
             kbar = kbar + W.T @ ebar
         return {"W": Wbar}, kbar, vbar
+    if kind == GELU:
+        W1, W2 = P["W1"], P["W2"]
+        h = W1 @ k
+        u = gelu(h)
+        gp = dgelu(h)
+        y = W2 @ u
+        e = (y - v) if loss == LOSS_MSE else -v
+        du = W2.T @ e
+        dh = du * gp
+        G1, G2 = gbar["W1"], gbar["W2"]
+        W2b = np.zeros_like(W2)
+        # gW1 = dh k^T
+        dhb = G1 @ k
+        kbar = G1.T @ dh
+        # dh = du * gelu'(h)
+        dub = dhb * gp
+        hb = dhb * du * d2gelu(h)
+        # du = W2^T e
+        W2b += np.outer(e, dub)
+        eb = W2 @ dub
+        # gW2 = e u^T
+        eb = eb + G2 @ u
+        ub = G2.T @ e
+        # e = y - v   (dot loss: e = -v)
+        vbar = -eb
+        if loss == LOSS_MSE:
+            W2b += np.outer(eb, u)       # y = W2 u
+            ub = ub + W2.T @ eb
+        # u = gelu(h) ; h = W1 k
+        hb = hb + ub * gp
+        kbar = kbar + W1.T @ hb
+        return {"W1": np.outer(hb, k), "W2": W2b}, kbar, vbar
     W1, W3, W2 = P["W1"], P["W3"], P["W2"]
     h1 = W1 @ k
     h3 = W3 @ k
@@ -202,6 +279,10 @@ def fast_apply_vjp(kind, P, x, ybar):
     """Reverse-mode pass through fast_apply: (Pbar, xbar)."""
     if kind == LINEAR:
         return {"W": np.outer(ybar, x)}, P["W"].T @ ybar
+    if kind == GELU:
+        h = P["W1"] @ x
+        hb = (P["W2"].T @ ybar) * dgelu(h)
+        return {"W1": np.outer(hb, x), "W2": np.outer(ybar, gelu(h))}, P["W1"].T @ hb
     W1, W3, W2 = P["W1"], P["W3"], P["W2"]
     h1 = W1 @ x
     h3 = W3 @ x
@@ -373,6 +454,12 @@ def chunk_grads(kind, loss, P, K, V):
         Y = K @ P["W"].T
         E = (Y - V) if loss == LOSS_MSE else -V
         return {"W": (E, K)}
+    if kind == GELU:
+        Hg = K @ P["W1"].T
+        U = gelu(Hg)
+        E = (U @ P["W2"].T - V) if loss == LOSS_MSE else -V
+        dH = (E @ P["W2"]) * dgelu(Hg)
+        return {"W1": (dH, K), "W2": (E, U)}
     H1 = K @ P["W1"].T
     H3 = K @ P["W3"].T
     S = silu(H1)
@@ -436,6 +523,8 @@ def closed_fwd(kind, q, k, v, lr, mom, decay, W0, M0, C, d_h=0, loss=LOSS_MSE,
 def _fast_apply_rows(kind, P, X):
     if kind == LINEAR:
         return X @ P["W"].T
+    if kind == GELU:
+        return gelu(X @ P["W1"].T) @ P["W2"].T
     return (silu(X @ P["W1"].T) * (X @ P["W3"].T)) @ P["W2"].T
 
 

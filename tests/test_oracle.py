@@ -24,7 +24,7 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 def small_case(kind, B=1, H=2, T=10, C=4, d_k=4, d_v=3, d_h=5, seed=0, m0=0.3,
                mom=(0.8, 0.99), decay=(0.9, 1.0), lr=(0.05, 0.5)):
-    w = gen.Workload("t", kind, gen.F32, B, H, d_k, d_v, d_h if kind == O.SWIGLU else 0, T, C,
+    w = gen.Workload("t", kind, gen.F32, B, H, d_k, d_v, d_h if kind != O.LINEAR else 0, T, C,
                      "uniform", decay[0], seed=seed, lr_lo=lr[0], lr_hi=lr[1], mom_lo=mom[0],
                      mom_hi=mom[1], decay_hi=decay[1])
     x = gen.generate(w, m0_scale=m0)
@@ -36,7 +36,7 @@ def fwd_args(w, x):
 
 
 # ------------------------------------------------------------------ P1: closed == per-token
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 @pytest.mark.parametrize("loss", [O.LOSS_MSE, O.LOSS_NEG_DOT])
 @pytest.mark.parametrize("T,C", [(12, 4), (11, 4), (9, 9), (7, 3)])
 def test_closed_equals_sequential(kind, loss, T, C):
@@ -48,7 +48,7 @@ def test_closed_equals_sequential(kind, loss, T, C):
     assert O.rel_fro(M2, M1) < 1e-12
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 @pytest.mark.parametrize("edge", ["mu0", "lam1", "lam0", "mixed0"])
 def test_closed_equals_sequential_gate_edges(kind, edge):
     w, x = small_case(kind, T=12, C=5, seed=3)
@@ -70,7 +70,7 @@ def test_closed_equals_sequential_gate_edges(kind, edge):
 
 
 # ------------------------------------------------------------------ P2: plain chunk update
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 def test_no_momentum_unit_decay_is_plain_chunk_update(kind):
     w, x = small_case(kind, T=6, C=6, H=1, seed=5)
     x["mom"][:] = 0.0
@@ -109,7 +109,7 @@ def test_constant_gates_geometric(mu, lam):
 
 
 # ------------------------------------------------------------------ P4: chunk size 1
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 def test_chunk_size_one_is_tokenwise(kind):
     w, x = small_case(kind, T=9, C=1, seed=11)
     o1, W1, M1 = O.seq_fwd(*fwd_args(w, x), d_h=w.d_h)
@@ -145,7 +145,7 @@ def _fd(f, x, d, eps=1e-6):
     return (f(x + eps * d) - f(x - eps * d)) / (2 * eps)
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 @pytest.mark.parametrize("loss", [O.LOSS_MSE, O.LOSS_NEG_DOT])
 def test_loss_grad_matches_fd(kind, loss):
     rng = np.random.default_rng(1)
@@ -161,7 +161,7 @@ def test_loss_grad_matches_fd(kind, loss):
         assert abs(fd - g @ d) <= 1e-8 * max(1.0, abs(fd))
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 @pytest.mark.parametrize("loss", [O.LOSS_MSE, O.LOSS_NEG_DOT])
 def test_loss_grad_vjp_matches_fd(kind, loss):
     rng = np.random.default_rng(2)
@@ -184,7 +184,7 @@ def test_loss_grad_vjp_matches_fd(kind, loss):
     assert abs(_fd(lambda z: phi(s, k, z), v, dv) - vb @ dv) < 1e-7
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 def test_fast_apply_and_vjp(kind):
     rng = np.random.default_rng(3)
     d_k, d_v, d_h = 5, 4, 6
@@ -195,7 +195,7 @@ def test_fast_apply_and_vjp(kind):
     P = O.unpack(kind, s, d_k, d_v, d_h)
     if kind == O.LINEAR:  # the linear fast weight is a plain matrix-vector product
         np.testing.assert_allclose(O.fast_apply(kind, P, x), np.dot(P["W"], x), rtol=1e-15)
-    else:
+    elif kind == O.SWIGLU:
         h1 = P["W1"] @ x
         np.testing.assert_allclose(O.silu(h1), h1 / (1 + np.exp(-h1)), rtol=1e-14)
     Pb, xb = O.fast_apply_vjp(kind, P, x, yb)
@@ -203,6 +203,27 @@ def test_fast_apply_and_vjp(kind):
     f = lambda s_, x_: O.fast_apply(kind, O.unpack(kind, s_, d_k, d_v, d_h), x_) @ yb
     assert abs(_fd(lambda z: f(z, x), s, ds) - O.pack(kind, Pb) @ ds) < 1e-8
     assert abs(_fd(lambda z: f(s, z), x, dx) - xb @ dx) < 1e-8
+
+
+def test_gelu_is_the_library_gelu_and_its_derivatives_fd():
+    """The GELU MLP's activation is the exact GELU (torch's default, the erf form),
+    and its first and second derivatives match finite differences."""
+    import torch
+    z = np.linspace(-7, 7, 57)
+    ref = torch.nn.functional.gelu(torch.from_numpy(z)).numpy()
+    np.testing.assert_allclose(O.gelu(z), ref, rtol=1e-13, atol=1e-15)
+    assert abs(O.gelu(np.array(1.0)) - 0.8413447460685429) < 1e-15   # Phi(1)
+    # atol: central-difference roundoff (eps = 1e-6) where gelu' crosses zero
+    np.testing.assert_allclose(O.dgelu(z), _fd(O.gelu, z, np.ones_like(z)), rtol=1e-8, atol=1e-9)
+    np.testing.assert_allclose(O.d2gelu(z), _fd(O.dgelu, z, np.ones_like(z)), rtol=1e-7, atol=1e-9)
+
+
+@pytest.mark.parametrize("loss", [O.LOSS_MSE, O.LOSS_NEG_DOT])
+def test_seq_bwd_fd_tiny_gelu(loss):
+    """Finite differences of the per-token recurrence with the GELU MLP fast weight
+    (second-order terms through gelu'' included), ragged last chunk."""
+    w, x = small_case(O.GELU, B=1, H=1, T=7, C=3, d_k=4, d_v=4, d_h=8, seed=61)
+    _check_bwd_fd(w, x, loss=loss, seed=3)
 
 
 def test_silu_derivatives_fd():
@@ -262,7 +283,7 @@ def test_seq_bwd_fd_linear_ragged():
     _check_bwd_fd(w, x, seed=9)
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 @pytest.mark.parametrize("loss", [O.LOSS_MSE, O.LOSS_NEG_DOT])
 def test_closed_bwd_equals_seq_bwd(kind, loss):
     w, x = small_case(kind, B=1, H=2, T=11, C=4, seed=21)
@@ -413,7 +434,7 @@ def test_bf16_rounding_ties_to_even():
 # ------------------------------------------------------------------ chunk-averaged variant
 # atlas.scime.ai summary, "Surprising findings": the per-token factors collapsed to
 # chunk scalars (read as the chunk means of a_t and b_t; P_U, P_L, c unchanged).
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 def test_chunk_mean_chunk_size_one_is_tokenwise(kind):
     """With one token per chunk the mean is the token's own factor: the variant is
     token-wise TTT (the independent third loop)."""
@@ -424,7 +445,7 @@ def test_chunk_mean_chunk_size_one_is_tokenwise(kind):
     assert O.rel_fro(o1, o2) < 1e-13 and O.rel_fro(W1, W2) < 1e-13 and O.rel_fro(M1, M2) < 1e-13
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 def test_chunk_mean_no_momentum_unit_decay(kind):
     """mu = 0, lam = 1: a_t = eta_t [t = C] and b_t = eta_t, so the variant is the
     plain chunk update with the chunk's mean learning rate,
@@ -466,7 +487,7 @@ def test_chunk_mean_constant_gates_geometric(mu, lam):
     assert abs(PU - mu ** C) <= 1e-15 and abs(PL - lam ** C) <= 1e-15
 
 
-@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU])
+@pytest.mark.parametrize("kind", [O.LINEAR, O.SWIGLU, O.GELU])
 def test_chunk_mean_bwd_matches_fd(kind):
     """closed_bwd of the variant against central finite differences of closed_fwd
     of the variant, every input group, ragged last chunk."""
