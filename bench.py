@@ -54,6 +54,11 @@ def phase_flops_per_token_head(w) -> dict:
     dk, dv, dh = w.d_k, w.d_v, w.d_h
     if w.kind == gen.LINEAR:
         return {"tc_g1_linear_out_e": 4 * dk * dv, "tc_g4_aggregate_state": 4 * dv * dk}
+    if w.kind == gen.GELU:
+        return {"tc_g1_gelu": 4 * dk * dh,             # [q; k] x W1^T
+                "tc_g2_y_out_e": 4 * dh * dv,          # [A_q; A_k] x W2^T
+                "tc_g3_gelu_dh": 2 * dv * dh,          # E x W2
+                "tc_g4_aggregate_state": 4 * dh * dk + 4 * dv * dh}  # two aggregations x 2 matrices
     return {"tc_g1_h_act": 8 * dk * dh,            # [q; k] x [W1; W3]^T
             "tc_g2_y_out_e": 4 * dh * dv,          # [A_q; A_k] x W2^T
             "tc_g3_da_dh": 2 * dv * dh,            # E x W2
@@ -85,22 +90,24 @@ def kernel_work(w, has_m0: bool) -> dict:
     BH, C, T, NC = w.B * w.H, w.C, w.T, w.T // w.C
     dk, dv, dh = w.d_k, w.d_v, w.d_h
     out = {"k1_chunk_coeffs": (0.0, 20.0 * BH * T), "k1_chunk_coeffs_bwd": (0.0, 32.0 * BH * T)}
-    if w.kind != gen.SWIGLU:
+    if w.kind == gen.LINEAR:
         return out
-    S13, S2 = 2 * dh * dk, dv * dh
+    nf = 2 if w.kind == gen.SWIGLU else 1            # activation factors per hidden unit
+    S13, S2 = nf * dh * dk, dv * dh
     S = S13 + S2
     N, Mk, Mv = C * dh, C * dk, C * dv
     st_read = (4 + 4 * has_m0) + 8 * (NC - 1)       # per state element, summed over chunks
     st_write = 8 * NC + 2 * (NC - 1)
     fl = phase_flops_per_token_head(w)
+    g1, g3 = ("tc_g1_h_act", "tc_g3_da_dh") if nf == 2 else ("tc_g1_gelu", "tc_g3_gelu_dh")
     per_head = {
-        "tc_g1_h_act": (fl["tc_g1_h_act"] * C, 2 * (2 * Mk + S13 + 2 * N + 2 * N)),
-        "tc_g2_y_out_e": (fl["tc_g2_y_out_e"] * 2 * C, 2 * (2 * N + S2 + Mv + 4 * Mv)),
-        "tc_g3_da_dh": (fl["tc_g3_da_dh"] * C, 2 * (Mv + S2 + 2 * N + 2 * N)),
+        g1: (fl[g1] * C, 2 * (2 * Mk + S13 + 2 * N + nf * N)),
+        "tc_g2_y_out_e": (fl["tc_g2_y_out_e"] * C, 2 * (2 * N + S2 + Mv + 4 * Mv)),
+        g3: (fl[g3] * C, 2 * (Mv + S2 + nf * N + nf * N)),
         "tc_g4_aggregate_state": (fl["tc_g4_aggregate_state"] * C,
-                                  2 * (2 * N + 2 * Mk + 2 * Mv + N) + S * (st_read + st_write) / NC),
+                                  2 * (nf * N + 2 * Mk + 2 * Mv + N) + S * (st_read + st_write) / NC),
     }
-    if dk == dv:
+    if dk == dv and nf == 2:
         dd = dk * dh
         b = {"tcb_r1_h": 4 * Mk + 2 * S13 + 12 * N, "tcb_r2_e": 2 * N + 2 * S2 + 4 * Mv,
              "tcb_r3_du": 2 * Mv + 2 * S2 + 12 * N, "tcb_d1_dir13": 2 * Mk + 4 * S13 + 12 * N,
@@ -336,14 +343,15 @@ def measure_extras(E, torch, dev, stream, args):
     """The metric's other operating points, device-timed like the main line:
     forward at T = 16K (the 8x length-extrapolation layer), forward+backward at
     T = 2K (the training workload), and the forward at T = 2K of the
-    chunk-averaged variant and of the no-momentum mode, each with its own
-    warm-up."""
+    chunk-averaged variant, of the no-momentum mode and of the GELU MLP fast
+    weight, each with its own warm-up."""
     out = {}
     f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
     for name, train, steps, coef, nomom in (("layer_1p3b_16k", False, args.extra_steps, 0, 0),
                                             ("train_1p3b_2k", True, max(2, args.extra_steps // 8), 0, 0),
                                             ("layer_1p3b_2k", False, args.extra_steps, 1, 0),
-                                            ("layer_1p3b_2k", False, args.extra_steps, 0, 1)):
+                                            ("layer_1p3b_2k", False, args.extra_steps, 0, 1),
+                                            ("layer_1p3b_2k_gelu", False, args.extra_steps, 0, 0)):
         w = gen.BY_NAME[name]
         x = gen.generate(w)
         q, k, v = f(x["q"], torch.bfloat16), f(x["k"], torch.bfloat16), f(x["v"], torch.bfloat16)

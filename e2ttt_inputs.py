@@ -86,6 +86,8 @@ WORKLOADS = [
     Workload("layer_1p3b_16k", SWIGLU, BF16, 1, 8, 256, 256, 512, 16384, 512, "softplus", 0.98, seed=3),
     Workload("train_1p3b_2k", SWIGLU, BF16, 4, 8, 256, 256, 512, 2048, 512, "softplus", 0.95, seed=4,
              with_bwd=True),
+    Workload("layer_1p3b_2k_gelu", GELU, BF16, 4, 8, 256, 256, 512, 2048, 512, "softplus", 0.95,
+             seed=5),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 

@@ -69,7 +69,10 @@ typedef enum {
   E2TTT_ERR_TIMEOUT = 4        /* a device-side bounded wait gave up                  */
 } e2ttt_status;
 
-typedef enum { E2TTT_LINEAR = 0, E2TTT_SWIGLU = 1 } e2ttt_fast_kind;
+/* Fast weight f_W: LINEAR W x; SWIGLU W2 (silu(W1 x) * (W3 x)); GELU_MLP
+ * W2 gelu(W1 x) with the exact GELU z Phi(z) (the MLP variant, "E2-TTT_MLP" in
+ * the atlas.scime.ai summary, "Key results"; forward only). */
+typedef enum { E2TTT_LINEAR = 0, E2TTT_SWIGLU = 1, E2TTT_GELU_MLP = 2 } e2ttt_fast_kind;
 typedef enum { E2TTT_F32 = 0, E2TTT_BF16 = 1 } e2ttt_dtype;
 typedef enum { E2TTT_LOSS_MSE = 0, E2TTT_LOSS_NEG_DOT = 1 } e2ttt_loss;
 /* Momentum / weight kernels. PER_TOKEN: a_t, b_t of every token (the method).
@@ -101,8 +104,9 @@ typedef struct {
   int momentum;
 } e2ttt_shape;
 
-/* Fast-weight state size S per (b, h): d_v*d_k (linear) or 2*d_h*d_k + d_v*d_h
- * (SwiGLU). Returns 0 for an invalid shape. */
+/* Fast-weight state size S per (b, h): d_v*d_k (linear), 2*d_h*d_k + d_v*d_h
+ * (SwiGLU, [W1 | W3 | W2]) or d_h*d_k + d_v*d_h (GELU MLP, [W1 | W2]). Returns
+ * 0 for an invalid shape. */
 size_t e2ttt_state_elems(const e2ttt_shape* shape);
 
 /* Bytes of device scratch the forward (for_bwd = 0) or backward (for_bwd = 1)
@@ -187,7 +191,8 @@ e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
  *            (act dtype), dW_end, dM_end (fp32 [B,H,S]; may be NULL = zero).
  *   Outputs: dq, dk, dv (act dtype), dlr, dmom, ddecay (fp32 [B,H,T]),
  *            dW0, dM0 (fp32 [B,H,S]).
- *   No-momentum mode: mom, dM_end, dmom and dM0 must be NULL. */
+ *   No-momentum mode: mom, dM_end, dmom and dM0 must be NULL.
+ *   E2TTT_GELU_MLP returns E2TTT_ERR_UNSUPPORTED (forward only). */
 e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
                                   const void* q, const void* k, const void* v,
                                   const float* lr, const float* mom, const float* decay,

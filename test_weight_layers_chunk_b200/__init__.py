@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libe2ttt.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "e2ttt.h")
 
-LINEAR, SWIGLU = 0, 1
+LINEAR, SWIGLU, GELU_MLP = 0, 1, 2
 F32, BF16 = 0, 1
 LOSS_MSE, LOSS_NEG_DOT = 0, 1
 COEF_PER_TOKEN, COEF_CHUNK_MEAN = 0, 1

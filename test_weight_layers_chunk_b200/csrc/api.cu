@@ -43,18 +43,18 @@ bool shape_ok(const e2ttt_shape* s, std::string* why) {
     *why = buf;
     return false;
   }
-  if (s->kind != E2TTT_LINEAR && s->kind != E2TTT_SWIGLU) { *why = "unknown fast-weight kind"; return false; }
+  if (s->kind != E2TTT_LINEAR && s->kind != E2TTT_SWIGLU && s->kind != E2TTT_GELU_MLP) { *why = "unknown fast-weight kind"; return false; }
   if (s->act != E2TTT_F32 && s->act != E2TTT_BF16) { *why = "unknown activation dtype"; return false; }
   if (s->loss != E2TTT_LOSS_MSE && s->loss != E2TTT_LOSS_NEG_DOT) { *why = "unknown loss"; return false; }
   if (s->coef != E2TTT_COEF_PER_TOKEN && s->coef != E2TTT_COEF_CHUNK_MEAN) { *why = "unknown coef"; return false; }
   if (s->momentum != E2TTT_MOMENTUM && s->momentum != E2TTT_NO_MOMENTUM) { *why = "unknown momentum mode"; return false; }
-  if (s->kind == E2TTT_SWIGLU && s->d_h < 1) { *why = "SwiGLU needs d_h >= 1"; return false; }
+  if (s->kind != E2TTT_LINEAR && s->d_h < 1) { *why = "SwiGLU and the GELU MLP need d_h >= 1"; return false; }
   if (s->C > 1024) { *why = "chunk size C must be <= 1024"; return false; }
   long long BH = (long long)s->B * s->H;
   if (BH > 65535) { *why = "B*H must be <= 65535"; return false; }
   long long dmax = s->d_k;
   if (s->d_v > dmax) dmax = s->d_v;
-  if (s->kind == E2TTT_SWIGLU && 2LL * s->d_h > dmax) dmax = 2LL * s->d_h;
+  if (s->kind != E2TTT_LINEAR && 2LL * s->d_h > dmax) dmax = 2LL * s->d_h;
   if (BH * s->T * dmax >= (1LL << 31)) { *why = "B*H*T*max(d) must be < 2^31"; return false; }
   return true;
 }
@@ -67,13 +67,14 @@ Dims make_dims(const e2ttt_shape* s) {
   d.NC = (s->T + s->C - 1) / s->C;
   d.d_k = s->d_k;
   d.d_v = s->d_v;
-  d.d_h = s->kind == E2TTT_SWIGLU ? s->d_h : 0;
+  d.d_h = s->kind != E2TTT_LINEAR ? s->d_h : 0;
   d.kind = s->kind;
   d.loss = s->loss;
   d.coef = s->coef;
   d.nomom = s->momentum == E2TTT_NO_MOMENTUM;
-  d.S = s->kind == E2TTT_LINEAR ? (long long)s->d_v * s->d_k
-                                : 2LL * s->d_h * s->d_k + (long long)s->d_v * s->d_h;
+  d.S = s->kind == E2TTT_LINEAR     ? (long long)s->d_v * s->d_k
+        : s->kind == E2TTT_GELU_MLP ? (long long)s->d_h * s->d_k + (long long)s->d_v * s->d_h
+                                    : 2LL * s->d_h * s->d_k + (long long)s->d_v * s->d_h;
   return d;
 }
 
@@ -108,9 +109,10 @@ FwdWs fwd_layout(const Dims& d, bool tc_shape) {
   const size_t region = w.off;
   Bump s;
   s.off = region;
-  if (d.kind == 1) L.H = s.take((size_t)d.BH * 2 * d.C * 2 * d.d_h * f);
+  const size_t nf = d.kind == 1 ? 2 : 1;  // activation factors per hidden unit
+  if (d.kind != 0) L.H = s.take((size_t)d.BH * 2 * d.C * nf * d.d_h * f);
   L.E = s.take((size_t)d.BH * d.C * d.d_v * f);
-  if (d.kind == 1) L.dH = s.take((size_t)d.BH * d.C * 2 * d.d_h * f);
+  if (d.kind != 0) L.dH = s.take((size_t)d.BH * d.C * nf * d.d_h * f);
   size_t end = s.off;
   L.tc = region;
   if (tc_shape) {
@@ -354,6 +356,8 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* s, const void* q, const voi
                   {ws, need, "workspace"}};
   if (!check_overlaps(in, 10, outr, 9, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
   if (d.nomom) dM0 = (float*)((char*)ws + dm_off);  // zero momentum adjoint, kept internal
+  if (d.kind == E2TTT_GELU_MLP)
+    return fail(E2TTT_ERR_UNSUPPORTED, "the backward of the GELU MLP fast weight is not implemented");
   BwdArgs A{d, q, k, v, lr, mom, decay, saved, dout, dW_end, dM_end, dq, dk, dv,
             dlr, dmom, ddecay, dW0, dM0, ws, (cudaStream_t)stream};
   cudaError_t e = bf ? bwd_run<bf16>(A) : bwd_run<float>(A);

@@ -40,4 +40,12 @@ struct Dims {
   long long S; // state elements per head
 };
 
+// Exact GELU z Phi(z) (Phi the standard normal CDF, through erff) and its
+// derivative Phi(z) + z phi(z), for the GELU MLP fast weight.
+__device__ __forceinline__ float gelu_cdf_f(float z) { return 0.5f * (1.0f + erff(z * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_f(float z) { return z * gelu_cdf_f(z); }
+__device__ __forceinline__ float dgelu_f(float z) {
+  return gelu_cdf_f(z) + z * 0.39894228040143268f * expf(-0.5f * z * z);
+}
+
 }  // namespace e2ttt

@@ -10,6 +10,8 @@
 //            E = Y_k - V,  dA = E W2,  dH1 = dA * H3_k * silu'(H1_k),
 //            dH3 = dA * silu(H1_k)
 //            d[W1; W3] = [dH1 | dH3]^T diag(.) K,   dW2 = E^T diag(.) A_k
+//   GELU MLP: H = [Q; K] W1^T,  A = gelu(H),  [out; Y_k] = A W2^T,  E = Y_k - V,
+//            dH = (E W2) * gelu'(H_k),  dW1 = dH^T diag(.) K,  dW2 = E^T diag(.) A_k
 //   epilogue (fp32): M_end = U(1,n) M0 - dM,  W_end = L(1,n) W0 + c M0 - dW
 // (E = -V for the dot-product loss.)
 #include "simt.cuh"
@@ -29,7 +31,13 @@ struct Fwd {
   float *H, *E, *dH;
   int ci, t0, n;
   __device__ __forceinline__ size_t tok(int z, int t) const { return (size_t)z * d.T + t0 + t; }
+  // row length of H and dH: [h1 | h3] (SwiGLU) or h (GELU MLP)
+  __device__ __forceinline__ int hld() const { return d.kind == 2 ? d.d_h : 2 * d.d_h; }
 };
+// the activation of hidden unit j of one row of H
+__device__ __forceinline__ float act_of(const Dims& d, const float* h, int j) {
+  return d.kind == 2 ? gelu_f(h[j]) : silu_f(h[j]) * h[d.d_h + j];
+}
 
 // rows of [Q_chunk; K_chunk]
 template <typename TA> struct LoadX {
@@ -57,13 +65,12 @@ template <typename TA> struct LoadW {
     return c.src.W[z * c.src.stride + off + (long long)kk * ld + j];
   }
 };
-// A = silu(H1) * H3 on the [q; k] rows
+// A = silu(H1) * H3 (or gelu(H)) on the [q; k] rows
 template <typename TA> struct LoadAct {
   Fwd<TA> c;
   int row0;
   __device__ __forceinline__ float operator()(int z, int r, int j) const {
-    const float* h = c.H + ((size_t)z * 2 * c.d.C + row0 + r) * 2 * c.d.d_h;
-    return silu_f(h[j]) * h[c.d.d_h + j];
+    return act_of(c.d, c.H + ((size_t)z * 2 * c.d.C + row0 + r) * c.hld(), j);
   }
 };
 // A(t, kk) = L[t, kk] with L [C, ld] per head in workspace
@@ -89,12 +96,11 @@ template <typename TA> struct LoadK {
     return to_f(c.k[c.tok(z, t) * c.d.d_k + j]);
   }
 };
-// B(t, j) = A_k[t, j] = silu(h1) * h3 of the key rows
+// B(t, j) = A_k[t, j], the activation of the key rows
 template <typename TA> struct LoadActK {
   Fwd<TA> c;
   __device__ __forceinline__ float operator()(int z, int t, int j) const {
-    const float* h = c.H + ((size_t)z * 2 * c.d.C + c.n + t) * 2 * c.d.d_h;
-    return silu_f(h[j]) * h[c.d.d_h + j];
+    return act_of(c.d, c.H + ((size_t)z * 2 * c.d.C + c.n + t) * c.hld(), j);
   }
 };
 template <typename TA> struct ScaleAB {
@@ -122,16 +128,20 @@ template <typename TA> struct EpiOutE {
 template <typename TA> struct EpiStoreH {
   Fwd<TA> c;
   __device__ __forceinline__ void operator()(int z, int r, int col, const float* acc) const {
-    c.H[((size_t)z * 2 * c.d.C + r) * 2 * c.d.d_h + col] = acc[0];
+    c.H[((size_t)z * 2 * c.d.C + r) * c.hld() + col] = acc[0];
   }
 };
 template <typename TA> struct EpiDH {
   Fwd<TA> c;
   __device__ __forceinline__ void operator()(int z, int t, int j, const float* acc) const {
     const int dh = c.d.d_h;
-    const float* h = c.H + ((size_t)z * 2 * c.d.C + c.n + t) * 2 * dh;
+    const float* h = c.H + ((size_t)z * 2 * c.d.C + c.n + t) * c.hld();
+    float* o = c.dH + ((size_t)z * c.d.C + t) * c.hld();
+    if (c.d.kind == 2) {
+      o[j] = acc[0] * dgelu_f(h[j]);
+      return;
+    }
     float h1 = h[j], h3 = h[dh + j];
-    float* o = c.dH + ((size_t)z * c.d.C + t) * 2 * dh;
     o[j] = acc[0] * h3 * dsilu_f(h1);
     o[dh + j] = acc[0] * silu_f(h1);
   }
@@ -158,8 +168,9 @@ cudaError_t fwd_chunk(const Fwd<TA>& c, cudaStream_t st) {
     return simt_gemm<2>(d.BH, d.d_v, d.d_k, n, LoadTok<TA>{c.E, d.C, d.d_v}, LoadK<TA>{c},
                         ScaleAB<TA>{c}, EpiState<TA>{c, 0, d.d_k}, st, "simt_aggregate_state");
   }
-  const long long o2 = 2LL * d.d_h * d.d_k;
-  e = simt_gemm<1>(d.BH, 2 * n, 2 * d.d_h, d.d_k, LoadX<TA>{c}, LoadWT<TA>{c, 0, d.d_k},
+  const int r13 = d.kind == 2 ? d.d_h : 2 * d.d_h;  // rows of W1 (GELU) or [W1; W3]
+  const long long o2 = (long long)r13 * d.d_k;
+  e = simt_gemm<1>(d.BH, 2 * n, r13, d.d_k, LoadX<TA>{c}, LoadWT<TA>{c, 0, d.d_k},
                    UnitScale{}, EpiStoreH<TA>{c}, st, "simt_g1_h");
   if (e != cudaSuccess) return e;
   e = simt_gemm<1>(d.BH, 2 * n, d.d_v, d.d_h, LoadAct<TA>{c, 0}, LoadWT<TA>{c, o2, d.d_h},
@@ -168,7 +179,7 @@ cudaError_t fwd_chunk(const Fwd<TA>& c, cudaStream_t st) {
   e = simt_gemm<1>(d.BH, n, d.d_h, d.d_v, LoadRow<TA>{c.E, d.C, d.d_v}, LoadW<TA>{c, o2, d.d_h},
                    UnitScale{}, EpiDH<TA>{c}, st, "simt_g3_da_dh");
   if (e != cudaSuccess) return e;
-  e = simt_gemm<2>(d.BH, 2 * d.d_h, d.d_k, n, LoadTok<TA>{c.dH, d.C, 2 * d.d_h}, LoadK<TA>{c},
+  e = simt_gemm<2>(d.BH, r13, d.d_k, n, LoadTok<TA>{c.dH, d.C, r13}, LoadK<TA>{c},
                    ScaleAB<TA>{c}, EpiState<TA>{c, 0, d.d_k}, st, "simt_g4_aggregate_w13");
   if (e != cudaSuccess) return e;
   return simt_gemm<2>(d.BH, d.d_v, d.d_h, n, LoadTok<TA>{c.E, d.C, d.d_v}, LoadActK<TA>{c},

@@ -175,6 +175,89 @@ struct EpiG1 {
   }
 };
 
+// G1, GELU MLP: H = X W1^T -> A = gelu(H) (query and key rows) and the key rows'
+// gelu'(H) (the factor G3 needs). Class 0 = query rows, class 1 = key rows.
+struct EpiG1Gelu {
+  static constexpr int kSmem = 4096;  // gelu(H) | gelu'(H) staging
+  template <int BN>
+  static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;
+    const int per = BN / c.nparts;
+    const int yA = c.z * 2 * d.C + c.cls * d.C + r0;
+    const int ySk = c.z * d.C + r0;
+    uint8_t* S = c.wsmem;
+    for (int g = c.part * per; g < (c.part + 1) * per; g += 32) {
+      const int j = c.n0 + g;
+      float h[32], gp[32];
+      ld1(c, 0, g, h);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        gp[i] = dgelu_f(h[i]);
+        h[i] = gelu_f(h[i]);
+      }
+      staging_free(lane);
+      stage32(S, lane, h);
+      if (c.cls == 1) stage32(S + 2048, lane, gp);
+      staging_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mA, S, j, yA);
+        if (c.cls == 1) tc::tma_store_2d(&p.mSk, S + 2048, j, ySk);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
+
+// G3, GELU MLP: dA = E W2 -> dH = dA gelu'(H_k) (rows: key tokens).
+struct EpiG3Gelu {
+  static constexpr int kSmem = 6144;  // gelu'(H) [2 groups] | dH staging
+  template <int BN>
+  static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;
+    const int per = BN / c.nparts;
+    const int col0 = c.n0 + c.part * per;
+    static_assert(BN <= 128, "factor buffers for at most two column groups per warp");
+    const int ngroups = per / 32;
+    const int y = c.z * d.C + r0;
+    uint8_t* F = c.wsmem;
+    uint8_t* S = c.wsmem + 4096;
+    if (lane == 0) {
+      tc::mbar_expect_tx(&c.wbar[0], 2048u * ngroups);
+      for (int gi = 0; gi < ngroups; ++gi)
+        tc::tma_load_2d(F + gi * 2048, &p.mSk, &c.wbar[0], col0 + gi * 32, y);
+    }
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      float da[32], gp[32];
+      ld1(c, 0, c.part * per + gi * 32, da);
+      if (gi == 0) {
+        const bool ok = tc::mbar_wait(&c.wbar[0], c.uses[0] & 1u);
+        c.uses[0] += 1;
+        if (!ok) {
+          if (lane == 0) atomicExch(p.status, tc2::kErrEpilogue);
+          return;
+        }
+      }
+      unstage32(F + gi * 2048, lane, gp);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) da[i] *= gp[i];
+      staging_free(lane);
+      stage32(S, lane, da);
+      staging_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mdH, S, col0 + gi * 32, y);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
+
 // Query rows -> out, key rows -> E (optional) and its a-/b-scaled copies, for a
 // warp's 32 rows and its column groups; V of the key rows is prefetched.
 template <int BN>
@@ -351,6 +434,8 @@ struct EpiG4 {
     if (c.cls == 0 && d.kind == 1) {
       const int which = r0 / d.d_h, rr = r0 % d.d_h;
       sh_row = c.z * 2 * d.d_h + w13_row(rr, which);
+    } else if (c.cls == 0 && d.kind == 2) {
+      sh_row = c.z * d.d_h + r0;  // W1 of the GELU MLP, not interleaved
     } else {
       sh_row = c.z * d.d_v + r0;
     }
@@ -445,6 +530,8 @@ struct EpiG4W {
     if (c.cls == 0 && d.kind == 1) {
       const int which = r0 / d.d_h, rr = r0 % d.d_h;
       sh_row = c.z * 2 * d.d_h + w13_row(rr, which);
+    } else if (c.cls == 0 && d.kind == 2) {
+      sh_row = c.z * d.d_h + r0;  // W1 of the GELU MLP, not interleaved
     } else {
       sh_row = c.z * d.d_v + r0;
     }
@@ -506,17 +593,20 @@ template <> struct EpiName<EpiG2> { static constexpr const char* v = "tc_g2_y_ou
 template <> struct EpiName<EpiG3> { static constexpr const char* v = "tc_g3_da_dh"; };
 template <> struct EpiName<EpiG4> { static constexpr const char* v = "tc_g4_aggregate_state"; };
 template <> struct EpiName<EpiG4W> { static constexpr const char* v = "tc_g4_aggregate_w"; };
+template <> struct EpiName<EpiG1Gelu> { static constexpr const char* v = "tc_g1_gelu"; };
+template <> struct EpiName<EpiG3Gelu> { static constexpr const char* v = "tc_g3_gelu_dh"; };
 template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 
 // ---------------------------------------------------------------- prep kernel
 // bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
 __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
-  // One warp per state row: rows [0, 2 d_h) of a head are W1 then W3 (d_k wide),
-  // rows [2 d_h, 2 d_h + d_v) are W2 (d_h wide); the linear state is d_v rows of d_k.
+  // One warp per state row: rows [0, 2 d_h) of a head are W1 then W3 (d_k wide;
+  // GELU MLP: [0, d_h) are W1), the next d_v rows are W2 (d_h wide); the linear
+  // state is d_v rows of d_k.
   const Dims& d = p.d;
   const int lane = threadIdx.x & 31;
-  const int r13 = d.kind == 1 ? 2 * d.d_h : d.d_v;
-  const int rows = d.kind == 1 ? r13 + d.d_v : r13;
+  const int r13 = d.kind == 1 ? 2 * d.d_h : d.kind == 2 ? d.d_h : d.d_v;
+  const int rows = d.kind != 0 ? r13 + d.d_v : r13;
   const long long total = (long long)d.BH * rows;
   const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
   for (long long gr = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); gr < total;
@@ -667,12 +757,13 @@ size_t carve(const Dims& d, char* base, Scratch* s) {
   if (d.kind == 0) {
     t.Wsh13 = take(BH * d.d_v * d.d_k * e);
   } else {
-    t.Wsh13 = take(BH * 2 * d.d_h * d.d_k * e);
+    const size_t nf = d.kind == 1 ? 2 : 1;  // activation factors per hidden unit
+    t.Wsh13 = take(BH * nf * d.d_h * d.d_k * e);
     t.W2sh = take(BH * d.d_v * d.d_h * e);
     t.A = take(BH * 2 * d.C * d.d_h * e);
-    t.Sk = take(BH * d.C * 2 * d.d_h * e);
+    t.Sk = take(BH * d.C * nf * d.d_h * e);
     t.E = take(BH * d.C * d.d_v * e);
-    t.dH = take(BH * d.C * 2 * d.d_h * e);
+    t.dH = take(BH * d.C * nf * d.d_h * e);
     t.Ka = take(BH * d.T * d.d_k * e);
     t.Kb = take(BH * d.T * d.d_k * e);
   }
@@ -688,7 +779,7 @@ bool tc_fwd_supported(const Dims& d, bool bf16_act) {
   if (!bf16_act) return false;
   if (d.T % d.C != 0 || d.C % 128 != 0) return false;
   if (d.d_k % 128 != 0 || d.d_v % 128 != 0) return false;
-  if (d.kind == 1 && d.d_h % 128 != 0) return false;
+  if (d.kind != 0 && d.d_h % 128 != 0) return false;
   return encode_fn() != nullptr;
 }
 
@@ -710,6 +801,8 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   p.A = s.A; p.Sk = s.Sk; p.E = s.E; p.Ea = s.Ea; p.Eb = s.Eb; p.dH = s.dH; p.Ka = s.Ka;
   p.Kb = s.Kb;
   const int BH = d.BH, T = d.T, C = d.C, NC = d.NC, dk = d.d_k, dv = d.d_v, dh = d.d_h;
+  const int nf = d.kind == 1 ? 2 : 1;           // activation factors per hidden unit
+  const int r13 = d.kind == 0 ? dv : nf * dh;   // rows of the first state block
 
   cudaError_t e = save_initial_state(d, W0, M0, saved, st);
   if (e != cudaSuccess) return e;
@@ -719,7 +812,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (d.kind == 1) {
+  if (d.kind != 0) {
     E2TTT_TRACE("tc_scale_keys", st);
     scale_keys_kernel<<<4 * num_sms(), 256, 0, st>>>(k, ca, cb, d.nomom ? nullptr : s.Ka, s.Kb,
                                                      (long long)BH * T, dk);
@@ -736,15 +829,22 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   }
   using tc2::kModeA1B2;
   using tc2::kModeA2B1;
-  if (d.kind == 1) {
-    // G1: classes = query rows, key rows; B = interleaved [W1; W3]
+  if (d.kind != 0) {
     ok &= make_map(&g1.maps[0].op0, q, (uint64_t)BH * T, dk, 128);
     ok &= make_map(&g1.maps[1].op0, k, (uint64_t)BH * T, dk, 128);
-    ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * 2 * dh, dk, 256);
-    g1.maps[1].op2 = g1.maps[0].op2;
     g1.n_cls = 2;
-    for (int c = 0; c < 2; ++c)
-      g1.cls[c] = tc2::Class{C / 128, 2 * dh / 256, dk / 64, {T, 0, 0}, {2 * dh, 0, 0}, 0};
+    if (d.kind == 1) {
+      // G1: classes = query rows, key rows; B = interleaved [W1; W3]
+      ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * 2 * dh, dk, 256);
+      for (int c = 0; c < 2; ++c)
+        g1.cls[c] = tc2::Class{C / 128, 2 * dh / 256, dk / 64, {T, 0, 0}, {2 * dh, 0, 0}, 0};
+    } else {
+      // G1, GELU MLP: B = W1 (N = d_h), 128-wide tiles
+      ok &= make_map(&g1.maps[0].op2, s.Wsh13, (uint64_t)BH * dh, dk, 128);
+      for (int c = 0; c < 2; ++c)
+        g1.cls[c] = tc2::Class{C / 128, dh / 128, dk / 64, {T, 0, 0}, {dh, 0, 0}, 0};
+    }
+    g1.maps[1].op2 = g1.maps[0].op2;
     // G2: A = [A_q; A_k], B = W2 (N = d_v)
     ok &= make_map(&g2.maps[0].op0, s.A, (uint64_t)BH * 2 * C, dh, 128);
     ok &= make_map(&g2.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 128);
@@ -755,8 +855,9 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     ok &= make_map(&g3.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 64);
     g3.n_cls = 1;
     g3.cls[0] = tc2::Class{C / 128, dh / 128, dv / 64, {C, 0, 0}, {dv, 0, 0}, 0};
-    // G4 class 0: A = dH (M = [W1; W3] rows, K = tokens), B0 = diag(a) K, B1 = diag(b) K
-    ok &= make_map(&g4.maps[0].op0, s.dH, (uint64_t)BH * C, 2 * dh, 64);
+    // G4 class 0: A = dH (M = [W1; W3] rows, or W1 rows for GELU; K = tokens),
+    // B0 = diag(a) K, B1 = diag(b) K
+    ok &= make_map(&g4.maps[0].op0, s.dH, (uint64_t)BH * C, r13, 64);
     ok &= make_map(&g4.maps[0].op1, s.Ka, (uint64_t)BH * T, dk, 64);
     ok &= make_map(&g4.maps[0].op2, s.Kb, (uint64_t)BH * T, dk, 64);
     // G4 class 1: A0 = diag(a) E, A1 = diag(b) E (M = W2 rows), B = A_k (rows [C, 2C) of A)
@@ -764,7 +865,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     ok &= make_map(&g4.maps[1].op1, s.Eb, (uint64_t)BH * C, dv, 64);
     ok &= make_map(&g4.maps[1].op2, s.A, (uint64_t)BH * 2 * C, dh, 64);
     g4.n_cls = 2;
-    g4.cls[0] = tc2::Class{2 * dh / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, kModeA1B2};
+    g4.cls[0] = tc2::Class{r13 / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, kModeA1B2};
     g4.cls[1] = tc2::Class{dv / 128, dh / 128, C / 64, {C, 0, 0}, {2 * C, C, 0}, kModeA2B1};
   } else {
     ok &= make_map(&g1.maps[0].op0, q, (uint64_t)BH * T, dk, 128);
@@ -786,13 +887,13 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   g4w.heads = BH;
   g4w.status = status;
   if (d.nomom) {
-    if (d.kind == 1) {
-      ok &= make_map(&g4w.maps[0].op0, s.dH, (uint64_t)BH * C, 2 * dh, 64);
+    if (d.kind != 0) {
+      ok &= make_map(&g4w.maps[0].op0, s.dH, (uint64_t)BH * C, r13, 64);
       ok &= make_map(&g4w.maps[0].op2, s.Kb, (uint64_t)BH * T, dk, 64);
       ok &= make_map(&g4w.maps[1].op0, s.Eb, (uint64_t)BH * C, dv, 64);
       ok &= make_map(&g4w.maps[1].op2, s.A, (uint64_t)BH * 2 * C, dh, 64);
       g4w.n_cls = 2;
-      g4w.cls[0] = tc2::Class{2 * dh / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, 0};
+      g4w.cls[0] = tc2::Class{r13 / 128, dk / 128, C / 64, {C, 0, 0}, {T, 0, 0}, 0};
       g4w.cls[1] = tc2::Class{dv / 128, dh / 128, C / 64, {C, 0, 0}, {2 * C, C, 0}, 0};
     } else {
       ok &= make_map(&g4w.maps[0].op0, s.Eb, (uint64_t)BH * C, dv, 64);
@@ -806,11 +907,11 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   ok &= make_map_box32(&p.mV, v, (uint64_t)BH * T, dv);
   ok &= make_map_box32(&p.mEa, s.Ea, (uint64_t)BH * C, dv);
   ok &= make_map_box32(&p.mEb, s.Eb, (uint64_t)BH * C, dv);
-  if (d.kind == 1) {
+  if (d.kind != 0) {
     ok &= make_map_box32(&p.mA, s.A, (uint64_t)BH * 2 * C, dh);
-    ok &= make_map_box32(&p.mSk, s.Sk, (uint64_t)BH * C, 2 * dh);
+    ok &= make_map_box32(&p.mSk, s.Sk, (uint64_t)BH * C, nf * dh);
     ok &= make_map_box32(&p.mE, s.E, (uint64_t)BH * C, dv);
-    ok &= make_map_box32(&p.mdH, s.dH, (uint64_t)BH * C, 2 * dh);
+    ok &= make_map_box32(&p.mdH, s.dH, (uint64_t)BH * C, nf * dh);
   }
   if (!ok) return cudaErrorInvalidValue;
 
@@ -820,10 +921,10 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     p.write_shadow = ci + 1 < NC;
     chunk_states(d, ci, W0, M0, W_end, M_end, saved, &p.src, &p.dst);
     {
-      const int ncls = d.kind == 1 ? 2 : 1;
+      const int ncls = d.kind != 0 ? 2 : 1;
       for (int c = 0; c < ncls; ++c) {
-        const long long off = c == 0 ? 0 : 2LL * dh * dk;
-        const uint64_t rows = c == 0 ? (d.kind == 1 ? 2 * dh : dv) : dv;
+        const long long off = c == 0 ? 0 : (long long)r13 * dk;
+        const uint64_t rows = c == 0 ? r13 : dv;
         const uint64_t cols = c == 0 ? dk : dh;
         ok &= make_state_map(&p.srcW[c], p.src.W + off, rows, cols, BH, p.src.stride);
         if (p.src.M) ok &= make_state_map(&p.srcM[c], p.src.M + off, rows, cols, BH, p.src.stride);
@@ -831,18 +932,25 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
         if (p.dst.M) ok &= make_state_map(&p.dstM[c], p.dst.M + off, rows, cols, BH, p.dst.stride);
       }
       if (ci == 0) {
-        ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * (d.kind == 1 ? 2 * dh : dv), dk);
-        if (d.kind == 1) ok &= make_map_box32(&p.shadow[1], s.W2sh, (uint64_t)BH * dv, dh);
+        ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * r13, dk);
+        if (d.kind != 0) ok &= make_map_box32(&p.shadow[1], s.W2sh, (uint64_t)BH * dv, dh);
       }
       if (!ok) return cudaErrorInvalidValue;
     }
     g1.cls[0].a.y_base = g1.cls[1].a.y_base = ci * C;  // query / key rows of this chunk
     g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
     g4w.cls[0].b.y_base = ci * C;
-    if (d.kind == 1) {
-      e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
+    if (d.kind != 0) {
+      if (d.kind == 1)
+        e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
+      else
+        e = launch<128, 1, false, false, 4, EpiG1Gelu, kEpiWarps, EpiG1Gelu::kSmem>(g1, p, st);
       if (e == cudaSuccess) e = launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
-      if (e == cudaSuccess) e = launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st);
+      if (e == cudaSuccess) {
+        e = d.kind == 1
+                ? launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st)
+                : launch<128, 1, false, true, 3, EpiG3Gelu, kEpiWarps, EpiG3Gelu::kSmem>(g3, p, st);
+      }
       if (e == cudaSuccess) {
         e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)
                     : launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);

@@ -97,6 +97,8 @@ F32_CASES = {
     "tiny_linear_m0": gen.WORKLOADS[0],
     "linear_ragged": gen.Workload("lr", gen.LINEAR, gen.F32, 2, 3, 40, 24, 0, 203, 48, "uniform",
                                   0.99, seed=11),
+    "gelu_f32": gen.Workload("gf", gen.GELU, gen.F32, 2, 2, 24, 20, 40, 100, 32, "uniform", 0.99,
+                             seed=14, lr_lo=0.005, lr_hi=0.05),
     "swiglu_f32": gen.Workload("sf", gen.SWIGLU, gen.F32, 2, 2, 24, 20, 40, 100, 32, "uniform",
                                0.99, seed=12, lr_lo=0.002, lr_hi=0.02, mom_lo=0.7, mom_hi=0.95),
     "swiglu_f32_dot": gen.Workload("sd", gen.SWIGLU, gen.F32, 1, 2, 16, 16, 32, 96, 32, "uniform",

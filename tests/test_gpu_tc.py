@@ -66,6 +66,11 @@ CASES = {
     "swiglu_dot": (gen.Workload("dot", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 256, "uniform",
                                 0.999, seed=22, lr_lo=0.0005, lr_hi=0.005, mom_lo=0.5, mom_hi=0.9,
                                 loss=gen.LOSS_NEG_DOT), None),
+    # the GELU MLP fast weight (state-preserving gates: W = 0 is a fixed point here too)
+    "gelu_d128_preserving": (gen.Workload("gelu", gen.GELU, gen.BF16, 1, 2, 128, 128, 256, 512, 128,
+                                          "uniform", 0.999, seed=24, lr_lo=0.002, lr_hi=0.02), None),
+    "layer_1p3b_2k_gelu_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_2k_gelu"]),
+                                      [(0, 1), (3, 6)]),
 }
 
 
@@ -137,3 +142,23 @@ def test_tc_and_cuda_core_paths_agree(E):
     b = run_fwd(E, w, d2)
     for i in range(3):
         assert err(host(a[i]), host(b[i])) < TOL
+
+
+def test_gelu_tc_and_cuda_core_paths_agree(E):
+    """The GELU MLP through both forward paths (an unaligned view of q routes the
+    call to the CUDA-core path)."""
+    import torch
+    w = gen.Workload("agree_gelu", gen.GELU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform",
+                     0.999, seed=25, lr_lo=0.002, lr_hi=0.02)
+    x = gen.generate(w, m0_scale=0.5)
+    d = device_inputs(w, x)
+    o1, W1, M1, _ = run_fwd(E, w, d)
+    buf = torch.empty(d["q"].numel() + 1, dtype=torch.bfloat16, device="cuda")
+    qu = buf[1:].view_as(d["q"])
+    qu.copy_(d["q"])
+    d2 = dict(d)
+    d2["q"] = qu
+    o2, W2, M2, _ = run_fwd(E, w, d2)
+    errs = (err(host(o1), host(o2)), err(host(W1), host(W2)), err(host(M1), host(M2)))
+    print(f"\ngelu tensor-core vs CUDA-core: {errs}")
+    assert max(errs) < 2e-2, errs
