@@ -71,7 +71,7 @@ typedef enum {
 
 /* Fast weight f_W: LINEAR W x; SWIGLU W2 (silu(W1 x) * (W3 x)); GELU_MLP
  * W2 gelu(W1 x) with the exact GELU z Phi(z) (the MLP variant, "E2-TTT_MLP" in
- * the atlas.scime.ai summary, "Key results"; forward only). */
+ * the atlas.scime.ai summary, "Key results"). */
 typedef enum { E2TTT_LINEAR = 0, E2TTT_SWIGLU = 1, E2TTT_GELU_MLP = 2 } e2ttt_fast_kind;
 typedef enum { E2TTT_F32 = 0, E2TTT_BF16 = 1 } e2ttt_dtype;
 typedef enum { E2TTT_LOSS_MSE = 0, E2TTT_LOSS_NEG_DOT = 1 } e2ttt_loss;
@@ -192,7 +192,9 @@ e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
  *   Outputs: dq, dk, dv (act dtype), dlr, dmom, ddecay (fp32 [B,H,T]),
  *            dW0, dM0 (fp32 [B,H,S]).
  *   No-momentum mode: mom, dM_end, dmom and dM0 must be NULL.
- *   E2TTT_GELU_MLP returns E2TTT_ERR_UNSUPPORTED (forward only). */
+ *   Paths: the SwiGLU backward with bf16 activations (shapes as for the
+ *   forward's tensor-core path) runs on the tensor cores; the GELU MLP, the
+ *   linear fast weight and fp32 activations run on fp32 CUDA cores. */
 e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
                                   const void* q, const void* k, const void* v,
                                   const float* lr, const float* mom, const float* decay,

@@ -658,7 +658,7 @@ def chunk_kernels_vjp(eta, mu, lam, abar, bbar, PUbar, PLbar, cbar):
 
 
 def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_end=None,
-               d_h=0, loss=LOSS_MSE, heads=None, coef=COEF_PER_TOKEN):
+               d_h=0, loss=LOSS_MSE, heads=None, coef=COEF_PER_TOKEN, starts=None):
     """Adjoint of closed_fwd, chunk by chunk in reverse. With D_W, D_M the
     adjoints of the chunk-end states and G_t = a_t D_M + b_t D_W:
         dM0 = P_U D_M + c D_W
@@ -667,7 +667,10 @@ def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_e
         PUbar = <D_M, M0>,  PLbar = <D_W, W0>,  cbar = <D_W, M0>
     then chunk_kernels_vjp gives the gate gradients. For the chunk-averaged
     variant every token's a_t is the mean of the per-token kernels, so each
-    per-token kernel receives the mean of abar (and of bbar) before the VJP."""
+    per-token kernel receives the mean of abar (and of bbar) before the VJP.
+    ``starts`` [n_chunks,B,H,2,S] optionally gives the chunk-start states to
+    differentiate at (the backward's saved-state input) instead of recomputing
+    them from W0, M0."""
     q, k, v, lr, mom, decay, W0, M0, dout = map(_f64, (q, k, v, lr, mom, decay, W0, M0, dout))
     B, H, T = lr.shape
     d_k, d_v, S = _dims(kind, q, v, W0, d_h)
@@ -677,8 +680,11 @@ def closed_bwd(kind, q, k, v, lr, mom, decay, W0, M0, C, dout, dW_end=None, dM_e
     res = {n: np.zeros(x.shape) for n, x in
            (("dq", q), ("dk", k), ("dv", v), ("dlr", lr), ("dmom", mom), ("ddecay", decay),
             ("dW0", W0), ("dM0", M0))}
-    _, _, _, starts = closed_fwd(kind, q, k, v, lr, mom, decay, W0, M0, C, d_h, loss,
-                                 return_starts=True, heads=heads, coef=coef)
+    if starts is None:
+        _, _, _, starts = closed_fwd(kind, q, k, v, lr, mom, decay, W0, M0, C, d_h, loss,
+                                     return_starts=True, heads=heads, coef=coef)
+    else:
+        starts = _f64(starts)
     hl = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
     for (b, h) in hl:
         DW = dW_end[b, h].copy()

@@ -356,8 +356,6 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* s, const void* q, const voi
                   {ws, need, "workspace"}};
   if (!check_overlaps(in, 10, outr, 9, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
   if (d.nomom) dM0 = (float*)((char*)ws + dm_off);  // zero momentum adjoint, kept internal
-  if (d.kind == E2TTT_GELU_MLP)
-    return fail(E2TTT_ERR_UNSUPPORTED, "the backward of the GELU MLP fast weight is not implemented");
   BwdArgs A{d, q, k, v, lr, mom, decay, saved, dout, dW_end, dM_end, dq, dk, dv,
             dlr, dmom, ddecay, dW0, dM0, ws, (cudaStream_t)stream};
   cudaError_t e = bf ? bwd_run<bf16>(A) : bwd_run<float>(A);

@@ -20,6 +20,12 @@
 //   h1b = dh1b du h3 s'' + sb s',  dv = -eb,
 //   dk = -(G1^T dh1 + G3^T dh3) + W1^T h1b + W3^T h3b,
 //   dW2 += e dub^T + eb u^T (MSE),  dW1 += h1b k^T,  dW3 += h3b k^T.
+// GELU MLP (h = W1 k, u = gelu(h), dh = du gelu'(h)), with P1 = G1 k, P2 = G2 u:
+//   dhb = -P1, dub = dhb gelu'(h), eb = W2 dub - P2, ub = -G2^T e + W2^T eb (MSE),
+//   hb = dhb du gelu''(h) + ub gelu'(h), dv = -eb, dk = -G1^T dh + W1^T hb,
+//   dW2 += e dub^T + eb u^T (MSE), dW1 += hb k^T.
+// Both MLPs share the code below with nf = 2 (SwiGLU: h1 | h3) or 1 (GELU: h)
+// activation factors per hidden unit.
 #include <stdint.h>
 
 #include <initializer_list>
@@ -55,17 +61,18 @@ BwdWs bwd_layout(const Dims& d) {
   L.bbar = take(BH * d.T);
   L.sbar = take(3 * BH * d.NC);
   L.part = take(3 * BH * 64);
-  if (d.kind == 1) {
-    L.H = take(BH * 2 * C * 2 * dh);
+  if (d.kind != 0) {
+    const size_t nf = d.kind == 1 ? 2 : 1;
+    L.H = take(BH * 2 * C * nf * dh);
     L.E = take(BH * C * dv);
     L.dA = take(BH * C * dh);
-    L.P = take(BH * C * 4 * dh);
+    L.P = take(BH * C * 2 * nf * dh);
     L.P2 = take(BH * C * 2 * dv);
     L.UB = take(BH * C * 2 * dh);
     L.DUB = take(BH * C * dh);
     L.EB = take(BH * C * dv);
     L.UB5 = take(BH * C * dh);
-    L.HB = take(BH * 2 * C * 2 * dh);
+    L.HB = take(BH * 2 * C * nf * dh);
   } else {
     L.E = take(BH * C * dv);
     L.P = take(BH * C * 2 * dv);
@@ -94,12 +101,22 @@ struct Bwd {
   __device__ __forceinline__ const float* w0(int z) const { return W0 + z * sst; }
   __device__ __forceinline__ const float* dWp(int z) const { return DW + z * d.S; }
   __device__ __forceinline__ const float* dMp(int z) const { return DM + z * d.S; }
-  // SwiGLU key-row quantities at (t, j)
+  // activation factors per hidden unit (SwiGLU h1 | h3: 2, GELU h: 1) and the
+  // row width nf d_h of H and HB
+  __device__ __forceinline__ int nf() const { return d.kind == 2 ? 1 : 2; }
+  __device__ __forceinline__ int hw() const { return nf() * d.d_h; }
+  // key-row quantities at (t, j): h1 (GELU: h), h3 (SwiGLU only), the activation u
   __device__ __forceinline__ float h1k(int z, int t, int j) const {
-    return H[((size_t)z * 2 * d.C + n + t) * 2 * d.d_h + j];
+    return H[((size_t)z * 2 * d.C + n + t) * hw() + j];
   }
   __device__ __forceinline__ float h3k(int z, int t, int j) const {
-    return H[((size_t)z * 2 * d.C + n + t) * 2 * d.d_h + d.d_h + j];
+    return H[((size_t)z * 2 * d.C + n + t) * hw() + d.d_h + j];
+  }
+  __device__ __forceinline__ float act_row(const float* h, int j) const {
+    return d.kind == 2 ? gelu_f(h[j]) : silu_f(h[j]) * h[d.d_h + j];
+  }
+  __device__ __forceinline__ float uk(int z, int t, int j) const {
+    return act_row(H + ((size_t)z * 2 * d.C + n + t) * hw(), j);
   }
 };
 
@@ -136,7 +153,7 @@ template <typename TA> struct LState {  // B(kk, col) = state matrix [kk][col] o
 };
 template <typename TA> struct LActK {  // u of key rows (t, j) from H
   Bwd<TA> c;
-  __device__ float operator()(int z, int t, int j) const { return silu_f(c.h1k(z, t, j)) * c.h3k(z, t, j); }
+  __device__ float operator()(int z, int t, int j) const { return c.uk(z, t, j); }
 };
 // B(kk, col) over [DM rows | DW rows] of a block with row length ld: col < half -> DM
 template <typename TA> struct LDirT {
@@ -193,13 +210,18 @@ template <typename TA> struct EEb {
     c.dv[c.tok(z, t) * dv + col] = from_f<TA>(-eb);
   }
 };
-// query rows: ub_q = dout W2 -> h1b_q = ub h3 s', h3b_q = ub s (rows [0, C) of HB)
+// query rows: ub_q = dout W2 -> h1b_q = ub h3 s', h3b_q = ub s (GELU: hb_q = ub
+// gelu'(h)) (rows [0, C) of HB)
 template <typename TA> struct EQrows {
   Bwd<TA> c;
   __device__ void operator()(int z, int t, int j, const float* acc) const {
     const int dh = c.d.d_h;
-    const float* h = c.H + ((size_t)z * 2 * c.d.C + t) * 2 * dh;
-    float* o = c.HB + ((size_t)z * 2 * c.d.C + t) * 2 * dh;
+    const float* h = c.H + ((size_t)z * 2 * c.d.C + t) * c.hw();
+    float* o = c.HB + ((size_t)z * 2 * c.d.C + t) * c.hw();
+    if (c.d.kind == 2) {
+      o[j] = acc[0] * dgelu_f(h[j]);
+      return;
+    }
     o[j] = acc[0] * h[dh + j] * dsilu_f(h[j]);
     o[dh + j] = acc[0] * silu_f(h[j]);
   }
@@ -218,29 +240,34 @@ template <typename TA> struct EdW {
 };
 
 // ------------------------------------------------------------------ SwiGLU stacked loaders
-// dk: A(t, kk') over [-a dh1 | -a dh3 | -b dh1 | -b dh3 | h1b | h3b] (6 d_h)
+// dk: A(t, kk') over [-a dh1 | -a dh3 | -b dh1 | -b dh3 | h1b | h3b] (6 d_h;
+// GELU: [-a dh | -b dh | hb], 3 d_h)
 template <typename TA> struct LdkA {
   Bwd<TA> c;
   __device__ float operator()(int z, int t, int kk) const {
-    const int dh = c.d.d_h;
+    const int dh = c.d.d_h, nf = c.nf();
     const int seg = kk / dh, j = kk - seg * dh;
-    if (seg >= 4) return c.HB[((size_t)z * 2 * c.d.C + c.d.C + t) * 2 * dh + (seg - 4) * dh + j];
-    const float h1 = c.h1k(z, t, j), h3 = c.h3k(z, t, j);
+    if (seg >= 2 * nf)
+      return c.HB[((size_t)z * 2 * c.d.C + c.d.C + t) * c.hw() + (seg - 2 * nf) * dh + j];
+    const float h1 = c.h1k(z, t, j);
     const float du = c.dA[((size_t)z * c.d.C + t) * dh + j];
-    const float dh_ = (seg & 1) ? du * silu_f(h1) : du * h3 * dsilu_f(h1);
-    const float sc = seg < 2 ? c.coef_a(z, t) : c.coef_b(z, t);
+    float dh_;
+    if (nf == 1) dh_ = du * dgelu_f(h1);
+    else dh_ = (seg & 1) ? du * silu_f(h1) : du * c.h3k(z, t, j) * dsilu_f(h1);
+    const float sc = seg < nf ? c.coef_a(z, t) : c.coef_b(z, t);
     return -sc * dh_;
   }
 };
-// dk: B(kk', col) over [DM1; DM3; DW1; DW3; W1; W3] rows (each d_h x d_k)
+// dk: B(kk', col) over [DM1; DM3; DW1; DW3; W1; W3] rows (each d_h x d_k; GELU:
+// [DM1; DW1; W1])
 template <typename TA> struct LdkB {
   Bwd<TA> c;
   __device__ float operator()(int z, int kk, int col) const {
-    const int dh = c.d.d_h, dk = c.d.d_k;
+    const int dh = c.d.d_h, dk = c.d.d_k, nf = c.nf();
     const int seg = kk / dh, j = kk - seg * dh;
-    const long long o = (long long)((seg & 1) * dh + j) * dk + col;  // W1 or W3 block row j
-    if (seg < 2) return c.dMp(z)[o];
-    if (seg < 4) return c.dWp(z)[o];
+    const long long o = (long long)((seg % nf) * dh + j) * dk + col;  // W1 (or W3) block row j
+    if (seg < nf) return c.dMp(z)[o];
+    if (seg < 2 * nf) return c.dWp(z)[o];
     return c.w0(z)[o];
   }
 };
@@ -249,7 +276,7 @@ template <typename TA> struct LdW13A {
   Bwd<TA> c;
   __device__ float operator()(int z, int i, int tt) const {
     const int row = tt < c.n ? c.d.C + tt : tt - c.n;
-    return c.HB[((size_t)z * 2 * c.d.C + row) * 2 * c.d.d_h + i];
+    return c.HB[((size_t)z * 2 * c.d.C + row) * c.hw() + i];
   }
 };
 template <typename TA> struct LdW13B {  // B(t', col) = k (t' < n) or q
@@ -274,9 +301,8 @@ template <typename TA> struct LdW2B {
   __device__ float operator()(int z, int tt, int j) const {
     const int n = c.n, dh = c.d.d_h;
     if (tt < n) return c.DUB[((size_t)z * c.d.C + tt) * dh + j];
-    if (tt < 2 * n) return silu_f(c.h1k(z, tt - n, j)) * c.h3k(z, tt - n, j);
-    const float* h = c.H + ((size_t)z * 2 * c.d.C + tt - 2 * n) * 2 * dh;
-    return silu_f(h[j]) * h[dh + j];
+    if (tt < 2 * n) return c.uk(z, tt - n, j);
+    return c.act_row(c.H + ((size_t)z * 2 * c.d.C + tt - 2 * n) * c.hw(), j);
   }
 };
 
@@ -328,14 +354,21 @@ __global__ void swiglu_rows_kernel(Bwd<TA> c) {
   const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (w >= c.d.BH * c.n) return;
   const int z = w / c.n, t = w - z * c.n;
-  const int dh = c.d.d_h, dv = c.d.d_v;
-  const float* P = c.P + ((size_t)z * c.d.C + t) * 4 * dh;
+  const int dh = c.d.d_h, dv = c.d.d_v, hw = c.hw();
+  const float* P = c.P + ((size_t)z * c.d.C + t) * 2 * hw;
   const float* P2 = c.P2 + ((size_t)z * c.d.C + t) * 2 * dv;
   const float* du = c.dA + ((size_t)z * c.d.C + t) * dh;
   const float* e = c.E + ((size_t)z * c.d.C + t) * dv;
   float am = 0.f, bw = 0.f;
   for (int j = lane; j < dh; j += 32) {
-    const float h1 = c.h1k(z, t, j), h3 = c.h3k(z, t, j);
+    const float h1 = c.h1k(z, t, j);
+    if (c.d.kind == 2) {
+      const float dhj = du[j] * dgelu_f(h1);
+      am += dhj * P[j];
+      bw += dhj * P[hw + j];
+      continue;
+    }
+    const float h3 = c.h3k(z, t, j);
     const float dh1 = du[j] * h3 * dsilu_f(h1), dh3 = du[j] * silu_f(h1);
     am += dh1 * P[j] + dh3 * P[dh + j];
     bw += dh1 * P[2 * dh + j] + dh3 * P[3 * dh + j];
@@ -367,6 +400,20 @@ __global__ void swiglu_elem_kernel(Bwd<TA> c, int stage) {
     const int t = (int)(r % c.n), z = (int)(r / c.n);
     const float a = c.coef_a(z, t), b = c.coef_b(z, t);
     const size_t row = (size_t)z * c.d.C + t;
+    if (c.d.kind == 2) {  // GELU MLP
+      const float* P = c.P + row * 2 * dh;
+      const float dhb = -(a * P[j] + b * P[dh + j]);
+      const float h = c.h1k(z, t, j), gp = dgelu_f(h);
+      if (stage == 1) {
+        c.DUB[row * dh + j] = dhb * gp;
+        continue;
+      }
+      const float du = c.dA[row * dh + j];
+      float ub = -(a * c.UB[row * 2 * dh + j] + b * c.UB[row * 2 * dh + dh + j]);
+      if (c.d.loss == 0) ub += c.UB5[row * dh + j];
+      c.HB[((size_t)z * 2 * c.d.C + c.d.C + t) * dh + j] = dhb * du * d2gelu_f(h) + ub * gp;
+      continue;
+    }
     const float* P = c.P + row * 4 * dh;
     const float dh1b = -(a * P[j] + b * P[2 * dh + j]);
     const float dh3b = -(a * P[dh + j] + b * P[3 * dh + j]);
@@ -509,17 +556,19 @@ cudaError_t chunk_bwd(const Bwd<TA>& c, cudaStream_t st) {
     return simt_gemm<1>(BH, dv, dk, 2 * n, LLinDwA<TA>{c}, LLinDwB<TA>{c}, UnitScale{},
                         EdW<TA>{c, 0, dk}, st, "bwd_linear_dw");
   }
-  const long long o2 = 2LL * dh * dk;
+  const int nf = d.kind == 2 ? 1 : 2;   // activation factors per hidden unit
+  const int hw = nf * dh;                // rows of W1 (GELU) or [W1; W3]
+  const long long o2 = (long long)hw * dk;
   // recompute the forward internals at W0
-  E2_CHECK(simt_gemm<1>(BH, 2 * n, 2 * dh, dk, LX<TA>{c}, LStateT<TA>{c, 0, dk}, UnitScale{},
-                        EStore<TA>{c.H, 2 * d.C, 2 * dh}, st, "bwd_h"));
+  E2_CHECK(simt_gemm<1>(BH, 2 * n, hw, dk, LX<TA>{c}, LStateT<TA>{c, 0, dk}, UnitScale{},
+                        EStore<TA>{c.H, 2 * d.C, hw}, st, "bwd_h"));
   E2_CHECK(simt_gemm<1>(BH, n, dv, dh, LActK<TA>{c}, LStateT<TA>{c, o2, dh}, UnitScale{}, EResid<TA>{c},
                         st, "bwd_residual"));
   E2_CHECK(simt_gemm<1>(BH, n, dh, dv, LBufRow<TA>{c.E, d.C, dv}, LState<TA>{c, o2, dh}, UnitScale{},
                         EStore<TA>{c.dA, d.C, dh}, st, "bwd_da"));
   // directional products with the state adjoints
-  E2_CHECK(simt_gemm<1>(BH, n, 4 * dh, dk, LRowAct<TA>{c, c.k, dk}, LDirT<TA>{c, 0, dk, 2 * dh},
-                        UnitScale{}, EStore<TA>{c.P, d.C, 4 * dh}, st, "bwd_dir_w13"));
+  E2_CHECK(simt_gemm<1>(BH, n, 2 * hw, dk, LRowAct<TA>{c, c.k, dk}, LDirT<TA>{c, 0, dk, hw},
+                        UnitScale{}, EStore<TA>{c.P, d.C, 2 * hw}, st, "bwd_dir_w13"));
   E2_CHECK(simt_gemm<1>(BH, n, 2 * dv, dh, LActK<TA>{c}, LDirT<TA>{c, o2, dh, dv}, UnitScale{},
                         EStore<TA>{c.P2, d.C, 2 * dv}, st, "bwd_dir_w2"));
   E2_CHECK(simt_gemm<1>(BH, n, 2 * dh, dv, LBufRow<TA>{c.E, d.C, dv}, LDir<TA>{c, o2, dh, dh},
@@ -545,9 +594,9 @@ cudaError_t chunk_bwd(const Bwd<TA>& c, cudaStream_t st) {
     E2_CHECK(cudaGetLastError());
   }
   // input gradients
-  E2_CHECK(simt_gemm<1>(BH, n, dk, 6 * dh, LdkA<TA>{c}, LdkB<TA>{c}, UnitScale{},
+  E2_CHECK(simt_gemm<1>(BH, n, dk, 3 * hw, LdkA<TA>{c}, LdkB<TA>{c}, UnitScale{},
                         EActOut<TA>{c, c.dk, dk}, st, "bwd_dk"));
-  E2_CHECK(simt_gemm<1>(BH, n, dk, 2 * dh, LBufRow<TA>{c.HB, 2 * d.C, 2 * dh}, LState<TA>{c, 0, dk},
+  E2_CHECK(simt_gemm<1>(BH, n, dk, hw, LBufRow<TA>{c.HB, 2 * d.C, hw}, LState<TA>{c, 0, dk},
                         UnitScale{}, EActOut<TA>{c, c.dq, dk}, st, "bwd_dq"));
   {
     E2TTT_TRACE("bwd_dm_update", st);
@@ -555,7 +604,7 @@ cudaError_t chunk_bwd(const Bwd<TA>& c, cudaStream_t st) {
     E2_CHECK(cudaGetLastError());
   }
   // state-gradient aggregations (in place into D_W)
-  E2_CHECK(simt_gemm<1>(BH, 2 * dh, dk, 2 * n, LdW13A<TA>{c}, LdW13B<TA>{c}, UnitScale{},
+  E2_CHECK(simt_gemm<1>(BH, hw, dk, 2 * n, LdW13A<TA>{c}, LdW13B<TA>{c}, UnitScale{},
                         EdW<TA>{c, 0, dk}, st, "bwd_dw13"));
   return simt_gemm<1>(BH, dv, dh, 3 * n, LdW2A<TA>{c}, LdW2B<TA>{c}, UnitScale{}, EdW<TA>{c, o2, dh},
                       st, "bwd_dw2");

@@ -47,5 +47,9 @@ __device__ __forceinline__ float gelu_f(float z) { return z * gelu_cdf_f(z); }
 __device__ __forceinline__ float dgelu_f(float z) {
   return gelu_cdf_f(z) + z * 0.39894228040143268f * expf(-0.5f * z * z);
 }
+// gelu''(z) = phi(z) (2 - z^2)
+__device__ __forceinline__ float d2gelu_f(float z) {
+  return 0.39894228040143268f * expf(-0.5f * z * z) * (2.0f - z * z);
+}
 
 }  // namespace e2ttt

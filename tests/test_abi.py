@@ -131,14 +131,7 @@ def test_no_momentum_pointer_rules(E):
     assert E.e2ttt_state_elems(bad) == 0
 
 
-def test_gelu_mlp_state_and_backward_unsupported(E):
+def test_gelu_mlp_state_size(E):
     g = E.make_shape(1, 2, 64, 16, 8, 6, 16, E.GELU_MLP, E.F32)
     assert E.e2ttt_state_elems(g) == 16 * 8 + 6 * 16
-    n = 1 << 30
-    args = dict(q=FAKE, k=FAKE + n, v=FAKE + 2 * n, lr=FAKE + 3 * n, mom=FAKE + 4 * n,
-                decay=FAKE + 5 * n, saved_states=FAKE + 6 * n, dout=FAKE + 7 * n, dW_end=None,
-                dM_end=None, dq=FAKE + 8 * n, dk=FAKE + 9 * n, dv=FAKE + 10 * n, dlr=FAKE + 11 * n,
-                dmom=FAKE + 12 * n, ddecay=FAKE + 13 * n, dW0=FAKE + 14 * n, dM0=FAKE + 15 * n,
-                workspace=FAKE + 16 * n, workspace_bytes=E.e2ttt_workspace_bytes(g, 1))
-    assert E.e2ttt_chunk_scan_bwd(g, raw=True, stream=None, **args) == E.ERR_UNSUPPORTED
-    assert "GELU" in E.e2ttt_last_error()
+    assert E.e2ttt_workspace_bytes(g, 0) > 0 and E.e2ttt_workspace_bytes(g, 1) > 0

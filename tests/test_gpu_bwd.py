@@ -67,6 +67,11 @@ F32 = {
     "swiglu_dot": gen.Workload("bsd", gen.SWIGLU, gen.F32, 2, 1, 12, 16, 20, 48, 16, "uniform", 0.99,
                                seed=44, loss=gen.LOSS_NEG_DOT, lr_lo=0.001, lr_hi=0.005,
                                mom_lo=0.5, mom_hi=0.9),
+    "gelu_mse": gen.Workload("bg", gen.GELU, gen.F32, 1, 2, 16, 12, 24, 50, 16, "uniform", 0.99,
+                             seed=47, lr_lo=0.002, lr_hi=0.02, mom_lo=0.7, mom_hi=0.95),
+    "gelu_dot": gen.Workload("bgd", gen.GELU, gen.F32, 2, 1, 12, 16, 20, 48, 16, "uniform", 0.99,
+                             seed=48, loss=gen.LOSS_NEG_DOT, lr_lo=0.001, lr_hi=0.005,
+                             mom_lo=0.5, mom_hi=0.9),
 }
 
 
@@ -133,3 +138,26 @@ def test_bwd_tensor_core_and_cuda_core_agree(E):
     errs = {n: err(host(g_tc[n]), host(g_cc[n])) for n in NAMES}
     print("\ntensor-core vs CUDA-core backward:", " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
     assert all(e < 2e-2 for e in errs.values()), errs
+
+
+def test_bwd_gelu_bf16_small(E):
+    """The GELU MLP with bf16 activations (CUDA-core backward), against the oracle's
+    adjoint at the saved chunk-start states the GPU forward produced (an input of
+    the backward). End to end against fp64 starts the gradients of this
+    configuration move by ~0.3 under the forward's correlated bf16 state rounding
+    (the oracle's own adjoint at these states shows the same); the fp32 GELU cases
+    above check the whole path."""
+    import torch
+    w = gen.Workload("bgb", gen.GELU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform", 0.999,
+                     seed=49, lr_lo=0.002, lr_hi=0.02)
+    x = gen.generate(w, m0_scale=0.5)
+    dW, dM = gen.upstream_state_grads(w, seed=8, scale=0.1)
+    d = device_inputs(w, x)
+    _, _, _, saved = run_fwd(E, w, d, save=True)
+    g = E.chunk_scan_bwd(d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], saved, d["dout"],
+                         dev(dW), dev(dM), C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss)
+    torch.cuda.synchronize()
+    gpu = {n: host(t) for n, t in g.items()}
+    ref = O.closed_bwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"],
+                       x["M0"], w.C, x["dout"], dW, dM, d_h=w.d_h, loss=w.loss, starts=host(saved))
+    check(gpu, ref, 2e-2, label="gelu_bf16_small (oracle at the GPU's saved states)")

@@ -517,3 +517,15 @@ def test_chunk_mean_bwd_matches_fd(kind):
     # and the variant really differs from the per-token kernels
     g0 = O.closed_bwd(*args(x), x["dout"], dW, dM, d_h=w.d_h)
     assert O.rel_fro(g["dlr"], g0["dlr"]) > 1e-3
+
+
+def test_closed_bwd_given_starts_equals_recomputed():
+    """closed_bwd with starts= the states closed_fwd computes equals closed_bwd that
+    recomputes them (the option only replaces the chunk-start states)."""
+    w, x = small_case(O.GELU, B=1, H=1, T=7, C=3, d_k=4, d_v=4, d_h=6, seed=71)
+    args = (w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"], x["M0"], w.C)
+    _, _, _, st = O.closed_fwd(*args, d_h=w.d_h, return_starts=True)
+    g1 = O.closed_bwd(*args, x["dout"], d_h=w.d_h)
+    g2 = O.closed_bwd(*args, x["dout"], d_h=w.d_h, starts=st)
+    for n in g1:
+        np.testing.assert_array_equal(g1[n], g2[n])
