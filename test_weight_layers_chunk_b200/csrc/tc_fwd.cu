@@ -413,20 +413,36 @@ struct EpiG3 {
 // G4: accumulator 0 = dM = sum_t a_t g_t, accumulator 1 = dW = sum_t b_t g_t.
 // Class 0 covers rows of [W1; W3] (or W for linear), class 1 the rows of W2.
 // Each of the four epilogue warps owns 32 rows x 128 columns of the tile and
-// moves the fp32 state with TMA through two 10 KB slots of its shared memory:
-// the W0/M0 tiles of column group g+2 load while group g is computed; results
-// are written back into the slot (W, M fp32 and the bf16 copy of W) and stored
-// with TMA, so the state never passes through the load/store units.
+// moves the fp32 state with TMA through two 10 KB slots of its shared memory, in
+// one sequence of 32-column groups q that continues across the CTA's tiles: the
+// W0/M0 tiles of group q + 2 load into group q's slot once its stores have read
+// it, so they arrive while group q + 1 is computed (the first groups of the next
+// tile load during the last groups of this one). Results are written back into
+// the slot (W, M fp32 and the bf16 copy of W) and stored with TMA, so the state
+// never passes through the load/store units. (Three slots, which would let a
+// store's read overlap the next group's math, only fit beside a two-slot k-block
+// ring, and the shallower ring costs more than they save.)
 struct EpiG4 {
   static constexpr int kSlot = 10240;  // W 4 KB | M 4 KB | bf16 copy 2 KB
+  static constexpr int kSlots = 2;
+  static constexpr int kSmem = kSlots * kSlot;
+  static __device__ __forceinline__ void issue(const FwdP& p, const uint8_t* wsmem, uint64_t* wbar,
+                                               int q, int g, int cls, int z, int r0, int n0) {
+    const int sidx = q % kSlots;
+    uint8_t* slot = const_cast<uint8_t*>(wsmem) + sidx * kSlot;
+    const bool hasM = p.src.M != nullptr;
+    tc::mbar_expect_tx(&wbar[sidx], hasM ? 8192u : 4096u);
+    tc::tma_load_3d(slot, &p.srcW[cls], &wbar[sidx], n0 + g * 32, r0, z);
+    if (hasM) tc::tma_load_3d(slot + 4096, &p.srcM[cls], &wbar[sidx], n0 + g * 32, r0, z);
+  }
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
     const int lane = c.row & 31;
     const int r0 = c.m0 + c.quad * 32;  // first state row of this warp
     constexpr int kGroups = BN / 32;
+    static_assert(kGroups >= 2, "two groups ahead");
     const bool hasM = p.src.M != nullptr;
-    const uint32_t tx = hasM ? 8192u : 4096u;
     const size_t plane = (size_t)d.BH * d.NC;
     const size_t so = (size_t)c.z * d.NC + p.ci;
     const float PU = p.scal[so], PL = p.scal[plane + so], cc = p.scal[2 * plane + so];
@@ -439,28 +455,25 @@ struct EpiG4 {
     } else {
       sh_row = c.z * d.d_v + r0;
     }
-    auto issue = [&](int g) {  // lane 0: TMA loads of column group g into slot g & 1
-      const int sidx = g & 1;
-      uint8_t* slot = c.wsmem + sidx * kSlot;
-      tc::mbar_expect_tx(&c.wbar[sidx], tx);
-      tc::tma_load_3d(slot, &p.srcW[c.cls], &c.wbar[sidx], c.n0 + g * 32, r0, c.z);
-      if (hasM) tc::tma_load_3d(slot + 4096, &p.srcM[c.cls], &c.wbar[sidx], c.n0 + g * 32, r0, c.z);
-    };
-    if (lane == 0) {
-      tc::bulk_wait_read<0>();  // the previous tile's stores no longer read our slots
-      issue(0);
-      if (kGroups > 1) issue(1);
+    const int q0 = c.iter * kGroups;
+    if (c.iter == 0 && lane == 0) {
+      issue(p, c.wsmem, c.wbar, q0, 0, c.cls, c.z, r0, c.n0);
+      issue(p, c.wsmem, c.wbar, q0 + 1, 1, c.cls, c.z, r0, c.n0);
     }
     __syncwarp();
     for (int g = 0; g < kGroups; ++g) {
-      const int sidx = g & 1;
+      const int q = q0 + g, sidx = q % kSlots;
       uint8_t* slot = c.wsmem + sidx * kSlot;
       float dM[32], dW[32];
       ld2(c, 0, g * 32, 1, g * 32, dM, dW);
       const bool ok = tc::mbar_wait(&c.wbar[sidx], c.uses[sidx] & 1u);
       c.uses[sidx] += 1;
       if (!ok) {
-        if (lane == 0) atomicExch(p.status, tc2::kErrEpilogue);
+        if (lane == 0) {
+          atomicExch(p.status, tc2::kErrEpilogue);
+          const int s1 = (q + 1) % kSlots;  // group q + 1's loads may still be in flight
+          if (g + 1 < kGroups || c.nxt_valid) (void)tc::mbar_wait(&c.wbar[s1], c.uses[s1] & 1u);
+        }
         return;
       }
       // row `lane` of the 128B-swizzled fp32 tiles; 64B-swizzled bf16 row
@@ -468,22 +481,22 @@ struct EpiG4 {
       uint8_t* mrow = slot + 4096 + lane * 128;
       uint8_t* srow = slot + 8192 + lane * 64;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int off = (q ^ (lane & 7)) << 4;
+      for (int k = 0; k < 8; ++k) {
+        const int off = (k ^ (lane & 7)) << 4;
         const float4 w = *reinterpret_cast<const float4*>(wrow + off);
         const float4 m = hasM ? *reinterpret_cast<const float4*>(mrow + off) : make_float4(0.f, 0.f, 0.f, 0.f);
         float4 wn, mn;
-        mn.x = PU * m.x - dM[4 * q + 0];
-        mn.y = PU * m.y - dM[4 * q + 1];
-        mn.z = PU * m.z - dM[4 * q + 2];
-        mn.w = PU * m.w - dM[4 * q + 3];
-        wn.x = PL * w.x + cc * m.x - dW[4 * q + 0];
-        wn.y = PL * w.y + cc * m.y - dW[4 * q + 1];
-        wn.z = PL * w.z + cc * m.z - dW[4 * q + 2];
-        wn.w = PL * w.w + cc * m.w - dW[4 * q + 3];
+        mn.x = PU * m.x - dM[4 * k + 0];
+        mn.y = PU * m.y - dM[4 * k + 1];
+        mn.z = PU * m.z - dM[4 * k + 2];
+        mn.w = PU * m.w - dM[4 * k + 3];
+        wn.x = PL * w.x + cc * m.x - dW[4 * k + 0];
+        wn.y = PL * w.y + cc * m.y - dW[4 * k + 1];
+        wn.z = PL * w.z + cc * m.z - dW[4 * k + 2];
+        wn.w = PL * w.w + cc * m.w - dW[4 * k + 3];
         *reinterpret_cast<float4*>(wrow + off) = wn;
         *reinterpret_cast<float4*>(mrow + off) = mn;
-        *reinterpret_cast<uint2*>(srow + ((((q >> 1) ^ ((lane >> 1) & 3)) << 4) | ((q & 1) << 3))) =
+        *reinterpret_cast<uint2*>(srow + ((((k >> 1) ^ ((lane >> 1) & 3)) << 4) | ((k & 1) << 3))) =
             make_uint2(pack2(wn.x, wn.y), pack2(wn.z, wn.w));
       }
       tc::fence_async_smem();
@@ -493,9 +506,13 @@ struct EpiG4 {
         tc::tma_store_3d(&p.dstM[c.cls], slot + 4096, c.n0 + g * 32, r0, c.z);
         if (p.write_shadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 8192, c.n0 + g * 32, sh_row);
         tc::bulk_commit();
-        if (g + 2 < kGroups) {
-          tc::bulk_wait_read<0>();  // slot reused for group g + 2
-          issue(g + 2);
+        tc::bulk_wait_read<0>();  // group q's stores have read the slot of group q + 2
+        const int gn = g + 2;
+        if (gn < kGroups) {
+          issue(p, c.wsmem, c.wbar, q + 2, gn, c.cls, c.z, r0, c.n0);
+        } else if (c.nxt_valid) {
+          issue(p, c.wsmem, c.wbar, q + 2, gn - kGroups, c.nxt_cls, c.nxt_z,
+                c.nxt_m0 + c.quad * 32, c.nxt_n0);
         }
       }
       __syncwarp();
@@ -953,13 +970,13 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
       }
       if (e == cudaSuccess) {
         e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)
-                    : launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
+                    : launch<128, 2, true, true, 3, EpiG4, 4, EpiG4::kSmem>(g4, p, st);
       }
     } else {
       e = launch<128, 1, false, false, 4, EpiG1Lin, kEpiWarps, EpiG1Lin::kSmem>(g1, p, st);
       if (e == cudaSuccess) {
         e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)
-                    : launch<128, 2, true, true, 3, EpiG4, 4, 2 * EpiG4::kSlot>(g4, p, st);
+                    : launch<128, 2, true, true, 3, EpiG4, 4, EpiG4::kSmem>(g4, p, st);
       }
     }
     if (e != cudaSuccess) return e;
