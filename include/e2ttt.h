@@ -144,10 +144,12 @@ e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* shape,
  *            chunk), saved_states (may be NULL; needed by the backward).
  *   No-momentum mode (shape->momentum = E2TTT_NO_MOMENTUM): mom, M0 and M_end
  *   must be NULL; saved_states then hold W and a zero M for every chunk.
- *   Paths: bf16 activations with T % C == 0, C % 128 == 0, d_k % 64 == 0,
- *   d_v % 64 == 0 (and d_h % 128 == 0 for SwiGLU) run on the tcgen05 tensor
- *   cores (bf16 operands, fp32 accumulation and state); every other shape and
- *   fp32 activations run on fp32 CUDA-core kernels. */
+ *   Paths: bf16 activations with C % 128 == 0 and d_k, d_v (and d_h for the
+ *   SwiGLU and GELU MLPs) multiples of 128 run on the tcgen05 tensor cores
+ *   (bf16 operands, fp32 accumulation and state); a shorter last chunk
+ *   (T % C != 0) runs there padded to C tokens, its padding rows adding
+ *   nothing. Every other shape and fp32 activations run on fp32 CUDA-core
+ *   kernels. */
 e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* shape,
                                   const void* q, const void* k, const void* v,
                                   const float* lr, const float* mom, const float* decay,
@@ -193,7 +195,8 @@ e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
  *            dW0, dM0 (fp32 [B,H,S]).
  *   No-momentum mode: mom, dM_end, dmom and dM0 must be NULL.
  *   Paths: the SwiGLU backward with bf16 activations (shapes as for the
- *   forward's tensor-core path) runs on the tensor cores; the GELU MLP, the
+ *   forward's tensor-core path, a shorter last chunk included) runs on the
+ *   tensor cores; the GELU MLP, the
  *   linear fast weight and fp32 activations run on fp32 CUDA cores. */
 e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
                                   const void* q, const void* k, const void* v,

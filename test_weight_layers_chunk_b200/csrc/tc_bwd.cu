@@ -35,8 +35,14 @@ struct BwdP {
   // 32 x 32 boxes for the epilogues' TMA-staged I/O (bf16: 64B swizzle, fp32: 128B)
   CUtensorMap mHc, mY3, mDH, mHB, fdu, fDB, fUBd;
   CUtensorMap mZ3, mv, mdv, mdk, mdq, fG2U, fdkp, fDW[2];
+  // mv, mdv, mdk, mdq are 3-D (columns, tokens, heads): a box past a head's last
+  // token reads as zero and is clipped on store
   Dims d;
   int ci, t0;
+  // tokens of this chunk: C, or T - t0 for a shorter last chunk, whose padding
+  // rows carry zero keys, queries, dout and v and a_t = b_t = 0, so every
+  // per-token term of theirs vanishes
+  int clen;
   const bf16 *v;
   bf16 *dq, *dk, *dv;
   const float *ca, *cb, *scal;
@@ -209,7 +215,7 @@ struct EpiR2 {
     const GroupAt ga = group_at(c, gi);
     if (!ga.valid) return;
     tc::mbar_expect_tx(&c.wbar[0], 2048u);
-    tc::tma_load_2d(c.wsmem, &p.mv, &c.wbar[0], ga.col, ga.z * p.d.T + p.t0 + ga.m0 + c.quad * 32);
+    tc::tma_load_3d(c.wsmem, &p.mv, &c.wbar[0], ga.col, p.t0 + ga.m0 + c.quad * 32, ga.z);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -322,7 +328,7 @@ struct EpiD1 {
     const int per = BN / c.nparts, ngroups = per / 32;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-    const float a = p.ca[tok], b = p.cb[tok];
+    const float a = t < p.clen ? p.ca[tok] : 0.f, b = t < p.clen ? p.cb[tok] : 0.f;
     const int yD = c.z * d.C + c.m0 + c.quad * 32;
     float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG;
     float* pb = pa + (size_t)d.BH * d.C * p.NG;
@@ -380,7 +386,7 @@ struct EpiD2 {
     const int per = BN / c.nparts, ngroups = per / 32;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-    const float a = p.ca[tok], b = p.cb[tok];
+    const float a = t < p.clen ? p.ca[tok] : 0.f, b = t < p.clen ? p.cb[tok] : 0.f;
     const int yG = c.z * d.C + c.m0 + c.quad * 32;
     float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG + 2 * d.d_h / 32;
     float* pb = pa + (size_t)d.BH * d.C * p.NG;
@@ -445,7 +451,7 @@ struct EpiE3 {
     const int per = BN / c.nparts, ngroups = per / 32;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-    const float a = p.ca[tok], b = p.cb[tok];
+    const float a = t < p.clen ? p.ca[tok] : 0.f, b = t < p.clen ? p.cb[tok] : 0.f;
     const int r0 = c.m0 + c.quad * 32;
     const uint8_t* IN = c.wsmem;
     uint8_t* F = c.wsmem + kIn;
@@ -504,7 +510,8 @@ struct EpiE4 {
     const int lane = c.row & 31;
     const int per = BN / c.nparts, ngroups = per / 32;
     const int r0 = c.m0 + c.quad * 32;
-    const int yV = c.z * d.T + p.t0 + r0, yB = c.z * 3 * d.C + d.C + r0;
+    const int tV = p.t0 + r0, yB = c.z * 3 * d.C + d.C + r0;
+    const bool any_real = r0 < p.clen;
     const uint8_t* IN = c.wsmem;
     uint8_t* OUT = c.wsmem + kIn;
     if (c.iter == 0 && lane == 0) issue(p, c, 0);
@@ -534,7 +541,7 @@ struct EpiE4 {
       stage_h(OUT + 2048, lane, eb);
       out_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.mdv, OUT, col, yV);
+        if (any_real) tc::tma_store_3d(&p.mdv, OUT, col, tV, c.z);
         tc::tma_store_2d(&p.mZ3, OUT + 2048, col, yB);
         tc::bulk_commit();
       }
@@ -699,7 +706,7 @@ struct EpiDk1 {
     const int lane = c.row & 31;
     const int t = c.m0 + c.row;
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
-    const float a = p.ca[tok], b = p.cb[tok];
+    const float a = t < p.clen ? p.ca[tok] : 0.f, b = t < p.clen ? p.cb[tok] : 0.f;
     const int y = c.z * d.C + c.m0 + c.quad * 32;
     uint8_t* F = c.wsmem;
     FOR_GROUPS(c, BN, g) {
@@ -735,7 +742,8 @@ struct EpiDkq {
     const Dims& d = p.d;
     const int lane = c.row & 31;
     const int per = BN / c.nparts, ngroups = per / 32;
-    const int yO = c.z * d.T + p.t0 + c.m0 + c.quad * 32;
+    const int tO = p.t0 + c.m0 + c.quad * 32;
+    const bool any_real = c.m0 + c.quad * 32 < p.clen;
     const uint8_t* IN = c.wsmem;
     uint8_t* OUT = c.wsmem + kIn;
     if (KEYS && c.iter == 0 && lane == 0) issue(p, c, 0);
@@ -760,7 +768,7 @@ struct EpiDkq {
       stage_h(OUT, lane, x);
       out_ready();
       if (lane == 0) {
-        tc::tma_store_2d(KEYS ? &p.mdk : &p.mdq, OUT, col, yO);
+        if (any_real) tc::tma_store_3d(KEYS ? &p.mdk : &p.mdq, OUT, col, tO, c.z);
         tc::bulk_commit();
       }
       __syncwarp();
@@ -913,10 +921,12 @@ __global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* 
   }
 }
 // abar_t, bbar_t = -(sum of the partial dot products), fixed order.
-__global__ void bwd_rows_kernel(const float* part, float* abar, float* bbar, Dims d, int t0, int NG) {
+__global__ void bwd_rows_kernel(const float* part, float* abar, float* bbar, Dims d, int t0, int clen,
+                                int NG) {
   const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= (long long)d.BH * d.C) return;
   const int z = (int)(r / d.C), t = (int)(r % d.C);
+  if (t >= clen) return;  // padding of a shorter last chunk
   const float* pa = part + (size_t)r * NG;
   const float* pb = pa + (size_t)d.BH * d.C * NG;
   float sa = 0.f, sb = 0.f;
@@ -970,6 +980,19 @@ bool box32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, bool 
   return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
             const_cast<void*>(base), dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE,
             f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3-D bf16 map over per-head token rows [heads][T][cols], box 32 x 32 x 1, 64B
+// swizzle: rows past a head's T read as zero and are clipped on store.
+bool tok_box32(CUtensorMap* m, const void* base, uint64_t T, uint64_t cols, uint64_t heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, T, heads};
+  cuuint64_t strides[2] = {cols * 2, T * cols * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t el[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, el,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 // 3-D fp32 map over [heads, rows, cols] of one block of every head's state
@@ -1124,12 +1147,11 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     mok &= box32(&p.fdu, B.du, rC, dh, true);
     mok &= box32(&p.fDB, B.DB, rC, 2 * dh, true);
     mok &= box32(&p.fUBd, B.UBd, rC, dh, true);
-    const uint64_t rT = (uint64_t)BH * T;
     mok &= box32(&p.mZ3, B.Z3, 3 * rC, dv, false);
-    mok &= box32(&p.mv, A.v, rT, dv, false);
-    mok &= box32(&p.mdv, A.dv, rT, dv, false);
-    mok &= box32(&p.mdk, A.dk, rT, dk, false);
-    mok &= box32(&p.mdq, A.dq, rT, dk, false);
+    mok &= tok_box32(&p.mv, A.v, T, dv, BH);
+    mok &= tok_box32(&p.mdv, A.dv, T, dv, BH);
+    mok &= tok_box32(&p.mdk, A.dk, T, dk, BH);
+    mok &= tok_box32(&p.mdq, A.dq, T, dk, BH);
     mok &= box32(&p.fG2U, B.G2U, rC, dv, true);
     mok &= box32(&p.fdkp, B.dkp, rC, dk, true);
     mok &= state_box32(&p.fDW[0], A.dW0, 2 * dh, dk, BH, d.S);
@@ -1211,21 +1233,32 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   const Dims dd = d;
   for (int ci = NC - 1; ci >= 0; --ci) {
     const int t0 = ci * C;
+    const int cl = T - t0 < C ? T - t0 : C;  // tokens of this chunk
     p.ci = ci;
     p.t0 = t0;
+    p.clen = cl;
     const float* W0 = A.saved + ci * per_chunk;
     const float* M0 = W0 + d.S;
-    // chunk rows of keys, queries, dout into the stacked operands
+    // chunk rows of keys, queries, dout into the stacked operands (zero padding
+    // rows after a shorter last chunk's tokens)
     e = cudaMemcpy2DAsync(B.X, (size_t)2 * C * dk * 2, (const bf16*)A.k + (size_t)t0 * dk,
-                          (size_t)T * dk * 2, (size_t)C * dk * 2, BH, cudaMemcpyDeviceToDevice, st);
+                          (size_t)T * dk * 2, (size_t)cl * dk * 2, BH, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess)
       e = cudaMemcpy2DAsync(B.X + (size_t)C * dk, (size_t)2 * C * dk * 2,
-                            (const bf16*)A.q + (size_t)t0 * dk, (size_t)T * dk * 2, (size_t)C * dk * 2,
+                            (const bf16*)A.q + (size_t)t0 * dk, (size_t)T * dk * 2, (size_t)cl * dk * 2,
                             BH, cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess)
       e = cudaMemcpy2DAsync(B.Z3 + (size_t)2 * C * dv, (size_t)3 * C * dv * 2,
                             (const bf16*)A.dout + (size_t)t0 * dv, (size_t)T * dv * 2,
-                            (size_t)C * dv * 2, BH, cudaMemcpyDeviceToDevice, st);
+                            (size_t)cl * dv * 2, BH, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess && cl < C) {
+      const size_t pk = (size_t)(C - cl) * dk * 2, pv = (size_t)(C - cl) * dv * 2;
+      e = cudaMemset2DAsync(B.X + (size_t)cl * dk, (size_t)2 * C * dk * 2, 0, pk, BH, st);
+      if (e == cudaSuccess)
+        e = cudaMemset2DAsync(B.X + (size_t)(C + cl) * dk, (size_t)2 * C * dk * 2, 0, pk, BH, st);
+      if (e == cudaSuccess)
+        e = cudaMemset2DAsync(B.Z3 + (size_t)(2 * C + cl) * dv, (size_t)3 * C * dv * 2, 0, pv, BH, st);
+    }
     if (e != cudaSuccess) return e;
     {
       E2TTT_TRACE("tcb_shadow", st);
@@ -1252,7 +1285,8 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     {
       E2TTT_TRACE("tcb_rows", st);
       const long long rows = (long long)BH * C;
-      bwd_rows_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(B.part, B.abar, B.bbar, dd, t0, p.NG);
+      bwd_rows_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(B.part, B.abar, B.bbar, dd, t0,
+                                                                         cl, p.NG);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }

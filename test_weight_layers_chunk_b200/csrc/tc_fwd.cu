@@ -39,10 +39,13 @@ struct FwdP {
   // and the bf16 operand copies it writes; index = tile class (0: [W1; W3] or W,
   // 1: W2). Rebuilt for every chunk.
   CUtensorMap srcW[2], srcM[2], dstW[2], dstM[2], shadow[2];
-  // 32 x 32 bf16 tiles (64B swizzle) moved by the other epilogues
+  // 32 x 32 bf16 tiles (64B swizzle) moved by the other epilogues; mOut and mV
+  // are 3-D (columns, tokens, heads), so a box past a head's last token is
+  // clipped on store and reads as zero
   CUtensorMap mA, mSk, mOut, mV, mE, mEa, mEb, mdH;
   Dims d;
   int ci, t0, write_shadow;
+  int clen;   // tokens of this chunk: C, or T - t0 for a shorter last chunk
   int nomom;  // no momentum: no a-scaled operands, W-only aggregation epilogue
   int* status;
   const bf16 *q, *k, *v;
@@ -271,19 +274,23 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
   const int ngroups = per / 32;
   uint8_t* V = c.wsmem;            // [2][2 KB]
   uint8_t* S = c.wsmem + 4096;     // E | Ea | Eb staging
-  const int ytok = c.z * d.T + p.t0 + r0;
+  const int ttok = p.t0 + r0;      // first token (within the head) of this warp's rows
   const int yrow = c.z * d.C + r0;
+  // Rows at or past the chunk's length (a shorter last chunk) are padding: no
+  // output, and E = a E = b E = 0, so they add nothing to any later sum over tokens.
+  const bool real = lane < p.clen - r0;
+  if (!key_rows && p.clen - r0 <= 0) return;  // no query row of this warp is real
   if (key_rows) {
     if (lane == 0) {
       tc::mbar_expect_tx(&c.wbar[0], 2048u * ngroups);
       for (int gi = 0; gi < ngroups; ++gi)
-        tc::tma_load_2d(V + gi * 2048, &p.mV, &c.wbar[0], col0 + gi * 32, ytok);
+        tc::tma_load_3d(V + gi * 2048, &p.mV, &c.wbar[0], col0 + gi * 32, ttok, c.z);
     }
     __syncwarp();
   }
   float at = 0.f, bt = 0.f;
-  if (key_rows) {
-    const size_t tok = (size_t)ytok + lane;
+  if (key_rows && real) {
+    const size_t tok = (size_t)c.z * d.T + ttok + lane;
     at = p.ca[tok];
     bt = p.cb[tok];
   }
@@ -296,7 +303,7 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
       stage32(S, lane, y);
       staging_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.mOut, S, col, ytok);
+        tc::tma_store_3d(&p.mOut, S, col, ttok, c.z);
         tc::bulk_commit();
       }
       __syncwarp();
@@ -313,7 +320,7 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
     float vv[32];
     unstage32(V + gi * 2048, lane, vv);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = d.loss == 0 ? y[i] - vv[i] : -vv[i];
+    for (int i = 0; i < 32; ++i) y[i] = !real ? 0.f : d.loss == 0 ? y[i] - vv[i] : -vv[i];
     staging_free(lane);
     if (write_e) stage32(S, lane, y);
     if (!p.nomom) {
@@ -723,6 +730,20 @@ bool make_state_map(CUtensorMap* m, const float* base, uint64_t rows, uint64_t c
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over per-head token rows [heads][T][cols], box 32 x 32 x 1, 64B
+// swizzle: rows past a head's T are clipped on stores and read as zero on loads.
+bool make_tok_map_box32(CUtensorMap* m, const void* base, uint64_t T, uint64_t cols, uint64_t heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, T, heads};
+  cuuint64_t strides[2] = {cols * 2, T * cols * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 map, box 32 columns x 32 rows, 64B swizzle (epilogue stores).
 bool make_map_box32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   EncodeTiledFn fn = encode_fn();
@@ -794,7 +815,7 @@ size_t carve(const Dims& d, char* base, Scratch* s) {
 
 bool tc_fwd_supported(const Dims& d, bool bf16_act) {
   if (!bf16_act) return false;
-  if (d.T % d.C != 0 || d.C % 128 != 0) return false;
+  if (d.C % 128 != 0) return false;  // a shorter last chunk runs padded to C tokens
   if (d.d_k % 128 != 0 || d.d_v % 128 != 0) return false;
   if (d.kind != 0 && d.d_h % 128 != 0) return false;
   return encode_fn() != nullptr;
@@ -920,8 +941,8 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     }
   }
   // 32 x 32 tiles of the epilogues (bf16, 64B swizzle)
-  ok &= make_map_box32(&p.mOut, out, (uint64_t)BH * T, dv);
-  ok &= make_map_box32(&p.mV, v, (uint64_t)BH * T, dv);
+  ok &= make_tok_map_box32(&p.mOut, out, T, dv, BH);
+  ok &= make_tok_map_box32(&p.mV, v, T, dv, BH);
   ok &= make_map_box32(&p.mEa, s.Ea, (uint64_t)BH * C, dv);
   ok &= make_map_box32(&p.mEb, s.Eb, (uint64_t)BH * C, dv);
   if (d.kind != 0) {
@@ -935,6 +956,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   for (int ci = 0; ci < NC; ++ci) {
     p.ci = ci;
     p.t0 = ci * C;
+    p.clen = T - ci * C < C ? T - ci * C : C;
     p.write_shadow = ci + 1 < NC;
     chunk_states(d, ci, W0, M0, W_end, M_end, saved, &p.src, &p.dst);
     {

@@ -140,6 +140,45 @@ def test_bwd_tensor_core_and_cuda_core_agree(E):
     assert all(e < 2e-2 for e in errs.values()), errs
 
 
+@pytest.mark.parametrize("T,C,B,H", [(600, 256, 2, 2), (200, 256, 1, 3), (640, 512, 1, 2)])
+def test_bwd_bf16_shorter_last_chunk(E, T, C, B, H):
+    """SwiGLU, bf16, T % C != 0: the tensor-core forward and backward run the last
+    chunk padded to C tokens (88 real tokens in two 128-row tiles; one chunk of
+    200; one real 128-row tile of four)."""
+    w = gen.Workload("btail", gen.SWIGLU, gen.BF16, B, H, 128, 128, 256, T, C, "uniform", 0.999,
+                     seed=47 + T, lr_lo=0.002, lr_hi=0.02)
+    assert E.e2ttt_fwd_uses_tensor_cores(
+        E.make_shape(B, H, T, C, 128, 128, 256, E.SWIGLU, E.BF16)) == 1
+    x = gen.generate(w, m0_scale=0.5)
+    dW, dM = gen.upstream_state_grads(w, seed=10, scale=0.1)
+    gpu, ref = run_bwd(E, w, x, dW, dM)
+    check(gpu, ref, 2e-2, label=f"swiglu_bf16 T={T} C={C}")
+
+
+def test_bwd_shorter_last_chunk_paths_agree(E):
+    """T % C != 0 through both backward paths (the unaligned view of dout routes
+    the call to the CUDA-core backward)."""
+    import torch
+    w = gen.Workload("agreet", gen.SWIGLU, gen.BF16, 2, 2, 128, 128, 256, 600, 256, "uniform", 0.999,
+                     seed=48, lr_lo=0.002, lr_hi=0.02)
+    x = gen.generate(w, m0_scale=0.5)
+    d = device_inputs(w, x)
+    _, _, _, saved = run_fwd(E, w, d, save=True)
+    dW, dM = (dev(a) for a in gen.upstream_state_grads(w, seed=11, scale=0.1))
+    args = (d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], saved)
+    kw = dict(C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss)
+    g_tc = E.chunk_scan_bwd(*args, d["dout"], dW, dM, **kw)
+    buf = torch.empty(d["dout"].numel() + 1, dtype=torch.bfloat16, device="cuda")
+    dout_u = buf[1:].view_as(d["dout"])
+    dout_u.copy_(d["dout"])
+    g_cc = E.chunk_scan_bwd(*args, dout_u, dW, dM, **kw)
+    torch.cuda.synchronize()
+    errs = {n: err(host(g_tc[n]), host(g_cc[n])) for n in NAMES}
+    print("\nshorter last chunk, tensor-core vs CUDA-core backward:",
+          " ".join(f"{n}={e:.2e}" for n, e in errs.items()))
+    assert all(e < 2e-2 for e in errs.values()), errs
+
+
 def test_bwd_gelu_bf16_small(E):
     """The GELU MLP with bf16 activations (CUDA-core backward), against the oracle's
     adjoint at the saved chunk-start states the GPU forward produced (an input of

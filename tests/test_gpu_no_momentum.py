@@ -36,6 +36,9 @@ CASES = {
                                    "uniform", 0.999, seed=55, lr_lo=0.002, lr_hi=0.02),
     "swiglu_bf16_tc": gen.Workload("nmsb", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128,
                                    "uniform", 0.999, seed=57, lr_lo=0.002, lr_hi=0.02),
+    # a shorter last chunk (T % C != 0) on the tensor cores: 44 real tokens of 128
+    "swiglu_bf16_tc_tail": gen.Workload("nmst", gen.SWIGLU, gen.BF16, 2, 2, 128, 128, 256, 300, 128,
+                                        "uniform", 0.999, seed=59, lr_lo=0.002, lr_hi=0.02),
 }
 
 

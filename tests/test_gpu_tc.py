@@ -71,6 +71,19 @@ CASES = {
                                           "uniform", 0.999, seed=24, lr_lo=0.002, lr_hi=0.02), None),
     "layer_1p3b_2k_gelu_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_2k_gelu"]),
                                       [(0, 1), (3, 6)]),
+    # a shorter last chunk (T % C != 0), run padded to C tokens: 88 real tokens
+    # in the last chunk (one part-filled 128-row tile, one all padding) ...
+    "swiglu_tail_88": (gen.Workload("tail88", gen.SWIGLU, gen.BF16, 2, 2, 128, 128, 256, 600, 256,
+                                    "uniform", 0.999, seed=26, lr_lo=0.002, lr_hi=0.02), None),
+    # ... a single chunk shorter than C ...
+    "swiglu_single_short": (gen.Workload("short", gen.SWIGLU, gen.BF16, 1, 3, 128, 128, 256, 200, 256,
+                                         "uniform", 0.999, seed=27, lr_lo=0.002, lr_hi=0.02), None),
+    # ... one whole 128-row tile real and the rest padding, linear fast weight ...
+    "linear_tail_128": (gen.Workload("lintail", gen.LINEAR, gen.BF16, 2, 2, 128, 256, 0, 640, 512,
+                                     "uniform", 0.999, seed=28, lr_lo=0.002, lr_hi=0.02), None),
+    # ... and the GELU MLP with 44 real tokens in the last of three chunks
+    "gelu_tail_44": (gen.Workload("geltail", gen.GELU, gen.BF16, 2, 2, 128, 128, 256, 300, 128,
+                                  "uniform", 0.999, seed=29, lr_lo=0.002, lr_hi=0.02), None),
 }
 
 
