@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace e2ttt {
 
 typedef __nv_bfloat16 bf16;
@@ -50,6 +52,35 @@ __device__ __forceinline__ float dgelu_f(float z) {
 // gelu''(z) = phi(z) (2 - z^2)
 __device__ __forceinline__ float d2gelu_f(float z) {
   return 0.39894228040143268f * expf(-0.5f * z * z) * (2.0f - z * z);
+}
+
+// Programmatic dependent launch (sm_90 and later). A kernel launched with the
+// programmatic stream serialization attribute (launch_pdl) may start while its
+// predecessor on the stream still runs: griddep_wait() blocks until that
+// predecessor has completed and its memory operations are visible, so it comes
+// before the kernel's first global memory access. griddep_launch_dependents()
+// lets the successor start early (its own griddep_wait() still orders it).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with programmatic stream serialization: the kernel must call
+// griddep_wait() before touching global memory.
+template <class... Params, class... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace e2ttt

@@ -869,6 +869,7 @@ __global__ void __launch_bounds__(256) bwd_shadow_kernel(
     const float* __restrict__ W0, const float* __restrict__ M0, long long sst,
     const float* __restrict__ DW, float* __restrict__ DM, bf16* W13, bf16* W2, bf16* DW13,
     bf16* DW2, bf16* DM13, bf16* DM2, float* part, const float* __restrict__ scal, Dims d, int ci) {
+  griddep_launch_dependents();  // the next kernel's set-up may start
   const int z = blockIdx.y, blk = blockIdx.x;
   const long long S = d.S, n13 = 2LL * d.d_h * d.d_k;
   const size_t plane = (size_t)d.BH * d.NC, so = (size_t)z * d.NC + ci;
@@ -911,6 +912,7 @@ __global__ void __launch_bounds__(256) bwd_shadow_kernel(
 }
 // chunk-scalar adjoints from the partials.
 __global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci) {
+  griddep_launch_dependents();  // the next kernel's set-up may start
   const int z = blockIdx.x * blockDim.x + threadIdx.x;
   if (z >= d.BH) return;
   const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
@@ -923,6 +925,7 @@ __global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* 
 // abar_t, bbar_t = -(sum of the partial dot products), fixed order.
 __global__ void bwd_rows_kernel(const float* part, float* abar, float* bbar, Dims d, int t0, int clen,
                                 int NG) {
+  griddep_launch_dependents();  // the next kernel's set-up may start
   const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= (long long)d.BH * d.C) return;
   const int z = (int)(r / d.C), t = (int)(r % d.C);
@@ -1050,8 +1053,7 @@ cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
   E2TTT_TRACE(Name<Epi>::v, st);
-  kern<<<grid, (2 + EW) * 32, smem, st>>>(job, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3((2 + EW) * 32), smem, st, job, p);
 }
 
 struct Buf {

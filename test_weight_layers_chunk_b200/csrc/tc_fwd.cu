@@ -624,6 +624,7 @@ template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_l
 // ---------------------------------------------------------------- prep kernel
 // bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
 __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
+  griddep_launch_dependents();  // the next kernel's set-up may start
   // One warp per state row: rows [0, 2 d_h) of a head are W1 then W3 (d_k wide;
   // GELU MLP: [0, d_h) are W1), the next d_v rows are W2 (d_h wide); the linear
   // state is d_v rows of d_k.
@@ -663,6 +664,7 @@ __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* _
 __global__ void scale_keys_kernel(const bf16* __restrict__ k, const float* __restrict__ ca,
                                   const float* __restrict__ cb, bf16* __restrict__ Ka,
                                   bf16* __restrict__ Kb, long long tokens, int d_k) {
+  griddep_launch_dependents();  // the next kernel's set-up may start
   const long long n8 = tokens * d_k / 8;
   for (long long e8 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e8 < n8;
        e8 += (long long)gridDim.x * blockDim.x) {
@@ -775,8 +777,7 @@ cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
   for (int c = 0; c < job.n_cls; ++c) job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
   const int grid = job.total_tiles < num_sms() ? job.total_tiles : num_sms();
   E2TTT_TRACE(EpiName<Epi>::v, st);
-  kern<<<grid, (2 + EW) * 32, smem, st>>>(job, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3((2 + EW) * 32), smem, st, job, p);
 }
 
 struct Scratch {

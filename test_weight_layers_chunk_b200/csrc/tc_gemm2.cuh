@@ -16,6 +16,10 @@
 // Every mbarrier wait is bounded (about 1 s of globaltimer). On expiry the CTA
 // records a code in the device status word, stops, waits (bounded) for its own
 // copies and MMAs in flight, frees TMEM and exits. No TMA multicast anywhere.
+// Launched with programmatic stream serialization: the set-up (barriers, TMEM,
+// tensor-map prefetch) overlaps the tail of the previous kernel on the stream,
+// and every thread waits for that kernel (griddep_wait) before its first global
+// access; the CTA at once lets the next kernel start its own set-up.
 #pragma once
 #include <cuda.h>
 #include <stdint.h>
@@ -205,6 +209,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
   __shared__ int s_err;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     s_err = 0;
     for (int s = 0; s < STAGES; ++s) {
@@ -234,6 +239,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   int mma_tiles = 0;
+  griddep_wait();  // the previous kernel's results are complete and visible
 
   if (warp == 0 && lane == 0) {
     // ---------------- producer
