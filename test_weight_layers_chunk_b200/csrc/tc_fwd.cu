@@ -263,7 +263,10 @@ struct EpiG3Gelu {
 
 // Query rows -> out, key rows -> E (optional) and its a-/b-scaled copies, for a
 // warp's 32 rows and its column groups; V of the key rows is prefetched.
-template <int BN>
+// PAD: the chunk may be shorter than C (a last chunk with T % C != 0), so rows at
+// or past its length are padding (compiled separately: the per-row masking
+// slows the full-chunk epilogue measurably).
+template <bool PAD, int BN>
 __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>& c, bool key_rows,
                                                 int r0, bool write_e) {
   const Dims& d = p.d;
@@ -276,10 +279,10 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
   uint8_t* S = c.wsmem + 4096;     // E | Ea | Eb staging
   const int ttok = p.t0 + r0;      // first token (within the head) of this warp's rows
   const int yrow = c.z * d.C + r0;
-  // Rows at or past the chunk's length (a shorter last chunk) are padding: no
-  // output, and E = a E = b E = 0, so they add nothing to any later sum over tokens.
-  const bool real = lane < p.clen - r0;
-  if (!key_rows && p.clen - r0 <= 0) return;  // no query row of this warp is real
+  // Padding rows: no output, and E = a E = b E = 0, so they add nothing to any
+  // later sum over tokens.
+  const bool real = !PAD || lane < p.clen - r0;
+  if (PAD && !key_rows && p.clen - r0 <= 0) return;  // no query row of this warp is real
   if (key_rows) {
     if (lane == 0) {
       tc::mbar_expect_tx(&c.wbar[0], 2048u * ngroups);
@@ -320,7 +323,7 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
     float vv[32];
     unstage32(V + gi * 2048, lane, vv);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) y[i] = !real ? 0.f : d.loss == 0 ? y[i] - vv[i] : -vv[i];
+    for (int i = 0; i < 32; ++i) y[i] = (PAD && !real) ? 0.f : d.loss == 0 ? y[i] - vv[i] : -vv[i];
     staging_free(lane);
     if (write_e) stage32(S, lane, y);
     if (!p.nomom) {
@@ -342,25 +345,32 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
   }
 }
 
-// G2, SwiGLU: rows [0, C) are queries (-> out), [C, 2C) keys (-> E).
-struct EpiG2 {
+// G2, SwiGLU: rows [0, C) are queries (-> out), [C, 2C) keys (-> E). PAD: a
+// shorter last chunk.
+template <bool PAD>
+struct EpiG2T {
   static constexpr int kSmem = 10240;  // V[2] | E | Ea | Eb
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const int r0 = c.m0 + c.quad * 32;
     const bool key_rows = c.m0 >= p.d.C;
-    out_or_residual(p, c, key_rows, key_rows ? r0 - p.d.C : r0, true);
+    out_or_residual<PAD>(p, c, key_rows, key_rows ? r0 - p.d.C : r0, true);
   }
 };
+using EpiG2 = EpiG2T<false>;
+using EpiG2Pad = EpiG2T<true>;
 
 // G1, linear: class 0 = queries (-> out), class 1 = keys (-> scaled E).
-struct EpiG1Lin {
+template <bool PAD>
+struct EpiG1LinT {
   static constexpr int kSmem = 10240;
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
-    out_or_residual(p, c, c.cls == 1, c.m0 + c.quad * 32, false);
+    out_or_residual<PAD>(p, c, c.cls == 1, c.m0 + c.quad * 32, false);
   }
 };
+using EpiG1Lin = EpiG1LinT<false>;
+using EpiG1LinPad = EpiG1LinT<true>;
 
 // G3, SwiGLU: dA -> dH1 = dA H3 silu'(H1), dH3 = dA silu(H1) (rows: tokens).
 struct EpiG3 {
@@ -614,32 +624,30 @@ struct EpiG4W {
 template <class Epi> struct EpiName;
 template <> struct EpiName<EpiG1> { static constexpr const char* v = "tc_g1_h_act"; };
 template <> struct EpiName<EpiG2> { static constexpr const char* v = "tc_g2_y_out_e"; };
+template <> struct EpiName<EpiG2Pad> { static constexpr const char* v = "tc_g2_y_out_e"; };
 template <> struct EpiName<EpiG3> { static constexpr const char* v = "tc_g3_da_dh"; };
 template <> struct EpiName<EpiG4> { static constexpr const char* v = "tc_g4_aggregate_state"; };
 template <> struct EpiName<EpiG4W> { static constexpr const char* v = "tc_g4_aggregate_w"; };
 template <> struct EpiName<EpiG1Gelu> { static constexpr const char* v = "tc_g1_gelu"; };
 template <> struct EpiName<EpiG3Gelu> { static constexpr const char* v = "tc_g3_gelu_dh"; };
 template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
+template <> struct EpiName<EpiG1LinPad> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 
 // ---------------------------------------------------------------- prep kernel
 // bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
 __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
   griddep_launch_dependents();  // the next kernel's set-up may start
-  // One warp per state row: rows [0, 2 d_h) of a head are W1 then W3 (d_k wide;
-  // GELU MLP: [0, d_h) are W1), the next d_v rows are W2 (d_h wide); the linear
-  // state is d_v rows of d_k.
+  // One warp per state row, two rows per pass with both rows' loads issued first:
+  // rows [0, 2 d_h) of a head are W1 then W3 (d_k wide; GELU MLP: [0, d_h) are
+  // W1), the next d_v rows are W2 (d_h wide); the linear state is d_v rows of d_k.
   const Dims& d = p.d;
   const int lane = threadIdx.x & 31;
   const int r13 = d.kind == 1 ? 2 * d.d_h : d.kind == 2 ? d.d_h : d.d_v;
   const int rows = d.kind != 0 ? r13 + d.d_v : r13;
   const long long total = (long long)d.BH * rows;
   const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
-  for (long long gr = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); gr < total;
-       gr += nwarps) {
+  auto row_of = [&](long long gr, const float*& src, bf16*& dst, int& len) {
     const int z = (int)(gr / rows), r = (int)(gr - (long long)z * rows);
-    const float* src;
-    bf16* dst;
-    int len;
     if (r < r13) {
       src = W0 + (size_t)z * d.S + (size_t)r * d.d_k;
       const int sr = d.kind == 1 ? w13_row(r % d.d_h, r / d.d_h) : r;
@@ -650,37 +658,75 @@ __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* _
       dst = p.W2sh + ((size_t)z * d.d_v + (r - r13)) * d.d_h;
       len = d.d_h;
     }
-    // len is a multiple of 128: every lane moves whole 8-float groups
-    for (int c = lane * 8; c < len; c += 256) {
-      const float4 f0 = *reinterpret_cast<const float4*>(src + c);
-      const float4 f1 = *reinterpret_cast<const float4*>(src + c + 4);
-      *reinterpret_cast<uint4*>(dst + c) =
-          make_uint4(pack2(f0.x, f0.y), pack2(f0.z, f0.w), pack2(f1.x, f1.y), pack2(f1.z, f1.w));
+  };
+  for (long long gr = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); gr < total;
+       gr += 2 * nwarps) {
+    const float *s0, *s1 = nullptr;
+    bf16 *d0, *d1 = nullptr;
+    int n0, n1 = 0;
+    row_of(gr, s0, d0, n0);
+    if (gr + nwarps < total) row_of(gr + nwarps, s1, d1, n1);
+    // row lengths are multiples of 128: every lane moves whole 8-float groups
+    for (int c = lane * 8; c < (n0 > n1 ? n0 : n1); c += 256) {
+      float4 f[4];
+      const bool h0 = c < n0, h1 = c < n1;
+      if (h0) {
+        f[0] = *reinterpret_cast<const float4*>(s0 + c);
+        f[1] = *reinterpret_cast<const float4*>(s0 + c + 4);
+      }
+      if (h1) {
+        f[2] = *reinterpret_cast<const float4*>(s1 + c);
+        f[3] = *reinterpret_cast<const float4*>(s1 + c + 4);
+      }
+      if (h0)
+        *reinterpret_cast<uint4*>(d0 + c) = make_uint4(pack2(f[0].x, f[0].y), pack2(f[0].z, f[0].w),
+                                                       pack2(f[1].x, f[1].y), pack2(f[1].z, f[1].w));
+      if (h1)
+        *reinterpret_cast<uint4*>(d1 + c) = make_uint4(pack2(f[2].x, f[2].y), pack2(f[2].z, f[2].w),
+                                                       pack2(f[3].x, f[3].y), pack2(f[3].z, f[3].w));
     }
   }
 }
 
 // diag(a) K and diag(b) K for every token (B operands of the W1/W3 aggregation).
+// Each thread moves kScaleVec 8-element groups per pass (all loads issued before
+// the stores), consecutive threads consecutive groups.
+constexpr int kScaleVec = 4;
 __global__ void scale_keys_kernel(const bf16* __restrict__ k, const float* __restrict__ ca,
                                   const float* __restrict__ cb, bf16* __restrict__ Ka,
                                   bf16* __restrict__ Kb, long long tokens, int d_k) {
   griddep_launch_dependents();  // the next kernel's set-up may start
   const long long n8 = tokens * d_k / 8;
-  for (long long e8 = (long long)blockIdx.x * blockDim.x + threadIdx.x; e8 < n8;
-       e8 += (long long)gridDim.x * blockDim.x) {
-    const long long tok = e8 * 8 / d_k;
-    const float a = ca[tok], b = cb[tok];
-    const uint4 u = reinterpret_cast<const uint4*>(k)[e8];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t oa[4], ob[4];
+  const long long step = (long long)gridDim.x * blockDim.x * kScaleVec;
+  for (long long base = (long long)blockIdx.x * blockDim.x * kScaleVec + threadIdx.x; base < n8;
+       base += step) {
+    uint4 u[kScaleVec];
+    float a[kScaleVec], b[kScaleVec];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-      oa[i] = pack2(a * f.x, a * f.y);
-      ob[i] = pack2(b * f.x, b * f.y);
+    for (int j = 0; j < kScaleVec; ++j) {
+      const long long e8 = base + (long long)j * blockDim.x;
+      if (e8 < n8) {
+        const long long tok = e8 * 8 / d_k;
+        u[j] = reinterpret_cast<const uint4*>(k)[e8];
+        a[j] = ca[tok];
+        b[j] = cb[tok];
+      }
     }
-    if (Ka) reinterpret_cast<uint4*>(Ka)[e8] = make_uint4(oa[0], oa[1], oa[2], oa[3]);  // NULL: no momentum
-    reinterpret_cast<uint4*>(Kb)[e8] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+#pragma unroll
+    for (int j = 0; j < kScaleVec; ++j) {
+      const long long e8 = base + (long long)j * blockDim.x;
+      if (e8 >= n8) continue;
+      const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+      uint32_t oa[4], ob[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        oa[i] = pack2(a[j] * f.x, a[j] * f.y);
+        ob[i] = pack2(b[j] * f.x, b[j] * f.y);
+      }
+      if (Ka) reinterpret_cast<uint4*>(Ka)[e8] = make_uint4(oa[0], oa[1], oa[2], oa[3]);  // NULL: no momentum
+      reinterpret_cast<uint4*>(Kb)[e8] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
   }
 }
 
@@ -985,7 +1031,10 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
         e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
       else
         e = launch<128, 1, false, false, 4, EpiG1Gelu, kEpiWarps, EpiG1Gelu::kSmem>(g1, p, st);
-      if (e == cudaSuccess) e = launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
+      if (e == cudaSuccess) {
+        e = p.clen < C ? launch<128, 1, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
+                       : launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
+      }
       if (e == cudaSuccess) {
         e = d.kind == 1
                 ? launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st)
@@ -996,7 +1045,8 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
                     : launch<128, 2, true, true, 3, EpiG4, 4, EpiG4::kSmem>(g4, p, st);
       }
     } else {
-      e = launch<128, 1, false, false, 4, EpiG1Lin, kEpiWarps, EpiG1Lin::kSmem>(g1, p, st);
+      e = p.clen < C ? launch<128, 1, false, false, 4, EpiG1LinPad, kEpiWarps, EpiG1LinPad::kSmem>(g1, p, st)
+                     : launch<128, 1, false, false, 4, EpiG1Lin, kEpiWarps, EpiG1Lin::kSmem>(g1, p, st);
       if (e == cudaSuccess) {
         e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)
                     : launch<128, 2, true, true, 3, EpiG4, 4, EpiG4::kSmem>(g4, p, st);
