@@ -130,9 +130,11 @@ def fwd_flops(w) -> float:
 
 
 def train_flops(w) -> float:
-    """Forward 26 d d_h plus backward 52 d d_h per token and head (SwiGLU,
-    d_k = d_v = d; the backward's recomputation of the forward is not counted)."""
-    return 78.0 * w.d_k * w.d_h * w.B * w.H * w.T
+    """Forward plus backward: the backward's algorithmic FLOPs are twice the
+    forward's (SwiGLU, d_k = d_v = d: 26 + 52 d d_h per token and head; the same
+    ratio is taken for the GELU MLP); the backward's recomputation of the forward
+    is not counted."""
+    return 3.0 * fwd_flops(w)
 
 
 def fp32_fma_peak_tflops(sm_mhz: float) -> float:
@@ -342,16 +344,18 @@ def _timed(torch, stream, fn, steps):
 def measure_extras(E, torch, dev, stream, args):
     """The metric's other operating points, device-timed like the main line:
     forward at T = 16K (the 8x length-extrapolation layer), forward+backward at
-    T = 2K (the training workload), and the forward at T = 2K of the
+    T = 2K (the training workload), the forward at T = 2K of the
     chunk-averaged variant, of the no-momentum mode and of the GELU MLP fast
-    weight, each with its own warm-up."""
+    weight, and the GELU MLP's forward+backward at T = 2K, each with its own
+    warm-up."""
     out = {}
     f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
     for name, train, steps, coef, nomom in (("layer_1p3b_16k", False, args.extra_steps, 0, 0),
                                             ("train_1p3b_2k", True, max(2, args.extra_steps // 8), 0, 0),
                                             ("layer_1p3b_2k", False, args.extra_steps, 1, 0),
                                             ("layer_1p3b_2k", False, args.extra_steps, 0, 1),
-                                            ("layer_1p3b_2k_gelu", False, args.extra_steps, 0, 0)):
+                                            ("layer_1p3b_2k_gelu", False, args.extra_steps, 0, 0),
+                                            ("layer_1p3b_2k_gelu", True, max(2, args.extra_steps // 8), 0, 0)):
         w = gen.BY_NAME[name]
         x = gen.generate(w)
         q, k, v = f(x["q"], torch.bfloat16), f(x["k"], torch.bfloat16), f(x["v"], torch.bfloat16)

@@ -1,4 +1,5 @@
-// tcgen05 tensor-core backward of the chunk scan (SwiGLU, bf16 activations).
+// tcgen05 tensor-core backward of the chunk scan (SwiGLU and GELU MLP, bf16
+// activations).
 //
 // Same mathematics as the CUDA-core backward (bwd.cu): the adjoint of the
 // closed-form chunk transition ("Rethinking Expressivity and Efficiency in
@@ -15,6 +16,11 @@
 //   dk = -(a dH D_M13 + b dH D_W13) + [h1b | h3b] [W1; W3] ;  dq = query-row [h1b | h3b] [W1; W3]
 //   dW13 += [h1b | h3b]^T [K; Q] ,  dW2 += [E; EB; dout]^T [dub; U_k; U_q]  (into D_W in place)
 //   dM0 = U(1,n) D_M + c D_W ; abar, bbar and the chunk-scalar adjoints for the gate gradients.
+// GELU MLP (h = W1 k, u = gelu(h); one activation factor per hidden unit, so the
+// [W1; W3] blocks above are W1 alone and h1 | h3 is h):
+//   R1  h = X W1^T ; u = gelu(h)     R3  dH = du gelu'(h)     E3  dub = dhb gelu'(h)
+//   E5  hb = dhb du gelu''(h) + ub gelu'(h)     Q1  query-row hb = (dout W2) gelu'(h)
+// and D1, D2, E4, dk, dq, dW as above with hw = d_h columns instead of 2 d_h.
 #include <cuda.h>
 
 #include <type_traits>
@@ -39,6 +45,7 @@ struct BwdP {
   // token reads as zero and is clipped on store
   Dims d;
   int ci, t0;
+  int hw;  // hidden columns of the first state block: 2 d_h (SwiGLU h1 | h3) or d_h (GELU h)
   // tokens of this chunk: C, or T - t0 for a shorter last chunk, whose padding
   // rows carry zero keys, queries, dout and v and a_t = b_t = 0, so every
   // per-token term of theirs vanishes
@@ -51,12 +58,12 @@ struct BwdP {
   bf16 *X;    // [2C, d_k]   rows: keys, then queries
   bf16 *Y3;   // [3C, d_h]   rows: dub | u_k | u_q
   bf16 *Z3;   // [3C, d_v]   rows: E | EB | dout
-  bf16 *Hc;   // [2C, 2 d_h] h1 | h3 (keys, then queries)
-  bf16 *DH;   // [C, 2 d_h]  dH1 | dH3
-  bf16 *HB;   // [2C, 2 d_h] h1b | h3b (keys, then queries)
+  bf16 *Hc;   // [2C, hw] h1 | h3 (GELU: h) (keys, then queries)
+  bf16 *DH;   // [C, hw]  dH1 | dH3 (GELU: dH)
+  bf16 *HB;   // [2C, hw] h1b | h3b (GELU: hb) (keys, then queries)
   // fp32 epilogue data (per head)
   float *du;     // [C, d_h]
-  float *DB;     // [C, 2 d_h]  dh1b | dh3b
+  float *DB;     // [C, hw]  dh1b | dh3b (GELU: dhb)
   float *G2U;    // [C, d_v]
   float *UBd;    // [C, d_h]
   float *dkp;    // [C, d_k]
@@ -388,7 +395,7 @@ struct EpiD2 {
     const size_t tok = (size_t)c.z * d.T + p.t0 + t;
     const float a = t < p.clen ? p.ca[tok] : 0.f, b = t < p.clen ? p.cb[tok] : 0.f;
     const int yG = c.z * d.C + c.m0 + c.quad * 32;
-    float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG + 2 * d.d_h / 32;
+    float* pa = p.part + ((size_t)c.z * d.C + t) * p.NG + p.hw / 32;
     float* pb = pa + (size_t)d.BH * d.C * p.NG;
     const uint8_t* IN = c.wsmem;
     uint8_t* F = c.wsmem + kIn;
@@ -697,6 +704,249 @@ struct EpiQ1 {
     }
   }
 };
+// ---- GELU MLP variants of R1, R3, E3, E5, Q1 (one activation factor per hidden unit)
+// R1: rows of X (keys then queries); h = acc -> Hc, u = gelu(h) -> Y3.
+struct EpiR1G {
+  static constexpr int kSmem = 4096;  // h | u staging (bf16)
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int r0 = c.m0 + c.quad * 32;
+    const int yH = c.z * 2 * d.C + r0, yU = c.z * 3 * d.C + d.C + r0;
+    uint8_t* S = c.wsmem;
+    FOR_GROUPS(c, BN, g) {
+      const int j = c.n0 + g;
+      float h[32];
+      acc1(c, g, h);
+      out_free(lane);
+      stage_h(S, lane, h);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h[i] = gelu_f(h[i]);
+      stage_h(S + 2048, lane, h);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mHc, S, j, yH);
+        tc::tma_store_2d(&p.mY3, S + 2048, j, yU);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
+// R3: du = E W2 -> du (fp32), dH = du gelu'(h) (key rows).
+struct EpiR3G {
+  static constexpr int kIn = 2048;            // h (bf16)
+  static constexpr int kSmem = kIn + 6144;    // | du (fp32) | dH (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
+    tc::tma_load_2d(c.wsmem, &p.mHc, &c.wbar[0], ga.col, ga.z * 2 * p.d.C + ga.m0 + c.quad * 32);
+  }
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int yD = c.z * d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* F = c.wsmem + kIn;
+    uint8_t* Hs = c.wsmem + kIn + 4096;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
+      float du[32], h[32];
+      acc1(c, g, du);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, h);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h[i] = du[i] * dgelu_f(h[i]);
+      out_free(lane);
+      stage_f(F, lane, du);
+      stage_h(Hs, lane, h);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fdu, F, j, yD);
+        tc::tma_store_2d(&p.mDH, Hs, j, yD);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
+// E3: acc0 = E D_M2, acc1 = E D_W2 (columns = hidden units) -> UBd = -(a . + b .)
+// (fp32) and dub = dhb gelu'(h) (bf16, rows [0, C) of Y3).
+struct EpiE3G {
+  static constexpr int kWarps = 4;
+  static constexpr int kIn = 6144;           // dhb (fp32) | h (bf16)
+  static constexpr int kSmem = kIn + 6144;   // | UBd (fp32) | dub (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    const Dims& d = p.d;
+    const int r = ga.m0 + c.quad * 32;
+    uint64_t* bar = &c.wbar[0];
+    tc::mbar_expect_tx(bar, 6144u);
+    tc::tma_load_2d(c.wsmem, &p.fDB, bar, ga.col, ga.z * d.C + r);
+    tc::tma_load_2d(c.wsmem + 4096, &p.mHc, bar, ga.col, ga.z * 2 * d.C + r);
+  }
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int t = c.m0 + c.row;
+    const size_t tok = (size_t)c.z * d.T + p.t0 + t;
+    const float a = t < p.clen ? p.ca[tok] : 0.f, b = t < p.clen ? p.cb[tok] : 0.f;
+    const int r0 = c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* F = c.wsmem + kIn;
+    uint8_t* Hs = c.wsmem + kIn + 4096;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
+      float m[32], w[32];
+      acc2(c, g, m, w);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
+      out_free(lane);
+      stage_f(F, lane, m);
+      if (!in_wait(p, c)) return;
+      float bh[32];
+      unstage_f(IN, lane, bh);
+      unstage_h(IN + 4096, lane, w);   // h
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) bh[i] *= dgelu_f(w[i]);
+      stage_h(Hs, lane, bh);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.fUBd, F, j, c.z * d.C + r0);
+        tc::tma_store_2d(&p.mY3, Hs, j, c.z * 3 * d.C + r0);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
+// E5: ub = UBd + eb W2 (MSE); the key rows' hb = dhb du gelu''(h) + ub gelu'(h).
+struct EpiE5G {
+  static constexpr int kWarps = 4;
+  static constexpr int kIn = 14336;          // UBd | du | dhb (fp32) | h (bf16)
+  static constexpr int kSmem = kIn + 2048;   // | hb (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    const Dims& d = p.d;
+    const int r = ga.m0 + c.quad * 32;
+    const int yC = ga.z * d.C + r, yH = ga.z * 2 * d.C + r;
+    uint64_t* bar = &c.wbar[0];
+    tc::mbar_expect_tx(bar, 14336u);
+    tc::tma_load_2d(c.wsmem, &p.fUBd, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 4096, &p.fdu, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 8192, &p.fDB, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 12288, &p.mHc, bar, ga.col, yH);
+  }
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int yH = c.z * 2 * d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
+      float acc[32], ubd[32], du[32], bh[32], h[32];
+      acc1(c, g, acc);
+      if (!in_wait(p, c)) return;
+      unstage_f(IN, lane, ubd);
+      unstage_f(IN + 4096, lane, du);
+      unstage_f(IN + 8192, lane, bh);
+      unstage_h(IN + 12288, lane, h);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float ub = ubd[i] + (d.loss == 0 ? acc[i] : 0.f);
+        h[i] = bh[i] * du[i] * d2gelu_f(h[i]) + ub * dgelu_f(h[i]);
+      }
+      out_free(lane);
+      stage_h(OUT, lane, h);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mHB, OUT, j, yH);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
+// Q1: ub_q = dout W2 -> query-row hb = ub gelu'(h).
+struct EpiQ1G {
+  static constexpr int kIn = 2048;           // query h (bf16)
+  static constexpr int kSmem = kIn + 2048;   // | hb (bf16)
+  template <int BN>
+  static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
+    const GroupAt ga = group_at(c, gi);
+    if (!ga.valid) return;
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
+    tc::tma_load_2d(c.wsmem, &p.mHc, &c.wbar[0], ga.col, ga.z * 2 * p.d.C + p.d.C + ga.m0 + c.quad * 32);
+  }
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    const Dims& d = p.d;
+    const int lane = c.row & 31;
+    const int per = BN / c.nparts, ngroups = per / 32;
+    const int y = c.z * 2 * d.C + d.C + c.m0 + c.quad * 32;
+    const uint8_t* IN = c.wsmem;
+    uint8_t* OUT = c.wsmem + kIn;
+    if (c.iter == 0 && lane == 0) issue(p, c, 0);
+    __syncwarp();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int g = c.part * per + gi * 32, j = c.n0 + g;
+      float ub[32], h[32];
+      acc1(c, g, ub);
+      if (!in_wait(p, c)) return;
+      unstage_h(IN, lane, h);
+      __syncwarp();
+      if (lane == 0) {
+        tc::fence_async_smem();
+        issue(p, c, gi + 1);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h[i] = ub[i] * dgelu_f(h[i]);
+      out_free(lane);
+      stage_h(OUT, lane, h);
+      out_ready();
+      if (lane == 0) {
+        tc::tma_store_2d(&p.mHB, OUT, j, y);
+        tc::bulk_commit();
+      }
+      __syncwarp();
+    }
+  }
+};
 // dk part 1: -(a dH D_M13 + b dH D_W13) (fp32) -> dkp.
 struct EpiDk1 {
   static constexpr int kSmem = 4096;  // dkp staging (fp32)
@@ -838,10 +1088,16 @@ template <> struct Name<EpiDk1> { static constexpr const char* v = "tcb_dk1"; };
 template <> struct Name<EpiDkq<true>> { static constexpr const char* v = "tcb_dk2"; };
 template <> struct Name<EpiDkq<false>> { static constexpr const char* v = "tcb_dq"; };
 template <> struct Name<EpiDW> { static constexpr const char* v = "tcb_dw"; };
+template <> struct Name<EpiR1G> { static constexpr const char* v = "tcb_r1_h"; };
+template <> struct Name<EpiR3G> { static constexpr const char* v = "tcb_r3_du"; };
+template <> struct Name<EpiE3G> { static constexpr const char* v = "tcb_e3_ub_dub"; };
+template <> struct Name<EpiE5G> { static constexpr const char* v = "tcb_e5_hb"; };
+template <> struct Name<EpiQ1G> { static constexpr const char* v = "tcb_q1_hbq"; };
 
 // ---------------------------------------------------------------- elementwise kernels
 // bf16 copies of the chunk-start weights and of the state adjoints, each split
-// into a [W1; W3] block [BH, 2 d_h, d_k] and a W2 block [BH, d_v, d_h]; the
+// into a [W1; W3] block [BH, 2 d_h, d_k] (GELU: W1, [BH, d_h, d_k]) and a W2 block
+// [BH, d_v, d_h]; the
 // partial sums of <D_M, M0>, <D_W, W0>, <D_W, M0> (64 blocks per head); and,
 // once the old D_M is read, D_M <- U(1,n) D_M + c D_W in place (the chunk-start
 // adjoint of M; the GEMM phases read only the bf16 copies).
@@ -871,7 +1127,7 @@ __global__ void __launch_bounds__(256) bwd_shadow_kernel(
     bf16* DW2, bf16* DM13, bf16* DM2, float* part, const float* __restrict__ scal, Dims d, int ci) {
   griddep_launch_dependents();  // the next kernel's set-up may start
   const int z = blockIdx.y, blk = blockIdx.x;
-  const long long S = d.S, n13 = 2LL * d.d_h * d.d_k;
+  const long long S = d.S, n13 = (d.kind == 1 ? 2LL : 1LL) * d.d_h * d.d_k;
   const size_t plane = (size_t)d.BH * d.NC, so = (size_t)z * d.NC + ci;
   const float U = scal[so], cc = scal[2 * plane + so];
   const float4* w0 = reinterpret_cast<const float4*>(W0 + z * sst);
@@ -1071,7 +1327,8 @@ Buf carve(const Dims& d, char* base) {
     return p;
   };
   const size_t BH = d.BH, C = d.C, dk = d.d_k, dv = d.d_v, dh = d.d_h, h = 2, f = 4;
-  const int NG = (int)(2 * dh / 32 + dv / 32);
+  const size_t hw = (d.kind == 1 ? 2 : 1) * dh;  // SwiGLU h1 | h3, GELU h
+  const int NG = (int)(hw / 32 + dv / 32);
   B.status = (int*)take(256);  // first bytes of the workspace (read by e2ttt_workspace_status)
   B.a = (float*)take(BH * d.T * f);
   B.b = (float*)take(BH * d.T * f);
@@ -1083,17 +1340,17 @@ Buf carve(const Dims& d, char* base) {
   B.X = (bf16*)take(BH * 2 * C * dk * h);
   B.Y3 = (bf16*)take(BH * 3 * C * dh * h);
   B.Z3 = (bf16*)take(BH * 3 * C * dv * h);
-  B.Hc = (bf16*)take(BH * 2 * C * 2 * dh * h);
-  B.DH = (bf16*)take(BH * C * 2 * dh * h);
-  B.HB = (bf16*)take(BH * 2 * C * 2 * dh * h);
-  B.W13 = (bf16*)take(BH * 2 * dh * dk * h);
+  B.Hc = (bf16*)take(BH * 2 * C * hw * h);
+  B.DH = (bf16*)take(BH * C * hw * h);
+  B.HB = (bf16*)take(BH * 2 * C * hw * h);
+  B.W13 = (bf16*)take(BH * hw * dk * h);
   B.W2 = (bf16*)take(BH * dv * dh * h);
-  B.DW13 = (bf16*)take(BH * 2 * dh * dk * h);
+  B.DW13 = (bf16*)take(BH * hw * dk * h);
   B.DW2 = (bf16*)take(BH * dv * dh * h);
-  B.DM13 = (bf16*)take(BH * 2 * dh * dk * h);
+  B.DM13 = (bf16*)take(BH * hw * dk * h);
   B.DM2 = (bf16*)take(BH * dv * dh * h);
   B.du = (float*)take(BH * C * dh * f);
-  B.DB = (float*)take(BH * C * 2 * dh * f);
+  B.DB = (float*)take(BH * C * hw * f);
   B.G2U = (float*)take(BH * C * dv * f);
   B.UBd = (float*)take(BH * C * dh * f);
   B.dkp = (float*)take(BH * C * dk * f);
@@ -1109,7 +1366,7 @@ tc2::Class cls(int tm, int tn, int kb, tc2::Opnd a, tc2::Opnd b, int mode = 0) {
 }  // namespace
 
 bool tc_bwd_supported(const Dims& d, bool bf16_act) {
-  return d.kind == 1 && tc_fwd_supported(d, bf16_act);
+  return (d.kind == 1 || d.kind == 2) && tc_fwd_supported(d, bf16_act);
 }
 size_t tc_bwd_workspace_bytes(const Dims& d) { return carve(d, nullptr).total; }
 
@@ -1138,16 +1395,19 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   p.DW = A.dW0; p.DM = A.dM0;
   p.X = B.X; p.Y3 = B.Y3; p.Z3 = B.Z3; p.Hc = B.Hc; p.DH = B.DH; p.HB = B.HB;
   p.du = B.du; p.DB = B.DB; p.G2U = B.G2U; p.UBd = B.UBd; p.dkp = B.dkp; p.part = B.part;
-  p.NG = (int)(2 * dh / 32 + dv / 32);
+  const bool gelu = d.kind == 2;
+  const int hw = (gelu ? 1 : 2) * dh;  // columns of the first state block's hidden side
+  p.hw = hw;
+  p.NG = hw / 32 + dv / 32;
   p.status = B.status;
   {
     const uint64_t rC = (uint64_t)BH * C;
-    bool mok = box32(&p.mHc, B.Hc, 2 * rC, 2 * dh, false);
+    bool mok = box32(&p.mHc, B.Hc, 2 * rC, hw, false);
     mok &= box32(&p.mY3, B.Y3, 3 * rC, dh, false);
-    mok &= box32(&p.mDH, B.DH, rC, 2 * dh, false);
-    mok &= box32(&p.mHB, B.HB, 2 * rC, 2 * dh, false);
+    mok &= box32(&p.mDH, B.DH, rC, hw, false);
+    mok &= box32(&p.mHB, B.HB, 2 * rC, hw, false);
     mok &= box32(&p.fdu, B.du, rC, dh, true);
-    mok &= box32(&p.fDB, B.DB, rC, 2 * dh, true);
+    mok &= box32(&p.fDB, B.DB, rC, hw, true);
     mok &= box32(&p.fUBd, B.UBd, rC, dh, true);
     mok &= box32(&p.mZ3, B.Z3, 3 * rC, dv, false);
     mok &= tok_box32(&p.mv, A.v, T, dv, BH);
@@ -1156,8 +1416,8 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     mok &= tok_box32(&p.mdq, A.dq, T, dk, BH);
     mok &= box32(&p.fG2U, B.G2U, rC, dv, true);
     mok &= box32(&p.fdkp, B.dkp, rC, dk, true);
-    mok &= state_box32(&p.fDW[0], A.dW0, 2 * dh, dk, BH, d.S);
-    mok &= state_box32(&p.fDW[1], A.dW0 + 2 * (size_t)dh * dk, dv, dh, BH, d.S);
+    mok &= state_box32(&p.fDW[0], A.dW0, hw, dk, BH, d.S);
+    mok &= state_box32(&p.fDW[1], A.dW0 + (size_t)hw * dk, dv, dh, BH, d.S);
     if (!mok) return cudaErrorInvalidValue;
   }
 
@@ -1166,17 +1426,22 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   bool ok = true;
   const uint64_t rX = (uint64_t)BH * 2 * C, rY = (uint64_t)BH * 3 * C, rZ = rY;
   const uint64_t rH = (uint64_t)BH * 2 * C, rD = (uint64_t)BH * C;
-  const uint64_t r13 = (uint64_t)BH * 2 * dh, r2w = (uint64_t)BH * dv;
+  const uint64_t r13 = (uint64_t)BH * hw, r2w = (uint64_t)BH * dv;
   for (tc2::Job* j : {&r1, &r2, &r3, &d1, &d2, &e3, &e4, &e5, &q1, &k1, &k2, &dq, &dw}) {
     j->heads = BH;
     j->n_cls = 1;
     j->status = B.status;
   }
-  // R1: X [2C x dk] x {W1, W3}^T (two B operands)
+  // R1: X [2C x dk] x {W1, W3}^T (two B operands; GELU: W1 alone)
   ok &= mk(&r1.maps[0].op0, B.X, rX, dk, 128);
-  ok &= mk(&r1.maps[0].op1, B.W13, r13, dk, 128);
-  ok &= mk(&r1.maps[0].op2, B.W13 + (size_t)dh * dk, r13 - dh, dk, 128);
-  r1.cls[0] = cls(2 * C / 128, dh / 128, dk / 64, {2 * C, 0, 0}, {2 * dh, 0, 0}, tc2::kModeA1B2);
+  if (gelu) {
+    ok &= mk(&r1.maps[0].op2, B.W13, r13, dk, 128);
+    r1.cls[0] = cls(2 * C / 128, dh / 128, dk / 64, {2 * C, 0, 0}, {hw, 0, 0});
+  } else {
+    ok &= mk(&r1.maps[0].op1, B.W13, r13, dk, 128);
+    ok &= mk(&r1.maps[0].op2, B.W13 + (size_t)dh * dk, r13 - dh, dk, 128);
+    r1.cls[0] = cls(2 * C / 128, dh / 128, dk / 64, {2 * C, 0, 0}, {hw, 0, 0}, tc2::kModeA1B2);
+  }
   // R2: U_k (rows [C, 2C) of Y3) x W2^T
   ok &= mk(&r2.maps[0].op0, B.Y3, rY, dh, 128);
   ok &= mk(&r2.maps[0].op2, B.W2, r2w, dh, 128);
@@ -1189,7 +1454,7 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   ok &= mk(&d1.maps[0].op0, B.X, rX, dk, 128);
   ok &= mk(&d1.maps[0].op1, B.DM13, r13, dk, 128);
   ok &= mk(&d1.maps[0].op2, B.DW13, r13, dk, 128);
-  d1.cls[0] = cls(C / 128, 2 * dh / 128, dk / 64, {2 * C, 0, 0}, {2 * dh, 0, 0}, tc2::kModeA1B2);
+  d1.cls[0] = cls(C / 128, hw / 128, dk / 64, {2 * C, 0, 0}, {hw, 0, 0}, tc2::kModeA1B2);
   // D2: U_k x {D_M2, D_W2}^T
   ok &= mk(&d2.maps[0].op0, B.Y3, rY, dh, 128);
   ok &= mk(&d2.maps[0].op1, B.DM2, r2w, dh, 128);
@@ -1211,23 +1476,23 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   q1.maps[0] = e5.maps[0];
   q1.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, 2 * C, 0}, {dv, 0, 0});
   // dk1: dH x {D_M13, D_W13} (MN-major: N = d_k, K = 2 d_h)
-  ok &= mk(&k1.maps[0].op0, B.DH, rD, 2 * dh, 128);
+  ok &= mk(&k1.maps[0].op0, B.DH, rD, hw, 128);
   ok &= mk(&k1.maps[0].op1, B.DM13, r13, dk, 64);
   ok &= mk(&k1.maps[0].op2, B.DW13, r13, dk, 64);
-  k1.cls[0] = cls(C / 128, dk / 128, 2 * dh / 64, {C, 0, 0}, {2 * dh, 0, 0}, tc2::kModeA1B2);
+  k1.cls[0] = cls(C / 128, dk / 128, hw / 64, {C, 0, 0}, {hw, 0, 0}, tc2::kModeA1B2);
   // dk2 / dq: [h1b | h3b] (rows [0, C) / [C, 2C) of HB) x [W1; W3] (MN-major)
-  ok &= mk(&k2.maps[0].op0, B.HB, rH, 2 * dh, 128);
+  ok &= mk(&k2.maps[0].op0, B.HB, rH, hw, 128);
   ok &= mk(&k2.maps[0].op2, B.W13, r13, dk, 64);
-  k2.cls[0] = cls(C / 128, dk / 128, 2 * dh / 64, {2 * C, 0, 0}, {2 * dh, 0, 0});
+  k2.cls[0] = cls(C / 128, dk / 128, hw / 64, {2 * C, 0, 0}, {hw, 0, 0});
   dq.maps[0] = k2.maps[0];
-  dq.cls[0] = cls(C / 128, dk / 128, 2 * dh / 64, {2 * C, C, 0}, {2 * dh, 0, 0});
+  dq.cls[0] = cls(C / 128, dk / 128, hw / 64, {2 * C, C, 0}, {hw, 0, 0});
   // dW: class 0 = [h1b | h3b]^T [K; Q] (2C tokens), class 1 = [E; EB; dout]^T [dub; u_k; u_q]
-  ok &= mk(&dw.maps[0].op0, B.HB, rH, 2 * dh, 64);
+  ok &= mk(&dw.maps[0].op0, B.HB, rH, hw, 64);
   ok &= mk(&dw.maps[0].op2, B.X, rX, dk, 64);
   ok &= mk(&dw.maps[1].op0, B.Z3, rZ, dv, 64);
   ok &= mk(&dw.maps[1].op2, B.Y3, rY, dh, 64);
   dw.n_cls = 2;
-  dw.cls[0] = cls(2 * dh / 128, dk / 128, 2 * C / 64, {2 * C, 0, 0}, {2 * C, 0, 0});
+  dw.cls[0] = cls(hw / 128, dk / 128, 2 * C / 64, {2 * C, 0, 0}, {2 * C, 0, 0});
   dw.cls[1] = cls(dv / 128, dh / 128, 3 * C / 64, {3 * C, 0, 0}, {3 * C, 0, 0});
   if (!ok) return cudaErrorInvalidValue;
 
@@ -1272,15 +1537,20 @@ cudaError_t tc_bwd(const BwdArgs& A) {
       if (e != cudaSuccess) return e;
     }
     using tc2::kModeA1B2;
-    if ((e = run_gemm<2, false, false, EpiR1>(r1, p, st)) != cudaSuccess) return e;
+    e = gelu ? run_gemm<1, false, false, EpiR1G>(r1, p, st) : run_gemm<2, false, false, EpiR1>(r1, p, st);
+    if (e != cudaSuccess) return e;
     if ((e = run_gemm<1, false, false, EpiR2>(r2, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<1, false, true, EpiR3>(r3, p, st)) != cudaSuccess) return e;
+    e = gelu ? run_gemm<1, false, true, EpiR3G>(r3, p, st) : run_gemm<1, false, true, EpiR3>(r3, p, st);
+    if (e != cudaSuccess) return e;
     if ((e = run_gemm<2, false, false, EpiD1>(d1, p, st)) != cudaSuccess) return e;
     if ((e = run_gemm<2, false, false, EpiD2>(d2, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<2, false, true, EpiE3>(e3, p, st)) != cudaSuccess) return e;
+    e = gelu ? run_gemm<2, false, true, EpiE3G>(e3, p, st) : run_gemm<2, false, true, EpiE3>(e3, p, st);
+    if (e != cudaSuccess) return e;
     if ((e = run_gemm<1, false, false, EpiE4>(e4, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<1, false, true, EpiE5>(e5, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<1, false, true, EpiQ1>(q1, p, st)) != cudaSuccess) return e;
+    e = gelu ? run_gemm<1, false, true, EpiE5G>(e5, p, st) : run_gemm<1, false, true, EpiE5>(e5, p, st);
+    if (e != cudaSuccess) return e;
+    e = gelu ? run_gemm<1, false, true, EpiQ1G>(q1, p, st) : run_gemm<1, false, true, EpiQ1>(q1, p, st);
+    if (e != cudaSuccess) return e;
     if ((e = run_gemm<2, false, true, EpiDk1>(k1, p, st)) != cudaSuccess) return e;
     if ((e = run_gemm<1, false, true, EpiDkq<true>>(k2, p, st)) != cudaSuccess) return e;
     if ((e = run_gemm<1, false, true, EpiDkq<false>>(dq, p, st)) != cudaSuccess) return e;
