@@ -194,10 +194,10 @@ e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
  *   Outputs: dq, dk, dv (act dtype), dlr, dmom, ddecay (fp32 [B,H,T]),
  *            dW0, dM0 (fp32 [B,H,S]).
  *   No-momentum mode: mom, dM_end, dmom and dM0 must be NULL.
- *   Paths: the SwiGLU backward with bf16 activations (shapes as for the
- *   forward's tensor-core path, a shorter last chunk included) runs on the
- *   tensor cores; the GELU MLP, the
- *   linear fast weight and fp32 activations run on fp32 CUDA cores. */
+ *   Paths: the SwiGLU and GELU MLP backward with bf16 activations (shapes as
+ *   for the forward's tensor-core path, a shorter last chunk included) runs on
+ *   the tensor cores; the linear fast weight and fp32 activations run on fp32
+ *   CUDA cores. */
 e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
                                   const void* q, const void* k, const void* v,
                                   const float* lr, const float* mom, const float* decay,
