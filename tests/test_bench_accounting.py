@@ -1,0 +1,111 @@
+"""The work figures bench.py divides by (host-side arithmetic, no GPU).
+
+The roofline fractions the bench reports are algorithmic work / measured time /
+measured peak, so the work must be right. These tests re-derive it another way:
+FLOPs per token and head from the matrix shapes of each GEMM phase, the
+aggregation's bytes chunk by chunk, and the whole call's compulsory bytes from
+its inputs and outputs, and check the recorded ncu traffic is only used for the
+kernel sources it was taken on.
+"""
+import os
+import shutil
+
+import pytest
+
+import e2ttt_inputs as gen
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def gemm_flops(m, n, k):
+    return 2 * m * n * k
+
+
+def test_forward_flops_from_gemm_shapes(bench):
+    """Per chunk of C tokens and one head: G1 multiplies the 2C query and key rows
+    by the hidden weights, G2 the 2C activation rows by W2, G3 the C residual rows
+    by W2, G4 forms two weighted sums (a and b) for every state matrix."""
+    for name in ("layer_1p3b_2k", "swiglu_d128", "layer_1p3b_2k_gelu", "tiny_linear"):
+        w = gen.BY_NAME[name]
+        C, dk, dv, dh = w.C, w.d_k, w.d_v, w.d_h
+        if w.kind == gen.LINEAR:
+            ref = gemm_flops(2 * C, dv, dk) + 2 * gemm_flops(dv, dk, C)
+        else:
+            nf = 2 if w.kind == gen.SWIGLU else 1
+            ref = (gemm_flops(2 * C, nf * dh, dk) + gemm_flops(2 * C, dv, dh) + gemm_flops(C, dh, dv)
+                   + 2 * (gemm_flops(nf * dh, dk, C) + gemm_flops(dv, dh, C)))
+        got = sum(bench.phase_flops_per_token_head(w).values()) * C
+        assert got == ref, (name, got, ref)
+    w = gen.BY_NAME["layer_1p3b_2k"]
+    assert bench.fwd_flops(w) == 26 * w.d_k * w.d_h * w.B * w.H * w.T
+    g = gen.BY_NAME["layer_1p3b_2k_gelu"]
+    assert bench.fwd_flops(g) == 18 * g.d_k * g.d_h * g.B * g.H * g.T
+
+
+def test_backward_flops(bench):
+    """The tensor-core backward's phases: 52 d d_h of adjoint work per token and
+    head plus 12 of recomputed forward (R1 8, R2 2, R3 2); training counts the
+    forward and the 52 (twice the forward's 26)."""
+    assert sum(bench.TC_BWD_FLOPS.values()) == 64
+    assert bench.TC_BWD_FLOPS["tcb_r1_h"] + bench.TC_BWD_FLOPS["tcb_r2_e"] + bench.TC_BWD_FLOPS["tcb_r3_du"] == 12
+    w = gen.BY_NAME["train_1p3b_2k"]
+    assert bench.train_flops(w) == 78 * w.d_k * w.d_h * w.B * w.H * w.T
+
+
+def test_aggregation_bytes_chunk_by_chunk(bench):
+    """G4 of the 1.3B layer, one launch averaged over the step's chunks: bf16
+    operands (dH, aK, bK, aE, bE, A_k) read once per chunk; the fp32 state read
+    once (W0 only in the first chunk, W and M after), W and M written every chunk
+    and the bf16 copy of W written for every chunk but the last."""
+    w = gen.BY_NAME["layer_1p3b_2k"]
+    BH, C, NC = w.B * w.H, w.C, w.T // w.C
+    dk, dv, dh = w.d_k, w.d_v, w.d_h
+    S = 2 * dh * dk + dv * dh
+    operands = 2 * (2 * C * dh + 2 * C * dk + 2 * C * dv + C * dh)   # dH, aK, bK, aE, bE, A_k (bf16)
+    total = 0
+    for ci in range(NC):
+        reads = S * 4 if ci == 0 else 2 * S * 4      # M0 = 0 is not read
+        writes = 2 * S * 4 + (S * 2 if ci + 1 < NC else 0)
+        total += operands + reads + writes
+    per_launch = total / NC * BH
+    got = bench.kernel_work(w, has_m0=False)["tc_g4_aggregate_state"][1]
+    assert got == per_launch == 291504128.0
+
+
+def test_call_bytes_match_the_compulsory_traffic(bench):
+    """One forward call of the 1.3B layer: q, k, v in and out out (bf16), three
+    fp32 gates per token, W0 and M0 in, W_end and M_end out (fp32): about 336 MB."""
+    w = gen.BY_NAME["layer_1p3b_2k"]
+    toks = w.B * w.H * w.T
+    S = 2 * w.d_h * w.d_k + w.d_v * w.d_h
+    ref = toks * 2 * (w.d_k + w.d_k + w.d_v + w.d_v) + toks * 3 * 4 + 4 * w.B * w.H * S * 4
+    assert bench.algorithmic_bytes(w) == ref
+    assert 335e6 < ref < 337e6
+
+
+def test_recorded_traffic_needs_matching_sources(bench, tmp_path, monkeypatch):
+    """A profile's traffic figure is used only while the kernel sources hash to
+    the value recorded with it."""
+    src = tmp_path / "test_weight_layers_chunk_b200" / "csrc"
+    src.mkdir(parents=True)
+    for rel in bench.KERNEL_SOURCES["tc_"]:
+        shutil.copy(os.path.join(ROOT, rel), tmp_path / rel)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_source_sha("tc_g4_aggregate_state")
+    (tmp_path / "profiles").mkdir()
+    prof = tmp_path / "profiles" / "tc_g4_aggregate_state__layer_1p3b_2k.md"
+    prof.write_text(f"kernel_source_sha: {sha}\ntraffic_bytes_per_launch: 123456\n")
+    assert bench.recorded_traffic("tc_g4_aggregate_state", "layer_1p3b_2k") == 123456.0
+    with open(tmp_path / bench.KERNEL_SOURCES["tc_"][-1], "a") as f:
+        f.write("\n// changed\n")
+    assert bench.recorded_traffic("tc_g4_aggregate_state", "layer_1p3b_2k") is None
+    assert bench.recorded_traffic("tc_g4_aggregate_state", "other_workload") is None
