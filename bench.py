@@ -43,9 +43,11 @@ METRIC = "E2-TTT layer tokens/sec (fwd, fwd+bwd) at T=2K/16K; % of bf16 TC roofl
 UNIT = "tokens/s"
 _CSRC = "test_weight_layers_chunk_b200/csrc/"
 # the sources a kernel's recorded ncu traffic depends on, by kernel-name prefix
-KERNEL_SOURCES = {"tcb_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_bwd.cu"],
-                  "tc_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_fwd.cu"],
-                  "": [_CSRC + "scan.cu", _CSRC + "simt.cuh", _CSRC + "simt_fwd.cu", _CSRC + "bwd.cu"]}
+# (its translation unit and every header that unit compiles)
+_SHARED = [_CSRC + "common.cuh", _CSRC + "state.cuh", _CSRC + "paths.h", _CSRC + "trace.h"]
+KERNEL_SOURCES = {"tcb_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_bwd.cu"] + _SHARED,
+                  "tc_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_fwd.cu"] + _SHARED,
+                  "": [_CSRC + "scan.cu", _CSRC + "simt.cuh", _CSRC + "simt_fwd.cu", _CSRC + "bwd.cu"] + _SHARED}
 
 
 # ----------------------------------------------------------------- algorithmic work
