@@ -343,6 +343,35 @@ def _timed(torch, stream, fn, steps):
     return ev0.elapsed_time(ev1) / steps
 
 
+def measure_k1_large(E, torch, dev, stream, reps: int = 20) -> dict:
+    """K1 alone on B*H*T = 2^26 token-heads (64 heads x 2^20 tokens, C = 512), large
+    enough that its bandwidth means something: 12 B of gates in and 8 B of a, b
+    out per token-head plus 12 B of chunk scalars per chunk, once each. Gates are
+    drawn on the device in the workload's ranges (lr U(0.01, 0.1), momentum
+    U(0.8, 0.99), decay U(0.95, 1)); CUDA events on the launching stream, after
+    warm-up; the 1.3 GB touched per launch is ten times L2."""
+    BH, T, C = 64, 1 << 20, 512
+    g = torch.Generator(device=dev).manual_seed(26)
+    u = lambda lo, hi: lo + (hi - lo) * torch.rand((BH, T), generator=g, device=dev)
+    lr, mom, decay = u(0.01, 0.1), u(0.8, 0.99), u(0.95, 1.0)
+    a, b = torch.empty_like(lr), torch.empty_like(lr)
+    nc = T // C
+    sc = torch.empty((3, BH, nc), device=dev)
+    shape = E.make_shape(BH, 1, T, C, 1, 1, 0, E.LINEAR, E.F32)
+    run = lambda: E.e2ttt_chunk_coeffs(shape, lr, mom, decay, a, b, sc, stream=stream)
+    for _ in range(3):
+        run()
+    ms = _timed(torch, stream, run, reps)
+    by = 20.0 * BH * T + 12.0 * BH * nc
+    gbs = by / (ms / 1e3) / 1e9
+    peak = measured_peaks()
+    out = {"token_heads": BH * T, "us_per_launch": ms * 1e3, "bytes_per_launch": by, "gbs": gbs,
+           "frac": gbs / peak["hbm_gbs"], "peak_source": peak["source"] + " (copy bandwidth)"}
+    del lr, mom, decay, a, b, sc
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_extras(E, torch, dev, stream, args):
     """The metric's other operating points, device-timed like the main line:
     forward at T = 16K (the 8x length-extrapolation layer), forward+backward at
@@ -552,6 +581,12 @@ def run_ours(args, w):
     extras = {}
     if args.extras and rank == 0 and world == 1 and not train:
         extras = measure_extras(E, torch, dev, stream, args)
+    k1_large = None
+    if rank == 0 and not train:
+        try:   # an auxiliary measurement: its failure is reported, the line still prints
+            k1_large = measure_k1_large(E, torch, dev, stream)
+        except Exception as exc:  # noqa: BLE001
+            k1_large = {"error": f"{type(exc).__name__}: {exc}"}
 
     # End to end through the public API with pinned host buffers, pipelined the way
     # a serving loop runs: every step copies its inputs in (one copy stream),
@@ -636,7 +671,7 @@ def run_ours(args, w):
                 "config": config_dict(w, argparse.Namespace(gpus=world, mode=args.mode)),
                 "roofline": roofline, "step_roofline": whole, "kernels": kernels,
                 "gpu_launches": trace["launches"] // tsteps * args.steps, "clocks": clocks,
-                "cpu_baseline": cpu_baseline, "e2e": e2e, "extra": extras}
+                "cpu_baseline": cpu_baseline, "e2e": e2e, "k1_2e26": k1_large, "extra": extras}
         print(json.dumps(line))
     del graph, run_step  # release the captured graph before the process group
     if world > 1:
