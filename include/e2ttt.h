@@ -20,6 +20,7 @@
  *       l = 1/2 |f_W(k) - v|^2   (E2TTT_LOSS_MSE)   or   -<f_W(k), v>   (E2TTT_LOSS_NEG_DOT)
  *       f_W(x) = W x                          (E2TTT_LINEAR,  W  [d_v, d_k])
  *       f_W(x) = W2 (silu(W1 x) * (W3 x))     (E2TTT_SWIGLU,  W1, W3 [d_h, d_k], W2 [d_v, d_h])
+ *       f_W(x) = W2 gelu(W1 x)                (E2TTT_GELU_MLP, W1 [d_h, d_k], W2 [d_v, d_h])
  *   closed form (what the library computes):
  *       a_t = eta_t U(t+1,C),  b_t = eta_t sum_{j=t..C} L(j+1,C) U(t+1,j)
  *       M_end = U(1,C) M0 - sum_t a_t g_t
@@ -33,7 +34,8 @@
  *   v, out      [B, H, T, d_v]   activation dtype
  *   lr, mom, decay              [B, H, T] fp32 gate VALUES (not logits)
  *   W0, M0, W_end, M_end        [B, H, S] fp32, S = e2ttt_state_elems(shape):
- *        linear: W [d_v, d_k];  SwiGLU: [W1 | W3 | W2] concatenated
+ *        linear: W [d_v, d_k];  SwiGLU: [W1 | W3 | W2] concatenated;
+ *        GELU MLP: [W1 | W2] concatenated
  *   saved_states                [n_chunks, B, H, 2, S] fp32: (W, M) at the
  *                               start of every chunk (written by the forward,
  *                               read by the backward)
@@ -93,7 +95,8 @@ typedef enum { E2TTT_MOMENTUM = 0, E2TTT_NO_MOMENTUM = 1 } e2ttt_momentum;
 /* Problem description. kind/act/loss/coef/momentum hold e2ttt_fast_kind /
  * e2ttt_dtype / e2ttt_loss / e2ttt_coef / e2ttt_momentum values. d_h is ignored
  * (may be 0) for E2TTT_LINEAR.
- * Limits: all sizes >= 1; B*H*T*max(d_k,d_v,d_h) < 2^31; 1 <= C <= 1024. */
+ * Limits: all sizes >= 1; B*H <= 65535; B*H*T*max(d_k, d_v, 2 d_h) < 2^31
+ * (d_h counted for the MLPs only); 1 <= C <= 1024. */
 typedef struct {
   int B, H, T, C;
   int d_k, d_v, d_h;
@@ -122,9 +125,10 @@ int e2ttt_num_chunks(const e2ttt_shape* shape);
 int e2ttt_fwd_uses_tensor_cores(const e2ttt_shape* shape);
 
 /* The two scalar kernels of every chunk (atlas.scime.ai summary, "Approach":
- * momentum kernel and weight kernel from unrolling the token-wise
- * momentum-plus-decay recurrence, via log-space cumulative sums; arxivlens
- * "Results": "log-space suffix, ratio sums").
+ * the token-wise recurrence with momentum and decay, unrolled over a chunk,
+ * gives a momentum kernel and a weight kernel, computed from sums of logarithms;
+ * arxivlens "Results": their cost is sums over the tokens after t, taken in log
+ * space, and sums of ratios of gate products).
  *   a[b,h,t] = eta_t U(t+1,C)                       momentum kernel
  *   b[b,h,t] = eta_t sum_{j=t..C} L(j+1,C) U(t+1,j) weight kernel
  *   chunk_scalars [3, B, H, n_chunks]: U(1,C), L(1,C), sum_j L(j+1,C) U(1,j)
@@ -186,7 +190,8 @@ e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
 
 /* Backward of e2ttt_chunk_scan_fwd for the scalar objective
  *     L = sum_t <dout_t, out_t> + <dW_end, W_end> + <dM_end, M_end>
- * (abstract: "fully parallelized chunk-level training"). Chunks run in reverse;
+ * (abstract: with the closed form, training proceeds chunk by chunk with all
+ * tokens of a chunk in parallel). Chunks run in reverse;
  * the gradient of the chunk-end states flows into the previous chunk. Second
  * order terms through g_t(W0, k_t, v_t) are included (no stop-gradient).
  *   Inputs:  q, k, v, lr, mom, decay, saved_states (from the forward), dout

@@ -1,8 +1,8 @@
 // Backward of the chunk scan on fp32 CUDA cores (any shape; fp32 or bf16 activations).
 //
 // Adjoint of the closed-form chunk transition ("Rethinking Expressivity and
-// Efficiency in Test-Time Training": abstract, "fully parallelized chunk-level
-// training" through the closed form), chunks in reverse. For the scalar
+// Efficiency in Test-Time Training": abstract, training through the closed form
+// with all tokens of a chunk in parallel), chunks in reverse. For the scalar
 //   L = sum_t <dout_t, out_t> + <dW_end, W_end> + <dM_end, M_end>,
 // with D_W, D_M the adjoints of a chunk's end states and G_t = a_t D_M + b_t D_W:
 //   dM0   = U(1,n) D_M + c D_W

@@ -1,10 +1,11 @@
 // K1: the two scalar kernels of E2-TTT and their adjoint.
 //
 // "Rethinking Expressivity and Efficiency in Test-Time Training", atlas.scime.ai
-// summary, "Approach": a momentum kernel and a weight kernel come from unrolling
-// the token-wise momentum-plus-decay recurrence and are computed with log-space
-// cumulative sums; arxivlens summary, "Results": the extra work is a log-space
-// suffix and ratio sums. Per chunk of n tokens (1-based t), with
+// summary, "Approach": unrolling the token-wise recurrence with momentum and
+// decay over a chunk gives a momentum kernel and a weight kernel, computed from
+// sums of logarithms; arxivlens summary, "Results": the added cost is sums over
+// later tokens in log space and sums of ratios of gate products. Per chunk of n
+// tokens (1-based t), with
 // U(i,j) = prod mu, L(i,j) = prod lam over tokens i..j:
 //   SU_t = sum_{s>t} log mu_s,  SL_t = sum_{s>t} log lam_s     (suffix log-sums)
 //   a_t  = eta_t exp(SU_t)                                     (momentum kernel)
