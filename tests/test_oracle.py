@@ -431,6 +431,27 @@ def test_bf16_rounding_ties_to_even():
     np.testing.assert_array_equal(r, np.array([1.0, 1.0, 1.0 + 2 ** -6, 1.0, -2.5], np.float32))
 
 
+def test_bf16_rounding_matches_torch_conversion():
+    """The input module's bf16 rounding against torch's own float -> bf16
+    conversion (round to nearest, ties to even) on a million values spread over
+    the exponent range, both signs, exact ties, subnormals, the largest finite
+    values (which round to infinity) and non-finite inputs."""
+    import torch
+    rng = np.random.default_rng(7)
+    mant = rng.integers(0, 1 << 23, size=1 << 20, dtype=np.uint32)
+    expo = rng.integers(1, 255, size=1 << 20, dtype=np.uint32)
+    sign = rng.integers(0, 2, size=1 << 20, dtype=np.uint32)
+    x = ((sign << 31) | (expo << 23) | mant).view(np.float32)
+    ties = (((sign[:4096] << 31) | (expo[:4096] << 23) | (mant[:4096] & ~np.uint32(0xFFFF))
+             | np.uint32(0x8000))).view(np.float32)
+    special = np.array([0.0, -0.0, 1e-45, -3e-39, 3.3e38, -3.4028235e38, np.inf, -np.inf], np.float32)
+    x = np.concatenate([x, ties, special])
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(gen.round_to_bf16(x), ref)
+    nan = gen.round_to_bf16(np.array([np.nan], np.float32))
+    assert np.isnan(nan[0])
+
+
 # ------------------------------------------------------------------ chunk-averaged variant
 # atlas.scime.ai summary, "Surprising findings": the per-token factors collapsed to
 # chunk scalars (read as the chunk means of a_t and b_t; P_U, P_L, c unchanged).
