@@ -84,14 +84,26 @@ TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_du": 2, "tcb_d1_dir13": 8,
 
 
 def kernel_work(w, has_m0: bool) -> dict:
-    """Algorithmic work of one launch of each kernel: (FLOPs, bytes). One launch
-    covers one chunk of every head (the prep kernels: the whole step). Bytes count
-    every operand read once from HBM and every result written once; the fp32
-    state traffic of the aggregation is averaged over the chunks of a step (the
-    first chunk reads M0 only if one is given, the last writes no bf16 copy)."""
-    BH, C, T, NC = w.B * w.H, w.C, w.T, w.T // w.C
+    """Work of one launch of each kernel: (FLOPs, algorithmic bytes,
+    implementation bytes). One launch covers one chunk of every head (the prep
+    kernels and K1: the whole call).
+
+    Algorithmic bytes are the method's compulsory traffic: q, k, v and out once
+    in the activation dtype, the three gates once, W0 and M0 read and W_end and
+    M_end written once per call (fp32), each charged to the kernel that moves it
+    (q, k to the first GEMM phase, v, out to the phase that forms out and E, the
+    state to the aggregation phase, one chunk's share per launch). K1 is judged
+    as an operator of its own: gates in, a and b out, chunk scalars out. Traffic
+    of intermediates (activations, residuals, scaled operand copies, bf16 state
+    copies) and the per-chunk round trip of the state through HBM are
+    implementation overhead: they are in the implementation bytes (every operand
+    read once and every result written once, the state traffic averaged over the
+    chunks of a call), never in the algorithmic ones."""
+    BH, C, T, NC = w.B * w.H, w.C, w.T, -(-w.T // w.C)
     dk, dv, dh = w.d_k, w.d_v, w.d_h
-    out = {"k1_chunk_coeffs": (0.0, 20.0 * BH * T), "k1_chunk_coeffs_bwd": (0.0, 32.0 * BH * T)}
+    k1 = 20.0 * BH * T + 12.0 * BH * NC
+    out = {"k1_chunk_coeffs": (0.0, k1, k1),
+           "k1_chunk_coeffs_bwd": (0.0, 32.0 * BH * T, 32.0 * BH * T)}
     if w.kind == gen.LINEAR:
         return out
     nf = 2 if w.kind == gen.SWIGLU else 1            # activation factors per hidden unit
@@ -102,11 +114,12 @@ def kernel_work(w, has_m0: bool) -> dict:
     st_write = 8 * NC + 2 * (NC - 1)
     fl = phase_flops_per_token_head(w)
     g1, g3 = ("tc_g1_h_act", "tc_g3_da_dh") if nf == 2 else ("tc_g1_gelu", "tc_g3_gelu_dh")
+    state_alg = 16.0 * S / NC                        # W0, M0 in, W_end, M_end out, once per call
     per_head = {
-        g1: (fl[g1] * C, 2 * (2 * Mk + S13 + 2 * N + nf * N)),
-        "tc_g2_y_out_e": (fl["tc_g2_y_out_e"] * C, 2 * (2 * N + S2 + Mv + 4 * Mv)),
-        g3: (fl[g3] * C, 2 * (Mv + S2 + nf * N + nf * N)),
-        "tc_g4_aggregate_state": (fl["tc_g4_aggregate_state"] * C,
+        g1: (fl[g1] * C, 2 * 2 * Mk, 2 * (2 * Mk + S13 + 2 * N + nf * N)),
+        "tc_g2_y_out_e": (fl["tc_g2_y_out_e"] * C, 2 * 2 * Mv, 2 * (2 * N + S2 + Mv + 4 * Mv)),
+        g3: (fl[g3] * C, 0.0, 2 * (Mv + S2 + nf * N + nf * N)),
+        "tc_g4_aggregate_state": (fl["tc_g4_aggregate_state"] * C, state_alg,
                                   2 * (nf * N + 2 * Mk + 2 * Mv + N) + S * (st_read + st_write) / NC),
     }
     if dk == dv and nf == 2:
@@ -118,13 +131,35 @@ def kernel_work(w, has_m0: bool) -> dict:
              "tcb_q1_hbq": 2 * Mv + 2 * S2 + 8 * N, "tcb_dk1": 4 * N + 4 * S13 + 4 * Mk,
              "tcb_dk2": 4 * N + 2 * S13 + 6 * Mk, "tcb_dq": 4 * N + 2 * S13 + 2 * Mk,
              "tcb_dw": 14 * N + 4 * Mk + 6 * Mv + 8 * S}
+        # algorithmic bytes of the backward: q, k, v, dout read and dq, dk, dv
+        # written once (bf16); the saved chunk-start states read once (the shadow
+        # pass); dW0, dM0 written once per call (the dW phase, one chunk's share)
+        alg = {"tcb_r1_h": 2 * 2 * Mk, "tcb_r2_e": 2 * Mv, "tcb_q1_hbq": 2 * Mv,
+               "tcb_e4_eb": 2 * Mv, "tcb_dk2": 2 * Mk, "tcb_dq": 2 * Mk, "tcb_dw": 8.0 * S / NC}
         for n, by in b.items():
-            per_head[n] = (TC_BWD_FLOPS[n] * dd * C, by)
-        per_head["tcb_shadow"] = (0.0, 26 * S)
-    out.update({n: (f * BH, by * BH) for n, (f, by) in per_head.items()})
-    out["tc_shadow_init"] = (0.0, 6.0 * S * BH)
-    out["tc_scale_keys"] = (0.0, 6.0 * T * dk * BH)
+            per_head[n] = (TC_BWD_FLOPS[n] * dd * C, float(alg.get(n, 0.0)), by)
+        per_head["tcb_shadow"] = (0.0, 8.0 * S, 26.0 * S)
+    out.update({n: (f * BH, a * BH, by * BH) for n, (f, a, by) in per_head.items()})
+    out["tc_shadow_init"] = (0.0, 0.0, 6.0 * S * BH)
+    out["tc_scale_keys"] = (0.0, 0.0, 6.0 * T * dk * BH)
     return out
+
+
+def roofline_of(flops: float, alg_bytes: float, seconds: float, peaks: dict) -> dict:
+    """Bound and fraction of one launch from its algorithmic work: the slower of
+    FLOPs at the measured bf16 peak and bytes at the measured copy bandwidth
+    decides the bound; the fraction is the achieved rate over that peak."""
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        a = flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": a / peaks["bf16_tflops"], "algorithmic_per_launch": flops,
+                "peak_source": peaks["source"] + " (burst bf16 GEMM)"}
+    a = alg_bytes / seconds / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": a / peaks["hbm_gbs"], "algorithmic_per_launch": alg_bytes,
+            "peak_source": peaks["source"] + " (copy bandwidth)"}
 
 
 def fwd_flops(w) -> float:
@@ -258,28 +293,65 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- CPU oracle timing
-def oracle_sample(w, x, budget_s: float, max_heads=None):
-    """Run the fp64 closed-form oracle head by head until `budget_s` is spent.
-    Returns (layer tokens processed, seconds, heads, threads)."""
+def _pool_threads() -> int:
+    """Threads of the BLAS / OpenMP pools the oracle's numpy calls run on."""
+    from threadpoolctl import threadpool_info
+    return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+
+
+def oracle_sample(w, x, budget_s: float, routine: str = "closed", max_heads=None,
+                  max_tokens=None):
+    """Run one fp64 oracle routine head by head until `budget_s` is spent.
+    routine "closed": closed_fwd over whole heads; "seq": the per-token
+    recurrence seq_fwd over the first `max_tokens` tokens of each head (a
+    bounded sample: it is about 30 times slower). Returns (layer tokens
+    processed, seconds, heads, token count per head)."""
     import oracle as O
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = os.cpu_count() or 1
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
     if max_heads:
         heads = heads[:max_heads]
+    T = min(w.T, max_tokens) if max_tokens else w.T
     done = 0
     t0 = time.perf_counter()
-    for hh in heads:
-        O.closed_fwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"],
-                     x["M0"], w.C, d_h=w.d_h, loss=w.loss, heads=[hh])
+    for (b, h) in heads:
+        if routine == "closed":
+            O.closed_fwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"],
+                         x["M0"], w.C, d_h=w.d_h, loss=w.loss, heads=[(b, h)])
+        else:
+            sl = lambda a: a[b:b + 1, h:h + 1, :T]
+            O.seq_fwd(w.kind, sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["lr"]), sl(x["mom"]),
+                      sl(x["decay"]), x["W0"][b:b + 1, h:h + 1], x["M0"][b:b + 1, h:h + 1], w.C,
+                      d_h=w.d_h, loss=w.loss)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return done * w.T / w.H, dt, done, threads
+    # layer tokens = token-heads / H (a layer token carries all H heads)
+    return done * T / w.H, dt, done, T
+
+
+def cpu_baselines(w, x, budget_s: float) -> dict:
+    """The fp64 oracle on the host cores: closed_fwd and the per-token seq_fwd,
+    each single-threaded and with every core, over bounded samples of the
+    workload. The line's value is closed_fwd with every core (the fastest)."""
+    cores = os.cpu_count() or 1
+    runs = []
+    from threadpoolctl import threadpool_limits
+    for routine, limit in (("closed", None), ("closed", 1), ("seq", None), ("seq", 1)):
+        with threadpool_limits(limits=limit):
+            n = _pool_threads()
+            if routine == "closed":
+                tok, dt, nh, T = oracle_sample(w, x, budget_s, "closed")
+                sample = f"closed_fwd on {nh} of {w.B * w.H} heads x {T} tokens ({dt:.1f} s)"
+            else:
+                tok, dt, nh, T = oracle_sample(w, x, budget_s / 2, "seq", max_heads=1,
+                                               max_tokens=min(w.T, w.C))
+                sample = f"seq_fwd on {nh} head x its first {T} tokens ({dt:.1f} s)"
+        runs.append({"routine": routine + "_fwd", "threads": n, "value": tok / dt, "unit": UNIT,
+                     "sample": sample})
+    best = runs[0]
+    return {"value": best["value"], "unit": UNIT, "cores": best["threads"], "kind": "oracle",
+            "sample": best["sample"] + f"; host has {cores} cores", "runs": runs}
 
 
 def run_reference(args, w):
@@ -291,9 +363,9 @@ def run_reference(args, w):
         oracle_sample(w, x, 0.0, max_heads=1)
     tok = 0.0
     t0 = time.perf_counter()
-    threads = 1
+    threads = _pool_threads()
     for _ in range(args.steps):
-        t, _, _, threads = oracle_sample(w, x, 0.0, max_heads=1)
+        t, _, _, _ = oracle_sample(w, x, 0.0, max_heads=1)
         tok += t
     dt = time.perf_counter() - t0
     v = tok / dt
@@ -308,8 +380,11 @@ def run_reference(args, w):
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
 
 
+KIND_NAMES = {gen.LINEAR: "linear", gen.SWIGLU: "swiglu", gen.GELU: "gelu_mlp"}
+
+
 def config_dict(w, args):
-    return {"workload": w.name, "kind": "swiglu" if w.kind == gen.SWIGLU else "linear",
+    return {"workload": w.name, "kind": KIND_NAMES[w.kind],
             "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "d_h": w.d_h, "T": w.T, "C": w.C,
             "global_batch": w.B * args.gpus, "seq_len": w.T, "mode": args.mode,
             "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
@@ -374,14 +449,17 @@ def measure_k1_large(E, torch, dev, stream, reps: int = 20) -> dict:
 
 def measure_extras(E, torch, dev, stream, args):
     """The metric's other operating points, device-timed like the main line:
-    forward at T = 16K (the 8x length-extrapolation layer), forward+backward at
+    the forward of the tiny linear workload (fp32, CUDA cores) and of the d = 128
+    SwiGLU workload (both latency-bound), forward at T = 16K (the 8x length-extrapolation layer), forward+backward at
     T = 2K (the training workload), the forward at T = 2K of the
     chunk-averaged variant, of the no-momentum mode and of the GELU MLP fast
     weight, and the GELU MLP's forward+backward at T = 2K, each with its own
     warm-up."""
     out = {}
     f = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
-    for name, train, steps, coef, nomom in (("layer_1p3b_16k", False, args.extra_steps, 0, 0),
+    for name, train, steps, coef, nomom in (("tiny_linear", False, args.extra_steps, 0, 0),
+                                            ("swiglu_d128", False, args.extra_steps, 0, 0),
+                                            ("layer_1p3b_16k", False, args.extra_steps, 0, 0),
                                             ("train_1p3b_2k", True, max(2, args.extra_steps // 8), 0, 0),
                                             ("layer_1p3b_2k", False, args.extra_steps, 1, 0),
                                             ("layer_1p3b_2k", False, args.extra_steps, 0, 1),
@@ -389,7 +467,8 @@ def measure_extras(E, torch, dev, stream, args):
                                             ("layer_1p3b_2k_gelu", True, max(2, args.extra_steps // 8), 0, 0)):
         w = gen.BY_NAME[name]
         x = gen.generate(w)
-        q, k, v = f(x["q"], torch.bfloat16), f(x["k"], torch.bfloat16), f(x["v"], torch.bfloat16)
+        ad = torch.bfloat16 if w.act == gen.BF16 else torch.float32
+        q, k, v = f(x["q"], ad), f(x["k"], ad), f(x["v"], ad)
         lr, mom, decay, W0 = f(x["lr"]), f(x["mom"]), f(x["decay"]), f(x["W0"])
         shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss,
                              coef=coef, momentum=nomom)
@@ -398,7 +477,7 @@ def measure_extras(E, torch, dev, stream, args):
         saved = torch.empty((nc, w.B, w.H, 2, w.state_elems), device=dev) if train else None
         ws = E.workspace(shape, False, dev)
         if train:
-            dout = f(x["dout"], torch.bfloat16)
+            dout = f(x["dout"], ad)
             g = [torch.empty_like(t) for t in (q, k, v, lr, mom, decay, W0, W0)]
             wsb = E.workspace(shape, True, dev)
 
@@ -445,10 +524,7 @@ def run_ours(args, w):
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         xs = gen.generate(w)
-        tok, dt, nh, threads = oracle_sample(w, xs, args.cpu_budget)
-        cpu_baseline = {"value": tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-                        "sample": f"closed-form fp64 oracle on {nh} of {w.B * w.H} heads "
-                                  f"x {w.T} tokens ({dt:.1f} s)"}
+        cpu_baseline = cpu_baselines(w, xs, args.cpu_budget)
         del xs
 
     x = gen.generate(w, seed=w.seed + 1000 * rank)
@@ -528,7 +604,7 @@ def run_ours(args, w):
     tokens = w.B * w.T * args.steps * world
     value = tokens / (ms_max / 1e3)
 
-    # roofline of the dominant kernel
+    # roofline of the dominant kernel, from its algorithmic work
     peaks = measured_peaks()
     clocks = clk.summary()
     kern = trace["kernels"]
@@ -536,47 +612,48 @@ def run_ours(args, w):
     if w.kind == gen.SWIGLU and w.d_k == w.d_v:
         dd = w.d_k * w.d_h * w.B * w.H * w.C
         for n, f in BWD_SIMT_FLOPS.items():
-            work[n] = ("alu", f * dd)
+            work[n] = ("alu", f * dd, None)
     dom = max((n for n in kern if n in work), key=lambda n: kern[n]["total_ms"])
     avg_ms = kern[dom]["total_ms"] / kern[dom]["launches"]
     if isinstance(work[dom][0], str):      # CUDA-core backward kernel: fp32 FMA bound
-        bound, flops_launch = work[dom]
+        flops_launch = work[dom][1]
         achieved = flops_launch / (avg_ms / 1e3) / 1e12
         peak = fp32_fma_peak_tflops(clocks.get("sm_max_mhz") or 1965.0)
-        psrc, unit, alg = "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock", "TFLOP/s", flops_launch
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "algorithmic_per_launch": flops_launch,
+                    "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x max SM clock"}
     else:
-        flops_launch, bytes_launch = work[dom]
-        t_tensor = flops_launch / (peaks["bf16_tflops"] * 1e12)
-        t_hbm = bytes_launch / (peaks["hbm_gbs"] * 1e9)
-        if t_tensor >= t_hbm:
-            bound, alg, unit = "tensor", flops_launch, "TFLOP/s"
-            achieved = flops_launch / (avg_ms / 1e3) / 1e12
-            peak, psrc = peaks["bf16_tflops"], peaks["source"] + " (burst bf16 GEMM)"
-        else:
-            bound, alg, unit = "hbm", bytes_launch, "GB/s"
-            achieved = bytes_launch / (avg_ms / 1e3) / 1e9
-            peak, psrc = peaks["hbm_gbs"], peaks["source"] + " (copy bandwidth)"
-    roofline = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak, "peak_source": psrc,
-                "algorithmic_per_launch": alg, "avg_launch_us": avg_ms * 1e3,
-                "traffic": recorded_traffic(dom, w.name),
-                "share_of_step": kern[dom]["total_ms"] / ms}
+        flops_launch, alg_launch, impl_launch = work[dom]
+        roofline = roofline_of(flops_launch, alg_launch, avg_ms / 1e3, peaks)
+        roofline["implementation_bytes_per_launch"] = impl_launch
+        roofline["algorithmic_bytes_per_launch"] = alg_launch
+    roofline.update({"kernel": dom, "avg_launch_us": avg_ms * 1e3,
+                     "traffic": recorded_traffic(dom, w.name),
+                     "share_of_step": kern[dom]["total_ms"] / ms})
     step_flops = train_flops(w) if train else fwd_flops(w)
+    impl_step = sum(kv["launches"] * work[n][2] for n, kv in kern.items()
+                    if n in work and work[n][2] is not None) / tsteps
+    alg_step = algorithmic_bytes(w)
     whole = {"achieved_tflops": step_flops / (ms_max / args.steps / 1e3) / 1e12,
              "traced_ms_per_step": ms / tsteps, "traced_steps": tsteps,
              "timed_as": "cuda_graph_replay" if graph is not None else "stream_launches",
-             "stream_launch_ms_per_step": stream_ms}
+             "stream_launch_ms_per_step": stream_ms,
+             "algorithmic_bytes_per_step": alg_step,
+             "implementation_bytes_per_step": impl_step,
+             "implementation_over_algorithmic": impl_step / alg_step}
     whole["frac"] = whole["achieved_tflops"] / peaks["bf16_tflops"]
+    if peaks.get("bf16_tflops_sustained"):
+        whole["frac_sustained"] = whole["achieved_tflops"] / peaks["bf16_tflops_sustained"]
     kernels = {}
     for n, kv in kern.items():
         avg_s = kv["total_ms"] / kv["launches"] / 1e3
         kernels[n] = {"launches": kv["launches"], "avg_us": avg_s * 1e6, "share": kv["total_ms"] / ms}
         if n in work and not isinstance(work[n][0], str):
-            f, by = work[n]
-            kernels[n]["tflops"] = f / avg_s / 1e12
-            kernels[n]["gbs"] = by / avg_s / 1e9
-            kernels[n]["frac"] = max(f / avg_s / 1e12 / peaks["bf16_tflops"],
-                                     by / avg_s / 1e9 / peaks["hbm_gbs"])
+            f, alg, impl = work[n]
+            r = roofline_of(f, alg, avg_s, peaks)
+            kernels[n].update({"bound": r["bound"], "frac": r["frac"], "tflops": f / avg_s / 1e12,
+                               "alg_gbs": alg / avg_s / 1e9, "impl_gbs": impl / avg_s / 1e9,
+                               "impl_frac_hbm": impl / avg_s / 1e9 / peaks["hbm_gbs"]})
 
     extras = {}
     if args.extras and rank == 0 and world == 1 and not train:

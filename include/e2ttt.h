@@ -41,9 +41,13 @@
  *                               read by the backward)
  *
  * Conventions:
- *   - The library allocates no memory. Scratch comes from `workspace`
- *     (device memory of at least e2ttt_workspace_bytes(shape, for_bwd) bytes,
- *     256-byte aligned); its contents on entry do not matter.
+ *   - The library allocates no memory at run time. Scratch comes from
+ *     `workspace` (device memory of at least e2ttt_workspace_bytes(shape,
+ *     for_bwd) bytes, 256-byte aligned); its contents on entry do not matter.
+ *     One exception is made at load time: the library holds a 32 MiB static
+ *     __device__ array on every GPU where its kernels are loaded, for the life
+ *     of the process; only e2ttt_chunk_scan_fwd_noalloc (and
+ *     e2ttt_noalloc_status) use it.
  *   - Every compute call is asynchronous on `stream` (a cudaStream_t passed as
  *     void*; NULL = the legacy default stream). Argument checks run on the host
  *     before anything is launched and return E2TTT_ERR_INVALID_ARG or
@@ -175,18 +179,34 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* shape,
  *     kernels are loaded, for the life of the process.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     Calls outside capture look it up again, so a context made anew on the
+ *     device (after cudaDeviceReset) gets its own address; calls under capture
+ *     reuse the address the last uncaptured call found, so after a reset make
+ *     one uncaptured call before capturing again.
  *   - Shapes whose workspace (e2ttt_workspace_bytes(shape, 0)) exceeds 32 MiB
  *     return E2TTT_ERR_INVALID_ARG with the sizes in e2ttt_last_error(); the
  *     tiny linear and the d=128 SwiGLU workloads fit, the 1.3B layer does not.
  *   - All calls share the array and it keeps the last call's contents; calls
  *     that overlap on the GPU (several streams or host threads) race on it and
- *     must be serialised by the caller. */
+ *     must be serialised by the caller.
+ *   - The status of the device-side bounded waits is read with
+ *     e2ttt_noalloc_status (the caller never sees the array's address). */
 e2ttt_status e2ttt_chunk_scan_fwd_noalloc(const e2ttt_shape* shape,
                                           const void* q, const void* k, const void* v,
                                           const float* lr, const float* mom, const float* decay,
                                           const float* W0, const float* M0,
                                           void* out, float* W_end, float* M_end,
                                           float* saved_states, void* stream);
+
+/* Status of the device-side bounded waits of the last
+ * e2ttt_chunk_scan_fwd_noalloc call on the current device (the no-allocation
+ * counterpart of e2ttt_workspace_status, whose status word lives in the
+ * library's static array): synchronizes `stream`, then returns
+ * E2TTT_ERR_TIMEOUT if a tensor-core kernel gave up waiting (that call's
+ * outputs are then invalid), else E2TTT_OK; E2TTT_ERR_CUDA if there is no
+ * usable current device. Not for use under stream capture. No counterpart in
+ * the paper. */
+e2ttt_status e2ttt_noalloc_status(void* stream);
 
 /* Backward of e2ttt_chunk_scan_fwd for the scalar objective
  *     L = sum_t <dout_t, out_t> + <dW_end, W_end> + <dM_end, M_end>

@@ -61,6 +61,7 @@ _SIGS = {
     "e2ttt_chunk_scan_fwd_noalloc": (ctypes.c_int, [_S] + [_P] * 13),
     "e2ttt_chunk_scan_bwd": (ctypes.c_int, [_S] + [_P] * 19 + [ctypes.c_size_t, _P]),
     "e2ttt_workspace_status": (ctypes.c_int, [_P, _P]),
+    "e2ttt_noalloc_status": (ctypes.c_int, [_P]),
     "e2ttt_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "e2ttt_last_error": (ctypes.c_char_p, []),
     "e2ttt_trace_enable": (None, [ctypes.c_int]),
@@ -175,6 +176,14 @@ def e2ttt_chunk_scan_fwd_noalloc(shape, q, k, v, lr, mom, decay, W0, M0, out, W_
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(lr), _ptr(mom), _ptr(decay), _ptr(W0),
         _ptr(M0), _ptr(out), _ptr(W_end), _ptr(M_end), _ptr(saved_states),
         _stream(stream) if not raw else stream)
+    if raw:
+        return st
+    _check(st)
+
+
+def e2ttt_noalloc_status(stream=None, raw=False):
+    """Status word of the last no-allocation forward on the current device."""
+    st = _lib.e2ttt_noalloc_status(_stream(stream) if not raw else stream)
     if raw:
         return st
     _check(st)

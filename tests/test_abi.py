@@ -135,3 +135,14 @@ def test_gelu_mlp_state_size(E):
     g = E.make_shape(1, 2, 64, 16, 8, 6, 16, E.GELU_MLP, E.F32)
     assert E.e2ttt_state_elems(g) == 16 * 8 + 6 * 16
     assert E.e2ttt_workspace_bytes(g, 0) > 0 and E.e2ttt_workspace_bytes(g, 1) > 0
+
+
+def test_noalloc_status_without_a_device(E):
+    """The no-allocation status readout needs a current device: with none (this
+    CPU-only host) it returns E2TTT_ERR_CUDA with a message, never crashes."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the readout is covered by the GPU test")
+    st = E.e2ttt_noalloc_status(raw=True, stream=None)
+    assert st == E.ERR_CUDA
+    assert "e2ttt_noalloc_status" in E.e2ttt_last_error()

@@ -77,8 +77,41 @@ def test_aggregation_bytes_chunk_by_chunk(bench):
         writes = 2 * S * 4 + (S * 2 if ci + 1 < NC else 0)
         total += operands + reads + writes
     per_launch = total / NC * BH
-    got = bench.kernel_work(w, has_m0=False)["tc_g4_aggregate_state"][1]
+    got = bench.kernel_work(w, has_m0=False)["tc_g4_aggregate_state"][2]
     assert got == per_launch == 291504128.0
+
+
+def test_algorithmic_bytes_are_the_calls_compulsory_traffic(bench):
+    """The algorithmic bytes charged to the forward's launches add up to the
+    call's compulsory traffic less the gates (which K1 reads): q, k with the
+    first GEMM phase, v, out with the phase that forms out, W0, M0, W_end, M_end
+    once per call with the aggregation; intermediates and the per-chunk state
+    round trips are implementation bytes only."""
+    w = gen.BY_NAME["layer_1p3b_2k"]
+    NC = w.T // w.C
+    work = bench.kernel_work(w, has_m0=True)
+    per_call = sum(NC * work[n][1] for n in ("tc_g1_h_act", "tc_g2_y_out_e", "tc_g3_da_dh",
+                                             "tc_g4_aggregate_state"))
+    gates = 12 * w.B * w.H * w.T
+    assert per_call == bench.algorithmic_bytes(w) - gates
+    assert work["tc_shadow_init"][1] == work["tc_scale_keys"][1] == 0.0
+    # implementation bytes never undercount the algorithmic ones
+    for n, (f, alg, impl) in work.items():
+        assert impl >= alg, n
+
+
+def test_roofline_bound_follows_the_algorithmic_work(bench):
+    """G4 of the 1.3B layer does 12 d d_h FLOPs per token and head and carries a
+    quarter of the call's state bytes: at the measured peaks that is
+    tensor-bound, and the fraction is FLOPs / time / bf16 peak."""
+    w = gen.BY_NAME["layer_1p3b_2k"]
+    f, alg, impl = bench.kernel_work(w, has_m0=False)["tc_g4_aggregate_state"]
+    assert f == 12 * w.d_k * w.d_h * w.B * w.H * w.C
+    peaks = {"hbm_gbs": 6557.4, "bf16_tflops": 1667.1, "source": "measured"}
+    r = bench.roofline_of(f, alg, 57.97e-6, peaks)
+    assert r["bound"] == "tensor"
+    assert abs(r["frac"] - f / 57.97e-6 / 1667.1e12) < 1e-12
+    assert 0.26 < r["frac"] < 0.27
 
 
 def test_call_bytes_match_the_compulsory_traffic(bench):
