@@ -241,6 +241,17 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* shape,
  * of the workspace and is reset by every compute call. */
 e2ttt_status e2ttt_workspace_status(const void* workspace, void* stream);
 
+/* Failure-detection test hook (no counterpart in the paper). on = 1 arms it:
+ * the next e2ttt_chunk_scan_fwd that runs on the tensor cores makes one CTA of
+ * its first GEMM launch wait on an mbarrier that nothing ever completes, and
+ * limits every wait of that launch to 1 ms instead of 1 s. The wait runs out,
+ * the CTA records the failure in the workspace status word, waits (bounded) for
+ * its own copies in flight, frees its tensor memory and exits; no memory access
+ * is changed. e2ttt_workspace_status then returns E2TTT_ERR_TIMEOUT, that call's
+ * outputs are invalid, and the CUDA context stays usable: the next call runs
+ * normally. The hook disarms itself once used; on = 0 disarms it. */
+void e2ttt_test_stall_next_forward(int on);
+
 /* Launch tracing. While enabled, every kernel the library launches is
  * bracketed by a pair of CUDA events recorded on its launch stream (events are
  * created by the library and reused; no device memory is allocated).

@@ -65,6 +65,7 @@ _SIGS = {
     "e2ttt_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "e2ttt_last_error": (ctypes.c_char_p, []),
     "e2ttt_trace_enable": (None, [ctypes.c_int]),
+    "e2ttt_test_stall_next_forward": (None, [ctypes.c_int]),
     "e2ttt_trace_summary": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -120,6 +121,11 @@ def e2ttt_workspace_status(workspace, stream=None, raw=False):
     if raw:
         return st
     _check(st)
+
+
+def e2ttt_test_stall_next_forward(on: bool = True) -> None:
+    """Failure-detection test hook: the next tensor-core forward times out."""
+    _lib.e2ttt_test_stall_next_forward(int(bool(on)))
 
 
 def e2ttt_trace_enable(on: bool = True) -> None:

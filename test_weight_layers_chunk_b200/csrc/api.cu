@@ -232,6 +232,8 @@ e2ttt_status e2ttt_workspace_status(const void* ws, void* stream) {
   return E2TTT_OK;
 }
 
+void e2ttt_test_stall_next_forward(int on) { arm_forward_stall(on != 0); }
+
 e2ttt_status e2ttt_chunk_coeffs(const e2ttt_shape* s, const float* lr, const float* mom,
                                 const float* decay, float* a, float* b, float* scal,
                                 void* stream) {

@@ -33,6 +33,9 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
                    const float* M0, float* W_end, float* M_end, float* saved, void* scratch,
                    int* status, cudaStream_t st);
 
+// Test hook behind e2ttt_test_stall_next_forward (tc_fwd.cu).
+void arm_forward_stall(bool on);
+
 // Backward (bwd.cu).
 struct BwdArgs {
   Dims d;

@@ -295,6 +295,185 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   }
 }
 
+// Vectorised block version for full chunks of C = PER x 128 tokens: thread i
+// owns tokens [PER i, PER i + PER) of its chunk, loads its gates with one
+// PER-wide vector load per gate (all of them in flight at once), keeps them and
+// their logs in registers, and writes a_t, b_t with one vector store each. The
+// arithmetic, its order and the cross-thread combination are those of
+// chunk_coeffs_block_kernel, so the results are the same bit for bit; only the
+// memory access differs (the block kernel's per-token loop waited on one load
+// round trip per token).
+template <int PER>
+__device__ __forceinline__ void load_vec(const float* __restrict__ p, float (&v)[PER]) {
+  if constexpr (PER == 1) {
+    v[0] = p[0];
+  } else if constexpr (PER == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x; v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int j = 0; j < PER; j += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(p + j);
+      v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
+    }
+  }
+}
+template <int PER>
+__device__ __forceinline__ void store_vec(float* __restrict__ p, const float (&v)[PER]) {
+  if constexpr (PER == 1) {
+    p[0] = v[0];
+  } else if constexpr (PER == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < PER; j += 4)
+      *reinterpret_cast<float4*>(p + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  }
+}
+
+template <int PER>
+__global__ void __launch_bounds__(kK1Threads)
+chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                        const float* __restrict__ decay, float* __restrict__ a_out,
+                        float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
+                        int NC, int coef) {
+  __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
+  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
+  const size_t base = (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER;
+  float eta[PER], mu[PER], lam[PER];
+  load_vec<PER>(lr + base, eta);
+  if (mom) {
+    load_vec<PER>(mom + base, mu);
+  } else {  // no-momentum mode: mu = 0
+#pragma unroll
+    for (int i = 0; i < PER; ++i) mu[i] = 0.f;
+  }
+  load_vec<PER>(decay + base, lam);
+  float lmu[PER], llam[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    lmu[i] = logf(mu[i]);
+    llam[i] = logf(lam[i]);
+  }
+  s_mu_first[tid] = mu[0];
+  if (tid == 0) s_mu_first[kK1Threads] = 0.f;  // no token after the chunk's last
+
+  // suffix log-sums: exclusive (tokens after this segment) and chunk totals
+  float su = 0.f, sl = 0.f;
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    su += lmu[i];
+    sl += llam[i];
+  }
+  const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
+  if (lane == 0) {
+    w_su[warp] = su_inc;
+    w_sl[warp] = sl_inc;
+  }
+  __syncthreads();
+  float su_later = 0.f, sl_later = 0.f;  // warps after this one
+  for (int w = kK1Warps - 1; w > warp; --w) {
+    su_later += w_su[w];
+    sl_later += w_sl[w];
+  }
+  float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
+  float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
+  if (lane == 31) {
+    su_excl = 0.f;
+    sl_excl = 0.f;
+  }
+  su_excl += su_later;
+  sl_excl += sl_later;
+  float su_all = 0.f, sl_all = 0.f;
+  for (int w = kK1Warps - 1; w >= 0; --w) {
+    su_all += w_su[w];
+    sl_all += w_sl[w];
+  }
+  const float mu_next = s_mu_first[tid + 1];
+
+  // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map
+  su = su_excl;
+  sl = sl_excl;
+  float Mseg = 1.f, Cseg = 0.f;
+  float asum = 0.f, bsum = 0.f;
+  float av[PER], bv[PER];
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    av[i] = eta[i] * expf(su);
+    asum += av[i];
+    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+    Cseg = expf(sl) + m * Cseg;
+    Mseg = m * Mseg;
+    su += lmu[i];
+    sl += llam[i];
+  }
+  float M = Mseg, Cc = Cseg;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float Mr = __shfl_down_sync(0xffffffffu, M, off);
+    const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+    if (lane + off < 32) {
+      Cc = Cc + M * Cr;
+      M = M * Mr;
+    }
+  }
+  if (lane == 0) {
+    w_M[warp] = M;
+    w_C[warp] = Cc;
+  }
+  __syncthreads();
+  float r_end = 0.f;
+  for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
+  const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
+  const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
+  float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
+
+  // reverse walk 2: R_t and the weight kernel b_t
+  sl = sl_excl;
+  float r1 = 0.f;
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+    const float r = expf(sl) + m * r_next;
+    bv[i] = eta[i] * r;
+    bsum += bv[i];
+    r_next = r;
+    if (i == 0) r1 = r;
+    sl += llam[i];
+  }
+  if (coef) {  // the chunk-averaged variant: every token carries the chunk means
+    const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
+    __syncthreads();  // w_su / w_sl are free again
+    if (lane == 0) {
+      w_su[warp] = ai;
+      w_sl[warp] = bi;
+    }
+    __syncthreads();
+    float at = 0.f, bt = 0.f;
+    for (int w = kK1Warps - 1; w >= 0; --w) {
+      at += w_su[w];
+      bt += w_sl[w];
+    }
+    const float n = (float)(PER * kK1Threads);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      av[i] = at / n;
+      bv[i] = bt / n;
+    }
+  }
+  store_vec<PER>(a_out + base, av);
+  store_vec<PER>(b_out + base, bv);
+  if (tid == 0) {  // the thread holding token 1
+    const size_t plane = (size_t)BH * NC;
+    const size_t o = (size_t)bh * NC + ci;
+    scal[o] = expf(su_all);
+    scal[plane + o] = expf(sl_all);
+    scal[2 * plane + o] = mu[0] * r1;
+  }
+}
+
 // Adjoint of chunk_coeffs_kernel. Given abar, bbar (per token) and the chunk
 // scalar adjoints (PUbar, PLbar, cbar), with
 //   X_1 = PUbar, X_{s+1} = mu_s X_s + abar_s eta_s
@@ -447,6 +626,21 @@ cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* 
                                 float* b, float* scal, int BH, int T, int C, int NC, int coef,
                                 cudaStream_t st) {
   E2TTT_TRACE("k1_chunk_coeffs", st);
+  // Full chunks of 128, 256, 512 or 1024 tokens with vector-aligned gates and
+  // outputs: the vectorised kernel (same results as the block kernel).
+  const int per = C / kK1Threads;
+  const int vb = per >= 4 ? 16 : per * 4;  // alignment of one vector access in bytes
+  auto vec_ok = [&](const void* p) { return p == nullptr || ((uintptr_t)p % vb) == 0; };
+  if (T % C == 0 && C % kK1Threads == 0 && (per == 1 || per == 2 || per == 4 || per == 8) &&
+      vec_ok(lr) && vec_ok(mom) && vec_ok(decay) && vec_ok(a) && vec_ok(b)) {
+    switch (per) {
+      case 1: chunk_coeffs_vec_kernel<1><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      case 2: chunk_coeffs_vec_kernel<2><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      case 4: chunk_coeffs_vec_kernel<4><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      default: chunk_coeffs_vec_kernel<8><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+    }
+    return cudaGetLastError();
+  }
   if (C <= kK1MaxC) {
     const size_t smem = (size_t)4 * C * sizeof(float);
     if (smem > 48 * 1024) {

@@ -18,6 +18,8 @@
 // them as MN-major operands, so nothing is ever transposed.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "paths.h"
 #include "state.cuh"
 #include "tc_gemm2.cuh"
@@ -858,7 +860,15 @@ size_t carve(const Dims& d, char* base, Scratch* s) {
   return off;
 }
 
+// Failure-detection test hook (e2ttt_test_stall_next_forward): armed, it makes
+// the first GEMM launch of the next tensor-core forward stall one CTA on an
+// mbarrier nothing completes, with every wait of that launch limited to 1 ms.
+std::atomic<int> g_stall_next{0};
+constexpr unsigned long long kStallWaitNs = 1000000ull;
+
 }  // namespace
+
+void arm_forward_stall(bool on) { g_stall_next.store(on ? 1 : 0); }
 
 bool tc_fwd_supported(const Dims& d, bool bf16_act) {
   if (!bf16_act) return false;
@@ -1024,6 +1034,8 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
       if (!ok) return cudaErrorInvalidValue;
     }
     g1.cls[0].a.y_base = g1.cls[1].a.y_base = ci * C;  // query / key rows of this chunk
+    g1.stall = ci == 0 && g_stall_next.exchange(0) ? 1 : 0;
+    g1.wait_ns = g1.stall ? kStallWaitNs : 0;
     g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
     g4w.cls[0].b.y_base = ci * C;
     if (d.kind != 0) {

@@ -50,19 +50,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait for the phase with the given parity; false once `limit_ns` of
+// globaltimer time has passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0 && globaltimer() - t0 > kWaitNs) return false;
+    if ((i & 63) == 0 && globaltimer() - t0 > limit_ns) return false;
   }
 }
 // Bounded wait for the hot producer / MMA loops: try_wait with a short
 // suspend-time hint (20 ns), so a thread whose phase completes while it is
 // suspended resumes promptly instead of after the default suspend interval.
-__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity,
+                                               unsigned long long limit_ns = kWaitNs) {
   const unsigned long long t0 = globaltimer();
   for (uint32_t i = 0;; ++i) {
     uint32_t ok;
@@ -74,7 +77,7 @@ __device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity) {
         : "r"(smem_u32(bar)), "r"(parity), "r"(20u)
         : "memory");
     if (ok) return true;
-    if ((i & 255) == 255 && globaltimer() - t0 > kWaitNs) return false;
+    if ((i & 255) == 255 && globaltimer() - t0 > limit_ns) return false;
   }
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

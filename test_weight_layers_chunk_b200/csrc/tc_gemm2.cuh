@@ -103,6 +103,11 @@ struct Job {
   int heads;
   int total_tiles;
   int* status;
+  // Failure-detection test hook (0 = off): CTA 0's MMA issuer first waits on an
+  // mbarrier that nothing completes, and every wait of the launch gives up
+  // after wait_ns; the launch then reports a timeout in *status and exits.
+  int stall;
+  unsigned long long wait_ns;  // 0: the default limit (tc::kWaitNs)
 };
 
 template <int BN>
@@ -207,6 +212,8 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
   uint64_t* epi_bar = acc_empty + 2;     // [kEpiBars per epilogue warp]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + kEpiBars * EPI_WARPS);
   __shared__ int s_err;
+  __shared__ uint64_t never;  // the stall hook's mbarrier: nothing ever arrives on it
+  const unsigned long long lim = job.wait_ns ? job.wait_ns : tc::kWaitNs;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   griddep_launch_dependents();
@@ -221,6 +228,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       mbar_init(&acc_empty[b], EPI_WARPS);
     }
     for (int w = 0; w < kEpiBars * EPI_WARPS; ++w) mbar_init(&epi_bar[w], 1);
+    mbar_init(&never, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -253,7 +261,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       for (int kb = 0; kb < K.kblocks; kb += KG, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (it >= STAGES && !mbar_wait_hint(&empty[s], ph ^ 1u)) {
+        if (it >= STAGES && !mbar_wait_hint(&empty[s], ph ^ 1u, lim)) {
           atomicExch(job.status, kErrProducer);
           s_err = 1;
           ok = false;
@@ -278,7 +286,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
     }
     // no copy of ours may still be in flight when the CTA exits
     for (int j = it - STAGES < 0 ? 0 : it - STAGES; j < it; ++j)
-      (void)mbar_wait(&full[j % STAGES], (uint32_t)(j / STAGES) & 1u);
+      (void)mbar_wait(&full[j % STAGES], (uint32_t)(j / STAGES) & 1u, lim);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     constexpr uint32_t id = idesc(BM, BN, A_MN, B_MN);
@@ -290,13 +298,18 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
     const uint64_t dB0 = sdesc(smem_u32(ring), B_MN);
     int it = 0, i = 0;
     bool ok = true;
+    if (job.stall && blockIdx.x == 0 && !mbar_wait(&never, 0u, lim)) {
+      atomicExch(job.status, kErrMma);
+      s_err = 1;
+      ok = false;
+    }
     for (int t = blockIdx.x; t < job.total_tiles && ok; t += gridDim.x, ++i) {
       int c, z, mt, nt;
       decode_tile(job, t, c, z, mt, nt);
       const int kblocks = job.cls[c].kblocks;
       const bool a1b2 = NUM_ACC > 1 && job.cls[c].mode == kModeA1B2;
       const int b = i & 1;
-      if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u)) {
+      if (!mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, lim)) {
         atomicExch(job.status, kErrMma);
         s_err = 1;
         break;
@@ -306,7 +319,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       for (int kb = 0; kb < kblocks; kb += KG, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (!mbar_wait_hint(&full[s], ph)) {
+        if (!mbar_wait_hint(&full[s], ph, lim)) {
           atomicExch(job.status, kErrMma);
           s_err = 1;
           ok = false;
@@ -385,7 +398,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
         if (t + (int)gridDim.x < job.total_tiles && !s_err)
           pend[(i + 1) & 1] = Epi::prefetch(prm, make_ctx(t + gridDim.x, i + 1));
       }
-      if (!mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u)) {
+      if (!mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, lim)) {
         atomicExch(job.status, kErrEpilogue);
         s_err = 1;
         break;
@@ -401,7 +414,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
     }
     // no prefetch of ours may still be in flight when the CTA exits
     for (int k = 0; k < 2; ++k)
-      if (kPre && pend[k]) (void)mbar_wait(&epi_bar[kEpiBars * ew + k], uses[k] & 1u);
+      if (kPre && pend[k]) (void)mbar_wait(&epi_bar[kEpiBars * ew + k], uses[k] & 1u, lim);
     if (EPI_SMEM > 0 && lane == 0) tc::bulk_wait_all();  // our TMA stores have completed
     __syncwarp();
   }
@@ -410,7 +423,7 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
     if (lane == 0 && mma_tiles > 0) {
       // wait (bounded) until the last committed accumulator set is complete
       const int last = mma_tiles - 1;
-      (void)mbar_wait(&acc_full[last & 1], (uint32_t)(last >> 1) & 1u);
+      (void)mbar_wait(&acc_full[last & 1], (uint32_t)(last >> 1) & 1u, lim);
     }
     __syncwarp();
     tc_fence_after();

@@ -67,6 +67,52 @@ def test_chunk_coeffs_match_oracle(E, wi):
             assert abs(sc[i, bb, hh, c] - ref) <= TOL_COEF * abs(ref) + 1e-30, (i, ref, sc[i, bb, hh, c])
 
 
+@pytest.mark.parametrize("C", [128, 256, 512, 1024])
+@pytest.mark.parametrize("mode", ["per_token", "chunk_mean", "no_momentum"])
+def test_chunk_coeffs_vector_path_matches_block_path(E, C, mode):
+    """Full chunks of C = 128 x {1, 2, 4, 8} tokens with aligned buffers run the
+    vectorised K1 kernel; the same gates in buffers shifted by one float (not
+    vector-aligned) run the block kernel. Same arithmetic in the same order:
+    the results must agree bit for bit, and match the oracle."""
+    import torch
+    T = 4 * C
+    w = gen.Workload("k1v", gen.LINEAR, gen.F32, 2, 3, 8, 8, 0, T, C, "uniform", 0.9, seed=C)
+    x = gen.generate(w)
+    coef = E.COEF_CHUNK_MEAN if mode == "chunk_mean" else E.COEF_PER_TOKEN
+    mom_mode = E.NO_MOMENTUM if mode == "no_momentum" else E.MOMENTUM
+    s = E.make_shape(w.B, w.H, w.T, w.C, 8, 8, 0, E.LINEAR, E.F32, coef=coef, momentum=mom_mode)
+    nc = E.e2ttt_num_chunks(s)
+
+    def run(shift):
+        bufs = []
+        for name in ("lr", "mom", "decay"):
+            if name == "mom" and mode == "no_momentum":
+                bufs.append(None)
+                continue
+            t = torch.empty(w.B * w.H * T + shift, device="cuda")
+            t[shift:] = dev(x[name]).reshape(-1)
+            bufs.append(t[shift:].view(w.B, w.H, T))
+        outs = [torch.empty(w.B * w.H * T + shift, device="cuda")[shift:].view(w.B, w.H, T)
+                for _ in range(2)]
+        sc = torch.empty((3, w.B, w.H, nc), device="cuda")
+        E.e2ttt_chunk_coeffs(s, *bufs, outs[0], outs[1], sc)
+        torch.cuda.synchronize()
+        return outs[0], outs[1], sc
+
+    va, vb, vs = run(0)
+    ba, bb, bs = run(1)
+    assert torch.equal(va, ba) and torch.equal(vb, bb) and torch.equal(vs, bs)
+    mom = np.zeros_like(x["mom"]) if mode == "no_momentum" else x["mom"]
+    kern = O.chunk_mean_kernels if mode == "chunk_mean" else O.chunk_kernels
+    a, b = host(va), host(vb)
+    for bh in range(w.B * w.H):
+        bi, hi = divmod(bh, w.H)
+        for c in range(nc):
+            sl = slice(c * C, (c + 1) * C)
+            ra, rb, pu, pl, cc = kern(x["lr"][bi, hi, sl], mom[bi, hi, sl], x["decay"][bi, hi, sl])
+            assert rel(a[bi, hi, sl], ra) < TOL_COEF and rel(b[bi, hi, sl], rb) < TOL_COEF
+
+
 @pytest.mark.parametrize("edge", ["mu0", "lam1", "lam0", "ragged", "C1", "C1024"])
 def test_chunk_coeffs_edges(E, edge):
     T, C = 300, 64
