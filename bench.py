@@ -140,6 +140,9 @@ def kernel_work(w, has_m0: bool) -> dict:
             per_head[n] = (TC_BWD_FLOPS[n] * dd * C, float(alg.get(n, 0.0)), by)
         per_head["tcb_shadow"] = (0.0, 8.0 * S, 26.0 * S)
     out.update({n: (f * BH, a * BH, by * BH) for n, (f, a, by) in per_head.items()})
+    # the persistent forward: every chunk's four GEMM phases in one launch
+    phases = (g1, "tc_g2_y_out_e", g3, "tc_g4_aggregate_state")
+    out["tc_fwd_persistent"] = tuple(NC * sum(out[n][i] for n in phases) for i in range(3))
     out["tc_shadow_init"] = (0.0, 0.0, 6.0 * S * BH)
     out["tc_scale_keys"] = (0.0, 0.0, 6.0 * T * dk * BH)
     return out

@@ -18,6 +18,8 @@
 // them as MN-major operands, so nothing is ever transposed.
 #include <cuda.h>
 
+#include <stdlib.h>
+
 #include <atomic>
 
 #include "paths.h"
@@ -38,23 +40,22 @@ constexpr int HB = 128;  // hidden units per G1 tile (its 256 columns hold h1 th
 
 struct FwdP {
   // fp32 state tiles of the aggregation epilogue (3-D maps: columns, rows, heads)
-  // and the bf16 operand copies it writes; index = tile class (0: [W1; W3] or W,
-  // 1: W2). Rebuilt for every chunk.
-  CUtensorMap srcW[2], srcM[2], dstW[2], dstM[2], shadow[2];
+  // and the bf16 operand copies it writes; second index = tile class (0: [W1; W3]
+  // or W, 1: W2); first index of the source maps: 0 = the tile's chunk is the
+  // call's first (it reads W0, M0), 1 = a later chunk. The per-phase launches
+  // rebuild them for every chunk and fill both entries alike.
+  CUtensorMap srcW[2][2], srcM[2][2], dstW[2], dstM[2], shadow[2];
+  int hasM[2];  // whether the source momentum of variant 0 / 1 exists (M0 may be NULL)
   // 32 x 32 bf16 tiles (64B swizzle) moved by the other epilogues; mOut and mV
   // are 3-D (columns, tokens, heads), so a box past a head's last token is
   // clipped on store and reads as zero
   CUtensorMap mA, mSk, mOut, mV, mE, mEa, mEb, mdH;
   Dims d;
-  int ci, t0, write_shadow;
-  int clen;   // tokens of this chunk: C, or T - t0 for a shorter last chunk
   int nomom;  // no momentum: no a-scaled operands, W-only aggregation epilogue
   int* status;
   const bf16 *q, *k, *v;
   bf16* out;
   const float *ca, *cb, *scal;
-  StateIn src;
-  StateOut dst;
   bf16 *Wsh13, *W2sh;  // bf16 copies of the chunk-start weights (Wsh13 = W for linear)
   bf16 *A, *Sk, *E, *Ea, *Eb, *dH, *Ka, *Kb;
 };
@@ -279,12 +280,12 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
   const int ngroups = per / 32;
   uint8_t* V = c.wsmem;            // [2][2 KB]
   uint8_t* S = c.wsmem + 4096;     // E | Ea | Eb staging
-  const int ttok = p.t0 + r0;      // first token (within the head) of this warp's rows
+  const int ttok = c.t0 + r0;      // first token (within the head) of this warp's rows
   const int yrow = c.z * d.C + r0;
   // Padding rows: no output, and E = a E = b E = 0, so they add nothing to any
   // later sum over tokens.
-  const bool real = !PAD || lane < p.clen - r0;
-  if (PAD && !key_rows && p.clen - r0 <= 0) return;  // no query row of this warp is real
+  const bool real = !PAD || lane < c.clen - r0;
+  if (PAD && !key_rows && c.clen - r0 <= 0) return;  // no query row of this warp is real
   if (key_rows) {
     if (lane == 0) {
       tc::mbar_expect_tx(&c.wbar[0], 2048u * ngroups);
@@ -375,8 +376,11 @@ using EpiG1Lin = EpiG1LinT<false>;
 using EpiG1LinPad = EpiG1LinT<true>;
 
 // G3, SwiGLU: dA -> dH1 = dA H3 silu'(H1), dH3 = dA silu(H1) (rows: tokens).
+// The silu factors of a column group arrive by TMA in a 4 KB buffer; once read
+// into registers, the same buffer stages that group's dH1 | dH3 for the TMA
+// stores (each lane reads and then writes only its own row).
 struct EpiG3 {
-  static constexpr int kSmem = 12288;  // silu factors [2 groups][2] | dH1 | dH3
+  static constexpr int kSmem = 8192;  // [2 groups][silu(H1) | H3 silu'(H1), then dH3 | dH1]
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
@@ -387,9 +391,9 @@ struct EpiG3 {
     static_assert(BN <= 128, "silu-factor buffers for at most two column groups per warp");
     const int ngroups = per / 32;
     const int y = c.z * d.C + r0;
-    uint8_t* F = c.wsmem;          // [group][s1 | s2] 2 KB each
-    uint8_t* S = c.wsmem + 8192;   // dH1 | dH3 staging
+    uint8_t* F = c.wsmem;  // [group][s1 | s2] 2 KB each
     if (lane == 0) {
+      tc::bulk_wait_read<0>();  // the previous tile's stores have read the buffers
       tc::mbar_expect_tx(&c.wbar[0], 4096u * ngroups);
       for (int gi = 0; gi < ngroups; ++gi) {
         tc::tma_load_2d(F + gi * 4096, &p.mSk, &c.wbar[0], col0 + gi * 32, y);
@@ -408,20 +412,20 @@ struct EpiG3 {
           return;
         }
       }
-      unstage32(F + gi * 4096, lane, s1);
-      unstage32(F + gi * 4096 + 2048, lane, s2);
+      uint8_t* G = F + gi * 4096;
+      unstage32(G, lane, s1);
+      unstage32(G + 2048, lane, s2);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         s2[i] *= da[i];  // dH1
         s1[i] *= da[i];  // dH3
       }
-      staging_free(lane);
-      stage32(S, lane, s2);
-      stage32(S + 2048, lane, s1);
+      stage32(G, lane, s2);
+      stage32(G + 2048, lane, s1);
       staging_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.mdH, S, col0 + gi * 32, y);
-        tc::tma_store_2d(&p.mdH, S + 2048, d.d_h + col0 + gi * 32, y);
+        tc::tma_store_2d(&p.mdH, G, col0 + gi * 32, y);
+        tc::tma_store_2d(&p.mdH, G + 2048, d.d_h + col0 + gi * 32, y);
         tc::bulk_commit();
       }
       __syncwarp();
@@ -446,13 +450,13 @@ struct EpiG4 {
   static constexpr int kSlots = 2;
   static constexpr int kSmem = kSlots * kSlot;
   static __device__ __forceinline__ void issue(const FwdP& p, const uint8_t* wsmem, uint64_t* wbar,
-                                               int q, int g, int cls, int z, int r0, int n0) {
+                                               int q, int g, int cls, int z, int r0, int n0, int var) {
     const int sidx = q % kSlots;
     uint8_t* slot = const_cast<uint8_t*>(wsmem) + sidx * kSlot;
-    const bool hasM = p.src.M != nullptr;
+    const bool hasM = p.hasM[var];
     tc::mbar_expect_tx(&wbar[sidx], hasM ? 8192u : 4096u);
-    tc::tma_load_3d(slot, &p.srcW[cls], &wbar[sidx], n0 + g * 32, r0, z);
-    if (hasM) tc::tma_load_3d(slot + 4096, &p.srcM[cls], &wbar[sidx], n0 + g * 32, r0, z);
+    tc::tma_load_3d(slot, &p.srcW[var][cls], &wbar[sidx], n0 + g * 32, r0, z);
+    if (hasM) tc::tma_load_3d(slot + 4096, &p.srcM[var][cls], &wbar[sidx], n0 + g * 32, r0, z);
   }
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
@@ -461,9 +465,10 @@ struct EpiG4 {
     const int r0 = c.m0 + c.quad * 32;  // first state row of this warp
     constexpr int kGroups = BN / 32;
     static_assert(kGroups >= 2, "two groups ahead");
-    const bool hasM = p.src.M != nullptr;
+    const int var = c.ci == 0 ? 0 : 1;
+    const bool hasM = p.hasM[var];
     const size_t plane = (size_t)d.BH * d.NC;
-    const size_t so = (size_t)c.z * d.NC + p.ci;
+    const size_t so = (size_t)c.z * d.NC + c.ci;
     const float PU = p.scal[so], PL = p.scal[plane + so], cc = p.scal[2 * plane + so];
     int sh_row;
     if (c.cls == 0 && d.kind == 1) {
@@ -474,10 +479,10 @@ struct EpiG4 {
     } else {
       sh_row = c.z * d.d_v + r0;
     }
-    const int q0 = c.iter * kGroups;
-    if (c.iter == 0 && lane == 0) {
-      issue(p, c.wsmem, c.wbar, q0, 0, c.cls, c.z, r0, c.n0);
-      issue(p, c.wsmem, c.wbar, q0 + 1, 1, c.cls, c.z, r0, c.n0);
+    const int q0 = c.seq * kGroups;
+    if (!c.pre && lane == 0) {
+      issue(p, c.wsmem, c.wbar, q0, 0, c.cls, c.z, r0, c.n0, var);
+      issue(p, c.wsmem, c.wbar, q0 + 1, 1, c.cls, c.z, r0, c.n0, var);
     }
     __syncwarp();
     for (int g = 0; g < kGroups; ++g) {
@@ -523,15 +528,15 @@ struct EpiG4 {
       if (lane == 0) {
         tc::tma_store_3d(&p.dstW[c.cls], slot, c.n0 + g * 32, r0, c.z);
         tc::tma_store_3d(&p.dstM[c.cls], slot + 4096, c.n0 + g * 32, r0, c.z);
-        if (p.write_shadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 8192, c.n0 + g * 32, sh_row);
+        if (c.wshadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 8192, c.n0 + g * 32, sh_row);
         tc::bulk_commit();
         tc::bulk_wait_read<0>();  // group q's stores have read the slot of group q + 2
         const int gn = g + 2;
         if (gn < kGroups) {
-          issue(p, c.wsmem, c.wbar, q + 2, gn, c.cls, c.z, r0, c.n0);
+          issue(p, c.wsmem, c.wbar, q + 2, gn, c.cls, c.z, r0, c.n0, var);
         } else if (c.nxt_valid) {
           issue(p, c.wsmem, c.wbar, q + 2, gn - kGroups, c.nxt_cls, c.nxt_z,
-                c.nxt_m0 + c.quad * 32, c.nxt_n0);
+                c.nxt_m0 + c.quad * 32, c.nxt_n0, c.nxt_ci == 0 ? 0 : 1);
         }
       }
       __syncwarp();
@@ -547,11 +552,11 @@ struct EpiG4W {
   static constexpr int kSlots = 3;
   static constexpr int kSmem = kSlots * kSlot;
   static __device__ __forceinline__ void issue(const FwdP& p, const uint8_t* wsmem, uint64_t* wbar,
-                                               int q, int g, int cls, int z, int r0, int n0) {
+                                               int q, int g, int cls, int z, int r0, int n0, int var) {
     const int sidx = q % kSlots;
     uint8_t* slot = const_cast<uint8_t*>(wsmem) + sidx * kSlot;
     tc::mbar_expect_tx(&wbar[sidx], 4096u);
-    tc::tma_load_3d(slot, &p.srcW[cls], &wbar[sidx], n0 + g * 32, r0, z);
+    tc::tma_load_3d(slot, &p.srcW[var][cls], &wbar[sidx], n0 + g * 32, r0, z);
   }
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
@@ -561,7 +566,8 @@ struct EpiG4W {
     constexpr int kGroups = BN / 32;
     static_assert(kGroups >= 2, "two groups ahead");
     const size_t plane = (size_t)d.BH * d.NC;
-    const float PL = p.scal[plane + (size_t)c.z * d.NC + p.ci];
+    const float PL = p.scal[plane + (size_t)c.z * d.NC + c.ci];
+    const int var = c.ci == 0 ? 0 : 1;
     int sh_row;
     if (c.cls == 0 && d.kind == 1) {
       const int which = r0 / d.d_h, rr = r0 % d.d_h;
@@ -571,10 +577,10 @@ struct EpiG4W {
     } else {
       sh_row = c.z * d.d_v + r0;
     }
-    const int q0 = c.iter * kGroups;
-    if (c.iter == 0 && lane == 0) {
-      issue(p, c.wsmem, c.wbar, q0, 0, c.cls, c.z, r0, c.n0);
-      issue(p, c.wsmem, c.wbar, q0 + 1, 1, c.cls, c.z, r0, c.n0);
+    const int q0 = c.seq * kGroups;
+    if (!c.pre && lane == 0) {
+      issue(p, c.wsmem, c.wbar, q0, 0, c.cls, c.z, r0, c.n0, var);
+      issue(p, c.wsmem, c.wbar, q0 + 1, 1, c.cls, c.z, r0, c.n0, var);
     }
     __syncwarp();
     for (int g = 0; g < kGroups; ++g) {
@@ -607,15 +613,15 @@ struct EpiG4W {
       __syncwarp();
       if (lane == 0) {
         tc::tma_store_3d(&p.dstW[c.cls], slot, c.n0 + g * 32, r0, c.z);
-        if (p.write_shadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 4096, c.n0 + g * 32, sh_row);
+        if (c.wshadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 4096, c.n0 + g * 32, sh_row);
         tc::bulk_commit();
         tc::bulk_wait_read<1>();  // the slot of group q - 1 is free for group q + 2
         const int gn = g + 2;
         if (gn < kGroups) {
-          issue(p, c.wsmem, c.wbar, q + 2, gn, c.cls, c.z, r0, c.n0);
+          issue(p, c.wsmem, c.wbar, q + 2, gn, c.cls, c.z, r0, c.n0, var);
         } else if (c.nxt_valid) {
           issue(p, c.wsmem, c.wbar, q + 2, gn - kGroups, c.nxt_cls, c.nxt_z,
-                c.nxt_m0 + c.quad * 32, c.nxt_n0);
+                c.nxt_m0 + c.quad * 32, c.nxt_n0, c.nxt_ci == 0 ? 0 : 1);
         }
       }
       __syncwarp();
@@ -634,6 +640,460 @@ template <> struct EpiName<EpiG1Gelu> { static constexpr const char* v = "tc_g1_
 template <> struct EpiName<EpiG3Gelu> { static constexpr const char* v = "tc_g3_gelu_dh"; };
 template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 template <> struct EpiName<EpiG1LinPad> { static constexpr const char* v = "tc_g1_linear_out_e"; };
+
+// ---------------------------------------------------------------- persistent forward
+// The whole SwiGLU forward (every chunk, G1 to G4) in one cooperative launch.
+// Each CTA (one per SM) walks a static list of the tiles of all four GEMM phases
+// of all chunks: chunk by chunk, and inside a chunk group by group of hg heads,
+// phase after phase within a group. A tile of phase p for head z and chunk ci
+// may start once the tiles its inputs come from are done: G1 after every G4
+// tile of (z, ci - 1) (the bf16 copy of the chunk-start weights, and no reader of
+// the previous chunk's scratch is left), G2 after G1 of (z, ci), G3 after G2, G4
+// after G3. Completed tiles are counted per (phase, head) in global counters
+// (release increments after the tile's stores have completed; bounded acquire
+// spins before the first read of a tile's inputs). Dependencies only point to
+// earlier tiles of the list, and every CTA is resident (cooperative launch), so
+// the earliest unfinished tile can always run. Heads of a later group (or a
+// later chunk) run while an earlier group aggregates: the HBM-bound state
+// epilogue of G4 overlaps the tensor-core phases of other heads, and no kernel
+// boundary separates the phases.
+//
+// One configuration serves the four phases: a ring of three 48 KB stages (G1:
+// A 16 KB + B 32 KB; G4: three 16 KB operand tiles; G2, G3: 32 KB), two TMEM
+// accumulator sets of 256 columns (G1: one 128 x 256 accumulator; G4: two 128 x
+// 128; G2, G3: one 128 x 128), eight epilogue warps of 10 KB (G4: four warps of
+// 20 KB, the other four idle for its tiles).
+namespace mk {
+constexpr int kStages = 3;
+constexpr uint32_t kSlot = 49152;
+constexpr int kEW = 8;
+constexpr int kEpiSmem = 10240;
+constexpr int kEpiSmemG4 = 20480;
+constexpr uint32_t kAcc = 256;
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kSlot + (size_t)kEW * kEpiSmem + 1024;
+static_assert(EpiG1::kSmem <= kEpiSmem && EpiG2::kSmem <= kEpiSmem && EpiG3::kSmem <= kEpiSmem,
+              "epilogue buffers of G1-G3 fit the 10 KB per warp");
+static_assert(4 * kEpiSmemG4 <= kEW * kEpiSmem && EpiG4::kSmem <= kEpiSmemG4, "G4 epilogue buffers fit");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+enum : int { kErrDep = 4 };
+}  // namespace mk
+
+struct MegaJob {
+  tc2::Job ph[4];   // maps and tile classes of G1..G4 (y_base of every operand 0)
+  int tph[4];       // tiles per head of each phase
+  int BH, NC, C, hg;
+  int per_group;    // tiles of one group of hg heads in one chunk (all phases)
+  int per_chunk;    // tiles of one chunk
+  int total;        // tiles of the call
+  int* cnt;         // [4][BH] completed tiles per (phase, head), zero at launch
+  int* status;
+  unsigned long long wait_ns;
+  int stall;        // failure-detection test hook, as in tc2::Job
+};
+
+struct MkTile {
+  int ph, ci, z, cls, mt, nt;
+};
+
+__device__ __forceinline__ MkTile mk_decode(const MegaJob& J, int t) {
+  MkTile r;
+  r.ci = t / J.per_chunk;
+  int x = t - r.ci * J.per_chunk;
+  const int g = x / J.per_group;
+  x -= g * J.per_group;
+  r.ph = 0;
+  while (r.ph < 3 && x >= J.hg * J.tph[r.ph]) {
+    x -= J.hg * J.tph[r.ph];
+    ++r.ph;
+  }
+  const tc2::Job& P = J.ph[r.ph];
+  r.cls = 0;
+  const int per0 = P.cls[0].tiles_m * P.cls[0].tiles_n * J.hg;
+  if (P.n_cls > 1 && x >= per0) {
+    x -= per0;
+    r.cls = 1;
+  }
+  const tc2::Class& K = P.cls[r.cls];
+  const int per_head = K.tiles_m * K.tiles_n;
+  const int zl = x / per_head;
+  x -= zl * per_head;
+  r.z = g * J.hg + zl;
+  r.mt = x / K.tiles_n;
+  r.nt = x - r.mt * K.tiles_n;
+  return r;
+}
+// Completed tiles of the producing phase that tile T needs (dphase < 0: none).
+__device__ __forceinline__ void mk_need(const MegaJob& J, const MkTile& T, int& dphase, int& target) {
+  if (T.ph == 0) {
+    dphase = T.ci > 0 ? 3 : -1;
+    target = T.ci * J.tph[3];
+  } else {
+    dphase = T.ph - 1;
+    target = (T.ci + 1) * J.tph[T.ph - 1];
+  }
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bounded wait until the tile's inputs are complete; then order the async-proxy
+// (TMA) reads that follow after the acquire.
+__device__ __forceinline__ bool mk_dep_wait(const MegaJob& J, const MkTile& T, unsigned long long lim) {
+  int dp, tg;
+  mk_need(J, T, dp, tg);
+  if (dp >= 0) {
+    const int* c = J.cnt + (size_t)dp * J.BH + T.z;
+    if (ld_acquire(c) < tg) {
+      const unsigned long long t0 = tc::globaltimer();
+      for (uint32_t i = 1;; ++i) {
+        __nanosleep(64);
+        if (ld_acquire(c) >= tg) break;
+        if ((i & 15) == 0 && tc::globaltimer() - t0 > lim) return false;
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+__device__ __forceinline__ bool mk_dep_ready(const MegaJob& J, const MkTile& T) {
+  int dp, tg;
+  mk_need(J, T, dp, tg);
+  return dp < 0 || ld_acquire(J.cnt + (size_t)dp * J.BH + T.z) >= tg;
+}
+__device__ __forceinline__ void epi_barrier() {  // the eight epilogue warps
+  asm volatile("bar.sync 1, %0;" ::"n"(mk::kEW * 32) : "memory");
+}
+
+template <bool MN, int ROWS>
+__device__ __forceinline__ void mk_load(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
+                                        const tc2::Opnd& o, int yoff, int z, int origin, int kb) {
+  tc2::Opnd q = o;
+  q.y_base += yoff;
+  tc2::load_opnd<MN, ROWS>(dst, map, bar, q, z, origin, kb);
+}
+
+__global__ void __launch_bounds__((2 + mk::kEW) * 32, 1)
+fwd_persistent(const __grid_constant__ MegaJob J, const __grid_constant__ FwdP prm) {
+  using namespace mk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint8_t* epi_smem = smem + (size_t)kStages * kSlot;
+  __shared__ uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2];
+  __shared__ uint64_t epi_bar[tc2::kEpiBars * kEW];
+  __shared__ uint64_t never;  // the stall hook's mbarrier: nothing ever arrives on it
+  __shared__ uint32_t tmem_slot;
+  __shared__ int s_err_;
+  volatile int& s_err = s_err_;  // set by any role on failure, read by all
+  const unsigned long long lim = J.wait_ns ? J.wait_ns : tc::kWaitNs;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    s_err = 0;
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&acc_full[b], 1);
+      tc::mbar_init(&acc_empty[b], kEW);
+    }
+    for (int w = 0; w < tc2::kEpiBars * kEW; ++w) tc::mbar_init(&epi_bar[w], 1);
+    tc::mbar_init(&never, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int p = 0; p < 4; ++p) {
+      tc::prefetch_tmap(&J.ph[p].maps[0].op0);
+      tc::prefetch_tmap(&J.ph[p].maps[0].op2);
+    }
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&tmem_slot, 2 * kAcc);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  int mma_tiles = 0;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < J.total && ok; t += gridDim.x) {
+      const MkTile T = mk_decode(J, t);
+      if (!mk_dep_wait(J, T, lim)) {
+        atomicExch(J.status, kErrDep);
+        s_err = 1;
+        break;
+      }
+      const tc2::Job& P = J.ph[T.ph];
+      const tc2::Class& K = P.cls[T.cls];
+      const tc2::Maps& M = P.maps[T.cls];
+      const int aoff = T.ph == 0 ? T.ci * J.C : 0;                // query / key rows of the chunk
+      const int boff = (T.ph == 3 && T.cls == 0) ? T.ci * J.C : 0;  // key rows (K dim) of the chunk
+      const uint32_t bytes = (T.ph == 1 || T.ph == 2) ? 32768u : 49152u;
+      for (int kb = 0; kb < K.kblocks; ++kb, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (it >= kStages && !tc::mbar_wait_hint(&empty[s], ph ^ 1u, lim)) {
+          atomicExch(J.status, tc2::kErrProducer);
+          s_err = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* st = ring + (size_t)s * kSlot;
+        tc::mbar_expect_tx(&full[s], bytes);
+        const int m0 = T.mt * tc::BM;
+        switch (T.ph) {
+          case 0:  // [q; k] rows x [W1; W3] (interleaved), both K-major, N = 256
+            mk_load<false, 128>(st, &M.op0, &full[s], K.a, aoff, T.z, m0, kb);
+            mk_load<false, 256>(st + 16384, &M.op2, &full[s], K.b, 0, T.z, T.nt * 256, kb);
+            break;
+          case 1:  // A = [u_q; u_k], B = W2, K-major, N = 128
+            mk_load<false, 128>(st, &M.op0, &full[s], K.a, 0, T.z, m0, kb);
+            mk_load<false, 128>(st + 16384, &M.op2, &full[s], K.b, 0, T.z, T.nt * 128, kb);
+            break;
+          case 2:  // A = E (K-major), B = W2 read MN-major, N = 128
+            mk_load<false, 128>(st, &M.op0, &full[s], K.a, 0, T.z, m0, kb);
+            mk_load<true, 128>(st + 16384, &M.op2, &full[s], K.b, 0, T.z, T.nt * 128, kb);
+            break;
+          default:  // the two aggregations, all operands MN-major
+            if (K.mode == tc2::kModeA2B1) {
+              mk_load<true, 128>(st, &M.op0, &full[s], K.a, 0, T.z, m0, kb);
+              mk_load<true, 128>(st + 16384, &M.op1, &full[s], K.a, 0, T.z, m0, kb);
+              mk_load<true, 128>(st + 32768, &M.op2, &full[s], K.b, boff, T.z, T.nt * 128, kb);
+            } else {
+              mk_load<true, 128>(st, &M.op0, &full[s], K.a, 0, T.z, m0, kb);
+              mk_load<true, 128>(st + 16384, &M.op1, &full[s], K.b, boff, T.z, T.nt * 128, kb);
+              mk_load<true, 128>(st + 32768, &M.op2, &full[s], K.b, boff, T.z, T.nt * 128, kb);
+            }
+            break;
+        }
+      }
+    }
+    for (int j = it - kStages < 0 ? 0 : it - kStages; j < it; ++j)
+      (void)tc::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, lim);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint64_t dK = tc2::sdesc(tc::smem_u32(ring), false);
+    const uint64_t dN = tc2::sdesc(tc::smem_u32(ring), true);
+    constexpr uint32_t kA = 16384 >> 4, kB2 = 32768 >> 4;
+    int it = 0, i = 0;
+    bool ok = true;
+    if (J.stall && blockIdx.x == 0 && !tc::mbar_wait(&never, 0u, lim)) {
+      atomicExch(J.status, tc2::kErrMma);
+      s_err = 1;
+      ok = false;
+    }
+    for (int t = blockIdx.x; t < J.total && ok; t += gridDim.x, ++i) {
+      const MkTile T = mk_decode(J, t);
+      const tc2::Class& K = J.ph[T.ph].cls[T.cls];
+      const int b = i & 1;
+      if (!tc::mbar_wait(&acc_empty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, lim)) {
+        atomicExch(J.status, tc2::kErrMma);
+        s_err = 1;
+        break;
+      }
+      tc::tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(b * kAcc);
+      for (int kb = 0; kb < K.kblocks; ++kb, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        if (!tc::mbar_wait_hint(&full[s], ph, lim)) {
+          atomicExch(J.status, tc2::kErrMma);
+          s_err = 1;
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t so = ((uint32_t)s * kSlot) >> 4;
+#pragma unroll
+        for (int k = 0; k < tc::BK / 16; ++k) {
+          const uint32_t accum = (kb | k) != 0;
+          switch (T.ph) {
+            case 0:
+              tc::mma_bf16(acc, dK + (so + k * 2), dK + (so + kA + k * 2), tc2::idesc(128, 256, false, false), accum);
+              break;
+            case 1:
+              tc::mma_bf16(acc, dK + (so + k * 2), dK + (so + kA + k * 2), tc2::idesc(128, 128, false, false), accum);
+              break;
+            case 2:
+              tc::mma_bf16(acc, dK + (so + k * 2), dN + (so + kA + k * 128), tc2::idesc(128, 128, false, true), accum);
+              break;
+            default: {
+              constexpr uint32_t id = tc2::idesc(128, 128, true, true);
+              if (K.mode == tc2::kModeA2B1) {
+                const uint64_t bd = dN + (so + kB2 + k * 128);
+                tc::mma_bf16(acc, dN + (so + k * 128), bd, id, accum);
+                tc::mma_bf16(acc + 128, dN + (so + kA + k * 128), bd, id, accum);
+              } else {
+                const uint64_t ad = dN + (so + k * 128);
+                tc::mma_bf16(acc, ad, dN + (so + kA + k * 128), id, accum);
+                tc::mma_bf16(acc + 128, ad, dN + (so + kB2 + k * 128), id, accum);
+              }
+              break;
+            }
+          }
+        }
+        tc::mma_commit(&empty[s]);
+      }
+      tc::mma_commit(&acc_full[b]);
+      ++mma_tiles;
+    }
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    // Every epilogue warp runs the same number of iterations and named barriers,
+    // also after a failure (then it only skips the work), so no warp can wait
+    // at the barrier for one that left.
+    const int ew = warp - 2;
+    const int quad = warp & 3;
+    uint32_t uses[tc2::kEpiBars] = {0u, 0u, 0u, 0u};
+    int seq4 = 0;    // G4 tiles this warp has finished
+    int pre4 = 0;    // the previous G4 tile issued this one's first state loads
+    int i = 0;
+    for (int t = blockIdx.x; t < J.total; t += gridDim.x, ++i) {
+      const MkTile T = mk_decode(J, t);
+      const int b = i & 1;
+      bool ok = !s_err;
+      if (ok && !tc::mbar_wait(&acc_full[b], (uint32_t)(i >> 1) & 1u, lim)) {
+        if (lane == 0) atomicExch(J.status, tc2::kErrEpilogue);
+        s_err = 1;
+        ok = false;
+      }
+      tc::tc_fence_after();
+      if (ok) {
+        int dep_ok = 1;
+        if (lane == 0) dep_ok = mk_dep_wait(J, T, lim) ? 1 : 0;  // satisfied already: the producer waited
+        dep_ok = __shfl_sync(0xffffffffu, dep_ok, 0);
+        if (!dep_ok) {
+          if (lane == 0) atomicExch(J.status, kErrDep);
+          s_err = 1;
+          ok = false;
+        }
+      }
+      const int chunk_t0 = T.ci * J.C;
+      const int clen = T.ci == J.NC - 1 ? prm.d.T - chunk_t0 : J.C;
+      if (ok) {
+        auto fill = [&](auto& c, int nparts, int part, uint8_t* ws) {
+          c.cls = T.cls;
+          c.z = T.z;
+          c.m0 = T.mt * tc::BM;
+          c.row = quad * 32 + lane;
+          c.quad = quad;
+          c.nparts = nparts;
+          c.part = part;
+          c.taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * kAcc);
+          c.wsmem = ws;
+          c.wbar = epi_bar + tc2::kEpiBars * ew;
+          c.uses = uses;
+          c.slot = i & 1;
+          c.iter = i;
+          c.seq = i;
+          c.pre = 0;
+          c.ci = T.ci;
+          c.t0 = chunk_t0;
+          c.clen = clen;
+          c.wshadow = T.ci + 1 < J.NC;
+          c.nxt_valid = 0;
+          c.nxt_cls = c.nxt_z = c.nxt_m0 = c.nxt_n0 = c.nxt_ci = 0;
+        };
+        switch (T.ph) {
+          case 0: {
+            tc2::EpiCtx<256> c;
+            fill(c, 2, ew >> 2, epi_smem + (size_t)ew * kEpiSmem);
+            c.n0 = T.nt * 256;
+            EpiG1::run(prm, c);
+            break;
+          }
+          case 1: {
+            tc2::EpiCtx<128> c;
+            fill(c, 2, ew >> 2, epi_smem + (size_t)ew * kEpiSmem);
+            c.n0 = T.nt * 128;
+            if (clen < J.C) EpiG2Pad::run(prm, c);
+            else EpiG2::run(prm, c);
+            break;
+          }
+          case 2: {
+            tc2::EpiCtx<128> c;
+            fill(c, 2, ew >> 2, epi_smem + (size_t)ew * kEpiSmem);
+            c.n0 = T.nt * 128;
+            EpiG3::run(prm, c);
+            break;
+          }
+          default:
+            if (ew < 4) {
+              tc2::EpiCtx<128> c;
+              fill(c, 1, 0, epi_smem + (size_t)ew * kEpiSmemG4);
+              c.n0 = T.nt * 128;
+              c.seq = seq4;
+              c.pre = pre4;
+              // the CTA's next tile: its first state groups load during this
+              // tile's last groups if it is a G4 tile whose inputs are complete
+              int nv = 0, ncls = 0, nz = 0, nmt = 0, nnt = 0, nci = 0;
+              const int tn = t + (int)gridDim.x;
+              if (lane == 0 && tn < J.total) {
+                const MkTile N = mk_decode(J, tn);
+                nv = N.ph == 3 && mk_dep_ready(J, N);
+                if (nv) fence_proxy_async_global();
+                ncls = N.cls; nz = N.z; nmt = N.mt; nnt = N.nt; nci = N.ci;
+              }
+              nv = __shfl_sync(0xffffffffu, nv, 0);
+              if (nv) {
+                c.nxt_valid = 1;
+                c.nxt_cls = __shfl_sync(0xffffffffu, ncls, 0);
+                c.nxt_z = __shfl_sync(0xffffffffu, nz, 0);
+                c.nxt_m0 = __shfl_sync(0xffffffffu, nmt, 0) * tc::BM;
+                c.nxt_n0 = __shfl_sync(0xffffffffu, nnt, 0) * 128;
+                c.nxt_ci = __shfl_sync(0xffffffffu, nci, 0);
+              }
+              EpiG4::run(prm, c);
+              seq4 += 1;
+              pre4 = nv;
+            }
+            break;
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        tc2::mbar_arrive(&acc_empty[b]);
+        tc::bulk_wait_all();             // this warp's stores of the tile have completed
+        fence_proxy_async_global();
+      }
+      __syncwarp();
+      epi_barrier();                     // ... and those of every epilogue warp
+      if (ew == 0 && lane == 0 && ok && !s_err) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(J.cnt + (size_t)T.ph * J.BH + T.z)
+                     : "memory");
+      }
+    }
+    // a G4 tile that prefetched for a next one that never ran (after a failure):
+    // its two state loads must land before the CTA exits
+    if (pre4 && lane == 0) {
+      (void)tc::mbar_wait(&epi_bar[tc2::kEpiBars * ew + 0], uses[0] & 1u, lim);
+      (void)tc::mbar_wait(&epi_bar[tc2::kEpiBars * ew + 1], uses[1] & 1u, lim);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0 && mma_tiles > 0) {
+      const int last = mma_tiles - 1;
+      (void)tc::mbar_wait(&acc_full[last & 1], (uint32_t)(last >> 1) & 1u, lim);
+    }
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 2 * kAcc);
+  }
+}
 
 // ---------------------------------------------------------------- prep kernel
 // bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
@@ -828,8 +1288,42 @@ cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
   return launch_pdl(kern, dim3(grid), dim3((2 + EW) * 32), smem, st, job, p);
 }
 
+// Heads per group in the persistent forward's tile order: the largest divisor
+// of B*H whose group (all four phases of one chunk) has no more tiles than the
+// GPU has SMs, at least one head.
+int mega_group_heads(int BH, int tiles_per_head, int sms) {
+  int hg = 1;
+  for (int h = 1; h <= BH; ++h)
+    if (BH % h == 0 && h * tiles_per_head <= sms) hg = h;
+  return hg;
+}
+
+cudaError_t launch_mega(const MegaJob& J, const FwdP& p, cudaStream_t st) {
+  constexpr size_t smem = mk::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(fwd_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fwd_persistent, (2 + mk::kEW) * 32, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  const int grid = J.total < num_sms() ? J.total : num_sms();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3((2 + mk::kEW) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: tiles wait on one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  E2TTT_TRACE("tc_fwd_persistent", st);
+  return cudaLaunchKernelEx(&cfg, fwd_persistent, J, p);
+}
+
 struct Scratch {
   bf16 *Wsh13, *W2sh, *A, *Sk, *E, *Ea, *Eb, *dH, *Ka, *Kb;
+  int* cnt;  // persistent forward: completed tiles per (phase, head)
 };
 
 size_t carve(const Dims& d, char* base, Scratch* s) {
@@ -856,6 +1350,7 @@ size_t carve(const Dims& d, char* base, Scratch* s) {
   }
   t.Ea = take(BH * d.C * d.d_v * e);
   t.Eb = take(BH * d.C * d.d_v * e);
+  t.cnt = (int*)take(4 * BH * sizeof(int));
   if (s) *s = t;
   return off;
 }
@@ -1010,22 +1505,82 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   }
   if (!ok) return cudaErrorInvalidValue;
 
+  // SwiGLU with momentum and no saved states may run every chunk in one
+  // persistent, cooperative launch; it is selected with E2TTT_PERSISTENT=1 in
+  // the environment (the per-phase launches are faster on the shapes measured).
+  const char* env_p = getenv("E2TTT_PERSISTENT");
+  const bool persistent = d.kind == 1 && !d.nomom && saved == nullptr && env_p && env_p[0] == '1';
+  if (persistent) {
+    MegaJob J{};
+    J.ph[0] = g1;
+    J.ph[1] = g2;
+    J.ph[2] = g3;
+    J.ph[3] = g4;
+    for (int ph = 0; ph < 4; ++ph) {
+      J.tph[ph] = 0;
+      for (int c = 0; c < J.ph[ph].n_cls; ++c)
+        J.tph[ph] += J.ph[ph].cls[c].tiles_m * J.ph[ph].cls[c].tiles_n;
+    }
+    const int tph_all = J.tph[0] + J.tph[1] + J.tph[2] + J.tph[3];
+    J.BH = BH;
+    J.NC = NC;
+    J.C = C;
+    const char* env_hg = getenv("E2TTT_PERSISTENT_HG");
+    J.hg = env_hg ? atoi(env_hg) : mega_group_heads(BH, tph_all, num_sms());
+    if (J.hg < 1 || BH % J.hg != 0) J.hg = 1;
+    J.per_group = J.hg * tph_all;
+    J.per_chunk = BH * tph_all;
+    J.total = NC * J.per_chunk;
+    J.cnt = s.cnt;
+    J.status = status;
+    J.stall = g_stall_next.exchange(0) != 0;
+    J.wait_ns = J.stall ? kStallWaitNs : 0;
+    // state maps: variant 0 = W0, M0 (first chunk), 1 = W_end, M_end in place
+    p.hasM[0] = M0 != nullptr;
+    p.hasM[1] = 1;
+    for (int c = 0; c < 2; ++c) {
+      const long long off = c == 0 ? 0 : (long long)r13 * dk;
+      const uint64_t rows = c == 0 ? r13 : dv;
+      const uint64_t cols = c == 0 ? dk : dh;
+      ok &= make_state_map(&p.srcW[0][c], W0 + off, rows, cols, BH, d.S);
+      if (M0) ok &= make_state_map(&p.srcM[0][c], M0 + off, rows, cols, BH, d.S);
+      ok &= make_state_map(&p.srcW[1][c], W_end + off, rows, cols, BH, d.S);
+      ok &= make_state_map(&p.srcM[1][c], M_end + off, rows, cols, BH, d.S);
+      ok &= make_state_map(&p.dstW[c], W_end + off, rows, cols, BH, d.S);
+      ok &= make_state_map(&p.dstM[c], M_end + off, rows, cols, BH, d.S);
+    }
+    ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * r13, dk);
+    ok &= make_map_box32(&p.shadow[1], s.W2sh, (uint64_t)BH * dv, dh);
+    if (!ok) return cudaErrorInvalidValue;
+    e = cudaMemsetAsync(s.cnt, 0, 4 * (size_t)BH * sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    return launch_mega(J, p, st);
+  }
+
   for (int ci = 0; ci < NC; ++ci) {
-    p.ci = ci;
-    p.t0 = ci * C;
-    p.clen = T - ci * C < C ? T - ci * C : C;
-    p.write_shadow = ci + 1 < NC;
-    chunk_states(d, ci, W0, M0, W_end, M_end, saved, &p.src, &p.dst);
+    const int clen = T - ci * C < C ? T - ci * C : C;
+    for (tc2::Job* j : {&g1, &g2, &g3, &g4, &g4w}) {
+      j->ci = ci;
+      j->t0 = ci * C;
+      j->clen = clen;
+      j->wshadow = ci + 1 < NC;
+    }
+    StateIn src;
+    StateOut dst;
+    chunk_states(d, ci, W0, M0, W_end, M_end, saved, &src, &dst);
     {
       const int ncls = d.kind != 0 ? 2 : 1;
+      p.hasM[0] = p.hasM[1] = src.M != nullptr;
       for (int c = 0; c < ncls; ++c) {
         const long long off = c == 0 ? 0 : (long long)r13 * dk;
         const uint64_t rows = c == 0 ? r13 : dv;
         const uint64_t cols = c == 0 ? dk : dh;
-        ok &= make_state_map(&p.srcW[c], p.src.W + off, rows, cols, BH, p.src.stride);
-        if (p.src.M) ok &= make_state_map(&p.srcM[c], p.src.M + off, rows, cols, BH, p.src.stride);
-        ok &= make_state_map(&p.dstW[c], p.dst.W + off, rows, cols, BH, p.dst.stride);
-        if (p.dst.M) ok &= make_state_map(&p.dstM[c], p.dst.M + off, rows, cols, BH, p.dst.stride);
+        ok &= make_state_map(&p.srcW[0][c], src.W + off, rows, cols, BH, src.stride);
+        if (src.M) ok &= make_state_map(&p.srcM[0][c], src.M + off, rows, cols, BH, src.stride);
+        p.srcW[1][c] = p.srcW[0][c];
+        p.srcM[1][c] = p.srcM[0][c];
+        ok &= make_state_map(&p.dstW[c], dst.W + off, rows, cols, BH, dst.stride);
+        if (dst.M) ok &= make_state_map(&p.dstM[c], dst.M + off, rows, cols, BH, dst.stride);
       }
       if (ci == 0) {
         ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * r13, dk);
@@ -1044,7 +1599,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
       else
         e = launch<128, 1, false, false, 4, EpiG1Gelu, kEpiWarps, EpiG1Gelu::kSmem>(g1, p, st);
       if (e == cudaSuccess) {
-        e = p.clen < C ? launch<128, 1, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
+        e = clen < C ? launch<128, 1, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
                        : launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
       }
       if (e == cudaSuccess) {
@@ -1057,7 +1612,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
                     : launch<128, 2, true, true, 3, EpiG4, 4, EpiG4::kSmem>(g4, p, st);
       }
     } else {
-      e = p.clen < C ? launch<128, 1, false, false, 4, EpiG1LinPad, kEpiWarps, EpiG1LinPad::kSmem>(g1, p, st)
+      e = clen < C ? launch<128, 1, false, false, 4, EpiG1LinPad, kEpiWarps, EpiG1LinPad::kSmem>(g1, p, st)
                      : launch<128, 1, false, false, 4, EpiG1Lin, kEpiWarps, EpiG1Lin::kSmem>(g1, p, st);
       if (e == cudaSuccess) {
         e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)

@@ -108,6 +108,9 @@ struct Job {
   // after wait_ns; the launch then reports a timeout in *status and exits.
   int stall;
   unsigned long long wait_ns;  // 0: the default limit (tc::kWaitNs)
+  // chunk of this launch, handed to the epilogues: index, first token, tokens in
+  // the chunk, and whether the bf16 operand copy of the end state is written
+  int ci, t0, clen, wshadow;
 };
 
 template <int BN>
@@ -122,9 +125,12 @@ struct EpiCtx {
   uint32_t* uses;     // completed-phase counters of wbar[], kept across tiles
   int slot;           // this tile's epilogue input buffer / wbar index (tile ordinal & 1)
   int iter;           // ordinal of this tile among the CTA's tiles
+  int seq;            // ordinal among the CTA's tiles of this epilogue type
+  int pre;            // 1 if the CTA's previous tile already issued this tile's first input loads
+  int ci, t0, clen, wshadow;  // the tile's chunk (see Job)
   // the CTA's next tile (nxt_valid = 0 if this is its last), for epilogues that
   // start loading the next tile's inputs while finishing this one
-  int nxt_valid, nxt_cls, nxt_z, nxt_m0, nxt_n0;
+  int nxt_valid, nxt_cls, nxt_z, nxt_m0, nxt_n0, nxt_ci;
   __device__ __forceinline__ void ld(int acc, int col, float (&v)[32]) const {
     tmem_ld32(taddr + (uint32_t)(acc * BN + col), v);
   }
@@ -374,8 +380,15 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
       ctx.uses = uses;
       ctx.slot = i & 1;
       ctx.iter = i;
+      ctx.seq = i;
+      ctx.pre = i > 0;
+      ctx.ci = job.ci;
+      ctx.t0 = job.t0;
+      ctx.clen = job.clen;
+      ctx.wshadow = job.wshadow;
       ctx.nxt_valid = t + (int)gridDim.x < job.total_tiles;
       ctx.nxt_cls = ctx.nxt_z = ctx.nxt_m0 = ctx.nxt_n0 = 0;
+      ctx.nxt_ci = job.ci;
       if (ctx.nxt_valid) {
         int c2, z2, mt2, nt2;
         decode_tile(job, t + gridDim.x, c2, z2, mt2, nt2);

@@ -142,3 +142,17 @@ def test_recorded_traffic_needs_matching_sources(bench, tmp_path, monkeypatch):
         f.write("\n// changed\n")
     assert bench.recorded_traffic("tc_g4_aggregate_state", "layer_1p3b_2k") is None
     assert bench.recorded_traffic("tc_g4_aggregate_state", "other_workload") is None
+
+
+def test_persistent_forward_work_is_the_sum_of_its_phases(bench):
+    """One launch of the persistent forward runs the four GEMM phases of every
+    chunk: its FLOPs are the forward's, its algorithmic bytes the call's
+    compulsory traffic less the gates."""
+    w = gen.BY_NAME["layer_1p3b_2k"]
+    work = bench.kernel_work(w, has_m0=False)
+    f, alg, impl = work["tc_fwd_persistent"]
+    assert f == bench.fwd_flops(w)
+    assert alg == bench.algorithmic_bytes(w) - 12 * w.B * w.H * w.T
+    NC = w.T // w.C
+    assert impl == NC * sum(work[n][2] for n in ("tc_g1_h_act", "tc_g2_y_out_e", "tc_g3_da_dh",
+                                                 "tc_g4_aggregate_state"))

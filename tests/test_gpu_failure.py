@@ -26,8 +26,14 @@ def E():
     return E
 
 
-def test_bounded_wait_runs_out_and_the_context_recovers(E):
+@pytest.mark.parametrize("persistent", [False, True])
+def test_bounded_wait_runs_out_and_the_context_recovers(E, persistent, monkeypatch):
+    """Both forward drivers: the per-phase launches, and the persistent kernel
+    (E2TTT_PERSISTENT=1, one launch for all chunks), where the stalled CTA's
+    tiles never complete and every CTA waiting on them gives up too."""
     import torch
+    monkeypatch.setenv("E2TTT_PERSISTENT", "1" if persistent else "0")
+    saved = False
     w = gen.Workload("stall", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform", 0.999,
                      seed=61, lr_lo=0.002, lr_hi=0.02)
     x = gen.generate(w, m0_scale=0.5)
@@ -36,11 +42,14 @@ def test_bounded_wait_runs_out_and_the_context_recovers(E):
     assert E.e2ttt_fwd_uses_tensor_cores(shape) == 1
     ws = E.workspace(shape)
 
+    nc = E.e2ttt_num_chunks(shape)
+    sv = torch.empty((nc, w.B, w.H, 2, w.state_elems), device="cuda") if saved else None
+
     def call():
         out = torch.empty_like(d["v"])
         We, Me = torch.empty_like(d["W0"]), torch.empty_like(d["W0"])
         E.e2ttt_chunk_scan_fwd(shape, d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"],
-                               d["W0"], d["M0"], out, We, Me, None, ws)
+                               d["W0"], d["M0"], out, We, Me, sv, ws)
         return out, We, Me
 
     before = call()
