@@ -332,7 +332,7 @@ __device__ __forceinline__ void store_vec(float* __restrict__ p, const float (&v
 }
 
 template <int PER>
-__global__ void __launch_bounds__(kK1Threads)
+__global__ void __launch_bounds__(kK1Threads, PER >= 8 ? 8 : 16)  // 16 blocks (2048 threads) per SM
 chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
                         const float* __restrict__ decay, float* __restrict__ a_out,
                         float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,

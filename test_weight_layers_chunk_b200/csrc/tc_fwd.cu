@@ -21,6 +21,7 @@
 #include <stdlib.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "paths.h"
 #include "state.cuh"
@@ -169,10 +170,11 @@ struct EpiG1 {
       }
       staging_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.mA, S, j0 + g, yA);
+        const uint64_t keep = tc::l2_evict_last();  // read by the next phases of the chunk
+        tc::tma_store_2d_hint(&p.mA, S, j0 + g, yA, keep);
         if (c.cls == 1) {
-          tc::tma_store_2d(&p.mSk, S + 2048, j0 + g, ySk);
-          tc::tma_store_2d(&p.mSk, S + 4096, d.d_h + j0 + g, ySk);
+          tc::tma_store_2d_hint(&p.mSk, S + 2048, j0 + g, ySk, keep);
+          tc::tma_store_2d_hint(&p.mSk, S + 4096, d.d_h + j0 + g, ySk, keep);
         }
         tc::bulk_commit();
       }
@@ -208,8 +210,9 @@ struct EpiG1Gelu {
       if (c.cls == 1) stage32(S + 2048, lane, gp);
       staging_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.mA, S, j, yA);
-        if (c.cls == 1) tc::tma_store_2d(&p.mSk, S + 2048, j, ySk);
+        const uint64_t keep = tc::l2_evict_last();  // read by the next phases of the chunk
+        tc::tma_store_2d_hint(&p.mA, S, j, yA, keep);
+        if (c.cls == 1) tc::tma_store_2d_hint(&p.mSk, S + 2048, j, ySk, keep);
         tc::bulk_commit();
       }
       __syncwarp();
@@ -276,24 +279,29 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
   const int lane = c.row & 31;
   const int per = BN / c.nparts;
   const int col0 = c.n0 + c.part * per;
-  static_assert(BN <= 128, "two V buffers: at most two 32-column groups per warp");
   const int ngroups = per / 32;
-  uint8_t* V = c.wsmem;            // [2][2 KB]
+  uint8_t* V = c.wsmem;            // [2][2 KB]: V of a pair of column groups
   uint8_t* S = c.wsmem + 4096;     // E | Ea | Eb staging
   const int ttok = c.t0 + r0;      // first token (within the head) of this warp's rows
   const int yrow = c.z * d.C + r0;
+  const uint64_t keep = tc::l2_evict_last();    // E, aE, bE: read by the next phases
+  const uint64_t stream = tc::l2_evict_first(); // out: never read again
   // Padding rows: no output, and E = a E = b E = 0, so they add nothing to any
   // later sum over tokens.
   const bool real = !PAD || lane < c.clen - r0;
   if (PAD && !key_rows && c.clen - r0 <= 0) return;  // no query row of this warp is real
-  if (key_rows) {
+  // V of key rows arrives by TMA, a pair of 32-column groups at a time
+  auto load_pair = [&](int g0) {
     if (lane == 0) {
-      tc::mbar_expect_tx(&c.wbar[0], 2048u * ngroups);
-      for (int gi = 0; gi < ngroups; ++gi)
-        tc::tma_load_3d(V + gi * 2048, &p.mV, &c.wbar[0], col0 + gi * 32, ttok, c.z);
+      const int n = ngroups - g0 < 2 ? ngroups - g0 : 2;
+      tc::fence_async_smem();  // the previous pair's reads of V precede the refill
+      tc::mbar_expect_tx(&c.wbar[0], 2048u * n);
+      for (int j = 0; j < n; ++j)
+        tc::tma_load_3d(V + j * 2048, &p.mV, &c.wbar[0], col0 + (g0 + j) * 32, ttok, c.z);
     }
     __syncwarp();
-  }
+  };
+  if (key_rows) load_pair(0);
   float at = 0.f, bt = 0.f;
   if (key_rows && real) {
     const size_t tok = (size_t)c.z * d.T + ttok + lane;
@@ -309,13 +317,14 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
       stage32(S, lane, y);
       staging_ready();
       if (lane == 0) {
-        tc::tma_store_3d(&p.mOut, S, col, ttok, c.z);
+        tc::tma_store_3d_hint(&p.mOut, S, col, ttok, c.z, stream);
         tc::bulk_commit();
       }
       __syncwarp();
       continue;
     }
-    if (gi == 0) {
+    if ((gi & 1) == 0) {
+      if (gi > 0) load_pair(gi);
       const bool ok = tc::mbar_wait(&c.wbar[0], c.uses[0] & 1u);
       c.uses[0] += 1;
       if (!ok) {
@@ -324,7 +333,7 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
       }
     }
     float vv[32];
-    unstage32(V + gi * 2048, lane, vv);
+    unstage32(V + (gi & 1) * 2048, lane, vv);
 #pragma unroll
     for (int i = 0; i < 32; ++i) y[i] = (PAD && !real) ? 0.f : d.loss == 0 ? y[i] - vv[i] : -vv[i];
     staging_free(lane);
@@ -339,9 +348,9 @@ __device__ __forceinline__ void out_or_residual(const FwdP& p, const EpiCtx<BN>&
     stage32(S + 4096, lane, vv);
     staging_ready();
     if (lane == 0) {
-      if (write_e) tc::tma_store_2d(&p.mE, S, col, yrow);
-      if (!p.nomom) tc::tma_store_2d(&p.mEa, S + 2048, col, yrow);
-      tc::tma_store_2d(&p.mEb, S + 4096, col, yrow);
+      if (write_e) tc::tma_store_2d_hint(&p.mE, S, col, yrow, keep);
+      if (!p.nomom) tc::tma_store_2d_hint(&p.mEa, S + 2048, col, yrow, keep);
+      tc::tma_store_2d_hint(&p.mEb, S + 4096, col, yrow, keep);
       tc::bulk_commit();
     }
     __syncwarp();
@@ -380,7 +389,7 @@ using EpiG1LinPad = EpiG1LinT<true>;
 // into registers, the same buffer stages that group's dH1 | dH3 for the TMA
 // stores (each lane reads and then writes only its own row).
 struct EpiG3 {
-  static constexpr int kSmem = 8192;  // [2 groups][silu(H1) | H3 silu'(H1), then dH3 | dH1]
+  static constexpr int kSmem = 8192;  // [2 groups][silu(H1) | H3 silu'(H1), then dH1 | dH3]
   template <int BN>
   static __device__ __forceinline__ void run(const FwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
@@ -388,23 +397,28 @@ struct EpiG3 {
     const int r0 = c.m0 + c.quad * 32;
     const int per = BN / c.nparts;
     const int col0 = c.n0 + c.part * per;
-    static_assert(BN <= 128, "silu-factor buffers for at most two column groups per warp");
     const int ngroups = per / 32;
     const int y = c.z * d.C + r0;
-    uint8_t* F = c.wsmem;  // [group][s1 | s2] 2 KB each
-    if (lane == 0) {
-      tc::bulk_wait_read<0>();  // the previous tile's stores have read the buffers
-      tc::mbar_expect_tx(&c.wbar[0], 4096u * ngroups);
-      for (int gi = 0; gi < ngroups; ++gi) {
-        tc::tma_load_2d(F + gi * 4096, &p.mSk, &c.wbar[0], col0 + gi * 32, y);
-        tc::tma_load_2d(F + gi * 4096 + 2048, &p.mSk, &c.wbar[0], d.d_h + col0 + gi * 32, y);
+    const uint64_t keep = tc::l2_evict_last();  // dH: read by the aggregation next
+    uint8_t* F = c.wsmem;  // [group of the pair][s1 | s2] 2 KB each
+    auto load_pair = [&](int g0) {
+      if (lane == 0) {
+        tc::bulk_wait_read<0>();  // earlier stores have read the buffers
+        const int n = ngroups - g0 < 2 ? ngroups - g0 : 2;
+        tc::mbar_expect_tx(&c.wbar[0], 4096u * n);
+        for (int j = 0; j < n; ++j) {
+          tc::tma_load_2d(F + j * 4096, &p.mSk, &c.wbar[0], col0 + (g0 + j) * 32, y);
+          tc::tma_load_2d(F + j * 4096 + 2048, &p.mSk, &c.wbar[0], d.d_h + col0 + (g0 + j) * 32, y);
+        }
       }
-    }
-    __syncwarp();
+      __syncwarp();
+    };
+    load_pair(0);
     for (int gi = 0; gi < ngroups; ++gi) {
       float da[32], s1[32], s2[32];
       ld1(c, 0, c.part * per + gi * 32, da);
-      if (gi == 0) {
+      if ((gi & 1) == 0) {
+        if (gi > 0) load_pair(gi);
         const bool ok = tc::mbar_wait(&c.wbar[0], c.uses[0] & 1u);
         c.uses[0] += 1;
         if (!ok) {
@@ -412,7 +426,7 @@ struct EpiG3 {
           return;
         }
       }
-      uint8_t* G = F + gi * 4096;
+      uint8_t* G = F + (gi & 1) * 4096;
       unstage32(G, lane, s1);
       unstage32(G + 2048, lane, s2);
 #pragma unroll
@@ -424,8 +438,8 @@ struct EpiG3 {
       stage32(G + 2048, lane, s1);
       staging_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.mdH, G, col0 + gi * 32, y);
-        tc::tma_store_2d(&p.mdH, G + 2048, d.d_h + col0 + gi * 32, y);
+        tc::tma_store_2d_hint(&p.mdH, G, col0 + gi * 32, y, keep);
+        tc::tma_store_2d_hint(&p.mdH, G + 2048, d.d_h + col0 + gi * 32, y, keep);
         tc::bulk_commit();
       }
       __syncwarp();
@@ -528,7 +542,8 @@ struct EpiG4 {
       if (lane == 0) {
         tc::tma_store_3d(&p.dstW[c.cls], slot, c.n0 + g * 32, r0, c.z);
         tc::tma_store_3d(&p.dstM[c.cls], slot + 4096, c.n0 + g * 32, r0, c.z);
-        if (c.wshadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 8192, c.n0 + g * 32, sh_row);
+        if (c.wshadow)  // the next chunk's first phases read the bf16 copy at once
+          tc::tma_store_2d_hint(&p.shadow[c.cls], slot + 8192, c.n0 + g * 32, sh_row, tc::l2_evict_last());
         tc::bulk_commit();
         tc::bulk_wait_read<0>();  // group q's stores have read the slot of group q + 2
         const int gn = g + 2;
@@ -613,7 +628,8 @@ struct EpiG4W {
       __syncwarp();
       if (lane == 0) {
         tc::tma_store_3d(&p.dstW[c.cls], slot, c.n0 + g * 32, r0, c.z);
-        if (c.wshadow) tc::tma_store_2d(&p.shadow[c.cls], slot + 4096, c.n0 + g * 32, sh_row);
+        if (c.wshadow)
+          tc::tma_store_2d_hint(&p.shadow[c.cls], slot + 4096, c.n0 + g * 32, sh_row, tc::l2_evict_last());
         tc::bulk_commit();
         tc::bulk_wait_read<1>();  // the slot of group q - 1 is free for group q + 2
         const int gn = g + 2;
@@ -1288,6 +1304,31 @@ cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
   return launch_pdl(kern, dim3(grid), dim3((2 + EW) * 32), smem, st, job, p);
 }
 
+// A side stream and two events per device and host thread (created once,
+// never freed; no device memory is involved), for the prep kernels that can run
+// beside others. Per thread, because a call records and waits on its own
+// events between its fork and its join.
+struct SideStream {
+  cudaStream_t s;
+  cudaEvent_t fork, join;
+};
+SideStream* side_stream() {
+  thread_local SideStream tab[64];
+  thread_local bool made[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!made[dev]) {
+    SideStream x{};
+    if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    tab[dev] = x;
+    made[dev] = true;
+  }
+  return &tab[dev];
+}
+
 // Heads per group in the persistent forward's tile order: the largest divisor
 // of B*H whose group (all four phases of one chunk) has no more tiles than the
 // GPU has SMs, at least one head.
@@ -1396,9 +1437,20 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
 
   cudaError_t e = save_initial_state(d, W0, M0, saved, st);
   if (e != cudaSuccess) return e;
+  // The bf16 copy of W0 does not depend on the scaled keys: it runs on a side
+  // stream, forked from and joined back to the caller's stream, so the two
+  // HBM-bound prep kernels overlap (also under stream capture).
+  SideStream* side = side_stream();
+  const bool fork = side != nullptr && d.kind != 0;
+  if (fork) {
+    e = cudaEventRecord(side->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+    if (e != cudaSuccess) return e;
+  }
   {
-    E2TTT_TRACE("tc_shadow_init", st);
-    shadow_init_kernel<<<8 * num_sms(), 256, 0, st>>>(p, W0);
+    cudaStream_t ss = fork ? side->s : st;
+    E2TTT_TRACE("tc_shadow_init", ss);
+    shadow_init_kernel<<<8 * num_sms(), 256, 0, ss>>>(p, W0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1409,7 +1461,23 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (fork) {
+    e = cudaEventRecord(side->join, side->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
+    if (e != cudaSuccess) return e;
+  }
 
+  // G2 and G3 run 128 x 256 tiles where their N (d_v, resp. d_h) allows: half
+  // the A-operand reloads and half the ring handshakes per FLOP of 128 x 128.
+  const char* env_p = getenv("E2TTT_PERSISTENT");
+  // the persistent kernel (below) runs 128 x 128 tiles in G2 and G3
+  const bool persistent = d.kind == 1 && !d.nomom && saved == nullptr && env_p && env_p[0] == '1';
+  const bool wide_ok = !persistent;
+  // (only while the wide tiles still fill every SM at least once: with few
+  // heads the narrower tiles keep more SMs busy)
+  const int sms = num_sms();
+  const bool wide2 = wide_ok && d.kind == 1 && dv % 256 == 0 && BH * (2 * C / 128) * (dv / 256) >= sms;
+  const bool wide3 = wide_ok && d.kind == 1 && dh % 256 == 0 && BH * (C / 128) * (dh / 256) >= sms;
   // Operand maps (chunk-independent; the chunk offset goes into the coordinates).
   tc2::Job g1{}, g2{}, g3{}, g4{};
   bool ok = true;
@@ -1437,14 +1505,14 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     g1.maps[1].op2 = g1.maps[0].op2;
     // G2: A = [A_q; A_k], B = W2 (N = d_v)
     ok &= make_map(&g2.maps[0].op0, s.A, (uint64_t)BH * 2 * C, dh, 128);
-    ok &= make_map(&g2.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 128);
+    ok &= make_map(&g2.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, wide2 ? 256 : 128);
     g2.n_cls = 1;
-    g2.cls[0] = tc2::Class{2 * C / 128, dv / 128, dh / 64, {2 * C, 0, 0}, {dv, 0, 0}, 0};
+    g2.cls[0] = tc2::Class{2 * C / 128, dv / (wide2 ? 256 : 128), dh / 64, {2 * C, 0, 0}, {dv, 0, 0}, 0};
     // G3: A = E, B = W2 read MN-major (N = d_h, K = d_v)
     ok &= make_map(&g3.maps[0].op0, s.E, (uint64_t)BH * C, dv, 128);
     ok &= make_map(&g3.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 64);
     g3.n_cls = 1;
-    g3.cls[0] = tc2::Class{C / 128, dh / 128, dv / 64, {C, 0, 0}, {dv, 0, 0}, 0};
+    g3.cls[0] = tc2::Class{C / 128, dh / (wide3 ? 256 : 128), dv / 64, {C, 0, 0}, {dv, 0, 0}, 0};
     // G4 class 0: A = dH (M = [W1; W3] rows, or W1 rows for GELU; K = tokens),
     // B0 = diag(a) K, B1 = diag(b) K
     ok &= make_map(&g4.maps[0].op0, s.dH, (uint64_t)BH * C, r13, 64);
@@ -1508,8 +1576,6 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   // SwiGLU with momentum and no saved states may run every chunk in one
   // persistent, cooperative launch; it is selected with E2TTT_PERSISTENT=1 in
   // the environment (the per-phase launches are faster on the shapes measured).
-  const char* env_p = getenv("E2TTT_PERSISTENT");
-  const bool persistent = d.kind == 1 && !d.nomom && saved == nullptr && env_p && env_p[0] == '1';
   if (persistent) {
     MegaJob J{};
     J.ph[0] = g1;
@@ -1599,13 +1665,17 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
       else
         e = launch<128, 1, false, false, 4, EpiG1Gelu, kEpiWarps, EpiG1Gelu::kSmem>(g1, p, st);
       if (e == cudaSuccess) {
-        e = clen < C ? launch<128, 1, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
-                       : launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
+        if (wide2)
+          e = clen < C ? launch<256, 1, false, false, 3, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
+                         : launch<256, 1, false, false, 3, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
+        else
+          e = clen < C ? launch<128, 1, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
+                         : launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
       }
       if (e == cudaSuccess) {
-        e = d.kind == 1
-                ? launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st)
-                : launch<128, 1, false, true, 3, EpiG3Gelu, kEpiWarps, EpiG3Gelu::kSmem>(g3, p, st);
+        e = d.kind != 1 ? launch<128, 1, false, true, 3, EpiG3Gelu, kEpiWarps, EpiG3Gelu::kSmem>(g3, p, st)
+            : wide3     ? launch<256, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st)
+                        : launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st);
       }
       if (e == cudaSuccess) {
         e = d.nomom ? launch<128, 1, true, true, 4, EpiG4W, 4, EpiG4W::kSmem>(g4w, p, st)

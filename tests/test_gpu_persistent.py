@@ -108,3 +108,22 @@ def test_persistent_forward_is_deterministic_and_resumable(E):
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([first[0], second[0]], dim=2), a[0])
     assert torch.equal(second[1], a[1]) and torch.equal(second[2], a[2])
+
+
+def test_wide_tiles_equal_the_persistent_kernels_tiles(E, monkeypatch):
+    """On the 1.3B layer's shapes the per-phase forward runs G2 and G3 with
+    128 x 256 tiles (they still fill every SM); the persistent kernel runs them
+    with 128 x 128 tiles. Each output element is the same sum over the same
+    k-blocks in the same order either way: equal bit for bit."""
+    import torch
+    w = gen.state_preserving(gen.BY_NAME["layer_1p3b_2k"])
+    x = gen.generate(w, m0_scale=0.5)
+    d = device_inputs(w, x)
+    kw = dict(C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss)
+    args = (d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], d["W0"], d["M0"])
+    a = E.chunk_scan_fwd(*args, **kw)      # persistent (E2TTT_PERSISTENT=1 by the fixture)
+    monkeypatch.setenv("E2TTT_PERSISTENT", "0")
+    b = E.chunk_scan_fwd(*args, **kw)      # per-phase, 128 x 256 tiles in G2 and G3
+    torch.cuda.synchronize()
+    for u, v, n in zip(a[:3], b[:3], ("out", "W_end", "M_end")):
+        assert torch.equal(u, v), n
