@@ -21,7 +21,6 @@
 #include <stdlib.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "paths.h"
 #include "state.cuh"
@@ -1304,31 +1303,6 @@ cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
   return launch_pdl(kern, dim3(grid), dim3((2 + EW) * 32), smem, st, job, p);
 }
 
-// A side stream and two events per device and host thread (created once,
-// never freed; no device memory is involved), for the prep kernels that can run
-// beside others. Per thread, because a call records and waits on its own
-// events between its fork and its join.
-struct SideStream {
-  cudaStream_t s;
-  cudaEvent_t fork, join;
-};
-SideStream* side_stream() {
-  thread_local SideStream tab[64];
-  thread_local bool made[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!made[dev]) {
-    SideStream x{};
-    if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-    if (cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess)
-      return nullptr;
-    tab[dev] = x;
-    made[dev] = true;
-  }
-  return &tab[dev];
-}
-
 // Heads per group in the persistent forward's tile order: the largest divisor
 // of B*H whose group (all four phases of one chunk) has no more tiles than the
 // GPU has SMs, at least one head.
@@ -1437,20 +1411,9 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
 
   cudaError_t e = save_initial_state(d, W0, M0, saved, st);
   if (e != cudaSuccess) return e;
-  // The bf16 copy of W0 does not depend on the scaled keys: it runs on a side
-  // stream, forked from and joined back to the caller's stream, so the two
-  // HBM-bound prep kernels overlap (also under stream capture).
-  SideStream* side = side_stream();
-  const bool fork = side != nullptr && d.kind != 0;
-  if (fork) {
-    e = cudaEventRecord(side->fork, st);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
-    if (e != cudaSuccess) return e;
-  }
   {
-    cudaStream_t ss = fork ? side->s : st;
-    E2TTT_TRACE("tc_shadow_init", ss);
-    shadow_init_kernel<<<8 * num_sms(), 256, 0, ss>>>(p, W0);
+    E2TTT_TRACE("tc_shadow_init", st);
+    shadow_init_kernel<<<8 * num_sms(), 256, 0, st>>>(p, W0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1459,11 +1422,6 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     scale_keys_kernel<<<4 * num_sms(), 256, 0, st>>>(k, ca, cb, d.nomom ? nullptr : s.Ka, s.Kb,
                                                      (long long)BH * T, dk);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  if (fork) {
-    e = cudaEventRecord(side->join, side->s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, side->join, 0);
     if (e != cudaSuccess) return e;
   }
 

@@ -148,11 +148,16 @@ struct EpiPrefetch<E, std::void_t<decltype(E::kPrefetch)>> : std::bool_constant<
 
 template <int BN, int NUM_ACC, bool A_MN, bool B_MN>
 struct Cfg {
-  static_assert(NUM_ACC == 1 || BN == BM, "two-accumulator tiles are 128 x 128");
+  static_assert(NUM_ACC == 1 || BN <= BM, "two-accumulator tiles are 128 x 128 or 128 x 64");
   static constexpr uint32_t kTileA = BM * BK * 2;
   static constexpr uint32_t kTileB = BN * BK * 2;
-  // slots: [A][B] for one accumulator; three 16 KB slots for two
-  static constexpr uint32_t kStage = NUM_ACC == 1 ? kTileA + kTileB : 3 * kTileA;
+  // stage layout: [A][B] for one accumulator; for two, [A0][A1][B] (two A
+  // operands share B) or [A][B0][B1] (one A shared by two B operands)
+  static constexpr uint32_t kOffA1B = kTileA;                  // A2B1: A1 at kTileA, B at 2 kTileA
+  static constexpr uint32_t kOffB1 = kTileA + kTileB;         // A1B2: B0 at kTileA, B1 here
+  static constexpr uint32_t kStage =
+      NUM_ACC == 1 ? kTileA + kTileB
+                   : (2 * kTileA + kTileB > kTileA + 2 * kTileB ? 2 * kTileA + kTileB : kTileA + 2 * kTileB);
   static constexpr uint32_t kAccCols = NUM_ACC * BN;  // one accumulator set
   static_assert(2 * kAccCols <= 512, "two accumulator sets must fit in TMEM");
   static constexpr uint32_t kTmemCols = 2 * kAccCols <= 128 ? 128 : 2 * kAccCols <= 256 ? 256 : 512;
@@ -281,11 +286,11 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
           if (NUM_ACC == 1) {
             load_opnd<B_MN, BN>(st + C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
           } else if (K.mode == kModeA2B1) {
-            load_opnd<A_MN, BM>(st + C_::kTileA, &M.op1, &full[s], K.a, z, mt * BM, kb + g);
+            load_opnd<A_MN, BM>(st + C_::kOffA1B, &M.op1, &full[s], K.a, z, mt * BM, kb + g);
             load_opnd<B_MN, BN>(st + 2 * C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
           } else {
             load_opnd<B_MN, BN>(st + C_::kTileA, &M.op1, &full[s], K.b, z, nt * BN, kb + g);
-            load_opnd<B_MN, BN>(st + 2 * C_::kTileA, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
+            load_opnd<B_MN, BN>(st + C_::kOffB1, &M.op2, &full[s], K.b, z, nt * BN, kb + g);
           }
         }
       }
@@ -344,10 +349,10 @@ gemm_persistent(const __grid_constant__ Job job, const __grid_constant__ P prm) 
             } else if (!a1b2) {
               const uint64_t bd = dB0 + (so + ((2 * C_::kTileA) >> 4) + k * kStepB);
               mma_bf16(acc, ad, bd, id, accum);
-              mma_bf16(acc + BN, dA0 + (so + (C_::kTileA >> 4) + k * kStepA), bd, id, accum);
+              mma_bf16(acc + BN, dA0 + (so + (C_::kOffA1B >> 4) + k * kStepA), bd, id, accum);
             } else {
               mma_bf16(acc, ad, dB0 + (so + (C_::kTileA >> 4) + k * kStepB), id, accum);
-              mma_bf16(acc + BN, ad, dB0 + (so + ((2 * C_::kTileA) >> 4) + k * kStepB), id, accum);
+              mma_bf16(acc + BN, ad, dB0 + (so + (C_::kOffB1 >> 4) + k * kStepB), id, accum);
             }
           }
         }
