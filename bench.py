@@ -143,6 +143,11 @@ def kernel_work(w, has_m0: bool) -> dict:
     # the persistent forward: every chunk's four GEMM phases in one launch
     phases = (g1, "tc_g2_y_out_e", g3, "tc_g4_aggregate_state")
     out["tc_fwd_persistent"] = tuple(NC * sum(out[n][i] for n in phases) for i in range(3))
+    # the fused G1 + G2 launch (SwiGLU, opt-in): both phases' work; its bytes
+    # drop the query rows' u, which stays on chip (written once, read once)
+    u_query = 2.0 * 2 * BH * C * dh
+    out["tc_ff12_h_y"] = (out[g1][0] + out["tc_g2_y_out_e"][0], out[g1][1] + out["tc_g2_y_out_e"][1],
+                          out[g1][2] + out["tc_g2_y_out_e"][2] - u_query)
     out["tc_shadow_init"] = (0.0, 0.0, 6.0 * S * BH)
     out["tc_scale_keys"] = (0.0, 0.0, 6.0 * T * dk * BH)
     return out

@@ -332,17 +332,9 @@ __device__ __forceinline__ void store_vec(float* __restrict__ p, const float (&v
 }
 
 template <int PER>
-__global__ void __launch_bounds__(kK1Threads, PER >= 8 ? 8 : 16)  // 16 blocks (2048 threads) per SM
-chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
-                        const float* __restrict__ decay, float* __restrict__ a_out,
-                        float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
-                        int NC, int coef) {
-  __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
-  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
-  const size_t base = (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER;
-  float eta[PER], mu[PER], lam[PER];
+__device__ __forceinline__ void load_gates(const float* __restrict__ lr, const float* __restrict__ mom,
+                                           const float* __restrict__ decay, size_t base,
+                                           float (&eta)[PER], float (&mu)[PER], float (&lam)[PER]) {
   load_vec<PER>(lr + base, eta);
   if (mom) {
     load_vec<PER>(mom + base, mu);
@@ -351,126 +343,166 @@ chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ 
     for (int i = 0; i < PER; ++i) mu[i] = 0.f;
   }
   load_vec<PER>(decay + base, lam);
-  float lmu[PER], llam[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    lmu[i] = logf(mu[i]);
-    llam[i] = logf(lam[i]);
-  }
-  s_mu_first[tid] = mu[0];
+}
+
+// Grid-stride over the (head, chunk) pairs: each block holds the next pair's
+// gates in flight (registers) while it scans the current one, so the loads of
+// a block overlap its own arithmetic and not only that of other blocks.
+template <int PER>
+__global__ void __launch_bounds__(kK1Threads, PER >= 8 ? 6 : PER >= 4 ? 10 : 16)  // no spills
+chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                        const float* __restrict__ decay, float* __restrict__ a_out,
+                        float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
+                        int NC, int coef) {
+  __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
+  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int pairs = BH * NC;
   if (tid == 0) s_mu_first[kK1Threads] = 0.f;  // no token after the chunk's last
-
-  // suffix log-sums: exclusive (tokens after this segment) and chunk totals
-  float su = 0.f, sl = 0.f;
-#pragma unroll
-  for (int i = PER - 1; i >= 0; --i) {
-    su += lmu[i];
-    sl += llam[i];
+  float eta[PER], mu[PER], lam[PER];
+  if ((int)blockIdx.x < pairs) {
+    const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
+    load_gates<PER>(lr, mom, decay, (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER, eta, mu, lam);
   }
-  const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
-  if (lane == 0) {
-    w_su[warp] = su_inc;
-    w_sl[warp] = sl_inc;
-  }
-  __syncthreads();
-  float su_later = 0.f, sl_later = 0.f;  // warps after this one
-  for (int w = kK1Warps - 1; w > warp; --w) {
-    su_later += w_su[w];
-    sl_later += w_sl[w];
-  }
-  float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
-  float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
-  if (lane == 31) {
-    su_excl = 0.f;
-    sl_excl = 0.f;
-  }
-  su_excl += su_later;
-  sl_excl += sl_later;
-  float su_all = 0.f, sl_all = 0.f;
-  for (int w = kK1Warps - 1; w >= 0; --w) {
-    su_all += w_su[w];
-    sl_all += w_sl[w];
-  }
-  const float mu_next = s_mu_first[tid + 1];
-
-  // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map
-  su = su_excl;
-  sl = sl_excl;
-  float Mseg = 1.f, Cseg = 0.f;
-  float asum = 0.f, bsum = 0.f;
-  float av[PER], bv[PER];
-#pragma unroll
-  for (int i = PER - 1; i >= 0; --i) {
-    av[i] = eta[i] * expf(su);
-    asum += av[i];
-    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
-    Cseg = expf(sl) + m * Cseg;
-    Mseg = m * Mseg;
-    su += lmu[i];
-    sl += llam[i];
-  }
-  float M = Mseg, Cc = Cseg;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float Mr = __shfl_down_sync(0xffffffffu, M, off);
-    const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
-    if (lane + off < 32) {
-      Cc = Cc + M * Cr;
-      M = M * Mr;
-    }
-  }
-  if (lane == 0) {
-    w_M[warp] = M;
-    w_C[warp] = Cc;
-  }
-  __syncthreads();
-  float r_end = 0.f;
-  for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
-  const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
-  const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
-  float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
-
-  // reverse walk 2: R_t and the weight kernel b_t
-  sl = sl_excl;
-  float r1 = 0.f;
-#pragma unroll
-  for (int i = PER - 1; i >= 0; --i) {
-    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
-    const float r = expf(sl) + m * r_next;
-    bv[i] = eta[i] * r;
-    bsum += bv[i];
-    r_next = r;
-    if (i == 0) r1 = r;
-    sl += llam[i];
-  }
-  if (coef) {  // the chunk-averaged variant: every token carries the chunk means
-    const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
-    __syncthreads();  // w_su / w_sl are free again
-    if (lane == 0) {
-      w_su[warp] = ai;
-      w_sl[warp] = bi;
-    }
-    __syncthreads();
-    float at = 0.f, bt = 0.f;
-    for (int w = kK1Warps - 1; w >= 0; --w) {
-      at += w_su[w];
-      bt += w_sl[w];
-    }
-    const float n = (float)(PER * kK1Threads);
+  for (int job = blockIdx.x; job < pairs; job += gridDim.x) {
+    const int bh = job / NC, ci = job % NC;
+    const size_t base = (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER;
+    float lmu[PER], llam[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      av[i] = at / n;
-      bv[i] = bt / n;
+      lmu[i] = logf(mu[i]);
+      llam[i] = logf(lam[i]);
     }
-  }
-  store_vec<PER>(a_out + base, av);
-  store_vec<PER>(b_out + base, bv);
-  if (tid == 0) {  // the thread holding token 1
-    const size_t plane = (size_t)BH * NC;
-    const size_t o = (size_t)bh * NC + ci;
-    scal[o] = expf(su_all);
-    scal[plane + o] = expf(sl_all);
-    scal[2 * plane + o] = mu[0] * r1;
+    const float mu0 = mu[0];
+    s_mu_first[tid] = mu0;
+    // the next pair's gates: issued now, first used at the next iteration
+    float eta_n[PER], mu_n[PER], lam_n[PER];
+    const int nxt = job + gridDim.x;
+    if (nxt < pairs) {
+      const int bn = nxt / NC, cn = nxt % NC;
+      load_gates<PER>(lr, mom, decay, (size_t)bn * T + (size_t)cn * C + (size_t)tid * PER, eta_n,
+                      mu_n, lam_n);
+    }
+
+    // suffix log-sums: exclusive (tokens after this segment) and chunk totals
+    float su = 0.f, sl = 0.f;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      su += lmu[i];
+      sl += llam[i];
+    }
+    const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
+    if (lane == 0) {
+      w_su[warp] = su_inc;
+      w_sl[warp] = sl_inc;
+    }
+    __syncthreads();
+    float su_later = 0.f, sl_later = 0.f;  // warps after this one
+    for (int w = kK1Warps - 1; w > warp; --w) {
+      su_later += w_su[w];
+      sl_later += w_sl[w];
+    }
+    float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
+    float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
+    if (lane == 31) {
+      su_excl = 0.f;
+      sl_excl = 0.f;
+    }
+    su_excl += su_later;
+    sl_excl += sl_later;
+    float su_all = 0.f, sl_all = 0.f;
+    for (int w = kK1Warps - 1; w >= 0; --w) {
+      su_all += w_su[w];
+      sl_all += w_sl[w];
+    }
+    const float mu_next = s_mu_first[tid + 1];
+
+    // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map; the
+    // decay products L(t+1, n) are kept for walk 2, which needs the same ones
+    su = su_excl;
+    sl = sl_excl;
+    float Mseg = 1.f, Cseg = 0.f;
+    float asum = 0.f, bsum = 0.f;
+    float av[PER], bv[PER], el[PER];
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      av[i] = eta[i] * expf(su);
+      asum += av[i];
+      const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+      el[i] = expf(sl);
+      Cseg = el[i] + m * Cseg;
+      Mseg = m * Mseg;
+      su += lmu[i];
+      sl += llam[i];
+    }
+    float M = Mseg, Cc = Cseg;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float Mr = __shfl_down_sync(0xffffffffu, M, off);
+      const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+      if (lane + off < 32) {
+        Cc = Cc + M * Cr;
+        M = M * Mr;
+      }
+    }
+    if (lane == 0) {
+      w_M[warp] = M;
+      w_C[warp] = Cc;
+    }
+    __syncthreads();
+    float r_end = 0.f;
+    for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
+    const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
+    const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
+    float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
+
+    // reverse walk 2: R_t and the weight kernel b_t
+    float r1 = 0.f;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+      const float r = el[i] + m * r_next;
+      bv[i] = eta[i] * r;
+      bsum += bv[i];
+      r_next = r;
+      if (i == 0) r1 = r;
+    }
+    if (coef) {  // the chunk-averaged variant: every token carries the chunk means
+      const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
+      __syncthreads();  // w_su / w_sl are free again
+      if (lane == 0) {
+        w_su[warp] = ai;
+        w_sl[warp] = bi;
+      }
+      __syncthreads();
+      float at = 0.f, bt = 0.f;
+      for (int w = kK1Warps - 1; w >= 0; --w) {
+        at += w_su[w];
+        bt += w_sl[w];
+      }
+      const float n = (float)(PER * kK1Threads);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        av[i] = at / n;
+        bv[i] = bt / n;
+      }
+      __syncthreads();  // every warp has read w_su / w_sl before the next pair writes them
+    }
+    store_vec<PER>(a_out + base, av);
+    store_vec<PER>(b_out + base, bv);
+    if (tid == 0) {  // the thread holding token 1
+      const size_t plane = (size_t)BH * NC;
+      const size_t o = (size_t)bh * NC + ci;
+      scal[o] = expf(su_all);
+      scal[plane + o] = expf(sl_all);
+      scal[2 * plane + o] = mu0 * r1;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      eta[i] = eta_n[i];
+      mu[i] = mu_n[i];
+      lam[i] = lam_n[i];
+    }
   }
 }
 
@@ -622,6 +654,33 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
 
 }  // namespace
 
+// One resident wave at most: every block then walks several (head, chunk)
+// pairs, prefetching the next one's gates.
+template <int PER>
+cudaError_t launch_vec(const float* lr, const float* mom, const float* decay, float* a, float* b,
+                       float* scal, int BH, int T, int C, int NC, int coef, cudaStream_t st) {
+  static int wave[4][64] = {};  // [log2 PER][device]: resident blocks on the whole GPU
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int pi = PER >= 8 ? 3 : PER >= 4 ? 2 : PER - 1;
+  int cap = (dev >= 0 && dev < 64) ? wave[pi][dev] : 0;
+  if (cap == 0) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_coeffs_vec_kernel<PER>,
+                                                      kK1Threads, 0);
+    if (e != cudaSuccess) return e;
+    cap = sms * (per_sm > 0 ? per_sm : 1);
+    if (dev >= 0 && dev < 64) wave[pi][dev] = cap;
+  }
+  const int pairs = BH * NC;
+  chunk_coeffs_vec_kernel<PER><<<pairs < cap ? pairs : cap, kK1Threads, 0, st>>>(
+      lr, mom, decay, a, b, scal, BH, T, C, NC, coef);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
                                 float* b, float* scal, int BH, int T, int C, int NC, int coef,
                                 cudaStream_t st) {
@@ -634,10 +693,10 @@ cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* 
   if (T % C == 0 && C % kK1Threads == 0 && (per == 1 || per == 2 || per == 4 || per == 8) &&
       vec_ok(lr) && vec_ok(mom) && vec_ok(decay) && vec_ok(a) && vec_ok(b)) {
     switch (per) {
-      case 1: chunk_coeffs_vec_kernel<1><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
-      case 2: chunk_coeffs_vec_kernel<2><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
-      case 4: chunk_coeffs_vec_kernel<4><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
-      default: chunk_coeffs_vec_kernel<8><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      case 1: return launch_vec<1>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
+      case 2: return launch_vec<2>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
+      case 4: return launch_vec<4>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
+      default: return launch_vec<8>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
     }
     return cudaGetLastError();
   }

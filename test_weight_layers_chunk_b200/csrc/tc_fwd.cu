@@ -656,6 +656,391 @@ template <> struct EpiName<EpiG3Gelu> { static constexpr const char* v = "tc_g3_
 template <> struct EpiName<EpiG1Lin> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 template <> struct EpiName<EpiG1LinPad> { static constexpr const char* v = "tc_g1_linear_out_e"; };
 
+// ---------------------------------------------------------------- fused G1 + G2
+// SwiGLU: one launch per chunk computes G1 and G2 together. A CTA takes a
+// 128-row tile of [q; k] rows of one head and, per block of 128 hidden units j,
+//   H_j = X [W1; W3]_j^T          (tensor memory, 256 columns: h1 | h3)
+//   u_j = silu(h1) h3             (epilogue warps -> shared memory, bf16, laid
+//                                  out as the K-major operand of the next MMA)
+//   Y  += u_j W2_j^T              (tensor memory, d_v columns)
+// and after the last block turns Y into out (query rows) or E, aE, bE (key
+// rows). The query rows' u never leaves the chip; the key rows' u (for the W2
+// aggregation) and their silu factors (for G3) are written once. The MMA of
+// H_{j+1} starts as soon as the epilogue has read H_j into registers, so the
+// silu math of block j overlaps it; Y_j is issued after H_{j+1}. Each u value
+// and each Y element is computed with the same operations in the same order as
+// by G1 then G2, so the results are the same bit for bit.
+// Named barrier of the eight epilogue warps (warps 2..9) of the fused and the
+// persistent kernels.
+__device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+namespace ff {
+constexpr int kStages = 3;
+constexpr uint32_t kStage = 49152;   // X k-block 16 KB + W13 k-block 32 KB, or a W2 k-block
+constexpr int kEW = 8;
+constexpr uint32_t kU = 32768;       // u of one block: 128 rows x 128 units, two 64-column tiles
+constexpr uint32_t kEpi = 81920;     // [u buffer 0 | u buffer 1 | 16 KB]: 8 x 10 KB of staging at the end
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStage + kEpi + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert(EpiG2::kSmem <= (int)(kEpi / kEW), "the Y epilogue's staging fits");
+}  // namespace ff
+
+struct FfJob {
+  CUtensorMap mX[2];  // query rows, key rows: [BH T, d_k], box 64 x 128
+  CUtensorMap mW13;   // interleaved [W1; W3] copy: [BH 2 d_h, d_k], box 64 x 256
+  CUtensorMap mW2;    // W2 copy: [BH d_v, d_h], box 64 x d_v
+  CUtensorMap mU;     // A = [u_q; u_k] per head: [BH 2C, d_h], box 64 x 32 (128B swizzle)
+  int mtiles;         // 128-row tiles per head and row class: C / 128
+  int nblk, kbh;      // hidden blocks (d_h / 128), k-blocks of H (d_k / 64)
+  int total;          // tiles: BH x 2 x mtiles (key-row tiles first)
+  int* status;
+  int ci, t0, clen;
+  int stall;          // failure-detection test hook, as in tc2::Job
+  unsigned long long wait_ns;
+};
+
+// The fused kernel's final epilogue (Y -> out, or E, aE, bE), kept out of line
+// so that its registers and those of the H epilogue are not live together.
+template <int DV>
+__device__ __noinline__ void ff_y_epilogue(const FwdP& p, const tc2::EpiCtx<DV>& c, bool key_rows,
+                                           int r0, int pad) {
+  if (pad) out_or_residual<true, DV>(p, c, key_rows, r0, true);
+  else out_or_residual<false, DV>(p, c, key_rows, r0, true);
+}
+
+template <int DV>
+__global__ void __launch_bounds__((2 + ff::kEW) * 32, 1)
+ff12_kernel(const __grid_constant__ FfJob J, const __grid_constant__ FwdP prm) {
+  using namespace ff;
+  constexpr uint32_t kW2Bytes = (uint32_t)DV * 128;  // one W2 k-block: DV rows x 64 bf16
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint8_t* epi = smem + (size_t)kStages * kStage;  // u buffers, then Y-epilogue staging
+  __shared__ uint64_t full[kStages], empty[kStages];
+  __shared__ uint64_t h_full, h_empty, u_full[2], u_empty[2], y_full, y_empty;
+  __shared__ uint64_t epi_bar[tc2::kEpiBars * kEW];
+  __shared__ uint64_t never;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int s_err_;
+  volatile int& s_err = s_err_;
+  const unsigned long long lim = J.wait_ns ? J.wait_ns : tc::kWaitNs;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Dims& d = prm.d;
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    s_err = 0;
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    tc::mbar_init(&h_full, 1);
+    tc::mbar_init(&h_empty, kEW);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&u_full[b], kEW);
+      tc::mbar_init(&u_empty[b], 1);
+    }
+    tc::mbar_init(&y_full, 1);
+    tc::mbar_init(&y_empty, kEW);
+    for (int w = 0; w < tc2::kEpiBars * kEW; ++w) tc::mbar_init(&epi_bar[w], 1);
+    tc::mbar_init(&never, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tmap(&J.mX[0]);
+    tc::prefetch_tmap(&J.mX[1]);
+    tc::prefetch_tmap(&J.mW13);
+    tc::prefetch_tmap(&J.mW2);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&tmem_slot, 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = tmem_slot;  // H at columns [0, 256), Y at [256, 256 + DV)
+  griddep_wait();
+  const int per_class = J.total / 2;
+  auto decode = [&](int t, int& cls, int& z, int& mt) {
+    cls = t < per_class ? 1 : 0;  // key-row tiles first (their epilogues do more)
+    const int r = cls ? t : t - per_class;
+    z = r / J.mtiles;
+    mt = r - z * J.mtiles;
+  };
+  int mma_done = 0;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- producer: per tile, the H k-blocks of block j, then W2 of block j - 1
+    int it = 0;
+    bool ok = true;
+    auto stage = [&](uint32_t bytes) -> uint8_t* {
+      const int s = it % kStages;
+      const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+      if (it >= kStages && !tc::mbar_wait_hint(&empty[s], ph ^ 1u, lim)) {
+        atomicExch(J.status, tc2::kErrProducer);
+        s_err = 1;
+        ok = false;
+        return nullptr;
+      }
+      tc::mbar_expect_tx(&full[s], bytes);
+      return ring + (size_t)s * kStage;
+    };
+    for (int t = blockIdx.x; t < J.total && ok; t += gridDim.x) {
+      int cls, z, mt;
+      decode(t, cls, z, mt);
+      const int xrow = z * d.T + J.t0 + mt * 128;
+      auto w2 = [&](int jj) {
+        for (int kb = 0; kb < 2 && ok; ++kb) {
+          uint8_t* st = stage(kW2Bytes);
+          if (!st) break;
+          tc::tma_load_2d(st, &J.mW2, &full[it % kStages], jj * 128 + kb * 64, z * DV);
+          ++it;
+        }
+      };
+      for (int j = 0; j < J.nblk && ok; ++j) {
+        for (int kb = 0; kb < J.kbh && ok; ++kb) {
+          uint8_t* st = stage(49152u);
+          if (!st) break;
+          tc::tma_load_2d(st, &J.mX[cls], &full[it % kStages], kb * 64, xrow);
+          tc::tma_load_2d(st + 16384, &J.mW13, &full[it % kStages], kb * 64, z * 2 * d.d_h + j * 256);
+          ++it;
+        }
+        if (j >= 1) w2(j - 1);
+      }
+      if (ok) w2(J.nblk - 1);
+    }
+    for (int j = it - kStages < 0 ? 0 : it - kStages; j < it; ++j)
+      (void)tc::mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, lim);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    const uint64_t dR = tc2::sdesc(tc::smem_u32(ring), false);
+    const uint64_t dU = tc2::sdesc(tc::smem_u32(epi), false);
+    constexpr uint32_t idH = tc2::idesc(128, 256, false, false);
+    constexpr uint32_t idY = tc2::idesc(128, DV, false, false);
+    int it = 0, gb = 0, ti = 0;
+    bool ok = !(J.stall && blockIdx.x == 0 && !tc::mbar_wait(&never, 0u, lim));
+    if (!ok) {
+      atomicExch(J.status, tc2::kErrMma);
+      s_err = 1;
+    }
+    auto take = [&]() -> uint32_t {  // the next ring stage, filled; returns its offset >> 4
+      const int s = it % kStages;
+      const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+      if (!tc::mbar_wait_hint(&full[s], ph, lim)) {
+        atomicExch(J.status, tc2::kErrMma);
+        s_err = 1;
+        ok = false;
+        return 0;
+      }
+      tc::tc_fence_after();
+      return ((uint32_t)s * kStage) >> 4;
+    };
+    auto release = [&]() {
+      tc::mma_commit(&empty[it % kStages]);
+      ++it;
+    };
+    auto issue_y = [&](int jj) {  // Y += u_jj W2_jj^T
+      const int g = gb + jj, b = g & 1;
+      if (!tc::mbar_wait(&u_full[b], (uint32_t)(g >> 1) & 1u, lim) ||
+          (jj == 0 && !tc::mbar_wait(&y_empty, ((uint32_t)ti & 1u) ^ 1u, lim))) {
+        atomicExch(J.status, tc2::kErrMma);
+        s_err = 1;
+        ok = false;
+        return;
+      }
+      tc::tc_fence_after();
+      for (int kb = 0; kb < 2 && ok; ++kb) {
+        const uint32_t so = take();
+        if (!ok) break;
+        const uint32_t uo = ((uint32_t)b * kU + (uint32_t)kb * 16384) >> 4;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_bf16(tmem + 256, dU + (uo + k * 2), dR + (so + k * 2), idY, (jj | kb | k) != 0);
+        release();
+      }
+      tc::mma_commit(&u_empty[b]);
+    };
+    for (int t = blockIdx.x; t < J.total && ok; t += gridDim.x, ++ti) {
+      for (int j = 0; j < J.nblk && ok; ++j) {
+        if (!tc::mbar_wait(&h_empty, ((uint32_t)(gb + j) & 1u) ^ 1u, lim)) {
+          atomicExch(J.status, tc2::kErrMma);
+          s_err = 1;
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        for (int kb = 0; kb < J.kbh && ok; ++kb) {
+          const uint32_t so = take();
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16(tmem, dR + (so + k * 2), dR + (so + (16384 >> 4) + k * 2), idH, (kb | k) != 0);
+          release();
+        }
+        tc::mma_commit(&h_full);
+        if (j >= 1 && ok) issue_y(j - 1);
+      }
+      if (ok) issue_y(J.nblk - 1);
+      if (ok) {
+        tc::mma_commit(&y_full);
+        ++mma_done;
+      }
+      gb += J.nblk;
+    }
+  } else if (warp >= 2) {
+    // ---------------- epilogue: every warp runs the same barriers on every tile,
+    // also after a failure (it then skips the work)
+    const int ew = warp - 2, quad = warp & 3, part = ew >> 2;
+    const int row = quad * 32 + lane;  // TMEM lane = row of the tile
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    uint32_t uses[tc2::kEpiBars] = {0u, 0u, 0u, 0u};
+    int gb = 0, ti = 0;
+    for (int t = blockIdx.x; t < J.total; t += gridDim.x, ++ti) {
+      int cls, z, mt;
+      decode(t, cls, z, mt);
+      const int r0 = mt * 128 + quad * 32;  // first row (within the chunk) of this warp
+      // the previous tile's staged stores have read the epilogue region
+      if (lane == 0) tc::bulk_wait_read<0>();
+      __syncwarp();
+      epi_barrier();
+      for (int j = 0; j < J.nblk; ++j) {
+        const int g = gb + j, b = g & 1;
+        bool ok = !s_err;
+        if (ok && !tc::mbar_wait(&h_full, (uint32_t)g & 1u, lim)) {
+          if (lane == 0) atomicExch(J.status, tc2::kErrEpilogue);
+          s_err = 1;
+          ok = false;
+        }
+        tc::tc_fence_after();
+        // buffer b is free once the MMA of its previous use and our store of it are done
+        if (ok && !tc::mbar_wait(&u_empty[b], ((uint32_t)(g >> 1) & 1u) ^ 1u, lim)) {
+          if (lane == 0) atomicExch(J.status, tc2::kErrEpilogue);
+          s_err = 1;
+          ok = false;
+        }
+        if (ok && lane == 0) tc::bulk_wait_read<0>();
+        __syncwarp();
+        uint8_t* ut = epi + (size_t)b * kU + (size_t)part * 16384;  // this warp's 64-column tile
+        uint8_t* urow = ut + row * 128;
+        bf16* sk = prm.Sk + ((size_t)z * d.C + r0 + lane) * (2 * d.d_h) + j * 128 + part * 64;
+        // u (and for key rows the silu factors s1 = silu(h1), s2 = h3 silu'(h1)),
+        // formed exactly as G1's epilogue forms them, in two halves of 32 units:
+        // H is released for the next block's MMA once the second half is read
+        for (int half = 0; half < 2; ++half) {
+          float h1[32], h3[32];
+          if (ok) {
+            const int cs = part * 64 + half * 32;
+            uint32_t a[32], c3[32];
+            tmem_ld32_nowait(tl + (uint32_t)cs, a);
+            tmem_ld32_nowait(tl + (uint32_t)(128 + cs), c3);
+            tmem_wait_ld2(a, c3);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              h1[i] = __uint_as_float(a[i]);
+              h3[i] = __uint_as_float(c3[i]);
+            }
+          }
+          if (half == 1) {
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc2::mbar_arrive(&h_empty);  // the next block's MMA may overwrite H
+          }
+          if (!ok) continue;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = half * 4 + kk;
+            float uu[8], f1[8], f2[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float x1 = h1[8 * kk + i], x3 = h3[8 * kk + i];
+              if (cls == 0) {
+                uu[i] = x1 * fast_sigmoid(x1) * x3;
+              } else {
+                const float sg = fast_sigmoid(x1);
+                const float s1 = x1 * sg;
+                f2[i] = x3 * sg * (1.0f + x1 * (1.0f - sg));
+                uu[i] = s1 * x3;
+                f1[i] = s1;
+              }
+            }
+            *reinterpret_cast<uint4*>(urow + ((k ^ (row & 7)) << 4)) =
+                make_uint4(pack2(uu[0], uu[1]), pack2(uu[2], uu[3]), pack2(uu[4], uu[5]), pack2(uu[6], uu[7]));
+            if (cls == 1) {
+              reinterpret_cast<uint4*>(sk)[k] =
+                  make_uint4(pack2(f1[0], f1[1]), pack2(f1[2], f1[3]), pack2(f1[4], f1[5]), pack2(f1[6], f1[7]));
+              reinterpret_cast<uint4*>(sk + d.d_h)[k] =
+                  make_uint4(pack2(f2[0], f2[1]), pack2(f2[2], f2[3]), pack2(f2[4], f2[5]), pack2(f2[6], f2[7]));
+            }
+          }
+        }
+        tc::fence_async_smem();  // the MMA (async proxy) reads what the threads wrote
+        __syncwarp();
+        if (lane == 0) tc2::mbar_arrive(&u_full[b]);
+        if (ok && cls == 1 && lane == 0) {
+          // key rows: u for the W2 aggregation (TMA store of this warp's 32 x 64 block)
+          tc::tma_store_2d_hint(&J.mU, ut + quad * 32 * 128, j * 128 + part * 64,
+                                z * 2 * d.C + d.C + r0, tc::l2_evict_last());
+          tc::bulk_commit();
+        }
+        __syncwarp();
+      }
+      gb += J.nblk;
+      // Y -> out (query rows) or E, aE, bE (key rows), staged through the epilogue
+      // region once every warp's u stores have read it
+      bool ok = !s_err;
+      if (ok && !tc::mbar_wait(&y_full, (uint32_t)ti & 1u, lim)) {
+        if (lane == 0) atomicExch(J.status, tc2::kErrEpilogue);
+        s_err = 1;
+        ok = false;
+      }
+      tc::tc_fence_after();
+      if (lane == 0) tc::bulk_wait_read<0>();
+      __syncwarp();
+      epi_barrier();
+      if (ok) {
+        tc2::EpiCtx<DV> c;
+        c.cls = cls;
+        c.z = z;
+        c.m0 = mt * 128;
+        c.n0 = 0;
+        c.row = row;
+        c.quad = quad;
+        c.part = part;
+        c.nparts = 2;
+        c.taddr = tl + 256u;
+        c.wsmem = epi + (size_t)ew * (kEpi / kEW);
+        c.wbar = epi_bar + tc2::kEpiBars * ew;
+        c.uses = uses;
+        c.slot = 0;
+        c.iter = ti;
+        c.seq = ti;
+        c.pre = 0;
+        c.ci = J.ci;
+        c.t0 = J.t0;
+        c.clen = J.clen;
+        c.wshadow = 0;
+        c.nxt_valid = 0;
+        c.nxt_cls = c.nxt_z = c.nxt_m0 = c.nxt_n0 = c.nxt_ci = 0;
+        ff_y_epilogue<DV>(prm, c, cls == 1, r0, J.clen < d.C);
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc2::mbar_arrive(&y_empty);
+    }
+    if (lane == 0) tc::bulk_wait_all();
+    __syncwarp();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    if (lane == 0 && mma_done > 0) (void)tc::mbar_wait(&y_full, (uint32_t)(mma_done - 1) & 1u, lim);
+    __syncwarp();
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------------- persistent forward
 // The whole SwiGLU forward (every chunk, G1 to G4) in one cooperative launch.
 // Each CTA (one per SM) walks a static list of the tiles of all four GEMM phases
@@ -778,9 +1163,6 @@ __device__ __forceinline__ bool mk_dep_ready(const MegaJob& J, const MkTile& T) 
   int dp, tg;
   mk_need(J, T, dp, tg);
   return dp < 0 || ld_acquire(J.cnt + (size_t)dp * J.BH + T.z) >= tg;
-}
-__device__ __forceinline__ void epi_barrier() {  // the eight epilogue warps
-  asm volatile("bar.sync 1, %0;" ::"n"(mk::kEW * 32) : "memory");
 }
 
 template <bool MN, int ROWS>
@@ -1336,6 +1718,17 @@ cudaError_t launch_mega(const MegaJob& J, const FwdP& p, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, fwd_persistent, J, p);
 }
 
+template <int DV>
+cudaError_t launch_ff12(const FfJob& J, const FwdP& p, cudaStream_t st) {
+  constexpr size_t smem = ff::kSmemBytes;
+  auto kern = ff12_kernel<DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = J.total < num_sms() ? J.total : num_sms();
+  E2TTT_TRACE("tc_ff12_h_y", st);
+  return launch_pdl(kern, dim3(grid), dim3((2 + ff::kEW) * 32), smem, st, J, p);
+}
+
 struct Scratch {
   bf16 *Wsh13, *W2sh, *A, *Sk, *E, *Ea, *Eb, *dH, *Ka, *Kb;
   int* cnt;  // persistent forward: completed tiles per (phase, head)
@@ -1531,6 +1924,29 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   }
   if (!ok) return cudaErrorInvalidValue;
 
+  // SwiGLU: G1 and G2 as one fused launch per chunk (u of the query rows stays
+  // on chip), selected with E2TTT_FUSED=1 in the environment. Not the default:
+  // on the 1.3B layer it is slower than the two launches it replaces (each
+  // 128-row tile streams its head's whole W1, W3 and W2 through a three-stage
+  // ring, behind a single H accumulator).
+  const char* env_f = getenv("E2TTT_FUSED");
+  const bool fused = d.kind == 1 && !persistent && (dv == 128 || dv == 256) && dh % 128 == 0 &&
+                     env_f && env_f[0] == '1';
+  FfJob fj{};
+  if (fused) {
+    fj.mX[0] = g1.maps[0].op0;
+    fj.mX[1] = g1.maps[1].op0;
+    fj.mW13 = g1.maps[0].op2;
+    ok &= make_map(&fj.mW2, s.W2sh, (uint64_t)BH * dv, dh, (uint32_t)dv);
+    ok &= make_map(&fj.mU, s.A, (uint64_t)BH * 2 * C, dh, 32);
+    fj.mtiles = C / 128;
+    fj.nblk = dh / 128;
+    fj.kbh = dk / 64;
+    fj.total = BH * 2 * fj.mtiles;
+    fj.status = status;
+    if (!ok) return cudaErrorInvalidValue;
+  }
+
   // SwiGLU with momentum and no saved states may run every chunk in one
   // persistent, cooperative launch; it is selected with E2TTT_PERSISTENT=1 in
   // the environment (the per-phase launches are faster on the shapes measured).
@@ -1618,11 +2034,19 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     g4.cls[0].b.y_base = ci * C;                        // key rows (K dimension) of this chunk
     g4w.cls[0].b.y_base = ci * C;
     if (d.kind != 0) {
-      if (d.kind == 1)
+      if (fused) {
+        fj.ci = ci;
+        fj.t0 = ci * C;
+        fj.clen = clen;
+        fj.stall = g1.stall;  // the stall hook, armed for this chunk's first launch
+        fj.wait_ns = g1.wait_ns;
+        e = dv == 256 ? launch_ff12<256>(fj, p, st) : launch_ff12<128>(fj, p, st);
+      } else if (d.kind == 1) {
         e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
-      else
+      } else {
         e = launch<128, 1, false, false, 4, EpiG1Gelu, kEpiWarps, EpiG1Gelu::kSmem>(g1, p, st);
-      if (e == cudaSuccess) {
+      }
+      if (e == cudaSuccess && !fused) {
         if (wide2)
           e = clen < C ? launch<256, 1, false, false, 3, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
                          : launch<256, 1, false, false, 3, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);

@@ -103,16 +103,21 @@ def test_bwd_bf16_small(E):
     check(gpu, ref, 2e-2, label="swiglu_bf16_small")
 
 
-@pytest.mark.parametrize("variant", ["stated", "preserving"])
+@pytest.mark.parametrize("variant", ["stated", "preserving", "preserving_upstream"])
 def test_bwd_training_workload(E, variant):
     """fwd then bwd at the 1.3B layer's shapes (B=4, H=8, d=256, d_h=512, T=2048,
-    C=512), upstream dOut ~ N(0,1); the oracle recomputes two heads."""
+    C=512), upstream dOut ~ N(0,1); the oracle recomputes two heads. The last
+    variant also feeds upstream gradients of the final states, dW_end and
+    dM_end ~ N(0, 0.1^2) (a layer whose carried state is read by a later
+    segment), on the state-preserving gates that keep them from decaying away."""
     w = gen.BY_NAME["train_1p3b_2k"]
-    if variant == "preserving":
+    if variant != "stated":
         w = gen.state_preserving(w)
     x = gen.generate(w, m0_scale=0.0 if variant == "stated" else 0.5)
+    dW, dM = (gen.upstream_state_grads(w, seed=11, scale=0.1) if variant == "preserving_upstream"
+              else (None, None))
     heads = [(0, 0), (3, 7)]
-    gpu, ref = run_bwd(E, w, x, None, None, heads=heads)
+    gpu, ref = run_bwd(E, w, x, dW, dM, heads=heads)
     check(gpu, ref, 2e-2, heads=heads, label=f"train_1p3b_2k {variant}")
 
 

@@ -113,6 +113,51 @@ def test_chunk_coeffs_vector_path_matches_block_path(E, C, mode):
             assert rel(a[bi, hi, sl], ra) < TOL_COEF and rel(b[bi, hi, sl], rb) < TOL_COEF
 
 
+@pytest.mark.parametrize("C", [128, 512, 1024])
+@pytest.mark.parametrize("mode", ["per_token", "chunk_mean"])
+def test_chunk_coeffs_vector_path_walks_several_chunks_per_block(E, C, mode):
+    """More (head, chunk) pairs than one resident wave of the vectorised K1
+    kernel holds (4096 pairs; at most 148 SMs x 16 blocks resident), so each
+    block scans several pairs, loading the next pair's gates during the current
+    scan. Bit-identical to the block kernel on every pair, and the oracle on a
+    sample that includes the first and last pairs."""
+    import torch
+    B, H, nc = 16, 16, 16
+    T = nc * C
+    w = gen.Workload("k1w", gen.LINEAR, gen.F32, B, H, 1, 1, 0, T, C, "uniform", 0.9, seed=C + 1)
+    x = gen.generate(w)
+    coef = E.COEF_CHUNK_MEAN if mode == "chunk_mean" else E.COEF_PER_TOKEN
+    s = E.make_shape(B, H, T, C, 1, 1, 0, E.LINEAR, E.F32, coef=coef)
+
+    def run(shift):
+        bufs = []
+        for name in ("lr", "mom", "decay"):
+            t = torch.empty(B * H * T + shift, device="cuda")
+            t[shift:] = dev(x[name]).reshape(-1)
+            bufs.append(t[shift:].view(B, H, T))
+        outs = [torch.empty(B * H * T + shift, device="cuda")[shift:].view(B, H, T) for _ in range(2)]
+        sc = torch.empty((3, B, H, nc), device="cuda")
+        E.e2ttt_chunk_coeffs(s, *bufs, outs[0], outs[1], sc)
+        torch.cuda.synchronize()
+        return outs[0], outs[1], sc
+
+    va, vb, vs = run(0)
+    ba, bb, bs = run(1)
+    assert torch.equal(va, ba) and torch.equal(vb, bb) and torch.equal(vs, bs)
+    kern = O.chunk_mean_kernels if mode == "chunk_mean" else O.chunk_kernels
+    a, b, sc = host(va), host(vb), host(vs)
+    rng = np.random.default_rng(C)
+    pairs = [0, B * H * nc - 1] + list(rng.choice(B * H * nc, 10, replace=False))
+    for p in pairs:
+        bh, c = divmod(int(p), nc)
+        bi, hi = divmod(bh, H)
+        sl = slice(c * C, (c + 1) * C)
+        ra, rb, pu, pl, cc = kern(x["lr"][bi, hi, sl], x["mom"][bi, hi, sl], x["decay"][bi, hi, sl])
+        assert rel(a[bi, hi, sl], ra) < TOL_COEF and rel(b[bi, hi, sl], rb) < TOL_COEF, (p,)
+        for i, ref in enumerate((pu, pl, cc)):
+            assert abs(sc[i, bi, hi, c] - ref) <= TOL_COEF * abs(ref) + 1e-30, (p, i)
+
+
 @pytest.mark.parametrize("edge", ["mu0", "lam1", "lam0", "ragged", "C1", "C1024"])
 def test_chunk_coeffs_edges(E, edge):
     T, C = 300, 64

@@ -127,3 +127,26 @@ def test_wide_tiles_equal_the_persistent_kernels_tiles(E, monkeypatch):
     torch.cuda.synchronize()
     for u, v, n in zip(a[:3], b[:3], ("out", "W_end", "M_end")):
         assert torch.equal(u, v), n
+
+
+@pytest.mark.parametrize("name", ["swiglu_d128", "layer_1p3b_2k_preserving", "ragged_tail", "neg_dot_loss"])
+def test_fused_g1_g2_equals_two_launches(E, name, monkeypatch):
+    """With E2TTT_FUSED=1 the per-phase forward runs G1 and G2 of the SwiGLU
+    fast weight as one fused launch per chunk (u of the query rows stays on
+    chip). Every u value and every element of Y is formed with the same
+    operations in the same order as by the two separate launches: equal bit for
+    bit, saved chunk-start states included."""
+    import torch
+    monkeypatch.setenv("E2TTT_PERSISTENT", "0")
+    w, m0, _ = CASES[name]
+    x = gen.generate(w, m0_scale=0.5)
+    d = device_inputs(w, x)
+    kw = dict(C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss, save_states=True)
+    args = (d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], d["W0"], d["M0"])
+    monkeypatch.setenv("E2TTT_FUSED", "1")
+    a = E.chunk_scan_fwd(*args, **kw)
+    monkeypatch.setenv("E2TTT_FUSED", "0")
+    b = E.chunk_scan_fwd(*args, **kw)
+    torch.cuda.synchronize()
+    for u, v, n in zip(a, b, ("out", "W_end", "M_end", "saved")):
+        assert torch.equal(u, v), (name, n, rel(host(u), host(v)))

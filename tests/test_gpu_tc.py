@@ -54,13 +54,15 @@ def shape_of(E, w):
 
 
 STATED = ("swiglu_d128", "layer_1p3b_2k", "layer_1p3b_16k")
+# one head of every batch row and every head index, for the 32-head 1.3B layer
+EIGHT_HEADS = [(0, 0), (0, 5), (1, 1), (1, 6), (2, 2), (2, 7), (3, 3), (3, 4)]
 CASES = {
     "swiglu_d128": (gen.BY_NAME["swiglu_d128"], None),
     "swiglu_d128_preserving": (gen.state_preserving(gen.BY_NAME["swiglu_d128"]), None),
     "layer_1p3b_2k": (gen.BY_NAME["layer_1p3b_2k"], None),
-    "layer_1p3b_2k_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_2k"]), [(0, 1), (3, 6)]),
+    "layer_1p3b_2k_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_2k"]), EIGHT_HEADS),
     "layer_1p3b_16k": (gen.BY_NAME["layer_1p3b_16k"], None),
-    "layer_1p3b_16k_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_16k"]), [(0, 2)]),
+    "layer_1p3b_16k_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_16k"]), None),
     "linear_bf16": (gen.Workload("lin", gen.LINEAR, gen.BF16, 2, 2, 128, 256, 0, 512, 128, "uniform",
                                  0.999, seed=21, lr_lo=0.002, lr_hi=0.02), None),
     "swiglu_dot": (gen.Workload("dot", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 256, "uniform",
@@ -70,7 +72,7 @@ CASES = {
     "gelu_d128_preserving": (gen.Workload("gelu", gen.GELU, gen.BF16, 1, 2, 128, 128, 256, 512, 128,
                                           "uniform", 0.999, seed=24, lr_lo=0.002, lr_hi=0.02), None),
     "layer_1p3b_2k_gelu_preserving": (gen.state_preserving(gen.BY_NAME["layer_1p3b_2k_gelu"]),
-                                      [(0, 1), (3, 6)]),
+                                      EIGHT_HEADS),
     # a shorter last chunk (T % C != 0), run padded to C tokens: 88 real tokens
     # in the last chunk (one part-filled 128-row tile, one all padding) ...
     "swiglu_tail_88": (gen.Workload("tail88", gen.SWIGLU, gen.BF16, 2, 2, 128, 128, 256, 600, 256,
