@@ -13,7 +13,11 @@
 //   b_t  = eta_t R_t                                           (weight kernel)
 //   U(1,n) = exp(SU_0), L(1,n) = exp(SL_0), c = mu_1 R_1        (chunk scalars)
 // No prefix sum is ever subtracted from another, so mu = 0 or lam = 0 (log = -inf)
-// gives exact zeros instead of NaN.
+// gives exact zeros instead of NaN. The logarithms and exponentials are taken in
+// base 2 (log2f, exp2f: the identities above hold in any base, and the base-2
+// functions cost fewer instructions at the same documented accuracy, 1 and 2
+// ulp), which matters where the scan is bound by its arithmetic rather than its
+// 20 bytes per token.
 //
 // Layout: one 128-thread block per (head, chunk) for chunks up to 8192 tokens
 // (thread i owns a contiguous segment of ceil(n/128) tokens; segment results are
@@ -58,8 +62,8 @@ __device__ __forceinline__ LogSums chunk_log_sums(const float* mu, const float* 
                                                   int lane) {
   float su = 0.f, sl = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
-    su += logf(mu_at(mu, t));
-    sl += logf(lam[t]);
+    su += log2f(mu_at(mu, t));
+    sl += log2f(lam[t]);
   }
   float su_inc = warp_suffix_sum(su, lane);
   float sl_inc = warp_suffix_sum(sl, lane);
@@ -97,14 +101,14 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   float Mseg = 1.f, Cseg = 0.f;
   float asum = 0.f, bsum = 0.f;  // segment sums (chunk means for coef = 1)
   for (int t = s1 - 1; t >= s0; --t) {
-    const float at = eta[t] * expf(su);
+    const float at = eta[t] * exp2f(su);
     a_out[base + t] = at;
     asum += at;
     float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
-    Cseg = expf(sl) + m * Cseg;
+    Cseg = exp2f(sl) + m * Cseg;
     Mseg = m * Mseg;
-    su += logf(mu_at(mu, t));
-    sl += logf(lam[t]);
+    su += log2f(mu_at(mu, t));
+    sl += log2f(lam[t]);
   }
   float M = Mseg, Cc = Cseg;
 #pragma unroll
@@ -124,13 +128,13 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   float r1 = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
     float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
-    float r = expf(sl) + m * r_next;
+    float r = exp2f(sl) + m * r_next;
     const float bt = eta[t] * r;
     b_out[base + t] = bt;
     bsum += bt;
     r_next = r;
     if (t == 0) r1 = r;
-    sl += logf(lam[t]);
+    sl += log2f(lam[t]);
   }
   if (coef) {  // the chunk-averaged variant: every token carries the chunk means
     const float am = __shfl_sync(0xffffffffu, warp_suffix_sum(asum, lane), 0) / (float)n;
@@ -143,8 +147,8 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   if (s0 == 0 && s1 > 0) {  // lane 0 holds token 1
     const size_t plane = (size_t)BH * NC;
     const size_t o = (size_t)bh * NC + ci;
-    scal[o] = expf(ls.su_all);
-    scal[plane + o] = expf(ls.sl_all);
+    scal[o] = exp2f(ls.su_all);
+    scal[plane + o] = exp2f(ls.sl_all);
     scal[2 * plane + o] = mu_at(mu, 0) * r1;
   }
 }
@@ -179,8 +183,8 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
     const float mu = mom ? mom[base + t] : 0.f;  // NULL: no-momentum mode
     s_eta[t] = lr[base + t];
     s_mu[t] = mu;
-    s_lmu[t] = logf(mu);
-    s_llam[t] = logf(decay[base + t]);
+    s_lmu[t] = log2f(mu);
+    s_llam[t] = log2f(decay[base + t]);
   }
   __syncthreads();
   const int per = (n + kK1Threads - 1) / kK1Threads;
@@ -223,11 +227,11 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   float Mseg = 1.f, Cseg = 0.f;
   float asum = 0.f, bsum = 0.f;  // segment sums (chunk means for coef = 1)
   for (int t = s1 - 1; t >= s0; --t) {
-    const float at = s_eta[t] * expf(su);
+    const float at = s_eta[t] * exp2f(su);
     a_out[base + t] = at;
     asum += at;
     const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
-    Cseg = expf(sl) + m * Cseg;
+    Cseg = exp2f(sl) + m * Cseg;
     Mseg = m * Mseg;
     su += s_lmu[t];
     sl += s_llam[t];
@@ -259,7 +263,7 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   float r1 = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
     const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
-    const float r = expf(sl) + m * r_next;
+    const float r = exp2f(sl) + m * r_next;
     const float bt = s_eta[t] * r;
     b_out[base + t] = bt;
     bsum += bt;
@@ -289,8 +293,8 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   if (s0 == 0 && s1 > 0) {  // the thread holding token 1
     const size_t plane = (size_t)BH * NC;
     const size_t o = (size_t)bh * NC + ci;
-    scal[o] = expf(su_all);
-    scal[plane + o] = expf(sl_all);
+    scal[o] = exp2f(su_all);
+    scal[plane + o] = exp2f(sl_all);
     scal[2 * plane + o] = s_mu[0] * r1;
   }
 }
@@ -332,9 +336,17 @@ __device__ __forceinline__ void store_vec(float* __restrict__ p, const float (&v
 }
 
 template <int PER>
-__device__ __forceinline__ void load_gates(const float* __restrict__ lr, const float* __restrict__ mom,
-                                           const float* __restrict__ decay, size_t base,
-                                           float (&eta)[PER], float (&mu)[PER], float (&lam)[PER]) {
+__global__ void __launch_bounds__(kK1Threads, PER >= 8 ? 8 : 16)  // 16 blocks (2048 threads) per SM
+chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                        const float* __restrict__ decay, float* __restrict__ a_out,
+                        float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
+                        int NC, int coef) {
+  __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
+  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
+  const size_t base = (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER;
+  float eta[PER], mu[PER], lam[PER];
   load_vec<PER>(lr + base, eta);
   if (mom) {
     load_vec<PER>(mom + base, mu);
@@ -343,166 +355,126 @@ __device__ __forceinline__ void load_gates(const float* __restrict__ lr, const f
     for (int i = 0; i < PER; ++i) mu[i] = 0.f;
   }
   load_vec<PER>(decay + base, lam);
-}
-
-// Grid-stride over the (head, chunk) pairs: each block holds the next pair's
-// gates in flight (registers) while it scans the current one, so the loads of
-// a block overlap its own arithmetic and not only that of other blocks.
-template <int PER>
-__global__ void __launch_bounds__(kK1Threads, PER >= 8 ? 6 : PER >= 4 ? 10 : 16)  // no spills
-chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
-                        const float* __restrict__ decay, float* __restrict__ a_out,
-                        float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
-                        int NC, int coef) {
-  __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
-  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int pairs = BH * NC;
-  if (tid == 0) s_mu_first[kK1Threads] = 0.f;  // no token after the chunk's last
-  float eta[PER], mu[PER], lam[PER];
-  if ((int)blockIdx.x < pairs) {
-    const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
-    load_gates<PER>(lr, mom, decay, (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER, eta, mu, lam);
+  float lmu[PER], llam[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    lmu[i] = log2f(mu[i]);
+    llam[i] = log2f(lam[i]);
   }
-  for (int job = blockIdx.x; job < pairs; job += gridDim.x) {
-    const int bh = job / NC, ci = job % NC;
-    const size_t base = (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER;
-    float lmu[PER], llam[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      lmu[i] = logf(mu[i]);
-      llam[i] = logf(lam[i]);
-    }
-    const float mu0 = mu[0];
-    s_mu_first[tid] = mu0;
-    // the next pair's gates: issued now, first used at the next iteration
-    float eta_n[PER], mu_n[PER], lam_n[PER];
-    const int nxt = job + gridDim.x;
-    if (nxt < pairs) {
-      const int bn = nxt / NC, cn = nxt % NC;
-      load_gates<PER>(lr, mom, decay, (size_t)bn * T + (size_t)cn * C + (size_t)tid * PER, eta_n,
-                      mu_n, lam_n);
-    }
+  s_mu_first[tid] = mu[0];
+  if (tid == 0) s_mu_first[kK1Threads] = 0.f;  // no token after the chunk's last
 
-    // suffix log-sums: exclusive (tokens after this segment) and chunk totals
-    float su = 0.f, sl = 0.f;
+  // suffix log-sums: exclusive (tokens after this segment) and chunk totals
+  float su = 0.f, sl = 0.f;
 #pragma unroll
-    for (int i = PER - 1; i >= 0; --i) {
-      su += lmu[i];
-      sl += llam[i];
+  for (int i = PER - 1; i >= 0; --i) {
+    su += lmu[i];
+    sl += llam[i];
+  }
+  const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
+  if (lane == 0) {
+    w_su[warp] = su_inc;
+    w_sl[warp] = sl_inc;
+  }
+  __syncthreads();
+  float su_later = 0.f, sl_later = 0.f;  // warps after this one
+  for (int w = kK1Warps - 1; w > warp; --w) {
+    su_later += w_su[w];
+    sl_later += w_sl[w];
+  }
+  float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
+  float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
+  if (lane == 31) {
+    su_excl = 0.f;
+    sl_excl = 0.f;
+  }
+  su_excl += su_later;
+  sl_excl += sl_later;
+  float su_all = 0.f, sl_all = 0.f;
+  for (int w = kK1Warps - 1; w >= 0; --w) {
+    su_all += w_su[w];
+    sl_all += w_sl[w];
+  }
+  const float mu_next = s_mu_first[tid + 1];
+
+  // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map
+  su = su_excl;
+  sl = sl_excl;
+  float Mseg = 1.f, Cseg = 0.f;
+  float asum = 0.f, bsum = 0.f;
+  float av[PER], bv[PER];
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    av[i] = eta[i] * exp2f(su);
+    asum += av[i];
+    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+    Cseg = exp2f(sl) + m * Cseg;
+    Mseg = m * Mseg;
+    su += lmu[i];
+    sl += llam[i];
+  }
+  float M = Mseg, Cc = Cseg;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float Mr = __shfl_down_sync(0xffffffffu, M, off);
+    const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+    if (lane + off < 32) {
+      Cc = Cc + M * Cr;
+      M = M * Mr;
     }
-    const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
+  }
+  if (lane == 0) {
+    w_M[warp] = M;
+    w_C[warp] = Cc;
+  }
+  __syncthreads();
+  float r_end = 0.f;
+  for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
+  const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
+  const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
+  float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
+
+  // reverse walk 2: R_t and the weight kernel b_t
+  sl = sl_excl;
+  float r1 = 0.f;
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+    const float r = exp2f(sl) + m * r_next;
+    bv[i] = eta[i] * r;
+    bsum += bv[i];
+    r_next = r;
+    if (i == 0) r1 = r;
+    sl += llam[i];
+  }
+  if (coef) {  // the chunk-averaged variant: every token carries the chunk means
+    const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
+    __syncthreads();  // w_su / w_sl are free again
     if (lane == 0) {
-      w_su[warp] = su_inc;
-      w_sl[warp] = sl_inc;
+      w_su[warp] = ai;
+      w_sl[warp] = bi;
     }
     __syncthreads();
-    float su_later = 0.f, sl_later = 0.f;  // warps after this one
-    for (int w = kK1Warps - 1; w > warp; --w) {
-      su_later += w_su[w];
-      sl_later += w_sl[w];
-    }
-    float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
-    float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
-    if (lane == 31) {
-      su_excl = 0.f;
-      sl_excl = 0.f;
-    }
-    su_excl += su_later;
-    sl_excl += sl_later;
-    float su_all = 0.f, sl_all = 0.f;
+    float at = 0.f, bt = 0.f;
     for (int w = kK1Warps - 1; w >= 0; --w) {
-      su_all += w_su[w];
-      sl_all += w_sl[w];
+      at += w_su[w];
+      bt += w_sl[w];
     }
-    const float mu_next = s_mu_first[tid + 1];
-
-    // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map; the
-    // decay products L(t+1, n) are kept for walk 2, which needs the same ones
-    su = su_excl;
-    sl = sl_excl;
-    float Mseg = 1.f, Cseg = 0.f;
-    float asum = 0.f, bsum = 0.f;
-    float av[PER], bv[PER], el[PER];
-#pragma unroll
-    for (int i = PER - 1; i >= 0; --i) {
-      av[i] = eta[i] * expf(su);
-      asum += av[i];
-      const float m = i + 1 < PER ? mu[i + 1] : mu_next;
-      el[i] = expf(sl);
-      Cseg = el[i] + m * Cseg;
-      Mseg = m * Mseg;
-      su += lmu[i];
-      sl += llam[i];
-    }
-    float M = Mseg, Cc = Cseg;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float Mr = __shfl_down_sync(0xffffffffu, M, off);
-      const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
-      if (lane + off < 32) {
-        Cc = Cc + M * Cr;
-        M = M * Mr;
-      }
-    }
-    if (lane == 0) {
-      w_M[warp] = M;
-      w_C[warp] = Cc;
-    }
-    __syncthreads();
-    float r_end = 0.f;
-    for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
-    const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
-    const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
-    float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
-
-    // reverse walk 2: R_t and the weight kernel b_t
-    float r1 = 0.f;
-#pragma unroll
-    for (int i = PER - 1; i >= 0; --i) {
-      const float m = i + 1 < PER ? mu[i + 1] : mu_next;
-      const float r = el[i] + m * r_next;
-      bv[i] = eta[i] * r;
-      bsum += bv[i];
-      r_next = r;
-      if (i == 0) r1 = r;
-    }
-    if (coef) {  // the chunk-averaged variant: every token carries the chunk means
-      const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
-      __syncthreads();  // w_su / w_sl are free again
-      if (lane == 0) {
-        w_su[warp] = ai;
-        w_sl[warp] = bi;
-      }
-      __syncthreads();
-      float at = 0.f, bt = 0.f;
-      for (int w = kK1Warps - 1; w >= 0; --w) {
-        at += w_su[w];
-        bt += w_sl[w];
-      }
-      const float n = (float)(PER * kK1Threads);
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        av[i] = at / n;
-        bv[i] = bt / n;
-      }
-      __syncthreads();  // every warp has read w_su / w_sl before the next pair writes them
-    }
-    store_vec<PER>(a_out + base, av);
-    store_vec<PER>(b_out + base, bv);
-    if (tid == 0) {  // the thread holding token 1
-      const size_t plane = (size_t)BH * NC;
-      const size_t o = (size_t)bh * NC + ci;
-      scal[o] = expf(su_all);
-      scal[plane + o] = expf(sl_all);
-      scal[2 * plane + o] = mu0 * r1;
-    }
+    const float n = (float)(PER * kK1Threads);
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-      eta[i] = eta_n[i];
-      mu[i] = mu_n[i];
-      lam[i] = lam_n[i];
+      av[i] = at / n;
+      bv[i] = bt / n;
     }
+  }
+  store_vec<PER>(a_out + base, av);
+  store_vec<PER>(b_out + base, bv);
+  if (tid == 0) {  // the thread holding token 1
+    const size_t plane = (size_t)BH * NC;
+    const size_t o = (size_t)bh * NC + ci;
+    scal[o] = exp2f(su_all);
+    scal[plane + o] = exp2f(sl_all);
+    scal[2 * plane + o] = mu[0] * r1;
   }
 }
 
@@ -563,13 +535,13 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float Mseg = 1.f, Cseg = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
     float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
-    float cl = expf(sl);
-    sU[t] = expf(su);
+    float cl = exp2f(sl);
+    sU[t] = exp2f(su);
     sL[t] = cl;
     Cseg = cl + m * Cseg;
     Mseg = m * Mseg;
-    su += logf(mu_at(mu, t));
-    sl += logf(lam[t]);
+    su += log2f(mu_at(mu, t));
+    sl += log2f(lam[t]);
   }
   float M = Mseg, Cc = Cseg;
 #pragma unroll
@@ -654,33 +626,6 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
 
 }  // namespace
 
-// One resident wave at most: every block then walks several (head, chunk)
-// pairs, prefetching the next one's gates.
-template <int PER>
-cudaError_t launch_vec(const float* lr, const float* mom, const float* decay, float* a, float* b,
-                       float* scal, int BH, int T, int C, int NC, int coef, cudaStream_t st) {
-  static int wave[4][64] = {};  // [log2 PER][device]: resident blocks on the whole GPU
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const int pi = PER >= 8 ? 3 : PER >= 4 ? 2 : PER - 1;
-  int cap = (dev >= 0 && dev < 64) ? wave[pi][dev] : 0;
-  if (cap == 0) {
-    int sms = 0, per_sm = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_coeffs_vec_kernel<PER>,
-                                                      kK1Threads, 0);
-    if (e != cudaSuccess) return e;
-    cap = sms * (per_sm > 0 ? per_sm : 1);
-    if (dev >= 0 && dev < 64) wave[pi][dev] = cap;
-  }
-  const int pairs = BH * NC;
-  chunk_coeffs_vec_kernel<PER><<<pairs < cap ? pairs : cap, kK1Threads, 0, st>>>(
-      lr, mom, decay, a, b, scal, BH, T, C, NC, coef);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
                                 float* b, float* scal, int BH, int T, int C, int NC, int coef,
                                 cudaStream_t st) {
@@ -693,10 +638,10 @@ cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* 
   if (T % C == 0 && C % kK1Threads == 0 && (per == 1 || per == 2 || per == 4 || per == 8) &&
       vec_ok(lr) && vec_ok(mom) && vec_ok(decay) && vec_ok(a) && vec_ok(b)) {
     switch (per) {
-      case 1: return launch_vec<1>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
-      case 2: return launch_vec<2>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
-      case 4: return launch_vec<4>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
-      default: return launch_vec<8>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef, st);
+      case 1: chunk_coeffs_vec_kernel<1><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      case 2: chunk_coeffs_vec_kernel<2><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      case 4: chunk_coeffs_vec_kernel<4><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
+      default: chunk_coeffs_vec_kernel<8><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, a, b, scal, BH, T, C, NC, coef); break;
     }
     return cudaGetLastError();
   }

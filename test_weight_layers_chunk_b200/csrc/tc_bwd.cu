@@ -23,6 +23,7 @@
 // and D1, D2, E4, dk, dq, dW as above with hw = d_h columns instead of 2 d_h.
 #include <cuda.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include "paths.h"
@@ -1121,7 +1122,7 @@ __device__ __forceinline__ void shadow4(const float4 w, const float4 m, const fl
   *reinterpret_cast<uint2*>(pa) = make_uint2(pack2(a.x, a.y), pack2(a.z, a.w));
   *reinterpret_cast<uint2*>(pb) = make_uint2(pack2(b.x, b.y), pack2(b.z, b.w));
 }
-__global__ void __launch_bounds__(256) bwd_shadow_kernel(
+__global__ void __launch_bounds__(256, 4) bwd_shadow_kernel(  // 4 blocks (64 registers) per SM
     const float* __restrict__ W0, const float* __restrict__ M0, long long sst,
     const float* __restrict__ DW, float* __restrict__ DM, bf16* W13, bf16* W2, bf16* DW13,
     bf16* DW2, bf16* DM13, bf16* DM2, float* part, const float* __restrict__ scal, Dims d, int ci) {
@@ -1164,17 +1165,18 @@ __global__ void __launch_bounds__(256) bwd_shadow_kernel(
     __syncthreads();
   }
   if (threadIdx.x == 0)
-    for (int q = 0; q < 3; ++q) part[((size_t)q * d.BH + z) * 64 + blk] = red[q][0];
+    for (int q = 0; q < 3; ++q) part[((size_t)q * d.BH + z) * 64 + blk] = red[q][0];  // blk < 64
 }
 // chunk-scalar adjoints from the partials.
-__global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci) {
+__global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci,
+                                   int nb) {
   griddep_launch_dependents();  // the next kernel's set-up may start
   const int z = blockIdx.x * blockDim.x + threadIdx.x;
   if (z >= d.BH) return;
   const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
   for (int q = 0; q < 3; ++q) {
     float s = 0.f;
-    for (int b = 0; b < 64; ++b) s += part[((size_t)q * d.BH + z) * 64 + b];
+    for (int b = 0; b < nb; ++b) s += part[((size_t)q * d.BH + z) * 64 + b];
     sbar[q * plane + o] = s;
   }
 }
@@ -1498,6 +1500,10 @@ cudaError_t tc_bwd(const BwdArgs& A) {
 
   const size_t per_chunk = (size_t)BH * 2 * d.S;
   const Dims dd = d;
+  // blocks per head of the shadow kernel: one resident wave (4 blocks per SM)
+  // over all heads, at most 64 (the partial-sum slots per head); fixed for a
+  // given device, so the partial sums keep their order from call to call
+  const int shadow_nb = std::max(1, std::min(64, 4 * num_sms() / BH));
   for (int ci = NC - 1; ci >= 0; --ci) {
     const int t0 = ci * C;
     const int cl = T - t0 < C ? T - t0 : C;  // tokens of this chunk
@@ -1529,10 +1535,10 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     if (e != cudaSuccess) return e;
     {
       E2TTT_TRACE("tcb_shadow", st);
-      bwd_shadow_kernel<<<dim3(64, BH), 256, 0, st>>>(W0, M0, 2 * d.S, A.dW0, A.dM0, B.W13, B.W2,
-                                                       B.DW13, B.DW2, B.DM13, B.DM2, B.spart,
-                                                       B.scal, dd, ci);
-      bwd_scalars_kernel<<<(BH + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci);
+      bwd_shadow_kernel<<<dim3(shadow_nb, BH), 256, 0, st>>>(W0, M0, 2 * d.S, A.dW0, A.dM0, B.W13,
+                                                              B.W2, B.DW13, B.DW2, B.DM13, B.DM2,
+                                                              B.spart, B.scal, dd, ci);
+      bwd_scalars_kernel<<<(BH + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci, shadow_nb);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
