@@ -517,6 +517,20 @@ def measure_extras(E, torch, dev, stream, args):
 
 
 # ----------------------------------------------------------------- our path
+def run_k1_only(args):
+    """K1 alone at 2^26 token-heads (the `k1_2e26` measurement of the main
+    line) as its own JSON line: --warmup launches, then --steps timed ones.
+    For profiling K1 by itself; not the benchmark's contract line."""
+    import torch
+    import test_weight_layers_chunk_b200 as E
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    r = measure_k1_large(E, torch, dev, stream, reps=args.steps)
+    print(json.dumps({"metric": "K1 token-heads/s at 2^26", "value": r["token_heads"] / (r["us_per_launch"] / 1e6),
+                      "unit": "token-heads/s", "k1_2e26": r}))
+
+
 def run_ours(args, w):
     import torch
     import test_weight_layers_chunk_b200 as E
@@ -784,7 +798,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, choices=[w.name for w in gen.WORKLOADS],
                     help="default: layer_1p3b_2k (fwd) or train_1p3b_2k (train)")
-    ap.add_argument("--mode", choices=["fwd", "train"], default="fwd")
+    ap.add_argument("--mode", choices=["fwd", "train", "k1"], default="fwd",
+                    help="k1: only K1 at 2^26 token-heads (for profiling it alone)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -798,7 +813,9 @@ def main():
     if args.workload is None:
         args.workload = "train_1p3b_2k" if args.mode == "train" else "layer_1p3b_2k"
     w = gen.BY_NAME[args.workload]
-    if args.impl == "reference":
+    if args.mode == "k1":
+        run_k1_only(args)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)
