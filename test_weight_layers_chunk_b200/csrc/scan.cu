@@ -14,10 +14,14 @@
 //   U(1,n) = exp(SU_0), L(1,n) = exp(SL_0), c = mu_1 R_1        (chunk scalars)
 // No prefix sum is ever subtracted from another, so mu = 0 or lam = 0 (log = -inf)
 // gives exact zeros instead of NaN. The logarithms and exponentials are taken in
-// base 2 (log2f, exp2f: the identities above hold in any base, and the base-2
-// functions cost fewer instructions at the same documented accuracy, 1 and 2
-// ulp), which matters where the scan is bound by its arithmetic rather than its
-// 20 bytes per token.
+// base 2 (log2f, exp2f: the identities above hold in any base, at the same
+// documented accuracy, 1 and 2 ulp, for fewer instructions). A thread's segment
+// of consecutive tokens enters the suffix log-sums through the log of its gate
+// product (one log per gate stream and segment), and inside the segment
+// U(t+1, n) and L(t+1, n) are the exponentials of the exclusive log-sums times
+// the segment's later gates: products of at most a segment's gates, no
+// division. Per token that leaves a few multiplications, so the scan is bound
+// by its 20 bytes per token rather than by its arithmetic.
 //
 // Layout: one 128-thread block per (head, chunk) for chunks up to 8192 tokens
 // (thread i owns a contiguous segment of ceil(n/128) tokens; segment results are
@@ -60,11 +64,12 @@ struct LogSums {
 
 __device__ __forceinline__ LogSums chunk_log_sums(const float* mu, const float* lam, int s0, int s1,
                                                   int lane) {
-  float su = 0.f, sl = 0.f;
+  float pu = 1.f, pl = 1.f;  // the segment's gate products, one log each
   for (int t = s1 - 1; t >= s0; --t) {
-    su += log2f(mu_at(mu, t));
-    sl += log2f(lam[t]);
+    pu *= mu_at(mu, t);
+    pl *= lam[t];
   }
+  const float su = log2f(pu), sl = log2f(pl);
   float su_inc = warp_suffix_sum(su, lane);
   float sl_inc = warp_suffix_sum(sl, lane);
   LogSums r;
@@ -96,19 +101,22 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
 
   LogSums ls = chunk_log_sums(mu, lam, s0, s1, lane);
 
-  // Reverse walk 1: momentum kernel a_t and the segment's ratio-sum map.
-  float su = ls.su_excl, sl = ls.sl_excl;
+  // Reverse walk 1: momentum kernel a_t and the segment's ratio-sum map. The
+  // products U(t+1, n), L(t+1, n) start from the exponential of the exclusive
+  // log-sum and pick up one gate per token inside the segment.
+  const float L_excl = exp2f(ls.sl_excl);
+  float U = exp2f(ls.su_excl), L = L_excl;
   float Mseg = 1.f, Cseg = 0.f;
   float asum = 0.f, bsum = 0.f;  // segment sums (chunk means for coef = 1)
   for (int t = s1 - 1; t >= s0; --t) {
-    const float at = eta[t] * exp2f(su);
+    const float at = eta[t] * U;
     a_out[base + t] = at;
     asum += at;
     float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
-    Cseg = exp2f(sl) + m * Cseg;
+    Cseg = L + m * Cseg;
     Mseg = m * Mseg;
-    su += log2f(mu_at(mu, t));
-    sl += log2f(lam[t]);
+    U *= mu_at(mu, t);
+    L *= lam[t];
   }
   float M = Mseg, Cc = Cseg;
 #pragma unroll
@@ -124,17 +132,17 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
   if (lane == 31) r_next = 0.f;
 
   // Reverse walk 2: R_t and the weight kernel b_t.
-  sl = ls.sl_excl;
+  L = L_excl;
   float r1 = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
     float m = (t + 1 < n) ? mu_at(mu, t + 1) : 0.f;
-    float r = exp2f(sl) + m * r_next;
+    float r = L + m * r_next;
     const float bt = eta[t] * r;
     b_out[base + t] = bt;
     bsum += bt;
     r_next = r;
     if (t == 0) r1 = r;
-    sl += log2f(lam[t]);
+    L *= lam[t];
   }
   if (coef) {  // the chunk-averaged variant: every token carries the chunk means
     const float am = __shfl_sync(0xffffffffu, warp_suffix_sum(asum, lane), 0) / (float)n;
@@ -154,14 +162,15 @@ chunk_coeffs_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
 }
 
 // Block version of chunk_coeffs_kernel: one 128-thread block per (head, chunk),
-// thread i owning a contiguous segment of ceil(n/128) tokens. The gates and their
-// logs are staged in shared memory (each log computed once); the segment
+// thread i owning a contiguous segment of ceil(n/128) tokens. The gates are
+// staged in shared memory; each segment's log-sums are the logs of its gate
+// products (one log per gate stream and segment); the segment
 // log-sums and the segment maps of the ratio-sum recurrence are combined with
 // warp shuffles and then across the four warps, suffix-wise and by additions and
 // products only (never by subtracting a prefix), as in the warp version.
 constexpr int kK1Threads = 128;
 constexpr int kK1Warps = kK1Threads / 32;
-constexpr int kK1MaxC = 8192;  // 4 C floats of shared memory
+constexpr int kK1MaxC = 8192;  // 3 C floats of shared memory
 
 __global__ void __launch_bounds__(kK1Threads)
 chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
@@ -171,8 +180,7 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   extern __shared__ float k1s[];
   float* s_eta = k1s;
   float* s_mu = k1s + C;
-  float* s_lmu = k1s + 2 * C;
-  float* s_llam = k1s + 3 * C;
+  float* s_lam = k1s + 2 * C;
   __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
@@ -183,19 +191,19 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
     const float mu = mom ? mom[base + t] : 0.f;  // NULL: no-momentum mode
     s_eta[t] = lr[base + t];
     s_mu[t] = mu;
-    s_lmu[t] = log2f(mu);
-    s_llam[t] = log2f(decay[base + t]);
+    s_lam[t] = decay[base + t];
   }
   __syncthreads();
   const int per = (n + kK1Threads - 1) / kK1Threads;
   const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
 
   // suffix log-sums: exclusive (tokens after this segment) and chunk totals
-  float su = 0.f, sl = 0.f;
+  float pu = 1.f, pl = 1.f;  // the segment's gate products
   for (int t = s1 - 1; t >= s0; --t) {
-    su += s_lmu[t];
-    sl += s_llam[t];
+    pu *= s_mu[t];
+    pl *= s_lam[t];
   }
+  const float su = log2f(pu), sl = log2f(pl);
   const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
   if (lane == 0) {
     w_su[warp] = su_inc;
@@ -221,20 +229,22 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
     sl_all += w_sl[w];
   }
 
-  // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map
-  su = su_excl;
-  sl = sl_excl;
+  // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map; the
+  // products U(t+1, n), L(t+1, n) start from the exponentials of the exclusive
+  // log-sums and pick up one gate per token inside the segment
+  const float L_excl = exp2f(sl_excl);
+  float U = exp2f(su_excl), L = L_excl;
   float Mseg = 1.f, Cseg = 0.f;
   float asum = 0.f, bsum = 0.f;  // segment sums (chunk means for coef = 1)
   for (int t = s1 - 1; t >= s0; --t) {
-    const float at = s_eta[t] * exp2f(su);
+    const float at = s_eta[t] * U;
     a_out[base + t] = at;
     asum += at;
     const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
-    Cseg = exp2f(sl) + m * Cseg;
+    Cseg = L + m * Cseg;
     Mseg = m * Mseg;
-    su += s_lmu[t];
-    sl += s_llam[t];
+    U *= s_mu[t];
+    L *= s_lam[t];
   }
   // inclusive suffix composition of the maps within the warp, then across warps
   float M = Mseg, Cc = Cseg;
@@ -259,17 +269,17 @@ chunk_coeffs_block_kernel(const float* __restrict__ lr, const float* __restrict_
   float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
 
   // reverse walk 2: R_t and the weight kernel b_t
-  sl = sl_excl;
+  L = L_excl;
   float r1 = 0.f;
   for (int t = s1 - 1; t >= s0; --t) {
     const float m = (t + 1 < n) ? s_mu[t + 1] : 0.f;
-    const float r = exp2f(sl) + m * r_next;
+    const float r = L + m * r_next;
     const float bt = s_eta[t] * r;
     b_out[base + t] = bt;
     bsum += bt;
     r_next = r;
     if (t == 0) r1 = r;
-    sl += s_llam[t];
+    L *= s_lam[t];
   }
   if (coef) {  // the chunk-averaged variant: every token carries the chunk means
     const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
@@ -355,22 +365,17 @@ chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ 
     for (int i = 0; i < PER; ++i) mu[i] = 0.f;
   }
   load_vec<PER>(decay + base, lam);
-  float lmu[PER], llam[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    lmu[i] = log2f(mu[i]);
-    llam[i] = log2f(lam[i]);
-  }
   s_mu_first[tid] = mu[0];
   if (tid == 0) s_mu_first[kK1Threads] = 0.f;  // no token after the chunk's last
 
   // suffix log-sums: exclusive (tokens after this segment) and chunk totals
-  float su = 0.f, sl = 0.f;
+  float pu = 1.f, pl = 1.f;  // the segment's gate products
 #pragma unroll
   for (int i = PER - 1; i >= 0; --i) {
-    su += lmu[i];
-    sl += llam[i];
+    pu *= mu[i];
+    pl *= lam[i];
   }
+  const float su = log2f(pu), sl = log2f(pl);
   const float su_inc = warp_suffix_sum(su, lane), sl_inc = warp_suffix_sum(sl, lane);
   if (lane == 0) {
     w_su[warp] = su_inc;
@@ -398,20 +403,20 @@ chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ 
   const float mu_next = s_mu_first[tid + 1];
 
   // reverse walk 1: momentum kernel a_t and the segment's ratio-sum map
-  su = su_excl;
-  sl = sl_excl;
+  const float L_excl = exp2f(sl_excl);
+  float U = exp2f(su_excl), L = L_excl;
   float Mseg = 1.f, Cseg = 0.f;
   float asum = 0.f, bsum = 0.f;
   float av[PER], bv[PER];
 #pragma unroll
   for (int i = PER - 1; i >= 0; --i) {
-    av[i] = eta[i] * exp2f(su);
+    av[i] = eta[i] * U;
     asum += av[i];
     const float m = i + 1 < PER ? mu[i + 1] : mu_next;
-    Cseg = exp2f(sl) + m * Cseg;
+    Cseg = L + m * Cseg;
     Mseg = m * Mseg;
-    su += lmu[i];
-    sl += llam[i];
+    U *= mu[i];
+    L *= lam[i];
   }
   float M = Mseg, Cc = Cseg;
 #pragma unroll
@@ -435,17 +440,17 @@ chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ 
   float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
 
   // reverse walk 2: R_t and the weight kernel b_t
-  sl = sl_excl;
+  L = L_excl;
   float r1 = 0.f;
 #pragma unroll
   for (int i = PER - 1; i >= 0; --i) {
     const float m = i + 1 < PER ? mu[i + 1] : mu_next;
-    const float r = exp2f(sl) + m * r_next;
+    const float r = L + m * r_next;
     bv[i] = eta[i] * r;
     bsum += bv[i];
     r_next = r;
     if (i == 0) r1 = r;
-    sl += llam[i];
+    L *= lam[i];
   }
   if (coef) {  // the chunk-averaged variant: every token carries the chunk means
     const float ai = warp_suffix_sum(asum, lane), bi = warp_suffix_sum(bsum, lane);
@@ -646,7 +651,7 @@ cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* 
     return cudaGetLastError();
   }
   if (C <= kK1MaxC) {
-    const size_t smem = (size_t)4 * C * sizeof(float);
+    const size_t smem = (size_t)3 * C * sizeof(float);
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(chunk_coeffs_block_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
