@@ -1167,36 +1167,53 @@ __global__ void __launch_bounds__(256, 4) bwd_shadow_kernel(  // 4 blocks (64 re
   if (threadIdx.x == 0)
     for (int q = 0; q < 3; ++q) part[((size_t)q * d.BH + z) * 64 + blk] = red[q][0];  // blk < 64
 }
-// chunk-scalar adjoints from the partials.
+// Sum over the 32 lanes of a warp in a fixed order (butterfly), every lane
+// receiving the total.
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+// chunk-scalar adjoints from the partials: one warp per (scalar, head), the
+// lanes reading consecutive partials.
 __global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci,
                                    int nb) {
   griddep_launch_dependents();  // the next kernel's set-up may start
-  const int z = blockIdx.x * blockDim.x + threadIdx.x;
-  if (z >= d.BH) return;
-  const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
-  for (int q = 0; q < 3; ++q) {
-    float s = 0.f;
-    for (int b = 0; b < nb; ++b) s += part[((size_t)q * d.BH + z) * 64 + b];
+  const int w = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+  if (w >= 3 * d.BH) return;  // warp-uniform
+  const int q = w / d.BH, z = w - q * d.BH;
+  const float* pp = part + ((size_t)q * d.BH + z) * 64;
+  float s = 0.f;
+  for (int b = lane; b < nb; b += 32) s += pp[b];
+  s = warp_sum(s);
+  if (lane == 0) {
+    const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
     sbar[q * plane + o] = s;
   }
 }
-// abar_t, bbar_t = -(sum of the partial dot products), fixed order.
+// abar_t, bbar_t = -(sum of the partial dot products), fixed order: one warp
+// per row, the lanes reading consecutive partials.
 __global__ void bwd_rows_kernel(const float* part, float* abar, float* bbar, Dims d, int t0, int clen,
                                 int NG) {
   griddep_launch_dependents();  // the next kernel's set-up may start
-  const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= (long long)d.BH * d.C) return;
+  const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= (long long)d.BH * d.C) return;  // warp-uniform
   const int z = (int)(r / d.C), t = (int)(r % d.C);
-  if (t >= clen) return;  // padding of a shorter last chunk
+  if (t >= clen) return;  // padding of a shorter last chunk (warp-uniform)
   const float* pa = part + (size_t)r * NG;
   const float* pb = pa + (size_t)d.BH * d.C * NG;
   float sa = 0.f, sb = 0.f;
-  for (int g = 0; g < NG; ++g) {
+  for (int g = lane; g < NG; g += 32) {
     sa += pa[g];
     sb += pb[g];
   }
-  abar[(size_t)z * d.T + t0 + t] = -sa;
-  bbar[(size_t)z * d.T + t0 + t] = -sb;
+  sa = warp_sum(sa);
+  sb = warp_sum(sb);
+  if (lane == 0) {
+    abar[(size_t)z * d.T + t0 + t] = -sa;
+    bbar[(size_t)z * d.T + t0 + t] = -sb;
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -1538,7 +1555,8 @@ cudaError_t tc_bwd(const BwdArgs& A) {
       bwd_shadow_kernel<<<dim3(shadow_nb, BH), 256, 0, st>>>(W0, M0, 2 * d.S, A.dW0, A.dM0, B.W13,
                                                               B.W2, B.DW13, B.DW2, B.DM13, B.DM2,
                                                               B.spart, B.scal, dd, ci);
-      bwd_scalars_kernel<<<(BH + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci, shadow_nb);
+      bwd_scalars_kernel<<<(3 * BH * 32 + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci,
+                                                                  shadow_nb);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
@@ -1563,8 +1581,8 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     {
       E2TTT_TRACE("tcb_rows", st);
       const long long rows = (long long)BH * C;
-      bwd_rows_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(B.part, B.abar, B.bbar, dd, t0,
-                                                                         cl, p.NG);
+      bwd_rows_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(B.part, B.abar, B.bbar, dd,
+                                                                              t0, cl, p.NG);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
