@@ -150,6 +150,8 @@ def kernel_work(w, has_m0: bool) -> dict:
                           out[g1][2] + out["tc_g2_y_out_e"][2] - u_query)
     out["tc_shadow_init"] = (0.0, 0.0, 6.0 * S * BH)
     out["tc_scale_keys"] = (0.0, 0.0, 6.0 * T * dk * BH)
+    # the two in one launch (the scaled keys only for the MLP fast weights)
+    out["tc_prep"] = (0.0, 0.0, out["tc_shadow_init"][2] + (out["tc_scale_keys"][2] if w.kind != gen.LINEAR else 0.0))
     return out
 
 

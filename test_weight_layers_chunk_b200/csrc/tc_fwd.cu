@@ -1494,8 +1494,9 @@ fwd_persistent(const __grid_constant__ MegaJob J, const __grid_constant__ FwdP p
 
 // ---------------------------------------------------------------- prep kernel
 // bf16 operand copies of the caller's W0 (W1/W3 rows interleaved in 128-row blocks).
-__global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* __restrict__ W0) {
-  griddep_launch_dependents();  // the next kernel's set-up may start
+// Block `bid` of `nblk` blocks (256 threads) of the bf16 copy of W0.
+__device__ __forceinline__ void shadow_init_blocks(const FwdP& p, const float* __restrict__ W0, int bid,
+                                                   int nblk) {
   // One warp per state row, two rows per pass with both rows' loads issued first:
   // rows [0, 2 d_h) of a head are W1 then W3 (d_k wide; GELU MLP: [0, d_h) are
   // W1), the next d_v rows are W2 (d_h wide); the linear state is d_v rows of d_k.
@@ -1504,7 +1505,7 @@ __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* _
   const int r13 = d.kind == 1 ? 2 * d.d_h : d.kind == 2 ? d.d_h : d.d_v;
   const int rows = d.kind != 0 ? r13 + d.d_v : r13;
   const long long total = (long long)d.BH * rows;
-  const long long nwarps = (long long)gridDim.x * (blockDim.x / 32);
+  const long long nwarps = (long long)nblk * (blockDim.x / 32);
   auto row_of = [&](long long gr, const float*& src, bf16*& dst, int& len) {
     const int z = (int)(gr / rows), r = (int)(gr - (long long)z * rows);
     if (r < r13) {
@@ -1518,7 +1519,7 @@ __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* _
       len = d.d_h;
     }
   };
-  for (long long gr = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); gr < total;
+  for (long long gr = (long long)bid * (blockDim.x / 32) + (threadIdx.x >> 5); gr < total;
        gr += 2 * nwarps) {
     const float *s0, *s1 = nullptr;
     bf16 *d0, *d1 = nullptr;
@@ -1551,13 +1552,14 @@ __global__ void __launch_bounds__(256) shadow_init_kernel(FwdP p, const float* _
 // Each thread moves kScaleVec 8-element groups per pass (all loads issued before
 // the stores), consecutive threads consecutive groups.
 constexpr int kScaleVec = 4;
-__global__ void scale_keys_kernel(const bf16* __restrict__ k, const float* __restrict__ ca,
-                                  const float* __restrict__ cb, bf16* __restrict__ Ka,
-                                  bf16* __restrict__ Kb, long long tokens, int d_k) {
-  griddep_launch_dependents();  // the next kernel's set-up may start
+// Block `bid` of `nblk` blocks (256 threads) of the key scaling.
+__device__ __forceinline__ void scale_keys_blocks(const bf16* __restrict__ k, const float* __restrict__ ca,
+                                                  const float* __restrict__ cb, bf16* __restrict__ Ka,
+                                                  bf16* __restrict__ Kb, long long tokens, int d_k,
+                                                  int bid, int nblk) {
   const long long n8 = tokens * d_k / 8;
-  const long long step = (long long)gridDim.x * blockDim.x * kScaleVec;
-  for (long long base = (long long)blockIdx.x * blockDim.x * kScaleVec + threadIdx.x; base < n8;
+  const long long step = (long long)nblk * blockDim.x * kScaleVec;
+  for (long long base = (long long)bid * blockDim.x * kScaleVec + threadIdx.x; base < n8;
        base += step) {
     uint4 u[kScaleVec];
     float a[kScaleVec], b[kScaleVec];
@@ -1586,6 +1588,25 @@ __global__ void scale_keys_kernel(const bf16* __restrict__ k, const float* __res
       if (Ka) reinterpret_cast<uint4*>(Ka)[e8] = make_uint4(oa[0], oa[1], oa[2], oa[3]);  // NULL: no momentum
       reinterpret_cast<uint4*>(Kb)[e8] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
     }
+  }
+}
+
+// The two prep jobs of a call in one launch: of every three blocks two copy W0
+// to bf16 and one scales the keys (k NULL: the copy alone), so both streams of
+// HBM traffic run side by side and the step has one prep launch, not two.
+__global__ void __launch_bounds__(256) prep_kernel(FwdP p, const float* __restrict__ W0,
+                                                   const bf16* __restrict__ k,
+                                                   const float* __restrict__ ca,
+                                                   const float* __restrict__ cb, bf16* Ka, bf16* Kb,
+                                                   long long tokens, int d_k) {
+  griddep_launch_dependents();  // the next kernel's set-up may start
+  const int b = blockIdx.x, n = gridDim.x;
+  if (k == nullptr) {
+    shadow_init_blocks(p, W0, b, n);
+  } else if (b % 3 == 2) {
+    scale_keys_blocks(k, ca, cb, Ka, Kb, tokens, d_k, b / 3, n / 3);
+  } else {
+    shadow_init_blocks(p, W0, b - b / 3, n - n / 3);
   }
 }
 
@@ -1805,15 +1826,11 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   cudaError_t e = save_initial_state(d, W0, M0, saved, st);
   if (e != cudaSuccess) return e;
   {
-    E2TTT_TRACE("tc_shadow_init", st);
-    shadow_init_kernel<<<8 * num_sms(), 256, 0, st>>>(p, W0);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  if (d.kind != 0) {
-    E2TTT_TRACE("tc_scale_keys", st);
-    scale_keys_kernel<<<4 * num_sms(), 256, 0, st>>>(k, ca, cb, d.nomom ? nullptr : s.Ka, s.Kb,
-                                                     (long long)BH * T, dk);
+    // the bf16 copy of W0 and (MLP fast weights) the scaled keys: 12 blocks per
+    // SM, a multiple of 3 (8 copy the state, 4 scale keys)
+    E2TTT_TRACE("tc_prep", st);
+    prep_kernel<<<12 * num_sms(), 256, 0, st>>>(p, W0, d.kind != 0 ? k : nullptr, ca, cb,
+                                               d.nomom ? nullptr : s.Ka, s.Kb, (long long)BH * T, dk);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

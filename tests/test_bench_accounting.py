@@ -94,7 +94,8 @@ def test_algorithmic_bytes_are_the_calls_compulsory_traffic(bench):
                                              "tc_g4_aggregate_state"))
     gates = 12 * w.B * w.H * w.T
     assert per_call == bench.algorithmic_bytes(w) - gates
-    assert work["tc_shadow_init"][1] == work["tc_scale_keys"][1] == 0.0
+    assert work["tc_shadow_init"][1] == work["tc_scale_keys"][1] == work["tc_prep"][1] == 0.0
+    assert work["tc_prep"][2] == work["tc_shadow_init"][2] + work["tc_scale_keys"][2]
     # implementation bytes never undercount the algorithmic ones
     for n, (f, alg, impl) in work.items():
         assert impl >= alg, n
