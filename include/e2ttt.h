@@ -95,9 +95,20 @@ typedef enum { E2TTT_COEF_PER_TOKEN = 0, E2TTT_COEF_CHUNK_MEAN = 1 } e2ttt_coef;
  * dmom and dM0 must be NULL in the backward. The forward moves only W through
  * HBM (about half the state traffic). */
 typedef enum { E2TTT_MOMENTUM = 0, E2TTT_NO_MOMENTUM = 1 } e2ttt_momentum;
+/* GEMM precision. AUTO: bf16 activations of tensor-core shapes (C, d_k, d_v,
+ * d_h multiples of 128, 16-byte aligned pointers) run on the tcgen05 tensor
+ * cores with bf16 operands (activations and bf16 copies of the chunk-start
+ * weights) and fp32 accumulation; everything else on the fp32 CUDA-core
+ * kernels. FP32: always the fp32 CUDA-core kernels (the bf16 activations are
+ * widened, the weights stay fp32), forward and backward: for problems whose
+ * gradients are sensitive to rounding the weights to bf16 (a GELU MLP fast
+ * weight with a non-zero M0 and upstream state gradients moves its exact
+ * gradients by 5-15 % under that rounding). Slower. */
+typedef enum { E2TTT_GEMM_AUTO = 0, E2TTT_GEMM_FP32 = 1 } e2ttt_gemm;
 
-/* Problem description. kind/act/loss/coef/momentum hold e2ttt_fast_kind /
- * e2ttt_dtype / e2ttt_loss / e2ttt_coef / e2ttt_momentum values. d_h is ignored
+/* Problem description. kind/act/loss/coef/momentum/gemm hold e2ttt_fast_kind /
+ * e2ttt_dtype / e2ttt_loss / e2ttt_coef / e2ttt_momentum / e2ttt_gemm values
+ * (a zero-initialised gemm field is E2TTT_GEMM_AUTO). d_h is ignored
  * (may be 0) for E2TTT_LINEAR.
  * Limits: all sizes >= 1; B*H <= 65535; B*H*T*max(d_k, d_v, 2 d_h) < 2^31
  * (d_h counted for the MLPs only); 1 <= C <= 1024. */
@@ -109,6 +120,7 @@ typedef struct {
   int loss;
   int coef;
   int momentum;
+  int gemm;
 } e2ttt_shape;
 
 /* Fast-weight state size S per (b, h): d_v*d_k (linear), 2*d_h*d_k + d_v*d_h
@@ -124,8 +136,8 @@ size_t e2ttt_workspace_bytes(const e2ttt_shape* shape, int for_bwd);
 int e2ttt_num_chunks(const e2ttt_shape* shape);
 
 /* 1 if e2ttt_chunk_scan_fwd runs `shape` on the tcgen05 tensor cores (given
- * 16-byte aligned pointers), 0 if on the fp32 CUDA-core kernels, -1 if the
- * shape is invalid. */
+ * 16-byte aligned pointers), 0 if on the fp32 CUDA-core kernels (always 0 with
+ * gemm = E2TTT_GEMM_FP32), -1 if the shape is invalid. */
 int e2ttt_fwd_uses_tensor_cores(const e2ttt_shape* shape);
 
 /* The two scalar kernels of every chunk (atlas.scime.ai summary, "Approach":

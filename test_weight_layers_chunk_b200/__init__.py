@@ -30,12 +30,14 @@ F32, BF16 = 0, 1
 LOSS_MSE, LOSS_NEG_DOT = 0, 1
 COEF_PER_TOKEN, COEF_CHUNK_MEAN = 0, 1
 MOMENTUM, NO_MOMENTUM = 0, 1
+GEMM_AUTO, GEMM_FP32 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 
 
 class e2ttt_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss", "coef", "momentum")]
+                ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss", "coef", "momentum",
+                 "gemm")]
 
 
 class E2TTTError(RuntimeError):
@@ -82,8 +84,8 @@ def header_functions() -> list[str]:
 
 
 def make_shape(B, H, T, C, d_k, d_v, d_h=0, kind=SWIGLU, act=BF16, loss=LOSS_MSE,
-               coef=COEF_PER_TOKEN, momentum=MOMENTUM) -> e2ttt_shape:
-    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef, momentum)
+               coef=COEF_PER_TOKEN, momentum=MOMENTUM, gemm=GEMM_AUTO) -> e2ttt_shape:
+    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef, momentum, gemm)
 
 
 def _ptr(x):
@@ -211,11 +213,11 @@ def e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved_states, dout, dW_
 
 
 # ---------------------------------------------------------------- conveniences
-def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN, momentum=MOMENTUM):
+def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN, momentum=MOMENTUM, gemm=GEMM_AUTO):
     import torch
     B, H, T, d_k = q.shape
     act = BF16 if q.dtype == torch.bfloat16 else F32
-    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef, momentum)
+    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef, momentum, gemm)
 
 
 def workspace(shape, for_bwd=False, device="cuda"):
@@ -228,12 +230,12 @@ def workspace(shape, for_bwd=False, device="cuda"):
 
 def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGLU,
                    loss=LOSS_MSE, coef=COEF_PER_TOKEN, momentum=MOMENTUM, save_states=False,
-                   ws=None, stream=None):
+                   ws=None, stream=None, gemm=GEMM_AUTO):
     """Allocate out / W_end / M_end (and saved_states) and run the forward.
     Returns (out, W_end, M_end, saved_states or None); M_end is None without
     momentum (momentum=NO_MOMENTUM: pass mom=None, M0=None)."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum, gemm)
     nc = e2ttt_num_chunks(shape)
     out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     W_end = torch.empty_like(W0)
@@ -249,11 +251,11 @@ def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGL
 
 def chunk_scan_bwd(q, k, v, lr, mom, decay, saved_states, dout, dW_end=None, dM_end=None, *, C,
                    d_h=0, kind=SWIGLU, loss=LOSS_MSE, coef=COEF_PER_TOKEN, momentum=MOMENTUM,
-                   ws=None, stream=None):
+                   ws=None, stream=None, gemm=GEMM_AUTO):
     """Allocate the gradients and run the backward. Returns a dict (dmom and dM0
     are None without momentum)."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum, gemm)
     nomom = momentum == NO_MOMENTUM
     g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
              dlr=torch.empty_like(lr), dmom=None if nomom else torch.empty_like(mom),

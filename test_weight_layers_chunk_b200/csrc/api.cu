@@ -48,6 +48,7 @@ bool shape_ok(const e2ttt_shape* s, std::string* why) {
   if (s->loss != E2TTT_LOSS_MSE && s->loss != E2TTT_LOSS_NEG_DOT) { *why = "unknown loss"; return false; }
   if (s->coef != E2TTT_COEF_PER_TOKEN && s->coef != E2TTT_COEF_CHUNK_MEAN) { *why = "unknown coef"; return false; }
   if (s->momentum != E2TTT_MOMENTUM && s->momentum != E2TTT_NO_MOMENTUM) { *why = "unknown momentum mode"; return false; }
+  if (s->gemm != E2TTT_GEMM_AUTO && s->gemm != E2TTT_GEMM_FP32) { *why = "unknown gemm precision"; return false; }
   if (s->kind != E2TTT_LINEAR && s->d_h < 1) { *why = "SwiGLU and the GELU MLP need d_h >= 1"; return false; }
   if (s->C > 1024) { *why = "chunk size C must be <= 1024"; return false; }
   long long BH = (long long)s->B * s->H;
@@ -72,6 +73,7 @@ Dims make_dims(const e2ttt_shape* s) {
   d.loss = s->loss;
   d.coef = s->coef;
   d.nomom = s->momentum == E2TTT_NO_MOMENTUM;
+  d.fp32_gemm = s->gemm == E2TTT_GEMM_FP32;
   d.S = s->kind == E2TTT_LINEAR     ? (long long)s->d_v * s->d_k
         : s->kind == E2TTT_GELU_MLP ? (long long)s->d_h * s->d_k + (long long)s->d_v * s->d_h
                                     : 2LL * s->d_h * s->d_k + (long long)s->d_v * s->d_h;

@@ -39,6 +39,7 @@ struct Dims {
   int kind, loss;
   int coef;    // 0: per-token kernels, 1: chunk means (the chunk-averaged variant)
   int nomom;   // 1: no momentum (mu = 0, no M state)
+  int fp32_gemm;  // 1: the fp32 CUDA-core kernels even where the tensor cores apply
   long long S; // state elements per head
 };
 

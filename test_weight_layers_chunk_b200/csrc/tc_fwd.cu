@@ -1795,7 +1795,7 @@ constexpr unsigned long long kStallWaitNs = 1000000ull;
 void arm_forward_stall(bool on) { g_stall_next.store(on ? 1 : 0); }
 
 bool tc_fwd_supported(const Dims& d, bool bf16_act) {
-  if (!bf16_act) return false;
+  if (!bf16_act || d.fp32_gemm) return false;
   if (d.C % 128 != 0) return false;  // a shorter last chunk runs padded to C tokens
   if (d.d_k % 128 != 0 || d.d_v % 128 != 0) return false;
   if (d.kind != 0 && d.d_h % 128 != 0) return false;

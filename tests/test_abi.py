@@ -137,6 +137,25 @@ def test_gelu_mlp_state_size(E):
     assert E.e2ttt_workspace_bytes(g, 0) > 0 and E.e2ttt_workspace_bytes(g, 1) > 0
 
 
+def test_gemm_precision_field(E):
+    """The shape's gemm field: GEMM_AUTO (zero) picks the tensor cores for a
+    tensor-core shape, GEMM_FP32 always the fp32 CUDA-core kernels (with their
+    smaller workspace), other values are rejected on the host."""
+    import ctypes
+    assert [n for n, _ in E.e2ttt_shape._fields_][-1] == "gemm"
+    assert ctypes.sizeof(E.e2ttt_shape) == 13 * ctypes.sizeof(ctypes.c_int)
+    auto = E.make_shape(1, 2, 512, 128, 128, 128, 256, E.GELU_MLP, E.BF16)
+    fp32 = E.make_shape(1, 2, 512, 128, 128, 128, 256, E.GELU_MLP, E.BF16, gemm=E.GEMM_FP32)
+    assert auto.gemm == E.GEMM_AUTO == 0
+    assert E.e2ttt_fwd_uses_tensor_cores(auto) in (0, 1)  # 1 where a GPU driver is present
+    assert E.e2ttt_fwd_uses_tensor_cores(fp32) == 0
+    for fb in (0, 1):
+        assert 0 < E.e2ttt_workspace_bytes(fp32, fb)
+    bad = E.make_shape(1, 2, 512, 128, 128, 128, 256, E.GELU_MLP, E.BF16, gemm=2)
+    assert E.e2ttt_fwd_uses_tensor_cores(bad) == -1
+    assert E.e2ttt_workspace_bytes(bad, 0) == 0
+
+
 def test_noalloc_status_without_a_device(E):
     """The no-allocation status readout needs a current device: with none (this
     CPU-only host) it returns E2TTT_ERR_CUDA with a message, never crashes."""

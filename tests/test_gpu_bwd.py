@@ -199,27 +199,36 @@ def test_bwd_gelu_bf16_small(E):
     check(gpu, ref, 2e-2, label="gelu_bf16_small end to end")
 
 
-def test_bwd_gelu_ill_conditioned_cuda_core(E):
-    """GELU MLP, bf16 activations, M0 != 0 and upstream state gradients: the exact
-    gradients move by 0.05-0.1 when the chunk-start weights are rounded to bf16,
-    so this case runs the fp32 CUDA-core backward (an unaligned view of dout
-    routes it there) against the oracle's adjoint at the GPU's saved states."""
+def test_bwd_gelu_ill_conditioned_fp32_gemms(E):
+    """GELU MLP, bf16 activations, M0 != 0 and upstream state gradients: rounding
+    the chunk-start weights to bf16 moves the exact gradients by 3-15 % (pinned
+    on the CPU by test_gelu_backward_conditioning_under_bf16_weights), so no
+    path with bf16 weight operands meets 2e-2 here. With gemm = GEMM_FP32 the
+    forward and the backward run the fp32 CUDA-core kernels; compared end to end
+    with the oracle from the inputs alone."""
     import torch
     w = gen.Workload("bgi", gen.GELU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform", 0.999,
                      seed=49, lr_lo=0.002, lr_hi=0.02)
     x = gen.generate(w, m0_scale=0.5)
     dW, dM = gen.upstream_state_grads(w, seed=8, scale=0.1)
     d = device_inputs(w, x)
-    _, _, _, saved = run_fwd(E, w, d, save=True)
-    buf = torch.empty(d["dout"].numel() + 1, dtype=torch.bfloat16, device="cuda")
-    dout_u = buf[1:].view_as(d["dout"])
-    dout_u.copy_(d["dout"])
-    g = E.chunk_scan_bwd(d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], saved, dout_u,
-                         dev(dW), dev(dM), C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss)
+    assert E.e2ttt_fwd_uses_tensor_cores(
+        E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, gemm=E.GEMM_FP32)) == 0
+    kw = dict(C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss, gemm=E.GEMM_FP32)
+    _, _, _, saved = E.chunk_scan_fwd(d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], d["W0"],
+                                      d["M0"], save_states=True, **kw)
+    g = E.chunk_scan_bwd(d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], saved, d["dout"],
+                         dev(dW), dev(dM), **kw)
     torch.cuda.synchronize()
     ref = O.closed_bwd(w.kind, x["q"], x["k"], x["v"], x["lr"], x["mom"], x["decay"], x["W0"],
-                       x["M0"], w.C, x["dout"], dW, dM, d_h=w.d_h, loss=w.loss, starts=host(saved))
-    check({n: host(t) for n, t in g.items()}, ref, 2e-2, label="gelu ill-conditioned, CUDA cores")
+                       x["M0"], w.C, x["dout"], dW, dM, d_h=w.d_h, loss=w.loss)
+    # dq, dk, dv come back in the activations' bf16 (rounding 2^-9 per element):
+    # 1e-2, a tenth of what bf16 weights move; the gate and state gradients are
+    # fp32 throughout: 1e-3
+    gpu = {n: host(t) for n, t in g.items()}
+    check(gpu, ref, 1e-2, label="gelu ill-conditioned, fp32 GEMMs, end to end")
+    for n in ("dlr", "dmom", "ddecay", "dW0", "dM0"):
+        assert err(gpu[n], ref[n]) < 1e-3, (n, err(gpu[n], ref[n]))
 
 
 def _gelu_bwd_at_saved_states(E, w, x, dW, dM, heads=None):
