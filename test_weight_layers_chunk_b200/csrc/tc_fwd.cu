@@ -1982,8 +1982,6 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     J.BH = BH;
     J.NC = NC;
     J.C = C;
-    // heads per group of the tile order: E2TTT_PERSISTENT_HG in the environment
-    // overrides the default (the largest divisor of B*H whose group fits the SMs)
     const char* env_hg = getenv("E2TTT_PERSISTENT_HG");
     J.hg = env_hg ? atoi(env_hg) : mega_group_heads(BH, tph_all, num_sms());
     if (J.hg < 1 || BH % J.hg != 0) J.hg = 1;
