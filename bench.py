@@ -75,12 +75,15 @@ BWD_SIMT_FLOPS = {"bwd_dk": 12, "bwd_dw2": 6, "bwd_dir_w13": 8, "bwd_h": 8, "bwd
                   "bwd_q_rows": 2, "bwd_da": 2, "bwd_ub_eb": 2}
 
 
-# Backward GEMM phases of the tensor-core path, FLOPs per token and head in units
-# of d d_h (SwiGLU, d_k = d_v = d): 52 for the adjoint plus 12 for recomputing
-# H, E and du at the chunk-start weights (r1, r2, r3).
-TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_du": 2, "tcb_d1_dir13": 8,
-                "tcb_d2_dir2": 4, "tcb_e3_ub_dub": 4, "tcb_e4_eb": 2, "tcb_e5_hb": 2,
-                "tcb_q1_hbq": 2, "tcb_dk1": 8, "tcb_dk2": 4, "tcb_dq": 4, "tcb_dw": 14}
+# Backward GEMM launches of the tensor-core path, FLOPs per token and head in units
+# of d d_h (SwiGLU, d_k = d_v = d): 52 for the adjoint plus 14 of recomputation:
+# H, E and du at the chunk-start weights (r1 8, r2 2, the du half of r3_q1 2) and
+# du once more in e5 (its second accumulator). Three launches carry two phases
+# each: r3_q1 (du, dH; the query rows' h1b, h3b), e3_dk1 (ub, dub; dk part 1),
+# dk2_dq (dk, dq).
+TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_q1": 4, "tcb_d1_dir13": 8,
+                "tcb_d2_dir2": 4, "tcb_e3_dk1": 12, "tcb_e4_eb": 2, "tcb_e5_hb": 4,
+                "tcb_dk2_dq": 8, "tcb_dw": 14}
 
 
 def kernel_work(w, has_m0: bool) -> dict:
@@ -125,17 +128,17 @@ def kernel_work(w, has_m0: bool) -> dict:
     if dk == dv and nf == 2:
         dd = dk * dh
         b = {"tcb_r1_h": 4 * Mk + 2 * S13 + 12 * N, "tcb_r2_e": 2 * N + 2 * S2 + 4 * Mv,
-             "tcb_r3_du": 2 * Mv + 2 * S2 + 12 * N, "tcb_d1_dir13": 2 * Mk + 4 * S13 + 12 * N,
-             "tcb_d2_dir2": 2 * N + 4 * S2 + 6 * Mv, "tcb_e3_ub_dub": 2 * Mv + 4 * S2 + 18 * N,
-             "tcb_e4_eb": 2 * N + 2 * S2 + 8 * Mv, "tcb_e5_hb": 2 * Mv + 2 * S2 + 24 * N,
-             "tcb_q1_hbq": 2 * Mv + 2 * S2 + 8 * N, "tcb_dk1": 4 * N + 4 * S13 + 4 * Mk,
-             "tcb_dk2": 4 * N + 2 * S13 + 6 * Mk, "tcb_dq": 4 * N + 2 * S13 + 2 * Mk,
+             "tcb_r3_q1": (2 * Mv + 2 * S2 + 8 * N) + (2 * Mv + 2 * S2 + 8 * N),
+             "tcb_d1_dir13": 2 * Mk + 4 * S13 + 12 * N, "tcb_d2_dir2": 2 * N + 4 * S2 + 6 * Mv,
+             "tcb_e3_dk1": (2 * Mv + 4 * S2 + 18 * N) + (4 * N + 4 * S13 + 4 * Mk),
+             "tcb_e4_eb": 2 * N + 2 * S2 + 8 * Mv, "tcb_e5_hb": 4 * Mv + 2 * S2 + 20 * N,
+             "tcb_dk2_dq": (4 * N + 2 * S13 + 6 * Mk) + (4 * N + 2 * S13 + 2 * Mk),
              "tcb_dw": 14 * N + 4 * Mk + 6 * Mv + 8 * S}
         # algorithmic bytes of the backward: q, k, v, dout read and dq, dk, dv
         # written once (bf16); the saved chunk-start states read once (the shadow
         # pass); dW0, dM0 written once per call (the dW phase, one chunk's share)
-        alg = {"tcb_r1_h": 2 * 2 * Mk, "tcb_r2_e": 2 * Mv, "tcb_q1_hbq": 2 * Mv,
-               "tcb_e4_eb": 2 * Mv, "tcb_dk2": 2 * Mk, "tcb_dq": 2 * Mk, "tcb_dw": 8.0 * S / NC}
+        alg = {"tcb_r1_h": 2 * 2 * Mk, "tcb_r2_e": 2 * Mv, "tcb_r3_q1": 2 * Mv,
+               "tcb_e4_eb": 2 * Mv, "tcb_dk2_dq": 2 * 2 * Mk, "tcb_dw": 8.0 * S / NC}
         for n, by in b.items():
             per_head[n] = (TC_BWD_FLOPS[n] * dd * C, float(alg.get(n, 0.0)), by)
         per_head["tcb_shadow"] = (0.0, 8.0 * S, 26.0 * S)

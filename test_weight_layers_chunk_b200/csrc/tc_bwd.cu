@@ -11,7 +11,7 @@
 //   D1  K [D_M13 | D_W13]^T -> dh1b/dh3b = -(a P_M + b P_W) and the abar/bbar dot products
 //   D2  U_k [D_M2 | D_W2]^T -> G2u = -(a P_M + b P_W) and the abar/bbar dot products
 //   E3  E [D_M2 | D_W2] -> -(a . + b .) ; dub = dh1b H3 silu'(H1) + dh3b silu(H1)
-//   E4  eb = dub W2^T + G2u (dv = -eb)    E5  ub = E3 term + eb W2 -> h1b, h3b
+//   E4  eb = dub W2^T + G2u (dv = -eb)    E5  [E; EB] W2: du again, ub = E3 term + eb W2 -> h1b, h3b
 //   Q1  dout W2 -> query-row h1b, h3b
 //   dk = -(a dH D_M13 + b dH D_W13) + [h1b | h3b] [W1; W3] ;  dq = query-row [h1b | h3b] [W1; W3]
 //   dW13 += [h1b | h3b]^T [K; Q] ,  dW2 += [E; EB; dout]^T [dub; U_k; U_q]  (into D_W in place)
@@ -40,7 +40,7 @@ constexpr int kEW = 8;  // epilogue warps
 
 struct BwdP {
   // 32 x 32 boxes for the epilogues' TMA-staged I/O (bf16: 64B swizzle, fp32: 128B)
-  CUtensorMap mHc, mY3, mDH, mHB, fdu, fDB, fUBd;
+  CUtensorMap mHc, mY3, mDH, mHB, fDB, fUBd;
   CUtensorMap mZ3, mv, mdv, mdk, mdq, fG2U, fdkp, fDW[2];
   // mv, mdv, mdk, mdq are 3-D (columns, tokens, heads): a box past a head's last
   // token reads as zero and is clipped on store
@@ -63,13 +63,13 @@ struct BwdP {
   bf16 *DH;   // [C, hw]  dH1 | dH3 (GELU: dH)
   bf16 *HB;   // [2C, hw] h1b | h3b (GELU: hb) (keys, then queries)
   // fp32 epilogue data (per head)
-  float *du;     // [C, d_h]
   float *DB;     // [C, hw]  dh1b | dh3b (GELU: dhb)
   float *G2U;    // [C, d_v]
   float *UBd;    // [C, d_h]
   float *dkp;    // [C, d_k]
   float *part;   // [C, NG]   partial dot products for abar (and bbar at + BH*C*NG)
   int NG;
+  int per0;  // two-phase launches (EpiPair): tiles of the first phase
   int* status;
 };
 
@@ -259,10 +259,11 @@ struct EpiR2 {
     }
   }
 };
-// R3: du = E W2 -> du (fp32), dH1 = du H3 silu'(H1), dH3 = du silu(H1) (key rows).
+// R3: du = E W2 -> dH1 = du H3 silu'(H1), dH3 = du silu(H1) (key rows). du itself
+// is not stored: E5 forms it again in a second accumulator of its own GEMM.
 struct EpiR3 {
   static constexpr int kIn = 4096;            // h1 | h3 (bf16)
-  static constexpr int kSmem = kIn + 8192;    // | du (fp32) | dH1 | dH3 (bf16)
+  static constexpr int kSmem = kIn + 4096;    // | dH1 | dH3 (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
@@ -279,8 +280,7 @@ struct EpiR3 {
     const int per = BN / c.nparts, ngroups = per / 32;
     const int yD = c.z * d.C + c.m0 + c.quad * 32;
     const uint8_t* IN = c.wsmem;
-    uint8_t* F = c.wsmem + kIn;
-    uint8_t* Hs = c.wsmem + kIn + 4096;
+    uint8_t* Hs = c.wsmem + kIn;
     if (c.iter == 0 && lane == 0) issue(p, c, 0);
     __syncwarp();
     for (int gi = 0; gi < ngroups; ++gi) {
@@ -303,12 +303,10 @@ struct EpiR3 {
         h1[i] = dh1;
       }
       out_free(lane);
-      stage_f(F, lane, du);
       stage_h(Hs, lane, h1);
       stage_h(Hs + 2048, lane, h3);
       out_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.fdu, F, j, yD);
         tc::tma_store_2d(&p.mDH, Hs, j, yD);
         tc::tma_store_2d(&p.mDH, Hs + 2048, d.d_h + j, yD);
         tc::bulk_commit();
@@ -557,10 +555,11 @@ struct EpiE4 {
     }
   }
 };
-// E5: ub = UBd + eb W2 (MSE); the key rows' h1b, h3b (8 columns at a time).
+// E5: two accumulators over the same W2 tile: du = E W2 (acc0) and eb W2 (acc1);
+// ub = UBd + eb W2 (MSE); the key rows' h1b, h3b (8 columns at a time).
 struct EpiE5 {
   static constexpr int kWarps = 4;
-  static constexpr int kIn = 20480;          // UBd | du | dh1b | dh3b (fp32) | h1 | h3 (bf16)
+  static constexpr int kIn = 16384;          // UBd | dh1b | dh3b (fp32) | h1 | h3 (bf16)
   static constexpr int kSmem = kIn + 4096;   // | h1b | h3b (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
@@ -570,13 +569,12 @@ struct EpiE5 {
     const int r = ga.m0 + c.quad * 32;
     const int yC = ga.z * d.C + r, yH = ga.z * 2 * d.C + r;
     uint64_t* bar = &c.wbar[0];
-    tc::mbar_expect_tx(bar, 20480u);
+    tc::mbar_expect_tx(bar, 16384u);
     tc::tma_load_2d(c.wsmem, &p.fUBd, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 4096, &p.fdu, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 8192, &p.fDB, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 12288, &p.fDB, bar, d.d_h + ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 16384, &p.mHc, bar, ga.col, yH);
-    tc::tma_load_2d(c.wsmem + 18432, &p.mHc, bar, d.d_h + ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 8192, &p.fDB, bar, d.d_h + ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 12288, &p.mHc, bar, ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 14336, &p.mHc, bar, d.d_h + ga.col, yH);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -590,8 +588,8 @@ struct EpiE5 {
     __syncwarp();
     for (int gi = 0; gi < ngroups; ++gi) {
       const int g = c.part * per + gi * 32, j = c.n0 + g;
-      float acc[32];
-      acc1(c, g, acc);
+      float dua[32], acc[32];
+      acc2(c, g, dua, acc);
       if (!in_wait(p, c)) return;
       out_free(lane);
 #pragma unroll
@@ -599,19 +597,17 @@ struct EpiE5 {
         // 8 consecutive columns: one 16-byte chunk of a bf16 row, two of an fp32 row
         const float4 u0 = *reinterpret_cast<const float4*>(IN + swz128(lane, 2 * s8));
         const float4 u1 = *reinterpret_cast<const float4*>(IN + swz128(lane, 2 * s8 + 1));
-        const float4 d0 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8));
-        const float4 d1 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8 + 1));
-        const float4 p0 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8));
-        const float4 p1 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8 + 1));
-        const float4 q0 = *reinterpret_cast<const float4*>(IN + 12288 + swz128(lane, 2 * s8));
-        const float4 q1 = *reinterpret_cast<const float4*>(IN + 12288 + swz128(lane, 2 * s8 + 1));
+        const float4 p0 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8));
+        const float4 p1 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8 + 1));
+        const float4 q0 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8));
+        const float4 q1 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8 + 1));
         const float ubd[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-        const float du[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        const float* du = dua + 8 * s8;
         const float b1[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
         const float b3[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
         float h1[8], h3[8];
-        const uint4 x1 = *reinterpret_cast<const uint4*>(IN + 16384 + swz64(lane, s8));
-        const uint4 x3 = *reinterpret_cast<const uint4*>(IN + 18432 + swz64(lane, s8));
+        const uint4 x1 = *reinterpret_cast<const uint4*>(IN + 12288 + swz64(lane, s8));
+        const uint4 x3 = *reinterpret_cast<const uint4*>(IN + 14336 + swz64(lane, s8));
         const uint32_t w1[4] = {x1.x, x1.y, x1.z, x1.w}, w3[4] = {x3.x, x3.y, x3.z, x3.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -735,10 +731,10 @@ struct EpiR1G {
     }
   }
 };
-// R3: du = E W2 -> du (fp32), dH = du gelu'(h) (key rows).
+// R3: du = E W2 -> dH = du gelu'(h) (key rows); du is formed again in E5.
 struct EpiR3G {
   static constexpr int kIn = 2048;            // h (bf16)
-  static constexpr int kSmem = kIn + 6144;    // | du (fp32) | dH (bf16)
+  static constexpr int kSmem = kIn + 2048;    // | dH (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
@@ -753,8 +749,7 @@ struct EpiR3G {
     const int per = BN / c.nparts, ngroups = per / 32;
     const int yD = c.z * d.C + c.m0 + c.quad * 32;
     const uint8_t* IN = c.wsmem;
-    uint8_t* F = c.wsmem + kIn;
-    uint8_t* Hs = c.wsmem + kIn + 4096;
+    uint8_t* Hs = c.wsmem + kIn;
     if (c.iter == 0 && lane == 0) issue(p, c, 0);
     __syncwarp();
     for (int gi = 0; gi < ngroups; ++gi) {
@@ -771,11 +766,9 @@ struct EpiR3G {
 #pragma unroll
       for (int i = 0; i < 32; ++i) h[i] = du[i] * dgelu_f(h[i]);
       out_free(lane);
-      stage_f(F, lane, du);
       stage_h(Hs, lane, h);
       out_ready();
       if (lane == 0) {
-        tc::tma_store_2d(&p.fdu, F, j, yD);
         tc::tma_store_2d(&p.mDH, Hs, j, yD);
         tc::bulk_commit();
       }
@@ -844,10 +837,11 @@ struct EpiE3G {
     }
   }
 };
-// E5: ub = UBd + eb W2 (MSE); the key rows' hb = dhb du gelu''(h) + ub gelu'(h).
+// E5: du = E W2 (acc0) and eb W2 (acc1); ub = UBd + eb W2 (MSE); the key rows'
+// hb = dhb du gelu''(h) + ub gelu'(h).
 struct EpiE5G {
   static constexpr int kWarps = 4;
-  static constexpr int kIn = 14336;          // UBd | du | dhb (fp32) | h (bf16)
+  static constexpr int kIn = 10240;          // UBd | dhb (fp32) | h (bf16)
   static constexpr int kSmem = kIn + 2048;   // | hb (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
@@ -857,11 +851,10 @@ struct EpiE5G {
     const int r = ga.m0 + c.quad * 32;
     const int yC = ga.z * d.C + r, yH = ga.z * 2 * d.C + r;
     uint64_t* bar = &c.wbar[0];
-    tc::mbar_expect_tx(bar, 14336u);
+    tc::mbar_expect_tx(bar, 10240u);
     tc::tma_load_2d(c.wsmem, &p.fUBd, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 4096, &p.fdu, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 8192, &p.fDB, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 12288, &p.mHc, bar, ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 8192, &p.mHc, bar, ga.col, yH);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -876,12 +869,11 @@ struct EpiE5G {
     for (int gi = 0; gi < ngroups; ++gi) {
       const int g = c.part * per + gi * 32, j = c.n0 + g;
       float acc[32], ubd[32], du[32], bh[32], h[32];
-      acc1(c, g, acc);
+      acc2(c, g, du, acc);
       if (!in_wait(p, c)) return;
       unstage_f(IN, lane, ubd);
-      unstage_f(IN + 4096, lane, du);
-      unstage_f(IN + 8192, lane, bh);
-      unstage_h(IN + 12288, lane, h);
+      unstage_f(IN + 4096, lane, bh);
+      unstage_h(IN + 8192, lane, h);
       __syncwarp();
       if (lane == 0) {
         tc::fence_async_smem();
@@ -1303,6 +1295,37 @@ struct EpiWarpsOf { static constexpr int v = kEW; };
 template <class E>
 struct EpiWarpsOf<E, std::void_t<decltype(E::kWarps)>> { static constexpr int v = E::kWarps; };
 
+// Two independent GEMM phases of a chunk in one launch (one launch ramp instead
+// of two): class 0 tiles run E0's epilogue, class 1 tiles E1's. All class-0
+// tiles precede the class-1 tiles in the tile order, so a CTA switches class at
+// most once. The epilogues chain their input loads from tile to tile within a
+// class only: a class-0 tile whose successor is of class 1 requests nothing for
+// it, and a CTA's first class-1 tile starts its own chain. The launch has E0's
+// epilogue warp count; the epilogues split a tile's columns over however many
+// warps there are.
+template <class E0, class E1>
+struct EpiPair {
+  static constexpr int kWarps = EpiWarpsOf<E0>::v;
+  static constexpr int kSmem = EpiSmemOf<E0>::v > EpiSmemOf<E1>::v ? EpiSmemOf<E0>::v : EpiSmemOf<E1>::v;
+  template <int BN>
+  static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
+    EpiCtx<BN> x = c;
+    if (x.nxt_valid && x.nxt_cls != x.cls) x.nxt_valid = 0;
+    if (c.cls == 0) {
+      E0::run(p, x);
+    } else {
+      const int t = (int)blockIdx.x + c.iter * (int)gridDim.x;  // this tile's index
+      if (t - (int)gridDim.x < p.per0) x.iter = 0;              // the CTA's first class-1 tile
+      E1::run(p, x);
+    }
+  }
+};
+template <> struct Name<EpiPair<EpiR3, EpiQ1>> { static constexpr const char* v = "tcb_r3_q1"; };
+template <> struct Name<EpiPair<EpiR3G, EpiQ1G>> { static constexpr const char* v = "tcb_r3_q1"; };
+template <> struct Name<EpiPair<EpiE3, EpiDk1>> { static constexpr const char* v = "tcb_e3_dk1"; };
+template <> struct Name<EpiPair<EpiE3G, EpiDk1>> { static constexpr const char* v = "tcb_e3_dk1"; };
+template <> struct Name<EpiPair<EpiDkq<true>, EpiDkq<false>>> { static constexpr const char* v = "tcb_dk2_dq"; };
+
 template <int NUM_ACC, bool A_MN, bool B_MN, class Epi>
 cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
   constexpr int EW = EpiWarpsOf<Epi>::v;
@@ -1334,7 +1357,7 @@ cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
 struct Buf {
   int* status;
   bf16 *X, *Y3, *Z3, *Hc, *DH, *HB, *W13, *W2, *DW13, *DW2, *DM13, *DM2;
-  float *a, *b, *scal, *abar, *bbar, *sbar, *spart, *du, *DB, *G2U, *UBd, *dkp, *part;
+  float *a, *b, *scal, *abar, *bbar, *sbar, *spart, *DB, *G2U, *UBd, *dkp, *part;
   size_t total;
 };
 Buf carve(const Dims& d, char* base) {
@@ -1368,7 +1391,6 @@ Buf carve(const Dims& d, char* base) {
   B.DW2 = (bf16*)take(BH * dv * dh * h);
   B.DM13 = (bf16*)take(BH * hw * dk * h);
   B.DM2 = (bf16*)take(BH * dv * dh * h);
-  B.du = (float*)take(BH * C * dh * f);
   B.DB = (float*)take(BH * C * hw * f);
   B.G2U = (float*)take(BH * C * dv * f);
   B.UBd = (float*)take(BH * C * dh * f);
@@ -1413,7 +1435,7 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   p.ca = B.a; p.cb = B.b; p.scal = B.scal;
   p.DW = A.dW0; p.DM = A.dM0;
   p.X = B.X; p.Y3 = B.Y3; p.Z3 = B.Z3; p.Hc = B.Hc; p.DH = B.DH; p.HB = B.HB;
-  p.du = B.du; p.DB = B.DB; p.G2U = B.G2U; p.UBd = B.UBd; p.dkp = B.dkp; p.part = B.part;
+  p.DB = B.DB; p.G2U = B.G2U; p.UBd = B.UBd; p.dkp = B.dkp; p.part = B.part;
   const bool gelu = d.kind == 2;
   const int hw = (gelu ? 1 : 2) * dh;  // columns of the first state block's hidden side
   p.hw = hw;
@@ -1425,7 +1447,6 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     mok &= box32(&p.mY3, B.Y3, 3 * rC, dh, false);
     mok &= box32(&p.mDH, B.DH, rC, hw, false);
     mok &= box32(&p.mHB, B.HB, 2 * rC, hw, false);
-    mok &= box32(&p.fdu, B.du, rC, dh, true);
     mok &= box32(&p.fDB, B.DB, rC, hw, true);
     mok &= box32(&p.fUBd, B.UBd, rC, dh, true);
     mok &= box32(&p.mZ3, B.Z3, 3 * rC, dv, false);
@@ -1488,10 +1509,13 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   ok &= mk(&e4.maps[0].op0, B.Y3, rY, dh, 128);
   ok &= mk(&e4.maps[0].op2, B.W2, r2w, dh, 128);
   e4.cls[0] = cls(C / 128, dv / 128, dh / 64, {3 * C, 0, 0}, {dv, 0, 0});
-  // E5: EB (rows [C, 2C) of Z3) x W2 (MN-major);  Q1: dout (rows [2C, 3C)) x W2
+  // E5: [E; EB] (rows [0, C) and [C, 2C) of Z3; the second map starts C rows
+  // into Z3, so both A operands share one set of coordinates) x W2 (MN-major);
+  // Q1: dout (rows [2C, 3C)) x W2
   ok &= mk(&e5.maps[0].op0, B.Z3, rZ, dv, 128);
+  ok &= mk(&e5.maps[0].op1, B.Z3 + (size_t)C * dv, rZ - C, dv, 128);
   ok &= mk(&e5.maps[0].op2, B.W2, r2w, dh, 64);
-  e5.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, C, 0}, {dv, 0, 0});
+  e5.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, 0, 0}, {dv, 0, 0}, tc2::kModeA2B1);
   q1.maps[0] = e5.maps[0];
   q1.cls[0] = cls(C / 128, dh / 128, dv / 64, {3 * C, 2 * C, 0}, {dv, 0, 0});
   // dk1: dH x {D_M13, D_W13} (MN-major: N = d_k, K = 2 d_h)
@@ -1514,6 +1538,17 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   dw.cls[0] = cls(hw / 128, dk / 128, 2 * C / 64, {2 * C, 0, 0}, {2 * C, 0, 0});
   dw.cls[1] = cls(dv / 128, dh / 128, 3 * C / 64, {3 * C, 0, 0}, {3 * C, 0, 0});
   if (!ok) return cudaErrorInvalidValue;
+  // two-phase launches: R3 with Q1 (both x W2), E3 with dk1 (both two-accumulator
+  // products with the bf16 state adjoints), dk2 with dq
+  auto pair = [](const tc2::Job& j0, const tc2::Job& j1) {
+    tc2::Job j = j0;
+    j.n_cls = 2;
+    j.maps[1] = j1.maps[0];
+    j.cls[1] = j1.cls[0];
+    return j;
+  };
+  tc2::Job r3q1 = pair(r3, q1), e3k1 = pair(e3, k1), kq = pair(k2, dq);
+  auto tiles0 = [](const tc2::Job& j) { return j.cls[0].tiles_m * j.cls[0].tiles_n * j.heads; };
 
   const size_t per_chunk = (size_t)BH * 2 * d.S;
   const Dims dd = d;
@@ -1564,20 +1599,21 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     e = gelu ? run_gemm<1, false, false, EpiR1G>(r1, p, st) : run_gemm<2, false, false, EpiR1>(r1, p, st);
     if (e != cudaSuccess) return e;
     if ((e = run_gemm<1, false, false, EpiR2>(r2, p, st)) != cudaSuccess) return e;
-    e = gelu ? run_gemm<1, false, true, EpiR3G>(r3, p, st) : run_gemm<1, false, true, EpiR3>(r3, p, st);
+    p.per0 = tiles0(r3q1);
+    e = gelu ? run_gemm<1, false, true, EpiPair<EpiR3G, EpiQ1G>>(r3q1, p, st)
+             : run_gemm<1, false, true, EpiPair<EpiR3, EpiQ1>>(r3q1, p, st);
     if (e != cudaSuccess) return e;
     if ((e = run_gemm<2, false, false, EpiD1>(d1, p, st)) != cudaSuccess) return e;
     if ((e = run_gemm<2, false, false, EpiD2>(d2, p, st)) != cudaSuccess) return e;
-    e = gelu ? run_gemm<2, false, true, EpiE3G>(e3, p, st) : run_gemm<2, false, true, EpiE3>(e3, p, st);
+    p.per0 = tiles0(e3k1);
+    e = gelu ? run_gemm<2, false, true, EpiPair<EpiE3G, EpiDk1>>(e3k1, p, st)
+             : run_gemm<2, false, true, EpiPair<EpiE3, EpiDk1>>(e3k1, p, st);
     if (e != cudaSuccess) return e;
     if ((e = run_gemm<1, false, false, EpiE4>(e4, p, st)) != cudaSuccess) return e;
-    e = gelu ? run_gemm<1, false, true, EpiE5G>(e5, p, st) : run_gemm<1, false, true, EpiE5>(e5, p, st);
+    e = gelu ? run_gemm<2, false, true, EpiE5G>(e5, p, st) : run_gemm<2, false, true, EpiE5>(e5, p, st);
     if (e != cudaSuccess) return e;
-    e = gelu ? run_gemm<1, false, true, EpiQ1G>(q1, p, st) : run_gemm<1, false, true, EpiQ1>(q1, p, st);
-    if (e != cudaSuccess) return e;
-    if ((e = run_gemm<2, false, true, EpiDk1>(k1, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<1, false, true, EpiDkq<true>>(k2, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<1, false, true, EpiDkq<false>>(dq, p, st)) != cudaSuccess) return e;
+    p.per0 = tiles0(kq);
+    if ((e = run_gemm<1, false, true, EpiPair<EpiDkq<true>, EpiDkq<false>>>(kq, p, st)) != cudaSuccess) return e;
     {
       E2TTT_TRACE("tcb_rows", st);
       const long long rows = (long long)BH * C;

@@ -52,11 +52,18 @@ def test_forward_flops_from_gemm_shapes(bench):
 
 
 def test_backward_flops(bench):
-    """The tensor-core backward's phases: 52 d d_h of adjoint work per token and
-    head plus 12 of recomputed forward (R1 8, R2 2, R3 2); training counts the
-    forward and the 52 (twice the forward's 26)."""
-    assert sum(bench.TC_BWD_FLOPS.values()) == 64
-    assert bench.TC_BWD_FLOPS["tcb_r1_h"] + bench.TC_BWD_FLOPS["tcb_r2_e"] + bench.TC_BWD_FLOPS["tcb_r3_du"] == 12
+    """The tensor-core backward's launches: 52 d d_h of adjoint work per token and
+    head plus 14 of recomputation (R1 8, R2 2, du 2 in R3 and 2 more in E5, whose
+    second accumulator forms it again); training counts the forward and the 52
+    (twice the forward's 26)."""
+    assert sum(bench.TC_BWD_FLOPS.values()) == 66
+    # the recomputed H, E, du (R1, R2, R3's share of its launch) and E5's du
+    assert bench.TC_BWD_FLOPS["tcb_r1_h"] + bench.TC_BWD_FLOPS["tcb_r2_e"] + 2 + 2 == 14
+    # the adjoint phases, two-phase launches split into their parts
+    f = bench.TC_BWD_FLOPS
+    adjoint = (f["tcb_d1_dir13"] + f["tcb_d2_dir2"] + f["tcb_e3_dk1"] + f["tcb_e4_eb"] + 2
+               + (f["tcb_r3_q1"] - 2) + f["tcb_dk2_dq"] + f["tcb_dw"])
+    assert adjoint == 52
     w = gen.BY_NAME["train_1p3b_2k"]
     assert bench.train_flops(w) == 78 * w.d_k * w.d_h * w.B * w.H * w.T
 
