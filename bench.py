@@ -78,12 +78,11 @@ BWD_SIMT_FLOPS = {"bwd_dk": 12, "bwd_dw2": 6, "bwd_dir_w13": 8, "bwd_h": 8, "bwd
 # Backward GEMM launches of the tensor-core path, FLOPs per token and head in units
 # of d d_h (SwiGLU, d_k = d_v = d): 52 for the adjoint plus 14 of recomputation:
 # H, E and du at the chunk-start weights (r1 8, r2 2, the du half of r3_q1 2) and
-# du once more in e5 (its second accumulator). Three launches carry two phases
-# each: r3_q1 (du, dH; the query rows' h1b, h3b), e3_dk1 (ub, dub; dk part 1),
-# dk2_dq (dk, dq).
-TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_q1": 4, "tcb_d1_dir13": 8,
-                "tcb_d2_dir2": 4, "tcb_e3_dk1": 12, "tcb_e4_eb": 2, "tcb_e5_hb": 4,
-                "tcb_dk2_dq": 8, "tcb_dw": 14}
+# du once more in e5 (its second accumulator). Four launches carry two phases
+# each: r3_q1 (du, dH; the query rows' h1b, h3b), d1_d2 (the directional
+# products with the state adjoints), e3_dk1 (ub, dub; dk part 1), dk2_dq (dk, dq).
+TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_q1": 4, "tcb_d1_d2": 12,
+                "tcb_e3_dk1": 12, "tcb_e4_eb": 2, "tcb_e5_hb": 4, "tcb_dk2_dq": 8, "tcb_dw": 14}
 
 
 def kernel_work(w, has_m0: bool) -> dict:
@@ -129,7 +128,7 @@ def kernel_work(w, has_m0: bool) -> dict:
         dd = dk * dh
         b = {"tcb_r1_h": 4 * Mk + 2 * S13 + 12 * N, "tcb_r2_e": 2 * N + 2 * S2 + 4 * Mv,
              "tcb_r3_q1": (2 * Mv + 2 * S2 + 8 * N) + (2 * Mv + 2 * S2 + 8 * N),
-             "tcb_d1_dir13": 2 * Mk + 4 * S13 + 12 * N, "tcb_d2_dir2": 2 * N + 4 * S2 + 6 * Mv,
+             "tcb_d1_d2": (2 * Mk + 4 * S13 + 12 * N) + (2 * N + 4 * S2 + 6 * Mv),
              "tcb_e3_dk1": (2 * Mv + 4 * S2 + 18 * N) + (4 * N + 4 * S13 + 4 * Mk),
              "tcb_e4_eb": 2 * N + 2 * S2 + 8 * Mv, "tcb_e5_hb": 4 * Mv + 2 * S2 + 20 * N,
              "tcb_dk2_dq": (4 * N + 2 * S13 + 6 * Mk) + (4 * N + 2 * S13 + 2 * Mk),

@@ -16,6 +16,8 @@
 //   dk = -(a dH D_M13 + b dH D_W13) + [h1b | h3b] [W1; W3] ;  dq = query-row [h1b | h3b] [W1; W3]
 //   dW13 += [h1b | h3b]^T [K; Q] ,  dW2 += [E; EB; dout]^T [dub; U_k; U_q]  (into D_W in place)
 //   dM0 = U(1,n) D_M + c D_W ; abar, bbar and the chunk-scalar adjoints for the gate gradients.
+// Launches per chunk: the shadow pass, R1, R2, R3 + Q1, D1 + D2, E3 + dk1, E4, E5,
+// dk2 + dq, the row sums, dW (a "+" joins two phases in one launch).
 // GELU MLP (h = W1 k, u = gelu(h); one activation factor per hidden unit, so the
 // [W1; W3] blocks above are W1 alone and h1 | h3 is h):
 //   R1  h = X W1^T ; u = gelu(h)     R3  dH = du gelu'(h)     E3  dub = dhb gelu'(h)
@@ -1322,15 +1324,16 @@ struct EpiPair {
 };
 template <> struct Name<EpiPair<EpiR3, EpiQ1>> { static constexpr const char* v = "tcb_r3_q1"; };
 template <> struct Name<EpiPair<EpiR3G, EpiQ1G>> { static constexpr const char* v = "tcb_r3_q1"; };
+template <> struct Name<EpiPair<EpiD1, EpiD2>> { static constexpr const char* v = "tcb_d1_d2"; };
 template <> struct Name<EpiPair<EpiE3, EpiDk1>> { static constexpr const char* v = "tcb_e3_dk1"; };
 template <> struct Name<EpiPair<EpiE3G, EpiDk1>> { static constexpr const char* v = "tcb_e3_dk1"; };
 template <> struct Name<EpiPair<EpiDkq<true>, EpiDkq<false>>> { static constexpr const char* v = "tcb_dk2_dq"; };
 
-template <int NUM_ACC, bool A_MN, bool B_MN, class Epi>
+template <int NUM_ACC, bool A_MN, bool B_MN, class Epi, int BN = 128>
 cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
   constexpr int EW = EpiWarpsOf<Epi>::v;
   constexpr int ESM = EpiSmemOf<Epi>::v;
-  constexpr uint32_t kStage = tc2::Cfg<128, NUM_ACC, A_MN, B_MN>::kStage;
+  constexpr uint32_t kStage = tc2::Cfg<BN, NUM_ACC, A_MN, B_MN>::kStage;
   // Epilogues without staging buffers: two 64-wide k-blocks per ring slot (one
   // producer/MMA handshake per 128 of K). With staging: single k-block slots, as
   // many (up to 4) as the shared memory left over holds.
@@ -1339,9 +1342,9 @@ cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
   constexpr int kFit = (int)(kFree / ((long long)KG * kStage));
   constexpr int STAGES = ESM == 0 ? (NUM_ACC == 1 ? 3 : 2) : (kFit > 4 ? 4 : kFit);
   static_assert(STAGES >= 2, "at least two ring slots");
-  constexpr size_t smem = tc2::smem_bytes<128, NUM_ACC, A_MN, B_MN, STAGES, EW, ESM, KG>();
+  constexpr size_t smem = tc2::smem_bytes<BN, NUM_ACC, A_MN, B_MN, STAGES, EW, ESM, KG>();
   static_assert(smem <= 232448, "shared memory per CTA");
-  auto kern = tc2::gemm_persistent<128, NUM_ACC, A_MN, B_MN, STAGES, EW, Epi, BwdP, ESM, KG>;
+  auto kern = tc2::gemm_persistent<BN, NUM_ACC, A_MN, B_MN, STAGES, EW, Epi, BwdP, ESM, KG>;
   job.total_tiles = 0;
   for (int c = 0; c < job.n_cls; ++c) {
     if (job.cls[c].kblocks % KG != 0) return cudaErrorInvalidValue;
@@ -1535,11 +1538,16 @@ cudaError_t tc_bwd(const BwdArgs& A) {
   ok &= mk(&dw.maps[1].op0, B.Z3, rZ, dv, 64);
   ok &= mk(&dw.maps[1].op2, B.Y3, rY, dh, 64);
   dw.n_cls = 2;
-  dw.cls[0] = cls(hw / 128, dk / 128, 2 * C / 64, {2 * C, 0, 0}, {2 * C, 0, 0});
-  dw.cls[1] = cls(dv / 128, dh / 128, 3 * C / 64, {3 * C, 0, 0}, {3 * C, 0, 0});
+  // 128 x 256 tiles where d_k and d_h allow and they still fill every SM: a
+  // quarter fewer operand bytes per FLOP than 128 x 128 (the phase streams its
+  // operands from L2) and 512-cycle MMAs per ring slot
+  const int dwn = dk % 256 == 0 && dh % 256 == 0 && BH * (hw / 128 * dk / 256 + dv / 128 * dh / 256) >= num_sms()
+                      ? 256 : 128;
+  dw.cls[0] = cls(hw / 128, dk / dwn, 2 * C / 64, {2 * C, 0, 0}, {2 * C, 0, 0});
+  dw.cls[1] = cls(dv / 128, dh / dwn, 3 * C / 64, {3 * C, 0, 0}, {3 * C, 0, 0});
   if (!ok) return cudaErrorInvalidValue;
-  // two-phase launches: R3 with Q1 (both x W2), E3 with dk1 (both two-accumulator
-  // products with the bf16 state adjoints), dk2 with dq
+  // two-phase launches: R3 with Q1 (both x W2), D1 with D2 and E3 with dk1 (both
+  // two-accumulator products with the bf16 state adjoints), dk2 with dq
   auto pair = [](const tc2::Job& j0, const tc2::Job& j1) {
     tc2::Job j = j0;
     j.n_cls = 2;
@@ -1547,7 +1555,7 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     j.cls[1] = j1.cls[0];
     return j;
   };
-  tc2::Job r3q1 = pair(r3, q1), e3k1 = pair(e3, k1), kq = pair(k2, dq);
+  tc2::Job r3q1 = pair(r3, q1), d12 = pair(d1, d2), e3k1 = pair(e3, k1), kq = pair(k2, dq);
   auto tiles0 = [](const tc2::Job& j) { return j.cls[0].tiles_m * j.cls[0].tiles_n * j.heads; };
 
   const size_t per_chunk = (size_t)BH * 2 * d.S;
@@ -1603,8 +1611,8 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     e = gelu ? run_gemm<1, false, true, EpiPair<EpiR3G, EpiQ1G>>(r3q1, p, st)
              : run_gemm<1, false, true, EpiPair<EpiR3, EpiQ1>>(r3q1, p, st);
     if (e != cudaSuccess) return e;
-    if ((e = run_gemm<2, false, false, EpiD1>(d1, p, st)) != cudaSuccess) return e;
-    if ((e = run_gemm<2, false, false, EpiD2>(d2, p, st)) != cudaSuccess) return e;
+    p.per0 = tiles0(d12);
+    if ((e = run_gemm<2, false, false, EpiPair<EpiD1, EpiD2>>(d12, p, st)) != cudaSuccess) return e;
     p.per0 = tiles0(e3k1);
     e = gelu ? run_gemm<2, false, true, EpiPair<EpiE3G, EpiDk1>>(e3k1, p, st)
              : run_gemm<2, false, true, EpiPair<EpiE3, EpiDk1>>(e3k1, p, st);
@@ -1622,7 +1630,8 @@ cudaError_t tc_bwd(const BwdArgs& A) {
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
-    if ((e = run_gemm<1, true, true, EpiDW>(dw, p, st)) != cudaSuccess) return e;
+    e = dwn == 256 ? run_gemm<1, true, true, EpiDW, 256>(dw, p, st) : run_gemm<1, true, true, EpiDW>(dw, p, st);
+    if (e != cudaSuccess) return e;
   }
   return launch_chunk_coeffs_bwd(A.lr, A.mom, A.decay, B.abar, B.bbar, B.sbar, A.dlr, A.dmom,
                                  A.ddecay, BH, T, C, NC, d.coef, st);

@@ -61,7 +61,7 @@ def test_backward_flops(bench):
     assert bench.TC_BWD_FLOPS["tcb_r1_h"] + bench.TC_BWD_FLOPS["tcb_r2_e"] + 2 + 2 == 14
     # the adjoint phases, two-phase launches split into their parts
     f = bench.TC_BWD_FLOPS
-    adjoint = (f["tcb_d1_dir13"] + f["tcb_d2_dir2"] + f["tcb_e3_dk1"] + f["tcb_e4_eb"] + 2
+    adjoint = (f["tcb_d1_d2"] + f["tcb_e3_dk1"] + f["tcb_e4_eb"] + 2
                + (f["tcb_r3_q1"] - 2) + f["tcb_dk2_dq"] + f["tcb_dw"])
     assert adjoint == 52
     w = gen.BY_NAME["train_1p3b_2k"]
