@@ -17,7 +17,8 @@
 //   dW13 += [h1b | h3b]^T [K; Q] ,  dW2 += [E; EB; dout]^T [dub; U_k; U_q]  (into D_W in place)
 //   dM0 = U(1,n) D_M + c D_W ; abar, bbar and the chunk-scalar adjoints for the gate gradients.
 // Launches per chunk: the shadow pass, R1, R2, R3 + Q1, D1 + D2, E3 + dk1, E4, E5,
-// dk2 + dq, the row sums, dW (a "+" joins two phases in one launch).
+// dk2 + dq, the sums (abar, bbar and the chunk-scalar adjoints), dW (a "+" joins
+// two phases in one launch).
 // GELU MLP (h = W1 k, u = gelu(h); one activation factor per hidden unit, so the
 // [W1; W3] blocks above are W1 alone and h1 | h3 is h):
 //   R1  h = X W1^T ; u = gelu(h)     R3  dH = du gelu'(h)     E3  dub = dhb gelu'(h)
@@ -1168,31 +1169,30 @@ __device__ __forceinline__ float warp_sum(float x) {
   for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
   return x;
 }
-// chunk-scalar adjoints from the partials: one warp per (scalar, head), the
-// lanes reading consecutive partials.
-__global__ void bwd_scalars_kernel(const float* part, float* sbar, const float* scal, Dims d, int ci,
-                                   int nb) {
-  griddep_launch_dependents();  // the next kernel's set-up may start
-  const int w = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
-  if (w >= 3 * d.BH) return;  // warp-uniform
-  const int q = w / d.BH, z = w - q * d.BH;
-  const float* pp = part + ((size_t)q * d.BH + z) * 64;
-  float s = 0.f;
-  for (int b = lane; b < nb; b += 32) s += pp[b];
-  s = warp_sum(s);
-  if (lane == 0) {
-    const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
-    sbar[q * plane + o] = s;
-  }
-}
-// abar_t, bbar_t = -(sum of the partial dot products), fixed order: one warp
-// per row, the lanes reading consecutive partials.
-__global__ void bwd_rows_kernel(const float* part, float* abar, float* bbar, Dims d, int t0, int clen,
-                                int NG) {
+// The chunk's sums, one warp each, the lanes reading consecutive partials in a
+// fixed order: warps [0, BH C) form abar_t, bbar_t = -(sum of the row's partial
+// dot products of D1 and D2); the next 3 BH warps the chunk-scalar adjoints
+// from the shadow pass's partials (nb per head and scalar).
+__global__ void bwd_sums_kernel(const float* part, float* abar, float* bbar, const float* spart,
+                                float* sbar, Dims d, int ci, int t0, int clen, int NG, int nb) {
   griddep_launch_dependents();  // the next kernel's set-up may start
   const long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (r >= (long long)d.BH * d.C) return;  // warp-uniform
+  const long long rows = (long long)d.BH * d.C;
+  if (r >= rows) {
+    const int w = (int)(r - rows);
+    if (w >= 3 * d.BH) return;  // warp-uniform
+    const int q = w / d.BH, z = w - q * d.BH;
+    const float* pp = spart + ((size_t)q * d.BH + z) * 64;
+    float s = 0.f;
+    for (int b = lane; b < nb; b += 32) s += pp[b];
+    s = warp_sum(s);
+    if (lane == 0) {
+      const size_t plane = (size_t)d.BH * d.NC, o = (size_t)z * d.NC + ci;
+      sbar[q * plane + o] = s;
+    }
+    return;
+  }
   const int z = (int)(r / d.C), t = (int)(r % d.C);
   if (t >= clen) return;  // padding of a shorter last chunk (warp-uniform)
   const float* pa = part + (size_t)r * NG;
@@ -1598,8 +1598,6 @@ cudaError_t tc_bwd(const BwdArgs& A) {
       bwd_shadow_kernel<<<dim3(shadow_nb, BH), 256, 0, st>>>(W0, M0, 2 * d.S, A.dW0, A.dM0, B.W13,
                                                               B.W2, B.DW13, B.DW2, B.DM13, B.DM2,
                                                               B.spart, B.scal, dd, ci);
-      bwd_scalars_kernel<<<(3 * BH * 32 + 127) / 128, 128, 0, st>>>(B.spart, B.sbar, B.scal, dd, ci,
-                                                                  shadow_nb);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
@@ -1623,10 +1621,10 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     p.per0 = tiles0(kq);
     if ((e = run_gemm<1, false, true, EpiPair<EpiDkq<true>, EpiDkq<false>>>(kq, p, st)) != cudaSuccess) return e;
     {
-      E2TTT_TRACE("tcb_rows", st);
-      const long long rows = (long long)BH * C;
-      bwd_rows_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(B.part, B.abar, B.bbar, dd,
-                                                                              t0, cl, p.NG);
+      E2TTT_TRACE("tcb_sums", st);
+      const long long warps = (long long)BH * C + 3 * BH;
+      bwd_sums_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+          B.part, B.abar, B.bbar, B.spart, B.sbar, dd, ci, t0, cl, p.NG, shadow_nb);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
