@@ -46,7 +46,8 @@ _CSRC = "test_weight_layers_chunk_b200/csrc/"
 # (its translation unit and every header that unit compiles)
 _SHARED = [_CSRC + "common.cuh", _CSRC + "state.cuh", _CSRC + "paths.h", _CSRC + "trace.h"]
 KERNEL_SOURCES = {"tcb_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_bwd.cu"] + _SHARED,
-                  "tc_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_fwd.cu"] + _SHARED,
+                  "tc_": [_CSRC + "tc_gemm.cuh", _CSRC + "tc_gemm2.cuh", _CSRC + "tc_gemm_pair.cuh",
+                          _CSRC + "tc_fwd.cu"] + _SHARED,
                   "": [_CSRC + "scan.cu", _CSRC + "simt.cuh", _CSRC + "simt_fwd.cu", _CSRC + "bwd.cu"] + _SHARED}
 
 

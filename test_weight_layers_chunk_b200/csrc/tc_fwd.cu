@@ -25,6 +25,7 @@
 #include "paths.h"
 #include "state.cuh"
 #include "tc_gemm2.cuh"
+#include "tc_gemm_pair.cuh"
 #include "trace.h"
 
 namespace e2ttt {
@@ -1706,6 +1707,37 @@ cudaError_t launch(tc2::Job& job, const FwdP& p, cudaStream_t st) {
   return launch_pdl(kern, dim3(grid), dim3((2 + EW) * 32), smem, st, job, p);
 }
 
+// CTA-pair launch: a cluster of two CTAs per 256-row tile (cta_group::2 MMAs,
+// each CTA holding half of the B tile), with programmatic stream serialization.
+template <int BN, bool A_MN, bool B_MN, int STAGES, class Epi, int EW = kEpiWarps, int ESM = 0>
+cudaError_t launch_pair(tc2::Job& job, const FwdP& p, cudaStream_t st) {
+  constexpr size_t smem = tcp::pair_smem_bytes<BN, A_MN, B_MN, STAGES, EW>(ESM);
+  static_assert(smem <= 232448, "shared memory per CTA");
+  auto kern = tcp::gemm_pair<BN, A_MN, B_MN, STAGES, EW, Epi, FwdP, ESM>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  job.total_tiles = 0;
+  for (int c = 0; c < job.n_cls; ++c) job.total_tiles += job.cls[c].tiles_m * job.cls[c].tiles_n * job.heads;
+  const int sms = num_sms() & ~1;
+  const int grid = 2 * job.total_tiles < sms ? 2 * job.total_tiles : sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3((2 + EW) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  E2TTT_TRACE(EpiName<Epi>::v, st);
+  return cudaLaunchKernelEx(&cfg, kern, job, p);
+}
+
 // Heads per group in the persistent forward's tile order: the largest divisor
 // of B*H whose group (all four phases of one chunk) has no more tiles than the
 // GPU has SMs, at least one head.
@@ -1941,6 +1973,25 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
   }
   if (!ok) return cudaErrorInvalidValue;
 
+  // SwiGLU with E2TTT_PAIRS=1: G1, G2 and G3 on CTA pairs (256-row tiles, each
+  // CTA of a pair loading half of the B tile), where the 128 x 256 tiles fill the
+  // GPU. Bit-identical to the one-CTA launches; measured slower on the 1.3B layer
+  // (G1 31 -> 38 us, G2 25 -> 25, G3 24 -> 27 per chunk), so not the default.
+  const char* env_pr = getenv("E2TTT_PAIRS");
+  const char* env_f0 = getenv("E2TTT_FUSED");
+  const bool pairs = d.kind == 1 && !persistent && C % 256 == 0 && wide2 && wide3 && env_pr &&
+                     env_pr[0] == '1' && !(env_f0 && env_f0[0] == '1');
+  tc2::Job p1 = g1, p2 = g2, p3 = g3;
+  if (pairs) {
+    ok &= make_map(&p1.maps[0].op2, s.Wsh13, (uint64_t)BH * 2 * dh, dk, 128);
+    p1.maps[1].op2 = p1.maps[0].op2;
+    for (int c = 0; c < 2; ++c) p1.cls[c].tiles_m = C / 256;
+    ok &= make_map(&p2.maps[0].op2, s.W2sh, (uint64_t)BH * dv, dh, 128);
+    p2.cls[0].tiles_m = 2 * C / 256;
+    p3.cls[0].tiles_m = C / 256;
+    if (!ok) return cudaErrorInvalidValue;
+  }
+
   // SwiGLU: G1 and G2 as one fused launch per chunk (u of the query rows stays
   // on chip), selected with E2TTT_FUSED=1 in the environment. Not the default:
   // on the 1.3B layer it is slower than the two launches it replaces (each
@@ -2058,12 +2109,27 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
         fj.stall = g1.stall;  // the stall hook, armed for this chunk's first launch
         fj.wait_ns = g1.wait_ns;
         e = dv == 256 ? launch_ff12<256>(fj, p, st) : launch_ff12<128>(fj, p, st);
+      } else if (pairs) {
+        for (tc2::Job* j : {&p1, &p2, &p3}) {
+          j->ci = ci;
+          j->t0 = ci * C;
+          j->clen = clen;
+          j->wshadow = ci + 1 < NC;
+        }
+        p1.cls[0].a.y_base = p1.cls[1].a.y_base = ci * C;
+        p1.stall = g1.stall;
+        p1.wait_ns = g1.wait_ns;
+        e = launch_pair<256, false, false, 5, EpiG1, kEpiWarps, EpiG1::kSmem>(p1, p, st);
+        if (e == cudaSuccess)
+          e = clen < C ? launch_pair<256, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(p2, p, st)
+                       : launch_pair<256, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(p2, p, st);
+        if (e == cudaSuccess) e = launch_pair<256, false, true, 5, EpiG3, kEpiWarps, EpiG3::kSmem>(p3, p, st);
       } else if (d.kind == 1) {
         e = launch<256, 1, false, false, 3, EpiG1, kEpiWarps, EpiG1::kSmem>(g1, p, st);
       } else {
         e = launch<128, 1, false, false, 4, EpiG1Gelu, kEpiWarps, EpiG1Gelu::kSmem>(g1, p, st);
       }
-      if (e == cudaSuccess && !fused) {
+      if (e == cudaSuccess && !fused && !pairs) {
         if (wide2)
           e = clen < C ? launch<256, 1, false, false, 3, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
                          : launch<256, 1, false, false, 3, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
@@ -2071,7 +2137,7 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
           e = clen < C ? launch<128, 1, false, false, 4, EpiG2Pad, kEpiWarps, EpiG2Pad::kSmem>(g2, p, st)
                          : launch<128, 1, false, false, 4, EpiG2, kEpiWarps, EpiG2::kSmem>(g2, p, st);
       }
-      if (e == cudaSuccess) {
+      if (e == cudaSuccess && !pairs) {
         e = d.kind != 1 ? launch<128, 1, false, true, 3, EpiG3Gelu, kEpiWarps, EpiG3Gelu::kSmem>(g3, p, st)
             : wide3     ? launch<256, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st)
                         : launch<128, 1, false, true, 3, EpiG3, kEpiWarps, EpiG3::kSmem>(g3, p, st);

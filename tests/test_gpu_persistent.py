@@ -1,4 +1,7 @@
-"""The persistent forward: every chunk of the SwiGLU forward in one cooperative
+"""The opt-in forward drivers against the per-phase launches (and the oracle):
+the persistent forward, the fused G1 + G2 launch and the CTA-pair launches.
+
+The persistent forward: every chunk of the SwiGLU forward in one cooperative
 launch, against the per-phase launches and the fp64 oracle.
 
 With E2TTT_PERSISTENT=1 in the environment, the SwiGLU forward with momentum
@@ -12,6 +15,7 @@ covers both: every head for the stated 1.3B workload (whose collapsing state
 puts single heads above 2e-2 while the tensor-level error stays near 1e-2),
 sampled heads for the state-preserving variants.
 """
+import dataclasses
 import os
 
 import numpy as np
@@ -146,6 +150,38 @@ def test_fused_g1_g2_equals_two_launches(E, name, monkeypatch):
     monkeypatch.setenv("E2TTT_FUSED", "1")
     a = E.chunk_scan_fwd(*args, **kw)
     monkeypatch.setenv("E2TTT_FUSED", "0")
+    b = E.chunk_scan_fwd(*args, **kw)
+    torch.cuda.synchronize()
+    for u, v, n in zip(a, b, ("out", "W_end", "M_end", "saved")):
+        assert torch.equal(u, v), (name, n, rel(host(u), host(v)))
+
+
+PAIR_CASES = {
+    "layer_1p3b_2k_preserving": CASES["layer_1p3b_2k_preserving"][0],
+    # a shorter last chunk (264 of 512 tokens) through the padded G2 epilogue
+    "layer_1p3b_tail": dataclasses.replace(gen.state_preserving(gen.BY_NAME["layer_1p3b_2k"]),
+                                           name="pair_tail", T=1800, seed=74),
+}
+
+
+@pytest.mark.parametrize("name", list(PAIR_CASES))
+def test_cta_pairs_equal_one_cta_launches(E, name, monkeypatch):
+    """With E2TTT_PAIRS=1, G1, G2 and G3 of the SwiGLU forward run on CTA pairs
+    (clusters of two, cta_group::2 MMAs over 256-row tiles, each CTA holding its
+    own 128 rows of A and half of the B tile) where the 128 x 256 tiles fill the
+    GPU. Every output element is the same dot product over the same k-blocks in
+    the same order as in the one-CTA launches: equal bit for bit, saved
+    chunk-start states included."""
+    import torch
+    monkeypatch.setenv("E2TTT_PERSISTENT", "0")
+    w = PAIR_CASES[name]
+    x = gen.generate(w, m0_scale=0.5)
+    d = device_inputs(w, x)
+    kw = dict(C=w.C, d_h=w.d_h, kind=w.kind, loss=w.loss, save_states=True)
+    args = (d["q"], d["k"], d["v"], d["lr"], d["mom"], d["decay"], d["W0"], d["M0"])
+    monkeypatch.setenv("E2TTT_PAIRS", "1")
+    a = E.chunk_scan_fwd(*args, **kw)
+    monkeypatch.setenv("E2TTT_PAIRS", "0")
     b = E.chunk_scan_fwd(*args, **kw)
     torch.cuda.synchronize()
     for u, v, n in zip(a, b, ("out", "W_end", "M_end", "saved")):
