@@ -82,8 +82,11 @@ BWD_SIMT_FLOPS = {"bwd_dk": 12, "bwd_dw2": 6, "bwd_dir_w13": 8, "bwd_h": 8, "bwd
 # du once more in e5 (its second accumulator). Four launches carry two phases
 # each: r3_q1 (du, dH; the query rows' h1b, h3b), d1_d2 (the directional
 # products with the state adjoints), e3_dk1 (ub, dub; dk part 1), dk2_dq (dk, dq).
+# With the forward's E and dH saved (save_acts) r2_e and r3_q1 do not run and Q1
+# runs alone (q1_hbq): 52 + 10.
 TC_BWD_FLOPS = {"tcb_r1_h": 8, "tcb_r2_e": 2, "tcb_r3_q1": 4, "tcb_d1_d2": 12,
-                "tcb_e3_dk1": 12, "tcb_e4_eb": 2, "tcb_e5_hb": 4, "tcb_dk2_dq": 8, "tcb_dw": 14}
+                "tcb_e3_dk1": 12, "tcb_e4_eb": 2, "tcb_e5_hb": 4, "tcb_dk2_dq": 8, "tcb_dw": 14,
+                "tcb_q1_hbq": 2}
 
 
 def kernel_work(w, has_m0: bool) -> dict:
@@ -129,6 +132,7 @@ def kernel_work(w, has_m0: bool) -> dict:
         dd = dk * dh
         b = {"tcb_r1_h": 4 * Mk + 2 * S13 + 12 * N, "tcb_r2_e": 2 * N + 2 * S2 + 4 * Mv,
              "tcb_r3_q1": (2 * Mv + 2 * S2 + 8 * N) + (2 * Mv + 2 * S2 + 8 * N),
+             "tcb_q1_hbq": 2 * Mv + 2 * S2 + 8 * N,
              "tcb_d1_d2": (2 * Mk + 4 * S13 + 12 * N) + (2 * N + 4 * S2 + 6 * Mv),
              "tcb_e3_dk1": (2 * Mv + 4 * S2 + 18 * N) + (4 * N + 4 * S13 + 4 * Mk),
              "tcb_e4_eb": 2 * N + 2 * S2 + 8 * Mv, "tcb_e5_hb": 4 * Mv + 2 * S2 + 20 * N,
@@ -137,7 +141,7 @@ def kernel_work(w, has_m0: bool) -> dict:
         # algorithmic bytes of the backward: q, k, v, dout read and dq, dk, dv
         # written once (bf16); the saved chunk-start states read once (the shadow
         # pass); dW0, dM0 written once per call (the dW phase, one chunk's share)
-        alg = {"tcb_r1_h": 2 * 2 * Mk, "tcb_r2_e": 2 * Mv, "tcb_r3_q1": 2 * Mv,
+        alg = {"tcb_r1_h": 2 * 2 * Mk, "tcb_r2_e": 2 * Mv, "tcb_r3_q1": 2 * Mv, "tcb_q1_hbq": 2 * Mv,
                "tcb_e4_eb": 2 * Mv, "tcb_dk2_dq": 2 * 2 * Mk, "tcb_dw": 8.0 * S / NC}
         for n, by in b.items():
             per_head[n] = (TC_BWD_FLOPS[n] * dd * C, float(alg.get(n, 0.0)), by)
@@ -400,6 +404,7 @@ def config_dict(w, args):
     return {"workload": w.name, "kind": KIND_NAMES[w.kind],
             "B": w.B, "H": w.H, "d_k": w.d_k, "d_v": w.d_v, "d_h": w.d_h, "T": w.T, "C": w.C,
             "global_batch": w.B * args.gpus, "seq_len": w.T, "mode": args.mode,
+            **({"save_acts": True} if args.mode == "train" else {}),
             "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
             "l2": "working set larger than L2 (no flush)"}
 
@@ -484,10 +489,10 @@ def measure_extras(E, torch, dev, stream, args):
         q, k, v = f(x["q"], ad), f(x["k"], ad), f(x["v"], ad)
         lr, mom, decay, W0 = f(x["lr"]), f(x["mom"]), f(x["decay"]), f(x["W0"])
         shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss,
-                             coef=coef, momentum=nomom)
-        nc = E.e2ttt_num_chunks(shape)
+                             coef=coef, momentum=nomom,
+                             save_acts=E.SAVE_ACTS if train and w.kind != gen.LINEAR else E.RECOMPUTE_ACTS)
         outb, We, Me = torch.empty_like(v), torch.empty_like(W0), torch.empty_like(W0)
-        saved = torch.empty((nc, w.B, w.H, 2, w.state_elems), device=dev) if train else None
+        saved = E.saved_states(shape, dev) if train else None
         ws = E.workspace(shape, False, dev)
         if train:
             dout = f(x["dout"], ad)
@@ -560,14 +565,16 @@ def run_ours(args, w):
     q, k, v = f(x["q"], ad), f(x["k"], ad), f(x["v"], ad)
     lr, mom, decay, W0 = f(x["lr"]), f(x["mom"]), f(x["decay"]), f(x["W0"])
     M0 = None if not np.any(x["M0"]) else f(x["M0"])   # the workload's M0 is zero
-    shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss)
+    train = args.mode == "train"
+    # training: the forward keeps its per-chunk E and dH for the backward
+    # (save_acts), which then does not recompute them
+    shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss,
+                         save_acts=E.SAVE_ACTS if train else E.RECOMPUTE_ACTS)
     assert E.e2ttt_fwd_uses_tensor_cores(shape) == 1
-    nc = E.e2ttt_num_chunks(shape)
     out = torch.empty_like(v)
     W_end = torch.empty_like(W0)
     M_end = torch.empty_like(W0)
-    train = args.mode == "train"
-    saved = torch.empty((nc, w.B, w.H, 2, w.state_elems), device=dev) if train else None
+    saved = E.saved_states(shape, dev) if train else None
     ws = E.workspace(shape, False, dev)
     stream = torch.cuda.current_stream(dev)
 

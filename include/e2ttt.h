@@ -38,7 +38,10 @@
  *        GELU MLP: [W1 | W2] concatenated
  *   saved_states                [n_chunks, B, H, 2, S] fp32: (W, M) at the
  *                               start of every chunk (written by the forward,
- *                               read by the backward)
+ *                               read by the backward); with shape->save_acts
+ *                               = 1 followed by the forward's per-chunk
+ *                               activations (e2ttt_saved_bytes(shape) bytes in
+ *                               all)
  *
  * Conventions:
  *   - The library allocates no memory at run time. Scratch comes from
@@ -106,10 +109,21 @@ typedef enum { E2TTT_MOMENTUM = 0, E2TTT_NO_MOMENTUM = 1 } e2ttt_momentum;
  * gradients by 5-15 % under that rounding). Slower. */
 typedef enum { E2TTT_GEMM_AUTO = 0, E2TTT_GEMM_FP32 = 1 } e2ttt_gemm;
 
-/* Problem description. kind/act/loss/coef/momentum/gemm hold e2ttt_fast_kind /
- * e2ttt_dtype / e2ttt_loss / e2ttt_coef / e2ttt_momentum / e2ttt_gemm values
- * (a zero-initialised gemm field is E2TTT_GEMM_AUTO). d_h is ignored
- * (may be 0) for E2TTT_LINEAR.
+/* Saved activations (save_acts). 0: saved_states holds the chunk-start states
+ * only, and the backward recomputes the forward's per-chunk intermediates it
+ * needs. 1 (SwiGLU and GELU MLPs on the tensor-core path only): the forward
+ * also keeps, for every chunk, the residual E of the key rows and the hidden
+ * gradient dH of the inner loss (bf16) in saved_states after the states, in
+ * place of its per-call scratch (no extra memory traffic), and the backward
+ * reads them instead of recomputing them. The forward and the backward of one
+ * step must be given the same shape, save_acts included. */
+typedef enum { E2TTT_RECOMPUTE_ACTS = 0, E2TTT_SAVE_ACTS = 1 } e2ttt_acts;
+
+/* Problem description. kind/act/loss/coef/momentum/gemm/save_acts hold
+ * e2ttt_fast_kind / e2ttt_dtype / e2ttt_loss / e2ttt_coef / e2ttt_momentum /
+ * e2ttt_gemm / e2ttt_acts values (zero-initialised gemm and save_acts fields
+ * are E2TTT_GEMM_AUTO and E2TTT_RECOMPUTE_ACTS). d_h is ignored (may be 0)
+ * for E2TTT_LINEAR.
  * Limits: all sizes >= 1; B*H <= 65535; B*H*T*max(d_k, d_v, 2 d_h) < 2^31
  * (d_h counted for the MLPs only); 1 <= C <= 1024. */
 typedef struct {
@@ -121,6 +135,7 @@ typedef struct {
   int coef;
   int momentum;
   int gemm;
+  int save_acts;
 } e2ttt_shape;
 
 /* Fast-weight state size S per (b, h): d_v*d_k (linear), 2*d_h*d_k + d_v*d_h
@@ -134,6 +149,13 @@ size_t e2ttt_workspace_bytes(const e2ttt_shape* shape, int for_bwd);
 
 /* Number of chunks, ceil(T / C); 0 for an invalid shape. */
 int e2ttt_num_chunks(const e2ttt_shape* shape);
+
+/* Bytes of saved_states for `shape`: n_chunks * B * H * 2 * S * 4, plus with
+ * save_acts = 1 the per-chunk activations ([n_chunks, B, H, C, d_v] bf16 E,
+ * then [n_chunks, B, H, C, 2 d_h] (SwiGLU) or [.., d_h] (GELU MLP) bf16 dH;
+ * each region 256-byte aligned). 0 for an invalid shape. The backward only
+ * reads saved_states. */
+size_t e2ttt_saved_bytes(const e2ttt_shape* shape);
 
 /* 1 if e2ttt_chunk_scan_fwd runs `shape` on the tcgen05 tensor cores (given
  * 16-byte aligned pointers), 0 if on the fp32 CUDA-core kernels (always 0 with

@@ -31,13 +31,14 @@ LOSS_MSE, LOSS_NEG_DOT = 0, 1
 COEF_PER_TOKEN, COEF_CHUNK_MEAN = 0, 1
 MOMENTUM, NO_MOMENTUM = 0, 1
 GEMM_AUTO, GEMM_FP32 = 0, 1
+RECOMPUTE_ACTS, SAVE_ACTS = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 
 
 class e2ttt_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("B", "H", "T", "C", "d_k", "d_v", "d_h", "kind", "act", "loss", "coef", "momentum",
-                 "gemm")]
+                 "gemm", "save_acts")]
 
 
 class E2TTTError(RuntimeError):
@@ -57,6 +58,7 @@ _SIGS = {
     "e2ttt_state_elems": (ctypes.c_size_t, [_S]),
     "e2ttt_workspace_bytes": (ctypes.c_size_t, [_S, ctypes.c_int]),
     "e2ttt_num_chunks": (ctypes.c_int, [_S]),
+    "e2ttt_saved_bytes": (ctypes.c_size_t, [_S]),
     "e2ttt_fwd_uses_tensor_cores": (ctypes.c_int, [_S]),
     "e2ttt_chunk_coeffs": (ctypes.c_int, [_S, _P, _P, _P, _P, _P, _P, _P]),
     "e2ttt_chunk_scan_fwd": (ctypes.c_int, [_S] + [_P] * 13 + [ctypes.c_size_t, _P]),
@@ -84,8 +86,9 @@ def header_functions() -> list[str]:
 
 
 def make_shape(B, H, T, C, d_k, d_v, d_h=0, kind=SWIGLU, act=BF16, loss=LOSS_MSE,
-               coef=COEF_PER_TOKEN, momentum=MOMENTUM, gemm=GEMM_AUTO) -> e2ttt_shape:
-    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef, momentum, gemm)
+               coef=COEF_PER_TOKEN, momentum=MOMENTUM, gemm=GEMM_AUTO,
+               save_acts=RECOMPUTE_ACTS) -> e2ttt_shape:
+    return e2ttt_shape(B, H, T, C, d_k, d_v, d_h, kind, act, loss, coef, momentum, gemm, save_acts)
 
 
 def _ptr(x):
@@ -151,6 +154,21 @@ def e2ttt_num_chunks(shape: e2ttt_shape) -> int:
     return _lib.e2ttt_num_chunks(ctypes.byref(shape))
 
 
+def e2ttt_saved_bytes(shape: e2ttt_shape) -> int:
+    return _lib.e2ttt_saved_bytes(ctypes.byref(shape))
+
+
+def saved_states(shape, device="cuda"):
+    """The saved-states buffer of `shape`: a float32 tensor viewed as
+    [n_chunks, B, H, 2, S] (the chunk-start states) whose storage also holds the
+    saved activations when shape.save_acts is set (e2ttt_saved_bytes in all)."""
+    import torch
+    nc, S = e2ttt_num_chunks(shape), e2ttt_state_elems(shape)
+    n = (e2ttt_saved_bytes(shape) + 3) // 4
+    flat = torch.empty(n, dtype=torch.float32, device=device)
+    return flat[:nc * shape.B * shape.H * 2 * S].view(nc, shape.B, shape.H, 2, S)
+
+
 def e2ttt_fwd_uses_tensor_cores(shape: e2ttt_shape) -> int:
     return _lib.e2ttt_fwd_uses_tensor_cores(ctypes.byref(shape))
 
@@ -213,11 +231,13 @@ def e2ttt_chunk_scan_bwd(shape, q, k, v, lr, mom, decay, saved_states, dout, dW_
 
 
 # ---------------------------------------------------------------- conveniences
-def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN, momentum=MOMENTUM, gemm=GEMM_AUTO):
+def _shape_of(q, v, lr, C, d_h, kind, loss, coef=COEF_PER_TOKEN, momentum=MOMENTUM, gemm=GEMM_AUTO,
+              save_acts=RECOMPUTE_ACTS):
     import torch
     B, H, T, d_k = q.shape
     act = BF16 if q.dtype == torch.bfloat16 else F32
-    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef, momentum, gemm)
+    return make_shape(B, H, T, C, d_k, v.shape[-1], d_h, kind, act, loss, coef, momentum, gemm,
+                      save_acts)
 
 
 def workspace(shape, for_bwd=False, device="cuda"):
@@ -230,18 +250,18 @@ def workspace(shape, for_bwd=False, device="cuda"):
 
 def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGLU,
                    loss=LOSS_MSE, coef=COEF_PER_TOKEN, momentum=MOMENTUM, save_states=False,
-                   ws=None, stream=None, gemm=GEMM_AUTO):
+                   ws=None, stream=None, gemm=GEMM_AUTO, save_acts=RECOMPUTE_ACTS):
     """Allocate out / W_end / M_end (and saved_states) and run the forward.
     Returns (out, W_end, M_end, saved_states or None); M_end is None without
-    momentum (momentum=NO_MOMENTUM: pass mom=None, M0=None)."""
+    momentum (momentum=NO_MOMENTUM: pass mom=None, M0=None). save_acts=SAVE_ACTS
+    (with save_states) keeps the per-chunk E and dH for the backward; pass the
+    same save_acts to chunk_scan_bwd."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum, gemm)
-    nc = e2ttt_num_chunks(shape)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum, gemm, save_acts)
     out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     W_end = torch.empty_like(W0)
     M_end = None if momentum == NO_MOMENTUM else torch.empty_like(W0)
-    saved = (torch.empty((nc,) + tuple(W0.shape[:2]) + (2, W0.shape[-1]), dtype=torch.float32,
-                         device=q.device) if save_states else None)
+    saved = saved_states(shape, q.device) if save_states else None
     if ws is None:
         ws = workspace(shape, False, q.device)
     e2ttt_chunk_scan_fwd(shape, q, k, v, lr, mom, decay, W0, M0, out, W_end, M_end, saved, ws,
@@ -251,11 +271,11 @@ def chunk_scan_fwd(q, k, v, lr, mom, decay, W0, M0=None, *, C, d_h=0, kind=SWIGL
 
 def chunk_scan_bwd(q, k, v, lr, mom, decay, saved_states, dout, dW_end=None, dM_end=None, *, C,
                    d_h=0, kind=SWIGLU, loss=LOSS_MSE, coef=COEF_PER_TOKEN, momentum=MOMENTUM,
-                   ws=None, stream=None, gemm=GEMM_AUTO):
+                   ws=None, stream=None, gemm=GEMM_AUTO, save_acts=RECOMPUTE_ACTS):
     """Allocate the gradients and run the backward. Returns a dict (dmom and dM0
     are None without momentum)."""
     import torch
-    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum, gemm)
+    shape = _shape_of(q, v, lr, C, d_h, kind, loss, coef, momentum, gemm, save_acts)
     nomom = momentum == NO_MOMENTUM
     g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
              dlr=torch.empty_like(lr), dmom=None if nomom else torch.empty_like(mom),

@@ -49,6 +49,7 @@ bool shape_ok(const e2ttt_shape* s, std::string* why) {
   if (s->coef != E2TTT_COEF_PER_TOKEN && s->coef != E2TTT_COEF_CHUNK_MEAN) { *why = "unknown coef"; return false; }
   if (s->momentum != E2TTT_MOMENTUM && s->momentum != E2TTT_NO_MOMENTUM) { *why = "unknown momentum mode"; return false; }
   if (s->gemm != E2TTT_GEMM_AUTO && s->gemm != E2TTT_GEMM_FP32) { *why = "unknown gemm precision"; return false; }
+  if (s->save_acts != E2TTT_RECOMPUTE_ACTS && s->save_acts != E2TTT_SAVE_ACTS) { *why = "unknown save_acts mode"; return false; }
   if (s->kind != E2TTT_LINEAR && s->d_h < 1) { *why = "SwiGLU and the GELU MLP need d_h >= 1"; return false; }
   if (s->C > 1024) { *why = "chunk size C must be <= 1024"; return false; }
   long long BH = (long long)s->B * s->H;
@@ -74,6 +75,7 @@ Dims make_dims(const e2ttt_shape* s) {
   d.coef = s->coef;
   d.nomom = s->momentum == E2TTT_NO_MOMENTUM;
   d.fp32_gemm = s->gemm == E2TTT_GEMM_FP32;
+  d.save_acts = s->save_acts == E2TTT_SAVE_ACTS;
   d.S = s->kind == E2TTT_LINEAR     ? (long long)s->d_v * s->d_k
         : s->kind == E2TTT_GELU_MLP ? (long long)s->d_h * s->d_k + (long long)s->d_v * s->d_h
                                     : 2LL * s->d_h * s->d_k + (long long)s->d_v * s->d_h;
@@ -194,6 +196,12 @@ int e2ttt_num_chunks(const e2ttt_shape* s) {
   return make_dims(s).NC;
 }
 
+size_t e2ttt_saved_bytes(const e2ttt_shape* s) {
+  std::string why;
+  if (!shape_ok(s, &why)) return 0;
+  return saved_layout(make_dims(s)).total;
+}
+
 int e2ttt_fwd_uses_tensor_cores(const e2ttt_shape* s) {
   std::string why;
   if (!shape_ok(s, &why)) return -1;
@@ -277,6 +285,15 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   const bool tc_shape = tc_fwd_supported(d, bf);
   FwdWs L = fwd_layout(d, tc_shape);
   const bool tc = tc_shape && aligned16({q, k, v, out, W0, M0, W_end, M_end, saved});
+  if (d.save_acts) {
+    if (d.kind == E2TTT_LINEAR)
+      return fail(E2TTT_ERR_UNSUPPORTED, "save_acts: only the SwiGLU and GELU MLP fast weights save activations");
+    if (!saved) return fail(E2TTT_ERR_INVALID_ARG, "save_acts needs saved_states");
+    if (!tc)
+      return fail(E2TTT_ERR_UNSUPPORTED, "save_acts needs the tensor-core path (bf16 activations, gemm auto, "
+                                         "tile-aligned sizes, 16-byte aligned pointers)");
+  }
+  const SavedLayout SL = saved_layout(d);
   if (!ws) return fail(E2TTT_ERR_INVALID_ARG, "workspace is NULL (needs %zu bytes)", L.total);
   if (ws_bytes < L.total)
     return fail(E2TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.total);
@@ -287,7 +304,7 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
   Range in[] = {{q, nq, "q"}, {k, nq, "k"}, {v, nv, "v"}, {lr, ng, "lr"}, {mom, ng, "mom"},
                 {decay, ng, "decay"}, {W0, ns, "W0"}, {M0, ns, "M0"}};
   Range outr[] = {{out, nv, "out"}, {W_end, ns, "W_end"}, {M_end, ns, "M_end"},
-                  {saved, (size_t)d.NC * 2 * ns, "saved_states"}, {ws, L.total, "workspace"}};
+                  {saved, SL.total, "saved_states"}, {ws, L.total, "workspace"}};
   if (!check_overlaps(in, 8, outr, 5, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
 
   cudaStream_t st = (cudaStream_t)stream;
@@ -307,8 +324,10 @@ e2ttt_status e2ttt_chunk_scan_fwd(const e2ttt_shape* s, const void* q, const voi
     if (e != cudaSuccess) return cuda_fail(e, "saved-state reset");
   }
   if (tc) {
+    bf16* acts_e = d.save_acts ? (bf16*)((char*)saved + SL.e) : nullptr;
+    bf16* acts_dh = d.save_acts ? (bf16*)((char*)saved + SL.dh) : nullptr;
     e = tc_fwd(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out, ca, cb, scal, W0, M0,
-               W_end, M_end, saved, w + L.tc, status, st);
+               W_end, M_end, saved, w + L.tc, status, st, acts_e, acts_dh);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core forward");
     return E2TTT_OK;
   }
@@ -352,16 +371,20 @@ e2ttt_status e2ttt_chunk_scan_bwd(const e2ttt_shape* s, const void* q, const voi
   const size_t es = bf ? 2 : 4;
   const size_t nq = (size_t)d.BH * d.T * d.d_k * es, nv = (size_t)d.BH * d.T * d.d_v * es;
   const size_t ng = (size_t)d.BH * d.T * sizeof(float), ns = (size_t)d.BH * d.S * sizeof(float);
+  const SavedLayout SL = saved_layout(d);
   Range in[] = {{q, nq, "q"}, {k, nq, "k"}, {v, nv, "v"}, {lr, ng, "lr"}, {mom, ng, "mom"},
-                {decay, ng, "decay"}, {saved, (size_t)d.NC * 2 * ns, "saved_states"},
+                {decay, ng, "decay"}, {saved, SL.total, "saved_states"},
                 {dout, nv, "dout"}, {dW_end, ns, "dW_end"}, {dM_end, ns, "dM_end"}};
   Range outr[] = {{dq, nq, "dq"}, {dk, nq, "dk"}, {dv, nv, "dv"}, {dlr, ng, "dlr"},
                   {dmom, ng, "dmom"}, {ddecay, ng, "ddecay"}, {dW0, ns, "dW0"}, {dM0, ns, "dM0"},
                   {ws, need, "workspace"}};
   if (!check_overlaps(in, 10, outr, 9, &why)) return fail(E2TTT_ERR_INVALID_ARG, "%s", why.c_str());
   if (d.nomom) dM0 = (float*)((char*)ws + dm_off);  // zero momentum adjoint, kept internal
+  const bool acts = d.save_acts && d.kind != E2TTT_LINEAR;
+  const bf16* acts_e = acts ? (const bf16*)((const char*)saved + SL.e) : nullptr;
+  const bf16* acts_dh = acts ? (const bf16*)((const char*)saved + SL.dh) : nullptr;
   BwdArgs A{d, q, k, v, lr, mom, decay, saved, dout, dW_end, dM_end, dq, dk, dv,
-            dlr, dmom, ddecay, dW0, dM0, ws, (cudaStream_t)stream};
+            dlr, dmom, ddecay, dW0, dM0, ws, (cudaStream_t)stream, acts_e, acts_dh};
   cudaError_t e = bf ? bwd_run<bf16>(A) : bwd_run<float>(A);
   if (e == cudaErrorNotSupported)
     return fail(E2TTT_ERR_UNSUPPORTED, "backward path not available for this shape");

@@ -40,6 +40,7 @@ struct Dims {
   int coef;    // 0: per-token kernels, 1: chunk means (the chunk-averaged variant)
   int nomom;   // 1: no momentum (mu = 0, no M state)
   int fp32_gemm;  // 1: the fp32 CUDA-core kernels even where the tensor cores apply
+  int save_acts;  // 1: per-chunk E and dH kept in saved_states after the states
   long long S; // state elements per head
 };
 

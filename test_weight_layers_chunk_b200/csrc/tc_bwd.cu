@@ -18,7 +18,9 @@
 //   dM0 = U(1,n) D_M + c D_W ; abar, bbar and the chunk-scalar adjoints for the gate gradients.
 // Launches per chunk: the shadow pass, R1, R2, R3 + Q1, D1 + D2, E3 + dk1, E4, E5,
 // dk2 + dq, the sums (abar, bbar and the chunk-scalar adjoints), dW (a "+" joins
-// two phases in one launch).
+// two phases in one launch). With the forward's E and dH saved (save_acts), R2
+// and the R3 half of R3 + Q1 are not run: E is copied into Z3 and dH read in
+// place from the saved activations.
 // GELU MLP (h = W1 k, u = gelu(h); one activation factor per hidden unit, so the
 // [W1; W3] blocks above are W1 alone and h1 | h3 is h):
 //   R1  h = X W1^T ; u = gelu(h)     R3  dH = du gelu'(h)     E3  dub = dhb gelu'(h)
@@ -1584,6 +1586,18 @@ cudaError_t tc_bwd(const BwdArgs& A) {
       e = cudaMemcpy2DAsync(B.Z3 + (size_t)2 * C * dv, (size_t)3 * C * dv * 2,
                             (const bf16*)A.dout + (size_t)t0 * dv, (size_t)T * dv * 2,
                             (size_t)cl * dv * 2, BH, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess && A.acts_e) {
+      // saved activations: the forward's E of this chunk into rows [0, C) of Z3
+      // (its padding rows are zero), its dH read in place
+      const bf16* Ec = A.acts_e + (size_t)ci * BH * C * dv;
+      const bf16* Dc = A.acts_dh + (size_t)ci * BH * C * hw;
+      e = cudaMemcpy2DAsync(B.Z3, (size_t)3 * C * dv * 2, Ec, (size_t)C * dv * 2, (size_t)C * dv * 2, BH,
+                            cudaMemcpyDeviceToDevice, st);
+      bool mok = box32(&p.mDH, Dc, (uint64_t)BH * C, hw, false);
+      mok &= mk(&k1.maps[0].op0, Dc, rD, hw, 128);
+      if (!mok) return cudaErrorInvalidValue;
+      e3k1 = pair(e3, k1);
+    }
     if (e == cudaSuccess && cl < C) {
       const size_t pk = (size_t)(C - cl) * dk * 2, pv = (size_t)(C - cl) * dv * 2;
       e = cudaMemset2DAsync(B.X + (size_t)cl * dk, (size_t)2 * C * dk * 2, 0, pk, BH, st);
@@ -1604,11 +1618,17 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     using tc2::kModeA1B2;
     e = gelu ? run_gemm<1, false, false, EpiR1G>(r1, p, st) : run_gemm<2, false, false, EpiR1>(r1, p, st);
     if (e != cudaSuccess) return e;
-    if ((e = run_gemm<1, false, false, EpiR2>(r2, p, st)) != cudaSuccess) return e;
-    p.per0 = tiles0(r3q1);
-    e = gelu ? run_gemm<1, false, true, EpiPair<EpiR3G, EpiQ1G>>(r3q1, p, st)
-             : run_gemm<1, false, true, EpiPair<EpiR3, EpiQ1>>(r3q1, p, st);
-    if (e != cudaSuccess) return e;
+    if (A.acts_e) {
+      // E and dH come from the forward: no R2, and of R3 + Q1 only Q1
+      e = gelu ? run_gemm<1, false, true, EpiQ1G>(q1, p, st) : run_gemm<1, false, true, EpiQ1>(q1, p, st);
+      if (e != cudaSuccess) return e;
+    } else {
+      if ((e = run_gemm<1, false, false, EpiR2>(r2, p, st)) != cudaSuccess) return e;
+      p.per0 = tiles0(r3q1);
+      e = gelu ? run_gemm<1, false, true, EpiPair<EpiR3G, EpiQ1G>>(r3q1, p, st)
+               : run_gemm<1, false, true, EpiPair<EpiR3, EpiQ1>>(r3q1, p, st);
+      if (e != cudaSuccess) return e;
+    }
     p.per0 = tiles0(d12);
     if ((e = run_gemm<2, false, false, EpiPair<EpiD1, EpiD2>>(d12, p, st)) != cudaSuccess) return e;
     p.per0 = tiles0(e3k1);

@@ -1839,7 +1839,7 @@ size_t tc_fwd_scratch_bytes(const Dims& d) { return carve(d, nullptr, nullptr); 
 cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, bf16* out,
                    const float* ca, const float* cb, const float* scal, const float* W0,
                    const float* M0, float* W_end, float* M_end, float* saved, void* scratch,
-                   int* status, cudaStream_t st) {
+                   int* status, cudaStream_t st, bf16* acts_e, bf16* acts_dh) {
   Scratch s;
   carve(d, (char*)scratch, &s);
   FwdP p;
@@ -2093,6 +2093,18 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
       if (ci == 0) {
         ok &= make_map_box32(&p.shadow[0], s.Wsh13, (uint64_t)BH * r13, dk);
         if (d.kind != 0) ok &= make_map_box32(&p.shadow[1], s.W2sh, (uint64_t)BH * dv, dh);
+      }
+      if (acts_e && d.kind != 0) {
+        // saved activations: this chunk's E and dH go to its slots of saved_states
+        // (same layouts as the scratch they replace), where G3 and G4 read them
+        bf16* Ec = acts_e + (size_t)ci * BH * C * dv;
+        bf16* Dc = acts_dh + (size_t)ci * BH * C * r13;
+        ok &= make_map_box32(&p.mE, Ec, (uint64_t)BH * C, dv);
+        ok &= make_map(&g3.maps[0].op0, Ec, (uint64_t)BH * C, dv, 128);
+        ok &= make_map_box32(&p.mdH, Dc, (uint64_t)BH * C, r13);
+        ok &= make_map(&g4.maps[0].op0, Dc, (uint64_t)BH * C, r13, 64);
+        g4w.maps[0].op0 = g4.maps[0].op0;  // no momentum: the W-only aggregation reads dH too
+        p3.maps[0].op0 = g3.maps[0].op0;
       }
       if (!ok) return cudaErrorInvalidValue;
     }

@@ -142,8 +142,8 @@ def test_gemm_precision_field(E):
     tensor-core shape, GEMM_FP32 always the fp32 CUDA-core kernels (with their
     smaller workspace), other values are rejected on the host."""
     import ctypes
-    assert [n for n, _ in E.e2ttt_shape._fields_][-1] == "gemm"
-    assert ctypes.sizeof(E.e2ttt_shape) == 13 * ctypes.sizeof(ctypes.c_int)
+    assert [n for n, _ in E.e2ttt_shape._fields_][-2:] == ["gemm", "save_acts"]
+    assert ctypes.sizeof(E.e2ttt_shape) == 14 * ctypes.sizeof(ctypes.c_int)
     auto = E.make_shape(1, 2, 512, 128, 128, 128, 256, E.GELU_MLP, E.BF16)
     fp32 = E.make_shape(1, 2, 512, 128, 128, 128, 256, E.GELU_MLP, E.BF16, gemm=E.GEMM_FP32)
     assert auto.gemm == E.GEMM_AUTO == 0
@@ -165,3 +165,33 @@ def test_noalloc_status_without_a_device(E):
     st = E.e2ttt_noalloc_status(raw=True, stream=None)
     assert st == E.ERR_CUDA
     assert "e2ttt_noalloc_status" in E.e2ttt_last_error()
+
+
+def test_save_acts_field(E):
+    """save_acts: the saved-states size grows by the per-chunk bf16 E ([NC, B, H,
+    C, d_v]) and dH ([NC, B, H, C, 2 d_h] for SwiGLU, d_h for the GELU MLP),
+    each region 256-byte aligned; the linear fast weight saves no activations;
+    other values are rejected; the forward refuses save_acts on the host where
+    it cannot keep them (no saved_states, the linear fast weight, fp32
+    activations)."""
+    up = lambda x: (x + 255) // 256 * 256
+    for kind, nf in ((E.SWIGLU, 2), (E.GELU_MLP, 1)):
+        B, H, T, C, dk, dv, dh = 2, 3, 1000, 256, 128, 128, 256
+        base = E.make_shape(B, H, T, C, dk, dv, dh, kind, E.BF16)
+        acts = E.make_shape(B, H, T, C, dk, dv, dh, kind, E.BF16, save_acts=E.SAVE_ACTS)
+        nc, S = E.e2ttt_num_chunks(base), E.e2ttt_state_elems(base)
+        states = nc * B * H * 2 * S * 4
+        assert E.e2ttt_saved_bytes(base) == states
+        e_off = up(states)
+        dh_off = up(e_off + nc * B * H * C * dv * 2)
+        assert E.e2ttt_saved_bytes(acts) == dh_off + nc * B * H * C * nf * dh * 2
+    lin = E.make_shape(1, 2, 64, 16, 8, 8, 0, E.LINEAR, E.F32, save_acts=E.SAVE_ACTS)
+    assert E.e2ttt_saved_bytes(lin) == E.e2ttt_num_chunks(lin) * 2 * 2 * E.e2ttt_state_elems(lin) * 4
+    bad = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32, save_acts=2)
+    assert E.e2ttt_saved_bytes(bad) == 0
+    f32 = E.make_shape(1, 2, 64, 16, 8, 8, 16, E.SWIGLU, E.F32, save_acts=E.SAVE_ACTS)
+    assert _fwd(E, f32) == E.ERR_INVALID_ARG                  # no saved_states
+    assert "saved_states" in E.e2ttt_last_error()
+    assert _fwd(E, f32, saved_states=FAKE + 11 * (1 << 30)) == E.ERR_UNSUPPORTED  # fp32: CUDA cores
+    assert "tensor-core" in E.e2ttt_last_error()
+    assert _fwd(E, lin, saved_states=FAKE + 11 * (1 << 30)) == E.ERR_UNSUPPORTED

@@ -54,16 +54,18 @@ def test_forward_flops_from_gemm_shapes(bench):
 def test_backward_flops(bench):
     """The tensor-core backward's launches: 52 d d_h of adjoint work per token and
     head plus 14 of recomputation (R1 8, R2 2, du 2 in R3 and 2 more in E5, whose
-    second accumulator forms it again); training counts the forward and the 52
-    (twice the forward's 26)."""
-    assert sum(bench.TC_BWD_FLOPS.values()) == 66
-    # the recomputed H, E, du (R1, R2, R3's share of its launch) and E5's du
-    assert bench.TC_BWD_FLOPS["tcb_r1_h"] + bench.TC_BWD_FLOPS["tcb_r2_e"] + 2 + 2 == 14
-    # the adjoint phases, two-phase launches split into their parts
+    second accumulator forms it again), or 10 with the forward's E and dH saved;
+    training counts the forward and the 52 (twice the forward's 26)."""
     f = bench.TC_BWD_FLOPS
-    adjoint = (f["tcb_d1_d2"] + f["tcb_e3_dk1"] + f["tcb_e4_eb"] + 2
-               + (f["tcb_r3_q1"] - 2) + f["tcb_dk2_dq"] + f["tcb_dw"])
-    assert adjoint == 52
+    recompute = ("tcb_r1_h", "tcb_r2_e", "tcb_r3_q1", "tcb_d1_d2", "tcb_e3_dk1", "tcb_e4_eb",
+                 "tcb_e5_hb", "tcb_dk2_dq", "tcb_dw")
+    saved = ("tcb_r1_h", "tcb_q1_hbq", "tcb_d1_d2", "tcb_e3_dk1", "tcb_e4_eb", "tcb_e5_hb",
+             "tcb_dk2_dq", "tcb_dw")
+    # one chunk's launches: 52 of adjoint plus the recomputed H (8), E (2), du
+    # (2, in R3) and du again (2, in E5); with saved E and dH only H and E5's du
+    assert sum(f[n] for n in recompute) == 52 + 14
+    assert sum(f[n] for n in saved) == 52 + 10
+    assert f["tcb_r3_q1"] == f["tcb_q1_hbq"] + 2
     w = gen.BY_NAME["train_1p3b_2k"]
     assert bench.train_flops(w) == 78 * w.d_k * w.d_h * w.B * w.H * w.T
 
