@@ -5,7 +5,8 @@
 // closed-form chunk transition ("Rethinking Expressivity and Efficiency in
 // Test-Time Training": abstract, fully parallelized chunk-level training),
 // chunks in reverse, second-order terms through the loss gradient included.
-// Per chunk, all heads at once (token-major bf16 operands, fp32 epilogue data):
+// Per chunk, all heads at once (token-major bf16 operands and epilogue data between
+// phases, fp32 accumulation):
 //   R1  [K; Q] -> H1 = X W1^T, H3 = X W3^T (two accumulators) ; u = silu(H1) H3
 //   R2  E = U_k W2^T - V            R3  du = E W2 -> dH1 = du H3 silu'(H1), dH3 = du silu(H1)
 //   D1  K [D_M13 | D_W13]^T -> dh1b/dh3b = -(a P_M + b P_W) and the abar/bbar dot products
@@ -67,11 +68,11 @@ struct BwdP {
   bf16 *Hc;   // [2C, hw] h1 | h3 (GELU: h) (keys, then queries)
   bf16 *DH;   // [C, hw]  dH1 | dH3 (GELU: dH)
   bf16 *HB;   // [2C, hw] h1b | h3b (GELU: hb) (keys, then queries)
-  // fp32 epilogue data (per head)
-  float *DB;     // [C, hw]  dh1b | dh3b (GELU: dhb)
-  float *G2U;    // [C, d_v]
-  float *UBd;    // [C, d_h]
-  float *dkp;    // [C, d_k]
+  // bf16 epilogue data between phases (per head)
+  bf16 *DB;      // [C, hw]  dh1b | dh3b (GELU: dhb)
+  bf16 *G2U;     // [C, d_v]
+  bf16 *UBd;     // [C, d_h]
+  bf16 *dkp;     // [C, d_k]
   float *part;   // [C, NG]   partial dot products for abar (and bbar at + BH*C*NG)
   int NG;
   int per0;  // two-phase launches (EpiPair): tiles of the first phase
@@ -138,6 +139,17 @@ __device__ __forceinline__ void unstage_h(const uint8_t* buf, int r, float (&v)[
       v[8 * q + 2 * j] = f.x;
       v[8 * q + 2 * j + 1] = f.y;
     }
+  }
+}
+// The 8 bf16 values of 16-byte chunk q of row r of a 64B-swizzled tile.
+__device__ __forceinline__ void unpack8(const uint8_t* buf, int r, int q, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(buf + swz64(r, q));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
   }
 }
 __device__ __forceinline__ void stage_f(uint8_t* buf, int r, const float (&v)[32]) {
@@ -321,10 +333,10 @@ struct EpiR3 {
   }
 };
 // D1: acc0 = K D_M13^T, acc1 = K D_W13^T over columns [0, 2 d_h) -> DB = -(a P_M + b P_W)
-// (fp32) and the abar / bbar partial dot products with dH.
+// (bf16) and the abar / bbar partial dot products with dH.
 struct EpiD1 {
   static constexpr int kIn = 2048;           // dH (bf16)
-  static constexpr int kSmem = kIn + 4096;   // | DB (fp32)
+  static constexpr int kSmem = kIn + 2048;   // | DB (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
@@ -366,7 +378,7 @@ struct EpiD1 {
         pm[i] = -(a * pm[i] + b * pw[i]);
       }
       out_free(lane);
-      stage_f(F, lane, pm);
+      stage_h(F, lane, pm);
       out_ready();
       if (lane == 0) {
         tc::tma_store_2d(&p.fDB, F, jj, yD);
@@ -379,10 +391,10 @@ struct EpiD1 {
   }
 };
 // D2: acc0 = U_k D_M2^T, acc1 = U_k D_W2^T over columns [0, d_v) -> G2u = -(a P_M + b P_W)
-// (fp32) and the abar / bbar partial dot products with E.
+// (bf16) and the abar / bbar partial dot products with E.
 struct EpiD2 {
   static constexpr int kIn = 2048;           // E (bf16)
-  static constexpr int kSmem = kIn + 4096;   // | G2u (fp32)
+  static constexpr int kSmem = kIn + 2048;   // | G2u (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
@@ -424,7 +436,7 @@ struct EpiD2 {
         pm[i] = -(a * pm[i] + b * pw[i]);
       }
       out_free(lane);
-      stage_f(F, lane, pm);
+      stage_h(F, lane, pm);
       out_ready();
       if (lane == 0) {
         tc::tma_store_2d(&p.fG2U, F, col, yG);
@@ -437,11 +449,11 @@ struct EpiD2 {
   }
 };
 // E3: acc0 = E D_M2, acc1 = E D_W2 (columns = hidden units) -> UBd = -(a . + b .)
-// (fp32) and dub = dh1b H3 silu'(H1) + dh3b silu(H1) (bf16, rows [0, C) of Y3).
+// (bf16) and dub = dh1b H3 silu'(H1) + dh3b silu(H1) (bf16, rows [0, C) of Y3).
 struct EpiE3 {
   static constexpr int kWarps = 4;
-  static constexpr int kIn = 12288;          // dh1b | dh3b (fp32) | h1 | h3 (bf16)
-  static constexpr int kSmem = kIn + 6144;   // | UBd (fp32) | dub (bf16)
+  static constexpr int kIn = 8192;           // dh1b | dh3b | h1 | h3 (bf16)
+  static constexpr int kSmem = kIn + 4096;   // | UBd | dub (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
@@ -449,11 +461,11 @@ struct EpiE3 {
     const Dims& d = p.d;
     const int r = ga.m0 + c.quad * 32;
     uint64_t* bar = &c.wbar[0];
-    tc::mbar_expect_tx(bar, 12288u);
+    tc::mbar_expect_tx(bar, 8192u);
     tc::tma_load_2d(c.wsmem, &p.fDB, bar, ga.col, ga.z * d.C + r);
-    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, d.d_h + ga.col, ga.z * d.C + r);
-    tc::tma_load_2d(c.wsmem + 8192, &p.mHc, bar, ga.col, ga.z * 2 * d.C + r);
-    tc::tma_load_2d(c.wsmem + 10240, &p.mHc, bar, d.d_h + ga.col, ga.z * 2 * d.C + r);
+    tc::tma_load_2d(c.wsmem + 2048, &p.fDB, bar, d.d_h + ga.col, ga.z * d.C + r);
+    tc::tma_load_2d(c.wsmem + 4096, &p.mHc, bar, ga.col, ga.z * 2 * d.C + r);
+    tc::tma_load_2d(c.wsmem + 6144, &p.mHc, bar, d.d_h + ga.col, ga.z * 2 * d.C + r);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -466,7 +478,7 @@ struct EpiE3 {
     const int r0 = c.m0 + c.quad * 32;
     const uint8_t* IN = c.wsmem;
     uint8_t* F = c.wsmem + kIn;
-    uint8_t* Hs = c.wsmem + kIn + 4096;
+    uint8_t* Hs = c.wsmem + kIn + 2048;
     if (c.iter == 0 && lane == 0) issue(p, c, 0);
     __syncwarp();
     for (int gi = 0; gi < ngroups; ++gi) {
@@ -476,13 +488,13 @@ struct EpiE3 {
 #pragma unroll
       for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
       out_free(lane);
-      stage_f(F, lane, m);
+      stage_h(F, lane, m);
       if (!in_wait(p, c)) return;
       float b1[32], b3[32];
-      unstage_f(IN, lane, b1);
-      unstage_f(IN + 4096, lane, b3);
-      unstage_h(IN + 8192, lane, m);       // h1
-      unstage_h(IN + 10240, lane, w);      // h3
+      unstage_h(IN, lane, b1);
+      unstage_h(IN + 2048, lane, b3);
+      unstage_h(IN + 4096, lane, m);       // h1
+      unstage_h(IN + 6144, lane, w);       // h3
       __syncwarp();
       if (lane == 0) {
         tc::fence_async_smem();
@@ -506,13 +518,13 @@ struct EpiE3 {
 };
 // E4: eb = dub W2^T + G2u; EB row (zero for the dot loss) -> rows [C, 2C) of Z3, dv = -eb.
 struct EpiE4 {
-  static constexpr int kIn = 4096;           // G2u (fp32)
+  static constexpr int kIn = 2048;           // G2u (bf16)
   static constexpr int kSmem = kIn + 4096;   // | dv | EB (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
     if (!ga.valid) return;
-    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
     tc::tma_load_2d(c.wsmem, &p.fG2U, &c.wbar[0], ga.col, ga.z * p.d.C + ga.m0 + c.quad * 32);
   }
   template <int BN>
@@ -532,7 +544,7 @@ struct EpiE4 {
       float eb[32], gu[32];
       acc1(c, g, eb);
       if (!in_wait(p, c)) return;
-      unstage_f(IN, lane, gu);
+      unstage_h(IN, lane, gu);
       __syncwarp();
       if (lane == 0) {
         tc::fence_async_smem();
@@ -564,7 +576,7 @@ struct EpiE4 {
 // ub = UBd + eb W2 (MSE); the key rows' h1b, h3b (8 columns at a time).
 struct EpiE5 {
   static constexpr int kWarps = 4;
-  static constexpr int kIn = 16384;          // UBd | dh1b | dh3b (fp32) | h1 | h3 (bf16)
+  static constexpr int kIn = 10240;          // UBd | dh1b | dh3b | h1 | h3 (bf16)
   static constexpr int kSmem = kIn + 4096;   // | h1b | h3b (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
@@ -574,12 +586,12 @@ struct EpiE5 {
     const int r = ga.m0 + c.quad * 32;
     const int yC = ga.z * d.C + r, yH = ga.z * 2 * d.C + r;
     uint64_t* bar = &c.wbar[0];
-    tc::mbar_expect_tx(bar, 16384u);
+    tc::mbar_expect_tx(bar, 10240u);
     tc::tma_load_2d(c.wsmem, &p.fUBd, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 8192, &p.fDB, bar, d.d_h + ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 12288, &p.mHc, bar, ga.col, yH);
-    tc::tma_load_2d(c.wsmem + 14336, &p.mHc, bar, d.d_h + ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 2048, &p.fDB, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, d.d_h + ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 6144, &p.mHc, bar, ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 8192, &p.mHc, bar, d.d_h + ga.col, yH);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -599,28 +611,14 @@ struct EpiE5 {
       out_free(lane);
 #pragma unroll
       for (int s8 = 0; s8 < 4; ++s8) {
-        // 8 consecutive columns: one 16-byte chunk of a bf16 row, two of an fp32 row
-        const float4 u0 = *reinterpret_cast<const float4*>(IN + swz128(lane, 2 * s8));
-        const float4 u1 = *reinterpret_cast<const float4*>(IN + swz128(lane, 2 * s8 + 1));
-        const float4 p0 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8));
-        const float4 p1 = *reinterpret_cast<const float4*>(IN + 4096 + swz128(lane, 2 * s8 + 1));
-        const float4 q0 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8));
-        const float4 q1 = *reinterpret_cast<const float4*>(IN + 8192 + swz128(lane, 2 * s8 + 1));
-        const float ubd[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        // 8 consecutive columns: one 16-byte chunk of each bf16 row
+        float ubd[8], b1[8], b3[8], h1[8], h3[8];
+        unpack8(IN, lane, s8, ubd);
+        unpack8(IN + 2048, lane, s8, b1);
+        unpack8(IN + 4096, lane, s8, b3);
+        unpack8(IN + 6144, lane, s8, h1);
+        unpack8(IN + 8192, lane, s8, h3);
         const float* du = dua + 8 * s8;
-        const float b1[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        const float b3[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        float h1[8], h3[8];
-        const uint4 x1 = *reinterpret_cast<const uint4*>(IN + 12288 + swz64(lane, s8));
-        const uint4 x3 = *reinterpret_cast<const uint4*>(IN + 14336 + swz64(lane, s8));
-        const uint32_t w1[4] = {x1.x, x1.y, x1.z, x1.w}, w3[4] = {x3.x, x3.y, x3.z, x3.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w1[k]));
-          const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w3[k]));
-          h1[2 * k] = f1.x; h1[2 * k + 1] = f1.y;
-          h3[2 * k] = f3.x; h3[2 * k + 1] = f3.y;
-        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float ub = ubd[i] + (d.loss == 0 ? acc[8 * s8 + i] : 0.f);
@@ -782,11 +780,11 @@ struct EpiR3G {
   }
 };
 // E3: acc0 = E D_M2, acc1 = E D_W2 (columns = hidden units) -> UBd = -(a . + b .)
-// (fp32) and dub = dhb gelu'(h) (bf16, rows [0, C) of Y3).
+// (bf16) and dub = dhb gelu'(h) (bf16, rows [0, C) of Y3).
 struct EpiE3G {
   static constexpr int kWarps = 4;
-  static constexpr int kIn = 6144;           // dhb (fp32) | h (bf16)
-  static constexpr int kSmem = kIn + 6144;   // | UBd (fp32) | dub (bf16)
+  static constexpr int kIn = 4096;           // dhb | h (bf16)
+  static constexpr int kSmem = kIn + 4096;   // | UBd | dub (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
@@ -794,9 +792,9 @@ struct EpiE3G {
     const Dims& d = p.d;
     const int r = ga.m0 + c.quad * 32;
     uint64_t* bar = &c.wbar[0];
-    tc::mbar_expect_tx(bar, 6144u);
+    tc::mbar_expect_tx(bar, 4096u);
     tc::tma_load_2d(c.wsmem, &p.fDB, bar, ga.col, ga.z * d.C + r);
-    tc::tma_load_2d(c.wsmem + 4096, &p.mHc, bar, ga.col, ga.z * 2 * d.C + r);
+    tc::tma_load_2d(c.wsmem + 2048, &p.mHc, bar, ga.col, ga.z * 2 * d.C + r);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -809,7 +807,7 @@ struct EpiE3G {
     const int r0 = c.m0 + c.quad * 32;
     const uint8_t* IN = c.wsmem;
     uint8_t* F = c.wsmem + kIn;
-    uint8_t* Hs = c.wsmem + kIn + 4096;
+    uint8_t* Hs = c.wsmem + kIn + 2048;
     if (c.iter == 0 && lane == 0) issue(p, c, 0);
     __syncwarp();
     for (int gi = 0; gi < ngroups; ++gi) {
@@ -819,11 +817,11 @@ struct EpiE3G {
 #pragma unroll
       for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
       out_free(lane);
-      stage_f(F, lane, m);
+      stage_h(F, lane, m);
       if (!in_wait(p, c)) return;
       float bh[32];
-      unstage_f(IN, lane, bh);
-      unstage_h(IN + 4096, lane, w);   // h
+      unstage_h(IN, lane, bh);
+      unstage_h(IN + 2048, lane, w);   // h
       __syncwarp();
       if (lane == 0) {
         tc::fence_async_smem();
@@ -846,7 +844,7 @@ struct EpiE3G {
 // hb = dhb du gelu''(h) + ub gelu'(h).
 struct EpiE5G {
   static constexpr int kWarps = 4;
-  static constexpr int kIn = 10240;          // UBd | dhb (fp32) | h (bf16)
+  static constexpr int kIn = 6144;           // UBd | dhb | h (bf16)
   static constexpr int kSmem = kIn + 2048;   // | hb (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
@@ -856,10 +854,10 @@ struct EpiE5G {
     const int r = ga.m0 + c.quad * 32;
     const int yC = ga.z * d.C + r, yH = ga.z * 2 * d.C + r;
     uint64_t* bar = &c.wbar[0];
-    tc::mbar_expect_tx(bar, 10240u);
+    tc::mbar_expect_tx(bar, 6144u);
     tc::tma_load_2d(c.wsmem, &p.fUBd, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 4096, &p.fDB, bar, ga.col, yC);
-    tc::tma_load_2d(c.wsmem + 8192, &p.mHc, bar, ga.col, yH);
+    tc::tma_load_2d(c.wsmem + 2048, &p.fDB, bar, ga.col, yC);
+    tc::tma_load_2d(c.wsmem + 4096, &p.mHc, bar, ga.col, yH);
   }
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
@@ -876,9 +874,9 @@ struct EpiE5G {
       float acc[32], ubd[32], du[32], bh[32], h[32];
       acc2(c, g, du, acc);
       if (!in_wait(p, c)) return;
-      unstage_f(IN, lane, ubd);
-      unstage_f(IN + 4096, lane, bh);
-      unstage_h(IN + 8192, lane, h);
+      unstage_h(IN, lane, ubd);
+      unstage_h(IN + 2048, lane, bh);
+      unstage_h(IN + 4096, lane, h);
       __syncwarp();
       if (lane == 0) {
         tc::fence_async_smem();
@@ -945,9 +943,9 @@ struct EpiQ1G {
     }
   }
 };
-// dk part 1: -(a dH D_M13 + b dH D_W13) (fp32) -> dkp.
+// dk part 1: -(a dH D_M13 + b dH D_W13) -> dkp (bf16).
 struct EpiDk1 {
-  static constexpr int kSmem = 4096;  // dkp staging (fp32)
+  static constexpr int kSmem = 2048;  // dkp staging (bf16)
   template <int BN>
   static __device__ void run(const BwdP& p, const EpiCtx<BN>& c) {
     const Dims& d = p.d;
@@ -963,7 +961,7 @@ struct EpiDk1 {
 #pragma unroll
       for (int i = 0; i < 32; ++i) m[i] = -(a * m[i] + b * w[i]);
       out_free(lane);
-      stage_f(F, lane, m);
+      stage_h(F, lane, m);
       out_ready();
       if (lane == 0) {
         tc::tma_store_2d(&p.fdkp, F, c.n0 + g, y);
@@ -976,13 +974,13 @@ struct EpiDk1 {
 // dk part 2 (adds part 1) and dq: [h1b | h3b] [W1; W3] -> the activation-dtype output.
 template <bool KEYS>
 struct EpiDkq {
-  static constexpr int kIn = KEYS ? 4096 : 0;  // dkp (fp32)
+  static constexpr int kIn = KEYS ? 2048 : 0;  // dkp (bf16)
   static constexpr int kSmem = kIn + 2048;     // | dk or dq (bf16)
   template <int BN>
   static __device__ __forceinline__ void issue(const BwdP& p, const EpiCtx<BN>& c, int gi) {
     const GroupAt ga = group_at(c, gi);
     if (!ga.valid) return;
-    tc::mbar_expect_tx(&c.wbar[0], 4096u);
+    tc::mbar_expect_tx(&c.wbar[0], 2048u);
     tc::tma_load_2d(c.wsmem, &p.fdkp, &c.wbar[0], ga.col, ga.z * p.d.C + ga.m0 + c.quad * 32);
   }
   template <int BN>
@@ -1003,7 +1001,7 @@ struct EpiDkq {
       if (KEYS) {
         float y[32];
         if (!in_wait(p, c)) return;
-        unstage_f(IN, lane, y);
+        unstage_h(IN, lane, y);
         __syncwarp();
         if (lane == 0) {
           tc::fence_async_smem();
@@ -1362,7 +1360,8 @@ cudaError_t run_gemm(tc2::Job& job, const BwdP& p, cudaStream_t st) {
 struct Buf {
   int* status;
   bf16 *X, *Y3, *Z3, *Hc, *DH, *HB, *W13, *W2, *DW13, *DW2, *DM13, *DM2;
-  float *a, *b, *scal, *abar, *bbar, *sbar, *spart, *DB, *G2U, *UBd, *dkp, *part;
+  float *a, *b, *scal, *abar, *bbar, *sbar, *spart, *part;
+  bf16 *DB, *G2U, *UBd, *dkp;
   size_t total;
 };
 Buf carve(const Dims& d, char* base) {
@@ -1396,10 +1395,10 @@ Buf carve(const Dims& d, char* base) {
   B.DW2 = (bf16*)take(BH * dv * dh * h);
   B.DM13 = (bf16*)take(BH * hw * dk * h);
   B.DM2 = (bf16*)take(BH * dv * dh * h);
-  B.DB = (float*)take(BH * C * hw * f);
-  B.G2U = (float*)take(BH * C * dv * f);
-  B.UBd = (float*)take(BH * C * dh * f);
-  B.dkp = (float*)take(BH * C * dk * f);
+  B.DB = (bf16*)take(BH * C * hw * h);
+  B.G2U = (bf16*)take(BH * C * dv * h);
+  B.UBd = (bf16*)take(BH * C * dh * h);
+  B.dkp = (bf16*)take(BH * C * dk * h);
   B.part = (float*)take(2 * BH * C * NG * f);
   B.total = off;
   return B;
@@ -1452,15 +1451,15 @@ cudaError_t tc_bwd(const BwdArgs& A) {
     mok &= box32(&p.mY3, B.Y3, 3 * rC, dh, false);
     mok &= box32(&p.mDH, B.DH, rC, hw, false);
     mok &= box32(&p.mHB, B.HB, 2 * rC, hw, false);
-    mok &= box32(&p.fDB, B.DB, rC, hw, true);
-    mok &= box32(&p.fUBd, B.UBd, rC, dh, true);
+    mok &= box32(&p.fDB, B.DB, rC, hw, false);
+    mok &= box32(&p.fUBd, B.UBd, rC, dh, false);
     mok &= box32(&p.mZ3, B.Z3, 3 * rC, dv, false);
     mok &= tok_box32(&p.mv, A.v, T, dv, BH);
     mok &= tok_box32(&p.mdv, A.dv, T, dv, BH);
     mok &= tok_box32(&p.mdk, A.dk, T, dk, BH);
     mok &= tok_box32(&p.mdq, A.dq, T, dk, BH);
-    mok &= box32(&p.fG2U, B.G2U, rC, dv, true);
-    mok &= box32(&p.fdkp, B.dkp, rC, dk, true);
+    mok &= box32(&p.fG2U, B.G2U, rC, dv, false);
+    mok &= box32(&p.fdkp, B.dkp, rC, dk, false);
     mok &= state_box32(&p.fDW[0], A.dW0, hw, dk, BH, d.S);
     mok &= state_box32(&p.fDW[1], A.dW0 + (size_t)hw * dk, dv, dh, BH, d.S);
     if (!mok) return cudaErrorInvalidValue;
