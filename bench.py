@@ -98,7 +98,7 @@ def kernel_work(w, has_m0: bool) -> dict:
     in the activation dtype, the three gates once, W0 and M0 read and W_end and
     M_end written once per call (fp32), each charged to the kernel that moves it
     (q, k to the first GEMM phase, v, out to the phase that forms out and E, the
-    state to the aggregation phase, one chunk's share per launch). K1 is judged
+    state to the aggregation phase, one chunk's share per launch). K1 is rated
     as an operator of its own: gates in, a and b out, chunk scalars out. Traffic
     of intermediates (activations, residuals, scaled operand copies, bf16 state
     copies) and the per-chunk round trip of the state through HBM are
