@@ -26,16 +26,24 @@ def E():
     return E
 
 
-@pytest.mark.parametrize("persistent", [False, True])
-def test_bounded_wait_runs_out_and_the_context_recovers(E, persistent, monkeypatch):
-    """Both forward drivers: the per-phase launches, and the persistent kernel
+@pytest.mark.parametrize("driver", ["phases", "persistent", "pairs"])
+def test_bounded_wait_runs_out_and_the_context_recovers(E, driver, monkeypatch):
+    """Three forward drivers: the per-phase launches; the persistent kernel
     (E2TTT_PERSISTENT=1, one launch for all chunks), where the stalled CTA's
-    tiles never complete and every CTA waiting on them gives up too."""
+    tiles never complete and every CTA waiting on them gives up too; and the
+    CTA-pair launches (E2TTT_PAIRS=1, at the 1.3B layer's shapes where they
+    apply), where the even CTA of the first pair stalls before its MMAs, its
+    partner's producer and both CTAs' epilogues give up, and the pair meets at
+    its cluster barrier before freeing tensor memory."""
     import torch
-    monkeypatch.setenv("E2TTT_PERSISTENT", "1" if persistent else "0")
+    monkeypatch.setenv("E2TTT_PERSISTENT", "1" if driver == "persistent" else "0")
+    monkeypatch.setenv("E2TTT_PAIRS", "1" if driver == "pairs" else "0")
     saved = False
-    w = gen.Workload("stall", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform", 0.999,
-                     seed=61, lr_lo=0.002, lr_hi=0.02)
+    if driver == "pairs":
+        w = gen.BY_NAME["layer_1p3b_2k"]
+    else:
+        w = gen.Workload("stall", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128, "uniform",
+                         0.999, seed=61, lr_lo=0.002, lr_hi=0.02)
     x = gen.generate(w, m0_scale=0.5)
     d = device_inputs(w, x)
     shape = E.make_shape(w.B, w.H, w.T, w.C, w.d_k, w.d_v, w.d_h, w.kind, w.act, w.loss)
