@@ -351,6 +351,10 @@ chunk_coeffs_vec_kernel(const float* __restrict__ lr, const float* __restrict__ 
                         const float* __restrict__ decay, float* __restrict__ a_out,
                         float* __restrict__ b_out, float* __restrict__ scal, int BH, int T, int C,
                         int NC, int coef) {
+  // A successor launched with programmatic stream serialization (the forward's
+  // prep launch) may start now: it waits (griddepcontrol.wait) before it reads
+  // a, b or the chunk scalars; plain launches still wait for this grid to end.
+  griddep_launch_dependents();
   __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
   __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

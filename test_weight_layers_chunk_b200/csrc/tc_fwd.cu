@@ -1595,20 +1595,28 @@ __device__ __forceinline__ void scale_keys_blocks(const bf16* __restrict__ k, co
 // The two prep jobs of a call in one launch: of every three blocks two copy W0
 // to bf16 and one scales the keys (k NULL: the copy alone), so both streams of
 // HBM traffic run side by side and the step has one prep launch, not two.
+// Launched with programmatic stream serialization behind K1: the copy blocks
+// read only W0, which every earlier operation of the stream has finished
+// writing (K1 itself is a plain launch), and write the bf16 shadow, which no
+// kernel still running reads, so they start while K1 runs; the key-scaling
+// blocks wait for K1's a and b. The next kernel (G1, which waits for this one
+// to finish) is released once this block's work is issued, so its CTAs do not
+// take registers from the copy while it runs.
 __global__ void __launch_bounds__(256) prep_kernel(FwdP p, const float* __restrict__ W0,
                                                    const bf16* __restrict__ k,
                                                    const float* __restrict__ ca,
                                                    const float* __restrict__ cb, bf16* Ka, bf16* Kb,
                                                    long long tokens, int d_k) {
-  griddep_launch_dependents();  // the next kernel's set-up may start
   const int b = blockIdx.x, n = gridDim.x;
   if (k == nullptr) {
     shadow_init_blocks(p, W0, b, n);
   } else if (b % 3 == 2) {
+    griddep_wait();  // K1's a_t and b_t are complete and visible
     scale_keys_blocks(k, ca, cb, Ka, Kb, tokens, d_k, b / 3, n / 3);
   } else {
     shadow_init_blocks(p, W0, b - b / 3, n - n / 3);
   }
+  griddep_launch_dependents();
 }
 
 // ---------------------------------------------------------------- host side
@@ -1861,9 +1869,9 @@ cudaError_t tc_fwd(const Dims& d, const bf16* q, const bf16* k, const bf16* v, b
     // the bf16 copy of W0 and (MLP fast weights) the scaled keys: 12 blocks per
     // SM, a multiple of 3 (8 copy the state, 4 scale keys)
     E2TTT_TRACE("tc_prep", st);
-    prep_kernel<<<12 * num_sms(), 256, 0, st>>>(p, W0, d.kind != 0 ? k : nullptr, ca, cb,
-                                               d.nomom ? nullptr : s.Ka, s.Kb, (long long)BH * T, dk);
-    e = cudaGetLastError();
+    e = launch_pdl(prep_kernel, dim3(12 * num_sms()), dim3(256), 0, st, p, W0,
+                   d.kind != 0 ? k : nullptr, ca, cb, d.nomom ? nullptr : s.Ka, s.Kb,
+                   (long long)BH * T, dk);
     if (e != cudaSuccess) return e;
   }
 
