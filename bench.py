@@ -812,7 +812,10 @@ def main():
                     help="default: layer_1p3b_2k (fwd) or train_1p3b_2k (train)")
     ap.add_argument("--mode", choices=["fwd", "train", "k1"], default="fwd",
                     help="k1: only K1 at 2^26 token-heads (for profiling it alone)")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=30,
+                    help="timed steps of the end-to-end loop; the first step's input copies and "
+                         "the last one's result copies overlap nothing, so more steps measure the "
+                         "steady state")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extras", type=int, default=1, help="also time T=16K fwd and T=2K fwd+bwd")
