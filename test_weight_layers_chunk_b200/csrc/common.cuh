@@ -44,17 +44,37 @@ struct Dims {
   long long S; // state elements per head
 };
 
-// Exact GELU z Phi(z) (Phi the standard normal CDF, through erff) and its
-// derivative Phi(z) + z phi(z), for the GELU MLP fast weight.
-__device__ __forceinline__ float gelu_cdf_f(float z) { return 0.5f * (1.0f + erff(z * 0.70710678118654752f)); }
-__device__ __forceinline__ float gelu_f(float z) { return z * gelu_cdf_f(z); }
+// The standard normal CDF Phi(z) and density phi(z) for the GELU MLP fast
+// weight (GELU z Phi(z), not the tanh form). Phi comes from erfc(|z| / sqrt 2)
+// by the rational approximation of Abramowitz and Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (after Hastings; absolute error at
+// most 1.5e-7 in erf): erfc(x) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5))))
+// exp(-x^2) with t = 1 / (1 + p x). At x = |z| / sqrt 2 its exponential is
+// exp(-z^2 / 2), which phi needs too, so one exponential and one reciprocal
+// give both. The negative side is taken as Phi(-|z|) = erfc(|z| / sqrt 2) / 2
+// directly, without the cancellation in 1 + erf.
+struct NormCdfPdf {
+  float cdf, pdf;
+};
+__device__ __forceinline__ NormCdfPdf norm_cdf_pdf(float z) {
+  const float e = exp2f(-0.72134752044448170f * z * z);  // exp(-z^2 / 2): -log2(e) / 2
+  const float x = fabsf(z) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+  float s = fmaf(t, 1.061405429f, -1.453152027f);
+  s = fmaf(t, s, 1.421413741f);
+  s = fmaf(t, s, -0.284496736f);
+  s = fmaf(t, s, 0.254829592f);
+  const float tail = 0.5f * t * s * e;  // Phi(-|z|)
+  return {z >= 0.0f ? 1.0f - tail : tail, 0.39894228040143268f * e};
+}
+__device__ __forceinline__ float gelu_f(float z) { return z * norm_cdf_pdf(z).cdf; }
+// gelu'(z) = Phi(z) + z phi(z)
 __device__ __forceinline__ float dgelu_f(float z) {
-  return gelu_cdf_f(z) + z * 0.39894228040143268f * expf(-0.5f * z * z);
+  const NormCdfPdf n = norm_cdf_pdf(z);
+  return fmaf(z, n.pdf, n.cdf);
 }
 // gelu''(z) = phi(z) (2 - z^2)
-__device__ __forceinline__ float d2gelu_f(float z) {
-  return 0.39894228040143268f * expf(-0.5f * z * z) * (2.0f - z * z);
-}
+__device__ __forceinline__ float d2gelu_f(float z) { return norm_cdf_pdf(z).pdf * (2.0f - z * z); }
 
 // Programmatic dependent launch (sm_90 and later). A kernel launched with the
 // programmatic stream serialization attribute (launch_pdl) may start while its

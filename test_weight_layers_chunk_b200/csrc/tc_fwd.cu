@@ -200,10 +200,15 @@ struct EpiG1Gelu {
       const int j = c.n0 + g;
       float h[32], gp[32];
       ld1(c, 0, g, h);
+      if (c.cls == 1) {  // key rows: gelu and gelu'
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        gp[i] = dgelu_f(h[i]);
-        h[i] = gelu_f(h[i]);
+        for (int i = 0; i < 32; ++i) {
+          gp[i] = dgelu_f(h[i]);
+          h[i] = gelu_f(h[i]);
+        }
+      } else {  // query rows: gelu alone
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h[i] = gelu_f(h[i]);
       }
       staging_free(lane);
       stage32(S, lane, h);
