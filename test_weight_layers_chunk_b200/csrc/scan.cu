@@ -633,6 +633,222 @@ chunk_coeffs_bwd_kernel(const float* __restrict__ lr, const float* __restrict__ 
   }
 }
 
+// Block version of chunk_coeffs_bwd_kernel for full chunks of C = PER x 128
+// tokens: one 128-thread block per (head, chunk), thread i owning tokens
+// [PER i, PER i + PER) with its gates and adjoints in registers (one vector
+// load each). U(t+1, n) and L(t+1, n) are the exponentials of the exclusive
+// suffix log-sums times the segment's later gates and R_t comes from the
+// segments' ratio-sum maps combined across lanes and warps, as in
+// chunk_coeffs_vec_kernel; the forward scans X and (Y, V) compose each
+// thread's segment map across lanes by shuffles and across the four warps
+// through shared memory. The same quantities as the warp kernel (one warp per
+// chunk, which leaves most of the GPU idle); the rounding differs.
+template <int PER>
+__global__ void __launch_bounds__(kK1Threads)
+chunk_coeffs_bwd_vec_kernel(const float* __restrict__ lr, const float* __restrict__ mom,
+                            const float* __restrict__ decay, const float* __restrict__ abar,
+                            const float* __restrict__ bbar, const float* __restrict__ scal_bar,
+                            float* __restrict__ deta, float* __restrict__ dmu,
+                            float* __restrict__ dlam, int BH, int T, int C, int NC, int coef) {
+  __shared__ float s_mu_first[kK1Threads + 1];  // first mu of every segment, then 0
+  __shared__ float w_su[kK1Warps], w_sl[kK1Warps], w_M[kK1Warps], w_C[kK1Warps];
+  __shared__ float w_map[kK1Warps][7];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.x / NC, ci = blockIdx.x % NC;
+  const size_t base = (size_t)bh * T + (size_t)ci * C + (size_t)tid * PER;
+  float eta[PER], mu[PER], lam[PER], ab[PER], bb[PER];
+  load_vec<PER>(lr + base, eta);
+  if (mom) {
+    load_vec<PER>(mom + base, mu);
+  } else {  // no-momentum mode: mu = 0
+#pragma unroll
+    for (int i = 0; i < PER; ++i) mu[i] = 0.f;
+  }
+  load_vec<PER>(decay + base, lam);
+  load_vec<PER>(abar + base, ab);
+  load_vec<PER>(bbar + base, bb);
+  s_mu_first[tid] = mu[0];
+  if (tid == 0) s_mu_first[kK1Threads] = 0.f;  // no token after the chunk's last
+  if (coef) {  // the chunk-averaged variant: every token takes the chunk means
+    float sa = 0.f, sb = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      sa += ab[i];
+      sb += bb[i];
+    }
+    const float ai = warp_suffix_sum(sa, lane), bi = warp_suffix_sum(sb, lane);
+    if (lane == 0) {
+      w_M[warp] = ai;
+      w_C[warp] = bi;
+    }
+    __syncthreads();
+    float at = 0.f, bt = 0.f;
+    for (int w = kK1Warps - 1; w >= 0; --w) {
+      at += w_M[w];
+      bt += w_C[w];
+    }
+    __syncthreads();  // w_M and w_C are written again below
+    const float n = (float)(PER * kK1Threads);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      ab[i] = at / n;
+      bb[i] = bt / n;
+    }
+  }
+
+  // exclusive suffix log-sums of the gates after this thread's segment
+  float pu = 1.f, pl = 1.f;
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    pu *= mu[i];
+    pl *= lam[i];
+  }
+  const float su_inc = warp_suffix_sum(log2f(pu), lane), sl_inc = warp_suffix_sum(log2f(pl), lane);
+  if (lane == 0) {
+    w_su[warp] = su_inc;
+    w_sl[warp] = sl_inc;
+  }
+  __syncthreads();
+  float su_excl = __shfl_down_sync(0xffffffffu, su_inc, 1);
+  float sl_excl = __shfl_down_sync(0xffffffffu, sl_inc, 1);
+  if (lane == 31) {
+    su_excl = 0.f;
+    sl_excl = 0.f;
+  }
+  for (int w = kK1Warps - 1; w > warp; --w) {
+    su_excl += w_su[w];
+    sl_excl += w_sl[w];
+  }
+  const float mu_next = s_mu_first[tid + 1];
+
+  // reverse walk 1: U(t+1, n), L(t+1, n) and the segment's ratio-sum map
+  float U = exp2f(su_excl), L = exp2f(sl_excl);
+  float Ut[PER], Lt[PER];
+  float Mseg = 1.f, Cseg = 0.f;
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    Ut[i] = U;
+    Lt[i] = L;
+    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+    Cseg = L + m * Cseg;
+    Mseg = m * Mseg;
+    U *= mu[i];
+    L *= lam[i];
+  }
+  float M = Mseg, Cc = Cseg;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float Mr = __shfl_down_sync(0xffffffffu, M, off);
+    const float Cr = __shfl_down_sync(0xffffffffu, Cc, off);
+    if (lane + off < 32) {
+      Cc = Cc + M * Cr;
+      M = M * Mr;
+    }
+  }
+  if (lane == 0) {
+    w_M[warp] = M;
+    w_C[warp] = Cc;
+  }
+  __syncthreads();
+  float r_end = 0.f;
+  for (int w = kK1Warps - 1; w > warp; --w) r_end = w_C[w] + w_M[w] * r_end;
+  const float Cn = __shfl_down_sync(0xffffffffu, Cc, 1);
+  const float Mn = __shfl_down_sync(0xffffffffu, M, 1);
+  float r_next = lane == 31 ? r_end : Cn + Mn * r_end;
+
+  // reverse walk 2: R_t and deta_t = abar_t U(t+1, n) + bbar_t R_t
+  float Rt[PER], out[PER];
+#pragma unroll
+  for (int i = PER - 1; i >= 0; --i) {
+    const float m = i + 1 < PER ? mu[i + 1] : mu_next;
+    const float r = Lt[i] + m * r_next;
+    Rt[i] = r;
+    out[i] = ab[i] * Ut[i] + bb[i] * r;
+    r_next = r;
+  }
+  store_vec<PER>(deta + base, out);
+
+  // Forward scans. The segment's map: X -> pX X + uX; (Y, V) -> (p Y + u, q Y + r V + w).
+  float pX = 1.f, uX = 0.f, p = 1.f, q = 0.f, r = 1.f, u = 0.f, w = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const float m_ = mu[i], l_ = lam[i];
+    const float al = ab[i] * eta[i], be = bb[i] * eta[i];
+    uX = m_ * uX + al;
+    pX = m_ * pX;
+    const float q2 = m_ * p + l_ * q;
+    const float w2 = m_ * u + l_ * w + be;
+    p = m_ * p;
+    r = l_ * r;
+    u = m_ * u + be;
+    q = q2;
+    w = w2;
+  }
+  // inclusive prefix composition across lanes (this lane's map after the earlier ones)
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float pXe = __shfl_up_sync(0xffffffffu, pX, off);
+    const float uXe = __shfl_up_sync(0xffffffffu, uX, off);
+    const float pe = __shfl_up_sync(0xffffffffu, p, off);
+    const float qe = __shfl_up_sync(0xffffffffu, q, off);
+    const float re = __shfl_up_sync(0xffffffffu, r, off);
+    const float ue = __shfl_up_sync(0xffffffffu, u, off);
+    const float we = __shfl_up_sync(0xffffffffu, w, off);
+    if (lane >= off) {
+      uX = pX * uXe + uX;
+      pX = pX * pXe;
+      const float np = p * pe;
+      const float nq = q * pe + r * qe;
+      const float nr = r * re;
+      const float nu = p * ue + u;
+      const float nw = q * ue + r * we + w;
+      p = np; q = nq; r = nr; u = nu; w = nw;
+    }
+  }
+  if (lane == 31) {  // the warp's whole map
+    w_map[warp][0] = pX; w_map[warp][1] = uX; w_map[warp][2] = p; w_map[warp][3] = q;
+    w_map[warp][4] = r; w_map[warp][5] = u; w_map[warp][6] = w;
+  }
+  __syncthreads();
+  // the chunk's initial values X_1 = PUbar, Y_1 = cbar, V_1 = PLbar, carried
+  // through the earlier warps' maps, then through this warp's earlier lanes
+  const size_t plane = (size_t)BH * NC;
+  const size_t o = (size_t)bh * NC + ci;
+  float X = scal_bar[o], Y = scal_bar[2 * plane + o], V = scal_bar[plane + o];
+  for (int wi = 0; wi < warp; ++wi) {
+    const float* mp = w_map[wi];
+    const float Xn = mp[0] * X + mp[1];
+    const float Yn = mp[2] * Y + mp[5];
+    V = mp[3] * Y + mp[4] * V + mp[6];
+    X = Xn;
+    Y = Yn;
+  }
+  {
+    float epX = __shfl_up_sync(0xffffffffu, pX, 1), euX = __shfl_up_sync(0xffffffffu, uX, 1);
+    float ep = __shfl_up_sync(0xffffffffu, p, 1), eq = __shfl_up_sync(0xffffffffu, q, 1);
+    float er = __shfl_up_sync(0xffffffffu, r, 1), eu = __shfl_up_sync(0xffffffffu, u, 1);
+    float ew = __shfl_up_sync(0xffffffffu, w, 1);
+    if (lane == 0) { epX = 1.f; euX = 0.f; ep = 1.f; eq = 0.f; er = 1.f; eu = 0.f; ew = 0.f; }
+    const float Xn = epX * X + euX;
+    const float Yn = ep * Y + eu;
+    V = eq * Y + er * V + ew;
+    X = Xn;
+    Y = Yn;
+  }
+  float om[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    om[i] = Ut[i] * X + Rt[i] * Y;
+    out[i] = Lt[i] * V;
+    X = mu[i] * X + ab[i] * eta[i];
+    const float Yn = mu[i] * Y + bb[i] * eta[i];
+    V = lam[i] * V + Yn;
+    Y = Yn;
+  }
+  if (dmu) store_vec<PER>(dmu + base, om);  // NULL in no-momentum mode
+  store_vec<PER>(dlam + base, out);
+}
+
 }  // namespace
 
 cudaError_t launch_chunk_coeffs(const float* lr, const float* mom, const float* decay, float* a,
@@ -676,6 +892,23 @@ cudaError_t launch_chunk_coeffs_bwd(const float* lr, const float* mom, const flo
                                     const float* abar, const float* bbar, const float* scal_bar,
                                     float* deta, float* dmu, float* dlam, int BH, int T, int C,
                                     int NC, int coef, cudaStream_t st) {
+  // Full chunks of 128, 256, 512 or 1024 tokens with vector-aligned buffers:
+  // one block per chunk.
+  const int per = C / kK1Threads;
+  const int vb = per >= 4 ? 16 : per * 4;  // alignment of one vector access in bytes
+  auto vec_ok = [&](const void* p) { return p == nullptr || ((uintptr_t)p % vb) == 0; };
+  if (T % C == 0 && C % kK1Threads == 0 && (per == 1 || per == 2 || per == 4 || per == 8) &&
+      vec_ok(lr) && vec_ok(mom) && vec_ok(decay) && vec_ok(abar) && vec_ok(bbar) &&
+      vec_ok(deta) && vec_ok(dmu) && vec_ok(dlam)) {
+    E2TTT_TRACE("k1_chunk_coeffs_bwd", st);
+    switch (per) {
+      case 1: chunk_coeffs_bwd_vec_kernel<1><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC, coef); break;
+      case 2: chunk_coeffs_bwd_vec_kernel<2><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC, coef); break;
+      case 4: chunk_coeffs_bwd_vec_kernel<4><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC, coef); break;
+      default: chunk_coeffs_bwd_vec_kernel<8><<<BH * NC, kK1Threads, 0, st>>>(lr, mom, decay, abar, bbar, scal_bar, deta, dmu, dlam, BH, T, C, NC, coef); break;
+    }
+    return cudaGetLastError();
+  }
   int warps = BH * NC;
   int blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
   size_t smem = (size_t)kWarpsPerBlock * 3 * C * sizeof(float);

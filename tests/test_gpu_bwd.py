@@ -72,6 +72,15 @@ F32 = {
     "gelu_dot": gen.Workload("bgd", gen.GELU, gen.F32, 2, 1, 12, 16, 20, 48, 16, "uniform", 0.99,
                              seed=48, loss=gen.LOSS_NEG_DOT, lr_lo=0.001, lr_hi=0.005,
                              mom_lo=0.5, mom_hi=0.9),
+    # full chunks of 128, 256 and 512 tokens, where the gate gradients come from
+    # the block-per-chunk form of the K1 adjoint (1, 2 and 4 tokens per thread;
+    # the chunks of 16 to 32 tokens above take its one-warp-per-chunk form)
+    "linear_c128": gen.Workload("blc1", gen.LINEAR, gen.F32, 1, 2, 16, 12, 0, 384, 128, "uniform",
+                                0.99, seed=61, lr_lo=0.002, lr_hi=0.02),
+    "swiglu_c256": gen.Workload("bsc2", gen.SWIGLU, gen.F32, 1, 2, 12, 16, 20, 512, 256, "uniform",
+                                0.99, seed=62, lr_lo=0.002, lr_hi=0.02, mom_lo=0.7, mom_hi=0.95),
+    "linear_c512": gen.Workload("blc5", gen.LINEAR, gen.F32, 2, 1, 8, 8, 0, 1024, 512, "uniform",
+                                0.99, seed=63, lr_lo=0.002, lr_hi=0.01),
 }
 
 

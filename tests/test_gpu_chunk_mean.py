@@ -56,6 +56,9 @@ CASES = {
                                seed=41),
     "swiglu_f32": gen.Workload("cms", gen.SWIGLU, gen.F32, 1, 2, 16, 12, 24, 50, 16, "uniform", 0.99,
                                seed=43, lr_lo=0.002, lr_hi=0.02, mom_lo=0.7, mom_hi=0.95),
+    # full chunks of 256 tokens: the block-per-chunk K1 adjoint with chunk means
+    "linear_f32_c256": gen.Workload("cmlc", gen.LINEAR, gen.F32, 1, 2, 16, 12, 0, 512, 256,
+                                    "uniform", 0.99, seed=65, lr_lo=0.002, lr_hi=0.02),
     "swiglu_bf16_tc": gen.Workload("cmb", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128,
                                    "uniform", 0.999, seed=45, lr_lo=0.002, lr_hi=0.02),
 }

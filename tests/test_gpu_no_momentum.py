@@ -32,6 +32,9 @@ CASES = {
                                seed=51),
     "swiglu_f32": gen.Workload("nms", gen.SWIGLU, gen.F32, 1, 2, 16, 12, 24, 50, 16, "uniform", 0.99,
                                seed=53, lr_lo=0.002, lr_hi=0.02),
+    # full chunks of 128 tokens: the block-per-chunk K1 adjoint with no momentum
+    "linear_f32_c128": gen.Workload("nmlc", gen.LINEAR, gen.F32, 1, 2, 16, 12, 0, 384, 128,
+                                    "uniform", 0.99, seed=67, lr_lo=0.002, lr_hi=0.02),
     "linear_bf16_tc": gen.Workload("nmlb", gen.LINEAR, gen.BF16, 1, 2, 128, 128, 0, 512, 128,
                                    "uniform", 0.999, seed=55, lr_lo=0.002, lr_hi=0.02),
     "swiglu_bf16_tc": gen.Workload("nmsb", gen.SWIGLU, gen.BF16, 1, 2, 128, 128, 256, 512, 128,
